@@ -1,0 +1,505 @@
+"""CPU oracle for the DFlash draft-proposal step (propose + inject + greedy verify).
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product path imports, links or runs
+this module: only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline
+leg of ``bench.py`` may call it.  It shares no code with the CUDA library; both
+sides only receive the same seeded inputs.
+
+What it is: a plain, slow, obviously correct restatement of what the DFlash
+pages say the proposal step computes, in float64 arithmetic (numpy), with a
+library matmul as the only non-elementary step.  Every function names the
+passage it follows.  The three pages are cited by title:
+
+  [NEURON]  "DFlash Speculative Decoding in the vLLM Neuron Framework"
+            (AWS Neuron design doc), sections as named there.
+  [VLLM]    "[Feat][Spec Decode] DFlash" (vLLM pull request #36847),
+            unit test ``test_set_inputs_first_pass_dflash`` and the
+            acceptance-metric helpers.
+  [QEFF]    "Dflash: Block Diffusion Speculative Decoding" (QEfficient pull
+            request #995), PR description and commit notes.
+
+Precision modes
+---------------
+``exact``   every intermediate stays float64.  Used for the logits check
+            (relative L2 against the bf16 GPU path).
+``bf16io``  rounds to bfloat16 (round-to-nearest-even, via float32) at the
+            storage points listed in ``BF16_STORAGE_POINTS``; everything else
+            stays float64.  Used for bit-exact draft / acceptance comparison.
+            Argmax decisions are taken on float32-rounded logits in both modes
+            (the kernel's decision precision).
+
+Readings where the pages are silent (each is also listed in the design notes):
+  * every norm is RMSNorm ``x * rsqrt(mean(x^2) + eps) * w`` (weight multiplies
+    directly), q/k norms are per head over head_dim;
+  * context vectors feed Wk/Wv directly (no input_layernorm on the context),
+    per [NEURON] "Context KV Injection" step 2;
+  * no biases anywhere; one final RMSNorm before the LM head;
+  * RoPE is the rotate-half form, pairs (i, i + d/2), inv_freq_i =
+    theta^(-2i/d), angles from integer positions in float64, attention scaling 1;
+  * softmax scale 1/sqrt(head_dim), no soft-cap, no window;
+  * argmax ties go to the lowest index, NaN compares equal to -inf;
+  * K = block_size - 1 drafts per request.
+
+Parity pins: see tests/test_oracle_pins.py.  The whole draft stack beyond the
+single-layer library comparison and the invariants there is "parity unpinned"
+in the sense that no page prints model outputs.
+"""
+
+from __future__ import annotations
+
+from dataclasses import dataclass
+from typing import Callable, Mapping, Sequence
+
+import numpy as np
+
+# Storage points at which the ``bf16io`` mode rounds to bfloat16.  The names
+# are the oracle's own; the GPU path rounds at the same points by design.
+BF16_STORAGE_POINTS = (
+    "context vector c = hidden_norm(fc(x))",
+    "injected context K (after k_norm + RoPE) and V",
+    "normed activations fed to a projection (input/post-attention norms)",
+    "block q after q_norm + RoPE; block K (after k_norm + RoPE) and V",
+    "attention output o",
+    "MLP hidden silu(gate) * up",
+    "final-normed rows fed to the LM head",
+)
+
+
+# ----------------------------------------------------------------------------
+# configuration
+# ----------------------------------------------------------------------------
+@dataclass(frozen=True)
+class OracleConfig:
+    """Draft-model geometry.  Field names follow the [NEURON] DFlashConfig
+    (block size, mask token id, target layer ids) plus the Qwen3 layer shape
+    ([NEURON] "DFlash Draft Model Architecture")."""
+
+    hidden: int
+    n_layers: int
+    n_q_heads: int
+    n_kv_heads: int
+    head_dim: int
+    intermediate: int
+    vocab: int
+    n_target_layers: int
+    block_size: int
+    mask_token_id: int
+    page_size: int = 16
+    rms_eps: float = 1e-6
+    rope_theta: float = 1e6
+
+    @staticmethod
+    def from_mapping(m: Mapping) -> "OracleConfig":
+        names = OracleConfig.__dataclass_fields__.keys()
+        return OracleConfig(**{k: m[k] for k in names if k in m})
+
+    @property
+    def num_drafts(self) -> int:
+        # [NEURON] "Configuration Parameters": one block slot is the bonus
+        # token, so the draft width is block_size - 1.
+        return self.block_size - 1
+
+
+# ----------------------------------------------------------------------------
+# rounding
+# ----------------------------------------------------------------------------
+def round_bf16(a) -> np.ndarray:
+    """Round to bfloat16 (nearest, ties to even) and return float64 values.
+
+    Goes through float32 first (float64 -> float32 is IEEE nearest-even), then
+    drops the low 16 bits of the float32 pattern with nearest-even rounding.
+    Inputs are finite in every workload this oracle sees."""
+    f = np.asarray(a, dtype=np.float64).astype(np.float32)
+    u = f.view(np.uint32).astype(np.uint64)
+    lsb = (u >> np.uint64(16)) & np.uint64(1)
+    u = (u + np.uint64(0x7FFF) + lsb) & np.uint64(0xFFFF0000)
+    return u.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+def _identity(a) -> np.ndarray:
+    return np.asarray(a, dtype=np.float64)
+
+
+def rounding(mode: str) -> Callable[[np.ndarray], np.ndarray]:
+    if mode == "exact":
+        return _identity
+    if mode == "bf16io":
+        return round_bf16
+    raise ValueError(f"unknown precision mode {mode!r}")
+
+
+# ----------------------------------------------------------------------------
+# elementary operations
+# ----------------------------------------------------------------------------
+def rms_norm(x: np.ndarray, w: np.ndarray, eps: float) -> np.ndarray:
+    """RMSNorm over the last axis: x / sqrt(mean(x^2) + eps) * w.
+
+    [NEURON] names "hidden_norm" and "pre-norms" of a standard Qwen3 decoder
+    layer without defining them; the Qwen3 norm is RMSNorm."""
+    x = np.asarray(x, dtype=np.float64)
+    ms = np.mean(x * x, axis=-1, keepdims=True)
+    return x / np.sqrt(ms + eps) * np.asarray(w, dtype=np.float64)
+
+
+def silu(x: np.ndarray) -> np.ndarray:
+    """SiLU(x) = x * sigmoid(x), the SwiGLU gate of a Qwen3 MLP."""
+    x = np.asarray(x, dtype=np.float64)
+    return x / (1.0 + np.exp(-x))
+
+
+def linear(x: np.ndarray, w: np.ndarray) -> np.ndarray:
+    """y = x @ w^T with w stored [out, in] (no bias).  float64 matmul."""
+    return np.asarray(x, dtype=np.float64) @ np.asarray(w, dtype=np.float64).T
+
+
+def rope_inv_freq(head_dim: int, theta: float) -> np.ndarray:
+    """inv_freq_i = theta^(-2i/d), i < d/2 (default RoPE, attention scaling 1;
+    [QEFF] commit notes fold attention_scaling into the sin/cos table)."""
+    i = np.arange(head_dim // 2, dtype=np.float64)
+    return theta ** (-(2.0 * i) / head_dim)
+
+
+def apply_rope(x: np.ndarray, positions: np.ndarray, theta: float) -> np.ndarray:
+    """Rotate-half RoPE on the last axis of ``x`` (shape [..., n, heads, d] or
+    [n, d]) at integer ``positions`` (shape [n]).
+
+    out[i]       = x[i] cos(a_i) - x[i + d/2] sin(a_i)
+    out[i + d/2] = x[i + d/2] cos(a_i) + x[i] sin(a_i),  a_i = pos * inv_freq_i
+    """
+    x = np.asarray(x, dtype=np.float64)
+    d = x.shape[-1]
+    half = d // 2
+    pos = np.asarray(positions, dtype=np.float64)
+    ang = pos[:, None] * rope_inv_freq(d, theta)[None, :]  # [n, d/2]
+    cos, sin = np.cos(ang), np.sin(ang)
+    # broadcast [n, d/2] against x's [n, (heads,) d/2]
+    extra = x.ndim - 2
+    shape = (ang.shape[0],) + (1,) * extra + (half,)
+    cos = cos.reshape(shape)
+    sin = sin.reshape(shape)
+    x1, x2 = x[..., :half], x[..., half:]
+    return np.concatenate([x1 * cos - x2 * sin, x2 * cos + x1 * sin], axis=-1)
+
+
+def argmax_f32(logits: np.ndarray) -> np.ndarray:
+    """Greedy pick over the last axis, decided on float32 values.
+
+    Ties go to the lowest index (np.argmax returns the first maximum); NaN is
+    treated as -inf so it never wins over a number."""
+    f = np.asarray(logits).astype(np.float32)
+    f = np.where(np.isnan(f), np.float32(-np.inf), f)
+    return np.argmax(f, axis=-1).astype(np.int64)
+
+
+# ----------------------------------------------------------------------------
+# paged KV addressing and block construction
+# ----------------------------------------------------------------------------
+def paged_slots(positions, req_ids, block_table, page_size: int) -> np.ndarray:
+    """Map absolute positions to cache slots, [NEURON] "Paged KV Integration":
+    page number = pos // page clamped to the table width - 1, page id looked
+    up in the request's block-table row, slot = page_id * page + pos % page."""
+    positions = np.asarray(positions, dtype=np.int64)
+    req_ids = np.asarray(req_ids, dtype=np.int64)
+    bt = np.asarray(block_table, dtype=np.int64)
+    max_blocks = bt.shape[1]
+    flat = bt.reshape(-1)
+    block_numbers = np.minimum(positions // page_size, max_blocks - 1)
+    block_ids = flat[req_ids * max_blocks + block_numbers]
+    return block_ids * page_size + positions % page_size
+
+
+@dataclass
+class QueryBlock:
+    input_ids: np.ndarray         # [B * bs]
+    positions: np.ndarray         # [B * bs]
+    req_ids: np.ndarray           # [B * bs]
+    keep_idx: np.ndarray          # [B * (bs - 1)]
+    query_start_loc: np.ndarray   # [B + 1]
+
+
+def build_query_block(bonus_tokens, seq_lens, block_size: int,
+                      mask_token_id: int) -> QueryBlock:
+    """[NEURON] "Draft Block Construction": each request contributes
+    [bonus, mask, ..., mask] (block_size slots) at positions
+    seq_len + [0 .. block_size-1]; keep_idx selects slots 1 .. block_size-1.
+    [VLLM] test_set_inputs_first_pass_dflash prints a worked example of the
+    same layout, with query_start_loc = [0, bs, 2 bs, ...]."""
+    bonus = np.asarray(bonus_tokens, dtype=np.int64)
+    lens = np.asarray(seq_lens, dtype=np.int64)
+    B = bonus.shape[0]
+    ids = np.full((B, block_size), mask_token_id, dtype=np.int64)
+    ids[:, 0] = bonus
+    pos = lens[:, None] + np.arange(block_size, dtype=np.int64)[None, :]
+    req = np.repeat(np.arange(B, dtype=np.int64), block_size)
+    keep = (np.arange(B, dtype=np.int64)[:, None] * block_size
+            + np.arange(1, block_size, dtype=np.int64)[None, :]).reshape(-1)
+    qsl = np.arange(B + 1, dtype=np.int64) * block_size
+    return QueryBlock(ids.reshape(-1), pos.reshape(-1), req, keep, qsl)
+
+
+# ----------------------------------------------------------------------------
+# (a1) context fusion, (a2) context K/V injection
+# ----------------------------------------------------------------------------
+def context_fusion(cfg: OracleConfig, W: Mapping, aux: np.ndarray,
+                   mode: str = "exact") -> np.ndarray:
+    """[NEURON] "Context KV Injection" step 1 and [QEFF] (concat -> fc ->
+    hidden_norm): ctx = hidden_norm(fc(aux)).  ``aux`` is the concatenation of
+    the tapped target states, [n, n_target * hidden]."""
+    rnd = rounding(mode)
+    aux = np.asarray(aux, dtype=np.float64)
+    assert aux.shape[-1] == cfg.n_target_layers * cfg.hidden
+    f = linear(aux, W["fc_w"])
+    return rnd(rms_norm(f, W["hidden_norm_w"], cfg.rms_eps))
+
+
+def context_kv(cfg: OracleConfig, W: Mapping, ctx: np.ndarray,
+               positions: np.ndarray, mode: str = "exact"):
+    """[NEURON] "Context KV Injection" step 2: one matmul of ctx against all
+    layers' stacked K/V weights, then each layer's keys are k-normed and
+    RoPE-encoded at the context's own positions.  Returns per-layer lists of
+    K and V, each [n, n_kv_heads, head_dim]."""
+    rnd = rounding(mode)
+    L, Hkv, d = cfg.n_layers, cfg.n_kv_heads, cfg.head_dim
+    fused = np.concatenate(
+        [np.concatenate([W["wk"][l], W["wv"][l]], axis=0) for l in range(L)],
+        axis=0)                                   # [L * 2 * Hkv * d, hidden]
+    kv = linear(ctx, fused).reshape(ctx.shape[0], L, 2, Hkv, d)
+    ks, vs = [], []
+    for l in range(L):
+        k = rms_norm(kv[:, l, 0], W["k_norm_w"][l], cfg.rms_eps)
+        k = apply_rope(k, positions, cfg.rope_theta)
+        ks.append(rnd(k))
+        vs.append(rnd(kv[:, l, 1]))
+    return ks, vs
+
+
+def write_slots(cache: np.ndarray, slots: np.ndarray, values: np.ndarray,
+                page_size: int) -> None:
+    """index_put of per-token [Hkv, d] rows into a [pages, Hkv, page, d]
+    cache ([NEURON] "Context KV Injection" step 3).  Negative slots are padding
+    rows and are skipped (vLLM slot-mapping convention)."""
+    slots = np.asarray(slots, dtype=np.int64)
+    for r, s in enumerate(slots):
+        if s < 0:
+            continue
+        cache[s // page_size, :, s % page_size, :] = values[r]
+
+
+def inject_context(cfg: OracleConfig, W: Mapping, aux, positions, slot_mapping,
+                   k_caches: Sequence[np.ndarray], v_caches: Sequence[np.ndarray],
+                   mode: str = "exact") -> None:
+    """precompute_and_store_context_kv ([NEURON] "Context KV Injection"
+    steps 1-3): fuse, project, norm + rotate keys, scatter into each layer's
+    paged cache at ``slot_mapping``."""
+    aux = np.asarray(aux, dtype=np.float64)
+    if aux.shape[0] == 0:
+        return
+    ctx = context_fusion(cfg, W, aux, mode)
+    ks, vs = context_kv(cfg, W, ctx, positions, mode)
+    for l in range(cfg.n_layers):
+        write_slots(k_caches[l], slot_mapping, ks[l], cfg.page_size)
+        write_slots(v_caches[l], slot_mapping, vs[l], cfg.page_size)
+
+
+# ----------------------------------------------------------------------------
+# (a5) non-causal block attention over the paged cache
+# ----------------------------------------------------------------------------
+def gather_kv(cache: np.ndarray, block_table_row, n_keys: int,
+              page_size: int) -> np.ndarray:
+    """Logical keys 0 .. n_keys-1 of one request, [n_keys, Hkv, d], gathered
+    through the request's block-table row with the paged-slot formula."""
+    pos = np.arange(n_keys, dtype=np.int64)
+    slots = paged_slots(pos, np.zeros(n_keys, dtype=np.int64),
+                        np.asarray(block_table_row)[None, :], page_size)
+    return cache[slots // page_size, :, slots % page_size, :]
+
+
+def attention_one_request(q: np.ndarray, k: np.ndarray, v: np.ndarray,
+                          n_q_heads: int, n_kv_heads: int) -> np.ndarray:
+    """Non-causal attention of every query row over every key
+    ([NEURON] "What is DFlash": each query position attends to the injected
+    context and the rest of the block; vLLM runs it with causal=False).
+
+    q [nq, Hq, d], k/v [nk, Hkv, d]  ->  o [nq, Hq, d].  Query head h reads
+    kv head h // (Hq / Hkv).  Scores scaled by 1/sqrt(d); plain softmax."""
+    G = n_q_heads // n_kv_heads
+    d = q.shape[-1]
+    out = np.empty(q.shape, dtype=np.float64)
+    for h in range(n_q_heads):
+        kh = k[:, h // G, :]
+        vh = v[:, h // G, :]
+        s = (q[:, h, :] @ kh.T) / np.sqrt(d)           # [nq, nk]
+        s = s - s.max(axis=1, keepdims=True)
+        p = np.exp(s)
+        p = p / p.sum(axis=1, keepdims=True)
+        out[:, h, :] = p @ vh
+    return out
+
+
+def block_attention(cfg: OracleConfig, q: np.ndarray, k_cache: np.ndarray,
+                    v_cache: np.ndarray, block_table, seq_lens) -> np.ndarray:
+    """q [B * bs, Hq, d] for the query blocks -> o [B * bs, Hq, d].  Request b
+    sees logical keys [0, seq_len_b + bs): its context plus its whole block."""
+    bs = cfg.block_size
+    bt = np.asarray(block_table)
+    o = np.empty(q.shape, dtype=np.float64)
+    for b, n_ctx in enumerate(np.asarray(seq_lens, dtype=np.int64)):
+        n_keys = int(n_ctx) + bs
+        k = gather_kv(k_cache, bt[b], n_keys, cfg.page_size)
+        v = gather_kv(v_cache, bt[b], n_keys, cfg.page_size)
+        rows = slice(b * bs, (b + 1) * bs)
+        o[rows] = attention_one_request(q[rows], k.astype(np.float64),
+                                        v.astype(np.float64),
+                                        cfg.n_q_heads, cfg.n_kv_heads)
+    return o
+
+
+# ----------------------------------------------------------------------------
+# (a3)-(a7) the proposal forward
+# ----------------------------------------------------------------------------
+@dataclass
+class Proposal:
+    draft_tokens: np.ndarray      # [B, K]
+    block_tokens: np.ndarray      # [B, bs]  (bonus + drafts)
+    logits: np.ndarray            # [B * K, V] float64 (before the float32 pick)
+    hidden: np.ndarray            # [B * bs, H] final residual stream (pre final norm)
+
+
+def draft_layer(cfg: OracleConfig, W: Mapping, l: int, x: np.ndarray,
+                qb: QueryBlock, block_table, seq_lens,
+                k_cache: np.ndarray, v_cache: np.ndarray,
+                rnd: Callable) -> np.ndarray:
+    """One DFlashQwen3DecoderLayer ([NEURON] "DFlash Draft Model
+    Architecture": a standard Qwen3 decoder layer, attention + MLP with
+    pre-norms, attention run non-causally):
+
+      n  = RMSNorm(x; input_norm)
+      q, k, v = Wq n, Wk n, Wv n;  q, k per-head RMSNorm; RoPE at block positions
+      block k, v written to the block's paged slots ([NEURON] "Paged KV
+      Integration": the same slot helper serves the query block)
+      o  = non-causal attention over [0, seq_len + bs)
+      x += Wo o
+      n2 = RMSNorm(x; post_attention_norm)
+      x += Wd (silu(Wg n2) * Wu n2)
+    """
+    Hq, Hkv, d, eps = cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim, cfg.rms_eps
+    M = x.shape[0]
+    n = rnd(rms_norm(x, W["in_norm_w"][l], eps))
+    q = linear(n, W["wq"][l]).reshape(M, Hq, d)
+    k = linear(n, W["wk"][l]).reshape(M, Hkv, d)
+    v = linear(n, W["wv"][l]).reshape(M, Hkv, d)
+    q = rnd(apply_rope(rms_norm(q, W["q_norm_w"][l], eps), qb.positions,
+                       cfg.rope_theta))
+    k = rnd(apply_rope(rms_norm(k, W["k_norm_w"][l], eps), qb.positions,
+                       cfg.rope_theta))
+    v = rnd(v)
+    slots = paged_slots(qb.positions, qb.req_ids, block_table, cfg.page_size)
+    write_slots(k_cache, slots, k, cfg.page_size)
+    write_slots(v_cache, slots, v, cfg.page_size)
+    o = rnd(block_attention(cfg, q, k_cache, v_cache, block_table, seq_lens))
+    x = x + linear(o.reshape(M, Hq * d), W["wo"][l])
+    n2 = rnd(rms_norm(x, W["post_norm_w"][l], eps))
+    h = rnd(silu(linear(n2, W["w_gate"][l])) * linear(n2, W["w_up"][l]))
+    return x + linear(h, W["w_down"][l])
+
+
+def lm_head_logits(W: Mapping, rows: np.ndarray, chunk: int = 16384) -> np.ndarray:
+    """rows @ lm_head^T in float64, a vocabulary chunk at a time."""
+    V = W["lm_head"].shape[0]
+    out = np.empty((rows.shape[0], V), dtype=np.float64)
+    for v0 in range(0, V, chunk):
+        out[:, v0:v0 + chunk] = linear(rows, W["lm_head"][v0:v0 + chunk])
+    return out
+
+
+def propose(cfg: OracleConfig, W: Mapping, bonus_tokens, seq_lens, block_table,
+            k_caches: Sequence[np.ndarray], v_caches: Sequence[np.ndarray],
+            mode: str = "exact") -> Proposal:
+    """DFlashQwen3ForCausalLM.forward after injection ([NEURON] code block):
+    build [bonus, mask..] blocks, embed with the (aliased) target embedding,
+    run the decoder stack non-causally over the injected context, keep slots
+    1..bs-1, final RMSNorm, (aliased) target LM head, greedy pick; the block
+    output is cat(bonus, drafts).  Writes the block's K/V into the caches."""
+    rnd = rounding(mode)
+    bonus = np.asarray(bonus_tokens, dtype=np.int64)
+    B, bs, K = bonus.shape[0], cfg.block_size, cfg.num_drafts
+    qb = build_query_block(bonus, seq_lens, bs, cfg.mask_token_id)
+    x = np.asarray(W["embed"])[qb.input_ids].astype(np.float64)
+    for l in range(cfg.n_layers):
+        x = draft_layer(cfg, W, l, x, qb, block_table, seq_lens,
+                        k_caches[l], v_caches[l], rnd)
+    kept = x[qb.keep_idx]
+    f = rnd(rms_norm(kept, W["final_norm_w"], cfg.rms_eps))
+    logits = lm_head_logits(W, f)
+    drafts = argmax_f32(logits).reshape(B, K)
+    block = np.concatenate([bonus[:, None], drafts], axis=1)
+    return Proposal(drafts, block, logits, x)
+
+
+# ----------------------------------------------------------------------------
+# (a8) greedy verification
+# ----------------------------------------------------------------------------
+@dataclass
+class Verification:
+    out_tokens: np.ndarray     # [B, K+1], -1 after the bonus
+    num_accepted: np.ndarray   # [B]
+    bonus: np.ndarray          # [B]
+
+
+def verify_greedy(drafts, target_logits) -> Verification:
+    """Greedy acceptance against the target's predictions.
+
+    Target row j (j = 0..K) predicts the token after block slot j, slot 0
+    being the previous bonus token and slot j the draft d_{j-1} (0-based
+    d_0..d_{K-1} = drafts[:, 0..K-1]).  Drafts are accepted while
+    d_j == argmax T_j; n = number accepted; the bonus token is argmax T_n; the
+    emitted row is [d_0 .. d_{n-1}, bonus, -1, ...] of length K+1 — the
+    sampler output with rejected slots marked -1 ([NEURON] "Async Rejection
+    and Position Correction" counts valid entries as != -1).  The output is
+    what plain greedy decoding of the target emits ([QEFF]: verification by
+    the frozen target guarantees output identical to standard decoding)."""
+    d = np.asarray(drafts, dtype=np.int64)
+    B, K = d.shape
+    t = argmax_f32(target_logits)                     # [B, K+1]
+    assert t.shape == (B, K + 1)
+    out = np.full((B, K + 1), -1, dtype=np.int64)
+    n_acc = np.zeros(B, dtype=np.int64)
+    bonus = np.zeros(B, dtype=np.int64)
+    for b in range(B):
+        n = 0
+        while n < K and d[b, n] == t[b, n]:
+            n += 1
+        out[b, :n] = d[b, :n]
+        out[b, n] = t[b, n]
+        n_acc[b] = n
+        bonus[b] = t[b, n]
+    return Verification(out, n_acc, bonus)
+
+
+def acceptance_length(num_accepted_tokens: int, num_drafts: int) -> float:
+    """[VLLM] compute_acceptance_len: 1 + accepted / drafts (1 if none)."""
+    return 1.0 if num_drafts == 0 else 1.0 + num_accepted_tokens / num_drafts
+
+
+def acceptance_rate(num_accepted_tokens: int, num_draft_tokens: int) -> float:
+    """[VLLM] compute_acceptance_rate: accepted / draft tokens (nan if none)."""
+    return float("nan") if num_draft_tokens == 0 else \
+        num_accepted_tokens / num_draft_tokens
+
+
+# ----------------------------------------------------------------------------
+# helpers for callers
+# ----------------------------------------------------------------------------
+def empty_caches(cfg: OracleConfig, num_pages: int, dtype=np.float64):
+    """Per-layer zeroed K and V pools, [num_pages, Hkv, page, d] each."""
+    shape = (num_pages, cfg.n_kv_heads, cfg.page_size, cfg.head_dim)
+    return ([np.zeros(shape, dtype=dtype) for _ in range(cfg.n_layers)],
+            [np.zeros(shape, dtype=dtype) for _ in range(cfg.n_layers)])
+
+
+def top2_gap_f32(logits: np.ndarray) -> np.ndarray:
+    """Gap between the largest and second-largest float32 logit per row; used
+    to flag near-ties whose greedy pick legitimately depends on rounding."""
+    f = np.asarray(logits).astype(np.float32).astype(np.float64)
+    part = np.partition(f, -2, axis=-1)
+    return part[..., -1] - part[..., -2]
