@@ -1,0 +1,360 @@
+// attention.cuh — non-causal block attention over a paged KV cache (sm_100a).
+//
+// One CTA serves one (request b, kv head h, key split): all bs * G query rows
+// of the kv group (bs block slots x G = Hq / Hkv query heads) attend, with no
+// mask inside the range, to keys [split * chunk, ...) of the request's logical
+// keys [0, seq_len + bs) — its injected context plus its whole block.  Each K
+// and V byte is read from HBM once per kv group.
+//
+// Pages are staged with TMA tile loads (128-byte swizzle, one 16-row x 128-byte
+// box per page and 64-wide half of head_dim) into a ring of shared-memory
+// stages of 64 keys; a producer warp walks the block table.  Compute warps own
+// 16 query rows each and run bf16 mma.sync (m16n8k16) for Q K^T and P V with an
+// fp32 online softmax whose row statistics are reduced with quad shuffles.
+// When the request needs more than one split, partial (O, m, l) go to a
+// workspace and attn_combine_kernel merges them in split order.
+#pragma once
+
+#include "dflash_device.cuh"
+
+namespace dflash {
+
+constexpr int kAttnTileKeys = 64;
+constexpr int kAttnStages = 4;
+constexpr int kAttnMaxComputeWarps = 8;
+
+template <int D>
+struct AttnCfg {
+  static constexpr int kBoxBytes = 16 * 128;          // 16 keys x 64 bf16
+  static constexpr int kBoxesPerPage = D / 64;
+  static constexpr int kPagesPerTile = kAttnTileKeys / 16;
+  static constexpr int kKVBytes = kPagesPerTile * kBoxesPerPage * kBoxBytes;
+  static constexpr int kQStride = D + 8;              // padded row (bf16 elements)
+  static constexpr int smem_bytes(int n_compute_warps) {
+    return 1024 + kAttnStages * 2 * kKVBytes + n_compute_warps * 16 * kQStride * 2 + 256;
+  }
+};
+
+struct AttnParams {
+  const bf16* q;       // [M, Hq, D]
+  bf16* o;             // [M, Hq * D]
+  float* part_o;       // [max_splits][B][Hkv][R][D]
+  float* part_ml;      // [max_splits][B][Hkv][R][2]
+  const int* seq_lens;
+  const int* block_table;
+  int B, W, bs, Hq, Hkv, G, R, num_pages, chunk_keys, max_splits;
+  float scale_log2;    // log2(e) / sqrt(D)
+  unsigned* err;
+};
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Byte offset of (key kt in tile, 16-byte chunk c of the D-wide row) inside a
+// K or V stage laid out as [page][box half][16 rows x 128 B, 128B-swizzled].
+template <int D>
+__device__ __forceinline__ uint32_t kv_off(int kt, int c) {
+  const int jp = kt >> 4, rp = kt & 15;
+  const int hf = c >> 3, cc = c & 7;
+  return static_cast<uint32_t>((jp * AttnCfg<D>::kBoxesPerPage + hf) * AttnCfg<D>::kBoxBytes +
+                               rp * 128 + ((cc ^ (rp & 7)) << 4));
+}
+
+template <int D>
+__global__ void __launch_bounds__(32 * (kAttnMaxComputeWarps + 1), 1)
+    attn_block_kernel(const __grid_constant__ CUtensorMap tmK,
+                      const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+  using C = AttnCfg<D>;
+  const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int n_keys = p.seq_lens[b] + p.bs;
+  const int k0 = split * p.chunk_keys;
+  if (k0 >= n_keys) return;
+  const int k1 = min(n_keys, k0 + p.chunk_keys);
+  const int n_splits_b = (n_keys + p.chunk_keys - 1) / p.chunk_keys;
+  const int nwc = (blockDim.x >> 5) - 1;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sK = smem;
+  uint8_t* sV = smem + kAttnStages * C::kKVBytes;
+  bf16* sQ = reinterpret_cast<bf16*>(sV + kAttnStages * C::kKVBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sQ + nwc * 16 * C::kQStride);
+  uint64_t* empty = full + kAttnStages;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kAttnStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], nwc);
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  const int n_tiles = (k1 - k0 + kAttnTileKeys - 1) / kAttnTileKeys;
+
+  if (warp == nwc) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      const int* bt = p.block_table + static_cast<size_t>(b) * p.W;
+      uint32_t stage = 0, phase = 0;
+      for (int t = 0; t < n_tiles; ++t) {
+        const int t0 = k0 + t * kAttnTileKeys;
+        const int nvalid = min(kAttnTileKeys, k1 - t0);
+        const int npages = (nvalid + 15) >> 4;
+        if (!mbar_wait(&empty[stage], phase ^ 1u, p.err)) break;
+        mbar_arrive_expect_tx(&full[stage], static_cast<uint32_t>(npages * C::kBoxesPerPage *
+                                                                  C::kBoxBytes * 2));
+        for (int j = 0; j < npages; ++j) {
+          const int pg = (t0 >> 4) + j;
+          int y;
+          if (pg >= p.W) {
+            raise_error(p.err, DFLASH_DEVERR_TABLE);
+            y = -16;  // fully out of bounds: TMA fills zeros
+          } else {
+            const int page = bt[pg];
+            if (page < 0 || page >= p.num_pages) {
+              raise_error(p.err, DFLASH_DEVERR_SLOT);
+              y = -16;
+            } else {
+              y = (page * p.Hkv + h) * 16;
+            }
+          }
+#pragma unroll
+          for (int hf = 0; hf < C::kBoxesPerPage; ++hf) {
+            const uint32_t off = (j * C::kBoxesPerPage + hf) * C::kBoxBytes;
+            tma_load_2d(sK + stage * C::kKVBytes + off, &tmK, &full[stage], hf * 64, y);
+            tma_load_2d(sV + stage * C::kKVBytes + off, &tmV, &full[stage], hf * 64, y);
+          }
+        }
+        if (++stage == kAttnStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------- compute warps
+  // Q rows of this warp: r = i * G + g  ->  q[(b*bs + i), h*G + g, :]
+  bf16* sQw = sQ + warp * 16 * C::kQStride;
+  for (int e = lane; e < 16 * (D / 8); e += 32) {
+    const int rr = e / (D / 8), c = e - rr * (D / 8);
+    const int r = warp * 16 + rr;
+    uint4 val = make_uint4(0, 0, 0, 0);
+    if (r < p.R) {
+      const int i = r / p.G, g = r - (r / p.G) * p.G;
+      const bf16* src = p.q + (static_cast<size_t>(b * p.bs + i) * p.Hq + h * p.G + g) * D;
+      val = *reinterpret_cast<const uint4*>(src + c * 8);
+    }
+    *reinterpret_cast<uint4*>(sQw + rr * C::kQStride + c * 8) = val;
+  }
+  __syncwarp();
+  uint32_t qa[D / 16][4];
+#pragma unroll
+  for (int ks = 0; ks < D / 16; ++ks) {
+    const int row = ((lane >> 3) & 1) * 8 + (lane & 7);
+    const int col = ks * 16 + (lane >> 4) * 8;
+    ldmatrix_x4(smem_u32(sQw + row * C::kQStride + col), qa[ks][0], qa[ks][1], qa[ks][2],
+                qa[ks][3]);
+  }
+
+  float o[D / 8][4];
+#pragma unroll
+  for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+  float m_run[2] = {-INFINITY, -INFINITY};
+  float l_run[2] = {0.f, 0.f};
+
+  uint32_t stage = 0, phase = 0;
+  for (int t = 0; t < n_tiles; ++t) {
+    const int t0 = k0 + t * kAttnTileKeys;
+    const int nvalid = min(kAttnTileKeys, k1 - t0);
+    if (!mbar_wait(&full[stage], phase, p.err)) break;
+    const uint32_t kbase = smem_u32(sK + stage * C::kKVBytes);
+    const uint32_t vbase = smem_u32(sV + stage * C::kKVBytes);
+
+    if (nvalid & 15) {
+      // Rows past the last key of a partly used page may hold anything
+      // (including NaN bit patterns); zero them so that P = 0 rows add 0.
+      const int jp = nvalid >> 4, r0 = nvalid & 15;
+      uint8_t* vb = sV + stage * C::kKVBytes;
+      const int n16 = (16 - r0) * C::kBoxesPerPage * 8;
+      for (int e = lane; e < n16; e += 32) {
+        const int hf = e / ((16 - r0) * 8);
+        const int rem = e - hf * (16 - r0) * 8;
+        const int rr = r0 + rem / 8, cc = rem & 7;
+        *reinterpret_cast<uint4*>(vb + (jp * C::kBoxesPerPage + hf) * C::kBoxBytes + rr * 128 +
+                                  cc * 16) = make_uint4(0, 0, 0, 0);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+    }
+
+    // S = Q K^T over the 64 keys of the tile (8 blocks of 8 keys)
+    float s[8][4];
+#pragma unroll
+    for (int nb = 0; nb < 8; ++nb) s[nb][0] = s[nb][1] = s[nb][2] = s[nb][3] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+#pragma unroll
+      for (int nbp = 0; nbp < 4; ++nbp) {
+        const int j = lane >> 3;
+        const int kt = (nbp * 2 + (j >> 1)) * 8 + (lane & 7);
+        const int c = ks * 2 + (j & 1);
+        uint32_t b00, b01, b10, b11;
+        ldmatrix_x4(kbase + kv_off<D>(kt, c), b00, b01, b10, b11);
+        mma_bf16_16816(s[2 * nbp], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b00, b01);
+        mma_bf16_16816(s[2 * nbp + 1], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b10, b11);
+      }
+    }
+
+    // scale into the log2 domain, mask keys past the range, online softmax
+    float mx[2] = {m_run[0], m_run[1]};
+#pragma unroll
+    for (int nb = 0; nb < 8; ++nb) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int kt = nb * 8 + 2 * (lane & 3) + (e & 1);
+        const float v = s[nb][e] * p.scale_log2;
+        s[nb][e] = (kt < nvalid) ? v : -INFINITY;
+        mx[e >> 1] = fmaxf(mx[e >> 1], s[nb][e]);
+      }
+    }
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      mx[hh] = fmaxf(mx[hh], __shfl_xor_sync(0xffffffffu, mx[hh], 1));
+      mx[hh] = fmaxf(mx[hh], __shfl_xor_sync(0xffffffffu, mx[hh], 2));
+    }
+    float ref[2], alpha[2];
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      ref[hh] = (mx[hh] == -INFINITY) ? 0.f : mx[hh];
+      alpha[hh] = exp2f(m_run[hh] - ref[hh]);  // m_run = -inf -> 0
+      m_run[hh] = mx[hh];
+      l_run[hh] *= alpha[hh];
+    }
+#pragma unroll
+    for (int i = 0; i < D / 8; ++i) {
+      o[i][0] *= alpha[0];
+      o[i][1] *= alpha[0];
+      o[i][2] *= alpha[1];
+      o[i][3] *= alpha[1];
+    }
+#pragma unroll
+    for (int nb = 0; nb < 8; ++nb) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float pv = exp2f(s[nb][e] - ref[e >> 1]);
+        s[nb][e] = pv;
+        l_run[e >> 1] += pv;
+      }
+    }
+
+    // O += P V, 16 keys (one page) per k-step
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      if (kk * 16 < nvalid) {
+        const uint32_t a0 = pack_bf16x2(s[2 * kk][0], s[2 * kk][1]);
+        const uint32_t a1 = pack_bf16x2(s[2 * kk][2], s[2 * kk][3]);
+        const uint32_t a2 = pack_bf16x2(s[2 * kk + 1][0], s[2 * kk + 1][1]);
+        const uint32_t a3 = pack_bf16x2(s[2 * kk + 1][2], s[2 * kk + 1][3]);
+#pragma unroll
+        for (int dbp = 0; dbp < D / 16; ++dbp) {
+          const int j = lane >> 3;
+          const int kt = kk * 16 + (j & 1) * 8 + (lane & 7);
+          const int c = dbp * 2 + (j >> 1);
+          uint32_t b0, b1, b2, b3;
+          ldmatrix_x4_trans(vbase + kv_off<D>(kt, c), b0, b1, b2, b3);
+          mma_bf16_16816(o[2 * dbp], a0, a1, a2, a3, b0, b1);
+          mma_bf16_16816(o[2 * dbp + 1], a0, a1, a2, a3, b2, b3);
+        }
+      }
+    }
+
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[stage]);
+    if (++stage == kAttnStages) {
+      stage = 0;
+      phase ^= 1u;
+    }
+  }
+
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+    l_run[hh] += __shfl_xor_sync(0xffffffffu, l_run[hh], 1);
+    l_run[hh] += __shfl_xor_sync(0xffffffffu, l_run[hh], 2);
+  }
+
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+    const int r = warp * 16 + (lane >> 2) + hh * 8;
+    if (r >= p.R) continue;
+    if (n_splits_b == 1) {
+      const int i = r / p.G, g = r - (r / p.G) * p.G;
+      bf16* dst = p.o + (static_cast<size_t>(b * p.bs + i) * p.Hq + h * p.G + g) * D;
+      const float inv = 1.f / l_run[hh];
+#pragma unroll
+      for (int db = 0; db < D / 8; ++db) {
+        const int d = db * 8 + 2 * (lane & 3);
+        *reinterpret_cast<uint32_t*>(dst + d) =
+            pack_bf16x2(o[db][2 * hh] * inv, o[db][2 * hh + 1] * inv);
+      }
+    } else {
+      const size_t prow = (static_cast<size_t>(split) * p.B + b) * p.Hkv + h;
+      float* dst = p.part_o + (prow * p.R + r) * D;
+#pragma unroll
+      for (int db = 0; db < D / 8; ++db) {
+        const int d = db * 8 + 2 * (lane & 3);
+        *reinterpret_cast<float2*>(dst + d) = make_float2(o[db][2 * hh], o[db][2 * hh + 1]);
+      }
+      if ((lane & 3) == 0) {
+        *reinterpret_cast<float2*>(p.part_ml + (prow * p.R + r) * 2) =
+            make_float2(m_run[hh], l_run[hh]);
+      }
+    }
+  }
+}
+
+// Merge the split partials of requests that needed more than one split:
+//   m = max_s m_s,  w_s = 2^(m_s - m),  o = sum_s w_s O_s / sum_s w_s l_s
+// One CTA per (request, kv head); splits are summed in index order.
+template <int D>
+__global__ void __launch_bounds__(256) attn_combine_kernel(const AttnParams p) {
+  const int h = blockIdx.x, b = blockIdx.y;
+  const int n_keys = p.seq_lens[b] + p.bs;
+  const int ns = (n_keys + p.chunk_keys - 1) / p.chunk_keys;
+  if (ns <= 1) return;
+  const int nsc = min(ns, p.max_splits);
+  for (int e = threadIdx.x; e < p.R * (D / 4); e += blockDim.x) {
+    const int r = e / (D / 4), d = (e - r * (D / 4)) * 4;
+    float mmax = -INFINITY;
+    for (int s = 0; s < nsc; ++s) {
+      const size_t prow = (static_cast<size_t>(s) * p.B + b) * p.Hkv + h;
+      mmax = fmaxf(mmax, p.part_ml[(prow * p.R + r) * 2]);
+    }
+    float l = 0.f, a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    for (int s = 0; s < nsc; ++s) {
+      const size_t prow = (static_cast<size_t>(s) * p.B + b) * p.Hkv + h;
+      const float2 ml = *reinterpret_cast<const float2*>(p.part_ml + (prow * p.R + r) * 2);
+      const float w = exp2f(ml.x - mmax);
+      const float4 ov = *reinterpret_cast<const float4*>(p.part_o + (prow * p.R + r) * D + d);
+      l += w * ml.y;
+      a0 += w * ov.x;
+      a1 += w * ov.y;
+      a2 += w * ov.z;
+      a3 += w * ov.w;
+    }
+    const float inv = 1.f / l;
+    const int i = r / p.G, g = r - (r / p.G) * p.G;
+    bf16* dst = p.o + (static_cast<size_t>(b * p.bs + i) * p.Hq + h * p.G + g) * D + d;
+    *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(a0 * inv, a1 * inv),
+                                                pack_bf16x2(a2 * inv, a3 * inv));
+  }
+}
+
+}  // namespace dflash

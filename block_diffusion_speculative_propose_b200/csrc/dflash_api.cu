@@ -1,0 +1,1002 @@
+// dflash_api.cu — the C ABI declared in include/dflash.h: argument checking,
+// handle / weight packing, launch planning (GEMM tiles and split-K, attention
+// key splits), TMA descriptor construction and the launch sequences of
+// inject / propose / verify.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <new>
+#include <tuple>
+#include <vector>
+
+#include "attention.cuh"
+#include "dflash.h"
+#include "gemm_tcgen05.cuh"
+#include "small_kernels.cuh"
+
+using namespace dflash;
+
+namespace {
+
+constexpr int kCounterSlots = 1 << 16;
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t v, size_t a = kAlign) { return (v + a - 1) / a * a; }
+int cdiv(int a, int b) { return (a + b - 1) / b; }
+
+// ---------------------------------------------------------------------------
+// driver entry point for tensor-map encoding (no link-time libcuda dependency)
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 view [rows][cols] (row pitch cols * 2 bytes), box [box_rows][64],
+// 128-byte swizzle.  Out-of-range box rows read as zeros.
+bool make_tmap(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t cols,
+               uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides,
+            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------------------
+// GEMM planning
+// ---------------------------------------------------------------------------
+struct GemmPlan {
+  int BN = 0, splits = 1, kb_per_split = 0, m_tiles = 0, n_tiles = 0, k_blocks = 0, units = 0,
+      grid = 0;
+  size_t partial_bytes = 0;
+};
+
+// Picks the tile width BN (a multiple of the epilogue group) and the K-split
+// count by minimising a per-SM time estimate: the busiest SM runs
+// ceil(units / SMs) units, each bounded by its weight bytes (HBM) or its
+// padded 128-row MMA work (tensor pipe), plus a fixed per-unit cost; splitting
+// K adds the round trip of fp32 partials.
+GemmPlan plan_gemm(int M, int N, int K, int group, int num_sms) {
+  GemmPlan best;
+  double best_t = 1e300;
+  const int k_blocks = K / kGemmBK;
+  const int m_tiles = cdiv(M, kGemmBM);
+  const double bw_sm = 6.5e12 / 148.0 * 1.6;  // bytes/s one SM can pull when peers idle
+  const double fl_sm = 1.6e15 / 148.0;
+  const double hbm = 6.5e12;
+  const int bns[4] = {256, 128, 64, 32};
+  for (int bi = 0; bi < 4; ++bi) {
+    const int BN = bns[bi];
+    if (BN < group || BN % group) continue;
+    const int n_tiles = cdiv(N, BN);
+    for (int S = 1; S <= 16; ++S) {
+      if (S > 1 && (m_tiles > 1 || k_blocks / S < 4)) break;
+      if (S > 1 && m_tiles * n_tiles > kCounterSlots) break;
+      const int kbps = cdiv(k_blocks, S);
+      const int splits = cdiv(k_blocks, kbps);
+      if (splits != S) continue;
+      const int units = m_tiles * n_tiles * S;
+      const int rounds = cdiv(units, num_sms);
+      const double kspan = static_cast<double>(kbps) * kGemmBK;
+      const double rows = std::min(M, kGemmBM);
+      const double unit_bytes = BN * kspan * 2.0 + rows * kspan * 2.0 * 0.25;
+      const double unit_flops = 2.0 * kGemmBM * BN * kspan;
+      double t = rounds * (std::max(unit_bytes / bw_sm, unit_flops / fl_sm) + 0.6e-6);
+      const double total_w = static_cast<double>(N) * K * 2.0;
+      t = std::max(t, total_w / hbm);
+      if (S > 1) t += static_cast<double>(S) * M * N * 4.0 * 2.0 / hbm + 1.0e-6;
+      if (t < best_t * 0.999) {
+        best_t = t;
+        best.BN = BN;
+        best.splits = S;
+        best.kb_per_split = kbps;
+        best.m_tiles = m_tiles;
+        best.n_tiles = n_tiles;
+        best.k_blocks = k_blocks;
+        best.units = units;
+        best.grid = std::min(units, num_sms);
+        best.partial_bytes = S > 1 ? static_cast<size_t>(S) * M * N * 4 : 0;
+      }
+    }
+  }
+  return best;
+}
+
+// ---------------------------------------------------------------------------
+// attention planning
+// ---------------------------------------------------------------------------
+struct AttnPlan {
+  int chunk_keys = 0, max_splits = 0, R = 0, nwc = 0;
+  size_t part_o_bytes = 0, part_ml_bytes = 0;
+};
+
+AttnPlan plan_attention(int B, int Hkv, int W, int P, int bs, int G, int D, int num_sms) {
+  AttnPlan a;
+  const int keys_max = W * P;
+  const double est = static_cast<double>(B) * Hkv * keys_max;
+  int chunk = static_cast<int>(std::ceil(est / (4.0 * num_sms)));
+  chunk = (chunk + kAttnTileKeys - 1) / kAttnTileKeys * kAttnTileKeys;
+  chunk = std::max(128, std::min(8192, chunk));
+  a.chunk_keys = chunk;
+  a.max_splits = cdiv(keys_max, chunk);
+  a.R = bs * G;
+  a.nwc = cdiv(a.R, 16);
+  a.part_o_bytes =
+      a.max_splits > 1 ? static_cast<size_t>(a.max_splits) * B * Hkv * a.R * D * 4 : 0;
+  a.part_ml_bytes =
+      a.max_splits > 1 ? static_cast<size_t>(a.max_splits) * B * Hkv * a.R * 2 * 4 : 0;
+  return a;
+}
+
+// ---------------------------------------------------------------------------
+// error helpers
+// ---------------------------------------------------------------------------
+#define DF_CUDA(expr)                                   \
+  do {                                                  \
+    if ((expr) != cudaSuccess) return DFLASH_ERR_CUDA;  \
+  } while (0)
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// handle
+// ---------------------------------------------------------------------------
+struct dflash_handle {
+  dflash_config cfg{};
+  std::vector<int> target_layer_ids;
+  int device = 0;
+  int num_sms = 148;
+  // aliased caller weights
+  const bf16 *fc_w = nullptr, *hidden_norm_w = nullptr, *embed = nullptr, *lm_head = nullptr,
+             *final_norm_w = nullptr;
+  std::vector<const bf16*> in_norm_w, post_norm_w, wo, q_norm_w, k_norm_w, w_down;
+  // packed copies owned by the handle
+  std::vector<bf16*> wqkv, wgu;
+  bf16* wkv = nullptr;      // [L * 2 * Hkv * D, H]
+  bf16* knorm_all = nullptr;  // [L, D]
+  float2* rope = nullptr;   // [max_position, D/2]
+  unsigned* dev_err = nullptr;
+  unsigned* counters = nullptr;
+  std::mutex mu;
+  std::map<std::tuple<const void*, uint64_t, uint64_t, uint32_t>, CUtensorMap> tmaps;
+
+  bool tmap(CUtensorMap* out, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    std::lock_guard<std::mutex> lk(mu);
+    auto key = std::make_tuple(ptr, rows, cols, box_rows);
+    auto it = tmaps.find(key);
+    if (it != tmaps.end()) {
+      *out = it->second;
+      return true;
+    }
+    if (tmaps.size() > 8192) tmaps.clear();
+    if (!make_tmap(out, ptr, rows, cols, box_rows)) return false;
+    tmaps.emplace(key, *out);
+    return true;
+  }
+};
+
+namespace {
+
+void free_handle(dflash_handle* h) {
+  if (!h) return;
+  for (auto p : h->wqkv) cudaFree(p);
+  for (auto p : h->wgu) cudaFree(p);
+  cudaFree(h->wkv);
+  cudaFree(h->knorm_all);
+  cudaFree(h->rope);
+  cudaFree(h->dev_err);
+  cudaFree(h->counters);
+  delete h;
+}
+
+// ---------------------------------------------------------------------------
+// GEMM launch
+// ---------------------------------------------------------------------------
+template <int BN, class Epi>
+cudaError_t set_gemm_attr() {
+  return cudaFuncSetAttribute(gemm_tcgen05_kernel<BN, Epi>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              GemmCfg<BN>::kSmemBytes);
+}
+
+template <class Epi>
+cudaError_t set_gemm_attrs_all() {
+  cudaError_t e = cudaSuccess;
+  if constexpr (256 % Epi::kGroup == 0)
+    if ((e = set_gemm_attr<256, Epi>()) != cudaSuccess) return e;
+  if constexpr (128 % Epi::kGroup == 0)
+    if ((e = set_gemm_attr<128, Epi>()) != cudaSuccess) return e;
+  if constexpr (Epi::kGroup <= 64)
+    if ((e = set_gemm_attr<64, Epi>()) != cudaSuccess) return e;
+  if constexpr (Epi::kGroup <= 32)
+    if ((e = set_gemm_attr<32, Epi>()) != cudaSuccess) return e;
+  return e;
+}
+
+template <int BN, class Epi>
+void launch_gemm_bn(const CUtensorMap& ta, const CUtensorMap& tw, const GemmParams& gp,
+                    const Epi& epi, int grid, cudaStream_t st) {
+  gemm_tcgen05_kernel<BN, Epi>
+      <<<grid, kGemmThreads, GemmCfg<BN>::kSmemBytes, st>>>(ta, tw, gp, epi);
+}
+
+// D = A[M, K] * W[N, K]^T with epilogue `epi`.  `partials` must hold
+// plan.partial_bytes.
+template <class Epi>
+dflash_status run_gemm(dflash_handle* h, const void* A, int M, int K, const void* Wt, int N,
+                       const Epi& epi, float* partials, size_t partial_cap, cudaStream_t st,
+                       int force_bn = 0, int force_splits = 0) {
+  if (M <= 0) return DFLASH_OK;
+  GemmPlan pl = plan_gemm(M, N, K, Epi::kGroup, h->num_sms);
+  if (force_bn || force_splits) {
+    const int BN = force_bn ? force_bn : pl.BN;
+    const int S = force_splits ? force_splits : pl.splits;
+    if ((BN != 32 && BN != 64 && BN != 128 && BN != 256) || BN % Epi::kGroup)
+      return DFLASH_ERR_INVALID_ARG;
+    pl.BN = BN;
+    pl.k_blocks = K / kGemmBK;
+    pl.m_tiles = cdiv(M, kGemmBM);
+    pl.n_tiles = cdiv(N, BN);
+    if (S < 1 || S > pl.k_blocks) return DFLASH_ERR_INVALID_ARG;
+    if (S > 1 && pl.m_tiles * pl.n_tiles > kCounterSlots) return DFLASH_ERR_UNSUPPORTED_SHAPE;
+    pl.kb_per_split = cdiv(pl.k_blocks, S);
+    pl.splits = cdiv(pl.k_blocks, pl.kb_per_split);
+    pl.units = pl.m_tiles * pl.n_tiles * pl.splits;
+    pl.grid = std::min(pl.units, h->num_sms);
+    pl.partial_bytes = pl.splits > 1 ? static_cast<size_t>(pl.splits) * M * N * 4 : 0;
+  }
+  if (pl.BN == 0) return DFLASH_ERR_UNSUPPORTED_SHAPE;
+  if (pl.partial_bytes > partial_cap) return DFLASH_ERR_WORKSPACE;
+  CUtensorMap ta, tw;
+  if (!h->tmap(&ta, A, M, K, kGemmBM)) return DFLASH_ERR_CUDA;
+  if (!h->tmap(&tw, Wt, N, K, pl.BN)) return DFLASH_ERR_CUDA;
+  GemmParams gp;
+  gp.M = M;
+  gp.N = N;
+  gp.K = K;
+  gp.m_tiles = pl.m_tiles;
+  gp.n_tiles = pl.n_tiles;
+  gp.k_blocks = pl.k_blocks;
+  gp.splits = pl.splits;
+  gp.kb_per_split = pl.kb_per_split;
+  gp.num_units = pl.units;
+  gp.partials = partials;
+  gp.counters = h->counters;
+  gp.err = h->dev_err;
+  switch (pl.BN) {
+    case 256:
+      if constexpr (256 % Epi::kGroup == 0) launch_gemm_bn<256>(ta, tw, gp, epi, pl.grid, st);
+      break;
+    case 128:
+      if constexpr (128 % Epi::kGroup == 0) launch_gemm_bn<128>(ta, tw, gp, epi, pl.grid, st);
+      break;
+    case 64:
+      if constexpr (Epi::kGroup <= 64) launch_gemm_bn<64>(ta, tw, gp, epi, pl.grid, st);
+      break;
+    case 32:
+      if constexpr (Epi::kGroup <= 32) launch_gemm_bn<32>(ta, tw, gp, epi, pl.grid, st);
+      break;
+    default:
+      return DFLASH_ERR_UNSUPPORTED_SHAPE;
+  }
+  return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// attention launch
+// ---------------------------------------------------------------------------
+template <int D>
+cudaError_t set_attn_attrs() {
+  return cudaFuncSetAttribute(attn_block_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              AttnCfg<D>::smem_bytes(kAttnMaxComputeWarps));
+}
+
+template <int D>
+dflash_status run_attention(dflash_handle* h, const AttnPlan& ap, AttnParams prm,
+                            const void* kc, const void* vc, int num_pages, cudaStream_t st) {
+  const dflash_config& c = h->cfg;
+  CUtensorMap tk, tv;
+  const uint64_t rows = static_cast<uint64_t>(num_pages) * c.n_kv_heads * c.page_size;
+  // box: 16 rows (one page of one head) x 64 columns
+  if (!h->tmap(&tk, kc, rows, D, 16)) return DFLASH_ERR_CUDA;
+  if (!h->tmap(&tv, vc, rows, D, 16)) return DFLASH_ERR_CUDA;
+  dim3 grid(ap.max_splits, c.n_kv_heads, prm.B);
+  const int threads = 32 * (ap.nwc + 1);
+  attn_block_kernel<D><<<grid, threads, AttnCfg<D>::smem_bytes(ap.nwc), st>>>(tk, tv, prm);
+  if (ap.max_splits > 1) attn_combine_kernel<D><<<dim3(c.n_kv_heads, prm.B), 256, 0, st>>>(prm);
+  return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// workspace layouts
+// ---------------------------------------------------------------------------
+struct InjectWs {
+  size_t fcx = 0, ctx = 0, partial = 0, total = 0, partial_cap = 0;
+};
+InjectWs inject_layout(const dflash_handle* h, int n) {
+  const dflash_config& c = h->cfg;
+  InjectWs w;
+  size_t off = 0;
+  w.fcx = off;
+  off += align_up(static_cast<size_t>(n) * c.hidden * 4);
+  w.ctx = off;
+  off += align_up(static_cast<size_t>(n) * c.hidden * 2);
+  size_t cap = 0;
+  for (int m = 1; m <= n; m = (m < 256 ? m + 1 : m * 2)) {
+    const int mm = std::min(m, n);
+    cap = std::max(cap, plan_gemm(mm, c.hidden, c.n_target_layers * c.hidden, 32, h->num_sms)
+                            .partial_bytes);
+    cap = std::max(cap, plan_gemm(mm, c.n_layers * 2 * c.n_kv_heads * c.head_dim, c.hidden,
+                                  c.head_dim, h->num_sms)
+                            .partial_bytes);
+  }
+  w.partial = off;
+  w.partial_cap = cap;
+  off += align_up(cap);
+  w.total = off;
+  return w;
+}
+
+struct ProposeWs {
+  size_t x = 0, nrm = 0, q = 0, o = 0, hm = 0, frows = 0, keys = 0, part_o = 0, part_ml = 0,
+         partial = 0, total = 0, partial_cap = 0, part_o_cap = 0, part_ml_cap = 0;
+};
+size_t propose_partial_need(const dflash_handle* h, int B) {
+  const dflash_config& c = h->cfg;
+  const int M = B * c.block_size, MK = B * (c.block_size - 1);
+  const int D = c.head_dim, Hq = c.n_q_heads, Hkv = c.n_kv_heads, H = c.hidden;
+  size_t cap = 0;
+  cap = std::max(cap, plan_gemm(M, (Hq + 2 * Hkv) * D, H, D, h->num_sms).partial_bytes);
+  cap = std::max(cap, plan_gemm(M, H, Hq * D, 32, h->num_sms).partial_bytes);
+  cap = std::max(cap, plan_gemm(M, 2 * c.intermediate, H, 32, h->num_sms).partial_bytes);
+  cap = std::max(cap, plan_gemm(M, H, c.intermediate, 32, h->num_sms).partial_bytes);
+  cap = std::max(cap, plan_gemm(MK, c.vocab, H, 32, h->num_sms).partial_bytes);
+  return cap;
+}
+ProposeWs propose_layout(const dflash_handle* h, int B, int W) {
+  const dflash_config& c = h->cfg;
+  const int bs = c.block_size, K = bs - 1, M = B * bs, MK = B * K;
+  const int D = c.head_dim, Hq = c.n_q_heads, Hkv = c.n_kv_heads, H = c.hidden;
+  ProposeWs w;
+  size_t off = 0;
+  auto take = [&off](size_t bytes) {
+    const size_t at = off;
+    off += align_up(bytes);
+    return at;
+  };
+  w.x = take(static_cast<size_t>(M) * H * 4);
+  w.nrm = take(static_cast<size_t>(M) * H * 2);
+  w.q = take(static_cast<size_t>(M) * Hq * D * 2);
+  w.o = take(static_cast<size_t>(M) * Hq * D * 2);
+  w.hm = take(static_cast<size_t>(M) * c.intermediate * 2);
+  w.frows = take(static_cast<size_t>(MK) * H * 2);
+  w.keys = take(static_cast<size_t>(MK) * 8);
+  size_t po = 0, pm = 0, pc = 0;
+  for (int b = 1; b <= B; b = (b < 256 ? b + 1 : b * 2)) {
+    const int bb = std::min(b, B);
+    const AttnPlan ap = plan_attention(bb, Hkv, W, c.page_size, bs, Hq / Hkv, D, h->num_sms);
+    po = std::max(po, ap.part_o_bytes);
+    pm = std::max(pm, ap.part_ml_bytes);
+    pc = std::max(pc, propose_partial_need(h, bb));
+  }
+  w.part_o = take(po);
+  w.part_ml = take(pm);
+  w.part_o_cap = po;
+  w.part_ml_cap = pm;
+  w.partial = take(pc);
+  w.partial_cap = pc;
+  w.total = off;
+  return w;
+}
+
+template <class T>
+T* at(void* base, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(base) + off);
+}
+
+dflash_status set_device_of(const void* p) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess || a.type != cudaMemoryTypeDevice) {
+    cudaGetLastError();
+    return DFLASH_ERR_INVALID_ARG;
+  }
+  DF_CUDA(cudaSetDevice(a.device));
+  return DFLASH_OK;
+}
+
+}  // namespace
+
+namespace {
+struct VerifyPlan {
+  int chunks = 1, chunk_len = 0;
+  size_t bytes = 0;
+};
+VerifyPlan plan_verify(int B, int K, int V) {
+  VerifyPlan v;
+  const int rows = B * (K + 1);
+  int chunks = std::max(1, cdiv(4 * 148, std::max(rows, 1)));
+  chunks = std::min(chunks, std::max(1, V / 4096));
+  int len = cdiv(V, chunks);
+  len = (len + 3) / 4 * 4;
+  v.chunk_len = len;
+  v.chunks = cdiv(V, len);
+  v.bytes = align_up(static_cast<size_t>(rows) * v.chunks * 8);
+  return v;
+}
+}  // namespace
+
+namespace {
+template <int D>
+dflash_status propose_layers(dflash_handle* h, const ProposeWs& lw, void* ws,
+                             const int32_t* seq_lens, const int32_t* block_table, int B, int W,
+                             void* const* k_cache, void* const* v_cache, int num_pages,
+                             cudaStream_t st) {
+  const dflash_config& c = h->cfg;
+  const int bs = c.block_size, M = B * bs, H = c.hidden, Hq = c.n_q_heads, Hkv = c.n_kv_heads,
+            I = c.intermediate, K = bs - 1;
+  float* x = at<float>(ws, lw.x);
+  bf16* nrm = at<bf16>(ws, lw.nrm);
+  bf16* q = at<bf16>(ws, lw.q);
+  bf16* o = at<bf16>(ws, lw.o);
+  bf16* hm = at<bf16>(ws, lw.hm);
+  bf16* frows = at<bf16>(ws, lw.frows);
+  float* partial = at<float>(ws, lw.partial);
+  const AttnPlan ap = plan_attention(B, Hkv, W, c.page_size, bs, Hq / Hkv, D, h->num_sms);
+  if (ap.part_o_bytes > lw.part_o_cap || ap.part_ml_bytes > lw.part_ml_cap)
+    return DFLASH_ERR_WORKSPACE;
+  AttnParams prm;
+  prm.q = q;
+  prm.o = o;
+  prm.part_o = at<float>(ws, lw.part_o);
+  prm.part_ml = at<float>(ws, lw.part_ml);
+  prm.seq_lens = seq_lens;
+  prm.block_table = block_table;
+  prm.B = B;
+  prm.W = W;
+  prm.bs = bs;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.G = Hq / Hkv;
+  prm.R = ap.R;
+  prm.num_pages = num_pages;
+  prm.chunk_keys = ap.chunk_keys;
+  prm.max_splits = ap.max_splits;
+  prm.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
+  prm.err = h->dev_err;
+
+  for (int l = 0; l < c.n_layers; ++l) {
+    // QKV projection with q/k norm, RoPE and the block's paged K/V write
+    EpiQKV<D> eq;
+    eq.q = q;
+    eq.q_norm_w = h->q_norm_w[l];
+    eq.k_norm_w = h->k_norm_w[l];
+    eq.rope = h->rope;
+    eq.k_cache = static_cast<bf16*>(k_cache[l]);
+    eq.v_cache = static_cast<bf16*>(v_cache[l]);
+    eq.seq_lens = seq_lens;
+    eq.block_table = block_table;
+    eq.max_pos = c.max_position;
+    eq.W = W;
+    eq.bs = bs;
+    eq.Hq = Hq;
+    eq.Hkv = Hkv;
+    eq.P = c.page_size;
+    eq.num_pages = num_pages;
+    eq.eps = c.rms_eps;
+    eq.err = h->dev_err;
+    dflash_status s =
+        run_gemm(h, nrm, M, H, h->wqkv[l], (Hq + 2 * Hkv) * D, eq, partial, lw.partial_cap, st);
+    if (s != DFLASH_OK) return s;
+    // non-causal block attention over context + block
+    s = run_attention<D>(h, ap, prm, k_cache[l], v_cache[l], num_pages, st);
+    if (s != DFLASH_OK) return s;
+    // x += Wo o
+    EpiResidAdd er{x, H};
+    s = run_gemm(h, o, M, Hq * D, h->wo[l], H, er, partial, lw.partial_cap, st);
+    if (s != DFLASH_OK) return s;
+    rmsnorm_rows_kernel<<<M, 256, 0, st>>>(x, h->post_norm_w[l], nrm, H, c.rms_eps, 0, bs);
+    if (cudaGetLastError() != cudaSuccess) return DFLASH_ERR_CUDA;
+    // h = silu(gate) * up
+    EpiSwiGLU eg{hm, I};
+    s = run_gemm(h, nrm, M, H, h->wgu[l], 2 * I, eg, partial, lw.partial_cap, st);
+    if (s != DFLASH_OK) return s;
+    // x += Wd h
+    s = run_gemm(h, hm, M, I, h->w_down[l], H, er, partial, lw.partial_cap, st);
+    if (s != DFLASH_OK) return s;
+    if (l + 1 < c.n_layers) {
+      rmsnorm_rows_kernel<<<M, 256, 0, st>>>(x, h->in_norm_w[l + 1], nrm, H, c.rms_eps, 0, bs);
+    } else {
+      // final norm on the kept rows (block slots 1..bs-1) only
+      rmsnorm_rows_kernel<<<B * K, 256, 0, st>>>(x, h->final_norm_w, frows, H, c.rms_eps, K,
+                                                 bs);
+    }
+    if (cudaGetLastError() != cudaSuccess) return DFLASH_ERR_CUDA;
+  }
+  return DFLASH_OK;
+}
+}  // namespace
+
+// ===========================================================================
+// C ABI
+// ===========================================================================
+extern "C" {
+
+const char* dflash_status_string(dflash_status s) {
+  switch (s) {
+    case DFLASH_OK: return "DFLASH_OK";
+    case DFLASH_ERR_INVALID_ARG: return "DFLASH_ERR_INVALID_ARG";
+    case DFLASH_ERR_CUDA: return "DFLASH_ERR_CUDA";
+    case DFLASH_ERR_WORKSPACE: return "DFLASH_ERR_WORKSPACE";
+    case DFLASH_ERR_UNSUPPORTED_SHAPE: return "DFLASH_ERR_UNSUPPORTED_SHAPE";
+    case DFLASH_ERR_DEVICE_BOUNDS: return "DFLASH_ERR_DEVICE_BOUNDS";
+    case DFLASH_ERR_UNIMPLEMENTED: return "DFLASH_ERR_UNIMPLEMENTED";
+    case DFLASH_ERR_DEVICE_TIMEOUT: return "DFLASH_ERR_DEVICE_TIMEOUT";
+  }
+  return "DFLASH_ERR_UNKNOWN";
+}
+
+const char* dflash_version(void) { return "dflash-b200 0.1 (sm_100a)"; }
+
+dflash_status dflash_create(const dflash_config* cfg, const dflash_weights* w, int device,
+                            dflash_handle** out) {
+  if (!out) return DFLASH_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!cfg || !w) return DFLASH_ERR_INVALID_ARG;
+  const dflash_config& c = *cfg;
+  if (c.hidden <= 0 || c.n_layers <= 0 || c.n_q_heads <= 0 || c.n_kv_heads <= 0 ||
+      c.head_dim <= 0 || c.intermediate <= 0 || c.vocab <= 0 || c.n_target_layers <= 0 ||
+      c.block_size <= 0 || c.page_size <= 0 || c.max_position <= 0 || !(c.rms_eps >= 0.f) ||
+      !(c.rope_theta > 0.f))
+    return DFLASH_ERR_INVALID_ARG;
+  if (c.mask_token_id < 0 || c.mask_token_id >= c.vocab) return DFLASH_ERR_INVALID_ARG;
+  if (c.head_dim != 64 && c.head_dim != 128) return DFLASH_ERR_UNSUPPORTED_SHAPE;
+  if (c.hidden % 64 || (c.n_q_heads * c.head_dim) % 64 || c.intermediate % 64 ||
+      c.vocab % 32 || c.n_q_heads % c.n_kv_heads || c.page_size != 16 || c.block_size < 2 ||
+      c.block_size > 64 || c.n_layers > kMaxLayers)
+    return DFLASH_ERR_UNSUPPORTED_SHAPE;
+  if (c.block_size * (c.n_q_heads / c.n_kv_heads) > 16 * kAttnMaxComputeWarps)
+    return DFLASH_ERR_UNSUPPORTED_SHAPE;
+  const int L = c.n_layers;
+  if (!w->fc_w || !w->hidden_norm_w || !w->embed || !w->lm_head || !w->final_norm_w ||
+      !w->in_norm_w || !w->post_norm_w || !w->wq || !w->wk || !w->wv || !w->wo ||
+      !w->q_norm_w || !w->k_norm_w || !w->w_gate || !w->w_up || !w->w_down)
+    return DFLASH_ERR_INVALID_ARG;
+  for (int l = 0; l < L; ++l)
+    if (!w->in_norm_w[l] || !w->post_norm_w[l] || !w->wq[l] || !w->wk[l] || !w->wv[l] ||
+        !w->wo[l] || !w->q_norm_w[l] || !w->k_norm_w[l] || !w->w_gate[l] || !w->w_up[l] ||
+        !w->w_down[l])
+      return DFLASH_ERR_INVALID_ARG;
+  if (c.target_layer_ids) {
+    for (int t = 0; t < c.n_target_layers; ++t)
+      if (c.target_layer_ids[t] < 0) return DFLASH_ERR_INVALID_ARG;
+  }
+  if (!encode_fn()) return DFLASH_ERR_CUDA;
+
+  dflash_handle* h = new (std::nothrow) dflash_handle();
+  if (!h) return DFLASH_ERR_CUDA;
+  h->cfg = c;
+  if (c.target_layer_ids) h->target_layer_ids.assign(c.target_layer_ids, c.target_layer_ids + c.n_target_layers);
+  h->cfg.target_layer_ids = h->target_layer_ids.empty() ? nullptr : h->target_layer_ids.data();
+  h->device = device;
+  auto fail = [h](dflash_status s) {
+    free_handle(h);
+    return s;
+  };
+  if (cudaSetDevice(device) != cudaSuccess) return fail(DFLASH_ERR_CUDA);
+  if (cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess)
+    return fail(DFLASH_ERR_CUDA);
+  int major = 0;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, device);
+  if (major != 10) return fail(DFLASH_ERR_UNSUPPORTED_SHAPE);
+
+  const int H = c.hidden, D = c.head_dim, Hq = c.n_q_heads, Hkv = c.n_kv_heads,
+            I = c.intermediate;
+  h->fc_w = static_cast<const bf16*>(w->fc_w);
+  h->hidden_norm_w = static_cast<const bf16*>(w->hidden_norm_w);
+  h->embed = static_cast<const bf16*>(w->embed);
+  h->lm_head = static_cast<const bf16*>(w->lm_head);
+  h->final_norm_w = static_cast<const bf16*>(w->final_norm_w);
+  for (int l = 0; l < L; ++l) {
+    h->in_norm_w.push_back(static_cast<const bf16*>(w->in_norm_w[l]));
+    h->post_norm_w.push_back(static_cast<const bf16*>(w->post_norm_w[l]));
+    h->wo.push_back(static_cast<const bf16*>(w->wo[l]));
+    h->q_norm_w.push_back(static_cast<const bf16*>(w->q_norm_w[l]));
+    h->k_norm_w.push_back(static_cast<const bf16*>(w->k_norm_w[l]));
+    h->w_down.push_back(static_cast<const bf16*>(w->w_down[l]));
+  }
+
+  cudaStream_t st;
+  if (cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking) != cudaSuccess)
+    return fail(DFLASH_ERR_CUDA);
+  auto fail_st = [&](dflash_status s) {
+    cudaStreamSynchronize(st);
+    cudaStreamDestroy(st);
+    return fail(s);
+  };
+  const size_t rowb = static_cast<size_t>(H) * 2;
+  // QKV: [wq; wk; wv]
+  for (int l = 0; l < L; ++l) {
+    bf16* p = nullptr;
+    if (cudaMalloc(&p, static_cast<size_t>(Hq + 2 * Hkv) * D * rowb) != cudaSuccess)
+      return fail_st(DFLASH_ERR_CUDA);
+    h->wqkv.push_back(p);
+    if (cudaMemcpyAsync(p, w->wq[l], static_cast<size_t>(Hq) * D * rowb,
+                        cudaMemcpyDeviceToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(p + static_cast<size_t>(Hq) * D * H, w->wk[l],
+                        static_cast<size_t>(Hkv) * D * rowb, cudaMemcpyDeviceToDevice,
+                        st) != cudaSuccess ||
+        cudaMemcpyAsync(p + static_cast<size_t>(Hq + Hkv) * D * H, w->wv[l],
+                        static_cast<size_t>(Hkv) * D * rowb, cudaMemcpyDeviceToDevice,
+                        st) != cudaSuccess)
+      return fail_st(DFLASH_ERR_CUDA);
+  }
+  // gate / up interleaved in blocks of 16 rows: [g 16 | u 16] per 32 packed rows
+  for (int l = 0; l < L; ++l) {
+    bf16* p = nullptr;
+    if (cudaMalloc(&p, static_cast<size_t>(2 * I) * rowb) != cudaSuccess)
+      return fail_st(DFLASH_ERR_CUDA);
+    h->wgu.push_back(p);
+    if (cudaMemcpy2DAsync(p, 32 * rowb, w->w_gate[l], 16 * rowb, 16 * rowb, I / 16,
+                          cudaMemcpyDeviceToDevice, st) != cudaSuccess ||
+        cudaMemcpy2DAsync(p + 16 * static_cast<size_t>(H), 32 * rowb, w->w_up[l], 16 * rowb,
+                          16 * rowb, I / 16, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+      return fail_st(DFLASH_ERR_CUDA);
+  }
+  // all layers' K/V projections stacked: per layer [wk; wv]
+  const size_t kvrows = static_cast<size_t>(Hkv) * D;
+  if (cudaMalloc(&h->wkv, static_cast<size_t>(L) * 2 * kvrows * rowb) != cudaSuccess)
+    return fail_st(DFLASH_ERR_CUDA);
+  for (int l = 0; l < L; ++l) {
+    if (cudaMemcpyAsync(h->wkv + (2 * l) * kvrows * H, w->wk[l], kvrows * rowb,
+                        cudaMemcpyDeviceToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(h->wkv + (2 * l + 1) * kvrows * H, w->wv[l], kvrows * rowb,
+                        cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+      return fail_st(DFLASH_ERR_CUDA);
+  }
+  if (cudaMalloc(&h->knorm_all, static_cast<size_t>(L) * D * 2) != cudaSuccess)
+    return fail_st(DFLASH_ERR_CUDA);
+  for (int l = 0; l < L; ++l)
+    if (cudaMemcpyAsync(h->knorm_all + static_cast<size_t>(l) * D, w->k_norm_w[l],
+                        static_cast<size_t>(D) * 2, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+      return fail_st(DFLASH_ERR_CUDA);
+  if (cudaMalloc(&h->rope, static_cast<size_t>(c.max_position) * (D / 2) * sizeof(float2)) !=
+      cudaSuccess)
+    return fail_st(DFLASH_ERR_CUDA);
+  rope_table_kernel<<<c.max_position, 64, 0, st>>>(h->rope, c.max_position, D / 2,
+                                                    static_cast<double>(c.rope_theta));
+  if (cudaGetLastError() != cudaSuccess) return fail_st(DFLASH_ERR_CUDA);
+  if (cudaMalloc(&h->dev_err, sizeof(unsigned)) != cudaSuccess ||
+      cudaMemsetAsync(h->dev_err, 0, sizeof(unsigned), st) != cudaSuccess)
+    return fail_st(DFLASH_ERR_CUDA);
+  if (cudaMalloc(&h->counters, kCounterSlots * sizeof(unsigned)) != cudaSuccess ||
+      cudaMemsetAsync(h->counters, 0, kCounterSlots * sizeof(unsigned), st) != cudaSuccess)
+    return fail_st(DFLASH_ERR_CUDA);
+
+  // kernel attributes (set once, outside any stream capture)
+  if (set_gemm_attrs_all<EpiStoreF32>() != cudaSuccess ||
+      set_gemm_attrs_all<EpiResidAdd>() != cudaSuccess ||
+      set_gemm_attrs_all<EpiSwiGLU>() != cudaSuccess ||
+      set_gemm_attrs_all<EpiArgmax>() != cudaSuccess ||
+      set_gemm_attrs_all<EpiQKV<64>>() != cudaSuccess ||
+      set_gemm_attrs_all<EpiQKV<128>>() != cudaSuccess ||
+      set_gemm_attrs_all<EpiKVInject<64>>() != cudaSuccess ||
+      set_gemm_attrs_all<EpiKVInject<128>>() != cudaSuccess ||
+      set_attn_attrs<64>() != cudaSuccess || set_attn_attrs<128>() != cudaSuccess)
+    return fail_st(DFLASH_ERR_CUDA);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return fail_st(DFLASH_ERR_CUDA);
+  cudaStreamDestroy(st);
+  *out = h;
+  return DFLASH_OK;
+}
+
+void dflash_destroy(dflash_handle* h) {
+  if (!h) return;
+  cudaSetDevice(h->device);
+  free_handle(h);
+}
+
+size_t dflash_inject_workspace_bytes(const dflash_handle* h, int max_rows) {
+  if (!h || max_rows <= 0) return 0;
+  return inject_layout(h, max_rows).total;
+}
+
+size_t dflash_propose_workspace_bytes(const dflash_handle* h, int max_batch,
+                                      int max_pages_per_seq) {
+  if (!h || max_batch <= 0 || max_pages_per_seq <= 0) return 0;
+  return propose_layout(h, max_batch, max_pages_per_seq).total;
+}
+
+
+size_t dflash_verify_workspace_bytes(int B, int K, int V) {
+  if (B <= 0 || K < 0 || V <= 0) return 0;
+  return plan_verify(B, K, V).bytes;
+}
+
+dflash_status dflash_paged_slots(const int64_t* positions, const int64_t* req_ids, int n,
+                                 const int32_t* block_table, int max_pages_per_seq,
+                                 int page_size, int64_t* slots, void* stream) {
+  if (n < 0 || max_pages_per_seq <= 0 || page_size <= 0) return DFLASH_ERR_INVALID_ARG;
+  if (n == 0) return DFLASH_OK;
+  if (!positions || !req_ids || !block_table || !slots) return DFLASH_ERR_INVALID_ARG;
+  dflash_status s = set_device_of(slots);
+  if (s != DFLASH_OK) return s;
+  paged_slots_kernel<<<cdiv(n, 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      positions, req_ids, block_table, n, max_pages_per_seq, page_size, slots);
+  return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ERR_CUDA;
+}
+
+dflash_status dflash_inject_context(dflash_handle* h, const void* aux, const int64_t* positions,
+                                    const int64_t* slot_mapping, int n, void* const* k_cache,
+                                    void* const* v_cache, int num_pages, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
+  if (!h || n < 0) return DFLASH_ERR_INVALID_ARG;
+  if (n == 0) return DFLASH_OK;
+  const dflash_config& c = h->cfg;
+  if (!aux || !positions || !slot_mapping || !k_cache || !v_cache || num_pages <= 0 ||
+      !workspace)
+    return DFLASH_ERR_INVALID_ARG;
+  for (int l = 0; l < c.n_layers; ++l)
+    if (!k_cache[l] || !v_cache[l]) return DFLASH_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return DFLASH_ERR_INVALID_ARG;
+  const InjectWs lw = inject_layout(h, n);
+  if (workspace_bytes < lw.total) return DFLASH_ERR_WORKSPACE;
+  DF_CUDA(cudaSetDevice(h->device));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int H = c.hidden, D = c.head_dim;
+  float* fcx = at<float>(workspace, lw.fcx);
+  bf16* ctx = at<bf16>(workspace, lw.ctx);
+  float* partial = at<float>(workspace, lw.partial);
+
+  // (1) fc over the concatenated tapped states
+  EpiStoreF32 e1{fcx, H};
+  dflash_status s = run_gemm(h, aux, n, c.n_target_layers * H, h->fc_w, H, e1, partial,
+                             lw.partial_cap, st);
+  if (s != DFLASH_OK) return s;
+  // (2) hidden_norm
+  rmsnorm_rows_kernel<<<n, 256, 0, st>>>(fcx, h->hidden_norm_w, ctx, H, c.rms_eps, 0, 0);
+  if (cudaGetLastError() != cudaSuccess) return DFLASH_ERR_CUDA;
+  // (3) every layer's K/V at once, k_norm + RoPE, paged scatter
+  const int NKV = c.n_layers * 2 * c.n_kv_heads * D;
+  if (D == 128) {
+    EpiKVInject<128> e3{};
+    for (int l = 0; l < c.n_layers; ++l) {
+      e3.k_cache[l] = static_cast<bf16*>(k_cache[l]);
+      e3.v_cache[l] = static_cast<bf16*>(v_cache[l]);
+    }
+    e3.k_norm_w = h->knorm_all;
+    e3.rope = h->rope;
+    e3.positions = positions;
+    e3.slots = slot_mapping;
+    e3.max_pos = c.max_position;
+    e3.Hkv = c.n_kv_heads;
+    e3.P = c.page_size;
+    e3.num_pages = num_pages;
+    e3.eps = c.rms_eps;
+    e3.err = h->dev_err;
+    s = run_gemm(h, ctx, n, H, h->wkv, NKV, e3, partial, lw.partial_cap, st);
+  } else {
+    EpiKVInject<64> e3{};
+    for (int l = 0; l < c.n_layers; ++l) {
+      e3.k_cache[l] = static_cast<bf16*>(k_cache[l]);
+      e3.v_cache[l] = static_cast<bf16*>(v_cache[l]);
+    }
+    e3.k_norm_w = h->knorm_all;
+    e3.rope = h->rope;
+    e3.positions = positions;
+    e3.slots = slot_mapping;
+    e3.max_pos = c.max_position;
+    e3.Hkv = c.n_kv_heads;
+    e3.P = c.page_size;
+    e3.num_pages = num_pages;
+    e3.eps = c.rms_eps;
+    e3.err = h->dev_err;
+    s = run_gemm(h, ctx, n, H, h->wkv, NKV, e3, partial, lw.partial_cap, st);
+  }
+  return s;
+}
+
+
+dflash_status dflash_propose(dflash_handle* h, const int32_t* bonus_tokens,
+                             const int32_t* seq_lens, const int32_t* block_table, int B,
+                             int max_pages_per_seq, void* const* k_cache, void* const* v_cache,
+                             int num_pages, int32_t* draft_tokens, int32_t* block_tokens,
+                             float* logits_out, void* workspace, size_t workspace_bytes,
+                             void* stream) {
+  if (!h || B < 0) return DFLASH_ERR_INVALID_ARG;
+  if (B == 0) return DFLASH_OK;
+  const dflash_config& c = h->cfg;
+  if (!bonus_tokens || !seq_lens || !block_table || max_pages_per_seq <= 0 || !k_cache ||
+      !v_cache || num_pages <= 0 || !draft_tokens || !workspace)
+    return DFLASH_ERR_INVALID_ARG;
+  for (int l = 0; l < c.n_layers; ++l)
+    if (!k_cache[l] || !v_cache[l]) return DFLASH_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return DFLASH_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(B) * c.block_size > (1 << 24)) return DFLASH_ERR_UNSUPPORTED_SHAPE;
+  const ProposeWs lw = propose_layout(h, B, max_pages_per_seq);
+  if (workspace_bytes < lw.total) return DFLASH_ERR_WORKSPACE;
+  DF_CUDA(cudaSetDevice(h->device));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int bs = c.block_size, K = bs - 1, M = B * bs, H = c.hidden;
+  float* x = at<float>(workspace, lw.x);
+  bf16* nrm = at<bf16>(workspace, lw.nrm);
+  bf16* frows = at<bf16>(workspace, lw.frows);
+  unsigned long long* keys = at<unsigned long long>(workspace, lw.keys);
+  float* partial = at<float>(workspace, lw.partial);
+
+  embed_norm_kernel<<<M, 256, 0, st>>>(bonus_tokens, c.mask_token_id, h->embed, h->in_norm_w[0],
+                                       x, nrm, keys, B * K, bs, H, c.vocab, c.rms_eps,
+                                       h->dev_err);
+  if (cudaGetLastError() != cudaSuccess) return DFLASH_ERR_CUDA;
+  dflash_status s = (c.head_dim == 128)
+                        ? propose_layers<128>(h, lw, workspace, seq_lens, block_table, B,
+                                              max_pages_per_seq, k_cache, v_cache, num_pages, st)
+                        : propose_layers<64>(h, lw, workspace, seq_lens, block_table, B,
+                                             max_pages_per_seq, k_cache, v_cache, num_pages, st);
+  if (s != DFLASH_OK) return s;
+  // aliased target LM head with the greedy pick fused into its epilogue
+  EpiArgmax ea{keys, logits_out, c.vocab};
+  s = run_gemm(h, frows, B * K, H, h->lm_head, c.vocab, ea, partial, lw.partial_cap, st);
+  if (s != DFLASH_OK) return s;
+  argmax_finalize_kernel<<<cdiv(M, 256), 256, 0, st>>>(keys, bonus_tokens, draft_tokens,
+                                                       block_tokens, B, bs);
+  return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ERR_CUDA;
+}
+
+dflash_status dflash_verify_greedy(const int32_t* drafts, const float* target_logits, int B,
+                                   int K, int V, int32_t* out_tokens, int32_t* num_accepted,
+                                   int32_t* bonus, void* workspace, size_t workspace_bytes,
+                                   void* stream) {
+  if (B < 0 || K < 0 || V <= 0 || K > 128) return DFLASH_ERR_INVALID_ARG;
+  if (B == 0) return DFLASH_OK;
+  if ((K > 0 && !drafts) || !target_logits || !out_tokens || !num_accepted || !bonus ||
+      !workspace)
+    return DFLASH_ERR_INVALID_ARG;
+  const VerifyPlan vp = plan_verify(B, K, V);
+  if (workspace_bytes < vp.bytes) return DFLASH_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(target_logits) % 16 && V % 4 == 0)
+    return DFLASH_ERR_INVALID_ARG;
+  dflash_status s = set_device_of(out_tokens);
+  if (s != DFLASH_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  unsigned long long* part = static_cast<unsigned long long*>(workspace);
+  verify_partial_kernel<<<dim3(vp.chunks, B * (K + 1)), 256, 0, st>>>(target_logits, V,
+                                                                      vp.chunk_len, vp.chunks,
+                                                                      part);
+  verify_final_kernel<<<B, 32, 0, st>>>(part, vp.chunks, drafts, K, out_tokens, num_accepted,
+                                        bonus);
+  return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ERR_CUDA;
+}
+
+size_t dflash_linear_workspace_bytes(const dflash_handle* h, int M, int N, int K) {
+  if (!h || M <= 0 || N <= 0 || K <= 0) return 0;
+  return align_up(std::max<size_t>(plan_gemm(M, N, K, 32, h->num_sms).partial_bytes, kAlign));
+}
+
+dflash_status dflash_linear(dflash_handle* h, const void* A, const void* W, int M, int N, int K,
+                            float* out, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!h || M < 0 || N <= 0 || K <= 0) return DFLASH_ERR_INVALID_ARG;
+  if (M == 0) return DFLASH_OK;
+  if (!A || !W || !out || !workspace) return DFLASH_ERR_INVALID_ARG;
+  if (K % 64 || N % 32) return DFLASH_ERR_UNSUPPORTED_SHAPE;
+  if (reinterpret_cast<uintptr_t>(A) % 16 || reinterpret_cast<uintptr_t>(W) % 16 ||
+      reinterpret_cast<uintptr_t>(out) % 16)
+    return DFLASH_ERR_INVALID_ARG;
+  const size_t need = dflash_linear_workspace_bytes(h, M, N, K);
+  if (workspace_bytes < need) return DFLASH_ERR_WORKSPACE;
+  DF_CUDA(cudaSetDevice(h->device));
+  EpiStoreF32 e{out, N};
+  return run_gemm(h, A, M, K, W, N, e, static_cast<float*>(workspace), workspace_bytes,
+                  static_cast<cudaStream_t>(stream));
+}
+
+dflash_status dflash_linear_ex(dflash_handle* h, const void* A, const void* W, int M, int N,
+                               int K, float* out, int block_n, int splits, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+  if (!h || M < 0 || N <= 0 || K <= 0 || block_n < 0 || splits < 0)
+    return DFLASH_ERR_INVALID_ARG;
+  if (M == 0) return DFLASH_OK;
+  if (!A || !W || !out || !workspace) return DFLASH_ERR_INVALID_ARG;
+  if (K % 64 || N % 32) return DFLASH_ERR_UNSUPPORTED_SHAPE;
+  if (reinterpret_cast<uintptr_t>(A) % 16 || reinterpret_cast<uintptr_t>(W) % 16 ||
+      reinterpret_cast<uintptr_t>(out) % 16)
+    return DFLASH_ERR_INVALID_ARG;
+  DF_CUDA(cudaSetDevice(h->device));
+  EpiStoreF32 e{out, N};
+  return run_gemm(h, A, M, K, W, N, e, static_cast<float*>(workspace), workspace_bytes,
+                  static_cast<cudaStream_t>(stream), block_n, splits);
+}
+
+size_t dflash_attention_workspace_bytes(const dflash_handle* h, int B, int max_pages_per_seq) {
+  if (!h || B <= 0 || max_pages_per_seq <= 0) return 0;
+  const dflash_config& c = h->cfg;
+  const AttnPlan ap = plan_attention(B, c.n_kv_heads, max_pages_per_seq, c.page_size,
+                                     c.block_size, c.n_q_heads / c.n_kv_heads, c.head_dim,
+                                     h->num_sms);
+  return align_up(ap.part_o_bytes) + align_up(ap.part_ml_bytes) + kAlign;
+}
+
+dflash_status dflash_block_attention(dflash_handle* h, const void* q, const int32_t* seq_lens,
+                                     const int32_t* block_table, int B, int max_pages_per_seq,
+                                     const void* k_cache, const void* v_cache, int num_pages,
+                                     void* o, void* workspace, size_t workspace_bytes,
+                                     void* stream) {
+  if (!h || B < 0) return DFLASH_ERR_INVALID_ARG;
+  if (B == 0) return DFLASH_OK;
+  if (!q || !seq_lens || !block_table || max_pages_per_seq <= 0 || !k_cache || !v_cache ||
+      num_pages <= 0 || !o || !workspace)
+    return DFLASH_ERR_INVALID_ARG;
+  const dflash_config& c = h->cfg;
+  if (workspace_bytes < dflash_attention_workspace_bytes(h, B, max_pages_per_seq))
+    return DFLASH_ERR_WORKSPACE;
+  DF_CUDA(cudaSetDevice(h->device));
+  const AttnPlan ap = plan_attention(B, c.n_kv_heads, max_pages_per_seq, c.page_size,
+                                     c.block_size, c.n_q_heads / c.n_kv_heads, c.head_dim,
+                                     h->num_sms);
+  AttnParams prm;
+  prm.q = static_cast<const bf16*>(q);
+  prm.o = static_cast<bf16*>(o);
+  prm.part_o = static_cast<float*>(workspace);
+  prm.part_ml = at<float>(workspace, align_up(ap.part_o_bytes));
+  prm.seq_lens = seq_lens;
+  prm.block_table = block_table;
+  prm.B = B;
+  prm.W = max_pages_per_seq;
+  prm.bs = c.block_size;
+  prm.Hq = c.n_q_heads;
+  prm.Hkv = c.n_kv_heads;
+  prm.G = c.n_q_heads / c.n_kv_heads;
+  prm.R = ap.R;
+  prm.num_pages = num_pages;
+  prm.chunk_keys = ap.chunk_keys;
+  prm.max_splits = ap.max_splits;
+  prm.scale_log2 =
+      static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(c.head_dim)));
+  prm.err = h->dev_err;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return c.head_dim == 128 ? run_attention<128>(h, ap, prm, k_cache, v_cache, num_pages, st)
+                           : run_attention<64>(h, ap, prm, k_cache, v_cache, num_pages, st);
+}
+
+dflash_status dflash_check_device_errors(dflash_handle* h, unsigned* bits) {
+  if (bits) *bits = 0;
+  if (!h) return DFLASH_ERR_INVALID_ARG;
+  DF_CUDA(cudaSetDevice(h->device));
+  DF_CUDA(cudaDeviceSynchronize());
+  unsigned v = 0;
+  DF_CUDA(cudaMemcpy(&v, h->dev_err, sizeof(unsigned), cudaMemcpyDeviceToHost));
+  DF_CUDA(cudaMemset(h->dev_err, 0, sizeof(unsigned)));
+  if (v & DFLASH_DEVERR_TIMEOUT) {
+    // a kernel that gave up may have left split-K arrival counters behind
+    DF_CUDA(cudaMemset(h->counters, 0, kCounterSlots * sizeof(unsigned)));
+  }
+  if (bits) *bits = v;
+  if (v == 0) return DFLASH_OK;
+  return (v & DFLASH_DEVERR_TIMEOUT) ? DFLASH_ERR_DEVICE_TIMEOUT : DFLASH_ERR_DEVICE_BOUNDS;
+}
+
+}  // extern "C"

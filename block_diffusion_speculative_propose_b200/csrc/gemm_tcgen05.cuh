@@ -1,0 +1,555 @@
+// gemm_tcgen05.cuh — persistent, warp-specialised bf16 GEMM for sm_100a with
+// fused epilogues.
+//
+//   D[m, n] = sum_k A[m, k] * W[n, k]      A: [M, K] bf16, W: [N, K] bf16 (both K-major)
+//
+// Tile 128 x BN x 64.  Warp 0 streams A and W tiles with TMA (128-byte swizzle)
+// into a ring of shared-memory stages; warp 1 issues tcgen05.mma (M=128, N=BN,
+// K=16, one thread) into a double-buffered fp32 accumulator in tensor memory;
+// warps 2..5 drain the accumulator with tcgen05.ld and run the epilogue functor
+// while the next tile accumulates.  Units of work are (k-split, n-tile, m-tile)
+// triples handed out round-robin to one CTA per SM.
+//
+// Split-K (used only when a weight-streaming GEMM has too few output tiles to
+// occupy every SM): each split writes its fp32 partial tile to global memory;
+// the CTA that finishes a tile's last split (detected with a per-tile arrival
+// counter, no waiting) sums the partials in split order — so the result is
+// deterministic — and runs the epilogue.  The counters are left at zero.
+//
+// Every pipeline wait is bounded (see mbar_wait); a wait that runs out sets the
+// timeout bit and the CTA winds down, frees its tensor memory and returns.
+#pragma once
+
+#include "dflash_device.cuh"
+
+namespace dflash {
+
+constexpr int kGemmBM = 128;
+constexpr int kGemmBK = 64;
+constexpr int kGemmThreads = 192;
+constexpr int kGemmSmemLimit = 232448;  // max dynamic shared memory per block on sm_100
+
+template <int BN>
+struct GemmCfg {
+  static constexpr int kABytes = kGemmBM * kGemmBK * 2;
+  static constexpr int kBBytes = BN * kGemmBK * 2;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kReserve = 1024 + 256;  // alignment slack + barriers
+  static constexpr int kStagesRaw = (kGemmSmemLimit - kReserve) / kStageBytes;
+  static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
+  static constexpr int kSmemBytes = kReserve + kStages * kStageBytes;
+  static constexpr int kTmemCols = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
+                                   : (2 * BN <= 256) ? 256 : 512;
+  static_assert(BN % 16 == 0 && BN >= 32 && BN <= 256, "UMMA N for M=128");
+};
+
+struct GemmParams {
+  int M, N, K;
+  int m_tiles, n_tiles, k_blocks;
+  int splits, kb_per_split, num_units;
+  float* partials;     // [splits][M][N] when splits > 1
+  unsigned* counters;  // [m_tiles * n_tiles], zero on entry, zero on exit
+  unsigned* err;
+};
+
+struct GemmUnit {
+  int m_tile, n_tile, split, kb0, kb1;
+};
+__device__ __forceinline__ GemmUnit decode_unit(const GemmParams& p, int u) {
+  GemmUnit t;
+  const int per_split = p.m_tiles * p.n_tiles;
+  t.split = u / per_split;
+  const int r = u - t.split * per_split;
+  t.n_tile = r / p.m_tiles;
+  t.m_tile = r - t.n_tile * p.m_tiles;
+  t.kb0 = t.split * p.kb_per_split;
+  t.kb1 = min(p.k_blocks, t.kb0 + p.kb_per_split);
+  return t;
+}
+
+template <int N>
+__device__ __forceinline__ void tmem_load_cols(uint32_t taddr, float* v) {
+  static_assert(N % 32 == 0, "");
+#pragma unroll
+  for (int c = 0; c < N / 32; ++c) {
+    float t[32];
+    tmem_ld_32x32b_x32(taddr + c * 32, t);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[c * 32 + j] = t[j];
+  }
+  tmem_ld_wait();
+}
+
+template <int BN, class Epi>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_tcgen05_kernel(const __grid_constant__ CUtensorMap tmA,
+                        const __grid_constant__ CUtensorMap tmW, const GemmParams p,
+                        const Epi epi) {
+  using C = GemmCfg<BN>;
+  constexpr int G = Epi::kGroup;
+  static_assert(BN % G == 0, "epilogue group must divide the tile width");
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + C::kStages * C::kABytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + C::kStages * C::kBBytes);
+  uint64_t* empty = full + C::kStages;
+  uint64_t* tfull = empty + C::kStages;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 4);
+    }
+    fence_barrier_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmW);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const uint64_t pol_w = policy_evict_first();
+      const uint64_t pol_a = policy_evict_last();
+      uint32_t stage = 0, phase = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
+        const GemmUnit t = decode_unit(p, u);
+        for (int kb = t.kb0; kb < t.kb1; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, p.err)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
+          tma_load_2d_hint(sA + stage * C::kABytes, &tmA, &full[stage], kb * kGemmBK,
+                           t.m_tile * kGemmBM, pol_a);
+          tma_load_2d_hint(sB + stage * C::kBBytes, &tmW, &full[stage], kb * kGemmBK,
+                           t.n_tile * BN, pol_w);
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = umma_idesc_bf16_f32(kGemmBM, BN);
+      uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
+        const GemmUnit t = decode_unit(p, u);
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, p.err)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = t.kb0; kb < t.kb1; ++kb) {
+          if (!mbar_wait(&full[stage], phase, p.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t adesc = umma_desc_sw128(smem_u32(sA + stage * C::kABytes));
+          const uint64_t bdesc = umma_desc_sw128(smem_u32(sB + stage * C::kBBytes));
+#pragma unroll
+          for (int k = 0; k < kGemmBK / 16; ++k) {
+            // +32 bytes along K inside the 128-byte swizzle atom = +2 in the
+            // descriptor's (address >> 4) field
+            umma_bf16(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc,
+                      (kb > t.kb0 || k > 0) ? 1u : 0u);
+          }
+          umma_commit(&empty[stage]);
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[acc]);
+        acc ^= 1u;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int ew = warp - 2;        // 0..3
+    const int sp = warp & 3;        // TMEM sub-partition this warp may read
+    const int row = sp * 32 + lane;
+    uint32_t acc = 0, acc_phase = 0;
+    for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
+      const GemmUnit t = decode_unit(p, u);
+      if (!mbar_wait(&tfull[acc], acc_phase, p.err)) break;
+      tc_fence_after();
+      const int m = t.m_tile * kGemmBM + row;
+      const bool row_ok = m < p.M;
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(sp * 32) << 16) + acc * BN;
+      if (p.splits == 1) {
+        typename Epi::State st;
+        epi.begin(st);
+#pragma unroll 1
+        for (int g = 0; g < BN / G; ++g) {
+          float v[G];
+          tmem_load_cols<G>(taddr + g * G, v);
+          const int n0 = t.n_tile * BN + g * G;
+          if (row_ok && n0 < p.N) epi.apply(st, m, n0, min(G, p.N - n0), v);
+        }
+        epi.end(st, m, row_ok);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[acc]);
+      } else {
+        float* part = p.partials + static_cast<size_t>(t.split) * p.M * p.N;
+#pragma unroll 1
+        for (int g = 0; g < BN / G; ++g) {
+          float v[G];
+          tmem_load_cols<G>(taddr + g * G, v);
+          const int n0 = t.n_tile * BN + g * G;
+          if (row_ok && n0 < p.N) {
+            float* dst = part + static_cast<size_t>(m) * p.N + n0;
+            const int nv = min(G, p.N - n0);
+            if (nv == G) {
+#pragma unroll
+              for (int j = 0; j < G; j += 4)
+                __stcg(reinterpret_cast<float4*>(dst + j),
+                       make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]));
+            } else {
+#pragma unroll
+              for (int j = 0; j < G; ++j)
+                if (j < nv) __stcg(dst + j, v[j]);
+            }
+          }
+        }
+        __threadfence();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[acc]);
+        named_bar_sync(1, 128);
+        if (ew == 0 && lane == 0) {
+          const int tile = t.m_tile * p.n_tiles + t.n_tile;
+          const unsigned prev = atomicAdd(&p.counters[tile], 1u);
+          const int last = (prev == static_cast<unsigned>(p.splits - 1)) ? 1 : 0;
+          if (last) p.counters[tile] = 0u;
+          *last_flag = last;
+        }
+        named_bar_sync(1, 128);
+        const int last = *last_flag;
+        if (last) {
+          __threadfence();
+          typename Epi::State st;
+          epi.begin(st);
+#pragma unroll 1
+          for (int g = 0; g < BN / G; ++g) {
+            const int n0 = t.n_tile * BN + g * G;
+            if (row_ok && n0 < p.N) {
+              const int nv = min(G, p.N - n0);
+              float v[G];
+#pragma unroll
+              for (int j = 0; j < G; ++j) v[j] = 0.f;
+              for (int s = 0; s < p.splits; ++s) {
+                const float* src = p.partials + (static_cast<size_t>(s) * p.M + m) * p.N + n0;
+                if (nv == G) {
+#pragma unroll
+                  for (int j = 0; j < G; j += 4) {
+                    const float4 q = __ldcg(reinterpret_cast<const float4*>(src + j));
+                    v[j] += q.x;
+                    v[j + 1] += q.y;
+                    v[j + 2] += q.z;
+                    v[j + 3] += q.w;
+                  }
+                } else {
+#pragma unroll
+                  for (int j = 0; j < G; ++j)
+                    if (j < nv) v[j] += __ldcg(src + j);
+                }
+              }
+              epi.apply(st, m, n0, nv, v);
+            }
+          }
+          epi.end(st, m, row_ok);
+        }
+        named_bar_sync(1, 128);  // last_flag is rewritten by the next unit
+      }
+      acc ^= 1u;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// epilogue functors
+//   kGroup columns (one contiguous group of output features) are handed to
+//   apply() at a time, as fp32 values of one output row.
+// ---------------------------------------------------------------------------
+struct EpiNoState {};
+
+// out[m, n] = acc  (fp32)
+struct EpiStoreF32 {
+  static constexpr int kGroup = 32;
+  using State = EpiNoState;
+  float* out;
+  int ldo;
+  __device__ void begin(State&) const {}
+  __device__ void end(State&, int, bool) const {}
+  __device__ void apply(State&, int m, int n0, int nv, const float* v) const {
+    float* dst = out + static_cast<size_t>(m) * ldo + n0;
+    if (nv == kGroup) {
+#pragma unroll
+      for (int j = 0; j < kGroup; j += 4)
+        *reinterpret_cast<float4*>(dst + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < kGroup; ++j)
+        if (j < nv) dst[j] = v[j];
+    }
+  }
+};
+
+// x[m, n] += acc  (fp32 residual stream)
+struct EpiResidAdd {
+  static constexpr int kGroup = 32;
+  using State = EpiNoState;
+  float* x;
+  int ldx;
+  __device__ void begin(State&) const {}
+  __device__ void end(State&, int, bool) const {}
+  __device__ void apply(State&, int m, int n0, int nv, const float* v) const {
+    float* dst = x + static_cast<size_t>(m) * ldx + n0;
+    if (nv == kGroup) {
+#pragma unroll
+      for (int j = 0; j < kGroup; j += 4) {
+        float4 r = *reinterpret_cast<float4*>(dst + j);
+        r.x += v[j];
+        r.y += v[j + 1];
+        r.z += v[j + 2];
+        r.w += v[j + 3];
+        *reinterpret_cast<float4*>(dst + j) = r;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < kGroup; ++j)
+        if (j < nv) dst[j] += v[j];
+    }
+  }
+};
+
+// Gate/up weights are packed in blocks of 32 rows: 16 gate rows then the 16 up
+// rows of the same features.  h[m, f] = bf16(silu(gate) * up).
+struct EpiSwiGLU {
+  static constexpr int kGroup = 32;
+  using State = EpiNoState;
+  bf16* h;
+  int ldh;
+  __device__ void begin(State&) const {}
+  __device__ void end(State&, int, bool) const {}
+  __device__ void apply(State&, int m, int n0, int nv, const float* v) const {
+    (void)nv;  // the packed width is a multiple of 32
+    uint32_t w[8];
+#pragma unroll
+    for (int j = 0; j < 16; j += 2) {
+      const float g0 = v[j], g1 = v[j + 1];
+      const float a0 = g0 / (1.f + expf(-g0)) * v[16 + j];
+      const float a1 = g1 / (1.f + expf(-g1)) * v[17 + j];
+      w[j / 2] = pack_bf16x2(a0, a1);
+    }
+    uint4* dst = reinterpret_cast<uint4*>(h + static_cast<size_t>(m) * ldh + (n0 >> 1));
+    dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+  }
+};
+
+// Per-head RMSNorm (weight w) then rotate-half RoPE with the (cos, sin) table
+// row `cs`, in place on D values.
+template <int D>
+__device__ __forceinline__ void head_norm_rope(float* v, const bf16* w, const float2* cs,
+                                               float eps) {
+  float ss = 0.f;
+#pragma unroll
+  for (int j = 0; j < D; ++j) ss += v[j] * v[j];
+  const float r = rsqrtf(ss / D + eps);
+#pragma unroll
+  for (int j = 0; j < D; ++j) v[j] = v[j] * r * bf2f(w[j]);
+#pragma unroll
+  for (int j = 0; j < D / 2; ++j) {
+    const float2 c = cs[j];
+    const float a = v[j], b = v[j + D / 2];
+    v[j] = a * c.x - b * c.y;
+    v[j + D / 2] = b * c.x + a * c.y;
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void store_bf16_row(bf16* dst, const float* v) {
+#pragma unroll
+  for (int j = 0; j < D; j += 8) {
+    uint4 q;
+    q.x = pack_bf16x2(v[j], v[j + 1]);
+    q.y = pack_bf16x2(v[j + 2], v[j + 3]);
+    q.z = pack_bf16x2(v[j + 4], v[j + 5]);
+    q.w = pack_bf16x2(v[j + 6], v[j + 7]);
+    *reinterpret_cast<uint4*>(dst + j) = q;
+  }
+}
+
+// Draft-layer QKV projection of the query block.  Output features are
+// [q heads | k heads | v heads], one head per group.  q, k: per-head RMSNorm +
+// RoPE at the block position seq_len + i; q goes to the q buffer, k and v to
+// the request's paged slot of this layer's cache.
+template <int D>
+struct EpiQKV {
+  static constexpr int kGroup = D;
+  using State = EpiNoState;
+  bf16* q;
+  const bf16* q_norm_w;
+  const bf16* k_norm_w;
+  const float2* rope;
+  bf16* k_cache;
+  bf16* v_cache;
+  const int* seq_lens;
+  const int* block_table;
+  int max_pos, W, bs, Hq, Hkv, P, num_pages;
+  float eps;
+  unsigned* err;
+  __device__ void begin(State&) const {}
+  __device__ void end(State&, int, bool) const {}
+  __device__ void apply(State&, int m, int n0, int nv, float* v) const {
+    (void)nv;
+    const int head = n0 / D;
+    const int b = m / bs, i = m - (m / bs) * bs;
+    const int pos = seq_lens[b] + i;
+    if (head < Hq + Hkv) {
+      if (pos < 0 || pos >= max_pos) {
+        raise_error(err, DFLASH_DEVERR_POSITION);
+        return;
+      }
+      head_norm_rope<D>(v, head < Hq ? q_norm_w : k_norm_w,
+                        rope + static_cast<size_t>(pos) * (D / 2), eps);
+    }
+    if (head < Hq) {
+      store_bf16_row<D>(q + (static_cast<size_t>(m) * Hq + head) * D, v);
+      return;
+    }
+    const int pg = pos / P;
+    if (pg >= W) {
+      raise_error(err, DFLASH_DEVERR_TABLE);
+      return;
+    }
+    const int page = block_table[static_cast<size_t>(b) * W + pg];
+    if (page < 0 || page >= num_pages) {
+      raise_error(err, DFLASH_DEVERR_SLOT);
+      return;
+    }
+    const bool is_k = head < Hq + Hkv;
+    const int kh = is_k ? head - Hq : head - Hq - Hkv;
+    bf16* cache = is_k ? k_cache : v_cache;
+    store_bf16_row<D>(cache + ((static_cast<size_t>(page) * Hkv + kh) * P + (pos - pg * P)) * D, v);
+  }
+};
+
+constexpr int kMaxLayers = 64;
+
+// Context K/V injection.  Output features are ordered per layer as
+// [k heads | v heads]; a group is one (layer, k|v, head).  Keys get the layer's
+// k_norm and RoPE at the row's own position; rows with a negative slot are
+// padding and are skipped.
+template <int D>
+struct EpiKVInject {
+  static constexpr int kGroup = D;
+  using State = EpiNoState;
+  bf16* k_cache[kMaxLayers];
+  bf16* v_cache[kMaxLayers];
+  const bf16* k_norm_w;  // [L][D]
+  const float2* rope;
+  const int64_t* positions;
+  const int64_t* slots;
+  int max_pos, Hkv, P, num_pages;
+  float eps;
+  unsigned* err;
+  __device__ void begin(State&) const {}
+  __device__ void end(State&, int, bool) const {}
+  __device__ void apply(State&, int m, int n0, int nv, float* v) const {
+    (void)nv;
+    const int64_t slot = slots[m];
+    if (slot < 0) return;
+    if (slot >= static_cast<int64_t>(num_pages) * P) {
+      raise_error(err, DFLASH_DEVERR_SLOT);
+      return;
+    }
+    const int hi = n0 / D;
+    const int l = hi / (2 * Hkv);
+    const int kind = (hi / Hkv) & 1;
+    const int kh = hi - (hi / Hkv) * Hkv;
+    if (kind == 0) {
+      const int64_t pos = positions[m];
+      if (pos < 0 || pos >= max_pos) {
+        raise_error(err, DFLASH_DEVERR_POSITION);
+        return;
+      }
+      head_norm_rope<D>(v, k_norm_w + static_cast<size_t>(l) * D,
+                        rope + static_cast<size_t>(pos) * (D / 2), eps);
+    }
+    const int64_t page = slot / P, off = slot - (slot / P) * P;
+    bf16* cache = kind == 0 ? k_cache[l] : v_cache[l];
+    store_bf16_row<D>(cache + ((page * Hkv + kh) * P + off) * D, v);
+  }
+};
+
+// LM head with greedy pick: per row, the ordered key of (max logit, lowest id)
+// is folded into keys[m] with one 64-bit atomicMax per tile.  Optionally also
+// writes the fp32 logits (debug).
+struct EpiArgmax {
+  static constexpr int kGroup = 32;
+  struct State {
+    unsigned long long best;
+  };
+  unsigned long long* keys;
+  float* logits;
+  int ldl;
+  __device__ void begin(State& s) const { s.best = 0ull; }
+  __device__ void apply(State& s, int m, int n0, int nv, const float* v) const {
+#pragma unroll
+    for (int j = 0; j < kGroup; ++j) {
+      if (j < nv) {
+        const unsigned long long k = argmax_key(v[j], static_cast<uint32_t>(n0 + j));
+        s.best = k > s.best ? k : s.best;
+      }
+    }
+    if (logits) {
+      float* dst = logits + static_cast<size_t>(m) * ldl + n0;
+#pragma unroll
+      for (int j = 0; j < kGroup; ++j)
+        if (j < nv) dst[j] = v[j];
+    }
+  }
+  __device__ void end(State& s, int m, bool row_ok) const {
+    if (row_ok && s.best) atomicMax(keys + m, s.best);
+  }
+};
+
+}  // namespace dflash

@@ -1,0 +1,240 @@
+// small_kernels.cuh — the light kernels around the GEMMs and attention:
+// block build + embedding + first RMSNorm, row RMSNorms, the draft-token
+// finalisation, greedy verification, paged-slot mapping and the RoPE table.
+#pragma once
+
+#include "dflash_device.cuh"
+
+namespace dflash {
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const unsigned long long w = __shfl_xor_sync(0xffffffffu, v, o);
+    v = w > v ? w : v;
+  }
+  return v;
+}
+// Sum over the block (blockDim.x a multiple of 32, <= 1024); every thread gets it.
+__device__ __forceinline__ float block_sum(float v, float* red) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  v = warp_sum(v);
+  __syncthreads();  // red may still be read by a previous call
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  float t = (lane < (blockDim.x >> 5)) ? red[lane] : 0.f;
+  return warp_sum(t);
+}
+
+// Block construction ([bonus, mask, ..., mask] per request), embedding with
+// the target table, and the first layer's input RMSNorm.
+//   x[r, :]   = embed[id_r, :]                       (fp32 residual stream)
+//   nrm[r, :] = bf16(x * rsqrt(mean(x^2) + eps) * w)
+// Also clears the LM-head argmax keys of the call.
+__global__ void __launch_bounds__(256) embed_norm_kernel(
+    const int32_t* __restrict__ bonus, int mask_id, const bf16* __restrict__ embed,
+    const bf16* __restrict__ w, float* __restrict__ x, bf16* __restrict__ nrm,
+    unsigned long long* __restrict__ keys, int n_keys, int bs, int H, int V, float eps,
+    unsigned* err) {
+  __shared__ float red[32];
+  const int r = blockIdx.x;
+  const int b = r / bs, i = r - (r / bs) * bs;
+  int tok = (i == 0) ? bonus[b] : mask_id;
+  if (tok < 0 || tok >= V) {
+    if (threadIdx.x == 0) raise_error(err, DFLASH_DEVERR_TOKEN);
+    tok = 0;
+  }
+  if (threadIdx.x == 0 && r < n_keys) keys[r] = 0ull;
+  const bf16* e = embed + static_cast<size_t>(tok) * H;
+  float* xr = x + static_cast<size_t>(r) * H;
+  float ss = 0.f;
+  for (int j = threadIdx.x * 8; j < H; j += blockDim.x * 8) {
+    const uint4 q = *reinterpret_cast<const uint4*>(e + j);
+    const bf16* qb = reinterpret_cast<const bf16*>(&q);
+    float v[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      v[k] = bf2f(qb[k]);
+      ss += v[k] * v[k];
+    }
+    *reinterpret_cast<float4*>(xr + j) = make_float4(v[0], v[1], v[2], v[3]);
+    *reinterpret_cast<float4*>(xr + j + 4) = make_float4(v[4], v[5], v[6], v[7]);
+  }
+  ss = block_sum(ss, red);
+  const float rinv = rsqrtf(ss / H + eps);
+  bf16* nr = nrm + static_cast<size_t>(r) * H;
+  for (int j = threadIdx.x * 8; j < H; j += blockDim.x * 8) {
+    const uint4 q = *reinterpret_cast<const uint4*>(e + j);
+    const uint4 wq = *reinterpret_cast<const uint4*>(w + j);
+    const bf16* qb = reinterpret_cast<const bf16*>(&q);
+    const bf16* wb = reinterpret_cast<const bf16*>(&wq);
+    uint4 o;
+    uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      ow[k] = pack_bf16x2(bf2f(qb[2 * k]) * rinv * bf2f(wb[2 * k]),
+                          bf2f(qb[2 * k + 1]) * rinv * bf2f(wb[2 * k + 1]));
+    *reinterpret_cast<uint4*>(nr + j) = o;
+  }
+}
+
+// out[r, :] = bf16(x[src(r), :] * rsqrt(mean(x^2) + eps) * w).
+// With gather_k > 0, src(r) = (r / gather_k) * bs + 1 + r % gather_k: the block
+// slots 1..bs-1 of each request (keep_idx), packed densely.
+__global__ void __launch_bounds__(256) rmsnorm_rows_kernel(
+    const float* __restrict__ x, const bf16* __restrict__ w, bf16* __restrict__ out, int H,
+    float eps, int gather_k, int bs) {
+  __shared__ float red[32];
+  const int r = blockIdx.x;
+  const int src = gather_k > 0 ? (r / gather_k) * bs + 1 + (r - (r / gather_k) * gather_k) : r;
+  const float* xr = x + static_cast<size_t>(src) * H;
+  float ss = 0.f;
+  for (int j = threadIdx.x * 8; j < H; j += blockDim.x * 8) {
+    const float4 a = *reinterpret_cast<const float4*>(xr + j);
+    const float4 c = *reinterpret_cast<const float4*>(xr + j + 4);
+    ss += a.x * a.x + a.y * a.y + a.z * a.z + a.w * a.w + c.x * c.x + c.y * c.y + c.z * c.z +
+          c.w * c.w;
+  }
+  ss = block_sum(ss, red);
+  const float rinv = rsqrtf(ss / H + eps);
+  bf16* orow = out + static_cast<size_t>(r) * H;
+  for (int j = threadIdx.x * 8; j < H; j += blockDim.x * 8) {
+    const float4 a = *reinterpret_cast<const float4*>(xr + j);
+    const float4 c = *reinterpret_cast<const float4*>(xr + j + 4);
+    const uint4 wq = *reinterpret_cast<const uint4*>(w + j);
+    const bf16* wb = reinterpret_cast<const bf16*>(&wq);
+    uint4 o;
+    o.x = pack_bf16x2(a.x * rinv * bf2f(wb[0]), a.y * rinv * bf2f(wb[1]));
+    o.y = pack_bf16x2(a.z * rinv * bf2f(wb[2]), a.w * rinv * bf2f(wb[3]));
+    o.z = pack_bf16x2(c.x * rinv * bf2f(wb[4]), c.y * rinv * bf2f(wb[5]));
+    o.w = pack_bf16x2(c.z * rinv * bf2f(wb[6]), c.w * rinv * bf2f(wb[7]));
+    *reinterpret_cast<uint4*>(orow + j) = o;
+  }
+}
+
+// drafts[b, i] = argmax of LM-head row (b, i); block[b] = [bonus_b, drafts[b]].
+__global__ void argmax_finalize_kernel(const unsigned long long* __restrict__ keys,
+                                       const int32_t* __restrict__ bonus,
+                                       int32_t* __restrict__ drafts,
+                                       int32_t* __restrict__ block, int B, int bs) {
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= B * bs) return;
+  const int K = bs - 1;
+  const int b = idx / bs, i = idx - (idx / bs) * bs;
+  int32_t tok;
+  if (i == 0) {
+    tok = bonus[b];
+  } else {
+    tok = static_cast<int32_t>(argmax_key_index(keys[b * K + i - 1]));
+    drafts[b * K + i - 1] = tok;
+  }
+  if (block) block[idx] = tok;
+}
+
+// Greedy verification, pass 1: per (row, chunk) ordered argmax key of the fp32
+// target logits.  Rows are [B * (K+1)], each V long.
+__global__ void __launch_bounds__(256) verify_partial_kernel(
+    const float* __restrict__ logits, int V, int chunk_len, int chunks,
+    unsigned long long* __restrict__ part) {
+  __shared__ unsigned long long red[32];
+  const size_t row = blockIdx.y;
+  const int beg = blockIdx.x * chunk_len;
+  const int end = min(V, beg + chunk_len);
+  const float* src = logits + row * static_cast<size_t>(V);
+  unsigned long long best = 0ull;
+  if ((V & 3) == 0) {
+    for (int j = beg + threadIdx.x * 4; j < end; j += blockDim.x * 4) {
+      const float4 v = __ldcs(reinterpret_cast<const float4*>(src + j));
+      unsigned long long k;
+      k = argmax_key(v.x, j);
+      best = k > best ? k : best;
+      k = argmax_key(v.y, j + 1);
+      best = k > best ? k : best;
+      k = argmax_key(v.z, j + 2);
+      best = k > best ? k : best;
+      k = argmax_key(v.w, j + 3);
+      best = k > best ? k : best;
+    }
+  } else {
+    for (int j = beg + threadIdx.x; j < end; j += blockDim.x) {
+      const unsigned long long k = argmax_key(__ldcs(src + j), j);
+      best = k > best ? k : best;
+    }
+  }
+  best = warp_max_u64(best);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) red[warp] = best;
+  __syncthreads();
+  if (warp == 0) {
+    unsigned long long t = lane < (blockDim.x >> 5) ? red[lane] : 0ull;
+    t = warp_max_u64(t);
+    if (lane == 0) part[row * chunks + blockIdx.x] = t;
+  }
+}
+
+// Pass 2 (one warp per request): t_j for j = 0..K, longest matching prefix,
+// bonus, and the -1 padded output row.
+__global__ void verify_final_kernel(const unsigned long long* __restrict__ part, int chunks,
+                                    const int32_t* __restrict__ drafts, int K,
+                                    int32_t* __restrict__ out, int32_t* __restrict__ n_acc,
+                                    int32_t* __restrict__ bonus) {
+  __shared__ int32_t t[130];
+  const int b = blockIdx.x, lane = threadIdx.x;
+  for (int j = 0; j <= K; ++j) {
+    const unsigned long long* pr = part + (static_cast<size_t>(b) * (K + 1) + j) * chunks;
+    unsigned long long best = 0ull;
+    for (int c = lane; c < chunks; c += 32) best = pr[c] > best ? pr[c] : best;
+    best = warp_max_u64(best);
+    if (lane == 0) t[j] = static_cast<int32_t>(argmax_key_index(best));
+  }
+  __syncwarp();
+  int n = 0;
+  while (n < K && drafts[static_cast<size_t>(b) * K + n] == t[n]) ++n;
+  for (int j = lane; j <= K; j += 32) {
+    int32_t v = -1;
+    if (j < n) v = drafts[static_cast<size_t>(b) * K + j];
+    else if (j == n) v = t[n];
+    out[static_cast<size_t>(b) * (K + 1) + j] = v;
+  }
+  if (lane == 0) {
+    n_acc[b] = n;
+    bonus[b] = t[n];
+  }
+}
+
+// slots[i] = block_table[req * W + min(pos / P, W - 1)] * P + pos % P
+__global__ void paged_slots_kernel(const int64_t* __restrict__ pos,
+                                   const int64_t* __restrict__ req,
+                                   const int32_t* __restrict__ table, int n, int W, int P,
+                                   int64_t* __restrict__ slots) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const int64_t p = pos[i];
+  if (p < 0) {
+    slots[i] = -1;
+    return;
+  }
+  int64_t pg = p / P;
+  if (pg > W - 1) pg = W - 1;
+  const int64_t page = table[req[i] * W + pg];
+  slots[i] = page * P + (p - (p / P) * P);
+}
+
+// cos / sin of pos * theta^(-2j/D), evaluated in double, stored as fp32 pairs.
+__global__ void rope_table_kernel(float2* __restrict__ table, int max_pos, int half,
+                                  double theta) {
+  const int pos = blockIdx.x;
+  for (int j = threadIdx.x; j < half; j += blockDim.x) {
+    const double inv = pow(theta, -2.0 * j / (2.0 * half));
+    const double a = static_cast<double>(pos) * inv;
+    table[static_cast<size_t>(pos) * half + j] =
+        make_float2(static_cast<float>(cos(a)), static_cast<float>(sin(a)));
+  }
+}
+
+}  // namespace dflash

@@ -1,0 +1,344 @@
+"""Thin Python binding over the C ABI in include/dflash.h (libdflash.so).
+
+Argument marshalling only: every step of the path runs in the library's CUDA
+kernels.  Torch tensors supply device memory and streams; outputs that the
+caller does not pass are allocated here with ``torch.empty``.  If the shared
+library is missing this module raises — there is no fallback.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Dict, List, Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdflash.so")
+
+STATUS = {
+    0: "DFLASH_OK",
+    -1: "DFLASH_ERR_INVALID_ARG",
+    -2: "DFLASH_ERR_CUDA",
+    -3: "DFLASH_ERR_WORKSPACE",
+    -4: "DFLASH_ERR_UNSUPPORTED_SHAPE",
+    -5: "DFLASH_ERR_DEVICE_BOUNDS",
+    -6: "DFLASH_ERR_UNIMPLEMENTED",
+    -7: "DFLASH_ERR_DEVICE_TIMEOUT",
+}
+DEVERR_TIMEOUT, DEVERR_SLOT, DEVERR_TABLE, DEVERR_TOKEN, DEVERR_POSITION = 1, 2, 4, 8, 16
+
+
+class DFlashError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)}")
+
+
+class _Config(ctypes.Structure):
+    _fields_ = [("hidden", ctypes.c_int), ("n_layers", ctypes.c_int),
+                ("n_q_heads", ctypes.c_int), ("n_kv_heads", ctypes.c_int),
+                ("head_dim", ctypes.c_int), ("intermediate", ctypes.c_int),
+                ("vocab", ctypes.c_int), ("n_target_layers", ctypes.c_int),
+                ("target_layer_ids", ctypes.POINTER(ctypes.c_int)),
+                ("block_size", ctypes.c_int), ("mask_token_id", ctypes.c_int),
+                ("page_size", ctypes.c_int), ("rms_eps", ctypes.c_float),
+                ("rope_theta", ctypes.c_float), ("max_position", ctypes.c_int)]
+
+
+_PP = ctypes.POINTER(ctypes.c_void_p)
+
+
+class _Weights(ctypes.Structure):
+    _fields_ = [("fc_w", ctypes.c_void_p), ("hidden_norm_w", ctypes.c_void_p),
+                ("embed", ctypes.c_void_p), ("lm_head", ctypes.c_void_p),
+                ("final_norm_w", ctypes.c_void_p)] + [
+        (n, _PP) for n in ("in_norm_w", "post_norm_w", "wq", "wk", "wv", "wo", "q_norm_w",
+                           "k_norm_w", "w_gate", "w_up", "w_down")]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libdflash.so (built in-tree by ``build.py``); raises if absent."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                           "block_diffusion_speculative_propose_b200/build.py")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    sig = {
+        "dflash_create": ([ctypes.POINTER(_Config), ctypes.POINTER(_Weights), i32,
+                           ctypes.POINTER(vp)], i32),
+        "dflash_destroy": ([vp], None),
+        "dflash_inject_workspace_bytes": ([vp, i32], sz),
+        "dflash_propose_workspace_bytes": ([vp, i32, i32], sz),
+        "dflash_verify_workspace_bytes": ([i32, i32, i32], sz),
+        "dflash_linear_workspace_bytes": ([vp, i32, i32, i32], sz),
+        "dflash_attention_workspace_bytes": ([vp, i32, i32], sz),
+        "dflash_paged_slots": ([vp, vp, i32, vp, i32, i32, vp, vp], i32),
+        "dflash_inject_context": ([vp, vp, vp, vp, i32, _PP, _PP, i32, vp, sz, vp], i32),
+        "dflash_propose": ([vp, vp, vp, vp, i32, i32, _PP, _PP, i32, vp, vp, vp, vp, sz, vp],
+                           i32),
+        "dflash_verify_greedy": ([vp, vp, i32, i32, i32, vp, vp, vp, vp, sz, vp], i32),
+        "dflash_linear": ([vp, vp, vp, i32, i32, i32, vp, vp, sz, vp], i32),
+        "dflash_linear_ex": ([vp, vp, vp, i32, i32, i32, vp, i32, i32, vp, sz, vp], i32),
+        "dflash_block_attention": ([vp, vp, vp, vp, i32, i32, vp, vp, i32, vp, vp, sz, vp],
+                                   i32),
+        "dflash_check_device_errors": ([vp, ctypes.POINTER(ctypes.c_uint)], i32),
+        "dflash_status_string": ([i32], ctypes.c_char_p),
+        "dflash_version": ([], ctypes.c_char_p),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(L, name)
+        f.argtypes = args
+        f.restype = res
+    _lib = L
+    return L
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        raise DFlashError(status, where)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return t.data_ptr()
+
+
+def _want(t: torch.Tensor, dtype: torch.dtype, name: str) -> None:
+    if t.dtype != dtype:
+        raise ValueError(f"{name}: expected {dtype}, got {t.dtype}")
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _ptr_array(ts: Sequence[torch.Tensor]):
+    arr = (ctypes.c_void_p * len(ts))(*[_ptr(t) for t in ts])
+    return ctypes.cast(arr, _PP), arr
+
+
+class Workspace:
+    """Device scratch owned by the caller (a uint8 tensor), grown on demand."""
+
+    def __init__(self, device):
+        self.device = torch.device(device)
+        self.buf = torch.empty(0, dtype=torch.uint8, device=self.device)
+
+    def get(self, nbytes: int) -> torch.Tensor:
+        if self.buf.numel() < nbytes:
+            self.buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=self.device)
+        return self.buf
+
+
+class DFlash:
+    """A library handle: packed draft weights + RoPE table on one device.
+
+    ``cfg`` uses the field names of ``dflash_config``; ``weights`` the names of
+    ``dflash_weights`` (bf16 CUDA tensors; per-layer entries are lists).  The
+    handle keeps references to every tensor whose pointer the library keeps."""
+
+    def __init__(self, cfg: Dict, weights: Dict, device: int = 0, max_position: int = 0):
+        L = lib()
+        self.cfg = dict(cfg)
+        self.device = torch.device("cuda", device)
+        n_layers = cfg["n_layers"]
+        self._keep: List = []
+        tl = cfg.get("target_layer_ids")
+        tl_arr = None
+        if tl is not None:
+            tl_arr = (ctypes.c_int * len(tl))(*tl)
+            self._keep.append(tl_arr)
+        maxpos = max_position or cfg.get("max_position", 65536)
+        self.max_position = maxpos
+        c = _Config(cfg["hidden"], n_layers, cfg["n_q_heads"], cfg["n_kv_heads"],
+                    cfg["head_dim"], cfg["intermediate"], cfg["vocab"],
+                    cfg["n_target_layers"],
+                    ctypes.cast(tl_arr, ctypes.POINTER(ctypes.c_int)) if tl_arr else None,
+                    cfg["block_size"], cfg["mask_token_id"], cfg.get("page_size", 16),
+                    cfg.get("rms_eps", 1e-6), cfg.get("rope_theta", 1e6), maxpos)
+        w = _Weights()
+        for k in ("fc_w", "hidden_norm_w", "embed", "lm_head", "final_norm_w"):
+            t = weights[k]
+            _want(t, torch.bfloat16, k)
+            self._keep.append(t)
+            setattr(w, k, _ptr(t))
+        for k in ("in_norm_w", "post_norm_w", "wq", "wk", "wv", "wo", "q_norm_w", "k_norm_w",
+                  "w_gate", "w_up", "w_down"):
+            ts = list(weights[k])
+            if len(ts) != n_layers:
+                raise ValueError(f"{k}: expected {n_layers} layers")
+            for t in ts:
+                _want(t, torch.bfloat16, k)
+            self._keep.extend(ts)
+            pp, arr = _ptr_array(ts)
+            self._keep.append(arr)
+            setattr(w, k, pp)
+        h = ctypes.c_void_p()
+        _check(L.dflash_create(ctypes.byref(c), ctypes.byref(w), device, ctypes.byref(h)),
+               "dflash_create")
+        self.h = h
+        self.ws = Workspace(self.device)
+
+    def close(self) -> None:
+        if getattr(self, "h", None):
+            torch.cuda.synchronize(self.device)
+            lib().dflash_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    # ---------------------------------------------------------------- sizes
+    def inject_workspace_bytes(self, n: int) -> int:
+        return lib().dflash_inject_workspace_bytes(self.h, n)
+
+    def propose_workspace_bytes(self, B: int, max_pages_per_seq: int) -> int:
+        return lib().dflash_propose_workspace_bytes(self.h, B, max_pages_per_seq)
+
+    # ---------------------------------------------------------------- calls
+    def inject_context(self, aux, positions, slot_mapping, k_cache, v_cache,
+                       workspace: Optional[torch.Tensor] = None, stream=None) -> None:
+        n = int(aux.shape[0])
+        _want(aux, torch.bfloat16, "aux")
+        _want(positions, torch.int64, "positions")
+        _want(slot_mapping, torch.int64, "slot_mapping")
+        need = self.inject_workspace_bytes(n) if n else 0
+        ws = workspace if workspace is not None else self.ws.get(need)
+        kp, ka = _ptr_array(k_cache)
+        vp, va = _ptr_array(v_cache)
+        _check(lib().dflash_inject_context(self.h, _ptr(aux), _ptr(positions),
+                                           _ptr(slot_mapping), n, kp, vp,
+                                           int(k_cache[0].shape[0]), _ptr(ws), ws.numel(),
+                                           _stream(stream)),
+               "dflash_inject_context")
+
+    def propose(self, bonus_tokens, seq_lens, block_table, k_cache, v_cache,
+                draft_tokens=None, block_tokens=None, logits_out=None,
+                workspace: Optional[torch.Tensor] = None, stream=None):
+        B = int(bonus_tokens.shape[0])
+        bs = self.cfg["block_size"]
+        _want(bonus_tokens, torch.int32, "bonus_tokens")
+        _want(seq_lens, torch.int32, "seq_lens")
+        _want(block_table, torch.int32, "block_table")
+        W = int(block_table.shape[1])
+        if draft_tokens is None:
+            draft_tokens = torch.empty(B, bs - 1, dtype=torch.int32, device=self.device)
+        need = self.propose_workspace_bytes(B, W) if B else 0
+        ws = workspace if workspace is not None else self.ws.get(need)
+        kp, ka = _ptr_array(k_cache)
+        vp, va = _ptr_array(v_cache)
+        _check(lib().dflash_propose(self.h, _ptr(bonus_tokens), _ptr(seq_lens),
+                                    _ptr(block_table), B, W, kp, vp, int(k_cache[0].shape[0]),
+                                    _ptr(draft_tokens), _ptr(block_tokens), _ptr(logits_out),
+                                    _ptr(ws), ws.numel(), _stream(stream)),
+               "dflash_propose")
+        return draft_tokens
+
+    def linear(self, A, W, out=None, block_n: int = 0, splits: int = 0, workspace=None,
+               stream=None):
+        M, K = A.shape
+        N = W.shape[0]
+        _want(A, torch.bfloat16, "A")
+        _want(W, torch.bfloat16, "W")
+        if out is None:
+            out = torch.empty(M, N, dtype=torch.float32, device=self.device)
+        need = lib().dflash_linear_workspace_bytes(self.h, M, N, K) if M else 0
+        if splits > 1:
+            need = max(need, splits * M * N * 4)
+        ws = workspace if workspace is not None else self.ws.get(need)
+        _check(lib().dflash_linear_ex(self.h, _ptr(A), _ptr(W), M, N, K, _ptr(out), block_n,
+                                      splits, _ptr(ws), ws.numel(), _stream(stream)),
+               "dflash_linear")
+        return out
+
+    def block_attention(self, q, seq_lens, block_table, k_cache, v_cache, o=None,
+                        workspace=None, stream=None):
+        B = int(seq_lens.shape[0])
+        W = int(block_table.shape[1])
+        if o is None:
+            o = torch.empty(q.shape[0], q.shape[1] * q.shape[2], dtype=torch.bfloat16,
+                            device=self.device)
+        need = lib().dflash_attention_workspace_bytes(self.h, B, W) if B else 0
+        ws = workspace if workspace is not None else self.ws.get(need)
+        _check(lib().dflash_block_attention(self.h, _ptr(q), _ptr(seq_lens), _ptr(block_table),
+                                            B, W, _ptr(k_cache), _ptr(v_cache),
+                                            int(k_cache.shape[0]), _ptr(o), _ptr(ws),
+                                            ws.numel(), _stream(stream)),
+               "dflash_block_attention")
+        return o
+
+    def check_device_errors(self) -> int:
+        bits = ctypes.c_uint(0)
+        lib().dflash_check_device_errors(self.h, ctypes.byref(bits))
+        return int(bits.value)
+
+
+def verify_workspace_bytes(B: int, K: int, V: int) -> int:
+    return lib().dflash_verify_workspace_bytes(B, K, V)
+
+
+def verify_greedy(drafts, target_logits, out_tokens=None, num_accepted=None, bonus=None,
+                  workspace=None, stream=None):
+    """Greedy acceptance (dflash_verify_greedy); returns (out_tokens, n, bonus)."""
+    B, K1, V = target_logits.shape
+    K = K1 - 1
+    dev = target_logits.device
+    _want(drafts, torch.int32, "drafts")
+    _want(target_logits, torch.float32, "target_logits")
+    if out_tokens is None:
+        out_tokens = torch.empty(B, K + 1, dtype=torch.int32, device=dev)
+    if num_accepted is None:
+        num_accepted = torch.empty(B, dtype=torch.int32, device=dev)
+    if bonus is None:
+        bonus = torch.empty(B, dtype=torch.int32, device=dev)
+    if workspace is None:
+        workspace = torch.empty(max(verify_workspace_bytes(B, K, V), 256), dtype=torch.uint8,
+                                device=dev)
+    _check(lib().dflash_verify_greedy(_ptr(drafts), _ptr(target_logits), B, K, V,
+                                      _ptr(out_tokens), _ptr(num_accepted), _ptr(bonus),
+                                      _ptr(workspace), workspace.numel(), _stream(stream)),
+           "dflash_verify_greedy")
+    return out_tokens, num_accepted, bonus
+
+
+def paged_slots(positions, req_ids, block_table, page_size: int = 16, slots=None,
+                stream=None):
+    """_paged_slots on the device (dflash_paged_slots)."""
+    n = int(positions.shape[0])
+    _want(positions, torch.int64, "positions")
+    _want(req_ids, torch.int64, "req_ids")
+    _want(block_table, torch.int32, "block_table")
+    if slots is None:
+        slots = torch.empty(n, dtype=torch.int64, device=positions.device)
+    _check(lib().dflash_paged_slots(_ptr(positions), _ptr(req_ids), n, _ptr(block_table),
+                                    int(block_table.shape[1]), page_size, _ptr(slots),
+                                    _stream(stream)), "dflash_paged_slots")
+    return slots
+
+
+def status_string(s: int) -> str:
+    return lib().dflash_status_string(s).decode()
+
+
+def version() -> str:
+    return lib().dflash_version().decode()

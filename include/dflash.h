@@ -1,0 +1,265 @@
+/*
+ * dflash.h — C ABI of the DFlash draft-proposal library for NVIDIA B200 (sm_100a).
+ *
+ * The library implements the data-parallel hot path of DFlash block-diffusion
+ * speculative decoding as described in "DFlash Speculative Decoding in the vLLM
+ * Neuron Framework" (AWS Neuron design doc) and the two pull requests
+ * "[Feat][Spec Decode] DFlash" (vLLM #36847) and "Dflash: Block Diffusion
+ * Speculative Decoding" (QEfficient #995):
+ *
+ *   dflash_inject_context  — §"Context KV Injection (Precompute)": concat'd target
+ *                            aux states -> fc -> hidden_norm -> all layers' K/V
+ *                            (k_norm + RoPE on keys) -> paged-cache scatter.
+ *   dflash_propose         — §"Draft Block Construction", §"DFlash Draft Model
+ *                            Architecture": [bonus, mask, ..., mask] block, non-causal
+ *                            Qwen3-style decoder stack over the injected context,
+ *                            aliased target LM head, greedy argmax -> K drafts.
+ *   dflash_verify_greedy   — §"Component Overview" (greedy rejection sampler):
+ *                            longest prefix of drafts matching the target's argmax,
+ *                            plus one bonus token; rejected slots are -1
+ *                            (§"Async Rejection and Position Correction").
+ *   dflash_paged_slots     — §"Paged KV Integration" (_paged_slots helper).
+ *
+ * Conventions for every call
+ *   - All tensor arguments are DEVICE pointers unless stated otherwise; bf16 means
+ *     IEEE bfloat16 stored as uint16.  Row-major, densely packed.
+ *   - `stream` is a cudaStream_t passed as void*.  Calls only enqueue work on it:
+ *     no call synchronizes the stream, and no call other than dflash_create
+ *     allocates memory.  Work may be captured into a CUDA graph.
+ *   - The caller owns every buffer it passes; the handle owns only the packed
+ *     weight copies and small tables it builds in dflash_create.
+ *   - Shape and argument errors are detected on the host before any launch and
+ *     returned as a negative dflash_status; nothing is enqueued in that case.
+ *   - Conditions that can only be seen on the device (a page id outside the pool,
+ *     a position past the block table or the RoPE table, a token id outside the
+ *     vocabulary, a pipeline wait that ran out) never trap: the kernel skips the
+ *     access and sets a bit in the handle's device error word, which
+ *     dflash_check_device_errors() reads and clears.
+ *   - A handle may be used by one stream at a time (calls on one handle must not
+ *     overlap on the GPU).
+ */
+#ifndef DFLASH_H_
+#define DFLASH_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DFLASH_OK = 0,
+  DFLASH_ERR_INVALID_ARG = -1,       /* null pointer, negative size, inconsistent arguments */
+  DFLASH_ERR_CUDA = -2,              /* a CUDA runtime/driver call or a launch failed        */
+  DFLASH_ERR_WORKSPACE = -3,         /* workspace smaller than the *_workspace_bytes value   */
+  DFLASH_ERR_UNSUPPORTED_SHAPE = -4, /* geometry outside what the kernels are built for       */
+  DFLASH_ERR_DEVICE_BOUNDS = -5,     /* returned by dflash_check_device_errors (see above)    */
+  DFLASH_ERR_UNIMPLEMENTED = -6,
+  DFLASH_ERR_DEVICE_TIMEOUT = -7     /* returned by dflash_check_device_errors                */
+} dflash_status;
+
+/* Device error bits reported by dflash_check_device_errors(). */
+#define DFLASH_DEVERR_TIMEOUT   0x1u  /* a bounded pipeline wait gave up                        */
+#define DFLASH_DEVERR_SLOT      0x2u  /* slot / page id outside the KV pool                     */
+#define DFLASH_DEVERR_TABLE     0x4u  /* position // page_size past the block-table row width   */
+#define DFLASH_DEVERR_TOKEN     0x8u  /* bonus token id outside [0, vocab)                      */
+#define DFLASH_DEVERR_POSITION  0x10u /* position outside [0, max_position) of the RoPE table   */
+
+/* Draft-model geometry.  block_size / mask_token_id / target_layer_ids are the
+ * fields of the pages' DFlashConfig; the rest is the Qwen3 layer shape.
+ * Supported: head_dim in {64, 128}; hidden, n_q_heads*head_dim, intermediate and
+ * n_target_layers*hidden multiples of 64; vocab a multiple of 32;
+ * n_q_heads % n_kv_heads == 0 with block_size*(n_q_heads/n_kv_heads) <= 128;
+ * 2 <= block_size <= 64; n_layers <= 64; page_size == 16. */
+typedef struct dflash_config {
+  int hidden;
+  int n_layers;
+  int n_q_heads;
+  int n_kv_heads;
+  int head_dim;
+  int intermediate;
+  int vocab;
+  int n_target_layers;            /* number of tapped target layers (T)                   */
+  const int* target_layer_ids;    /* HOST array [n_target_layers], concat order; recorded */
+                                  /* for validation only (may be NULL)                    */
+  int block_size;                 /* bs; the call proposes K = bs - 1 drafts              */
+  int mask_token_id;
+  int page_size;                  /* tokens per KV page (16)                              */
+  float rms_eps;
+  float rope_theta;
+  int max_position;               /* RoPE table covers positions [0, max_position)        */
+} dflash_config;
+
+/* Draft weights: DEVICE pointers, bf16, row-major [out_features, in_features].
+ * Per-layer entries are HOST arrays of n_layers device pointers.
+ *   fc_w [H, T*H]   hidden_norm_w [H]   embed [V, H]   lm_head [V, H]   final_norm_w [H]
+ *   in_norm_w/post_norm_w [H]   wq [Hq*d, H]   wk, wv [Hkv*d, H]   wo [H, Hq*d]
+ *   q_norm_w, k_norm_w [d]      w_gate, w_up [I, H]   w_down [H, I]
+ * dflash_create copies wq/wk/wv, w_gate/w_up and the stacked K/V weights into
+ * packed buffers it owns; every other pointer is kept and must stay valid (and
+ * unchanged) for the lifetime of the handle (embed / lm_head are the target's
+ * aliased tables and are not copied). */
+typedef struct dflash_weights {
+  const void* fc_w;
+  const void* hidden_norm_w;
+  const void* embed;
+  const void* lm_head;
+  const void* final_norm_w;
+  const void* const* in_norm_w;
+  const void* const* post_norm_w;
+  const void* const* wq;
+  const void* const* wk;
+  const void* const* wv;
+  const void* const* wo;
+  const void* const* q_norm_w;
+  const void* const* k_norm_w;
+  const void* const* w_gate;
+  const void* const* w_up;
+  const void* const* w_down;
+} dflash_weights;
+
+typedef struct dflash_handle dflash_handle;
+
+/* Validates the geometry, makes `device` current, packs the weights and builds
+ * the RoPE table (cos/sin of pos * theta^(-2i/d), evaluated in double precision
+ * on the device).  Synchronizes the device once at the end.  On success *out
+ * receives the handle; on failure *out is NULL and nothing is leaked. */
+dflash_status dflash_create(const dflash_config* cfg, const dflash_weights* w,
+                            int device, dflash_handle** out);
+
+/* Frees everything the handle owns.  The caller must make sure no work that
+ * uses the handle is still pending.  NULL is a no-op. */
+void dflash_destroy(dflash_handle* h);
+
+/* Workspace (device memory, >= 256-byte aligned, contents need not be
+ * initialised) needed by dflash_inject_context for up to `max_rows` rows. */
+size_t dflash_inject_workspace_bytes(const dflash_handle* h, int max_rows);
+
+/* Workspace needed by dflash_propose for a batch of up to `max_batch` requests
+ * with block tables `max_pages_per_seq` entries wide. */
+size_t dflash_propose_workspace_bytes(const dflash_handle* h, int max_batch,
+                                      int max_pages_per_seq);
+
+/* Workspace needed by dflash_verify_greedy for [B, K+1, V] target logits. */
+size_t dflash_verify_workspace_bytes(int B, int K, int V);
+
+/* _paged_slots (§"Paged KV Integration"), exactly as the page writes it:
+ *   page_no = min(positions[i] / page_size, max_pages_per_seq - 1)
+ *   slots[i] = block_table[req_ids[i] * max_pages_per_seq + page_no] * page_size
+ *              + positions[i] % page_size
+ * positions, req_ids: [n] int64 (>= 0); block_table: [*, max_pages_per_seq] int32;
+ * slots: [n] int64 out.  Note the clamp: a position past the table aliases the
+ * row's last page.  A negative position yields slot -1 (a padding row).
+ * req_ids must index existing block-table rows.  n == 0 is a no-op. */
+dflash_status dflash_paged_slots(const int64_t* positions, const int64_t* req_ids,
+                                 int n, const int32_t* block_table,
+                                 int max_pages_per_seq, int page_size,
+                                 int64_t* slots, void* stream);
+
+/* precompute_and_store_context_kv (§"Context KV Injection (Precompute)"):
+ *   ctx = hidden_norm(fc(aux))                       [n, H]
+ *   for every layer l and kv head h:
+ *     k = RoPE(k_norm_l(Wk_l,h ctx), positions)      written to k_cache[l]
+ *     v = Wv_l,h ctx                                 written to v_cache[l]
+ * at slot_mapping (slot s -> page s / page_size, offset s % page_size).
+ *   aux          [n, T*H] bf16, the target's tapped states concatenated in
+ *                target_layer_ids order
+ *   positions    [n] int64 absolute positions (RoPE), 0 <= pos < max_position
+ *   slot_mapping [n] int64; a negative slot marks a padding row, skipped
+ *   k_cache, v_cache: HOST arrays of n_layers device pointers, each pool
+ *                [num_pages, n_kv_heads, page_size, head_dim] bf16
+ * n == 0 is a no-op.  Needs dflash_inject_workspace_bytes(h, n) of workspace. */
+dflash_status dflash_inject_context(dflash_handle* h, const void* aux,
+                                    const int64_t* positions,
+                                    const int64_t* slot_mapping, int n,
+                                    void* const* k_cache, void* const* v_cache,
+                                    int num_pages, void* workspace,
+                                    size_t workspace_bytes, void* stream);
+
+/* One draft proposal for B requests (DFlashQwen3ForCausalLM.forward after
+ * injection).  Request b's block is [bonus_tokens[b], mask, ..., mask] at
+ * positions seq_lens[b] + [0, bs); every block query attends (non-causally) to
+ * the request's keys [0, seq_lens[b] + bs): its injected context and its whole
+ * block.  The block's own K/V are written to the cache at those positions
+ * (they are scratch until the next injection overwrites them).
+ *   bonus_tokens  [B] int32        seq_lens [B] int32 (context tokens injected)
+ *   block_table   [B, max_pages_per_seq] int32; must cover seq_len + bs - 1
+ *   draft_tokens  [B, K] int32 out (K = bs - 1), greedy argmax of the LM head on
+ *                 block slots 1..bs-1 (ties -> lowest id; NaN counts as -inf)
+ *   block_tokens  [B, bs] int32 out, cat(bonus, drafts); may be NULL
+ *   logits_out    [B*K, V] fp32 out (debug); may be NULL
+ * B == 0 is a no-op.  Needs dflash_propose_workspace_bytes(h, B, max_pages_per_seq). */
+dflash_status dflash_propose(dflash_handle* h, const int32_t* bonus_tokens,
+                             const int32_t* seq_lens, const int32_t* block_table,
+                             int B, int max_pages_per_seq, void* const* k_cache,
+                             void* const* v_cache, int num_pages,
+                             int32_t* draft_tokens, int32_t* block_tokens,
+                             float* logits_out, void* workspace,
+                             size_t workspace_bytes, void* stream);
+
+/* Greedy verification.  target_logits row j (j = 0..K) of request b is the
+ * target's prediction after block slot j (slot 0 = previous bonus token,
+ * slot j = drafts[b][j-1]).  With t_j = argmax_v target_logits[b][j][v] (fp32
+ * compare, ties -> lowest index, NaN counts as -inf):
+ *   n = largest m <= K with drafts[b][i] == t_i for all i < m
+ *   out_tokens[b] = [drafts[b][0..n-1], t_n, -1, ..., -1]   ([B, K+1] int32)
+ *   num_accepted[b] = n, bonus[b] = t_n                      ([B] int32 each)
+ * drafts [B, K] int32; target_logits [B, K+1, V] fp32.  Bit-exact by construction.
+ * B == 0 is a no-op.  Needs dflash_verify_workspace_bytes(B, K, V). */
+dflash_status dflash_verify_greedy(const int32_t* drafts, const float* target_logits,
+                                   int B, int K, int V, int32_t* out_tokens,
+                                   int32_t* num_accepted, int32_t* bonus,
+                                   void* workspace, size_t workspace_bytes,
+                                   void* stream);
+
+/* ---- component entry points (each runs one kernel family of the path) ---- */
+
+/* out[m, n] = sum_k A[m, k] * W[n, k] in fp32 — the tcgen05 GEMM that every
+ * projection of the path runs on, with a plain fp32 store as its epilogue.
+ *   A [M, K] bf16, W [N, K] bf16 (row-major), out [M, N] fp32.
+ * K must be a multiple of 64 and N a multiple of 32.  M == 0 is a no-op.
+ * Needs dflash_linear_workspace_bytes(h, M, N, K) of workspace. */
+size_t dflash_linear_workspace_bytes(const dflash_handle* h, int M, int N, int K);
+dflash_status dflash_linear(dflash_handle* h, const void* A, const void* W, int M, int N,
+                            int K, float* out, void* workspace, size_t workspace_bytes,
+                            void* stream);
+/* Same with the launch plan chosen by the caller: tile width block_n in
+ * {32, 64, 128, 256} and K-split count `splits` (>= 1, <= K/64); 0 for either
+ * means "as the automatic plan".  Split-K needs splits*M*N*4 bytes of
+ * workspace (dflash_linear_workspace_bytes covers only the automatic plan). */
+dflash_status dflash_linear_ex(dflash_handle* h, const void* A, const void* W, int M, int N,
+                               int K, float* out, int block_n, int splits, void* workspace,
+                               size_t workspace_bytes, void* stream);
+
+/* One layer of non-causal block attention (§"What is DFlash": every block query
+ * attends to the injected context and the whole block), on a layer's caches:
+ *   q [B*bs, n_q_heads, head_dim] bf16 (block rows in request order)
+ *   o [B*bs, n_q_heads*head_dim] bf16 out
+ * Request b attends to its logical keys [0, seq_lens[b] + bs), located through
+ * block_table exactly as in dflash_propose; scale 1/sqrt(head_dim).
+ * Needs dflash_attention_workspace_bytes(h, B, max_pages_per_seq). */
+size_t dflash_attention_workspace_bytes(const dflash_handle* h, int B, int max_pages_per_seq);
+dflash_status dflash_block_attention(dflash_handle* h, const void* q, const int32_t* seq_lens,
+                                     const int32_t* block_table, int B, int max_pages_per_seq,
+                                     const void* k_cache, const void* v_cache, int num_pages,
+                                     void* o, void* workspace, size_t workspace_bytes,
+                                     void* stream);
+
+/* Synchronizes the device, reads and clears the handle's device error word.
+ * Returns DFLASH_OK if it was zero, DFLASH_ERR_DEVICE_TIMEOUT if the timeout bit
+ * was set, DFLASH_ERR_DEVICE_BOUNDS otherwise; *bits (may be NULL) receives the
+ * raw DFLASH_DEVERR_* mask.  (verify and paged_slots take no handle and have
+ * no device-detected error conditions.) */
+dflash_status dflash_check_device_errors(dflash_handle* h, unsigned* bits);
+
+/* Static, human-readable name of a status code. */
+const char* dflash_status_string(dflash_status s);
+
+/* Library build identification (static string). */
+const char* dflash_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DFLASH_H_ */

@@ -1,0 +1,262 @@
+"""GPU parity of the library's kernel families, called through the C ABI.
+
+  * dflash_linear(_ex)        the tcgen05 GEMM, every tile width and split-K,
+                              against a float64 torch matmul of the same bf16 inputs
+  * dflash_block_attention    against the oracle's non-causal paged attention
+  * dflash_inject_context     against the oracle's injection (bf16 storage mode)
+  * dflash_verify_greedy      bit-exact against the oracle
+  * dflash_paged_slots        bit-exact against the oracle
+"""
+
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from block_diffusion_speculative_propose_b200 import DFlash, paged_slots, synth, verify_greedy
+from tests._util import rel_l2, to_np, weights_np, weights_to
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+@pytest.fixture(scope="module")
+def tiny():
+    cfg = synth.model_config("tiny")
+    Wt = synth.make_weights(cfg, seed=0)
+    h = DFlash(cfg, weights_to(Wt, DEV), max_position=4096)
+    yield cfg, Wt, h
+    h.close()
+
+
+# ----------------------------------------------------------------------------
+# GEMM
+# ----------------------------------------------------------------------------
+GEMM_CASES = [
+    # (M, N, K, block_n, splits)   0 = automatic plan
+    (1, 256, 64, 0, 0),
+    (16, 4096, 4096, 0, 0),
+    (15, 4096, 1024, 32, 1),
+    (15, 4096, 1024, 64, 1),
+    (15, 4096, 1024, 128, 1),
+    (15, 4096, 1024, 256, 1),
+    (16, 1024, 4096, 128, 4),
+    (16, 1024, 4096, 32, 3),
+    (129, 96, 192, 32, 1),
+    (129, 96, 192, 32, 3),
+    (300, 1536, 512, 0, 0),
+    (512, 4096, 4096, 256, 1),
+    (1000, 2080, 640, 0, 0),
+    (2048, 1024, 1024, 256, 1),
+]
+
+
+@pytest.mark.parametrize("M,N,K,bn,splits", GEMM_CASES)
+def test_linear_matches_float64_matmul(tiny, M, N, K, bn, splits):
+    h = tiny[2]
+    g = torch.Generator().manual_seed(M * 7919 + N * 31 + K)
+    A = torch.randn(M, K, generator=g).to(torch.bfloat16)
+    W = (0.05 * torch.randn(N, K, generator=g)).to(torch.bfloat16)
+    ref = A.double() @ W.double().T
+    out = h.linear(A.to(DEV), W.to(DEV), block_n=bn, splits=splits)
+    torch.cuda.synchronize()
+    got = out.cpu().double()
+    err = (got - ref).abs().max().item()
+    scale = ref.abs().max().item()
+    assert err <= 2e-5 * scale + 1e-6, (err, scale)
+    assert h.check_device_errors() == 0
+
+
+def test_linear_split_k_is_deterministic(tiny):
+    h = tiny[2]
+    g = torch.Generator().manual_seed(5)
+    A = torch.randn(16, 4096, generator=g).to(torch.bfloat16).to(DEV)
+    W = (0.05 * torch.randn(2048, 4096, generator=g)).to(torch.bfloat16).to(DEV)
+    a = h.linear(A, W, block_n=64, splits=8).clone()
+    b = h.linear(A, W, block_n=64, splits=8).clone()
+    assert torch.equal(a, b)
+
+
+# ----------------------------------------------------------------------------
+# attention
+# ----------------------------------------------------------------------------
+def _pool(cfg, seq_lens, seed, extra=5):
+    """Shuffled page pool large enough for every request's seq_len + bs keys."""
+    rng = np.random.default_rng(seed)
+    P, bs = cfg["page_size"], cfg["block_size"]
+    need = [-(-(s + bs) // P) for s in seq_lens]
+    W = max(need) + 2
+    num_pages = sum(need) + extra
+    perm = rng.permutation(num_pages)
+    table = np.zeros((len(seq_lens), W), dtype=np.int32)
+    cur = 0
+    for b, n in enumerate(need):
+        table[b, :n] = perm[cur:cur + n]
+        cur += n
+    return table, num_pages
+
+
+def _attention_case(cfg, seq_lens, seed):
+    oc = O.OracleConfig.from_mapping(cfg)
+    table, num_pages = _pool(cfg, seq_lens, seed)
+    g = torch.Generator().manual_seed(seed)
+    shape = (num_pages, cfg["n_kv_heads"], cfg["page_size"], cfg["head_dim"])
+    kc = torch.randn(shape, generator=g).to(torch.bfloat16)
+    vc = torch.randn(shape, generator=g).to(torch.bfloat16)
+    # NaN in unused slots must not leak into results (P = 0 rows)
+    kc.view(-1)[-cfg["head_dim"]:] = float("nan")
+    B = len(seq_lens)
+    q = torch.randn(B * cfg["block_size"], cfg["n_q_heads"], cfg["head_dim"],
+                    generator=g).to(torch.bfloat16)
+    ref = O.block_attention(oc, to_np(q).astype(np.float64), to_np(kc).astype(np.float64),
+                            to_np(vc).astype(np.float64), table, seq_lens)
+    return q, kc, vc, table, ref
+
+
+@pytest.mark.parametrize("model,seq_lens", [
+    ("tiny", [64]),
+    ("tiny", [0, 1, 15, 16, 17, 63, 64, 65, 200]),
+    ("qwen3_8b", [2048]),
+    ("qwen3_8b", [0, 7, 100, 1000, 5000]),
+    ("llama31_8b", [3, 333, 4097]),
+])
+def test_block_attention_matches_oracle(model, seq_lens):
+    cfg = synth.model_config(model)
+    # the attention entry point needs only geometry: a handle with tiny weights
+    # of the same head layout
+    small = dict(cfg, intermediate=256, vocab=1024, n_layers=1, mask_token_id=1023,
+                 n_target_layers=1)
+    W = synth.make_weights(small, seed=1)
+    h = DFlash(small, weights_to(W, DEV), max_position=4096)
+    try:
+        q, kc, vc, table, ref = _attention_case(cfg, seq_lens, seed=len(seq_lens))
+        o = h.block_attention(q.to(DEV), torch.tensor(seq_lens, dtype=torch.int32, device=DEV),
+                              torch.tensor(table, device=DEV), kc.to(DEV), vc.to(DEV))
+        torch.cuda.synchronize()
+        got = to_np(o).astype(np.float64).reshape(ref.shape)
+        assert np.isfinite(got).all()
+        for b in range(len(seq_lens)):
+            rows = slice(b * cfg["block_size"], (b + 1) * cfg["block_size"])
+            assert rel_l2(got[rows], ref[rows]) < 8e-3, (b, seq_lens[b])
+        assert h.check_device_errors() == 0
+    finally:
+        h.close()
+
+
+# ----------------------------------------------------------------------------
+# verify / paged slots
+# ----------------------------------------------------------------------------
+@pytest.mark.parametrize("B,K,V", [(1, 3, 1024), (3, 15, 151936), (37, 9, 128256),
+                                   (5, 0, 1000), (4, 4, 1027)])
+def test_verify_bit_exact(B, K, V):
+    g = torch.Generator().manual_seed(B * 100 + K)
+    n_acc = torch.randint(0, K + 1, (B,), generator=g)
+    drafts = torch.randint(0, V, (B, K), generator=g, dtype=torch.int32)
+    T = synth.make_target_logits(g, drafts, n_acc, V)
+    if B > 2 and K > 1:
+        T[0, 1, :] = 0.5                        # all-equal row -> index 0
+        T[1, 0, 7] = float("nan")
+        T[2, 1, :] = float("-inf")
+    ref = O.verify_greedy(to_np(drafts), to_np(T))
+    out, n, bonus = verify_greedy(drafts.to(DEV), T.to(DEV))
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(to_np(out), ref.out_tokens)
+    np.testing.assert_array_equal(to_np(n), ref.num_accepted)
+    np.testing.assert_array_equal(to_np(bonus), ref.bonus)
+
+
+def test_verify_full_size_logits():
+    """[128, 16, 151936] fp32 logits with geometric acceptance (mean tau ~ 6)."""
+    cfg = synth.model_config("qwen3_8b")
+    sb = synth.make_step_batch(cfg, 128, 8192, 32768, accept="geometric", seed=3,
+                               with_aux=False)
+    ref = O.verify_greedy(to_np(sb.prev_drafts), to_np(sb.target_logits))
+    np.testing.assert_array_equal(ref.num_accepted, to_np(sb.n_accept))
+    out, n, bonus = verify_greedy(sb.prev_drafts.to(DEV), sb.target_logits.to(DEV))
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(to_np(out), ref.out_tokens)
+    np.testing.assert_array_equal(to_np(n), ref.num_accepted)
+    np.testing.assert_array_equal(to_np(bonus), ref.bonus)
+
+
+def test_paged_slots_bit_exact():
+    rng = np.random.default_rng(0)
+    table = rng.integers(0, 10000, (7, 33)).astype(np.int32)
+    pos = rng.integers(0, 33 * 16 + 40, 5000)          # includes clamped positions
+    req = rng.integers(0, 7, 5000)
+    ref = O.paged_slots(pos, req, table, 16)
+    got = paged_slots(torch.tensor(pos, device=DEV), torch.tensor(req, device=DEV),
+                      torch.tensor(table, device=DEV))
+    np.testing.assert_array_equal(to_np(got), ref)
+    neg = paged_slots(torch.tensor([-1, 3], device=DEV), torch.tensor([0, 0], device=DEV),
+                      torch.tensor(table, device=DEV))
+    assert to_np(neg).tolist() == [-1, int(table[0, 0]) * 16 + 3]
+
+
+# ----------------------------------------------------------------------------
+# injection
+# ----------------------------------------------------------------------------
+def _inject_case(cfg, Wt, h, n, seed, sample=None):
+    oc = O.OracleConfig.from_mapping(cfg)
+    rng = np.random.default_rng(seed)
+    P = cfg["page_size"]
+    num_pages = -(-(n + 40) // P) + 7
+    table = rng.permutation(num_pages)[None, :].astype(np.int32)
+    pos = np.arange(n, dtype=np.int64) + 40
+    slots = O.paged_slots(pos, np.zeros(n, np.int64), table, P)
+    slots[rng.random(n) < 0.1] = -1                      # padding rows
+    aux = synth.make_aux(n, cfg, seed)
+    shape = (num_pages, cfg["n_kv_heads"], P, cfg["head_dim"])
+    sentinel = 7.0
+    kc = [torch.full(shape, sentinel, dtype=torch.bfloat16, device=DEV)
+          for _ in range(cfg["n_layers"])]
+    vc = [torch.full(shape, sentinel, dtype=torch.bfloat16, device=DEV)
+          for _ in range(cfg["n_layers"])]
+    h.inject_context(aux.to(DEV), torch.tensor(pos, device=DEV),
+                     torch.tensor(slots, device=DEV), kc, vc)
+    torch.cuda.synchronize()
+    assert h.check_device_errors() == 0
+    rows = np.arange(n) if sample is None else sample
+    W = weights_np(Wt) if not isinstance(Wt["fc_w"], np.ndarray) else Wt
+    auxn = to_np(aux)[rows].astype(np.float64)
+    ctx_io = O.context_fusion(oc, W, auxn, "bf16io")
+    k_io, v_io = O.context_kv(oc, W, ctx_io, pos[rows], "bf16io")
+    ctx_ex = O.context_fusion(oc, W, auxn, "exact")
+    k_ex, v_ex = O.context_kv(oc, W, ctx_ex, pos[rows], "exact")
+    for l in range(cfg["n_layers"]):
+        kg, vg = to_np(kc[l]), to_np(vc[l])
+        for j, r in enumerate(rows):
+            s = slots[r]
+            if s < 0:
+                continue
+            gk, gv = kg[s // P, :, s % P], vg[s // P, :, s % P]
+            # one bf16 ulp against the bf16-storage oracle, 1e-2 rel-L2 against exact
+            assert np.all(np.abs(gk - k_io[l][j]) <= 2 ** -7 * np.abs(k_io[l][j]) + 1e-6), (l, r)
+            assert np.all(np.abs(gv - v_io[l][j]) <= 2 ** -7 * np.abs(v_io[l][j]) + 1e-6), (l, r)
+            assert rel_l2(gk, k_ex[l][j]) < 1e-2 and rel_l2(gv, v_ex[l][j]) < 1e-2
+        # padding rows and untouched slots keep the sentinel
+        for r in np.nonzero(slots < 0)[0][:8]:
+            s = O.paged_slots(pos[r:r + 1], np.zeros(1, np.int64), table, P)[0]
+            assert (kg[s // P, :, s % P] == sentinel).all()
+
+
+def test_inject_tiny(tiny):
+    cfg, Wt, h = tiny
+    for n in (1, 5, 64, 130):
+        _inject_case(cfg, Wt, h, n, seed=n)
+
+
+def test_inject_qwen3_shape_sampled():
+    cfg = synth.model_config("qwen3_8b")
+    Wt = synth.make_weights(cfg, seed=0)
+    h = DFlash(cfg, weights_to(Wt, DEV), max_position=40960)
+    try:
+        rng = np.random.default_rng(1)
+        W = weights_np({k: Wt[k] for k in ("fc_w", "hidden_norm_w", "wk", "wv", "k_norm_w")})
+        for n in (16, 2048):
+            sample = np.sort(rng.choice(n, size=min(n, 12), replace=False))
+            _inject_case(cfg, W, h, n, seed=n, sample=sample)
+    finally:
+        h.close()
