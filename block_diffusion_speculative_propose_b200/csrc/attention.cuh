@@ -4,7 +4,9 @@
 // of the kv group (bs block slots x G = Hq / Hkv query heads) attend, with no
 // mask inside the range, to keys [split * chunk, ...) of the request's logical
 // keys [0, seq_len + bs) — its injected context plus its whole block.  Each K
-// and V byte is read from HBM once per kv group.
+// and V byte is read from HBM once per kv group.  Compute warps are laid out as
+// (row group of 16 query rows) x (key part of each 64-key tile); the parts'
+// softmax states are merged in shared memory after the last tile.
 //
 // Pages are staged with TMA tile loads (128-byte swizzle, one 16-row x 128-byte
 // box per page and 64-wide half of head_dim) into a ring of shared-memory
@@ -33,11 +35,15 @@ struct AttnCfg {
   static constexpr int smem_bytes(int n_compute_warps) {
     return 1024 + kAttnStages * 2 * kKVBytes + n_compute_warps * 16 * kQStride * 2 + 256;
   }
+  static_assert(kAttnStages * 2 * kKVBytes >= 7 * 16 * D * 4 + 7 * 32 * 16,
+                "the stage buffers hold the key-part merge");
 };
 
 struct AttnParams {
+  int row_groups;      // ceil(R / 16)
+  int key_parts;       // compute warps per row group (each takes 64 / key_parts keys of a tile)
   const bf16* q;       // [M, Hq, D]
-  bf16* o;             // [M, Hq * D]
+  f16* o;              // [M, Hq * D] (convex combinations of V rows: fp16)
   float* part_o;       // [max_splits][B][Hkv][R][D]
   float* part_ml;      // [max_splits][B][Hkv][R][2]
   const int* seq_lens;
@@ -61,18 +67,20 @@ __device__ __forceinline__ uint32_t kv_off(int kt, int c) {
                                rp * 128 + ((cc ^ (rp & 7)) << 4));
 }
 
-template <int D>
+template <int D, int KP>
 __global__ void __launch_bounds__(32 * (kAttnMaxComputeWarps + 1), 1)
     attn_block_kernel(const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
   using C = AttnCfg<D>;
+  constexpr int NB = KP / 8;    // 8-key blocks of this warp's part of a tile
+  constexpr int KS = KP / 16;   // 16-key (one page) PV steps
   const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int n_keys = p.seq_lens[b] + p.bs;
   const int k0 = split * p.chunk_keys;
   if (k0 >= n_keys) return;
   const int k1 = min(n_keys, k0 + p.chunk_keys);
   const int n_splits_b = (n_keys + p.chunk_keys - 1) / p.chunk_keys;
-  const int nwc = (blockDim.x >> 5) - 1;
+  const int nwc = p.row_groups * p.key_parts;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   extern __shared__ uint8_t smem_raw[];
@@ -141,11 +149,13 @@ __global__ void __launch_bounds__(32 * (kAttnMaxComputeWarps + 1), 1)
   }
 
   // -------------------------------------------------------------- compute warps
+  const int rg = warp % p.row_groups;   // query rows rg*16 .. rg*16+15
+  const int kp = warp / p.row_groups;   // keys kp*KP .. kp*KP+KP-1 of every tile
   // Q rows of this warp: r = i * G + g  ->  q[(b*bs + i), h*G + g, :]
   bf16* sQw = sQ + warp * 16 * C::kQStride;
   for (int e = lane; e < 16 * (D / 8); e += 32) {
     const int rr = e / (D / 8), c = e - rr * (D / 8);
-    const int r = warp * 16 + rr;
+    const int r = rg * 16 + rr;
     uint4 val = make_uint4(0, 0, 0, 0);
     if (r < p.R) {
       const int i = r / p.G, g = r - (r / p.G) * p.G;
@@ -173,109 +183,112 @@ __global__ void __launch_bounds__(32 * (kAttnMaxComputeWarps + 1), 1)
   uint32_t stage = 0, phase = 0;
   for (int t = 0; t < n_tiles; ++t) {
     const int t0 = k0 + t * kAttnTileKeys;
-    const int nvalid = min(kAttnTileKeys, k1 - t0);
+    const int nvalid = min(kAttnTileKeys, k1 - t0) - kp * KP;   // valid keys of this part
     if (!mbar_wait(&full[stage], phase, p.err)) break;
-    const uint32_t kbase = smem_u32(sK + stage * C::kKVBytes);
-    const uint32_t vbase = smem_u32(sV + stage * C::kKVBytes);
-
-    if (nvalid & 15) {
-      // Rows past the last key of a partly used page may hold anything
-      // (including NaN bit patterns); zero them so that P = 0 rows add 0.
-      const int jp = nvalid >> 4, r0 = nvalid & 15;
-      uint8_t* vb = sV + stage * C::kKVBytes;
-      const int n16 = (16 - r0) * C::kBoxesPerPage * 8;
-      for (int e = lane; e < n16; e += 32) {
-        const int hf = e / ((16 - r0) * 8);
-        const int rem = e - hf * (16 - r0) * 8;
-        const int rr = r0 + rem / 8, cc = rem & 7;
-        *reinterpret_cast<uint4*>(vb + (jp * C::kBoxesPerPage + hf) * C::kBoxBytes + rr * 128 +
-                                  cc * 16) = make_uint4(0, 0, 0, 0);
+    if (nvalid > 0) {
+      const uint32_t kbase = smem_u32(sK + stage * C::kKVBytes);
+      const uint32_t vbase = smem_u32(sV + stage * C::kKVBytes);
+      if (nvalid < KP && (nvalid & 15)) {
+        // Rows past the last key of a partly used page may hold anything
+        // (including NaN bit patterns); zero them so that P = 0 rows add 0.
+        const int jp = (kp * KP + nvalid) >> 4, r0 = nvalid & 15;
+        uint8_t* vb = sV + stage * C::kKVBytes;
+        const int n16 = (16 - r0) * C::kBoxesPerPage * 8;
+        for (int e = lane; e < n16; e += 32) {
+          const int hf = e / ((16 - r0) * 8);
+          const int rem = e - hf * (16 - r0) * 8;
+          const int rr = r0 + rem / 8, cc = rem & 7;
+          *reinterpret_cast<uint4*>(vb + (jp * C::kBoxesPerPage + hf) * C::kBoxBytes +
+                                    rr * 128 + cc * 16) = make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
       }
-      fence_proxy_async_smem();
-      __syncwarp();
-    }
 
-    // S = Q K^T over the 64 keys of the tile (8 blocks of 8 keys)
-    float s[8][4];
+      // S = Q K^T over this part's keys
+      float s[NB][4];
 #pragma unroll
-    for (int nb = 0; nb < 8; ++nb) s[nb][0] = s[nb][1] = s[nb][2] = s[nb][3] = 0.f;
+      for (int nb = 0; nb < NB; ++nb) s[nb][0] = s[nb][1] = s[nb][2] = s[nb][3] = 0.f;
 #pragma unroll
-    for (int ks = 0; ks < D / 16; ++ks) {
+      for (int ks = 0; ks < D / 16; ++ks) {
+        if constexpr (NB >= 2) {
 #pragma unroll
-      for (int nbp = 0; nbp < 4; ++nbp) {
-        const int j = lane >> 3;
-        const int kt = (nbp * 2 + (j >> 1)) * 8 + (lane & 7);
-        const int c = ks * 2 + (j & 1);
-        uint32_t b00, b01, b10, b11;
-        ldmatrix_x4(kbase + kv_off<D>(kt, c), b00, b01, b10, b11);
-        mma_bf16_16816(s[2 * nbp], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b00, b01);
-        mma_bf16_16816(s[2 * nbp + 1], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b10, b11);
+          for (int nbp = 0; nbp < NB / 2; ++nbp) {
+            const int j = lane >> 3;
+            const int kt = kp * KP + (nbp * 2 + (j >> 1)) * 8 + (lane & 7);
+            const int c = ks * 2 + (j & 1);
+            uint32_t b00, b01, b10, b11;
+            ldmatrix_x4(kbase + kv_off<D>(kt, c), b00, b01, b10, b11);
+            mma_bf16_16816(s[2 * nbp], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b00, b01);
+            mma_bf16_16816(s[2 * nbp + 1], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b10,
+                           b11);
+          }
+        }
       }
-    }
 
-    // scale into the log2 domain, mask keys past the range, online softmax
-    float mx[2] = {m_run[0], m_run[1]};
+      // scale into the log2 domain, mask keys past the range, online softmax
+      float mx[2] = {m_run[0], m_run[1]};
 #pragma unroll
-    for (int nb = 0; nb < 8; ++nb) {
+      for (int nb = 0; nb < NB; ++nb) {
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int kt = nb * 8 + 2 * (lane & 3) + (e & 1);
-        const float v = s[nb][e] * p.scale_log2;
-        s[nb][e] = (kt < nvalid) ? v : -INFINITY;
-        mx[e >> 1] = fmaxf(mx[e >> 1], s[nb][e]);
+        for (int e = 0; e < 4; ++e) {
+          const int kt = nb * 8 + 2 * (lane & 3) + (e & 1);
+          const float v = s[nb][e] * p.scale_log2;
+          s[nb][e] = (kt < nvalid) ? v : -INFINITY;
+          mx[e >> 1] = fmaxf(mx[e >> 1], s[nb][e]);
+        }
       }
-    }
 #pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      mx[hh] = fmaxf(mx[hh], __shfl_xor_sync(0xffffffffu, mx[hh], 1));
-      mx[hh] = fmaxf(mx[hh], __shfl_xor_sync(0xffffffffu, mx[hh], 2));
-    }
-    float ref[2], alpha[2];
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      ref[hh] = (mx[hh] == -INFINITY) ? 0.f : mx[hh];
-      alpha[hh] = exp2f(m_run[hh] - ref[hh]);  // m_run = -inf -> 0
-      m_run[hh] = mx[hh];
-      l_run[hh] *= alpha[hh];
-    }
-#pragma unroll
-    for (int i = 0; i < D / 8; ++i) {
-      o[i][0] *= alpha[0];
-      o[i][1] *= alpha[0];
-      o[i][2] *= alpha[1];
-      o[i][3] *= alpha[1];
-    }
-#pragma unroll
-    for (int nb = 0; nb < 8; ++nb) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float pv = exp2f(s[nb][e] - ref[e >> 1]);
-        s[nb][e] = pv;
-        l_run[e >> 1] += pv;
+      for (int hh = 0; hh < 2; ++hh) {
+        mx[hh] = fmaxf(mx[hh], __shfl_xor_sync(0xffffffffu, mx[hh], 1));
+        mx[hh] = fmaxf(mx[hh], __shfl_xor_sync(0xffffffffu, mx[hh], 2));
       }
-    }
+      float ref[2], alpha[2];
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        ref[hh] = (mx[hh] == -INFINITY) ? 0.f : mx[hh];
+        alpha[hh] = exp2f(m_run[hh] - ref[hh]);  // m_run = -inf -> 0
+        m_run[hh] = mx[hh];
+        l_run[hh] *= alpha[hh];
+      }
+#pragma unroll
+      for (int i = 0; i < D / 8; ++i) {
+        o[i][0] *= alpha[0];
+        o[i][1] *= alpha[0];
+        o[i][2] *= alpha[1];
+        o[i][3] *= alpha[1];
+      }
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float pv = exp2f(s[nb][e] - ref[e >> 1]);
+          s[nb][e] = pv;
+          l_run[e >> 1] += pv;
+        }
+      }
 
-    // O += P V, 16 keys (one page) per k-step
+      // O += P V, 16 keys (one page) per k-step
 #pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      if (kk * 16 < nvalid) {
-        const uint32_t a0 = pack_bf16x2(s[2 * kk][0], s[2 * kk][1]);
-        const uint32_t a1 = pack_bf16x2(s[2 * kk][2], s[2 * kk][3]);
-        const uint32_t a2 = pack_bf16x2(s[2 * kk + 1][0], s[2 * kk + 1][1]);
-        const uint32_t a3 = pack_bf16x2(s[2 * kk + 1][2], s[2 * kk + 1][3]);
+      for (int kk = 0; kk < KS; ++kk) {
+        if (kk * 16 < nvalid) {
+          const uint32_t a0 = pack_bf16x2(s[2 * kk][0], s[2 * kk][1]);
+          const uint32_t a1 = pack_bf16x2(s[2 * kk][2], s[2 * kk][3]);
+          const uint32_t a2 = pack_bf16x2(s[2 * kk + 1][0], s[2 * kk + 1][1]);
+          const uint32_t a3 = pack_bf16x2(s[2 * kk + 1][2], s[2 * kk + 1][3]);
 #pragma unroll
-        for (int dbp = 0; dbp < D / 16; ++dbp) {
-          const int j = lane >> 3;
-          const int kt = kk * 16 + (j & 1) * 8 + (lane & 7);
-          const int c = dbp * 2 + (j >> 1);
-          uint32_t b0, b1, b2, b3;
-          ldmatrix_x4_trans(vbase + kv_off<D>(kt, c), b0, b1, b2, b3);
-          mma_bf16_16816(o[2 * dbp], a0, a1, a2, a3, b0, b1);
-          mma_bf16_16816(o[2 * dbp + 1], a0, a1, a2, a3, b2, b3);
+          for (int dbp = 0; dbp < D / 16; ++dbp) {
+            const int j = lane >> 3;
+            const int kt = kp * KP + kk * 16 + (j & 1) * 8 + (lane & 7);
+            const int c = dbp * 2 + (j >> 1);
+            uint32_t b0, b1, b2, b3;
+            ldmatrix_x4_trans(vbase + kv_off<D>(kt, c), b0, b1, b2, b3);
+            mma_bf16_16816(o[2 * dbp], a0, a1, a2, a3, b0, b1);
+            mma_bf16_16816(o[2 * dbp + 1], a0, a1, a2, a3, b2, b3);
+          }
         }
       }
     }
-
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[stage]);
     if (++stage == kAttnStages) {
@@ -290,19 +303,62 @@ __global__ void __launch_bounds__(32 * (kAttnMaxComputeWarps + 1), 1)
     l_run[hh] += __shfl_xor_sync(0xffffffffu, l_run[hh], 2);
   }
 
+  if (p.key_parts > 1) {
+    // merge the key parts of each row group through the (now idle) stage buffers
+    named_bar_sync(1, nwc * 32);
+    float* mo = reinterpret_cast<float*>(smem);
+    float* mml = mo + (p.key_parts - 1) * p.row_groups * 16 * D;
+    if (kp > 0) {
+      const int slot = (kp - 1) * p.row_groups + rg;
+      float* dst = mo + static_cast<size_t>(slot) * 16 * D;
+#pragma unroll
+      for (int db = 0; db < D / 8; ++db)
+        *reinterpret_cast<float4*>(dst + (db * 32 + lane) * 4) =
+            make_float4(o[db][0], o[db][1], o[db][2], o[db][3]);
+      *reinterpret_cast<float4*>(mml + (slot * 32 + lane) * 4) =
+          make_float4(m_run[0], m_run[1], l_run[0], l_run[1]);
+    }
+    named_bar_sync(1, nwc * 32);
+    if (kp > 0) return;
+    for (int j = 1; j < p.key_parts; ++j) {
+      const int slot = (j - 1) * p.row_groups + rg;
+      const float4 ml = *reinterpret_cast<const float4*>(mml + (slot * 32 + lane) * 4);
+      const float mj[2] = {ml.x, ml.y}, lj[2] = {ml.z, ml.w};
+      float a_self[2], a_other[2];
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const float mm = fmaxf(m_run[hh], mj[hh]);
+        const float rf = (mm == -INFINITY) ? 0.f : mm;
+        a_self[hh] = exp2f(m_run[hh] - rf);
+        a_other[hh] = exp2f(mj[hh] - rf);
+        l_run[hh] = l_run[hh] * a_self[hh] + lj[hh] * a_other[hh];
+        m_run[hh] = mm;
+      }
+      const float* src = mo + static_cast<size_t>(slot) * 16 * D;
+#pragma unroll
+      for (int db = 0; db < D / 8; ++db) {
+        const float4 v = *reinterpret_cast<const float4*>(src + (db * 32 + lane) * 4);
+        o[db][0] = o[db][0] * a_self[0] + v.x * a_other[0];
+        o[db][1] = o[db][1] * a_self[0] + v.y * a_other[0];
+        o[db][2] = o[db][2] * a_self[1] + v.z * a_other[1];
+        o[db][3] = o[db][3] * a_self[1] + v.w * a_other[1];
+      }
+    }
+  }
+
 #pragma unroll
   for (int hh = 0; hh < 2; ++hh) {
-    const int r = warp * 16 + (lane >> 2) + hh * 8;
+    const int r = rg * 16 + (lane >> 2) + hh * 8;
     if (r >= p.R) continue;
     if (n_splits_b == 1) {
       const int i = r / p.G, g = r - (r / p.G) * p.G;
-      bf16* dst = p.o + (static_cast<size_t>(b * p.bs + i) * p.Hq + h * p.G + g) * D;
+      f16* dst = p.o + (static_cast<size_t>(b * p.bs + i) * p.Hq + h * p.G + g) * D;
       const float inv = 1.f / l_run[hh];
 #pragma unroll
       for (int db = 0; db < D / 8; ++db) {
         const int d = db * 8 + 2 * (lane & 3);
         *reinterpret_cast<uint32_t*>(dst + d) =
-            pack_bf16x2(o[db][2 * hh] * inv, o[db][2 * hh + 1] * inv);
+            pack_f16x2(o[db][2 * hh] * inv, o[db][2 * hh + 1] * inv);
       }
     } else {
       const size_t prow = (static_cast<size_t>(split) * p.B + b) * p.Hkv + h;
@@ -322,38 +378,65 @@ __global__ void __launch_bounds__(32 * (kAttnMaxComputeWarps + 1), 1)
 
 // Merge the split partials of requests that needed more than one split:
 //   m = max_s m_s,  w_s = 2^(m_s - m),  o = sum_s w_s O_s / sum_s w_s l_s
-// One CTA per (request, kv head); splits are summed in index order.
+// One warp per (request, kv head, query row); splits are summed in index order.
 template <int D>
 __global__ void __launch_bounds__(256) attn_combine_kernel(const AttnParams p) {
-  const int h = blockIdx.x, b = blockIdx.y;
+  constexpr int PER = D / 32;   // elements of the row per lane
+  const int gw = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (gw >= p.B * p.Hkv * p.R) return;
+  const int r = gw % p.R;
+  const int h = (gw / p.R) % p.Hkv;
+  const int b = gw / (p.R * p.Hkv);
   const int n_keys = p.seq_lens[b] + p.bs;
-  const int ns = (n_keys + p.chunk_keys - 1) / p.chunk_keys;
+  const int ns = min((n_keys + p.chunk_keys - 1) / p.chunk_keys, p.max_splits);
   if (ns <= 1) return;
-  const int nsc = min(ns, p.max_splits);
-  for (int e = threadIdx.x; e < p.R * (D / 4); e += blockDim.x) {
-    const int r = e / (D / 4), d = (e - r * (D / 4)) * 4;
-    float mmax = -INFINITY;
-    for (int s = 0; s < nsc; ++s) {
-      const size_t prow = (static_cast<size_t>(s) * p.B + b) * p.Hkv + h;
-      mmax = fmaxf(mmax, p.part_ml[(prow * p.R + r) * 2]);
+  auto row_of = [&](int s) {
+    return ((static_cast<size_t>(s) * p.B + b) * p.Hkv + h) * p.R + r;
+  };
+  float mmax = -INFINITY;
+  for (int s = lane; s < ns; s += 32) mmax = fmaxf(mmax, p.part_ml[row_of(s) * 2]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) mmax = fmaxf(mmax, __shfl_xor_sync(0xffffffffu, mmax, off));
+  float acc[PER];
+#pragma unroll
+  for (int j = 0; j < PER; ++j) acc[j] = 0.f;
+  float l = 0.f;
+  for (int s0 = 0; s0 < ns; s0 += 32) {
+    float w = 0.f, wl = 0.f;
+    if (s0 + lane < ns) {
+      const float2 ml = *reinterpret_cast<const float2*>(p.part_ml + row_of(s0 + lane) * 2);
+      w = exp2f(ml.x - mmax);
+      wl = w * ml.y;
     }
-    float l = 0.f, a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-    for (int s = 0; s < nsc; ++s) {
-      const size_t prow = (static_cast<size_t>(s) * p.B + b) * p.Hkv + h;
-      const float2 ml = *reinterpret_cast<const float2*>(p.part_ml + (prow * p.R + r) * 2);
-      const float w = exp2f(ml.x - mmax);
-      const float4 ov = *reinterpret_cast<const float4*>(p.part_o + (prow * p.R + r) * D + d);
-      l += w * ml.y;
-      a0 += w * ov.x;
-      a1 += w * ov.y;
-      a2 += w * ov.z;
-      a3 += w * ov.w;
+    l += wl;
+    const int cnt = min(32, ns - s0);
+    for (int j = 0; j < cnt; ++j) {
+      const float ws = __shfl_sync(0xffffffffu, w, j);
+      const float* src = p.part_o + row_of(s0 + j) * D + lane * PER;
+      if constexpr (PER == 4) {
+        const float4 v = *reinterpret_cast<const float4*>(src);
+        acc[0] += ws * v.x;
+        acc[1] += ws * v.y;
+        acc[2] += ws * v.z;
+        acc[3] += ws * v.w;
+      } else {
+        const float2 v = *reinterpret_cast<const float2*>(src);
+        acc[0] += ws * v.x;
+        acc[1] += ws * v.y;
+      }
     }
-    const float inv = 1.f / l;
-    const int i = r / p.G, g = r - (r / p.G) * p.G;
-    bf16* dst = p.o + (static_cast<size_t>(b * p.bs + i) * p.Hq + h * p.G + g) * D + d;
-    *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(a0 * inv, a1 * inv),
-                                                pack_bf16x2(a2 * inv, a3 * inv));
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
+  const float inv = 1.f / l;
+  const int i = r / p.G, g = r - (r / p.G) * p.G;
+  f16* dst = p.o + (static_cast<size_t>(b * p.bs + i) * p.Hq + h * p.G + g) * D + lane * PER;
+  if constexpr (PER == 4) {
+    *reinterpret_cast<uint2*>(dst) = make_uint2(pack_f16x2(acc[0] * inv, acc[1] * inv),
+                                                pack_f16x2(acc[2] * inv, acc[3] * inv));
+  } else {
+    *reinterpret_cast<uint32_t*>(dst) = pack_f16x2(acc[0] * inv, acc[1] * inv);
   }
 }
 

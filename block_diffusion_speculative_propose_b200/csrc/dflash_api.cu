@@ -51,17 +51,19 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D bf16 view [rows][cols] (row pitch cols * 2 bytes), box [box_rows][64],
-// 128-byte swizzle.  Out-of-range box rows read as zeros.
+// 2-D view of 16-bit elements (bf16, or fp16 when f16) [rows][cols] (row pitch
+// cols * 2 bytes), box [box_rows][64], 128-byte swizzle.  Out-of-range box
+// rows read as zeros.
 bool make_tmap(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t cols,
-               uint32_t box_rows) {
+               uint32_t box_rows, bool f16) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {cols * 2};
   cuuint32_t box[2] = {64, box_rows};
   cuuint32_t estr[2] = {1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides,
+  return fn(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+            const_cast<void*>(ptr), dims, strides,
             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
@@ -72,9 +74,25 @@ bool make_tmap(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t cols,
 // ---------------------------------------------------------------------------
 struct GemmPlan {
   int BN = 0, splits = 1, kb_per_split = 0, m_tiles = 0, n_tiles = 0, k_blocks = 0, units = 0,
-      grid = 0;
+      grid = 0, a_rows = 128, stages = 1, smem = 0;
   size_t partial_bytes = 0;
 };
+
+// A box / slot rows: all 128 once there is more than one M tile, else M
+// rounded up to 16 (multiples of 8 rows keep every slot 1024-byte aligned).
+int gemm_a_rows(int M) { return M >= kGemmBM ? kGemmBM : std::max(16, (M + 15) / 16 * 16); }
+
+int gemm_stages(int a_rows, int bn) {
+  int st = kGemmMaxStages;
+  while (st > 2 && gemm_smem_bytes(a_rows, bn, st) > kGemmSmemLimit) --st;
+  return st;
+}
+
+void finish_plan(GemmPlan& pl, int M) {
+  pl.a_rows = gemm_a_rows(M);
+  pl.stages = gemm_stages(pl.a_rows, pl.BN);
+  pl.smem = gemm_smem_bytes(pl.a_rows, pl.BN, pl.stages);
+}
 
 // Picks the tile width BN (a multiple of the epilogue group) and the K-split
 // count by minimising a per-SM time estimate: the busiest SM runs
@@ -86,9 +104,10 @@ GemmPlan plan_gemm(int M, int N, int K, int group, int num_sms) {
   double best_t = 1e300;
   const int k_blocks = K / kGemmBK;
   const int m_tiles = cdiv(M, kGemmBM);
-  const double bw_sm = 6.5e12 / 148.0 * 1.6;  // bytes/s one SM can pull when peers idle
+  const double bw_sm = 90e9;                 // bytes/s one SM's TMA ring sustains
   const double fl_sm = 1.6e15 / 148.0;
   const double hbm = 6.5e12;
+  const double a_rows = gemm_a_rows(M);
   const int bns[4] = {256, 128, 64, 32};
   for (int bi = 0; bi < 4; ++bi) {
     const int BN = bns[bi];
@@ -103,10 +122,9 @@ GemmPlan plan_gemm(int M, int N, int K, int group, int num_sms) {
       const int units = m_tiles * n_tiles * S;
       const int rounds = cdiv(units, num_sms);
       const double kspan = static_cast<double>(kbps) * kGemmBK;
-      const double rows = std::min(M, kGemmBM);
-      const double unit_bytes = BN * kspan * 2.0 + rows * kspan * 2.0 * 0.25;
+      const double unit_bytes = (BN + a_rows) * kspan * 2.0;
       const double unit_flops = 2.0 * kGemmBM * BN * kspan;
-      double t = rounds * (std::max(unit_bytes / bw_sm, unit_flops / fl_sm) + 0.6e-6);
+      double t = rounds * (std::max(unit_bytes / bw_sm, unit_flops / fl_sm) + 1.0e-6);
       const double total_w = static_cast<double>(N) * K * 2.0;
       t = std::max(t, total_w / hbm);
       if (S > 1) t += static_cast<double>(S) * M * N * 4.0 * 2.0 / hbm + 1.0e-6;
@@ -124,6 +142,7 @@ GemmPlan plan_gemm(int M, int N, int K, int group, int num_sms) {
       }
     }
   }
+  if (best.BN) finish_plan(best, M);
   return best;
 }
 
@@ -131,7 +150,7 @@ GemmPlan plan_gemm(int M, int N, int K, int group, int num_sms) {
 // attention planning
 // ---------------------------------------------------------------------------
 struct AttnPlan {
-  int chunk_keys = 0, max_splits = 0, R = 0, nwc = 0;
+  int chunk_keys = 0, max_splits = 0, R = 0, row_groups = 0, key_parts = 0, nwc = 0;
   size_t part_o_bytes = 0, part_ml_bytes = 0;
 };
 
@@ -145,7 +164,11 @@ AttnPlan plan_attention(int B, int Hkv, int W, int P, int bs, int G, int D, int 
   a.chunk_keys = chunk;
   a.max_splits = cdiv(keys_max, chunk);
   a.R = bs * G;
-  a.nwc = cdiv(a.R, 16);
+  a.row_groups = cdiv(a.R, 16);
+  a.key_parts = 1;
+  while (a.key_parts < 4 && a.row_groups * a.key_parts * 2 <= kAttnMaxComputeWarps)
+    a.key_parts *= 2;
+  a.nwc = a.row_groups * a.key_parts;
   a.part_o_bytes =
       a.max_splits > 1 ? static_cast<size_t>(a.max_splits) * B * Hkv * a.R * D * 4 : 0;
   a.part_ml_bytes =
@@ -174,27 +197,36 @@ struct dflash_handle {
   // aliased caller weights
   const bf16 *fc_w = nullptr, *hidden_norm_w = nullptr, *embed = nullptr, *lm_head = nullptr,
              *final_norm_w = nullptr;
-  std::vector<const bf16*> in_norm_w, post_norm_w, wo, q_norm_w, k_norm_w, w_down;
-  // packed copies owned by the handle
-  std::vector<bf16*> wqkv, wgu;
-  bf16* wkv = nullptr;      // [L * 2 * Hkv * D, H]
+  std::vector<const bf16*> in_norm_w, post_norm_w, q_norm_w, k_norm_w, w_down;
+  // copies owned by the handle; the ones multiplied against fp16 operands are
+  // held as fp16 (bf16 -> fp16 is exact in fp16's normal range)
+  std::vector<f16*> wqkv, wgu, wo;
+  f16* wkv = nullptr;       // [L * 2 * Hkv * D, H]
+  f16* lm_head16 = nullptr; // [V, H]
   bf16* knorm_all = nullptr;  // [L, D]
   float2* rope = nullptr;   // [max_position, D/2]
   unsigned* dev_err = nullptr;
   unsigned* counters = nullptr;
   std::mutex mu;
-  std::map<std::tuple<const void*, uint64_t, uint64_t, uint32_t>, CUtensorMap> tmaps;
+  std::map<std::tuple<const void*, uint64_t, uint64_t, uint32_t, bool>, CUtensorMap> tmaps;
+  // launch accounting and optional per-launch event profiling (diagnostics)
+  unsigned long long launches = 0;
+  bool prof_on = false;
+  std::vector<cudaEvent_t> prof_events;
+  size_t prof_next = 0;
+  std::vector<int> prof_kind;
 
-  bool tmap(CUtensorMap* out, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  bool tmap(CUtensorMap* out, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows,
+            bool f16 = false) {
     std::lock_guard<std::mutex> lk(mu);
-    auto key = std::make_tuple(ptr, rows, cols, box_rows);
+    auto key = std::make_tuple(ptr, rows, cols, box_rows, f16);
     auto it = tmaps.find(key);
     if (it != tmaps.end()) {
       *out = it->second;
       return true;
     }
     if (tmaps.size() > 8192) tmaps.clear();
-    if (!make_tmap(out, ptr, rows, cols, box_rows)) return false;
+    if (!make_tmap(out, ptr, rows, cols, box_rows, f16)) return false;
     tmaps.emplace(key, *out);
     return true;
   }
@@ -204,9 +236,12 @@ namespace {
 
 void free_handle(dflash_handle* h) {
   if (!h) return;
+  for (auto e : h->prof_events) cudaEventDestroy(e);
   for (auto p : h->wqkv) cudaFree(p);
   for (auto p : h->wgu) cudaFree(p);
+  for (auto p : h->wo) cudaFree(p);
   cudaFree(h->wkv);
+  cudaFree(h->lm_head16);
   cudaFree(h->knorm_all);
   cudaFree(h->rope);
   cudaFree(h->dev_err);
@@ -214,14 +249,34 @@ void free_handle(dflash_handle* h) {
   delete h;
 }
 
+// Counts every kernel launch a handle's call makes and, while profiling is on,
+// brackets it with a pair of events recorded on the launching stream.
+struct LaunchScope {
+  dflash_handle* h;
+  cudaStream_t st;
+  cudaEvent_t stop = nullptr;
+  LaunchScope(dflash_handle* h_, int kind, cudaStream_t st_) : h(h_), st(st_) {
+    ++h->launches;
+    if (h->prof_on && h->prof_next + 2 <= h->prof_events.size()) {
+      cudaEvent_t a = h->prof_events[h->prof_next];
+      stop = h->prof_events[h->prof_next + 1];
+      h->prof_next += 2;
+      h->prof_kind.push_back(kind);
+      cudaEventRecord(a, st);
+    }
+  }
+  ~LaunchScope() {
+    if (stop) cudaEventRecord(stop, st);
+  }
+};
+
 // ---------------------------------------------------------------------------
 // GEMM launch
 // ---------------------------------------------------------------------------
 template <int BN, class Epi>
 cudaError_t set_gemm_attr() {
   return cudaFuncSetAttribute(gemm_tcgen05_kernel<BN, Epi>,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              GemmCfg<BN>::kSmemBytes);
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemLimit);
 }
 
 template <class Epi>
@@ -240,17 +295,17 @@ cudaError_t set_gemm_attrs_all() {
 
 template <int BN, class Epi>
 void launch_gemm_bn(const CUtensorMap& ta, const CUtensorMap& tw, const GemmParams& gp,
-                    const Epi& epi, int grid, cudaStream_t st) {
-  gemm_tcgen05_kernel<BN, Epi>
-      <<<grid, kGemmThreads, GemmCfg<BN>::kSmemBytes, st>>>(ta, tw, gp, epi);
+                    const Epi& epi, int grid, int smem, cudaStream_t st) {
+  gemm_tcgen05_kernel<BN, Epi><<<grid, kGemmThreads, smem, st>>>(ta, tw, gp, epi);
 }
 
 // D = A[M, K] * W[N, K]^T with epilogue `epi`.  `partials` must hold
 // plan.partial_bytes.
 template <class Epi>
-dflash_status run_gemm(dflash_handle* h, const void* A, int M, int K, const void* Wt, int N,
-                       const Epi& epi, float* partials, size_t partial_cap, cudaStream_t st,
-                       int force_bn = 0, int force_splits = 0) {
+dflash_status run_gemm(dflash_handle* h, int kind, bool f16, const void* A, int M, int K,
+                       const void* Wt, int N, const Epi& epi, float* partials,
+                       size_t partial_cap, cudaStream_t st, int force_bn = 0,
+                       int force_splits = 0) {
   if (M <= 0) return DFLASH_OK;
   GemmPlan pl = plan_gemm(M, N, K, Epi::kGroup, h->num_sms);
   if (force_bn || force_splits) {
@@ -269,12 +324,13 @@ dflash_status run_gemm(dflash_handle* h, const void* A, int M, int K, const void
     pl.units = pl.m_tiles * pl.n_tiles * pl.splits;
     pl.grid = std::min(pl.units, h->num_sms);
     pl.partial_bytes = pl.splits > 1 ? static_cast<size_t>(pl.splits) * M * N * 4 : 0;
+    finish_plan(pl, M);
   }
   if (pl.BN == 0) return DFLASH_ERR_UNSUPPORTED_SHAPE;
   if (pl.partial_bytes > partial_cap) return DFLASH_ERR_WORKSPACE;
   CUtensorMap ta, tw;
-  if (!h->tmap(&ta, A, M, K, kGemmBM)) return DFLASH_ERR_CUDA;
-  if (!h->tmap(&tw, Wt, N, K, pl.BN)) return DFLASH_ERR_CUDA;
+  if (!h->tmap(&ta, A, M, K, pl.a_rows, f16)) return DFLASH_ERR_CUDA;
+  if (!h->tmap(&tw, Wt, N, K, pl.BN, f16)) return DFLASH_ERR_CUDA;
   GemmParams gp;
   gp.M = M;
   gp.N = N;
@@ -285,21 +341,25 @@ dflash_status run_gemm(dflash_handle* h, const void* A, int M, int K, const void
   gp.splits = pl.splits;
   gp.kb_per_split = pl.kb_per_split;
   gp.num_units = pl.units;
+  gp.a_rows = pl.a_rows;
+  gp.stages = pl.stages;
+  gp.f16 = f16 ? 1 : 0;
   gp.partials = partials;
   gp.counters = h->counters;
   gp.err = h->dev_err;
+  LaunchScope scope(h, kind, st);
   switch (pl.BN) {
     case 256:
-      if constexpr (256 % Epi::kGroup == 0) launch_gemm_bn<256>(ta, tw, gp, epi, pl.grid, st);
+      if constexpr (256 % Epi::kGroup == 0) launch_gemm_bn<256>(ta, tw, gp, epi, pl.grid, pl.smem, st);
       break;
     case 128:
-      if constexpr (128 % Epi::kGroup == 0) launch_gemm_bn<128>(ta, tw, gp, epi, pl.grid, st);
+      if constexpr (128 % Epi::kGroup == 0) launch_gemm_bn<128>(ta, tw, gp, epi, pl.grid, pl.smem, st);
       break;
     case 64:
-      if constexpr (Epi::kGroup <= 64) launch_gemm_bn<64>(ta, tw, gp, epi, pl.grid, st);
+      if constexpr (Epi::kGroup <= 64) launch_gemm_bn<64>(ta, tw, gp, epi, pl.grid, pl.smem, st);
       break;
     case 32:
-      if constexpr (Epi::kGroup <= 32) launch_gemm_bn<32>(ta, tw, gp, epi, pl.grid, st);
+      if constexpr (Epi::kGroup <= 32) launch_gemm_bn<32>(ta, tw, gp, epi, pl.grid, pl.smem, st);
       break;
     default:
       return DFLASH_ERR_UNSUPPORTED_SHAPE;
@@ -312,8 +372,16 @@ dflash_status run_gemm(dflash_handle* h, const void* A, int M, int K, const void
 // ---------------------------------------------------------------------------
 template <int D>
 cudaError_t set_attn_attrs() {
-  return cudaFuncSetAttribute(attn_block_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              AttnCfg<D>::smem_bytes(kAttnMaxComputeWarps));
+  const int bytes = AttnCfg<D>::smem_bytes(kAttnMaxComputeWarps);
+  cudaError_t e;
+  if ((e = cudaFuncSetAttribute(attn_block_kernel<D, 64>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, bytes)) != cudaSuccess)
+    return e;
+  if ((e = cudaFuncSetAttribute(attn_block_kernel<D, 32>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, bytes)) != cudaSuccess)
+    return e;
+  return cudaFuncSetAttribute(attn_block_kernel<D, 16>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
 
 template <int D>
@@ -327,8 +395,23 @@ dflash_status run_attention(dflash_handle* h, const AttnPlan& ap, AttnParams prm
   if (!h->tmap(&tv, vc, rows, D, 16)) return DFLASH_ERR_CUDA;
   dim3 grid(ap.max_splits, c.n_kv_heads, prm.B);
   const int threads = 32 * (ap.nwc + 1);
-  attn_block_kernel<D><<<grid, threads, AttnCfg<D>::smem_bytes(ap.nwc), st>>>(tk, tv, prm);
-  if (ap.max_splits > 1) attn_combine_kernel<D><<<dim3(c.n_kv_heads, prm.B), 256, 0, st>>>(prm);
+  const int smem = AttnCfg<D>::smem_bytes(ap.nwc);
+  prm.row_groups = ap.row_groups;
+  prm.key_parts = ap.key_parts;
+  {
+    LaunchScope scope(h, DFLASH_KERNEL_ATTENTION, st);
+    if (ap.key_parts == 1)
+      attn_block_kernel<D, 64><<<grid, threads, smem, st>>>(tk, tv, prm);
+    else if (ap.key_parts == 2)
+      attn_block_kernel<D, 32><<<grid, threads, smem, st>>>(tk, tv, prm);
+    else
+      attn_block_kernel<D, 16><<<grid, threads, smem, st>>>(tk, tv, prm);
+  }
+  if (ap.max_splits > 1) {
+    LaunchScope scope(h, DFLASH_KERNEL_ATTN_COMBINE, st);
+    const int rows = prm.B * c.n_kv_heads * prm.R;
+    attn_combine_kernel<D><<<cdiv(rows, 8), 256, 0, st>>>(prm);
+  }
   return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ERR_CUDA;
 }
 
@@ -419,13 +502,32 @@ T* at(void* base, size_t off) {
   return reinterpret_cast<T*>(static_cast<uint8_t*>(base) + off);
 }
 
-dflash_status set_device_of(const void* p) {
-  cudaPointerAttributes a;
-  if (cudaPointerGetAttributes(&a, p) != cudaSuccess || a.type != cudaMemoryTypeDevice) {
-    cudaGetLastError();
-    return DFLASH_ERR_INVALID_ARG;
+// Makes `dev` current for this library's runtime (a no-op when it already is,
+// so calls stay cheap and legal inside stream capture).
+cudaError_t use_device(int dev) {
+  int cur = -1;
+  if (cudaGetDevice(&cur) == cudaSuccess && cur == dev) return cudaSuccess;
+  return cudaSetDevice(dev);
+}
+
+// Handle-free calls run on the device of their stream (or, on the legacy
+// default stream, of their output buffer).
+dflash_status set_device_for(cudaStream_t st, const void* p) {
+  int dev = -1;
+  if (st != nullptr) {
+    if (cudaStreamGetDevice(st, &dev) != cudaSuccess) {
+      cudaGetLastError();
+      return DFLASH_ERR_INVALID_ARG;
+    }
+  } else {
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess || a.type != cudaMemoryTypeDevice) {
+      cudaGetLastError();
+      return DFLASH_ERR_INVALID_ARG;
+    }
+    dev = a.device;
   }
-  DF_CUDA(cudaSetDevice(a.device));
+  DF_CUDA(use_device(dev));
   return DFLASH_OK;
 }
 
@@ -460,11 +562,11 @@ dflash_status propose_layers(dflash_handle* h, const ProposeWs& lw, void* ws,
   const int bs = c.block_size, M = B * bs, H = c.hidden, Hq = c.n_q_heads, Hkv = c.n_kv_heads,
             I = c.intermediate, K = bs - 1;
   float* x = at<float>(ws, lw.x);
-  bf16* nrm = at<bf16>(ws, lw.nrm);
+  f16* nrm = at<f16>(ws, lw.nrm);
   bf16* q = at<bf16>(ws, lw.q);
-  bf16* o = at<bf16>(ws, lw.o);
+  f16* o = at<f16>(ws, lw.o);
   bf16* hm = at<bf16>(ws, lw.hm);
-  bf16* frows = at<bf16>(ws, lw.frows);
+  f16* frows = at<f16>(ws, lw.frows);
   float* partial = at<float>(ws, lw.partial);
   const AttnPlan ap = plan_attention(B, Hkv, W, c.page_size, bs, Hq / Hkv, D, h->num_sms);
   if (ap.part_o_bytes > lw.part_o_cap || ap.part_ml_bytes > lw.part_ml_cap)
@@ -509,25 +611,32 @@ dflash_status propose_layers(dflash_handle* h, const ProposeWs& lw, void* ws,
     eq.num_pages = num_pages;
     eq.eps = c.rms_eps;
     eq.err = h->dev_err;
-    dflash_status s =
-        run_gemm(h, nrm, M, H, h->wqkv[l], (Hq + 2 * Hkv) * D, eq, partial, lw.partial_cap, st);
+    dflash_status s = run_gemm(h, DFLASH_KERNEL_GEMM_QKV, true, nrm, M, H, h->wqkv[l],
+                               (Hq + 2 * Hkv) * D, eq, partial, lw.partial_cap, st);
     if (s != DFLASH_OK) return s;
     // non-causal block attention over context + block
     s = run_attention<D>(h, ap, prm, k_cache[l], v_cache[l], num_pages, st);
     if (s != DFLASH_OK) return s;
     // x += Wo o
     EpiResidAdd er{x, H};
-    s = run_gemm(h, o, M, Hq * D, h->wo[l], H, er, partial, lw.partial_cap, st);
+    s = run_gemm(h, DFLASH_KERNEL_GEMM_O, true, o, M, Hq * D, h->wo[l], H, er, partial,
+                 lw.partial_cap, st);
     if (s != DFLASH_OK) return s;
-    rmsnorm_rows_kernel<<<M, 256, 0, st>>>(x, h->post_norm_w[l], nrm, H, c.rms_eps, 0, bs);
+    {
+      LaunchScope scope(h, DFLASH_KERNEL_RMSNORM, st);
+      rmsnorm_rows_kernel<<<M, 256, 0, st>>>(x, h->post_norm_w[l], nrm, H, c.rms_eps, 0, bs);
+    }
     if (cudaGetLastError() != cudaSuccess) return DFLASH_ERR_CUDA;
     // h = silu(gate) * up
     EpiSwiGLU eg{hm, I};
-    s = run_gemm(h, nrm, M, H, h->wgu[l], 2 * I, eg, partial, lw.partial_cap, st);
+    s = run_gemm(h, DFLASH_KERNEL_GEMM_GATE_UP, true, nrm, M, H, h->wgu[l], 2 * I, eg, partial,
+                 lw.partial_cap, st);
     if (s != DFLASH_OK) return s;
     // x += Wd h
-    s = run_gemm(h, hm, M, I, h->w_down[l], H, er, partial, lw.partial_cap, st);
+    s = run_gemm(h, DFLASH_KERNEL_GEMM_DOWN, false, hm, M, I, h->w_down[l], H, er, partial,
+                 lw.partial_cap, st);
     if (s != DFLASH_OK) return s;
+    LaunchScope scope(h, DFLASH_KERNEL_RMSNORM, st);
     if (l + 1 < c.n_layers) {
       rmsnorm_rows_kernel<<<M, 256, 0, st>>>(x, h->in_norm_w[l + 1], nrm, H, c.rms_eps, 0, bs);
     } else {
@@ -624,7 +733,6 @@ dflash_status dflash_create(const dflash_config* cfg, const dflash_weights* w, i
   for (int l = 0; l < L; ++l) {
     h->in_norm_w.push_back(static_cast<const bf16*>(w->in_norm_w[l]));
     h->post_norm_w.push_back(static_cast<const bf16*>(w->post_norm_w[l]));
-    h->wo.push_back(static_cast<const bf16*>(w->wo[l]));
     h->q_norm_w.push_back(static_cast<const bf16*>(w->q_norm_w[l]));
     h->k_norm_w.push_back(static_cast<const bf16*>(w->k_norm_w[l]));
     h->w_down.push_back(static_cast<const bf16*>(w->w_down[l]));
@@ -641,7 +749,7 @@ dflash_status dflash_create(const dflash_config* cfg, const dflash_weights* w, i
   const size_t rowb = static_cast<size_t>(H) * 2;
   // QKV: [wq; wk; wv]
   for (int l = 0; l < L; ++l) {
-    bf16* p = nullptr;
+    f16* p = nullptr;
     if (cudaMalloc(&p, static_cast<size_t>(Hq + 2 * Hkv) * D * rowb) != cudaSuccess)
       return fail_st(DFLASH_ERR_CUDA);
     h->wqkv.push_back(p);
@@ -657,7 +765,7 @@ dflash_status dflash_create(const dflash_config* cfg, const dflash_weights* w, i
   }
   // gate / up interleaved in blocks of 16 rows: [g 16 | u 16] per 32 packed rows
   for (int l = 0; l < L; ++l) {
-    bf16* p = nullptr;
+    f16* p = nullptr;
     if (cudaMalloc(&p, static_cast<size_t>(2 * I) * rowb) != cudaSuccess)
       return fail_st(DFLASH_ERR_CUDA);
     h->wgu.push_back(p);
@@ -684,6 +792,35 @@ dflash_status dflash_create(const dflash_config* cfg, const dflash_weights* w, i
     if (cudaMemcpyAsync(h->knorm_all + static_cast<size_t>(l) * D, w->k_norm_w[l],
                         static_cast<size_t>(D) * 2, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
       return fail_st(DFLASH_ERR_CUDA);
+  // O projections and the LM head: fp16 copies
+  for (int l = 0; l < L; ++l) {
+    f16* p = nullptr;
+    if (cudaMalloc(&p, static_cast<size_t>(H) * Hq * D * 2) != cudaSuccess)
+      return fail_st(DFLASH_ERR_CUDA);
+    h->wo.push_back(p);
+    if (cudaMemcpyAsync(p, w->wo[l], static_cast<size_t>(H) * Hq * D * 2,
+                        cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+      return fail_st(DFLASH_ERR_CUDA);
+  }
+  if (cudaMalloc(&h->lm_head16, static_cast<size_t>(c.vocab) * rowb) != cudaSuccess ||
+      cudaMemcpyAsync(h->lm_head16, w->lm_head, static_cast<size_t>(c.vocab) * rowb,
+                      cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return fail_st(DFLASH_ERR_CUDA);
+  {
+    auto to_f16 = [&](void* ptr, size_t n) {
+      bf16_to_f16_kernel<<<1184, 256, 0, st>>>(static_cast<uint16_t*>(ptr), n);
+      return cudaGetLastError() == cudaSuccess;
+    };
+    bool ok = true;
+    for (int l = 0; l < L; ++l) {
+      ok = ok && to_f16(h->wqkv[l], static_cast<size_t>(Hq + 2 * Hkv) * D * H);
+      ok = ok && to_f16(h->wgu[l], static_cast<size_t>(2 * I) * H);
+      ok = ok && to_f16(h->wo[l], static_cast<size_t>(H) * Hq * D);
+    }
+    ok = ok && to_f16(h->wkv, static_cast<size_t>(L) * 2 * kvrows * H);
+    ok = ok && to_f16(h->lm_head16, static_cast<size_t>(c.vocab) * H);
+    if (!ok) return fail_st(DFLASH_ERR_CUDA);
+  }
   if (cudaMalloc(&h->rope, static_cast<size_t>(c.max_position) * (D / 2) * sizeof(float2)) !=
       cudaSuccess)
     return fail_st(DFLASH_ERR_CUDA);
@@ -743,7 +880,7 @@ dflash_status dflash_paged_slots(const int64_t* positions, const int64_t* req_id
   if (n < 0 || max_pages_per_seq <= 0 || page_size <= 0) return DFLASH_ERR_INVALID_ARG;
   if (n == 0) return DFLASH_OK;
   if (!positions || !req_ids || !block_table || !slots) return DFLASH_ERR_INVALID_ARG;
-  dflash_status s = set_device_of(slots);
+  dflash_status s = set_device_for(static_cast<cudaStream_t>(stream), slots);
   if (s != DFLASH_OK) return s;
   paged_slots_kernel<<<cdiv(n, 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
       positions, req_ids, block_table, n, max_pages_per_seq, page_size, slots);
@@ -765,20 +902,23 @@ dflash_status dflash_inject_context(dflash_handle* h, const void* aux, const int
   if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return DFLASH_ERR_INVALID_ARG;
   const InjectWs lw = inject_layout(h, n);
   if (workspace_bytes < lw.total) return DFLASH_ERR_WORKSPACE;
-  DF_CUDA(cudaSetDevice(h->device));
+  DF_CUDA(use_device(h->device));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int H = c.hidden, D = c.head_dim;
   float* fcx = at<float>(workspace, lw.fcx);
-  bf16* ctx = at<bf16>(workspace, lw.ctx);
+  f16* ctx = at<f16>(workspace, lw.ctx);
   float* partial = at<float>(workspace, lw.partial);
 
   // (1) fc over the concatenated tapped states
   EpiStoreF32 e1{fcx, H};
-  dflash_status s = run_gemm(h, aux, n, c.n_target_layers * H, h->fc_w, H, e1, partial,
-                             lw.partial_cap, st);
+  dflash_status s = run_gemm(h, DFLASH_KERNEL_GEMM_FC, false, aux, n, c.n_target_layers * H,
+                             h->fc_w, H, e1, partial, lw.partial_cap, st);
   if (s != DFLASH_OK) return s;
   // (2) hidden_norm
-  rmsnorm_rows_kernel<<<n, 256, 0, st>>>(fcx, h->hidden_norm_w, ctx, H, c.rms_eps, 0, 0);
+  {
+    LaunchScope scope(h, DFLASH_KERNEL_RMSNORM, st);
+    rmsnorm_rows_kernel<<<n, 256, 0, st>>>(fcx, h->hidden_norm_w, ctx, H, c.rms_eps, 0, 0);
+  }
   if (cudaGetLastError() != cudaSuccess) return DFLASH_ERR_CUDA;
   // (3) every layer's K/V at once, k_norm + RoPE, paged scatter
   const int NKV = c.n_layers * 2 * c.n_kv_heads * D;
@@ -798,7 +938,8 @@ dflash_status dflash_inject_context(dflash_handle* h, const void* aux, const int
     e3.num_pages = num_pages;
     e3.eps = c.rms_eps;
     e3.err = h->dev_err;
-    s = run_gemm(h, ctx, n, H, h->wkv, NKV, e3, partial, lw.partial_cap, st);
+    s = run_gemm(h, DFLASH_KERNEL_GEMM_KV_INJECT, true, ctx, n, H, h->wkv, NKV, e3, partial,
+                 lw.partial_cap, st);
   } else {
     EpiKVInject<64> e3{};
     for (int l = 0; l < c.n_layers; ++l) {
@@ -815,7 +956,8 @@ dflash_status dflash_inject_context(dflash_handle* h, const void* aux, const int
     e3.num_pages = num_pages;
     e3.eps = c.rms_eps;
     e3.err = h->dev_err;
-    s = run_gemm(h, ctx, n, H, h->wkv, NKV, e3, partial, lw.partial_cap, st);
+    s = run_gemm(h, DFLASH_KERNEL_GEMM_KV_INJECT, true, ctx, n, H, h->wkv, NKV, e3, partial,
+                 lw.partial_cap, st);
   }
   return s;
 }
@@ -839,18 +981,21 @@ dflash_status dflash_propose(dflash_handle* h, const int32_t* bonus_tokens,
   if (static_cast<int64_t>(B) * c.block_size > (1 << 24)) return DFLASH_ERR_UNSUPPORTED_SHAPE;
   const ProposeWs lw = propose_layout(h, B, max_pages_per_seq);
   if (workspace_bytes < lw.total) return DFLASH_ERR_WORKSPACE;
-  DF_CUDA(cudaSetDevice(h->device));
+  DF_CUDA(use_device(h->device));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int bs = c.block_size, K = bs - 1, M = B * bs, H = c.hidden;
   float* x = at<float>(workspace, lw.x);
-  bf16* nrm = at<bf16>(workspace, lw.nrm);
-  bf16* frows = at<bf16>(workspace, lw.frows);
+  f16* nrm = at<f16>(workspace, lw.nrm);
+  f16* frows = at<f16>(workspace, lw.frows);
   unsigned long long* keys = at<unsigned long long>(workspace, lw.keys);
   float* partial = at<float>(workspace, lw.partial);
 
-  embed_norm_kernel<<<M, 256, 0, st>>>(bonus_tokens, c.mask_token_id, h->embed, h->in_norm_w[0],
-                                       x, nrm, keys, B * K, bs, H, c.vocab, c.rms_eps,
-                                       h->dev_err);
+  {
+    LaunchScope scope(h, DFLASH_KERNEL_EMBED_NORM, st);
+    embed_norm_kernel<<<M, 256, 0, st>>>(bonus_tokens, c.mask_token_id, h->embed,
+                                         h->in_norm_w[0], x, nrm, keys, B * K, bs, H, c.vocab,
+                                         c.rms_eps, h->dev_err);
+  }
   if (cudaGetLastError() != cudaSuccess) return DFLASH_ERR_CUDA;
   dflash_status s = (c.head_dim == 128)
                         ? propose_layers<128>(h, lw, workspace, seq_lens, block_table, B,
@@ -860,10 +1005,14 @@ dflash_status dflash_propose(dflash_handle* h, const int32_t* bonus_tokens,
   if (s != DFLASH_OK) return s;
   // aliased target LM head with the greedy pick fused into its epilogue
   EpiArgmax ea{keys, logits_out, c.vocab};
-  s = run_gemm(h, frows, B * K, H, h->lm_head, c.vocab, ea, partial, lw.partial_cap, st);
+  s = run_gemm(h, DFLASH_KERNEL_GEMM_LM_HEAD, true, frows, B * K, H, h->lm_head16, c.vocab, ea,
+               partial, lw.partial_cap, st);
   if (s != DFLASH_OK) return s;
-  argmax_finalize_kernel<<<cdiv(M, 256), 256, 0, st>>>(keys, bonus_tokens, draft_tokens,
-                                                       block_tokens, B, bs);
+  {
+    LaunchScope scope(h, DFLASH_KERNEL_ARGMAX_FINALIZE, st);
+    argmax_finalize_kernel<<<cdiv(M, 256), 256, 0, st>>>(keys, bonus_tokens, draft_tokens,
+                                                         block_tokens, B, bs);
+  }
   return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ERR_CUDA;
 }
 
@@ -880,9 +1029,9 @@ dflash_status dflash_verify_greedy(const int32_t* drafts, const float* target_lo
   if (workspace_bytes < vp.bytes) return DFLASH_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(target_logits) % 16 && V % 4 == 0)
     return DFLASH_ERR_INVALID_ARG;
-  dflash_status s = set_device_of(out_tokens);
-  if (s != DFLASH_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  dflash_status s = set_device_for(st, out_tokens);
+  if (s != DFLASH_OK) return s;
   unsigned long long* part = static_cast<unsigned long long*>(workspace);
   verify_partial_kernel<<<dim3(vp.chunks, B * (K + 1)), 256, 0, st>>>(target_logits, V,
                                                                       vp.chunk_len, vp.chunks,
@@ -908,9 +1057,10 @@ dflash_status dflash_linear(dflash_handle* h, const void* A, const void* W, int 
     return DFLASH_ERR_INVALID_ARG;
   const size_t need = dflash_linear_workspace_bytes(h, M, N, K);
   if (workspace_bytes < need) return DFLASH_ERR_WORKSPACE;
-  DF_CUDA(cudaSetDevice(h->device));
+  DF_CUDA(use_device(h->device));
   EpiStoreF32 e{out, N};
-  return run_gemm(h, A, M, K, W, N, e, static_cast<float*>(workspace), workspace_bytes,
+  return run_gemm(h, DFLASH_KERNEL_LINEAR, false, A, M, K, W, N, e,
+                  static_cast<float*>(workspace), workspace_bytes,
                   static_cast<cudaStream_t>(stream));
 }
 
@@ -925,9 +1075,10 @@ dflash_status dflash_linear_ex(dflash_handle* h, const void* A, const void* W, i
   if (reinterpret_cast<uintptr_t>(A) % 16 || reinterpret_cast<uintptr_t>(W) % 16 ||
       reinterpret_cast<uintptr_t>(out) % 16)
     return DFLASH_ERR_INVALID_ARG;
-  DF_CUDA(cudaSetDevice(h->device));
+  DF_CUDA(use_device(h->device));
   EpiStoreF32 e{out, N};
-  return run_gemm(h, A, M, K, W, N, e, static_cast<float*>(workspace), workspace_bytes,
+  return run_gemm(h, DFLASH_KERNEL_LINEAR, false, A, M, K, W, N, e,
+                  static_cast<float*>(workspace), workspace_bytes,
                   static_cast<cudaStream_t>(stream), block_n, splits);
 }
 
@@ -953,13 +1104,13 @@ dflash_status dflash_block_attention(dflash_handle* h, const void* q, const int3
   const dflash_config& c = h->cfg;
   if (workspace_bytes < dflash_attention_workspace_bytes(h, B, max_pages_per_seq))
     return DFLASH_ERR_WORKSPACE;
-  DF_CUDA(cudaSetDevice(h->device));
+  DF_CUDA(use_device(h->device));
   const AttnPlan ap = plan_attention(B, c.n_kv_heads, max_pages_per_seq, c.page_size,
                                      c.block_size, c.n_q_heads / c.n_kv_heads, c.head_dim,
                                      h->num_sms);
   AttnParams prm;
   prm.q = static_cast<const bf16*>(q);
-  prm.o = static_cast<bf16*>(o);
+  prm.o = static_cast<f16*>(o);
   prm.part_o = static_cast<float*>(workspace);
   prm.part_ml = at<float>(workspace, align_up(ap.part_o_bytes));
   prm.seq_lens = seq_lens;
@@ -982,10 +1133,78 @@ dflash_status dflash_block_attention(dflash_handle* h, const void* q, const int3
                            : run_attention<64>(h, ap, prm, k_cache, v_cache, num_pages, st);
 }
 
+unsigned long long dflash_launch_count(const dflash_handle* h) { return h ? h->launches : 0; }
+
+const char* dflash_kernel_name(int kind) {
+  switch (kind) {
+    case DFLASH_KERNEL_EMBED_NORM: return "embed_norm";
+    case DFLASH_KERNEL_GEMM_QKV: return "gemm_qkv";
+    case DFLASH_KERNEL_ATTENTION: return "attention";
+    case DFLASH_KERNEL_ATTN_COMBINE: return "attn_combine";
+    case DFLASH_KERNEL_GEMM_O: return "gemm_o";
+    case DFLASH_KERNEL_RMSNORM: return "rmsnorm";
+    case DFLASH_KERNEL_GEMM_GATE_UP: return "gemm_gate_up";
+    case DFLASH_KERNEL_GEMM_DOWN: return "gemm_down";
+    case DFLASH_KERNEL_GEMM_LM_HEAD: return "gemm_lm_head";
+    case DFLASH_KERNEL_ARGMAX_FINALIZE: return "argmax_finalize";
+    case DFLASH_KERNEL_GEMM_FC: return "gemm_fc";
+    case DFLASH_KERNEL_GEMM_KV_INJECT: return "gemm_kv_inject";
+    case DFLASH_KERNEL_LINEAR: return "linear";
+  }
+  return nullptr;
+}
+
+dflash_status dflash_profile_enable(dflash_handle* h, int max_launches) {
+  if (!h || max_launches <= 0) return DFLASH_ERR_INVALID_ARG;
+  DF_CUDA(use_device(h->device));
+  for (auto e : h->prof_events) cudaEventDestroy(e);
+  h->prof_events.clear();
+  h->prof_kind.clear();
+  h->prof_next = 0;
+  for (int i = 0; i < 2 * max_launches; ++i) {
+    cudaEvent_t e;
+    DF_CUDA(cudaEventCreate(&e));
+    h->prof_events.push_back(e);
+  }
+  h->prof_on = true;
+  return DFLASH_OK;
+}
+
+dflash_status dflash_profile_read(dflash_handle* h, int n_kinds, int* launches,
+                                  double* total_ms) {
+  if (!h || n_kinds < 0 || (n_kinds && (!launches || !total_ms))) return DFLASH_ERR_INVALID_ARG;
+  DF_CUDA(use_device(h->device));
+  for (int k = 0; k < n_kinds; ++k) {
+    launches[k] = 0;
+    total_ms[k] = 0.0;
+  }
+  DF_CUDA(cudaDeviceSynchronize());
+  for (size_t i = 0; i < h->prof_kind.size(); ++i) {
+    float ms = 0.f;
+    DF_CUDA(cudaEventElapsedTime(&ms, h->prof_events[2 * i], h->prof_events[2 * i + 1]));
+    const int k = h->prof_kind[i];
+    if (k >= 0 && k < n_kinds) {
+      launches[k] += 1;
+      total_ms[k] += ms;
+    }
+  }
+  h->prof_kind.clear();
+  h->prof_next = 0;
+  return DFLASH_OK;
+}
+
+dflash_status dflash_profile_disable(dflash_handle* h) {
+  if (!h) return DFLASH_ERR_INVALID_ARG;
+  h->prof_on = false;
+  h->prof_kind.clear();
+  h->prof_next = 0;
+  return DFLASH_OK;
+}
+
 dflash_status dflash_check_device_errors(dflash_handle* h, unsigned* bits) {
   if (bits) *bits = 0;
   if (!h) return DFLASH_ERR_INVALID_ARG;
-  DF_CUDA(cudaSetDevice(h->device));
+  DF_CUDA(use_device(h->device));
   DF_CUDA(cudaDeviceSynchronize());
   unsigned v = 0;
   DF_CUDA(cudaMemcpy(&v, h->dev_err, sizeof(unsigned), cudaMemcpyDeviceToHost));

@@ -1,7 +1,8 @@
 // gemm_tcgen05.cuh — persistent, warp-specialised bf16 GEMM for sm_100a with
 // fused epilogues.
 //
-//   D[m, n] = sum_k A[m, k] * W[n, k]      A: [M, K] bf16, W: [N, K] bf16 (both K-major)
+//   D[m, n] = sum_k A[m, k] * W[n, k]      A: [M, K], W: [N, K], both K-major and both
+//                                          fp16 or both bf16; fp32 accumulation
 //
 // Tile 128 x BN x 64.  Warp 0 streams A and W tiles with TMA (128-byte swizzle)
 // into a ring of shared-memory stages; warp 1 issues tcgen05.mma (M=128, N=BN,
@@ -29,24 +30,33 @@ constexpr int kGemmBK = 64;
 constexpr int kGemmThreads = 192;
 constexpr int kGemmSmemLimit = 232448;  // max dynamic shared memory per block on sm_100
 
+constexpr int kGemmMaxStages = 32;
+constexpr int kGemmBarrierBytes = 2 * kGemmMaxStages * 8 + 4 * 8 + 16;
+
 template <int BN>
 struct GemmCfg {
-  static constexpr int kABytes = kGemmBM * kGemmBK * 2;
   static constexpr int kBBytes = BN * kGemmBK * 2;
-  static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kReserve = 1024 + 256;  // alignment slack + barriers
-  static constexpr int kStagesRaw = (kGemmSmemLimit - kReserve) / kStageBytes;
-  static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
-  static constexpr int kSmemBytes = kReserve + kStages * kStageBytes;
   static constexpr int kTmemCols = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
                                    : (2 * BN <= 256) ? 256 : 512;
   static_assert(BN % 16 == 0 && BN >= 32 && BN <= 256, "UMMA N for M=128");
 };
 
+// Shared memory of one launch: [a_rows x 128 B A slots][BN x 128 B W slots]
+// [barriers].  With fewer than 128 rows of A (a_rows < 128) the MMA still
+// reads a full 128-row A operand; the rows past a_rows alias the following
+// slots, which only feeds accumulator rows that the epilogue never stores.
+__host__ __device__ inline int gemm_smem_bytes(int a_rows, int bn, int stages) {
+  const int tail = kGemmBM * 128 - a_rows * 128 - stages * bn * 128;  // keep A overreads inside
+  return 1024 + stages * (a_rows + bn) * 128 + kGemmBarrierBytes + (tail > 0 ? tail : 0);
+}
+
 struct GemmParams {
   int M, N, K;
   int m_tiles, n_tiles, k_blocks;
   int splits, kb_per_split, num_units;
+  int a_rows;          // rows of the A box / slot (128, or M rounded up to 16 when M < 128)
+  int stages;          // pipeline depth (<= kGemmMaxStages)
+  int f16;             // operands are fp16 (1) or bf16 (0)
   float* partials;     // [splits][M][N] when splits > 1
   unsigned* counters;  // [m_tiles * n_tiles], zero on entry, zero on exit
   unsigned* err;
@@ -92,11 +102,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
+  const int stages = p.stages;
+  const int a_bytes = p.a_rows * 128;
+  const uint32_t stage_tx = static_cast<uint32_t>(a_bytes + C::kBBytes);
   uint8_t* sA = smem;
-  uint8_t* sB = smem + C::kStages * C::kABytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + C::kStages * C::kBBytes);
-  uint64_t* empty = full + C::kStages;
-  uint64_t* tfull = empty + C::kStages;
+  uint8_t* sB = smem + stages * a_bytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + stages * C::kBBytes);
+  uint64_t* empty = full + kGemmMaxStages;
+  uint64_t* tfull = empty + kGemmMaxStages;
   uint64_t* tempty = tfull + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
   volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -105,7 +118,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::kStages; ++s) {
+    for (int s = 0; s < stages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
@@ -140,12 +153,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
-          tma_load_2d_hint(sA + stage * C::kABytes, &tmA, &full[stage], kb * kGemmBK,
+          mbar_arrive_expect_tx(&full[stage], stage_tx);
+          tma_load_2d_hint(sA + stage * a_bytes, &tmA, &full[stage], kb * kGemmBK,
                            t.m_tile * kGemmBM, pol_a);
           tma_load_2d_hint(sB + stage * C::kBBytes, &tmW, &full[stage], kb * kGemmBK,
                            t.n_tile * BN, pol_w);
-          if (++stage == C::kStages) {
+          if (++stage == static_cast<uint32_t>(stages)) {
             stage = 0;
             phase ^= 1u;
           }
@@ -155,7 +168,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = umma_idesc_bf16_f32(kGemmBM, BN);
+      const uint32_t idesc = umma_idesc_f32acc(kGemmBM, BN, p.f16 != 0);
       uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
       bool ok = true;
       for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
@@ -169,17 +182,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint64_t adesc = umma_desc_sw128(smem_u32(sA + stage * C::kABytes));
+          const uint64_t adesc = umma_desc_sw128(smem_u32(sA + stage * a_bytes));
           const uint64_t bdesc = umma_desc_sw128(smem_u32(sB + stage * C::kBBytes));
 #pragma unroll
           for (int k = 0; k < kGemmBK / 16; ++k) {
             // +32 bytes along K inside the 128-byte swizzle atom = +2 in the
             // descriptor's (address >> 4) field
-            umma_bf16(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc,
+            umma_f16kind(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc,
                       (kb > t.kb0 || k > 0) ? 1u : 0u);
           }
           umma_commit(&empty[stage]);
-          if (++stage == C::kStages) {
+          if (++stage == static_cast<uint32_t>(stages)) {
             stage = 0;
             phase ^= 1u;
           }

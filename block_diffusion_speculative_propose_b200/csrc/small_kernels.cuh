@@ -34,11 +34,11 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
 // Block construction ([bonus, mask, ..., mask] per request), embedding with
 // the target table, and the first layer's input RMSNorm.
 //   x[r, :]   = embed[id_r, :]                       (fp32 residual stream)
-//   nrm[r, :] = bf16(x * rsqrt(mean(x^2) + eps) * w)
+//   nrm[r, :] = fp16(x * rsqrt(mean(x^2) + eps) * w)
 // Also clears the LM-head argmax keys of the call.
 __global__ void __launch_bounds__(256) embed_norm_kernel(
     const int32_t* __restrict__ bonus, int mask_id, const bf16* __restrict__ embed,
-    const bf16* __restrict__ w, float* __restrict__ x, bf16* __restrict__ nrm,
+    const bf16* __restrict__ w, float* __restrict__ x, f16* __restrict__ nrm,
     unsigned long long* __restrict__ keys, int n_keys, int bs, int H, int V, float eps,
     unsigned* err) {
   __shared__ float red[32];
@@ -67,7 +67,7 @@ __global__ void __launch_bounds__(256) embed_norm_kernel(
   }
   ss = block_sum(ss, red);
   const float rinv = rsqrtf(ss / H + eps);
-  bf16* nr = nrm + static_cast<size_t>(r) * H;
+  f16* nr = nrm + static_cast<size_t>(r) * H;
   for (int j = threadIdx.x * 8; j < H; j += blockDim.x * 8) {
     const uint4 q = *reinterpret_cast<const uint4*>(e + j);
     const uint4 wq = *reinterpret_cast<const uint4*>(w + j);
@@ -77,17 +77,18 @@ __global__ void __launch_bounds__(256) embed_norm_kernel(
     uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
 #pragma unroll
     for (int k = 0; k < 4; ++k)
-      ow[k] = pack_bf16x2(bf2f(qb[2 * k]) * rinv * bf2f(wb[2 * k]),
-                          bf2f(qb[2 * k + 1]) * rinv * bf2f(wb[2 * k + 1]));
+      ow[k] = pack_f16x2(bf2f(qb[2 * k]) * rinv * bf2f(wb[2 * k]),
+                         bf2f(qb[2 * k + 1]) * rinv * bf2f(wb[2 * k + 1]));
     *reinterpret_cast<uint4*>(nr + j) = o;
   }
 }
 
-// out[r, :] = bf16(x[src(r), :] * rsqrt(mean(x^2) + eps) * w).
+// out[r, :] = fp16(x[src(r), :] * rsqrt(mean(x^2) + eps) * w)  (RMSNorm outputs are
+// bounded by sqrt(H) * max|w|, so fp16 holds them with 8x finer rounding than bf16).
 // With gather_k > 0, src(r) = (r / gather_k) * bs + 1 + r % gather_k: the block
 // slots 1..bs-1 of each request (keep_idx), packed densely.
 __global__ void __launch_bounds__(256) rmsnorm_rows_kernel(
-    const float* __restrict__ x, const bf16* __restrict__ w, bf16* __restrict__ out, int H,
+    const float* __restrict__ x, const bf16* __restrict__ w, f16* __restrict__ out, int H,
     float eps, int gather_k, int bs) {
   __shared__ float red[32];
   const int r = blockIdx.x;
@@ -102,17 +103,17 @@ __global__ void __launch_bounds__(256) rmsnorm_rows_kernel(
   }
   ss = block_sum(ss, red);
   const float rinv = rsqrtf(ss / H + eps);
-  bf16* orow = out + static_cast<size_t>(r) * H;
+  f16* orow = out + static_cast<size_t>(r) * H;
   for (int j = threadIdx.x * 8; j < H; j += blockDim.x * 8) {
     const float4 a = *reinterpret_cast<const float4*>(xr + j);
     const float4 c = *reinterpret_cast<const float4*>(xr + j + 4);
     const uint4 wq = *reinterpret_cast<const uint4*>(w + j);
     const bf16* wb = reinterpret_cast<const bf16*>(&wq);
     uint4 o;
-    o.x = pack_bf16x2(a.x * rinv * bf2f(wb[0]), a.y * rinv * bf2f(wb[1]));
-    o.y = pack_bf16x2(a.z * rinv * bf2f(wb[2]), a.w * rinv * bf2f(wb[3]));
-    o.z = pack_bf16x2(c.x * rinv * bf2f(wb[4]), c.y * rinv * bf2f(wb[5]));
-    o.w = pack_bf16x2(c.z * rinv * bf2f(wb[6]), c.w * rinv * bf2f(wb[7]));
+    o.x = pack_f16x2(a.x * rinv * bf2f(wb[0]), a.y * rinv * bf2f(wb[1]));
+    o.y = pack_f16x2(a.z * rinv * bf2f(wb[2]), a.w * rinv * bf2f(wb[3]));
+    o.z = pack_f16x2(c.x * rinv * bf2f(wb[4]), c.y * rinv * bf2f(wb[5]));
+    o.w = pack_f16x2(c.z * rinv * bf2f(wb[6]), c.w * rinv * bf2f(wb[7]));
     *reinterpret_cast<uint4*>(orow + j) = o;
   }
 }
@@ -223,6 +224,16 @@ __global__ void paged_slots_kernel(const int64_t* __restrict__ pos,
   if (pg > W - 1) pg = W - 1;
   const int64_t page = table[req[i] * W + pg];
   slots[i] = page * P + (p - (p / P) * P);
+}
+
+// In-place bf16 -> fp16 conversion of weights (exact in fp16's normal range).
+__global__ void bf16_to_f16_kernel(uint16_t* __restrict__ data, size_t n) {
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const bf16 v = *reinterpret_cast<const bf16*>(data + i);
+    const f16 o = __float2half_rn(__bfloat162float(v));
+    data[i] = *reinterpret_cast<const uint16_t*>(&o);
+  }
 }
 
 // cos / sin of pos * theta^(-2j/D), evaluated in double, stored as fp32 pairs.

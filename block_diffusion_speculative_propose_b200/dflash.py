@@ -28,6 +28,7 @@ STATUS = {
     -7: "DFLASH_ERR_DEVICE_TIMEOUT",
 }
 DEVERR_TIMEOUT, DEVERR_SLOT, DEVERR_TABLE, DEVERR_TOKEN, DEVERR_POSITION = 1, 2, 4, 8, 16
+KERNEL_KINDS = 13
 
 
 class DFlashError(RuntimeError):
@@ -90,6 +91,12 @@ def lib() -> ctypes.CDLL:
         "dflash_block_attention": ([vp, vp, vp, vp, i32, i32, vp, vp, i32, vp, vp, sz, vp],
                                    i32),
         "dflash_check_device_errors": ([vp, ctypes.POINTER(ctypes.c_uint)], i32),
+        "dflash_launch_count": ([vp], ctypes.c_ulonglong),
+        "dflash_kernel_name": ([i32], ctypes.c_char_p),
+        "dflash_profile_enable": ([vp, i32], i32),
+        "dflash_profile_read": ([vp, i32, ctypes.POINTER(ctypes.c_int),
+                                 ctypes.POINTER(ctypes.c_double)], i32),
+        "dflash_profile_disable": ([vp], i32),
         "dflash_status_string": ([i32], ctypes.c_char_p),
         "dflash_version": ([], ctypes.c_char_p),
     }
@@ -276,7 +283,7 @@ class DFlash:
         B = int(seq_lens.shape[0])
         W = int(block_table.shape[1])
         if o is None:
-            o = torch.empty(q.shape[0], q.shape[1] * q.shape[2], dtype=torch.bfloat16,
+            o = torch.empty(q.shape[0], q.shape[1] * q.shape[2], dtype=torch.float16,
                             device=self.device)
         need = lib().dflash_attention_workspace_bytes(self.h, B, W) if B else 0
         ws = workspace if workspace is not None else self.ws.get(need)
@@ -286,6 +293,25 @@ class DFlash:
                                             ws.numel(), _stream(stream)),
                "dflash_block_attention")
         return o
+
+    # ---------------------------------------------------------- diagnostics
+    def launch_count(self) -> int:
+        return int(lib().dflash_launch_count(self.h))
+
+    def profile_enable(self, max_launches: int) -> None:
+        _check(lib().dflash_profile_enable(self.h, max_launches), "dflash_profile_enable")
+
+    def profile_disable(self) -> None:
+        _check(lib().dflash_profile_disable(self.h), "dflash_profile_disable")
+
+    def profile_read(self) -> Dict[str, tuple]:
+        """{kernel family: (launches, total ms)} since the last read."""
+        n = KERNEL_KINDS
+        cnt = (ctypes.c_int * n)()
+        tot = (ctypes.c_double * n)()
+        _check(lib().dflash_profile_read(self.h, n, cnt, tot), "dflash_profile_read")
+        return {lib().dflash_kernel_name(k).decode(): (cnt[k], tot[k])
+                for k in range(n) if cnt[k]}
 
     def check_device_errors(self) -> int:
         bits = ctypes.c_uint(0)

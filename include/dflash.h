@@ -96,10 +96,13 @@ typedef struct dflash_config {
  *   fc_w [H, T*H]   hidden_norm_w [H]   embed [V, H]   lm_head [V, H]   final_norm_w [H]
  *   in_norm_w/post_norm_w [H]   wq [Hq*d, H]   wk, wv [Hkv*d, H]   wo [H, Hq*d]
  *   q_norm_w, k_norm_w [d]      w_gate, w_up [I, H]   w_down [H, I]
- * dflash_create copies wq/wk/wv, w_gate/w_up and the stacked K/V weights into
- * packed buffers it owns; every other pointer is kept and must stay valid (and
- * unchanged) for the lifetime of the handle (embed / lm_head are the target's
- * aliased tables and are not copied). */
+ * Storage precision of the path: the projections whose inputs are bounded by
+ * construction (RMSNorm outputs, attention outputs) run with fp16 operands, so
+ * dflash_create keeps fp16 copies of wq|wk|wv (packed), w_gate|w_up (packed in
+ * 16-row blocks), the stacked per-layer [wk; wv], wo and lm_head (bf16 -> fp16
+ * is exact in fp16's normal range).  fc_w and w_down are used in bf16 in place,
+ * as are the norm weights and the embedding (the target's aliased table): those
+ * pointers must stay valid and unchanged for the lifetime of the handle. */
 typedef struct dflash_weights {
   const void* fc_w;
   const void* hidden_norm_w;
@@ -235,7 +238,7 @@ dflash_status dflash_linear_ex(dflash_handle* h, const void* A, const void* W, i
 /* One layer of non-causal block attention (§"What is DFlash": every block query
  * attends to the injected context and the whole block), on a layer's caches:
  *   q [B*bs, n_q_heads, head_dim] bf16 (block rows in request order)
- *   o [B*bs, n_q_heads*head_dim] bf16 out
+ *   o [B*bs, n_q_heads*head_dim] fp16 out (as the proposal path stores it)
  * Request b attends to its logical keys [0, seq_lens[b] + bs), located through
  * block_table exactly as in dflash_propose; scale 1/sqrt(head_dim).
  * Needs dflash_attention_workspace_bytes(h, B, max_pages_per_seq). */
@@ -245,6 +248,44 @@ dflash_status dflash_block_attention(dflash_handle* h, const void* q, const int3
                                      const void* k_cache, const void* v_cache, int num_pages,
                                      void* o, void* workspace, size_t workspace_bytes,
                                      void* stream);
+
+/* ---- launch accounting and per-launch timing (diagnostics) ---- */
+
+/* Kernel families launched by the calls above (ids for dflash_profile_read). */
+enum {
+  DFLASH_KERNEL_EMBED_NORM = 0,      /* block build + embedding + first RMSNorm       */
+  DFLASH_KERNEL_GEMM_QKV = 1,        /* QKV GEMM + q/k norm + RoPE + block K/V write  */
+  DFLASH_KERNEL_ATTENTION = 2,       /* non-causal paged block attention             */
+  DFLASH_KERNEL_ATTN_COMBINE = 3,    /* split-KV merge                               */
+  DFLASH_KERNEL_GEMM_O = 4,          /* O projection + residual                      */
+  DFLASH_KERNEL_RMSNORM = 5,         /* row RMSNorms (post-attn, next input, final, hidden_norm) */
+  DFLASH_KERNEL_GEMM_GATE_UP = 6,    /* gate/up GEMM + SwiGLU                        */
+  DFLASH_KERNEL_GEMM_DOWN = 7,       /* down projection + residual                   */
+  DFLASH_KERNEL_GEMM_LM_HEAD = 8,    /* LM head + fused greedy argmax                */
+  DFLASH_KERNEL_ARGMAX_FINALIZE = 9, /* draft / block token write-out                */
+  DFLASH_KERNEL_GEMM_FC = 10,        /* fc over the tapped states                    */
+  DFLASH_KERNEL_GEMM_KV_INJECT = 11, /* all layers' K/V + k_norm + RoPE + scatter    */
+  DFLASH_KERNEL_LINEAR = 12,         /* dflash_linear / dflash_linear_ex             */
+  DFLASH_KERNEL_KINDS = 13
+};
+
+/* Number of kernel launches the handle's calls have issued so far (launches
+ * captured into a CUDA graph are counted once, at capture). */
+unsigned long long dflash_launch_count(const dflash_handle* h);
+
+/* Static name of a kernel family id, or NULL. */
+const char* dflash_kernel_name(int kind);
+
+/* While enabled, each launch of the handle's calls (up to max_launches of them
+ * until the next read) is bracketed by two CUDA events recorded on the call's
+ * stream.  dflash_profile_read synchronizes the device, returns per family k <
+ * n_kinds the number of recorded launches and their summed event time (ms),
+ * and restarts the recording.  Enabling allocates the events (a set-up call,
+ * not for use inside stream capture). */
+dflash_status dflash_profile_enable(dflash_handle* h, int max_launches);
+dflash_status dflash_profile_read(dflash_handle* h, int n_kinds, int* launches,
+                                  double* total_ms);
+dflash_status dflash_profile_disable(dflash_handle* h);
 
 /* Synchronizes the device, reads and clears the handle's device error word.
  * Returns DFLASH_OK if it was zero, DFLASH_ERR_DEVICE_TIMEOUT if the timeout bit

@@ -5,4 +5,4 @@ and the CPU-baseline leg of ``bench.py``; never by the library package.
 """
 from .dflash_oracle import *  # noqa: F401,F403
 from .dflash_oracle import (OracleConfig, Proposal, QueryBlock, Verification,  # noqa: F401
-                            BF16_STORAGE_POINTS)
+                            STORAGE_POINTS, FP16_WEIGHTS)

@@ -21,12 +21,16 @@ passage it follows.  The three pages are cited by title:
 Precision modes
 ---------------
 ``exact``   every intermediate stays float64.  Used for the logits check
-            (relative L2 against the bf16 GPU path).
-``bf16io``  rounds to bfloat16 (round-to-nearest-even, via float32) at the
-            storage points listed in ``BF16_STORAGE_POINTS``; everything else
-            stays float64.  Used for bit-exact draft / acceptance comparison.
-            Argmax decisions are taken on float32-rounded logits in both modes
-            (the kernel's decision precision).
+            (relative L2 against the GPU path).
+``device``  rounds (round-to-nearest-even, via float32) at the storage points
+            of ``STORAGE_POINTS`` to the format the device path stores there,
+            and uses the fp16 copies of the weights that the device path
+            multiplies in fp16; everything else stays float64.  Used for
+            bit-exact draft / acceptance comparison.
+``bf16``    rounds every storage point to bfloat16 (an all-bf16 pipeline; for
+            error analysis).
+Argmax decisions are taken on float32-rounded logits in every mode (the
+kernel's decision precision).
 
 Readings where the pages are silent (each is also listed in the design notes):
   * every norm is RMSNorm ``x * rsqrt(mean(x^2) + eps) * w`` (weight multiplies
@@ -52,17 +56,22 @@ from typing import Callable, Mapping, Sequence
 
 import numpy as np
 
-# Storage points at which the ``bf16io`` mode rounds to bfloat16.  The names
-# are the oracle's own; the GPU path rounds at the same points by design.
-BF16_STORAGE_POINTS = (
-    "context vector c = hidden_norm(fc(x))",
-    "injected context K (after k_norm + RoPE) and V",
-    "normed activations fed to a projection (input/post-attention norms)",
-    "block q after q_norm + RoPE; block K (after k_norm + RoPE) and V",
-    "attention output o",
-    "MLP hidden silu(gate) * up",
-    "final-normed rows fed to the LM head",
-)
+# Storage points of the proposal path and the format the device path keeps
+# there.  Operands that are bounded by construction (RMSNorm outputs: |y_i| <=
+# sqrt(H) max|w|; attention outputs: convex combinations of V rows) are held in
+# fp16; the KV cache, q (attended against that cache) and the MLP hidden stay
+# bf16.  ``device`` mode rounds to these formats; ``bf16`` mode to bf16 everywhere.
+STORAGE_POINTS = {
+    "context": "fp16",     # c = hidden_norm(fc(x)), fed to the K/V projection
+    "kv": "bf16",          # K (after k_norm + RoPE) and V entries of the paged cache
+    "norm": "fp16",        # input / post-attention RMSNorm outputs fed to projections
+    "q": "bf16",           # block q after q_norm + RoPE
+    "attn_out": "fp16",    # attention output o, fed to Wo
+    "mlp_hidden": "bf16",  # silu(gate) * up, fed to Wd
+    "final": "fp16",       # final-normed kept rows, fed to the LM head
+}
+# Weights multiplied in fp16 by the device path (held there as fp16 copies).
+FP16_WEIGHTS = ("wq", "wk", "wv", "wo", "w_gate", "w_up", "lm_head")
 
 
 # ----------------------------------------------------------------------------
@@ -116,16 +125,46 @@ def round_bf16(a) -> np.ndarray:
     return u.astype(np.uint32).view(np.float32).astype(np.float64)
 
 
+def round_fp16(a) -> np.ndarray:
+    """Round to IEEE binary16 (nearest, ties to even; via float32, subnormals
+    kept, overflow to inf) and return float64 values."""
+    f = np.asarray(a, dtype=np.float64).astype(np.float32)
+    with np.errstate(over="ignore"):
+        return f.astype(np.float16).astype(np.float64)
+
+
 def _identity(a) -> np.ndarray:
     return np.asarray(a, dtype=np.float64)
 
 
-def rounding(mode: str) -> Callable[[np.ndarray], np.ndarray]:
-    if mode == "exact":
-        return _identity
-    if mode == "bf16io":
-        return round_bf16
-    raise ValueError(f"unknown precision mode {mode!r}")
+_ROUND = {"bf16": round_bf16, "fp16": round_fp16}
+MODES = ("exact", "device", "bf16")
+
+
+class Rounding:
+    """Callable ``rnd(point, value)`` for one precision mode."""
+
+    def __init__(self, mode: str):
+        if mode not in MODES:
+            raise ValueError(f"unknown precision mode {mode!r}")
+        self.mode = mode
+
+    def __call__(self, point: str, a) -> np.ndarray:
+        if self.mode == "exact":
+            return _identity(a)
+        if self.mode == "bf16":
+            return round_bf16(a)
+        return _ROUND[STORAGE_POINTS[point]](a)
+
+    def weight(self, name: str, w) -> np.ndarray:
+        """A weight as the mode's GEMM sees it (fp16 copies in device mode)."""
+        if self.mode == "device" and name in FP16_WEIGHTS:
+            return round_fp16(w)
+        return w
+
+
+def rounding(mode: str) -> Rounding:
+    return Rounding(mode)
 
 
 # ----------------------------------------------------------------------------
@@ -249,7 +288,7 @@ def context_fusion(cfg: OracleConfig, W: Mapping, aux: np.ndarray,
     aux = np.asarray(aux, dtype=np.float64)
     assert aux.shape[-1] == cfg.n_target_layers * cfg.hidden
     f = linear(aux, W["fc_w"])
-    return rnd(rms_norm(f, W["hidden_norm_w"], cfg.rms_eps))
+    return rnd("context", rms_norm(f, W["hidden_norm_w"], cfg.rms_eps))
 
 
 def context_kv(cfg: OracleConfig, W: Mapping, ctx: np.ndarray,
@@ -261,15 +300,15 @@ def context_kv(cfg: OracleConfig, W: Mapping, ctx: np.ndarray,
     rnd = rounding(mode)
     L, Hkv, d = cfg.n_layers, cfg.n_kv_heads, cfg.head_dim
     fused = np.concatenate(
-        [np.concatenate([W["wk"][l], W["wv"][l]], axis=0) for l in range(L)],
-        axis=0)                                   # [L * 2 * Hkv * d, hidden]
+        [np.concatenate([rnd.weight("wk", W["wk"][l]), rnd.weight("wv", W["wv"][l])], axis=0)
+         for l in range(L)], axis=0)              # [L * 2 * Hkv * d, hidden]
     kv = linear(ctx, fused).reshape(ctx.shape[0], L, 2, Hkv, d)
     ks, vs = [], []
     for l in range(L):
         k = rms_norm(kv[:, l, 0], W["k_norm_w"][l], cfg.rms_eps)
         k = apply_rope(k, positions, cfg.rope_theta)
-        ks.append(rnd(k))
-        vs.append(rnd(kv[:, l, 1]))
+        ks.append(rnd("kv", k))
+        vs.append(rnd("kv", kv[:, l, 1]))
     return ks, vs
 
 
@@ -368,7 +407,7 @@ class Proposal:
 def draft_layer(cfg: OracleConfig, W: Mapping, l: int, x: np.ndarray,
                 qb: QueryBlock, block_table, seq_lens,
                 k_cache: np.ndarray, v_cache: np.ndarray,
-                rnd: Callable) -> np.ndarray:
+                rnd: Rounding) -> np.ndarray:
     """One DFlashQwen3DecoderLayer ([NEURON] "DFlash Draft Model
     Architecture": a standard Qwen3 decoder layer, attention + MLP with
     pre-norms, attention run non-causally):
@@ -384,31 +423,34 @@ def draft_layer(cfg: OracleConfig, W: Mapping, l: int, x: np.ndarray,
     """
     Hq, Hkv, d, eps = cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim, cfg.rms_eps
     M = x.shape[0]
-    n = rnd(rms_norm(x, W["in_norm_w"][l], eps))
-    q = linear(n, W["wq"][l]).reshape(M, Hq, d)
-    k = linear(n, W["wk"][l]).reshape(M, Hkv, d)
-    v = linear(n, W["wv"][l]).reshape(M, Hkv, d)
-    q = rnd(apply_rope(rms_norm(q, W["q_norm_w"][l], eps), qb.positions,
-                       cfg.rope_theta))
-    k = rnd(apply_rope(rms_norm(k, W["k_norm_w"][l], eps), qb.positions,
-                       cfg.rope_theta))
-    v = rnd(v)
+    w = rnd.weight
+    n = rnd("norm", rms_norm(x, W["in_norm_w"][l], eps))
+    q = linear(n, w("wq", W["wq"][l])).reshape(M, Hq, d)
+    k = linear(n, w("wk", W["wk"][l])).reshape(M, Hkv, d)
+    v = linear(n, w("wv", W["wv"][l])).reshape(M, Hkv, d)
+    q = rnd("q", apply_rope(rms_norm(q, W["q_norm_w"][l], eps), qb.positions,
+                            cfg.rope_theta))
+    k = rnd("kv", apply_rope(rms_norm(k, W["k_norm_w"][l], eps), qb.positions,
+                             cfg.rope_theta))
+    v = rnd("kv", v)
     slots = paged_slots(qb.positions, qb.req_ids, block_table, cfg.page_size)
     write_slots(k_cache, slots, k, cfg.page_size)
     write_slots(v_cache, slots, v, cfg.page_size)
-    o = rnd(block_attention(cfg, q, k_cache, v_cache, block_table, seq_lens))
-    x = x + linear(o.reshape(M, Hq * d), W["wo"][l])
-    n2 = rnd(rms_norm(x, W["post_norm_w"][l], eps))
-    h = rnd(silu(linear(n2, W["w_gate"][l])) * linear(n2, W["w_up"][l]))
+    o = rnd("attn_out", block_attention(cfg, q, k_cache, v_cache, block_table, seq_lens))
+    x = x + linear(o.reshape(M, Hq * d), w("wo", W["wo"][l]))
+    n2 = rnd("norm", rms_norm(x, W["post_norm_w"][l], eps))
+    h = rnd("mlp_hidden", silu(linear(n2, w("w_gate", W["w_gate"][l])))
+            * linear(n2, w("w_up", W["w_up"][l])))
     return x + linear(h, W["w_down"][l])
 
 
-def lm_head_logits(W: Mapping, rows: np.ndarray, chunk: int = 16384) -> np.ndarray:
+def lm_head_logits(W: Mapping, rows: np.ndarray, chunk: int = 16384,
+                   weight: Callable = lambda name, w: w) -> np.ndarray:
     """rows @ lm_head^T in float64, a vocabulary chunk at a time."""
     V = W["lm_head"].shape[0]
     out = np.empty((rows.shape[0], V), dtype=np.float64)
     for v0 in range(0, V, chunk):
-        out[:, v0:v0 + chunk] = linear(rows, W["lm_head"][v0:v0 + chunk])
+        out[:, v0:v0 + chunk] = linear(rows, weight("lm_head", W["lm_head"][v0:v0 + chunk]))
     return out
 
 
@@ -429,8 +471,8 @@ def propose(cfg: OracleConfig, W: Mapping, bonus_tokens, seq_lens, block_table,
         x = draft_layer(cfg, W, l, x, qb, block_table, seq_lens,
                         k_caches[l], v_caches[l], rnd)
     kept = x[qb.keep_idx]
-    f = rnd(rms_norm(kept, W["final_norm_w"], cfg.rms_eps))
-    logits = lm_head_logits(W, f)
+    f = rnd("final", rms_norm(kept, W["final_norm_w"], cfg.rms_eps))
+    logits = lm_head_logits(W, f, weight=rnd.weight)
     drafts = argmax_f32(logits).reshape(B, K)
     block = np.concatenate([bonus[:, None], drafts], axis=1)
     return Proposal(drafts, block, logits, x)

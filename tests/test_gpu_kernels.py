@@ -105,13 +105,26 @@ def _attention_case(cfg, seq_lens, seed):
     shape = (num_pages, cfg["n_kv_heads"], cfg["page_size"], cfg["head_dim"])
     kc = torch.randn(shape, generator=g).to(torch.bfloat16)
     vc = torch.randn(shape, generator=g).to(torch.bfloat16)
-    # NaN in unused slots must not leak into results (P = 0 rows)
-    kc.view(-1)[-cfg["head_dim"]:] = float("nan")
+    # NaN wherever no request reads (past each request's last key in its last
+    # page, and unused pages) must not leak into results
+    used = set()
+    P = cfg["page_size"]
+    for b, s in enumerate(seq_lens):
+        n = s + cfg["block_size"]
+        used.update(int(x) for x in table[b, :-(-n // P)])
+        if n % P:
+            last = int(table[b, (n - 1) // P])
+            kc[last, :, n % P:] = float("nan")
+            vc[last, :, n % P:] = float("nan")
+    for pg in set(range(num_pages)) - used:
+        kc[pg] = float("nan")
+        vc[pg] = float("nan")
     B = len(seq_lens)
     q = torch.randn(B * cfg["block_size"], cfg["n_q_heads"], cfg["head_dim"],
                     generator=g).to(torch.bfloat16)
     ref = O.block_attention(oc, to_np(q).astype(np.float64), to_np(kc).astype(np.float64),
                             to_np(vc).astype(np.float64), table, seq_lens)
+    assert np.isfinite(ref).all()
     return q, kc, vc, table, ref
 
 
@@ -221,8 +234,8 @@ def _inject_case(cfg, Wt, h, n, seed, sample=None):
     rows = np.arange(n) if sample is None else sample
     W = weights_np(Wt) if not isinstance(Wt["fc_w"], np.ndarray) else Wt
     auxn = to_np(aux)[rows].astype(np.float64)
-    ctx_io = O.context_fusion(oc, W, auxn, "bf16io")
-    k_io, v_io = O.context_kv(oc, W, ctx_io, pos[rows], "bf16io")
+    ctx_io = O.context_fusion(oc, W, auxn, "device")
+    k_io, v_io = O.context_kv(oc, W, ctx_io, pos[rows], "device")
     ctx_ex = O.context_fusion(oc, W, auxn, "exact")
     k_ex, v_ex = O.context_kv(oc, W, ctx_ex, pos[rows], "exact")
     for l in range(cfg["n_layers"]):
@@ -232,9 +245,14 @@ def _inject_case(cfg, Wt, h, n, seed, sample=None):
             if s < 0:
                 continue
             gk, gv = kg[s // P, :, s % P], vg[s // P, :, s % P]
-            # one bf16 ulp against the bf16-storage oracle, 1e-2 rel-L2 against exact
-            assert np.all(np.abs(gk - k_io[l][j]) <= 2 ** -7 * np.abs(k_io[l][j]) + 1e-6), (l, r)
-            assert np.all(np.abs(gv - v_io[l][j]) <= 2 ** -7 * np.abs(v_io[l][j]) + 1e-6), (l, r)
+            # Against the storage-precision oracle: one bf16 ulp of the larger
+            # value plus 2e-3 of the head's RMS (pre-rounding values differ by
+            # fp32 accumulation order, which can move a value across a bf16
+            # rounding boundary); against the exact oracle: 1e-2 relative L2.
+            for got, want in ((gk, k_io[l][j]), (gv, v_io[l][j])):
+                tol = (2.0 ** -7 * np.maximum(np.abs(got), np.abs(want))
+                       + 2e-3 * np.sqrt(np.mean(want ** 2, axis=-1, keepdims=True)))
+                assert np.all(np.abs(got - want) <= tol), (l, r)
             assert rel_l2(gk, k_ex[l][j]) < 1e-2 and rel_l2(gv, v_ex[l][j]) < 1e-2
         # padding rows and untouched slots keep the sentinel
         for r in np.nonzero(slots < 0)[0][:8]:

@@ -1,9 +1,9 @@
 """GPU parity of the whole proposal (inject -> propose) against the oracle.
 
-Drafts (greedy picks) must be bit-exact against the oracle's bf16-storage mode,
-except rows whose top-2 logit gap in that oracle is below 1e-3 (counted and
-reported, not compared); the LM-head logits must be within relative L2 1e-2 of
-the oracle's exact (float64) mode.  The GPU chain and the oracle chain each
+Drafts (greedy picks) must be bit-exact against the oracle's ``device``
+storage-precision mode, except rows whose top-2 logit gap in that oracle is
+below 1e-3 (counted and reported, not compared); the LM-head logits must be
+within relative L2 1e-2 of the oracle's exact (float64) mode.  The GPU chain and the oracle chain each
 inject the same context with their own code; nothing flows from one to the
 other.
 """
@@ -107,7 +107,7 @@ def test_tiny_chain(tiny, ctx_lens):
     cfg, Wt, h = tiny
     ch = Chain(cfg, Wt, h, ctx_lens, seed=sum(ctx_lens) + len(ctx_lens))
     d, lo, blk = ch.gpu()
-    p_io, p_ex = ch.oracle("bf16io"), ch.oracle("exact")
+    p_io, p_ex = ch.oracle("device"), ch.oracle("exact")
     K = cfg["block_size"] - 1
     excluded = compare_drafts(d, lo, p_io, p_ex, K)
     assert excluded <= max(1, len(ctx_lens) * K // 10)
@@ -220,14 +220,14 @@ def test_qwen3_b1_step():
         assert h.check_device_errors() == 0
         Wn = weights_np(Wt)
         res = {}
-        for mode in ("bf16io", "exact"):
+        for mode in ("device", "exact"):
             ko = [to_np(t).astype(np.float64) for t in kc]
             vo = [to_np(t).astype(np.float64) for t in vc]
             O.inject_context(oc, Wn, to_np(sb.aux).astype(np.float64),
                              to_np(sb.inject_positions), slots, ko, vo, mode)
             res[mode] = O.propose(oc, Wn, to_np(sb.bonus), to_np(sb.seq_lens),
                                   to_np(sb.block_table), ko, vo, mode)
-        excluded = compare_drafts(to_np(d), to_np(lo), res["bf16io"], res["exact"], K)
+        excluded = compare_drafts(to_np(d), to_np(lo), res["device"], res["exact"], K)
         assert excluded <= 3
     finally:
         h.close()

@@ -109,6 +109,29 @@ def test_round_bf16_matches_torch():
     np.testing.assert_array_equal(O.round_bf16(x), ref)
 
 
+def test_round_fp16_matches_torch():
+    rng = np.random.default_rng(14)
+    x = np.concatenate([rng.standard_normal(10000) * 10.0 ** rng.integers(-9, 6, 10000),
+                        [70000.0, -1e6, 6.1e-5, 3e-8, 65504.0, 65520.0]])
+    ref = torch.tensor(x, dtype=torch.float64).float().to(torch.float16).double().numpy()
+    np.testing.assert_array_equal(O.round_fp16(x), ref)
+
+
+def test_storage_modes():
+    """device mode rounds each storage point to its declared format; weights
+    multiplied in fp16 are fp16-rounded; exact mode leaves values alone."""
+    x = np.array([1.0 + 2.0 ** -9, 1.0 + 2.0 ** -12, 3.0e-6])
+    dev, ex, b16 = O.rounding("device"), O.rounding("exact"), O.rounding("bf16")
+    for point, fmt in O.STORAGE_POINTS.items():
+        want = O.round_fp16(x) if fmt == "fp16" else O.round_bf16(x)
+        np.testing.assert_array_equal(dev(point, x), want)
+        np.testing.assert_array_equal(b16(point, x), O.round_bf16(x))
+        np.testing.assert_array_equal(ex(point, x), x)
+    np.testing.assert_array_equal(dev.weight("lm_head", x), O.round_fp16(x))
+    np.testing.assert_array_equal(dev.weight("fc_w", x), x)
+    np.testing.assert_array_equal(dev.weight("w_down", x), x)
+
+
 def test_argmax_ties_and_nan():
     rng = np.random.default_rng(3)
     a = rng.integers(0, 4, (200, 9)).astype(np.float32)  # many ties
