@@ -512,9 +512,17 @@ cudaError_t use_device(int dev) {
 
 // Handle-free calls run on the device of their stream (or, on the legacy
 // default stream, of their output buffer).
+// Under stream capture the device is not queried (a stream query would
+// invalidate a global-mode capture); the current device is used as is.
 dflash_status set_device_for(cudaStream_t st, const void* p) {
   int dev = -1;
   if (st != nullptr) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) {
+      cudaGetLastError();
+      return DFLASH_ERR_INVALID_ARG;
+    }
+    if (cs != cudaStreamCaptureStatusNone) return DFLASH_OK;
     if (cudaStreamGetDevice(st, &dev) != cudaSuccess) {
       cudaGetLastError();
       return DFLASH_ERR_INVALID_ARG;
