@@ -1227,3 +1227,77 @@ dflash_status dflash_check_device_errors(dflash_handle* h, unsigned* bits) {
 }
 
 }  // extern "C"
+
+// ===========================================================================
+// Greedy verification that allocates nothing
+// ===========================================================================
+// Some callers cannot hand this library a workspace: an embedding runtime that
+// reserved all device memory for its own pool at start-up (a cudaMalloc from
+// here could fail or fragment that pool), a plugin that only ever receives its
+// input and output buffers from the host framework and owns no allocator, or
+// a latency-critical decode loop where cudaMalloc / cudaFree would synchronize
+// the device.  dflash_verify_greedy_noalloc serves them with scratch that the
+// library already owns: a fixed array in this module's device memory.
+namespace {
+
+// One 64-bit partial argmax key per (request, target row, vocabulary chunk).
+// Every device that loads this library holds these 64 KiB until the process
+// exits.  Calls share the array; it keeps whatever the last call wrote.
+constexpr int kNoAllocVerifyKeys = DFLASH_VERIFY_NOALLOC_MAX_PARTIALS;
+static __device__ __align__(256) unsigned long long g_verify_scratch[kNoAllocVerifyKeys];
+
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_verify_scratch_mu;
+unsigned long long* g_verify_scratch_dev[kNoAllocMaxDevices] = {};
+
+// On the host, g_verify_scratch only names the symbol; a kernel given that
+// name would read the wrong memory.  The array's device address is looked up
+// once per device (with that device current) and cached.
+dflash_status verify_scratch_on_current_device(unsigned long long** out) {
+  int dev = -1;
+  DF_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return DFLASH_ERR_UNSUPPORTED_SHAPE;
+  std::lock_guard<std::mutex> lk(g_verify_scratch_mu);
+  if (!g_verify_scratch_dev[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_verify_scratch) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      return DFLASH_ERR_CUDA;
+    }
+    g_verify_scratch_dev[dev] = static_cast<unsigned long long*>(p);
+  }
+  *out = g_verify_scratch_dev[dev];
+  return DFLASH_OK;
+}
+
+}  // namespace
+
+extern "C" dflash_status dflash_verify_greedy_noalloc(const int32_t* drafts,
+                                                      const float* target_logits, int B, int K,
+                                                      int V, int32_t* out_tokens,
+                                                      int32_t* num_accepted, int32_t* bonus,
+                                                      void* stream) {
+  if (B < 0 || K < 0 || V <= 0 || K > 128) return DFLASH_ERR_INVALID_ARG;
+  if (B == 0) return DFLASH_OK;
+  if ((K > 0 && !drafts) || !target_logits || !out_tokens || !num_accepted || !bonus)
+    return DFLASH_ERR_INVALID_ARG;
+  const VerifyPlan vp = plan_verify(B, K, V);
+  if (static_cast<int64_t>(B) * (K + 1) * vp.chunks > kNoAllocVerifyKeys)
+    return DFLASH_ERR_WORKSPACE;  // needs more partial keys than the fixed scratch holds
+  if (reinterpret_cast<uintptr_t>(target_logits) % 16 && V % 4 == 0)
+    return DFLASH_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  dflash_status s = set_device_for(st, out_tokens);
+  if (s != DFLASH_OK) return s;
+  unsigned long long* part = nullptr;
+  s = verify_scratch_on_current_device(&part);
+  if (s != DFLASH_OK) return s;
+  // Nothing in the scratch has to start at zero: the second kernel reads only
+  // the keys the first one writes in this same call.
+  verify_partial_kernel<<<dim3(vp.chunks, B * (K + 1)), 256, 0, st>>>(target_logits, V,
+                                                                      vp.chunk_len, vp.chunks,
+                                                                      part);
+  verify_final_kernel<<<B, 32, 0, st>>>(part, vp.chunks, drafts, K, out_tokens, num_accepted,
+                                        bonus);
+  return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ERR_CUDA;
+}

@@ -86,6 +86,7 @@ def lib() -> ctypes.CDLL:
         "dflash_propose": ([vp, vp, vp, vp, i32, i32, _PP, _PP, i32, vp, vp, vp, vp, sz, vp],
                            i32),
         "dflash_verify_greedy": ([vp, vp, i32, i32, i32, vp, vp, vp, vp, sz, vp], i32),
+        "dflash_verify_greedy_noalloc": ([vp, vp, i32, i32, i32, vp, vp, vp, vp], i32),
         "dflash_linear": ([vp, vp, vp, i32, i32, i32, vp, vp, sz, vp], i32),
         "dflash_linear_ex": ([vp, vp, vp, i32, i32, i32, vp, i32, i32, vp, sz, vp], i32),
         "dflash_block_attention": ([vp, vp, vp, vp, i32, i32, vp, vp, i32, vp, vp, sz, vp],
@@ -344,6 +345,29 @@ def verify_greedy(drafts, target_logits, out_tokens=None, num_accepted=None, bon
                                       _ptr(out_tokens), _ptr(num_accepted), _ptr(bonus),
                                       _ptr(workspace), workspace.numel(), _stream(stream)),
            "dflash_verify_greedy")
+    return out_tokens, num_accepted, bonus
+
+
+def verify_greedy_noalloc(drafts, target_logits, out_tokens=None, num_accepted=None,
+                          bonus=None, stream=None):
+    """Greedy acceptance without a workspace (dflash_verify_greedy_noalloc), for
+    callers that cannot allocate device scratch; returns (out_tokens, n, bonus).
+    The library's fixed scratch is shared by all calls: keep calls on one stream."""
+    B, K1, V = target_logits.shape
+    K = K1 - 1
+    dev = target_logits.device
+    _want(drafts, torch.int32, "drafts")
+    _want(target_logits, torch.float32, "target_logits")
+    if out_tokens is None:
+        out_tokens = torch.empty(B, K + 1, dtype=torch.int32, device=dev)
+    if num_accepted is None:
+        num_accepted = torch.empty(B, dtype=torch.int32, device=dev)
+    if bonus is None:
+        bonus = torch.empty(B, dtype=torch.int32, device=dev)
+    _check(lib().dflash_verify_greedy_noalloc(_ptr(drafts), _ptr(target_logits), B, K, V,
+                                              _ptr(out_tokens), _ptr(num_accepted), _ptr(bonus),
+                                              _stream(stream)),
+           "dflash_verify_greedy_noalloc")
     return out_tokens, num_accepted, bonus
 
 

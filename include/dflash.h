@@ -147,6 +147,34 @@ size_t dflash_propose_workspace_bytes(const dflash_handle* h, int max_batch,
 /* Workspace needed by dflash_verify_greedy for [B, K+1, V] target logits. */
 size_t dflash_verify_workspace_bytes(int B, int K, int V);
 
+/* Maximum number of partial keys (request x target row x vocabulary chunk)
+ * that dflash_verify_greedy_noalloc can hold: 8192 (64 KiB of device memory). */
+#define DFLASH_VERIFY_NOALLOC_MAX_PARTIALS 8192
+
+/* The same greedy verification as dflash_verify_greedy, for callers that cannot
+ * allocate device memory for a workspace: an embedding runtime that reserved
+ * all device memory for its own pool, a plugin that only receives its input
+ * and output buffers, or a latency-critical loop where cudaMalloc/cudaFree
+ * would synchronize the device.  (The pages have no counterpart of this call;
+ * it is an addition of this library.)
+ * Arguments, outputs and results are exactly those of dflash_verify_greedy,
+ * without the workspace.  Its scratch is a fixed 64 KiB array inside this
+ * library's device memory, present on every device that loads the library
+ * until the process exits; the call allocates nothing.
+ *   - The first call on a device looks up that array's device address (with
+ *     the device current) and caches it; make that first call before any
+ *     stream capture.
+ *   - Every call shares the one array and leaves its last contents behind.
+ *     Calls that overlap on the GPU (e.g. on two streams at once) race on it
+ *     and give wrong results; order them on one stream.
+ *   - Batches needing more than DFLASH_VERIFY_NOALLOC_MAX_PARTIALS partial keys
+ *     are rejected with DFLASH_ERR_WORKSPACE before any launch (every batch up
+ *     to 512 requests with K = 15 fits). */
+dflash_status dflash_verify_greedy_noalloc(const int32_t* drafts, const float* target_logits,
+                                           int B, int K, int V, int32_t* out_tokens,
+                                           int32_t* num_accepted, int32_t* bonus,
+                                           void* stream);
+
 /* _paged_slots (§"Paged KV Integration"), exactly as the page writes it:
  *   page_no = min(positions[i] / page_size, max_pages_per_seq - 1)
  *   slots[i] = block_table[req_ids[i] * max_pages_per_seq + page_no] * page_size
