@@ -268,14 +268,17 @@ __global__ void __launch_bounds__(32 * (kAttnMaxComputeWarps + 1), 1)
         }
       }
 
-      // O += P V, 16 keys (one page) per k-step
+      // O += P V, 16 keys (one page) per k-step.  P is split into bf16 hi + lo
+      // parts (P = hi + lo to ~2^-17) so that the tensor-core product does not
+      // add bf16 rounding of the probabilities to the output.
 #pragma unroll
       for (int kk = 0; kk < KS; ++kk) {
         if (kk * 16 < nvalid) {
-          const uint32_t a0 = pack_bf16x2(s[2 * kk][0], s[2 * kk][1]);
-          const uint32_t a1 = pack_bf16x2(s[2 * kk][2], s[2 * kk][3]);
-          const uint32_t a2 = pack_bf16x2(s[2 * kk + 1][0], s[2 * kk + 1][1]);
-          const uint32_t a3 = pack_bf16x2(s[2 * kk + 1][2], s[2 * kk + 1][3]);
+          uint32_t ah[4], al[4];
+          split_bf16x2(s[2 * kk][0], s[2 * kk][1], ah[0], al[0]);
+          split_bf16x2(s[2 * kk][2], s[2 * kk][3], ah[1], al[1]);
+          split_bf16x2(s[2 * kk + 1][0], s[2 * kk + 1][1], ah[2], al[2]);
+          split_bf16x2(s[2 * kk + 1][2], s[2 * kk + 1][3], ah[3], al[3]);
 #pragma unroll
           for (int dbp = 0; dbp < D / 16; ++dbp) {
             const int j = lane >> 3;
@@ -283,8 +286,10 @@ __global__ void __launch_bounds__(32 * (kAttnMaxComputeWarps + 1), 1)
             const int c = dbp * 2 + (j >> 1);
             uint32_t b0, b1, b2, b3;
             ldmatrix_x4_trans(vbase + kv_off<D>(kt, c), b0, b1, b2, b3);
-            mma_bf16_16816(o[2 * dbp], a0, a1, a2, a3, b0, b1);
-            mma_bf16_16816(o[2 * dbp + 1], a0, a1, a2, a3, b2, b3);
+            mma_bf16_16816(o[2 * dbp], ah[0], ah[1], ah[2], ah[3], b0, b1);
+            mma_bf16_16816(o[2 * dbp + 1], ah[0], ah[1], ah[2], ah[3], b2, b3);
+            mma_bf16_16816(o[2 * dbp], al[0], al[1], al[2], al[3], b0, b1);
+            mma_bf16_16816(o[2 * dbp + 1], al[0], al[1], al[2], al[3], b2, b3);
           }
         }
       }
@@ -411,20 +416,33 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const AttnParams p) {
     }
     l += wl;
     const int cnt = min(32, ns - s0);
-    for (int j = 0; j < cnt; ++j) {
-      const float ws = __shfl_sync(0xffffffffu, w, j);
-      const float* src = p.part_o + row_of(s0 + j) * D + lane * PER;
-      if constexpr (PER == 4) {
-        const float4 v = *reinterpret_cast<const float4*>(src);
-        acc[0] += ws * v.x;
-        acc[1] += ws * v.y;
-        acc[2] += ws * v.z;
-        acc[3] += ws * v.w;
-      } else {
-        const float2 v = *reinterpret_cast<const float2*>(src);
-        acc[0] += ws * v.x;
-        acc[1] += ws * v.y;
+    // four splits' loads in flight at a time; past-the-end slots reread the
+    // last split with weight 0
+    for (int j = 0; j < cnt; j += 4) {
+      float ws[4];
+      float v[4][PER];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int jj = min(j + u, cnt - 1);
+        const float wsu = __shfl_sync(0xffffffffu, w, jj);
+        ws[u] = (j + u < cnt) ? wsu : 0.f;
+        const float* src = p.part_o + row_of(s0 + jj) * D + lane * PER;
+        if constexpr (PER == 4) {
+          const float4 q = *reinterpret_cast<const float4*>(src);
+          v[u][0] = q.x;
+          v[u][1] = q.y;
+          v[u][2] = q.z;
+          v[u][3] = q.w;
+        } else {
+          const float2 q = *reinterpret_cast<const float2*>(src);
+          v[u][0] = q.x;
+          v[u][1] = q.y;
+        }
       }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int e = 0; e < PER; ++e) acc[e] += ws[u] * v[u][e];
     }
   }
 #pragma unroll

@@ -73,8 +73,9 @@ bool make_tmap(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t cols,
 // GEMM planning
 // ---------------------------------------------------------------------------
 struct GemmPlan {
-  int BN = 0, splits = 1, kb_per_split = 0, m_tiles = 0, n_tiles = 0, k_blocks = 0, units = 0,
-      grid = 0, a_rows = 128, stages = 1, smem = 0;
+  int BN = 0, m_tiles = 0, n_tiles = 0, k_blocks = 0, tiles = 0, stream_k = 0, ipc = 0,
+      total_iters = 0, nacc = 1, tmem_cols = 32, grid = 0, a_rows = 128, stages = 1, smem = 0,
+      slot_rows = 0;
   size_t partial_bytes = 0;
 };
 
@@ -88,62 +89,53 @@ int gemm_stages(int a_rows, int bn) {
   return st;
 }
 
-void finish_plan(GemmPlan& pl, int M) {
+// Tile width, accumulator chains and schedule.  Small M (weight-streaming):
+// BN = 128 with two accumulator chains; M >= 256 (tensor-bound): BN = 256
+// with one.  Whole tiles are handed out round-robin when they fill the SMs
+// evenly (>= 90% of the last round busy); otherwise stream-K splits the
+// (tile, k-block) iterations evenly over the SMs.  force_bn / force_splits
+// (0 = automatic) pin the tile width and the schedule: 1 = whole tiles,
+// n >= 2 = stream-K with ceil(k_blocks / n) iterations per CTA.
+GemmPlan plan_gemm(int M, int N, int K, int group, int num_sms, int force_bn = 0,
+                   int force_splits = 0) {
+  GemmPlan pl;
+  pl.k_blocks = K / kGemmBK;
+  pl.m_tiles = cdiv(M, kGemmBM);
+  pl.BN = force_bn ? force_bn : (M >= 2 * kGemmBM ? 256 : 128);
+  if (pl.BN < group || pl.BN % group) pl.BN = std::max(group, 128);
+  pl.nacc = pl.BN >= 256 ? 1 : pl.BN >= 128 ? 2 : 4;
+  pl.tmem_cols = 32;
+  while (pl.tmem_cols < 2 * pl.nacc * pl.BN) pl.tmem_cols *= 2;
+  pl.n_tiles = cdiv(N, pl.BN);
+  pl.tiles = pl.m_tiles * pl.n_tiles;
+  const int rounds = cdiv(pl.tiles, num_sms);
+  const double fill = static_cast<double>(pl.tiles) / (static_cast<double>(rounds) * num_sms);
+  bool sk = fill < 0.9;
+  if (force_splits == 1) sk = false;
+  if (force_splits >= 2) sk = true;
+  if (sk && pl.tiles > kCounterSlots) sk = false;
+  pl.total_iters = pl.tiles * pl.k_blocks;
+  if (sk) {
+    pl.stream_k = 1;
+    if (force_splits >= 2) {
+      pl.ipc = cdiv(pl.k_blocks, force_splits);
+    } else {
+      pl.ipc = std::max(cdiv(pl.total_iters, num_sms), std::min(pl.k_blocks, 4));
+    }
+    pl.grid = cdiv(pl.total_iters, pl.ipc);
+    pl.slot_rows = std::min(M, kGemmBM);
+    pl.partial_bytes = static_cast<size_t>(pl.grid) * 2 * pl.slot_rows * pl.BN * 4;
+  } else {
+    pl.stream_k = 0;
+    pl.ipc = pl.k_blocks;
+    pl.grid = std::min(pl.tiles, num_sms);
+    pl.slot_rows = std::min(M, kGemmBM);
+    pl.partial_bytes = 0;
+  }
   pl.a_rows = gemm_a_rows(M);
   pl.stages = gemm_stages(pl.a_rows, pl.BN);
   pl.smem = gemm_smem_bytes(pl.a_rows, pl.BN, pl.stages);
-}
-
-// Picks the tile width BN (a multiple of the epilogue group) and the K-split
-// count by minimising a per-SM time estimate: the busiest SM runs
-// ceil(units / SMs) units, each bounded by its weight bytes (HBM) or its
-// padded 128-row MMA work (tensor pipe), plus a fixed per-unit cost; splitting
-// K adds the round trip of fp32 partials.
-GemmPlan plan_gemm(int M, int N, int K, int group, int num_sms) {
-  GemmPlan best;
-  double best_t = 1e300;
-  const int k_blocks = K / kGemmBK;
-  const int m_tiles = cdiv(M, kGemmBM);
-  const double bw_sm = 90e9;                 // bytes/s one SM's TMA ring sustains
-  const double fl_sm = 1.6e15 / 148.0;
-  const double hbm = 6.5e12;
-  const double a_rows = gemm_a_rows(M);
-  const int bns[4] = {256, 128, 64, 32};
-  for (int bi = 0; bi < 4; ++bi) {
-    const int BN = bns[bi];
-    if (BN < group || BN % group) continue;
-    const int n_tiles = cdiv(N, BN);
-    for (int S = 1; S <= 16; ++S) {
-      if (S > 1 && (m_tiles > 1 || k_blocks / S < 4)) break;
-      if (S > 1 && m_tiles * n_tiles > kCounterSlots) break;
-      const int kbps = cdiv(k_blocks, S);
-      const int splits = cdiv(k_blocks, kbps);
-      if (splits != S) continue;
-      const int units = m_tiles * n_tiles * S;
-      const int rounds = cdiv(units, num_sms);
-      const double kspan = static_cast<double>(kbps) * kGemmBK;
-      const double unit_bytes = (BN + a_rows) * kspan * 2.0;
-      const double unit_flops = 2.0 * kGemmBM * BN * kspan;
-      double t = rounds * (std::max(unit_bytes / bw_sm, unit_flops / fl_sm) + 1.0e-6);
-      const double total_w = static_cast<double>(N) * K * 2.0;
-      t = std::max(t, total_w / hbm);
-      if (S > 1) t += static_cast<double>(S) * M * N * 4.0 * 2.0 / hbm + 1.0e-6;
-      if (t < best_t * 0.999) {
-        best_t = t;
-        best.BN = BN;
-        best.splits = S;
-        best.kb_per_split = kbps;
-        best.m_tiles = m_tiles;
-        best.n_tiles = n_tiles;
-        best.k_blocks = k_blocks;
-        best.units = units;
-        best.grid = std::min(units, num_sms);
-        best.partial_bytes = S > 1 ? static_cast<size_t>(S) * M * N * 4 : 0;
-      }
-    }
-  }
-  if (best.BN) finish_plan(best, M);
-  return best;
+  return pl;
 }
 
 // ---------------------------------------------------------------------------
@@ -307,26 +299,12 @@ dflash_status run_gemm(dflash_handle* h, int kind, bool f16, const void* A, int 
                        size_t partial_cap, cudaStream_t st, int force_bn = 0,
                        int force_splits = 0) {
   if (M <= 0) return DFLASH_OK;
-  GemmPlan pl = plan_gemm(M, N, K, Epi::kGroup, h->num_sms);
-  if (force_bn || force_splits) {
-    const int BN = force_bn ? force_bn : pl.BN;
-    const int S = force_splits ? force_splits : pl.splits;
-    if ((BN != 32 && BN != 64 && BN != 128 && BN != 256) || BN % Epi::kGroup)
-      return DFLASH_ERR_INVALID_ARG;
-    pl.BN = BN;
-    pl.k_blocks = K / kGemmBK;
-    pl.m_tiles = cdiv(M, kGemmBM);
-    pl.n_tiles = cdiv(N, BN);
-    if (S < 1 || S > pl.k_blocks) return DFLASH_ERR_INVALID_ARG;
-    if (S > 1 && pl.m_tiles * pl.n_tiles > kCounterSlots) return DFLASH_ERR_UNSUPPORTED_SHAPE;
-    pl.kb_per_split = cdiv(pl.k_blocks, S);
-    pl.splits = cdiv(pl.k_blocks, pl.kb_per_split);
-    pl.units = pl.m_tiles * pl.n_tiles * pl.splits;
-    pl.grid = std::min(pl.units, h->num_sms);
-    pl.partial_bytes = pl.splits > 1 ? static_cast<size_t>(pl.splits) * M * N * 4 : 0;
-    finish_plan(pl, M);
-  }
-  if (pl.BN == 0) return DFLASH_ERR_UNSUPPORTED_SHAPE;
+  if (force_bn && ((force_bn != 32 && force_bn != 64 && force_bn != 128 && force_bn != 256) ||
+                   force_bn % Epi::kGroup))
+    return DFLASH_ERR_INVALID_ARG;
+  if (force_splits < 0 || force_splits > K / kGemmBK) return DFLASH_ERR_INVALID_ARG;
+  const GemmPlan pl = plan_gemm(M, N, K, Epi::kGroup, h->num_sms, force_bn, force_splits);
+  if (pl.stream_k && pl.tiles > kCounterSlots) return DFLASH_ERR_UNSUPPORTED_SHAPE;
   if (pl.partial_bytes > partial_cap) return DFLASH_ERR_WORKSPACE;
   CUtensorMap ta, tw;
   if (!h->tmap(&ta, A, M, K, pl.a_rows, f16)) return DFLASH_ERR_CUDA;
@@ -338,12 +316,16 @@ dflash_status run_gemm(dflash_handle* h, int kind, bool f16, const void* A, int 
   gp.m_tiles = pl.m_tiles;
   gp.n_tiles = pl.n_tiles;
   gp.k_blocks = pl.k_blocks;
-  gp.splits = pl.splits;
-  gp.kb_per_split = pl.kb_per_split;
-  gp.num_units = pl.units;
+  gp.tiles = pl.tiles;
+  gp.stream_k = pl.stream_k;
+  gp.ipc = pl.ipc;
+  gp.total_iters = pl.total_iters;
+  gp.nacc = pl.nacc;
+  gp.tmem_cols = pl.tmem_cols;
   gp.a_rows = pl.a_rows;
   gp.stages = pl.stages;
   gp.f16 = f16 ? 1 : 0;
+  gp.slot_rows = pl.slot_rows;
   gp.partials = partials;
   gp.counters = h->counters;
   gp.err = h->dev_err;
@@ -1044,7 +1026,7 @@ dflash_status dflash_verify_greedy(const int32_t* drafts, const float* target_lo
   verify_partial_kernel<<<dim3(vp.chunks, B * (K + 1)), 256, 0, st>>>(target_logits, V,
                                                                       vp.chunk_len, vp.chunks,
                                                                       part);
-  verify_final_kernel<<<B, 32, 0, st>>>(part, vp.chunks, drafts, K, out_tokens, num_accepted,
+  verify_final_kernel<<<B, 256, 0, st>>>(part, vp.chunks, drafts, K, out_tokens, num_accepted,
                                         bonus);
   return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ERR_CUDA;
 }
@@ -1297,7 +1279,7 @@ extern "C" dflash_status dflash_verify_greedy_noalloc(const int32_t* drafts,
   verify_partial_kernel<<<dim3(vp.chunks, B * (K + 1)), 256, 0, st>>>(target_logits, V,
                                                                       vp.chunk_len, vp.chunks,
                                                                       part);
-  verify_final_kernel<<<B, 32, 0, st>>>(part, vp.chunks, drafts, K, out_tokens, num_accepted,
+  verify_final_kernel<<<B, 256, 0, st>>>(part, vp.chunks, drafts, K, out_tokens, num_accepted,
                                         bonus);
   return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ERR_CUDA;
 }

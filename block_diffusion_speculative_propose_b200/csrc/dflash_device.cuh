@@ -47,6 +47,15 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// (a, b) -> bf16x2 hi = rn(a, b) and lo = rn(a - hi, b - hi), so hi + lo
+// carries a and b to ~2^-17 relative.
+__device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t& hi, uint32_t& lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  const __nv_bfloat162 l = __floats2bfloat162_rn(a - __low2float(h), b - __high2float(h));
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+
 // Ordered 64-bit key for a greedy pick: the high word orders fp32 values
 // (NaN is mapped onto -inf, -0 onto +0), the low word is ~index so that the
 // numerically largest key is the largest value with the lowest index.
@@ -209,7 +218,7 @@ __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
 
 // 32 lanes x 32 consecutive fp32 columns; thread t of the warp gets lane
 // (warp's sub-partition base + t), columns [col, col + 32).
-__device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, float (&v)[32]) {
+__device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, float* v) {
   uint32_t r[32];
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 "

@@ -8,14 +8,19 @@
 // into a ring of shared-memory stages; warp 1 issues tcgen05.mma (M=128, N=BN,
 // K=16, one thread) into a double-buffered fp32 accumulator in tensor memory;
 // warps 2..5 drain the accumulator with tcgen05.ld and run the epilogue functor
-// while the next tile accumulates.  Units of work are (k-split, n-tile, m-tile)
-// triples handed out round-robin to one CTA per SM.
+// while the next tile accumulates.  A tile's K=16 steps are spread over `nacc`
+// independent accumulator chains (summed in chain order by the epilogue) so
+// that narrow, weight-streaming tiles are not paced by the latency of one
+// dependent MMA chain.
 //
-// Split-K (used only when a weight-streaming GEMM has too few output tiles to
-// occupy every SM): each split writes its fp32 partial tile to global memory;
-// the CTA that finishes a tile's last split (detected with a per-tile arrival
-// counter, no waiting) sums the partials in split order — so the result is
-// deterministic — and runs the epilogue.  The counters are left at zero.
+// Scheduling: whole tiles round-robin over one CTA per SM when there are
+// enough of them to fill the GPU evenly; otherwise stream-K — every CTA takes
+// an equal contiguous range of the (tile, k-block) iteration space, so every
+// SM streams weights.  A tile split across CTAs has each piece written as an
+// fp32 partial (at most two slots per CTA); the CTA that finishes the tile's
+// last piece (a per-tile arrival counter, no waiting) sums the pieces in CTA
+// order — so the result is deterministic — and runs the epilogue.  The
+// counters are left at zero.
 //
 // Every pipeline wait is bounded (see mbar_wait); a wait that runs out sets the
 // timeout bit and the CTA winds down, frees its tensor memory and returns.
@@ -36,8 +41,6 @@ constexpr int kGemmBarrierBytes = 2 * kGemmMaxStages * 8 + 4 * 8 + 16;
 template <int BN>
 struct GemmCfg {
   static constexpr int kBBytes = BN * kGemmBK * 2;
-  static constexpr int kTmemCols = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
-                                   : (2 * BN <= 256) ? 256 : 512;
   static_assert(BN % 16 == 0 && BN >= 32 && BN <= 256, "UMMA N for M=128");
 };
 
@@ -53,41 +56,87 @@ __host__ __device__ inline int gemm_smem_bytes(int a_rows, int bn, int stages) {
 struct GemmParams {
   int M, N, K;
   int m_tiles, n_tiles, k_blocks;
-  int splits, kb_per_split, num_units;
+  int tiles;           // m_tiles * n_tiles
+  int stream_k;        // 0: whole tiles round-robin; 1: equal ranges of (tile, k-block) iterations
+  int ipc;             // stream-K: k-block iterations per CTA
+  int total_iters;     // stream-K: tiles * k_blocks
+  int nacc;            // independent accumulator chains per tile (1, 2 or 4)
+  int tmem_cols;       // allocated TMEM columns (>= 2 * nacc * BN, power of two)
   int a_rows;          // rows of the A box / slot (128, or M rounded up to 16 when M < 128)
   int stages;          // pipeline depth (<= kGemmMaxStages)
   int f16;             // operands are fp16 (1) or bf16 (0)
-  float* partials;     // [splits][M][N] when splits > 1
-  unsigned* counters;  // [m_tiles * n_tiles], zero on entry, zero on exit
+  int slot_rows;       // rows held per partial slot (min(M, 128))
+  float* partials;     // stream-K: [gridDim.x * 2][slot_rows][BN] fp32
+  unsigned* counters;  // [tiles], zero on entry, zero on exit
   unsigned* err;
 };
 
-struct GemmUnit {
-  int m_tile, n_tile, split, kb0, kb1;
+// One contiguous piece of one output tile's K range, as processed by one CTA.
+struct GemmSeg {
+  int tile, m_tile, n_tile, kb0, kb1;
+  int first_cta, nseg;  // CTAs contributing to this tile (stream-K), 1 for whole tiles
+  int slot;             // this CTA's partial slot for the tile when nseg > 1
 };
-__device__ __forceinline__ GemmUnit decode_unit(const GemmParams& p, int u) {
-  GemmUnit t;
-  const int per_split = p.m_tiles * p.n_tiles;
-  t.split = u / per_split;
-  const int r = u - t.split * per_split;
-  t.n_tile = r / p.m_tiles;
-  t.m_tile = r - t.n_tile * p.m_tiles;
-  t.kb0 = t.split * p.kb_per_split;
-  t.kb1 = min(p.k_blocks, t.kb0 + p.kb_per_split);
-  return t;
+
+// Iterates the segments of this CTA.  Every warp role walks the same sequence.
+struct GemmSegIter {
+  int cur, end, step;
+  __device__ __forceinline__ explicit GemmSegIter(const GemmParams& p) {
+    if (p.stream_k) {
+      cur = blockIdx.x * p.ipc;
+      end = min(p.total_iters, cur + p.ipc);
+      step = 0;
+    } else {
+      cur = blockIdx.x;
+      end = p.tiles;
+      step = gridDim.x;
+    }
+  }
+  __device__ __forceinline__ bool next(const GemmParams& p, GemmSeg& s) {
+    if (cur >= end) return false;
+    if (p.stream_k) {
+      s.tile = cur / p.k_blocks;
+      s.kb0 = cur - s.tile * p.k_blocks;
+      s.kb1 = min(p.k_blocks, s.kb0 + (end - cur));
+      const int tile_beg = s.tile * p.k_blocks;
+      s.first_cta = tile_beg / p.ipc;
+      s.nseg = (tile_beg + p.k_blocks - 1) / p.ipc - s.first_cta + 1;
+      s.slot = blockIdx.x * 2 + (cur == static_cast<int>(blockIdx.x) * p.ipc ? 0 : 1);
+      cur += s.kb1 - s.kb0;
+    } else {
+      s.tile = cur;
+      s.kb0 = 0;
+      s.kb1 = p.k_blocks;
+      s.first_cta = 0;
+      s.nseg = 1;
+      s.slot = 0;
+      cur += step;
+    }
+    s.n_tile = s.tile / p.m_tiles;
+    s.m_tile = s.tile - s.n_tile * p.m_tiles;
+    return true;
+  }
+};
+
+// Partial slot that CTA c used for `tile` (the slot index rule of GemmSegIter).
+__device__ __forceinline__ int gemm_slot_of(const GemmParams& p, int tile, int c) {
+  const int seg_beg = max(tile * p.k_blocks, c * p.ipc);
+  return c * 2 + (seg_beg == c * p.ipc ? 0 : 1);
 }
 
-template <int N>
-__device__ __forceinline__ void tmem_load_cols(uint32_t taddr, float* v) {
-  static_assert(N % 32 == 0, "");
-#pragma unroll
-  for (int c = 0; c < N / 32; ++c) {
-    float t[32];
-    tmem_ld_32x32b_x32(taddr + c * 32, t);
-#pragma unroll
-    for (int j = 0; j < 32; ++j) v[c * 32 + j] = t[j];
-  }
+// Sum of the nacc accumulator chains for 32 columns at TMEM address taddr
+// (chains BN columns apart), in chain order.
+template <int BN>
+__device__ __forceinline__ void tmem_load_sum32(uint32_t taddr, int nacc, float* v) {
+  tmem_ld_32x32b_x32(taddr, v);
   tmem_ld_wait();
+  for (int j = 1; j < nacc; ++j) {
+    float t[32];
+    tmem_ld_32x32b_x32(taddr + j * BN, t);
+    tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] += t[i];
+  }
 }
 
 template <int BN, class Epi>
@@ -131,13 +180,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tma_prefetch_desc(&tmW);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_alloc(tmem_slot, static_cast<uint32_t>(p.tmem_cols));
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  const int acc_cols = p.nacc * BN;   // TMEM columns of one accumulator buffer
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -146,18 +196,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint64_t pol_a = policy_evict_last();
       uint32_t stage = 0, phase = 0;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
-        const GemmUnit t = decode_unit(p, u);
-        for (int kb = t.kb0; kb < t.kb1; ++kb) {
+      GemmSegIter it(p);
+      GemmSeg sg;
+      while (ok && it.next(p, sg)) {
+        for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, p.err)) {
             ok = false;
             break;
           }
           mbar_arrive_expect_tx(&full[stage], stage_tx);
           tma_load_2d_hint(sA + stage * a_bytes, &tmA, &full[stage], kb * kGemmBK,
-                           t.m_tile * kGemmBM, pol_a);
+                           sg.m_tile * kGemmBM, pol_a);
           tma_load_2d_hint(sB + stage * C::kBBytes, &tmW, &full[stage], kb * kGemmBK,
-                           t.n_tile * BN, pol_w);
+                           sg.n_tile * BN, pol_w);
           if (++stage == static_cast<uint32_t>(stages)) {
             stage = 0;
             phase ^= 1u;
@@ -171,12 +222,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint32_t idesc = umma_idesc_f32acc(kGemmBM, BN, p.f16 != 0);
       uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
-        const GemmUnit t = decode_unit(p, u);
+      GemmSegIter it(p);
+      GemmSeg sg;
+      while (ok && it.next(p, sg)) {
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, p.err)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc * BN;
-        for (int kb = t.kb0; kb < t.kb1; ++kb) {
+        const uint32_t d_base = tmem_base + acc * acc_cols;
+        int t = 0;   // K=16 step index within the segment; chain = t % nacc
+        for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
           if (!mbar_wait(&full[stage], phase, p.err)) {
             ok = false;
             break;
@@ -185,11 +238,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const uint64_t adesc = umma_desc_sw128(smem_u32(sA + stage * a_bytes));
           const uint64_t bdesc = umma_desc_sw128(smem_u32(sB + stage * C::kBBytes));
 #pragma unroll
-          for (int k = 0; k < kGemmBK / 16; ++k) {
+          for (int k = 0; k < kGemmBK / 16; ++k, ++t) {
             // +32 bytes along K inside the 128-byte swizzle atom = +2 in the
             // descriptor's (address >> 4) field
-            umma_f16kind(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc,
-                      (kb > t.kb0 || k > 0) ? 1u : 0u);
+            const int chain = t % p.nacc;
+            umma_f16kind(d_base + chain * BN, adesc + 2 * k, bdesc + 2 * k, idesc,
+                         t >= p.nacc ? 1u : 0u);
           }
           umma_commit(&empty[stage]);
           if (++stage == static_cast<uint32_t>(stages)) {
@@ -209,21 +263,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int sp = warp & 3;        // TMEM sub-partition this warp may read
     const int row = sp * 32 + lane;
     uint32_t acc = 0, acc_phase = 0;
-    for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
-      const GemmUnit t = decode_unit(p, u);
+    GemmSegIter it(p);
+    GemmSeg sg;
+    while (it.next(p, sg)) {
       if (!mbar_wait(&tfull[acc], acc_phase, p.err)) break;
       tc_fence_after();
-      const int m = t.m_tile * kGemmBM + row;
+      const int m = sg.m_tile * kGemmBM + row;
       const bool row_ok = m < p.M;
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(sp * 32) << 16) + acc * BN;
-      if (p.splits == 1) {
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(sp * 32) << 16) + acc * acc_cols;
+      if (sg.nseg == 1) {
         typename Epi::State st;
         epi.begin(st);
 #pragma unroll 1
         for (int g = 0; g < BN / G; ++g) {
           float v[G];
-          tmem_load_cols<G>(taddr + g * G, v);
-          const int n0 = t.n_tile * BN + g * G;
+#pragma unroll
+          for (int c = 0; c < G / 32; ++c) tmem_load_sum32<BN>(taddr + g * G + c * 32, p.nacc, v + c * 32);
+          const int n0 = sg.n_tile * BN + g * G;
           if (row_ok && n0 < p.N) epi.apply(st, m, n0, min(G, p.N - n0), v);
         }
         epi.end(st, m, row_ok);
@@ -231,25 +287,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&tempty[acc]);
       } else {
-        float* part = p.partials + static_cast<size_t>(t.split) * p.M * p.N;
+        float* part = p.partials + static_cast<size_t>(sg.slot) * p.slot_rows * BN;
 #pragma unroll 1
         for (int g = 0; g < BN / G; ++g) {
           float v[G];
-          tmem_load_cols<G>(taddr + g * G, v);
-          const int n0 = t.n_tile * BN + g * G;
-          if (row_ok && n0 < p.N) {
-            float* dst = part + static_cast<size_t>(m) * p.N + n0;
-            const int nv = min(G, p.N - n0);
-            if (nv == G) {
 #pragma unroll
-              for (int j = 0; j < G; j += 4)
-                __stcg(reinterpret_cast<float4*>(dst + j),
-                       make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]));
-            } else {
+          for (int c = 0; c < G / 32; ++c) tmem_load_sum32<BN>(taddr + g * G + c * 32, p.nacc, v + c * 32);
+          if (row_ok) {
+            float* dst = part + static_cast<size_t>(row) * BN + g * G;
 #pragma unroll
-              for (int j = 0; j < G; ++j)
-                if (j < nv) __stcg(dst + j, v[j]);
-            }
+            for (int j = 0; j < G; j += 4)
+              __stcg(reinterpret_cast<float4*>(dst + j),
+                     make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]));
           }
         }
         __threadfence();
@@ -258,10 +307,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (lane == 0) mbar_arrive(&tempty[acc]);
         named_bar_sync(1, 128);
         if (ew == 0 && lane == 0) {
-          const int tile = t.m_tile * p.n_tiles + t.n_tile;
-          const unsigned prev = atomicAdd(&p.counters[tile], 1u);
-          const int last = (prev == static_cast<unsigned>(p.splits - 1)) ? 1 : 0;
-          if (last) p.counters[tile] = 0u;
+          const unsigned prev = atomicAdd(&p.counters[sg.tile], 1u);
+          const int last = (prev == static_cast<unsigned>(sg.nseg - 1)) ? 1 : 0;
+          if (last) p.counters[sg.tile] = 0u;
           *last_flag = last;
         }
         named_bar_sync(1, 128);
@@ -272,35 +320,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           epi.begin(st);
 #pragma unroll 1
           for (int g = 0; g < BN / G; ++g) {
-            const int n0 = t.n_tile * BN + g * G;
+            const int n0 = sg.n_tile * BN + g * G;
             if (row_ok && n0 < p.N) {
-              const int nv = min(G, p.N - n0);
               float v[G];
 #pragma unroll
               for (int j = 0; j < G; ++j) v[j] = 0.f;
-              for (int s = 0; s < p.splits; ++s) {
-                const float* src = p.partials + (static_cast<size_t>(s) * p.M + m) * p.N + n0;
-                if (nv == G) {
+              for (int c = sg.first_cta; c < sg.first_cta + sg.nseg; ++c) {
+                const float* src = p.partials +
+                                   (static_cast<size_t>(gemm_slot_of(p, sg.tile, c)) *
+                                        p.slot_rows + row) * BN + g * G;
 #pragma unroll
-                  for (int j = 0; j < G; j += 4) {
-                    const float4 q = __ldcg(reinterpret_cast<const float4*>(src + j));
-                    v[j] += q.x;
-                    v[j + 1] += q.y;
-                    v[j + 2] += q.z;
-                    v[j + 3] += q.w;
-                  }
-                } else {
-#pragma unroll
-                  for (int j = 0; j < G; ++j)
-                    if (j < nv) v[j] += __ldcg(src + j);
+                for (int j = 0; j < G; j += 4) {
+                  const float4 q = __ldcg(reinterpret_cast<const float4*>(src + j));
+                  v[j] += q.x;
+                  v[j + 1] += q.y;
+                  v[j + 2] += q.z;
+                  v[j + 3] += q.w;
                 }
               }
-              epi.apply(st, m, n0, nv, v);
+              epi.apply(st, m, n0, min(G, p.N - n0), v);
             }
           }
           epi.end(st, m, row_ok);
         }
-        named_bar_sync(1, 128);  // last_flag is rewritten by the next unit
+        named_bar_sync(1, 128);  // last_flag is rewritten by the next segment
       }
       acc ^= 1u;
       if (acc == 0) acc_phase ^= 1u;
@@ -311,7 +354,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, C::kTmemCols);
+    tmem_dealloc(tmem_base, static_cast<uint32_t>(p.tmem_cols));
   }
 }
 

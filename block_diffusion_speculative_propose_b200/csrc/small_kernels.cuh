@@ -178,33 +178,40 @@ __global__ void __launch_bounds__(256) verify_partial_kernel(
   }
 }
 
-// Pass 2 (one warp per request): t_j for j = 0..K, longest matching prefix,
-// bonus, and the -1 padded output row.
-__global__ void verify_final_kernel(const unsigned long long* __restrict__ part, int chunks,
-                                    const int32_t* __restrict__ drafts, int K,
-                                    int32_t* __restrict__ out, int32_t* __restrict__ n_acc,
-                                    int32_t* __restrict__ bonus) {
+// Pass 2 (one CTA per request, one warp per target row): t_j for j = 0..K,
+// longest matching prefix, bonus, and the -1 padded output row.
+__global__ void __launch_bounds__(256) verify_final_kernel(
+    const unsigned long long* __restrict__ part, int chunks,
+    const int32_t* __restrict__ drafts, int K, int32_t* __restrict__ out,
+    int32_t* __restrict__ n_acc, int32_t* __restrict__ bonus) {
   __shared__ int32_t t[130];
-  const int b = blockIdx.x, lane = threadIdx.x;
-  for (int j = 0; j <= K; ++j) {
+  __shared__ int32_t d[130];
+  __shared__ int n_sh;
+  const int b = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nw = blockDim.x >> 5;
+  for (int j = threadIdx.x; j < K; j += blockDim.x) d[j] = drafts[static_cast<size_t>(b) * K + j];
+  for (int j = warp; j <= K; j += nw) {
     const unsigned long long* pr = part + (static_cast<size_t>(b) * (K + 1) + j) * chunks;
     unsigned long long best = 0ull;
     for (int c = lane; c < chunks; c += 32) best = pr[c] > best ? pr[c] : best;
     best = warp_max_u64(best);
     if (lane == 0) t[j] = static_cast<int32_t>(argmax_key_index(best));
   }
-  __syncwarp();
-  int n = 0;
-  while (n < K && drafts[static_cast<size_t>(b) * K + n] == t[n]) ++n;
-  for (int j = lane; j <= K; j += 32) {
-    int32_t v = -1;
-    if (j < n) v = drafts[static_cast<size_t>(b) * K + j];
-    else if (j == n) v = t[n];
-    out[static_cast<size_t>(b) * (K + 1) + j] = v;
-  }
-  if (lane == 0) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int n = 0;
+    while (n < K && d[n] == t[n]) ++n;
+    n_sh = n;
     n_acc[b] = n;
     bonus[b] = t[n];
+  }
+  __syncthreads();
+  const int n = n_sh;
+  for (int j = threadIdx.x; j <= K; j += blockDim.x) {
+    int32_t v = -1;
+    if (j < n) v = d[j];
+    else if (j == n) v = t[n];
+    out[static_cast<size_t>(b) * (K + 1) + j] = v;
   }
 }
 

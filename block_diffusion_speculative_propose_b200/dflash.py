@@ -272,7 +272,9 @@ class DFlash:
             out = torch.empty(M, N, dtype=torch.float32, device=self.device)
         need = lib().dflash_linear_workspace_bytes(self.h, M, N, K) if M else 0
         if splits > 1:
-            need = max(need, splits * M * N * 4)
+            bn = block_n or 256
+            tiles = -(-M // 128) * -(-N // bn)
+            need = max(need, 2 * (tiles * splits + 1) * min(M, 128) * bn * 4)
         ws = workspace if workspace is not None else self.ws.get(need)
         _check(lib().dflash_linear_ex(self.h, _ptr(A), _ptr(W), M, N, K, _ptr(out), block_n,
                                       splits, _ptr(ws), ws.numel(), _stream(stream)),

@@ -256,9 +256,11 @@ dflash_status dflash_linear(dflash_handle* h, const void* A, const void* W, int 
                             int K, float* out, void* workspace, size_t workspace_bytes,
                             void* stream);
 /* Same with the launch plan chosen by the caller: tile width block_n in
- * {32, 64, 128, 256} and K-split count `splits` (>= 1, <= K/64); 0 for either
- * means "as the automatic plan".  Split-K needs splits*M*N*4 bytes of
- * workspace (dflash_linear_workspace_bytes covers only the automatic plan). */
+ * {32, 64, 128, 256}; `splits` = 1 schedules whole tiles, n >= 2 schedules
+ * stream-K with ceil(K/64 / n) k-blocks per CTA (<= K/64); 0 for either means
+ * "as the automatic plan".  Stream-K needs 2 * CTAs * min(M,128) * block_n * 4
+ * bytes of workspace, CTAs <= tiles * n + 1 (dflash_linear_workspace_bytes
+ * covers only the automatic plan). */
 dflash_status dflash_linear_ex(dflash_handle* h, const void* A, const void* W, int M, int N,
                                int K, float* out, int block_n, int splits, void* workspace,
                                size_t workspace_bytes, void* stream);

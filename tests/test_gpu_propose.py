@@ -33,8 +33,13 @@ def compare_drafts(gpu_drafts, gpu_logits, prop_io, prop_ex, K):
     assert mism.size == 0, f"draft mismatch at rows {mism[:10]} gaps {gap[mism[:10]]}"
     if gpu_logits is not None:
         gl = np.asarray(gpu_logits, dtype=np.float64)
+        ex = [rel_l2(gl[r], prop_ex.logits[r]) for r in range(gl.shape[0])]
+        dv = [rel_l2(gl[r], prop_io.logits[r]) for r in range(gl.shape[0])]
+        print(f"logits rel-L2 vs exact: max {max(ex):.3e} mean {np.mean(ex):.3e}; "
+              f"vs device-precision oracle: max {max(dv):.3e}; near-ties excluded "
+              f"{int((~ok).sum())} of {ok.size}")
         for r in range(gl.shape[0]):
-            assert rel_l2(gl[r], prop_ex.logits[r]) < 1e-2, r
+            assert ex[r] < 1e-2, r
     return int((~ok).sum())
 
 
