@@ -74,6 +74,8 @@ __global__ void __launch_bounds__(32 * (kAttnMaxComputeWarps + 1), 1)
   using C = AttnCfg<D>;
   constexpr int NB = KP / 8;    // 8-key blocks of this warp's part of a tile
   constexpr int KS = KP / 16;   // 16-key (one page) PV steps
+  pdl_trigger();
+  pdl_wait();
   const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int n_keys = p.seq_lens[b] + p.bs;
   const int k0 = split * p.chunk_keys;
@@ -387,6 +389,8 @@ __global__ void __launch_bounds__(32 * (kAttnMaxComputeWarps + 1), 1)
 template <int D>
 __global__ void __launch_bounds__(256) attn_combine_kernel(const AttnParams p) {
   constexpr int PER = D / 32;   // elements of the row per lane
+  pdl_trigger();
+  pdl_wait();
   const int gw = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (gw >= p.B * p.Hkv * p.R) return;

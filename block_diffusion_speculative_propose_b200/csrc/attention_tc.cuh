@@ -1,0 +1,392 @@
+// attention_tc.cuh — non-causal block attention on the 5th-generation tensor
+// cores (tcgen05 MMA, accumulators in tensor memory).
+//
+// Same contract as attn_block_kernel (attention.cuh): one CTA per (request b,
+// kv head h, key split); every query row of the kv group (bs block slots x G
+// heads, zero-padded to 64 rows) attends to the request's keys
+// [split * chunk, ...) of [0, seq_len + bs) with no mask inside the range.
+//
+//   warp 0      TMA producer: walks the block table, stages 128-key tiles of
+//               K and V (eight 16-key pages, 128-byte swizzle) in a 2-deep ring
+//   warp 1      MMA issuer (one thread): S = Q K^T into a double-buffered TMEM
+//               S (M=64 rows x 128 keys), then O += P_hi V + P_lo V into TMEM
+//               O (64 x d); S of tile t+1 is issued before P V of tile t
+//   warps 2..5  softmax: each reads its 16 rows of S with tcgen05.ld.16x256b
+//               (the mma.sync accumulator-fragment layout), applies the online
+//               softmax (row statistics by quad shuffles), writes P split into
+//               bf16 hi + lo parts to shared memory as the next MMA's operand.
+//               O is rescaled in TMEM only when a row maximum grows by more than
+//               2^8 since the last rescale (the reference maximum is shared by P,
+//               the row sum and O, so the result is exact either way).
+//
+// Shared memory: K/V ring 2 x (K + V) tiles, Q (64 x d), P hi/lo x 2 buffers.
+// TMEM: S buffers at columns [0, 256), O at [256, 256 + d).  Every wait is
+// bounded; a wait that runs out sets the timeout bit and the CTA winds down.
+#pragma once
+
+#include "attention.cuh"
+
+namespace dflash {
+
+constexpr int kTcKeys = 128;        // keys per tile (8 pages)
+constexpr int kTcStages = 2;        // K/V ring depth
+constexpr int kTcM = 64;            // MMA M: query rows of a kv group, zero-padded
+constexpr int kTcThreads = 192;     // warp 0 TMA, warp 1 MMA, warps 2..5 softmax
+constexpr float kTcLazyRescale = 8.f;  // log2 of the growth that forces an O rescale
+
+template <int D>
+struct TcAttnCfg {
+  static constexpr int kHalves = D / 64;                      // 64-element halves of a row
+  static constexpr int kKVBytes = kHalves * kTcKeys * 128;    // one K (or V) tile
+  static constexpr int kQBytes = kHalves * kTcM * 128;
+  static constexpr int kPBytes = (kTcKeys / 64) * kTcM * 128; // P hi (or lo) of one tile
+  static constexpr int kOffV = kTcStages * kKVBytes;
+  static constexpr int kOffQ = 2 * kTcStages * kKVBytes;
+  static constexpr int kOffP = kOffQ + kQBytes;
+  static constexpr int kOffBar = kOffP + 4 * kPBytes;
+  static constexpr int kSmem = 1024 + kOffBar + 256;
+  static constexpr int kOCol = 2 * kTcKeys;                   // TMEM column of O
+  static_assert(kOCol + D <= 512, "TMEM budget");
+};
+
+template <int D>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    attn_block_tc_kernel(const __grid_constant__ CUtensorMap tmK,
+                         const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+  using C = TcAttnCfg<D>;
+  pdl_trigger();
+  pdl_wait();
+  const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int n_keys = p.seq_lens[b] + p.bs;
+  const int k0 = split * p.chunk_keys;
+  if (k0 >= n_keys) return;
+  const int k1 = min(n_keys, k0 + p.chunk_keys);
+  const int n_splits_b = (n_keys + p.chunk_keys - 1) / p.chunk_keys;
+  const int n_tiles = (k1 - k0 + kTcKeys - 1) / kTcKeys;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sQ = smem + C::kOffQ;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint64_t* kv_full = bars;        // [2]
+  uint64_t* kv_empty = bars + 2;   // [2]
+  uint64_t* s_full = bars + 4;     // [2]
+  uint64_t* s_empty = bars + 6;    // [2]
+  uint64_t* p_full = bars + 8;     // [2]
+  uint64_t* p_empty = bars + 10;   // [2]
+  uint64_t* o_ready = bars + 12;   // one phase per tile: P V of that tile landed
+  uint64_t* q_full = bars + 13;
+  uint64_t* o_final = bars + 14;   // the last tile's P V landed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
+  auto sK = [&](int s) { return smem + s * C::kKVBytes; };
+  auto sV = [&](int s) { return smem + C::kOffV + s * C::kKVBytes; };
+  auto sP = [&](int lohi, int buf) { return smem + C::kOffP + (buf * 2 + lohi) * C::kPBytes; };
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_empty[i], 4);
+      mbar_init(&p_full[i], 4);
+      mbar_init(&p_empty[i], 1);
+    }
+    mbar_init(o_ready, 1);
+    mbar_init(q_full, 4);
+    mbar_init(o_final, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      const int* bt = p.block_table + static_cast<size_t>(b) * p.W;
+      for (int t = 0; t < n_tiles; ++t) {
+        const int s = t & 1, u = t >> 1;
+        if (!mbar_wait(&kv_empty[s], (u & 1) ^ 1u, p.err)) break;
+        const int t0 = k0 + t * kTcKeys;
+        const int nvalid = min(kTcKeys, k1 - t0);
+        const int npages = (nvalid + 15) >> 4;
+        mbar_arrive_expect_tx(&kv_full[s],
+                              static_cast<uint32_t>(8 * C::kHalves * 2048 * 2));
+        for (int j = 0; j < 8; ++j) {
+          int y = -16;  // pages past the range: fully out of bounds, TMA fills zeros
+          if (j < npages) {
+            const int pg = (t0 >> 4) + j;
+            if (pg >= p.W) {
+              raise_error(p.err, DFLASH_DEVERR_TABLE);
+            } else {
+              const int page = bt[pg];
+              if (page < 0 || page >= p.num_pages) raise_error(p.err, DFLASH_DEVERR_SLOT);
+              else y = (page * p.Hkv + h) * 16;
+            }
+          }
+#pragma unroll
+          for (int hf = 0; hf < C::kHalves; ++hf) {
+            const int off = hf * kTcKeys * 128 + j * 2048;
+            tma_load_2d(sK(s) + off, &tmK, &kv_full[s], hf * 64, y);
+            tma_load_2d(sV(s) + off, &tmV, &kv_full[s], hf * 64, y);
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_qk = umma_idesc_bf16(kTcM, kTcKeys, false);
+      const uint32_t idesc_pv = umma_idesc_bf16(kTcM, D, true);
+      bool ok = mbar_wait(q_full, 0, p.err);
+      tc_fence_after();
+      auto issue_qk = [&](int t) -> bool {
+        const int s = t & 1, u = t >> 1;
+        if (!mbar_wait(&kv_full[s], u & 1, p.err)) return false;
+        if (!mbar_wait(&s_empty[s], (u & 1) ^ 1u, p.err)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int half = kk >> 2, w = kk & 3;
+          const uint64_t ad = umma_desc_sw128(smem_u32(sQ + half * kTcM * 128 + w * 32));
+          const uint64_t bd = umma_desc_sw128(smem_u32(sK(s) + half * kTcKeys * 128 + w * 32));
+          umma_f16kind(tmem_base + s * kTcKeys, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&s_full[s]);
+        return true;
+      };
+      if (ok) ok = issue_qk(0);
+      for (int t = 0; ok && t < n_tiles; ++t) {
+        if (t + 1 < n_tiles && !issue_qk(t + 1)) break;
+        const int s = t & 1, u = t >> 1;
+        if (!mbar_wait(&p_full[s], u & 1, p.err)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int lohi = 0; lohi < 2; ++lohi) {
+#pragma unroll
+          for (int kk = 0; kk < kTcKeys / 16; ++kk) {
+            const int kh = kk >> 2, w = kk & 3;
+            const uint64_t ad = umma_desc_sw128(smem_u32(sP(lohi, s) + kh * kTcM * 128 + w * 32));
+            const uint64_t bd = umma_desc_sw128_mn(smem_u32(sV(s) + kk * 16 * 128),
+                                                   kTcKeys * 128, 1024);
+            umma_f16kind(tmem_base + C::kOCol, ad, bd, idesc_pv,
+                         (t > 0 || lohi > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        umma_commit(&kv_empty[s]);
+        umma_commit(&p_empty[s]);
+        umma_commit(o_ready);
+        if (t + 1 == n_tiles) umma_commit(o_final);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ softmax warps
+    const int sp = warp & 3;                    // TMEM sub-partition = 16-row group
+    const int tid = threadIdx.x - 64;           // 0..127
+    // Q rows r = i * G + g of this kv group -> K-major, 128B-swizzled operand
+    for (int e = tid; e < kTcM * (D / 8); e += 128) {
+      const int r = e / (D / 8), c = e - r * (D / 8);
+      uint4 val = make_uint4(0, 0, 0, 0);
+      if (r < p.R) {
+        const int i = r / p.G, g = r - (r / p.G) * p.G;
+        const bf16* src = p.q + (static_cast<size_t>(b * p.bs + i) * p.Hq + h * p.G + g) * D;
+        val = *reinterpret_cast<const uint4*>(src + c * 8);
+      }
+      *reinterpret_cast<uint4*>(sQ + (c >> 3) * kTcM * 128 + r * 128 + (((c & 7) ^ (r & 7)) << 4)) =
+          val;
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(q_full);
+
+    const uint32_t lane_base = static_cast<uint32_t>(32 * sp) << 16;
+    const int r0 = 16 * sp + (lane >> 2);       // this thread's rows r0 and r0 + 8
+    float m_ref[2] = {-INFINITY, -INFINITY};
+    float l_run[2] = {0.f, 0.f};
+    bool ok = true;
+    for (int t = 0; t < n_tiles; ++t) {
+      const int s = t & 1, u = t >> 1;
+      if (!mbar_wait(&s_full[s], u & 1, p.err)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float sv[4 * (kTcKeys / 8)];
+      tmem_ld_16x256b_x8(tmem_base + lane_base + s * kTcKeys, sv);
+      tmem_ld_16x256b_x8(tmem_base + lane_base + s * kTcKeys + 64, sv + 32);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_empty[s]);
+
+      const int t0 = k0 + t * kTcKeys;
+      const int nvalid = min(kTcKeys, k1 - t0);
+      float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+      for (int j = 0; j < kTcKeys / 8; ++j) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int kt = j * 8 + 2 * (lane & 3) + (e & 1);
+          const float v = sv[4 * j + e] * p.scale_log2;
+          sv[4 * j + e] = (kt < nvalid) ? v : -INFINITY;
+          mx[e >> 1] = fmaxf(mx[e >> 1], sv[4 * j + e]);
+        }
+      }
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        mx[hh] = fmaxf(mx[hh], __shfl_xor_sync(0xffffffffu, mx[hh], 1));
+        mx[hh] = fmaxf(mx[hh], __shfl_xor_sync(0xffffffffu, mx[hh], 2));
+      }
+      bool need[2];
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh)
+        need[hh] = mx[hh] != -INFINITY &&
+                   (m_ref[hh] == -INFINITY || mx[hh] > m_ref[hh] + kTcLazyRescale);
+      if (__any_sync(0xffffffffu, need[0] || need[1])) {
+        float nref[2], alpha[2];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          nref[hh] = need[hh] ? mx[hh] : m_ref[hh];
+          alpha[hh] = (m_ref[hh] == -INFINITY) ? 0.f : exp2f(m_ref[hh] - nref[hh]);
+        }
+        if (t > 0) {
+          // O holds P V of tiles < t against the old reference: rescale it once
+          // the previous tile's P V has landed.  (s_full of tile t implies P V
+          // of tile t-2 is complete, so o_ready is at most one phase behind and
+          // its parity names tile t-1 unambiguously.)
+          if (!mbar_wait(o_ready, (t - 1) & 1, p.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c) {
+            float ov[32];
+            tmem_ld_16x256b_x8(tmem_base + lane_base + C::kOCol + c * 64, ov);
+            tmem_ld_wait();
+#pragma unroll
+            for (int q = 0; q < 32; ++q) ov[q] *= alpha[(q >> 1) & 1];
+            tmem_st_16x256b_x8(tmem_base + lane_base + C::kOCol + c * 64, ov);
+          }
+          tmem_st_wait();
+        }
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          l_run[hh] *= alpha[hh];
+          m_ref[hh] = nref[hh];
+        }
+      }
+      float ref[2];
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) ref[hh] = (m_ref[hh] == -INFINITY) ? 0.f : m_ref[hh];
+#pragma unroll
+      for (int q = 0; q < 4 * (kTcKeys / 8); ++q) {
+        const float pv = exp2f(sv[q] - ref[(q >> 1) & 1]);
+        sv[q] = pv;
+        l_run[(q >> 1) & 1] += pv;
+      }
+      if (!mbar_wait(&p_empty[s], (u & 1) ^ 1u, p.err)) {
+        ok = false;
+        break;
+      }
+      uint8_t* ph = sP(0, s);
+      uint8_t* pl = sP(1, s);
+#pragma unroll
+      for (int j = 0; j < kTcKeys / 8; ++j) {
+        const int kh = j >> 3, ch = j & 7;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const int r = r0 + 8 * hh;
+          uint32_t hi, lo;
+          split_bf16x2(sv[4 * j + 2 * hh], sv[4 * j + 2 * hh + 1], hi, lo);
+          const int off = kh * kTcM * 128 + r * 128 + ((ch ^ (r & 7)) << 4) + (lane & 3) * 4;
+          *reinterpret_cast<uint32_t*>(ph + off) = hi;
+          *reinterpret_cast<uint32_t*>(pl + off) = lo;
+        }
+      }
+      if (sp == 0 && (nvalid & 15)) {
+        // rows past the last key of a partly used page may hold anything
+        // (NaN patterns included): zero them so that P = 0 rows add 0
+        const int jp = nvalid >> 4, rr0 = nvalid & 15;
+        const int n16 = (16 - rr0) * C::kHalves * 8;
+        for (int e = lane; e < n16; e += 32) {
+          const int hf = e / ((16 - rr0) * 8);
+          const int rem = e - hf * (16 - rr0) * 8;
+          const int rr = rr0 + rem / 8, cc = rem & 7;
+          *reinterpret_cast<uint4*>(sV(s) + hf * kTcKeys * 128 + jp * 2048 + rr * 128 + cc * 16) =
+              make_uint4(0, 0, 0, 0);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[s]);
+    }
+
+    float o[D / 8][4];
+    if (ok && mbar_wait(o_final, 0, p.err)) {
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) {
+        float ov[32];
+        tmem_ld_16x256b_x8(tmem_base + lane_base + C::kOCol + c * 64, ov);
+        tmem_ld_wait();
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) o[c * 8 + jj][e] = ov[4 * jj + e];
+      }
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        l_run[hh] += __shfl_xor_sync(0xffffffffu, l_run[hh], 1);
+        l_run[hh] += __shfl_xor_sync(0xffffffffu, l_run[hh], 2);
+      }
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int r = r0 + hh * 8;
+        if (r >= p.R) continue;
+        if (n_splits_b == 1) {
+          const int i = r / p.G, g = r - (r / p.G) * p.G;
+          f16* dst = p.o + (static_cast<size_t>(b * p.bs + i) * p.Hq + h * p.G + g) * D;
+          const float inv = 1.f / l_run[hh];
+#pragma unroll
+          for (int db = 0; db < D / 8; ++db) {
+            const int d = db * 8 + 2 * (lane & 3);
+            *reinterpret_cast<uint32_t*>(dst + d) =
+                pack_f16x2(o[db][2 * hh] * inv, o[db][2 * hh + 1] * inv);
+          }
+        } else {
+          const size_t prow = (static_cast<size_t>(split) * p.B + b) * p.Hkv + h;
+          float* dst = p.part_o + (prow * p.R + r) * D;
+#pragma unroll
+          for (int db = 0; db < D / 8; ++db) {
+            const int d = db * 8 + 2 * (lane & 3);
+            *reinterpret_cast<float2*>(dst + d) = make_float2(o[db][2 * hh], o[db][2 * hh + 1]);
+          }
+          if ((lane & 3) == 0) {
+            *reinterpret_cast<float2*>(p.part_ml + (prow * p.R + r) * 2) =
+                make_float2(m_ref[hh], l_run[hh]);
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+}  // namespace dflash

@@ -7,6 +7,7 @@
 
 #include <algorithm>
 #include <cmath>
+#include <cstdlib>
 #include <cstring>
 #include <map>
 #include <mutex>
@@ -15,6 +16,7 @@
 #include <vector>
 
 #include "attention.cuh"
+#include "attention_tc.cuh"
 #include "dflash.h"
 #include "gemm_tcgen05.cuh"
 #include "small_kernels.cuh"
@@ -74,8 +76,8 @@ bool make_tmap(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t cols,
 // ---------------------------------------------------------------------------
 struct GemmPlan {
   int BN = 0, m_tiles = 0, n_tiles = 0, k_blocks = 0, tiles = 0, stream_k = 0, ipc = 0,
-      total_iters = 0, nacc = 1, tmem_cols = 32, grid = 0, a_rows = 128, stages = 1, smem = 0,
-      slot_rows = 0;
+      total_iters = 0, nacc = 1, nbuf = 2, tmem_cols = 32, grid = 0, a_rows = 128, stages = 1,
+      smem = 0, slot_rows = 0;
   size_t partial_bytes = 0;
 };
 
@@ -89,28 +91,38 @@ int gemm_stages(int a_rows, int bn) {
   return st;
 }
 
-// Tile width, accumulator chains and schedule.  Small M (weight-streaming):
-// BN = 128 with two accumulator chains; M >= 256 (tensor-bound): BN = 256
-// with one.  Whole tiles are handed out round-robin when they fill the SMs
-// evenly (>= 90% of the last round busy); otherwise stream-K splits the
-// (tile, k-block) iterations evenly over the SMs.  force_bn / force_splits
-// (0 = automatic) pin the tile width and the schedule: 1 = whole tiles,
-// n >= 2 = stream-K with ceil(k_blocks / n) iterations per CTA.
+// Tile width, accumulator chains and schedule.  BN = 256.  One M tile (the
+// weight-streaming regime, M <= 128): two accumulator chains in a single TMEM
+// buffer, and stream-K (the (tile, k-block) iterations split evenly over the
+// SMs) unless whole tiles already fill >= 90% of the last round.  Several M
+// tiles (tensor-bound): one chain, double-buffered, whole tiles round-robin;
+// stream-K only when the tiles cannot occupy half of the SMs.  force_bn /
+// force_splits (0 = automatic) pin the tile width and the schedule: 1 = whole
+// tiles, n >= 2 = stream-K with ceil(k_blocks / n) iterations per CTA.
 GemmPlan plan_gemm(int M, int N, int K, int group, int num_sms, int force_bn = 0,
                    int force_splits = 0) {
   GemmPlan pl;
   pl.k_blocks = K / kGemmBK;
   pl.m_tiles = cdiv(M, kGemmBM);
-  pl.BN = force_bn ? force_bn : (M >= 2 * kGemmBM ? 256 : 128);
-  if (pl.BN < group || pl.BN % group) pl.BN = std::max(group, 128);
-  pl.nacc = pl.BN >= 256 ? 1 : pl.BN >= 128 ? 2 : 4;
+  pl.BN = force_bn ? force_bn : 256;
+  if (pl.BN < group || pl.BN % group) pl.BN = 256;
+  const bool one_m_tile = pl.m_tiles == 1;
+  if (one_m_tile) {
+    // the staged epilogue (M <= 32) frees the accumulator as soon as it is
+    // copied out, so one buffer suffices there
+    pl.nacc = pl.BN >= 256 ? 2 : 4;
+    pl.nbuf = (M > kGemmStagedRows && 2 * pl.nacc * pl.BN <= 512) ? 2 : 1;
+  } else {
+    pl.nacc = pl.BN >= 256 ? 1 : pl.BN >= 128 ? 2 : 4;
+    pl.nbuf = 2;
+  }
   pl.tmem_cols = 32;
-  while (pl.tmem_cols < 2 * pl.nacc * pl.BN) pl.tmem_cols *= 2;
+  while (pl.tmem_cols < pl.nbuf * pl.nacc * pl.BN) pl.tmem_cols *= 2;
   pl.n_tiles = cdiv(N, pl.BN);
   pl.tiles = pl.m_tiles * pl.n_tiles;
   const int rounds = cdiv(pl.tiles, num_sms);
   const double fill = static_cast<double>(pl.tiles) / (static_cast<double>(rounds) * num_sms);
-  bool sk = fill < 0.9;
+  bool sk = one_m_tile ? fill < 0.9 : 2 * pl.tiles < num_sms;
   if (force_splits == 1) sk = false;
   if (force_splits >= 2) sk = true;
   if (sk && pl.tiles > kCounterSlots) sk = false;
@@ -138,11 +150,19 @@ GemmPlan plan_gemm(int M, int N, int K, int group, int num_sms, int force_bn = 0
   return pl;
 }
 
+// Upper bound of GemmPlan::partial_bytes over every automatic plan with M
+// rows: stream-K never uses more CTAs than SMs, each CTA owns two slots of
+// min(M, 128) x 256 fp32.  Monotonic in M, so it also bounds smaller calls.
+size_t gemm_partial_bound(int M, int num_sms) {
+  return static_cast<size_t>(num_sms) * 2 * std::min(M, kGemmBM) * 256 * 4;
+}
+
 // ---------------------------------------------------------------------------
 // attention planning
 // ---------------------------------------------------------------------------
 struct AttnPlan {
   int chunk_keys = 0, max_splits = 0, R = 0, row_groups = 0, key_parts = 0, nwc = 0;
+  bool tc = false;   // tcgen05 kernel (kv groups of up to 64 query rows)
   size_t part_o_bytes = 0, part_ml_bytes = 0;
 };
 
@@ -150,12 +170,14 @@ AttnPlan plan_attention(int B, int Hkv, int W, int P, int bs, int G, int D, int 
   AttnPlan a;
   const int keys_max = W * P;
   const double est = static_cast<double>(B) * Hkv * keys_max;
+  a.R = bs * G;
+  a.tc = a.R <= kTcM;
+  const int tile = a.tc ? kTcKeys : kAttnTileKeys;
   int chunk = static_cast<int>(std::ceil(est / (4.0 * num_sms)));
-  chunk = (chunk + kAttnTileKeys - 1) / kAttnTileKeys * kAttnTileKeys;
+  chunk = (chunk + tile - 1) / tile * tile;
   chunk = std::max(128, std::min(8192, chunk));
   a.chunk_keys = chunk;
   a.max_splits = cdiv(keys_max, chunk);
-  a.R = bs * G;
   a.row_groups = cdiv(a.R, 16);
   a.key_parts = 1;
   while (a.key_parts < 4 && a.row_groups * a.key_parts * 2 <= kAttnMaxComputeWarps)
@@ -177,6 +199,16 @@ AttnPlan plan_attention(int B, int Hkv, int W, int P, int bs, int G, int D, int 
   } while (0)
 
 }  // namespace
+
+// Programmatic dependent launch unless the environment sets DFLASH_PDL=0
+// (read once per process).
+bool pdl_default() {
+  static const bool on = [] {
+    const char* e = std::getenv("DFLASH_PDL");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
 
 // ---------------------------------------------------------------------------
 // handle
@@ -204,6 +236,9 @@ struct dflash_handle {
   // launch accounting and optional per-launch event profiling (diagnostics)
   unsigned long long launches = 0;
   bool prof_on = false;
+  // hot-path kernels are launched with programmatic dependent launch (the
+  // environment variable DFLASH_PDL=0 turns it off)
+  bool pdl = pdl_default();
   std::vector<cudaEvent_t> prof_events;
   size_t prof_next = 0;
   std::vector<int> prof_kind;
@@ -262,6 +297,25 @@ struct LaunchScope {
   }
 };
 
+// Launch of a hot-path kernel; with `pdl` the launch may overlap the tail of
+// the previous kernel in the stream (every such kernel calls pdl_wait() before
+// it touches memory that an earlier kernel writes or a later one overwrites).
+template <typename... KArgs, typename... Args>
+void launch_k(bool pdl, void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+              cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 // ---------------------------------------------------------------------------
 // GEMM launch
 // ---------------------------------------------------------------------------
@@ -286,9 +340,10 @@ cudaError_t set_gemm_attrs_all() {
 }
 
 template <int BN, class Epi>
-void launch_gemm_bn(const CUtensorMap& ta, const CUtensorMap& tw, const GemmParams& gp,
-                    const Epi& epi, int grid, int smem, cudaStream_t st) {
-  gemm_tcgen05_kernel<BN, Epi><<<grid, kGemmThreads, smem, st>>>(ta, tw, gp, epi);
+void launch_gemm_bn(const dflash_handle* h, const CUtensorMap& ta, const CUtensorMap& tw,
+                    const GemmParams& gp, const Epi& epi, int grid, int smem, cudaStream_t st) {
+  launch_k(h->pdl, gemm_tcgen05_kernel<BN, Epi>, dim3(grid), dim3(kGemmThreads), smem, st, ta, tw, gp,
+           epi);
 }
 
 // D = A[M, K] * W[N, K]^T with epilogue `epi`.  `partials` must hold
@@ -321,6 +376,7 @@ dflash_status run_gemm(dflash_handle* h, int kind, bool f16, const void* A, int 
   gp.ipc = pl.ipc;
   gp.total_iters = pl.total_iters;
   gp.nacc = pl.nacc;
+  gp.nbuf = pl.nbuf;
   gp.tmem_cols = pl.tmem_cols;
   gp.a_rows = pl.a_rows;
   gp.stages = pl.stages;
@@ -332,16 +388,16 @@ dflash_status run_gemm(dflash_handle* h, int kind, bool f16, const void* A, int 
   LaunchScope scope(h, kind, st);
   switch (pl.BN) {
     case 256:
-      if constexpr (256 % Epi::kGroup == 0) launch_gemm_bn<256>(ta, tw, gp, epi, pl.grid, pl.smem, st);
+      if constexpr (256 % Epi::kGroup == 0) launch_gemm_bn<256>(h, ta, tw, gp, epi, pl.grid, pl.smem, st);
       break;
     case 128:
-      if constexpr (128 % Epi::kGroup == 0) launch_gemm_bn<128>(ta, tw, gp, epi, pl.grid, pl.smem, st);
+      if constexpr (128 % Epi::kGroup == 0) launch_gemm_bn<128>(h, ta, tw, gp, epi, pl.grid, pl.smem, st);
       break;
     case 64:
-      if constexpr (Epi::kGroup <= 64) launch_gemm_bn<64>(ta, tw, gp, epi, pl.grid, pl.smem, st);
+      if constexpr (Epi::kGroup <= 64) launch_gemm_bn<64>(h, ta, tw, gp, epi, pl.grid, pl.smem, st);
       break;
     case 32:
-      if constexpr (Epi::kGroup <= 32) launch_gemm_bn<32>(ta, tw, gp, epi, pl.grid, pl.smem, st);
+      if constexpr (Epi::kGroup <= 32) launch_gemm_bn<32>(h, ta, tw, gp, epi, pl.grid, pl.smem, st);
       break;
     default:
       return DFLASH_ERR_UNSUPPORTED_SHAPE;
@@ -362,8 +418,11 @@ cudaError_t set_attn_attrs() {
   if ((e = cudaFuncSetAttribute(attn_block_kernel<D, 32>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, bytes)) != cudaSuccess)
     return e;
-  return cudaFuncSetAttribute(attn_block_kernel<D, 16>,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if ((e = cudaFuncSetAttribute(attn_block_kernel<D, 16>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, bytes)) != cudaSuccess)
+    return e;
+  return cudaFuncSetAttribute(attn_block_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              TcAttnCfg<D>::kSmem);
 }
 
 template <int D>
@@ -380,19 +439,23 @@ dflash_status run_attention(dflash_handle* h, const AttnPlan& ap, AttnParams prm
   const int smem = AttnCfg<D>::smem_bytes(ap.nwc);
   prm.row_groups = ap.row_groups;
   prm.key_parts = ap.key_parts;
-  {
+  if (ap.tc) {
+    LaunchScope scope(h, DFLASH_KERNEL_ATTENTION, st);
+    launch_k(h->pdl, attn_block_tc_kernel<D>, grid, dim3(kTcThreads), TcAttnCfg<D>::kSmem, st, tk, tv,
+             prm);
+  } else {
     LaunchScope scope(h, DFLASH_KERNEL_ATTENTION, st);
     if (ap.key_parts == 1)
-      attn_block_kernel<D, 64><<<grid, threads, smem, st>>>(tk, tv, prm);
+      launch_k(h->pdl, attn_block_kernel<D, 64>, grid, dim3(threads), smem, st, tk, tv, prm);
     else if (ap.key_parts == 2)
-      attn_block_kernel<D, 32><<<grid, threads, smem, st>>>(tk, tv, prm);
+      launch_k(h->pdl, attn_block_kernel<D, 32>, grid, dim3(threads), smem, st, tk, tv, prm);
     else
-      attn_block_kernel<D, 16><<<grid, threads, smem, st>>>(tk, tv, prm);
+      launch_k(h->pdl, attn_block_kernel<D, 16>, grid, dim3(threads), smem, st, tk, tv, prm);
   }
   if (ap.max_splits > 1) {
     LaunchScope scope(h, DFLASH_KERNEL_ATTN_COMBINE, st);
     const int rows = prm.B * c.n_kv_heads * prm.R;
-    attn_combine_kernel<D><<<cdiv(rows, 8), 256, 0, st>>>(prm);
+    launch_k(h->pdl, attn_combine_kernel<D>, dim3(cdiv(rows, 8)), dim3(256), 0, st, prm);
   }
   return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ERR_CUDA;
 }
@@ -411,15 +474,7 @@ InjectWs inject_layout(const dflash_handle* h, int n) {
   off += align_up(static_cast<size_t>(n) * c.hidden * 4);
   w.ctx = off;
   off += align_up(static_cast<size_t>(n) * c.hidden * 2);
-  size_t cap = 0;
-  for (int m = 1; m <= n; m = (m < 256 ? m + 1 : m * 2)) {
-    const int mm = std::min(m, n);
-    cap = std::max(cap, plan_gemm(mm, c.hidden, c.n_target_layers * c.hidden, 32, h->num_sms)
-                            .partial_bytes);
-    cap = std::max(cap, plan_gemm(mm, c.n_layers * 2 * c.n_kv_heads * c.head_dim, c.hidden,
-                                  c.head_dim, h->num_sms)
-                            .partial_bytes);
-  }
+  const size_t cap = gemm_partial_bound(n, h->num_sms);
   w.partial = off;
   w.partial_cap = cap;
   off += align_up(cap);
@@ -432,16 +487,7 @@ struct ProposeWs {
          partial = 0, total = 0, partial_cap = 0, part_o_cap = 0, part_ml_cap = 0;
 };
 size_t propose_partial_need(const dflash_handle* h, int B) {
-  const dflash_config& c = h->cfg;
-  const int M = B * c.block_size, MK = B * (c.block_size - 1);
-  const int D = c.head_dim, Hq = c.n_q_heads, Hkv = c.n_kv_heads, H = c.hidden;
-  size_t cap = 0;
-  cap = std::max(cap, plan_gemm(M, (Hq + 2 * Hkv) * D, H, D, h->num_sms).partial_bytes);
-  cap = std::max(cap, plan_gemm(M, H, Hq * D, 32, h->num_sms).partial_bytes);
-  cap = std::max(cap, plan_gemm(M, 2 * c.intermediate, H, 32, h->num_sms).partial_bytes);
-  cap = std::max(cap, plan_gemm(M, H, c.intermediate, 32, h->num_sms).partial_bytes);
-  cap = std::max(cap, plan_gemm(MK, c.vocab, H, 32, h->num_sms).partial_bytes);
-  return cap;
+  return gemm_partial_bound(B * h->cfg.block_size, h->num_sms);
 }
 ProposeWs propose_layout(const dflash_handle* h, int B, int W) {
   const dflash_config& c = h->cfg;
@@ -462,13 +508,13 @@ ProposeWs propose_layout(const dflash_handle* h, int B, int W) {
   w.frows = take(static_cast<size_t>(MK) * H * 2);
   w.keys = take(static_cast<size_t>(MK) * 8);
   size_t po = 0, pm = 0, pc = 0;
-  for (int b = 1; b <= B; b = (b < 256 ? b + 1 : b * 2)) {
-    const int bb = std::min(b, B);
+  // the attention split plan is not monotonic in the batch: cover every size
+  for (int bb = 1; bb <= B; ++bb) {
     const AttnPlan ap = plan_attention(bb, Hkv, W, c.page_size, bs, Hq / Hkv, D, h->num_sms);
     po = std::max(po, ap.part_o_bytes);
     pm = std::max(pm, ap.part_ml_bytes);
-    pc = std::max(pc, propose_partial_need(h, bb));
   }
+  pc = propose_partial_need(h, B);
   w.part_o = take(po);
   w.part_ml = take(pm);
   w.part_o_cap = po;
@@ -614,7 +660,8 @@ dflash_status propose_layers(dflash_handle* h, const ProposeWs& lw, void* ws,
     if (s != DFLASH_OK) return s;
     {
       LaunchScope scope(h, DFLASH_KERNEL_RMSNORM, st);
-      rmsnorm_rows_kernel<<<M, 256, 0, st>>>(x, h->post_norm_w[l], nrm, H, c.rms_eps, 0, bs);
+      launch_k(h->pdl, rmsnorm_rows_kernel, dim3(M), dim3(256), 0, st, x, h->post_norm_w[l], nrm, H,
+               c.rms_eps, 0, bs);
     }
     if (cudaGetLastError() != cudaSuccess) return DFLASH_ERR_CUDA;
     // h = silu(gate) * up
@@ -628,11 +675,12 @@ dflash_status propose_layers(dflash_handle* h, const ProposeWs& lw, void* ws,
     if (s != DFLASH_OK) return s;
     LaunchScope scope(h, DFLASH_KERNEL_RMSNORM, st);
     if (l + 1 < c.n_layers) {
-      rmsnorm_rows_kernel<<<M, 256, 0, st>>>(x, h->in_norm_w[l + 1], nrm, H, c.rms_eps, 0, bs);
+      launch_k(h->pdl, rmsnorm_rows_kernel, dim3(M), dim3(256), 0, st, x, h->in_norm_w[l + 1], nrm,
+               H, c.rms_eps, 0, bs);
     } else {
       // final norm on the kept rows (block slots 1..bs-1) only
-      rmsnorm_rows_kernel<<<B * K, 256, 0, st>>>(x, h->final_norm_w, frows, H, c.rms_eps, K,
-                                                 bs);
+      launch_k(h->pdl, rmsnorm_rows_kernel, dim3(B * K), dim3(256), 0, st, x, h->final_norm_w,
+               frows, H, c.rms_eps, K, bs);
     }
     if (cudaGetLastError() != cudaSuccess) return DFLASH_ERR_CUDA;
   }
@@ -872,8 +920,9 @@ dflash_status dflash_paged_slots(const int64_t* positions, const int64_t* req_id
   if (!positions || !req_ids || !block_table || !slots) return DFLASH_ERR_INVALID_ARG;
   dflash_status s = set_device_for(static_cast<cudaStream_t>(stream), slots);
   if (s != DFLASH_OK) return s;
-  paged_slots_kernel<<<cdiv(n, 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      positions, req_ids, block_table, n, max_pages_per_seq, page_size, slots);
+  launch_k(pdl_default(), paged_slots_kernel, dim3(cdiv(n, 256)), dim3(256), 0,
+           static_cast<cudaStream_t>(stream), positions, req_ids, block_table, n,
+           max_pages_per_seq, page_size, slots);
   return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ERR_CUDA;
 }
 
@@ -907,7 +956,8 @@ dflash_status dflash_inject_context(dflash_handle* h, const void* aux, const int
   // (2) hidden_norm
   {
     LaunchScope scope(h, DFLASH_KERNEL_RMSNORM, st);
-    rmsnorm_rows_kernel<<<n, 256, 0, st>>>(fcx, h->hidden_norm_w, ctx, H, c.rms_eps, 0, 0);
+    launch_k(h->pdl, rmsnorm_rows_kernel, dim3(n), dim3(256), 0, st, fcx, h->hidden_norm_w, ctx, H,
+             c.rms_eps, 0, 0);
   }
   if (cudaGetLastError() != cudaSuccess) return DFLASH_ERR_CUDA;
   // (3) every layer's K/V at once, k_norm + RoPE, paged scatter
@@ -982,9 +1032,9 @@ dflash_status dflash_propose(dflash_handle* h, const int32_t* bonus_tokens,
 
   {
     LaunchScope scope(h, DFLASH_KERNEL_EMBED_NORM, st);
-    embed_norm_kernel<<<M, 256, 0, st>>>(bonus_tokens, c.mask_token_id, h->embed,
-                                         h->in_norm_w[0], x, nrm, keys, B * K, bs, H, c.vocab,
-                                         c.rms_eps, h->dev_err);
+    launch_k(h->pdl, embed_norm_kernel, dim3(M), dim3(256), 0, st, bonus_tokens, c.mask_token_id,
+             h->embed, h->in_norm_w[0], x, nrm, keys, B * K, bs, H, c.vocab, c.rms_eps,
+             h->dev_err);
   }
   if (cudaGetLastError() != cudaSuccess) return DFLASH_ERR_CUDA;
   dflash_status s = (c.head_dim == 128)
@@ -1000,8 +1050,8 @@ dflash_status dflash_propose(dflash_handle* h, const int32_t* bonus_tokens,
   if (s != DFLASH_OK) return s;
   {
     LaunchScope scope(h, DFLASH_KERNEL_ARGMAX_FINALIZE, st);
-    argmax_finalize_kernel<<<cdiv(M, 256), 256, 0, st>>>(keys, bonus_tokens, draft_tokens,
-                                                         block_tokens, B, bs);
+    launch_k(h->pdl, argmax_finalize_kernel, dim3(cdiv(M, 256)), dim3(256), 0, st, keys,
+             bonus_tokens, draft_tokens, block_tokens, B, bs);
   }
   return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ERR_CUDA;
 }
@@ -1023,11 +1073,10 @@ dflash_status dflash_verify_greedy(const int32_t* drafts, const float* target_lo
   dflash_status s = set_device_for(st, out_tokens);
   if (s != DFLASH_OK) return s;
   unsigned long long* part = static_cast<unsigned long long*>(workspace);
-  verify_partial_kernel<<<dim3(vp.chunks, B * (K + 1)), 256, 0, st>>>(target_logits, V,
-                                                                      vp.chunk_len, vp.chunks,
-                                                                      part);
-  verify_final_kernel<<<B, 256, 0, st>>>(part, vp.chunks, drafts, K, out_tokens, num_accepted,
-                                        bonus);
+  launch_k(pdl_default(), verify_partial_kernel, dim3(vp.chunks, B * (K + 1)), dim3(256), 0, st,
+           target_logits, V, vp.chunk_len, vp.chunks, part);
+  launch_k(pdl_default(), verify_final_kernel, dim3(B), dim3(256), 0, st, part, vp.chunks, drafts,
+           K, out_tokens, num_accepted, bonus);
   return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ERR_CUDA;
 }
 
@@ -1276,10 +1325,9 @@ extern "C" dflash_status dflash_verify_greedy_noalloc(const int32_t* drafts,
   if (s != DFLASH_OK) return s;
   // Nothing in the scratch has to start at zero: the second kernel reads only
   // the keys the first one writes in this same call.
-  verify_partial_kernel<<<dim3(vp.chunks, B * (K + 1)), 256, 0, st>>>(target_logits, V,
-                                                                      vp.chunk_len, vp.chunks,
-                                                                      part);
-  verify_final_kernel<<<B, 256, 0, st>>>(part, vp.chunks, drafts, K, out_tokens, num_accepted,
-                                        bonus);
+  launch_k(pdl_default(), verify_partial_kernel, dim3(vp.chunks, B * (K + 1)), dim3(256), 0, st,
+           target_logits, V, vp.chunk_len, vp.chunks, part);
+  launch_k(pdl_default(), verify_final_kernel, dim3(B), dim3(256), 0, st, part, vp.chunks, drafts,
+           K, out_tokens, num_accepted, bonus);
   return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ERR_CUDA;
 }

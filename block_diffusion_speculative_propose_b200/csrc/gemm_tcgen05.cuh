@@ -36,6 +36,8 @@ constexpr int kGemmThreads = 192;
 constexpr int kGemmSmemLimit = 232448;  // max dynamic shared memory per block on sm_100
 
 constexpr int kGemmMaxStages = 32;
+// full/empty per stage, tfull/tempty per accumulator, then 4 words: TMEM base,
+// last-arriver flag and the two epilogue wait verdicts
 constexpr int kGemmBarrierBytes = 2 * kGemmMaxStages * 8 + 4 * 8 + 16;
 
 template <int BN>
@@ -44,13 +46,29 @@ struct GemmCfg {
   static_assert(BN % 16 == 0 && BN >= 32 && BN <= 256, "UMMA N for M=128");
 };
 
+// Tiles of at most this many rows (M <= 32) take the staged epilogue: one warp
+// copies the accumulator from tensor memory into a shared-memory tile, then all
+// 128 epilogue threads run the stream-K fixup and the epilogue functor over it,
+// so that a handful of rows does not leave 3/4 of the threads idle and the
+// rest walking the tile with one dependent global round trip per step.
+constexpr int kGemmStagedRows = 32;
+
+__host__ __device__ inline bool gemm_staged(int a_rows) { return a_rows <= kGemmStagedRows; }
+
+// fp32 staging tile [a_rows][bn + 4] (the pad spreads rows over the banks)
+__host__ __device__ inline int gemm_staging_bytes(int a_rows, int bn) {
+  return gemm_staged(a_rows) ? a_rows * (bn + 4) * 4 : 0;
+}
+
 // Shared memory of one launch: [a_rows x 128 B A slots][BN x 128 B W slots]
-// [barriers].  With fewer than 128 rows of A (a_rows < 128) the MMA still
-// reads a full 128-row A operand; the rows past a_rows alias the following
-// slots, which only feeds accumulator rows that the epilogue never stores.
+// [barriers][staging tile].  With fewer than 128 rows of A (a_rows < 128) the
+// MMA still reads a full 128-row A operand; the rows past a_rows alias the
+// following slots, which only feeds accumulator rows that the epilogue never
+// stores.
 __host__ __device__ inline int gemm_smem_bytes(int a_rows, int bn, int stages) {
   const int tail = kGemmBM * 128 - a_rows * 128 - stages * bn * 128;  // keep A overreads inside
-  return 1024 + stages * (a_rows + bn) * 128 + kGemmBarrierBytes + (tail > 0 ? tail : 0);
+  return 1024 + stages * (a_rows + bn) * 128 + kGemmBarrierBytes +
+         gemm_staging_bytes(a_rows, bn) + (tail > 0 ? tail : 0);
 }
 
 struct GemmParams {
@@ -61,7 +79,8 @@ struct GemmParams {
   int ipc;             // stream-K: k-block iterations per CTA
   int total_iters;     // stream-K: tiles * k_blocks
   int nacc;            // independent accumulator chains per tile (1, 2 or 4)
-  int tmem_cols;       // allocated TMEM columns (>= 2 * nacc * BN, power of two)
+  int nbuf;            // accumulator buffers (2: next tile accumulates during the epilogue)
+  int tmem_cols;       // allocated TMEM columns (>= nbuf * nacc * BN, power of two)
   int a_rows;          // rows of the A box / slot (128, or M rounded up to 16 when M < 128)
   int stages;          // pipeline depth (<= kGemmMaxStages)
   int f16;             // operands are fp16 (1) or bf16 (0)
@@ -162,9 +181,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* tempty = tfull + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
   volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  // [2]: verdict of the elected epilogue wait, alternating by segment (a
+  // thread can be at most one segment ahead of the slowest reader)
+  volatile int* wait_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
+  float* staging = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(full) + kGemmBarrierBytes);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  pdl_trigger();
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) {
@@ -194,21 +218,40 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (lane == 0) {
       const uint64_t pol_w = policy_evict_first();
       const uint64_t pol_a = policy_evict_last();
+      // The weights are never written by an earlier kernel: the W tiles of the
+      // first `stages` k-blocks are requested before waiting for the grid that
+      // produces A (the fresh stages need no empty-slot wait).
+      int pre = 0;
+      {
+        GemmSegIter it0(p);
+        GemmSeg s0;
+        while (pre < stages && it0.next(p, s0)) {
+          for (int kb = s0.kb0; kb < s0.kb1 && pre < stages; ++kb, ++pre) {
+            mbar_arrive_expect_tx(&full[pre], stage_tx);
+            tma_load_2d_hint(sB + pre * C::kBBytes, &tmW, &full[pre], kb * kGemmBK,
+                             s0.n_tile * BN, pol_w);
+          }
+        }
+      }
+      pdl_wait();
       uint32_t stage = 0, phase = 0;
+      int idx = 0;
       bool ok = true;
       GemmSegIter it(p);
       GemmSeg sg;
       while (ok && it.next(p, sg)) {
-        for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, p.err)) {
-            ok = false;
-            break;
+        for (int kb = sg.kb0; kb < sg.kb1; ++kb, ++idx) {
+          if (idx >= pre) {
+            if (!mbar_wait(&empty[stage], phase ^ 1u, p.err)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&full[stage], stage_tx);
+            tma_load_2d_hint(sB + stage * C::kBBytes, &tmW, &full[stage], kb * kGemmBK,
+                             sg.n_tile * BN, pol_w);
           }
-          mbar_arrive_expect_tx(&full[stage], stage_tx);
           tma_load_2d_hint(sA + stage * a_bytes, &tmA, &full[stage], kb * kGemmBK,
                            sg.m_tile * kGemmBM, pol_a);
-          tma_load_2d_hint(sB + stage * C::kBBytes, &tmW, &full[stage], kb * kGemmBK,
-                           sg.n_tile * BN, pol_w);
           if (++stage == static_cast<uint32_t>(stages)) {
             stage = 0;
             phase ^= 1u;
@@ -253,20 +296,149 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         if (!ok) break;
         umma_commit(&tfull[acc]);
-        acc ^= 1u;
-        if (acc == 0) acc_phase ^= 1u;
+        if (++acc == static_cast<uint32_t>(p.nbuf)) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
       }
     }
-  } else {
-    // ------------------------------------------------------------ epilogue
-    const int ew = warp - 2;        // 0..3
-    const int sp = warp & 3;        // TMEM sub-partition this warp may read
-    const int row = sp * 32 + lane;
-    uint32_t acc = 0, acc_phase = 0;
+  } else if (gemm_staged(p.a_rows)) {
+    // ------------------------------------------------------------ staged epilogue
+    pdl_wait();
+    constexpr int LD = BN + 4;
+    constexpr int F4 = BN / 4;             // float4 per row
+    const int tid = threadIdx.x - 64;      // 0..127
+    const int sp = warp & 3;
+    uint32_t acc = 0, acc_phase = 0, nseen = 0;
     GemmSegIter it(p);
     GemmSeg sg;
     while (it.next(p, sg)) {
-      if (!mbar_wait(&tfull[acc], acc_phase, p.err)) break;
+      // one thread waits (bounded) and the verdict is shared, so that the
+      // named barriers below are always reached by all 128 threads or none
+      if (tid == 0) wait_flag[nseen & 1] = mbar_wait(&tfull[acc], acc_phase, p.err) ? 1 : 0;
+      named_bar_sync(1, 128);
+      if (!wait_flag[nseen++ & 1]) break;
+      tc_fence_after();
+      if (sp == 0) {
+        // rows 0..31 live in TMEM lanes 0..31: the sub-partition-0 warp reads
+        // them (the load is warp-wide), one row per lane, and the lanes below
+        // a_rows park theirs in the staging tile, which holds a_rows rows
+        const uint32_t taddr = tmem_base + acc * acc_cols;
+        const bool keep = lane < p.a_rows;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          float v[32];
+          tmem_load_sum32<BN>(taddr + c * 32, p.nacc, v);
+          float* dst = staging + lane * LD + c * 32;
+          if (keep) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 4)
+              *reinterpret_cast<float4*>(dst + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (++acc == static_cast<uint32_t>(p.nbuf)) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+      named_bar_sync(1, 128);
+      const int rows = p.M;                // one M tile: M <= a_rows <= 32
+      const int nf4 = rows * F4;
+      if (sg.nseg > 1) {
+        float* part = p.partials + static_cast<size_t>(sg.slot) * p.slot_rows * BN;
+        for (int i = tid; i < nf4; i += 128) {
+          const int r = i / F4, c4 = i - r * F4;
+          __stcg(reinterpret_cast<float4*>(part) + i,
+                 *reinterpret_cast<const float4*>(staging + r * LD + c4 * 4));
+        }
+        __threadfence();
+        named_bar_sync(1, 128);
+        if (tid == 0) {
+          const unsigned prev = atomicAdd(&p.counters[sg.tile], 1u);
+          const int last = (prev == static_cast<unsigned>(sg.nseg - 1)) ? 1 : 0;
+          if (last) p.counters[sg.tile] = 0u;
+          *last_flag = last;
+        }
+        named_bar_sync(1, 128);
+        if (!*last_flag) {
+          named_bar_sync(1, 128);  // last_flag and staging are rewritten by the next segment
+          continue;
+        }
+        __threadfence();
+        // sum the pieces in CTA order; up to 8 float4 per thread in flight per piece
+        for (int i0 = tid; i0 < nf4; i0 += 128 * 8) {
+          float4 sum[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) sum[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 1
+          for (int c = sg.first_cta; c < sg.first_cta + sg.nseg; ++c) {
+            const float4* src = reinterpret_cast<const float4*>(
+                p.partials + static_cast<size_t>(gemm_slot_of(p, sg.tile, c)) * p.slot_rows * BN);
+            float4 q[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const int i = i0 + u * 128;
+              q[u] = i < nf4 ? __ldcg(src + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              sum[u].x += q[u].x;
+              sum[u].y += q[u].y;
+              sum[u].z += q[u].z;
+              sum[u].w += q[u].w;
+            }
+          }
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int i = i0 + u * 128;
+            if (i < nf4) {
+              const int r = i / F4, c4 = i - r * F4;
+              *reinterpret_cast<float4*>(staging + r * LD + c4 * 4) = sum[u];
+            }
+          }
+        }
+        named_bar_sync(1, 128);
+      }
+      // epilogue items (row, group of G columns); adjacent threads take adjacent
+      // rows of one group, which keeps the staging reads free of bank conflicts
+      constexpr int NG = BN / G;
+      for (int item = tid; item < rows * NG; item += 128) {
+        const int g = item / rows, r = item - g * rows;
+        const int n0 = sg.n_tile * BN + g * G;
+        if (n0 >= p.N) continue;
+        float v[G];
+        const float* src = staging + r * LD + g * G;
+#pragma unroll
+        for (int j = 0; j < G; j += 4) {
+          const float4 q = *reinterpret_cast<const float4*>(src + j);
+          v[j] = q.x;
+          v[j + 1] = q.y;
+          v[j + 2] = q.z;
+          v[j + 3] = q.w;
+        }
+        typename Epi::State st;
+        epi.begin(st);
+        epi.apply(st, r, n0, min(G, p.N - n0), v);
+        epi.end(st, r, true);
+      }
+      named_bar_sync(1, 128);  // staging and last_flag are rewritten by the next segment
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    pdl_wait();
+    const int ew = warp - 2;        // 0..3
+    const int sp = warp & 3;        // TMEM sub-partition this warp may read
+    const int row = sp * 32 + lane;
+    uint32_t acc = 0, acc_phase = 0, nseen = 0;
+    GemmSegIter it(p);
+    GemmSeg sg;
+    while (it.next(p, sg)) {
+      if (ew == 0 && lane == 0) wait_flag[nseen & 1] = mbar_wait(&tfull[acc], acc_phase, p.err) ? 1 : 0;
+      named_bar_sync(1, 128);
+      if (!wait_flag[nseen++ & 1]) break;
       tc_fence_after();
       const int m = sg.m_tile * kGemmBM + row;
       const bool row_ok = m < p.M;
@@ -345,8 +517,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         named_bar_sync(1, 128);  // last_flag is rewritten by the next segment
       }
-      acc ^= 1u;
-      if (acc == 0) acc_phase ^= 1u;
+      if (++acc == static_cast<uint32_t>(p.nbuf)) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
     }
   }
 

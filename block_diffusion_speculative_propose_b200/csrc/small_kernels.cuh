@@ -41,6 +41,8 @@ __global__ void __launch_bounds__(256) embed_norm_kernel(
     const bf16* __restrict__ w, float* __restrict__ x, f16* __restrict__ nrm,
     unsigned long long* __restrict__ keys, int n_keys, int bs, int H, int V, float eps,
     unsigned* err) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float red[32];
   const int r = blockIdx.x;
   const int b = r / bs, i = r - (r / bs) * bs;
@@ -90,6 +92,8 @@ __global__ void __launch_bounds__(256) embed_norm_kernel(
 __global__ void __launch_bounds__(256) rmsnorm_rows_kernel(
     const float* __restrict__ x, const bf16* __restrict__ w, f16* __restrict__ out, int H,
     float eps, int gather_k, int bs) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float red[32];
   const int r = blockIdx.x;
   const int src = gather_k > 0 ? (r / gather_k) * bs + 1 + (r - (r / gather_k) * gather_k) : r;
@@ -123,6 +127,8 @@ __global__ void argmax_finalize_kernel(const unsigned long long* __restrict__ ke
                                        const int32_t* __restrict__ bonus,
                                        int32_t* __restrict__ drafts,
                                        int32_t* __restrict__ block, int B, int bs) {
+  pdl_trigger();
+  pdl_wait();
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= B * bs) return;
   const int K = bs - 1;
@@ -142,6 +148,8 @@ __global__ void argmax_finalize_kernel(const unsigned long long* __restrict__ ke
 __global__ void __launch_bounds__(256) verify_partial_kernel(
     const float* __restrict__ logits, int V, int chunk_len, int chunks,
     unsigned long long* __restrict__ part) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ unsigned long long red[32];
   const size_t row = blockIdx.y;
   const int beg = blockIdx.x * chunk_len;
@@ -184,6 +192,8 @@ __global__ void __launch_bounds__(256) verify_final_kernel(
     const unsigned long long* __restrict__ part, int chunks,
     const int32_t* __restrict__ drafts, int K, int32_t* __restrict__ out,
     int32_t* __restrict__ n_acc, int32_t* __restrict__ bonus) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ int32_t t[130];
   __shared__ int32_t d[130];
   __shared__ int n_sh;
@@ -220,6 +230,8 @@ __global__ void paged_slots_kernel(const int64_t* __restrict__ pos,
                                    const int64_t* __restrict__ req,
                                    const int32_t* __restrict__ table, int n, int W, int P,
                                    int64_t* __restrict__ slots) {
+  pdl_trigger();
+  pdl_wait();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= n) return;
   const int64_t p = pos[i];

@@ -18,7 +18,7 @@ import oracle as O
 from block_diffusion_speculative_propose_b200 import (DFlash, paged_slots, synth,
                                                       verify_greedy)
 from tests._util import rel_l2, to_np, weights_np, weights_to
-from tests.test_gpu_propose import compare_drafts
+from tests.test_gpu_propose import compare_drafts, max_excluded
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
@@ -119,7 +119,7 @@ def test_full_step_at_bench_size(workload, samples):
             O.inject_context(oc, Wn, aux, pos, local_slots, ko, vo, mode)
             res[mode] = O.propose(oc, Wn, to_np(sb.bonus)[pick], seq[pick], table, ko, vo, mode)
         excluded = compare_drafts(gpu_drafts, gpu_logits, res["device"], res["exact"], K)
-        assert excluded <= max(2, len(pick) * K // 10)
+        assert excluded <= max_excluded(len(pick) * K)
     finally:
         h.close()
         gc.collect()

@@ -44,6 +44,12 @@ GEMM_CASES = [
     (15, 4096, 1024, 256, 1),
     (16, 1024, 4096, 128, 4),
     (16, 1024, 4096, 32, 3),
+    # staged epilogue (M <= 32): boundary rows, ragged N, many pieces per tile
+    (32, 2048, 2048, 0, 0),
+    (33, 2048, 2048, 0, 0),
+    (7, 1056, 640, 0, 0),
+    (17, 4096, 2048, 64, 5),
+    (1, 4096, 4096, 0, 0),
     (129, 96, 192, 32, 1),
     (129, 96, 192, 32, 3),
     (300, 1536, 512, 0, 0),
@@ -134,9 +140,14 @@ def _attention_case(cfg, seq_lens, seed):
     ("qwen3_8b", [2048]),
     ("qwen3_8b", [0, 7, 100, 1000, 5000]),
     ("llama31_8b", [3, 333, 4097]),
+    # 8 query heads per kv head: 128 rows per kv group (the mma.sync kernel)
+    ("qwen3_8b_g8", [0, 77, 3000]),
 ])
 def test_block_attention_matches_oracle(model, seq_lens):
-    cfg = synth.model_config(model)
+    if model == "qwen3_8b_g8":
+        cfg = dict(synth.model_config("qwen3_8b"), n_kv_heads=4)
+    else:
+        cfg = synth.model_config(model)
     # the attention entry point needs only geometry: a handle with tiny weights
     # of the same head layout
     small = dict(cfg, intermediate=256, vocab=1024, n_layers=1, mask_token_id=1023,
@@ -150,9 +161,15 @@ def test_block_attention_matches_oracle(model, seq_lens):
         torch.cuda.synchronize()
         got = to_np(o).astype(np.float64).reshape(ref.shape)
         assert np.isfinite(got).all()
+        # bf16 inputs are exact in the oracle; what remains is the fp32
+        # accumulation, P carried as bf16 hi + lo (about 2^-16 relative) and
+        # the fp16 output (2^-11 relative per element, ~3e-4 rel-L2)
+        errs = []
         for b in range(len(seq_lens)):
             rows = slice(b * cfg["block_size"], (b + 1) * cfg["block_size"])
-            assert rel_l2(got[rows], ref[rows]) < 8e-3, (b, seq_lens[b])
+            errs.append(rel_l2(got[rows], ref[rows]))
+        print(f"attention rel-L2 per request: {['%.2e' % e for e in errs]}")
+        assert max(errs) < 1e-3, errs
         assert h.check_device_errors() == 0
     finally:
         h.close()
