@@ -101,7 +101,7 @@ __global__ void __launch_bounds__(32 * (kAttnMaxComputeWarps + 1), 1)
     }
     fence_barrier_init();
   }
-  __syncthreads();
+  cta_sync();
 
   const int n_tiles = (k1 - k0 + kAttnTileKeys - 1) / kAttnTileKeys;
 

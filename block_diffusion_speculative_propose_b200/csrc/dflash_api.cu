@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <array>
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
@@ -75,7 +76,7 @@ bool make_tmap(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t cols,
 // GEMM planning
 // ---------------------------------------------------------------------------
 struct GemmPlan {
-  int BN = 0, m_tiles = 0, n_tiles = 0, k_blocks = 0, tiles = 0, stream_k = 0, ipc = 0,
+  int BN = 0, m_tiles = 0, n_tiles = 0, k_blocks = 0, tiles = 0, stream_k = 0, cluster_s = 1, ipc = 0,
       total_iters = 0, nacc = 1, nbuf = 2, tmem_cols = 32, grid = 0, a_rows = 128, stages = 1,
       smem = 0, slot_rows = 0;
   size_t partial_bytes = 0;
@@ -99,8 +100,14 @@ int gemm_stages(int a_rows, int bn) {
 // stream-K only when the tiles cannot occupy half of the SMs.  force_bn /
 // force_splits (0 = automatic) pin the tile width and the schedule: 1 = whole
 // tiles, n >= 2 = stream-K with ceil(k_blocks / n) iterations per CTA.
+//
+// Few rows (the staged epilogue, M <= 32) and fewer tiles than SMs: cluster
+// split-K with the largest cluster size S <= 8 (and <= the k-blocks) for which
+// every tile's cluster is resident at once (cluster_cap[S] = clusters of S CTAs
+// that fit on the GPU, 0 = unknown); with no such S, whole tiles when they
+// occupy at least half of the SMs, else stream-K.
 GemmPlan plan_gemm(int M, int N, int K, int group, int num_sms, int force_bn = 0,
-                   int force_splits = 0) {
+                   int force_splits = 0, const int* cluster_cap = nullptr) {
   GemmPlan pl;
   pl.k_blocks = K / kGemmBK;
   pl.m_tiles = cdiv(M, kGemmBM);
@@ -127,6 +134,24 @@ GemmPlan plan_gemm(int M, int N, int K, int group, int num_sms, int force_bn = 0
   if (force_splits >= 2) sk = true;
   if (sk && pl.tiles > kCounterSlots) sk = false;
   pl.total_iters = pl.tiles * pl.k_blocks;
+  pl.a_rows = gemm_a_rows(M);
+  if (!force_splits && cluster_cap && gemm_staged(pl.a_rows) && pl.tiles <= num_sms) {
+    int best = 1;
+    for (int S = 2; S <= std::min(8, pl.k_blocks); ++S)
+      if (cluster_cap[S] >= pl.tiles && pl.tiles * S <= num_sms) best = S;
+    if (best > 1) {
+      pl.cluster_s = best;
+      pl.stream_k = 0;
+      pl.ipc = cdiv(pl.k_blocks, best);
+      pl.grid = pl.tiles * best;
+      pl.slot_rows = std::min(M, kGemmBM);
+      pl.partial_bytes = 0;
+      pl.stages = gemm_stages(pl.a_rows, pl.BN);
+      pl.smem = gemm_smem_bytes(pl.a_rows, pl.BN, pl.stages);
+      return pl;
+    }
+    if (2 * pl.tiles >= num_sms) sk = false;
+  }
   if (sk) {
     pl.stream_k = 1;
     if (force_splits >= 2) {
@@ -218,21 +243,24 @@ struct dflash_handle {
   std::vector<int> target_layer_ids;
   int device = 0;
   int num_sms = 148;
-  // aliased caller weights
-  const bf16 *fc_w = nullptr, *hidden_norm_w = nullptr, *embed = nullptr, *lm_head = nullptr,
-             *final_norm_w = nullptr;
-  std::vector<const bf16*> in_norm_w, post_norm_w, q_norm_w, k_norm_w, w_down;
-  // copies owned by the handle; the ones multiplied against fp16 operands are
-  // held as fp16 (bf16 -> fp16 is exact in fp16's normal range)
-  std::vector<f16*> wqkv, wgu, wo;
-  f16* wkv = nullptr;       // [L * 2 * Hkv * D, H]
-  f16* lm_head16 = nullptr; // [V, H]
+  // aliased caller weights (embedding table and norm weights)
+  const bf16 *hidden_norm_w = nullptr, *embed = nullptr, *final_norm_w = nullptr;
+  std::vector<const bf16*> in_norm_w, post_norm_w, q_norm_w, k_norm_w;
+  // GEMM weights: copies owned by the handle, in the tile-contiguous layout of
+  // pack_tiles_kernel; the ones multiplied against fp16 operands are held as
+  // fp16 (bf16 -> fp16 is exact in fp16's normal range)
+  std::vector<f16*> wqkv, wgu, wo;  // [Wq; Wk; Wv], gate/up interleaved by 16 rows, Wo
+  std::vector<bf16*> wdown;         // W_down (bf16: multiplied against the bf16 MLP hidden)
+  bf16* fcw = nullptr;              // fc (bf16: multiplied against the bf16 target states)
+  f16* wkv = nullptr;               // all layers' [Wk; Wv], [L * 2 * Hkv * D, H]
+  f16* lm_head16 = nullptr;         // [V, H]
   bf16* knorm_all = nullptr;  // [L, D]
   float2* rope = nullptr;   // [max_position, D/2]
   unsigned* dev_err = nullptr;
   unsigned* counters = nullptr;
   std::mutex mu;
   std::map<std::tuple<const void*, uint64_t, uint64_t, uint32_t, bool>, CUtensorMap> tmaps;
+  std::map<std::pair<const void*, int>, std::array<int, 9>> cluster_caps;
   // launch accounting and optional per-launch event profiling (diagnostics)
   unsigned long long launches = 0;
   bool prof_on = false;
@@ -267,6 +295,8 @@ void free_handle(dflash_handle* h) {
   for (auto p : h->wqkv) cudaFree(p);
   for (auto p : h->wgu) cudaFree(p);
   for (auto p : h->wo) cudaFree(p);
+  for (auto p : h->wdown) cudaFree(p);
+  cudaFree(h->fcw);
   cudaFree(h->wkv);
   cudaFree(h->lm_head16);
   cudaFree(h->knorm_all);
@@ -300,20 +330,38 @@ struct LaunchScope {
 // Launch of a hot-path kernel; with `pdl` the launch may overlap the tail of
 // the previous kernel in the stream (every such kernel calls pdl_wait() before
 // it touches memory that an earlier kernel writes or a later one overwrites).
+// `cluster` > 1 launches thread-block clusters of that many CTAs along x.
 template <typename... KArgs, typename... Args>
-void launch_k(bool pdl, void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
-              cudaStream_t st, Args&&... args) {
+void launch_kc(bool pdl, int cluster, void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+               cudaStream_t st, Args&&... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  if (pdl) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  if (cluster > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = static_cast<unsigned>(cluster);
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
+  cfg.numAttrs = n;
   cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
+template <typename... KArgs, typename... Args>
+void launch_k(bool pdl, void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+              cudaStream_t st, Args&&... args) {
+  launch_kc(pdl, 1, kern, grid, block, smem, st, std::forward<Args>(args)...);
 }
 
 // ---------------------------------------------------------------------------
@@ -342,14 +390,66 @@ cudaError_t set_gemm_attrs_all() {
 template <int BN, class Epi>
 void launch_gemm_bn(const dflash_handle* h, const CUtensorMap& ta, const CUtensorMap& tw,
                     const GemmParams& gp, const Epi& epi, int grid, int smem, cudaStream_t st) {
-  launch_k(h->pdl, gemm_tcgen05_kernel<BN, Epi>, dim3(grid), dim3(kGemmThreads), smem, st, ta, tw, gp,
-           epi);
+  launch_kc(h->pdl, gp.cluster_s, gemm_tcgen05_kernel<BN, Epi>, dim3(grid), dim3(kGemmThreads),
+            smem, st, ta, tw, gp, epi);
+}
+
+// cap[S] = clusters of S CTAs (S = 2..8) of this GEMM instantiation that can be
+// resident at once with `smem` bytes each; cached per handle.  nullptr if the
+// occupancy query fails (cluster split-K is then not used).
+template <int BN, class Epi>
+const int* gemm_cluster_caps_bn(dflash_handle* h, int smem) {
+  const void* key = reinterpret_cast<const void*>(gemm_tcgen05_kernel<BN, Epi>);
+  std::lock_guard<std::mutex> lk(h->mu);
+  auto it = h->cluster_caps.find(std::make_pair(key, smem));
+  if (it != h->cluster_caps.end()) return it->second.data();
+  std::array<int, 9> cap{};
+  for (int S = 2; S <= 8; ++S) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(S);
+    cfg.blockDim = dim3(kGemmThreads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(S);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, gemm_tcgen05_kernel<BN, Epi>, &cfg) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    cap[S] = n;
+  }
+  return h->cluster_caps.emplace(std::make_pair(key, smem), cap).first->second.data();
+}
+
+template <class Epi>
+const int* gemm_cluster_caps(dflash_handle* h, int bn, int smem) {
+  switch (bn) {
+    case 256:
+      if constexpr (256 % Epi::kGroup == 0) return gemm_cluster_caps_bn<256, Epi>(h, smem);
+      break;
+    case 128:
+      if constexpr (128 % Epi::kGroup == 0) return gemm_cluster_caps_bn<128, Epi>(h, smem);
+      break;
+    case 64:
+      if constexpr (Epi::kGroup <= 64) return gemm_cluster_caps_bn<64, Epi>(h, smem);
+      break;
+    case 32:
+      if constexpr (Epi::kGroup <= 32) return gemm_cluster_caps_bn<32, Epi>(h, smem);
+      break;
+  }
+  return nullptr;
 }
 
 // D = A[M, K] * W[N, K]^T with epilogue `epi`.  `partials` must hold
 // plan.partial_bytes.
 template <class Epi>
-dflash_status run_gemm(dflash_handle* h, int kind, bool f16, const void* A, int M, int K,
+dflash_status run_gemm(dflash_handle* h, int kind, bool f16, bool w_packed, const void* A, int M,
+                       int K,
                        const void* Wt, int N, const Epi& epi, float* partials,
                        size_t partial_cap, cudaStream_t st, int force_bn = 0,
                        int force_splits = 0) {
@@ -358,12 +458,23 @@ dflash_status run_gemm(dflash_handle* h, int kind, bool f16, const void* A, int 
                    force_bn % Epi::kGroup))
     return DFLASH_ERR_INVALID_ARG;
   if (force_splits < 0 || force_splits > K / kGemmBK) return DFLASH_ERR_INVALID_ARG;
-  const GemmPlan pl = plan_gemm(M, N, K, Epi::kGroup, h->num_sms, force_bn, force_splits);
+  if (w_packed) force_bn = kPackRows;  // the packed layout fixes the tile width
+  GemmPlan pl = plan_gemm(M, N, K, Epi::kGroup, h->num_sms, force_bn, force_splits);
+  if (gemm_staged(pl.a_rows) && pl.tiles <= h->num_sms && !force_splits) {
+    const int* cap = gemm_cluster_caps<Epi>(h, pl.BN, pl.smem);
+    if (cap) pl = plan_gemm(M, N, K, Epi::kGroup, h->num_sms, force_bn, force_splits, cap);
+  }
   if (pl.stream_k && pl.tiles > kCounterSlots) return DFLASH_ERR_UNSUPPORTED_SHAPE;
   if (pl.partial_bytes > partial_cap) return DFLASH_ERR_WORKSPACE;
   CUtensorMap ta, tw;
   if (!h->tmap(&ta, A, M, K, pl.a_rows, f16)) return DFLASH_ERR_CUDA;
-  if (!h->tmap(&tw, Wt, N, K, pl.BN, f16)) return DFLASH_ERR_CUDA;
+  if (w_packed) {
+    if (!h->tmap(&tw, Wt, static_cast<uint64_t>(pl.n_tiles) * pl.k_blocks * kPackRows, kGemmBK,
+                 kPackRows, f16))
+      return DFLASH_ERR_CUDA;
+  } else if (!h->tmap(&tw, Wt, N, K, pl.BN, f16)) {
+    return DFLASH_ERR_CUDA;
+  }
   GemmParams gp;
   gp.M = M;
   gp.N = N;
@@ -373,6 +484,7 @@ dflash_status run_gemm(dflash_handle* h, int kind, bool f16, const void* A, int 
   gp.k_blocks = pl.k_blocks;
   gp.tiles = pl.tiles;
   gp.stream_k = pl.stream_k;
+  gp.cluster_s = pl.cluster_s;
   gp.ipc = pl.ipc;
   gp.total_iters = pl.total_iters;
   gp.nacc = pl.nacc;
@@ -381,6 +493,7 @@ dflash_status run_gemm(dflash_handle* h, int kind, bool f16, const void* A, int 
   gp.a_rows = pl.a_rows;
   gp.stages = pl.stages;
   gp.f16 = f16 ? 1 : 0;
+  gp.w_packed = w_packed ? 1 : 0;
   gp.slot_rows = pl.slot_rows;
   gp.partials = partials;
   gp.counters = h->counters;
@@ -647,7 +760,7 @@ dflash_status propose_layers(dflash_handle* h, const ProposeWs& lw, void* ws,
     eq.num_pages = num_pages;
     eq.eps = c.rms_eps;
     eq.err = h->dev_err;
-    dflash_status s = run_gemm(h, DFLASH_KERNEL_GEMM_QKV, true, nrm, M, H, h->wqkv[l],
+    dflash_status s = run_gemm(h, DFLASH_KERNEL_GEMM_QKV, true, true, nrm, M, H, h->wqkv[l],
                                (Hq + 2 * Hkv) * D, eq, partial, lw.partial_cap, st);
     if (s != DFLASH_OK) return s;
     // non-causal block attention over context + block
@@ -655,7 +768,7 @@ dflash_status propose_layers(dflash_handle* h, const ProposeWs& lw, void* ws,
     if (s != DFLASH_OK) return s;
     // x += Wo o
     EpiResidAdd er{x, H};
-    s = run_gemm(h, DFLASH_KERNEL_GEMM_O, true, o, M, Hq * D, h->wo[l], H, er, partial,
+    s = run_gemm(h, DFLASH_KERNEL_GEMM_O, true, true, o, M, Hq * D, h->wo[l], H, er, partial,
                  lw.partial_cap, st);
     if (s != DFLASH_OK) return s;
     {
@@ -666,11 +779,11 @@ dflash_status propose_layers(dflash_handle* h, const ProposeWs& lw, void* ws,
     if (cudaGetLastError() != cudaSuccess) return DFLASH_ERR_CUDA;
     // h = silu(gate) * up
     EpiSwiGLU eg{hm, I};
-    s = run_gemm(h, DFLASH_KERNEL_GEMM_GATE_UP, true, nrm, M, H, h->wgu[l], 2 * I, eg, partial,
+    s = run_gemm(h, DFLASH_KERNEL_GEMM_GATE_UP, true, true, nrm, M, H, h->wgu[l], 2 * I, eg, partial,
                  lw.partial_cap, st);
     if (s != DFLASH_OK) return s;
     // x += Wd h
-    s = run_gemm(h, DFLASH_KERNEL_GEMM_DOWN, false, hm, M, I, h->w_down[l], H, er, partial,
+    s = run_gemm(h, DFLASH_KERNEL_GEMM_DOWN, false, true, hm, M, I, h->wdown[l], H, er, partial,
                  lw.partial_cap, st);
     if (s != DFLASH_OK) return s;
     LaunchScope scope(h, DFLASH_KERNEL_RMSNORM, st);
@@ -738,6 +851,14 @@ dflash_status dflash_create(const dflash_config* cfg, const dflash_weights* w, i
         !w->wo[l] || !w->q_norm_w[l] || !w->k_norm_w[l] || !w->w_gate[l] || !w->w_up[l] ||
         !w->w_down[l])
       return DFLASH_ERR_INVALID_ARG;
+  // the GEMM weights are read with 16-byte loads when the handle packs them
+  auto misaligned = [](const void* q) { return reinterpret_cast<uintptr_t>(q) % 16 != 0; };
+  if (misaligned(w->fc_w)) return DFLASH_ERR_INVALID_ARG;
+  for (int l = 0; l < L; ++l)
+    if (misaligned(w->wq[l]) || misaligned(w->wk[l]) || misaligned(w->wv[l]) ||
+        misaligned(w->wo[l]) || misaligned(w->w_gate[l]) || misaligned(w->w_up[l]) ||
+        misaligned(w->w_down[l]))
+      return DFLASH_ERR_INVALID_ARG;
   if (c.target_layer_ids) {
     for (int t = 0; t < c.n_target_layers; ++t)
       if (c.target_layer_ids[t] < 0) return DFLASH_ERR_INVALID_ARG;
@@ -763,17 +884,14 @@ dflash_status dflash_create(const dflash_config* cfg, const dflash_weights* w, i
 
   const int H = c.hidden, D = c.head_dim, Hq = c.n_q_heads, Hkv = c.n_kv_heads,
             I = c.intermediate;
-  h->fc_w = static_cast<const bf16*>(w->fc_w);
   h->hidden_norm_w = static_cast<const bf16*>(w->hidden_norm_w);
   h->embed = static_cast<const bf16*>(w->embed);
-  h->lm_head = static_cast<const bf16*>(w->lm_head);
   h->final_norm_w = static_cast<const bf16*>(w->final_norm_w);
   for (int l = 0; l < L; ++l) {
     h->in_norm_w.push_back(static_cast<const bf16*>(w->in_norm_w[l]));
     h->post_norm_w.push_back(static_cast<const bf16*>(w->post_norm_w[l]));
     h->q_norm_w.push_back(static_cast<const bf16*>(w->q_norm_w[l]));
     h->k_norm_w.push_back(static_cast<const bf16*>(w->k_norm_w[l]));
-    h->w_down.push_back(static_cast<const bf16*>(w->w_down[l]));
   }
 
   cudaStream_t st;
@@ -858,6 +976,50 @@ dflash_status dflash_create(const dflash_config* cfg, const dflash_weights* w, i
     ok = ok && to_f16(h->wkv, static_cast<size_t>(L) * 2 * kvrows * H);
     ok = ok && to_f16(h->lm_head16, static_cast<size_t>(c.vocab) * H);
     if (!ok) return fail_st(DFLASH_ERR_CUDA);
+  }
+  // every GEMM weight into the tile-contiguous layout
+  {
+    // packs row-major [N, K] `src` into a new buffer stored at *out
+    auto pack = [&](const void* src, int N, int K, void** out) {
+      const size_t bytes = static_cast<size_t>(cdiv(N, kPackRows)) * kPackRows * K * 2;
+      if (cudaMalloc(out, bytes) != cudaSuccess) {
+        *out = nullptr;
+        return false;
+      }
+      pack_tiles_kernel<<<1184, 256, 0, st>>>(static_cast<const uint16_t*>(src),
+                                              static_cast<uint16_t*>(*out), N, K, bytes / 16, 0);
+      return cudaGetLastError() == cudaSuccess;
+    };
+    // replaces a row-major copy owned by the handle with its packed form
+    auto repack = [&](f16*& rm, int N, int K) {
+      void* p = nullptr;
+      if (!pack(rm, N, K, &p) || cudaStreamSynchronize(st) != cudaSuccess) {
+        cudaFree(p);
+        return false;
+      }
+      cudaFree(rm);
+      rm = static_cast<f16*>(p);
+      return true;
+    };
+    bool ok = true;
+    for (int l = 0; ok && l < L; ++l) {
+      ok = ok && repack(h->wqkv[l], (Hq + 2 * Hkv) * D, H);
+      ok = ok && repack(h->wgu[l], 2 * I, H);
+      ok = ok && repack(h->wo[l], H, Hq * D);
+    }
+    ok = ok && repack(h->wkv, L * 2 * Hkv * D, H);
+    ok = ok && repack(h->lm_head16, c.vocab, H);
+    for (int l = 0; ok && l < L; ++l) {
+      void* p = nullptr;
+      ok = pack(w->w_down[l], H, I, &p);
+      if (p) h->wdown.push_back(static_cast<bf16*>(p));
+    }
+    if (ok) {
+      void* p = nullptr;
+      ok = pack(w->fc_w, H, c.n_target_layers * H, &p);
+      h->fcw = static_cast<bf16*>(p);
+    }
+    if (!ok || cudaStreamSynchronize(st) != cudaSuccess) return fail_st(DFLASH_ERR_CUDA);
   }
   if (cudaMalloc(&h->rope, static_cast<size_t>(c.max_position) * (D / 2) * sizeof(float2)) !=
       cudaSuccess)
@@ -950,8 +1112,8 @@ dflash_status dflash_inject_context(dflash_handle* h, const void* aux, const int
 
   // (1) fc over the concatenated tapped states
   EpiStoreF32 e1{fcx, H};
-  dflash_status s = run_gemm(h, DFLASH_KERNEL_GEMM_FC, false, aux, n, c.n_target_layers * H,
-                             h->fc_w, H, e1, partial, lw.partial_cap, st);
+  dflash_status s = run_gemm(h, DFLASH_KERNEL_GEMM_FC, false, true, aux, n, c.n_target_layers * H,
+                             h->fcw, H, e1, partial, lw.partial_cap, st);
   if (s != DFLASH_OK) return s;
   // (2) hidden_norm
   {
@@ -978,7 +1140,7 @@ dflash_status dflash_inject_context(dflash_handle* h, const void* aux, const int
     e3.num_pages = num_pages;
     e3.eps = c.rms_eps;
     e3.err = h->dev_err;
-    s = run_gemm(h, DFLASH_KERNEL_GEMM_KV_INJECT, true, ctx, n, H, h->wkv, NKV, e3, partial,
+    s = run_gemm(h, DFLASH_KERNEL_GEMM_KV_INJECT, true, true, ctx, n, H, h->wkv, NKV, e3, partial,
                  lw.partial_cap, st);
   } else {
     EpiKVInject<64> e3{};
@@ -996,7 +1158,7 @@ dflash_status dflash_inject_context(dflash_handle* h, const void* aux, const int
     e3.num_pages = num_pages;
     e3.eps = c.rms_eps;
     e3.err = h->dev_err;
-    s = run_gemm(h, DFLASH_KERNEL_GEMM_KV_INJECT, true, ctx, n, H, h->wkv, NKV, e3, partial,
+    s = run_gemm(h, DFLASH_KERNEL_GEMM_KV_INJECT, true, true, ctx, n, H, h->wkv, NKV, e3, partial,
                  lw.partial_cap, st);
   }
   return s;
@@ -1045,7 +1207,7 @@ dflash_status dflash_propose(dflash_handle* h, const int32_t* bonus_tokens,
   if (s != DFLASH_OK) return s;
   // aliased target LM head with the greedy pick fused into its epilogue
   EpiArgmax ea{keys, logits_out, c.vocab};
-  s = run_gemm(h, DFLASH_KERNEL_GEMM_LM_HEAD, true, frows, B * K, H, h->lm_head16, c.vocab, ea,
+  s = run_gemm(h, DFLASH_KERNEL_GEMM_LM_HEAD, true, true, frows, B * K, H, h->lm_head16, c.vocab, ea,
                partial, lw.partial_cap, st);
   if (s != DFLASH_OK) return s;
   {
@@ -1098,7 +1260,7 @@ dflash_status dflash_linear(dflash_handle* h, const void* A, const void* W, int 
   if (workspace_bytes < need) return DFLASH_ERR_WORKSPACE;
   DF_CUDA(use_device(h->device));
   EpiStoreF32 e{out, N};
-  return run_gemm(h, DFLASH_KERNEL_LINEAR, false, A, M, K, W, N, e,
+  return run_gemm(h, DFLASH_KERNEL_LINEAR, false, false, A, M, K, W, N, e,
                   static_cast<float*>(workspace), workspace_bytes,
                   static_cast<cudaStream_t>(stream));
 }
@@ -1116,7 +1278,7 @@ dflash_status dflash_linear_ex(dflash_handle* h, const void* A, const void* W, i
     return DFLASH_ERR_INVALID_ARG;
   DF_CUDA(use_device(h->device));
   EpiStoreF32 e{out, N};
-  return run_gemm(h, DFLASH_KERNEL_LINEAR, false, A, M, K, W, N, e,
+  return run_gemm(h, DFLASH_KERNEL_LINEAR, false, false, A, M, K, W, N, e,
                   static_cast<float*>(workspace), workspace_bytes,
                   static_cast<cudaStream_t>(stream), block_n, splits);
 }

@@ -14,9 +14,12 @@
 // dependent MMA chain.
 //
 // Scheduling: whole tiles round-robin over one CTA per SM when there are
-// enough of them to fill the GPU evenly; otherwise stream-K — every CTA takes
-// an equal contiguous range of the (tile, k-block) iteration space, so every
-// SM streams weights.  A tile split across CTAs has each piece written as an
+// enough of them to fill the GPU evenly; for a few rows (the staged epilogue)
+// and fewer tiles than SMs, cluster split-K — the S CTAs of a thread-block
+// cluster share one tile, each taking 1/S of its k-blocks, and reduce the
+// pieces through distributed shared memory (no global partials, no fence, no
+// arrival counter); otherwise stream-K — every CTA takes an equal contiguous
+// range of the (tile, k-block) iteration space, so every SM streams weights.  A tile split across CTAs has each piece written as an
 // fp32 partial (at most two slots per CTA); the CTA that finishes the tile's
 // last piece (a per-tile arrival counter, no waiting) sums the pieces in CTA
 // order — so the result is deterministic — and runs the epilogue.  The
@@ -76,6 +79,7 @@ struct GemmParams {
   int m_tiles, n_tiles, k_blocks;
   int tiles;           // m_tiles * n_tiles
   int stream_k;        // 0: whole tiles round-robin; 1: equal ranges of (tile, k-block) iterations
+  int cluster_s;       // > 1: cluster split-K, S CTAs per tile (grid = tiles * S, cluster S x 1 x 1)
   int ipc;             // stream-K: k-block iterations per CTA
   int total_iters;     // stream-K: tiles * k_blocks
   int nacc;            // independent accumulator chains per tile (1, 2 or 4)
@@ -84,6 +88,7 @@ struct GemmParams {
   int a_rows;          // rows of the A box / slot (128, or M rounded up to 16 when M < 128)
   int stages;          // pipeline depth (<= kGemmMaxStages)
   int f16;             // operands are fp16 (1) or bf16 (0)
+  int w_packed;        // W in the tile-contiguous layout (BN = 256 row chunks), else row-major
   int slot_rows;       // rows held per partial slot (min(M, 128))
   float* partials;     // stream-K: [gridDim.x * 2][slot_rows][BN] fp32
   unsigned* counters;  // [tiles], zero on entry, zero on exit
@@ -101,7 +106,11 @@ struct GemmSeg {
 struct GemmSegIter {
   int cur, end, step;
   __device__ __forceinline__ explicit GemmSegIter(const GemmParams& p) {
-    if (p.stream_k) {
+    if (p.cluster_s > 1) {
+      cur = blockIdx.x;  // one segment: this CTA's share of tile blockIdx.x / S
+      end = blockIdx.x + 1;
+      step = 1;
+    } else if (p.stream_k) {
       cur = blockIdx.x * p.ipc;
       end = min(p.total_iters, cur + p.ipc);
       step = 0;
@@ -113,7 +122,17 @@ struct GemmSegIter {
   }
   __device__ __forceinline__ bool next(const GemmParams& p, GemmSeg& s) {
     if (cur >= end) return false;
-    if (p.stream_k) {
+    if (p.cluster_s > 1) {
+      const int S = p.cluster_s;
+      s.tile = cur / S;
+      const int rank = cur - s.tile * S;
+      s.kb0 = rank * p.k_blocks / S;
+      s.kb1 = (rank + 1) * p.k_blocks / S;
+      s.first_cta = s.tile * S;
+      s.nseg = 1;  // reduced through the cluster, not through global partials
+      s.slot = 0;
+      cur += 1;
+    } else if (p.stream_k) {
       s.tile = cur / p.k_blocks;
       s.kb0 = cur - s.tile * p.k_blocks;
       s.kb1 = min(p.k_blocks, s.kb0 + (end - cur));
@@ -156,6 +175,16 @@ __device__ __forceinline__ void tmem_load_sum32(uint32_t taddr, int nacc, float*
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] += t[i];
   }
+}
+
+// Coordinates of the W box of (n_tile, k-block kb): row-major W is addressed by
+// (k, row); the tile-contiguous layout stores each 256 x 64 tile as one chunk.
+__device__ __forceinline__ int w_x(const GemmParams& p, int kb) {
+  return p.w_packed ? 0 : kb * kGemmBK;
+}
+template <int BN>
+__device__ __forceinline__ int w_y(const GemmParams& p, int n_tile, int kb) {
+  return p.w_packed ? (n_tile * p.k_blocks + kb) * 256 : n_tile * BN;
 }
 
 template <int BN, class Epi>
@@ -208,7 +237,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tmem_relinquish();
   }
   tc_fence_before();
-  __syncthreads();
+  cta_sync();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int acc_cols = p.nacc * BN;   // TMEM columns of one accumulator buffer
@@ -228,8 +257,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         while (pre < stages && it0.next(p, s0)) {
           for (int kb = s0.kb0; kb < s0.kb1 && pre < stages; ++kb, ++pre) {
             mbar_arrive_expect_tx(&full[pre], stage_tx);
-            tma_load_2d_hint(sB + pre * C::kBBytes, &tmW, &full[pre], kb * kGemmBK,
-                             s0.n_tile * BN, pol_w);
+            tma_load_2d_hint(sB + pre * C::kBBytes, &tmW, &full[pre], w_x(p, kb),
+                             w_y<BN>(p, s0.n_tile, kb), pol_w);
           }
         }
       }
@@ -247,8 +276,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               break;
             }
             mbar_arrive_expect_tx(&full[stage], stage_tx);
-            tma_load_2d_hint(sB + stage * C::kBBytes, &tmW, &full[stage], kb * kGemmBK,
-                             sg.n_tile * BN, pol_w);
+            tma_load_2d_hint(sB + stage * C::kBBytes, &tmW, &full[stage], w_x(p, kb),
+                             w_y<BN>(p, sg.n_tile, kb), pol_w);
           }
           tma_load_2d_hint(sA + stage * a_bytes, &tmA, &full[stage], kb * kGemmBK,
                            sg.m_tile * kGemmBM, pol_a);
@@ -345,6 +374,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         acc_phase ^= 1u;
       }
       named_bar_sync(1, 128);
+      if (p.cluster_s > 1) break;          // reduced across the cluster below
       const int rows = p.M;                // one M tile: M <= a_rows <= 32
       const int nf4 = rows * F4;
       if (sg.nseg > 1) {
@@ -524,8 +554,53 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   }
 
+  if (p.cluster_s > 1) {
+    // Every thread of every CTA of the cluster reaches both barriers exactly
+    // once (no early exits above, all waits bounded).  Between them, CTA rank q
+    // reduces the column groups g = q, q + S, ... of the tile over the S
+    // staging tiles in rank order (deterministic) and runs the epilogue.
+    cluster_sync();
+    if (warp >= 2) {
+      constexpr int LD = BN + 4;
+      constexpr int NG = BN / G;
+      const int S = p.cluster_s;
+      const int rank = static_cast<int>(cluster_rank());
+      const int tile = blockIdx.x / S;
+      const int n_tile = tile / p.m_tiles;
+      const int rows = p.M;
+      const int my_groups = (NG - rank + S - 1) / S;
+      const int tid = threadIdx.x - 64;
+      for (int item = tid; item < my_groups * rows; item += 128) {
+        const int lg = item / rows, r = item - lg * rows;
+        const int g = rank + lg * S;
+        const int n0 = n_tile * BN + g * G;
+        if (n0 >= p.N) continue;
+        float v[G];
+#pragma unroll
+        for (int j = 0; j < G; ++j) v[j] = 0.f;
+        const float* src = staging + r * LD + g * G;
+#pragma unroll 1
+        for (int q = 0; q < S; ++q) {
+#pragma unroll
+          for (int j = 0; j < G; j += 4) {
+            const float4 t = ld_peer_f4(src + j, static_cast<uint32_t>(q));
+            v[j] += t.x;
+            v[j + 1] += t.y;
+            v[j + 2] += t.z;
+            v[j + 3] += t.w;
+          }
+        }
+        typename Epi::State st;
+        epi.begin(st);
+        epi.apply(st, r, n0, min(G, p.N - n0), v);
+        epi.end(st, r, true);
+      }
+    }
+    cluster_sync();  // no CTA leaves while a peer may still read its staging tile
+  }
+
   tc_fence_before();
-  __syncthreads();
+  cta_sync();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, static_cast<uint32_t>(p.tmem_cols));

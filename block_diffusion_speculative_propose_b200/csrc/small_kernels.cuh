@@ -255,6 +255,42 @@ __global__ void bf16_to_f16_kernel(uint16_t* __restrict__ data, size_t n) {
   }
 }
 
+// Tile-contiguous GEMM weight layout: the kPackRows x 64 tile (n_tile, k_block)
+// of a row-major W [N, K] becomes one contiguous chunk (kPackRows rows of 128
+// bytes, in order) at chunk index n_tile * (K / 64) + k_block; rows past N are
+// zero.  Every TMA box of the weight stream is then a single contiguous read.
+// With to_f16 the bf16 values are converted to fp16 on the way.
+constexpr int kPackRows = 256;
+
+__global__ void pack_tiles_kernel(const uint16_t* __restrict__ src, uint16_t* __restrict__ dst,
+                                  int N, int K, size_t units, int to_f16) {
+  const int kb_count = K / 64;
+  for (size_t u = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; u < units;
+       u += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const size_t chunk = u / (kPackRows * 8);
+    const int within = static_cast<int>(u - chunk * (kPackRows * 8));
+    const int r = within >> 3, j8 = within & 7;
+    const int nt = static_cast<int>(chunk / kb_count);
+    const int kb = static_cast<int>(chunk - static_cast<size_t>(nt) * kb_count);
+    const int row = nt * kPackRows + r;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (row < N)
+      v = *reinterpret_cast<const uint4*>(src + static_cast<size_t>(row) * K + kb * 64 + j8 * 8);
+    if (to_f16) {
+      uint32_t* w = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const bf16* b2 = reinterpret_cast<const bf16*>(&w[q]);
+        const f16 lo = __float2half_rn(__bfloat162float(b2[0]));
+        const f16 hi = __float2half_rn(__bfloat162float(b2[1]));
+        w[q] = static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(&lo)) |
+               (static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(&hi)) << 16);
+      }
+    }
+    *reinterpret_cast<uint4*>(dst + u * 8) = v;
+  }
+}
+
 // cos / sin of pos * theta^(-2j/D), evaluated in double, stored as fp32 pairs.
 __global__ void rope_table_kernel(float2* __restrict__ table, int max_pos, int half,
                                   double theta) {

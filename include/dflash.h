@@ -96,13 +96,18 @@ typedef struct dflash_config {
  *   fc_w [H, T*H]   hidden_norm_w [H]   embed [V, H]   lm_head [V, H]   final_norm_w [H]
  *   in_norm_w/post_norm_w [H]   wq [Hq*d, H]   wk, wv [Hkv*d, H]   wo [H, Hq*d]
  *   q_norm_w, k_norm_w [d]      w_gate, w_up [I, H]   w_down [H, I]
- * Storage precision of the path: the projections whose inputs are bounded by
- * construction (RMSNorm outputs, attention outputs) run with fp16 operands, so
- * dflash_create keeps fp16 copies of wq|wk|wv (packed), w_gate|w_up (packed in
- * 16-row blocks), the stacked per-layer [wk; wv], wo and lm_head (bf16 -> fp16
- * is exact in fp16's normal range).  fc_w and w_down are used in bf16 in place,
- * as are the norm weights and the embedding (the target's aliased table): those
- * pointers must stay valid and unchanged for the lifetime of the handle. */
+ * Every weight of a GEMM is copied by dflash_create into a tile-contiguous
+ * layout (each 256-row x 64-column tile one contiguous 32 KB chunk, so that the
+ * weight stream reads whole chunks).  Storage precision of the path: the
+ * projections whose inputs are bounded by construction (RMSNorm outputs,
+ * attention outputs) run with fp16 operands, so the copies of wq|wk|wv
+ * (stacked), w_gate|w_up (interleaved in 16-row blocks), the stacked per-layer
+ * [wk; wv], wo and lm_head are fp16 (bf16 -> fp16 is exact in fp16's normal
+ * range); fc_w and w_down stay bf16.  Those source buffers may be freed after
+ * dflash_create returns.  The norm weights and the embedding (the target's
+ * aliased table) are used in place: those pointers must stay valid and
+ * unchanged for the lifetime of the handle.  The GEMM weight pointers must be
+ * 16-byte aligned (DFLASH_ERR_INVALID_ARG otherwise). */
 typedef struct dflash_weights {
   const void* fc_w;
   const void* hidden_norm_w;
