@@ -49,6 +49,8 @@ struct AttnParams {
   const int* seq_lens;
   const int* block_table;
   int B, W, bs, Hq, Hkv, G, R, num_pages, chunk_keys, max_splits;
+  int cluster;         // tcgen05 kernel: the max_splits splits of a (request, kv head) form one
+                       // thread-block cluster and are combined through distributed shared memory
   float scale_log2;    // log2(e) / sqrt(D)
   unsigned* err;
 };

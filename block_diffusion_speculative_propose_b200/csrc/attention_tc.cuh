@@ -22,6 +22,14 @@
 // Shared memory: K/V ring 2 x (K + V) tiles, Q (64 x d), P hi/lo x 2 buffers.
 // TMEM: S buffers at columns [0, 256), O at [256, 256 + d).  Every wait is
 // bounded; a wait that runs out sets the timeout bit and the CTA winds down.
+//
+// Cluster mode (few requests: splitting the keys is what fills the GPU): the
+// splits of one (request, kv head) are the CTAs of one cluster.  Each parks
+// its unnormalised O rows and (m, l) in its K/V ring once the last P V has
+// landed; after a cluster barrier, CTA rank q combines rows q, q + S, ... over
+// the S pieces in rank order and writes the fp16 output, so no partials reach
+// global memory and no combine kernel runs.  A split past the request's last
+// key contributes (m, l) = (-inf, 0).
 #pragma once
 
 #include "attention.cuh"
@@ -46,6 +54,10 @@ struct TcAttnCfg {
   static constexpr int kOffBar = kOffP + 4 * kPBytes;
   static constexpr int kSmem = 1024 + kOffBar + 256;
   static constexpr int kOCol = 2 * kTcKeys;                   // TMEM column of O
+  // cluster combine, inside the (then idle) K/V ring: O rows, (m, l), weights
+  static constexpr int kCombOffML = kTcM * (D + 8) * 4;
+  static constexpr int kCombOffW = kCombOffML + kTcM * 8;
+  static_assert(kCombOffW + kTcM * 8 * 4 <= 2 * kTcStages * kKVBytes, "combine staging");
   static_assert(kOCol + D <= 512, "TMEM budget");
 };
 
@@ -59,10 +71,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int n_keys = p.seq_lens[b] + p.bs;
   const int k0 = split * p.chunk_keys;
-  if (k0 >= n_keys) return;
+  // (every CTA of a cluster stays to the end: its peers read its shared memory)
+  if (k0 >= n_keys && !p.cluster) return;
   const int k1 = min(n_keys, k0 + p.chunk_keys);
   const int n_splits_b = (n_keys + p.chunk_keys - 1) / p.chunk_keys;
-  const int n_tiles = (k1 - k0 + kTcKeys - 1) / kTcKeys;
+  const int n_tiles = k0 < n_keys ? (k1 - k0 + kTcKeys - 1) / kTcKeys : 0;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   extern __shared__ uint8_t smem_raw[];
@@ -147,7 +160,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (lane == 0) {
       const uint32_t idesc_qk = umma_idesc_bf16(kTcM, kTcKeys, false);
       const uint32_t idesc_pv = umma_idesc_bf16(kTcM, D, true);
-      bool ok = mbar_wait(q_full, 0, p.err);
+      bool ok = n_tiles > 0 && mbar_wait(q_full, 0, p.err);
       tc_fence_after();
       auto issue_qk = [&](int t) -> bool {
         const int s = t & 1, u = t >> 1;
@@ -333,7 +346,47 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
 
     float o[D / 8][4];
-    if (ok && mbar_wait(o_final, 0, p.err)) {
+    if (p.cluster) {
+      // park this split's unnormalised O rows and (m, l) in the K/V ring
+      // (every TMA load and MMA of the CTA has completed once o_final fired)
+      const bool have = ok && n_tiles > 0 && mbar_wait(o_final, 0, p.err);
+#pragma unroll
+      for (int db = 0; db < D / 8; ++db)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[db][e] = 0.f;
+      if (have) {
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c) {
+          float ov[32];
+          tmem_ld_16x256b_x8(tmem_base + lane_base + C::kOCol + c * 64, ov);
+          tmem_ld_wait();
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) o[c * 8 + jj][e] = ov[4 * jj + e];
+        }
+      }
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        l_run[hh] += __shfl_xor_sync(0xffffffffu, l_run[hh], 1);
+        l_run[hh] += __shfl_xor_sync(0xffffffffu, l_run[hh], 2);
+      }
+      float* so = reinterpret_cast<float*>(smem);                  // [64][D + 8]
+      float2* sml = reinterpret_cast<float2*>(smem + C::kCombOffML); // [64]
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int r = r0 + 8 * hh;
+#pragma unroll
+        for (int db = 0; db < D / 8; ++db) {
+          const int d = db * 8 + 2 * (lane & 3);
+          *reinterpret_cast<float2*>(so + r * (D + 8) + d) =
+              make_float2(o[db][2 * hh], o[db][2 * hh + 1]);
+        }
+        if ((lane & 3) == 0)
+          sml[r] = have ? make_float2(m_ref[hh], l_run[hh]) : make_float2(-INFINITY, 0.f);
+      }
+    } else if (ok && mbar_wait(o_final, 0, p.err)) {
       tc_fence_after();
 #pragma unroll
       for (int c = 0; c < D / 64; ++c) {
@@ -379,6 +432,55 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
       }
     }
+  }
+
+  if (p.cluster) {
+    cluster_sync();
+    if (warp >= 2) {
+      const int S = p.max_splits;
+      const int q = static_cast<int>(cluster_rank());
+      const int tid = threadIdx.x - 64;
+      const float* so = reinterpret_cast<const float*>(smem);
+      const float2* sml = reinterpret_cast<const float2*>(smem + C::kCombOffML);
+      float* wsc = reinterpret_cast<float*>(smem + C::kCombOffW);  // [64 / S rows][S]
+      const int my_rows = (p.R - q + S - 1) / S;                   // rows q, q + S, ...
+      // per-row weights 2^(m_p - M) / L of the S pieces
+      if (tid < my_rows) {
+        const int r = q + tid * S;
+        float mp[8], lp[8], M = -INFINITY;
+        for (int s = 0; s < S; ++s) {
+          const float4 t = ld_peer_f4(sml + (r & ~1), static_cast<uint32_t>(s));
+          mp[s] = (r & 1) ? t.z : t.x;
+          lp[s] = (r & 1) ? t.w : t.y;
+          M = fmaxf(M, mp[s]);
+        }
+        float L = 0.f;
+        for (int s = 0; s < S; ++s) {
+          mp[s] = mp[s] == -INFINITY ? 0.f : exp2f(mp[s] - M);
+          L += lp[s] * mp[s];
+        }
+        const float inv = 1.f / L;
+        for (int s = 0; s < S; ++s) wsc[tid * 8 + s] = mp[s] * inv;
+      }
+      named_bar_sync(2, 128);
+      for (int item = tid; item < my_rows * (D / 4); item += 128) {
+        const int lr = item / (D / 4), d = (item - lr * (D / 4)) * 4;
+        const int r = q + lr * S;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int s = 0; s < S; ++s) {
+          const float w = wsc[lr * 8 + s];
+          const float4 t = ld_peer_f4(so + r * (D + 8) + d, static_cast<uint32_t>(s));
+          acc.x += w * t.x;
+          acc.y += w * t.y;
+          acc.z += w * t.z;
+          acc.w += w * t.w;
+        }
+        const int i = r / p.G, g = r - (r / p.G) * p.G;
+        f16* dst = p.o + (static_cast<size_t>(b * p.bs + i) * p.Hq + h * p.G + g) * D + d;
+        *reinterpret_cast<uint2*>(dst) = make_uint2(pack_f16x2(acc.x, acc.y), pack_f16x2(acc.z, acc.w));
+      }
+    }
+    cluster_sync();  // no CTA leaves while a peer may still read its shared memory
   }
 
   tc_fence_before();

@@ -188,6 +188,7 @@ size_t gemm_partial_bound(int M, int num_sms) {
 struct AttnPlan {
   int chunk_keys = 0, max_splits = 0, R = 0, row_groups = 0, key_parts = 0, nwc = 0;
   bool tc = false;   // tcgen05 kernel (kv groups of up to 64 query rows)
+  bool cluster = false;  // tcgen05 kernel, splits of a (request, kv head) combined in a cluster
   size_t part_o_bytes = 0, part_ml_bytes = 0;
 };
 
@@ -212,6 +213,23 @@ AttnPlan plan_attention(int B, int Hkv, int W, int P, int bs, int G, int D, int 
       a.max_splits > 1 ? static_cast<size_t>(a.max_splits) * B * Hkv * a.R * D * 4 : 0;
   a.part_ml_bytes =
       a.max_splits > 1 ? static_cast<size_t>(a.max_splits) * B * Hkv * a.R * 2 * 4 : 0;
+  // Few (request, kv head) pairs: the key splits are what fills the GPU, and
+  // they are combined inside a cluster of up to 8 CTAs instead of through
+  // global partials and a second kernel.
+  if (a.tc && 2 * B * Hkv <= num_sms) {
+    const int S = std::min(8, num_sms / (B * Hkv));
+    if (S >= 2) {
+      const int chunk = cdiv(cdiv(keys_max, S), kTcKeys) * kTcKeys;
+      const int splits = cdiv(keys_max, chunk);
+      if (splits >= 2) {
+        a.cluster = true;
+        a.chunk_keys = chunk;
+        a.max_splits = splits;
+        a.part_o_bytes = 0;
+        a.part_ml_bytes = 0;
+      }
+    }
+  }
   return a;
 }
 
@@ -552,10 +570,11 @@ dflash_status run_attention(dflash_handle* h, const AttnPlan& ap, AttnParams prm
   const int smem = AttnCfg<D>::smem_bytes(ap.nwc);
   prm.row_groups = ap.row_groups;
   prm.key_parts = ap.key_parts;
+  prm.cluster = ap.cluster ? 1 : 0;
   if (ap.tc) {
     LaunchScope scope(h, DFLASH_KERNEL_ATTENTION, st);
-    launch_k(h->pdl, attn_block_tc_kernel<D>, grid, dim3(kTcThreads), TcAttnCfg<D>::kSmem, st, tk, tv,
-             prm);
+    launch_kc(h->pdl, ap.cluster ? ap.max_splits : 1, attn_block_tc_kernel<D>, grid,
+              dim3(kTcThreads), TcAttnCfg<D>::kSmem, st, tk, tv, prm);
   } else {
     LaunchScope scope(h, DFLASH_KERNEL_ATTENTION, st);
     if (ap.key_parts == 1)
@@ -565,7 +584,7 @@ dflash_status run_attention(dflash_handle* h, const AttnPlan& ap, AttnParams prm
     else
       launch_k(h->pdl, attn_block_kernel<D, 16>, grid, dim3(threads), smem, st, tk, tv, prm);
   }
-  if (ap.max_splits > 1) {
+  if (ap.max_splits > 1 && !ap.cluster) {
     LaunchScope scope(h, DFLASH_KERNEL_ATTN_COMBINE, st);
     const int rows = prm.B * c.n_kv_heads * prm.R;
     launch_k(h->pdl, attn_combine_kernel<D>, dim3(cdiv(rows, 8)), dim3(256), 0, st, prm);
