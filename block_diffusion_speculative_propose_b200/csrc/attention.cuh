@@ -157,16 +157,28 @@ __global__ void __launch_bounds__(32 * (kAttnMaxComputeWarps + 1), 1)
   const int kp = warp / p.row_groups;   // keys kp*KP .. kp*KP+KP-1 of every tile
   // Q rows of this warp: r = i * G + g  ->  q[(b*bs + i), h*G + g, :]
   bf16* sQw = sQ + warp * 16 * C::kQStride;
-  for (int e = lane; e < 16 * (D / 8); e += 32) {
-    const int rr = e / (D / 8), c = e - rr * (D / 8);
-    const int r = rg * 16 + rr;
-    uint4 val = make_uint4(0, 0, 0, 0);
-    if (r < p.R) {
-      const int i = r / p.G, g = r - (r / p.G) * p.G;
-      const bf16* src = p.q + (static_cast<size_t>(b * p.bs + i) * p.Hq + h * p.G + g) * D;
-      val = *reinterpret_cast<const uint4*>(src + c * 8);
+  {
+    // all of a lane's loads are issued before any store
+    constexpr int kQPer = 16 * (D / 8) / 32;
+    uint4 qv[kQPer];
+#pragma unroll
+    for (int u = 0; u < kQPer; ++u) {
+      const int e = lane + u * 32;
+      const int rr = e / (D / 8), c = e - rr * (D / 8);
+      const int r = rg * 16 + rr;
+      qv[u] = make_uint4(0, 0, 0, 0);
+      if (r < p.R) {
+        const int i = r / p.G, g = r - (r / p.G) * p.G;
+        const bf16* src = p.q + (static_cast<size_t>(b * p.bs + i) * p.Hq + h * p.G + g) * D;
+        qv[u] = *reinterpret_cast<const uint4*>(src + c * 8);
+      }
     }
-    *reinterpret_cast<uint4*>(sQw + rr * C::kQStride + c * 8) = val;
+#pragma unroll
+    for (int u = 0; u < kQPer; ++u) {
+      const int e = lane + u * 32;
+      const int rr = e / (D / 8), c = e - rr * (D / 8);
+      *reinterpret_cast<uint4*>(sQw + rr * C::kQStride + c * 8) = qv[u];
+    }
   }
   __syncwarp();
   uint32_t qa[D / 16][4];

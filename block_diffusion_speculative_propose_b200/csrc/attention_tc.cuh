@@ -24,12 +24,14 @@
 // bounded; a wait that runs out sets the timeout bit and the CTA winds down.
 //
 // Cluster mode (few requests: splitting the keys is what fills the GPU): the
-// splits of one (request, kv head) are the CTAs of one cluster.  Each parks
-// its unnormalised O rows and (m, l) in its K/V ring once the last P V has
-// landed; after a cluster barrier, CTA rank q combines rows q, q + S, ... over
-// the S pieces in rank order and writes the fp16 output, so no partials reach
-// global memory and no combine kernel runs.  A split past the request's last
-// key contributes (m, l) = (-inf, 0).
+// splits of one (request, kv head) are the CTAs of one cluster; CTA rank q
+// owns rows q, q + S, ...  Once every CTA of the cluster is past its key loop
+// (first cluster barrier), each pushes its unnormalised O rows and (m, l)
+// with remote shared-memory stores into the owners' (now idle) K/V rings;
+// after the second barrier each owner combines its rows from local shared
+// memory over the S pieces in rank order and writes the fp16 output.  No
+// partials reach global memory and no combine kernel runs.  A split past the
+// request's last key contributes (m, l) = (-inf, 0).
 #pragma once
 
 #include "attention.cuh"
@@ -54,10 +56,11 @@ struct TcAttnCfg {
   static constexpr int kOffBar = kOffP + 4 * kPBytes;
   static constexpr int kSmem = 1024 + kOffBar + 256;
   static constexpr int kOCol = 2 * kTcKeys;                   // TMEM column of O
-  // cluster combine, inside the (then idle) K/V ring: O rows, (m, l), weights
-  static constexpr int kCombOffML = kTcM * (D + 8) * 4;
-  static constexpr int kCombOffW = kCombOffML + kTcM * 8;
-  static_assert(kCombOffW + kTcM * 8 * 4 <= 2 * kTcStages * kKVBytes, "combine staging");
+  // cluster combine, inside the (then idle) K/V ring: received O rows
+  // [lr * S + src][D + 8] and (m, l) [lr * S + src] (S * ceil(64 / S) <= 71 slots)
+  static constexpr int kCombSlots = kTcM + 7;
+  static constexpr int kCombOffML = kCombSlots * (D + 8) * 4;
+  static_assert(kCombOffML + kCombSlots * 8 <= 2 * kTcStages * kKVBytes, "combine buffers");
   static_assert(kOCol + D <= 512, "TMEM budget");
 };
 
@@ -119,6 +122,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   cta_sync();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // softmax warps, cluster mode: this thread's O rows (r0, r0 + 8) and (m, l)
+  float o[D / 8][4];
+  float m_fin[2] = {-INFINITY, -INFINITY}, l_fin[2] = {0.f, 0.f};
+  bool have = false;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -179,7 +186,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       };
       if (ok) ok = issue_qk(0);
       for (int t = 0; ok && t < n_tiles; ++t) {
-        if (t + 1 < n_tiles && !issue_qk(t + 1)) break;
+        // S of tile t+1 goes ahead of P V of tile t when its K/V have landed
+        // (its softmax then overlaps P V); otherwise P V(t) is issued first
+        // instead of waiting on the load
+        const int s1 = (t + 1) & 1, u1 = (t + 1) >> 1;
+        const bool qk_first = t + 1 < n_tiles && mbar_try_wait(&kv_full[s1], u1 & 1) &&
+                              mbar_try_wait(&s_empty[s1], (u1 & 1) ^ 1u);
+        if (qk_first && !issue_qk(t + 1)) break;
         const int s = t & 1, u = t >> 1;
         if (!mbar_wait(&p_full[s], u & 1, p.err)) break;
         tc_fence_after();
@@ -199,23 +212,34 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         umma_commit(&p_empty[s]);
         umma_commit(o_ready);
         if (t + 1 == n_tiles) umma_commit(o_final);
+        if (!qk_first && t + 1 < n_tiles && !issue_qk(t + 1)) break;
       }
     }
   } else {
     // ------------------------------------------------------------ softmax warps
     const int sp = warp & 3;                    // TMEM sub-partition = 16-row group
     const int tid = threadIdx.x - 64;           // 0..127
-    // Q rows r = i * G + g of this kv group -> K-major, 128B-swizzled operand
-    for (int e = tid; e < kTcM * (D / 8); e += 128) {
+    // Q rows r = i * G + g of this kv group -> K-major, 128B-swizzled operand;
+    // all of a thread's loads are issued before any store
+    constexpr int kQPer = kTcM * (D / 8) / 128;
+    uint4 qv[kQPer];
+#pragma unroll
+    for (int u = 0; u < kQPer; ++u) {
+      const int e = tid + u * 128;
       const int r = e / (D / 8), c = e - r * (D / 8);
-      uint4 val = make_uint4(0, 0, 0, 0);
+      qv[u] = make_uint4(0, 0, 0, 0);
       if (r < p.R) {
         const int i = r / p.G, g = r - (r / p.G) * p.G;
         const bf16* src = p.q + (static_cast<size_t>(b * p.bs + i) * p.Hq + h * p.G + g) * D;
-        val = *reinterpret_cast<const uint4*>(src + c * 8);
+        qv[u] = *reinterpret_cast<const uint4*>(src + c * 8);
       }
+    }
+#pragma unroll
+    for (int u = 0; u < kQPer; ++u) {
+      const int e = tid + u * 128;
+      const int r = e / (D / 8), c = e - r * (D / 8);
       *reinterpret_cast<uint4*>(sQ + (c >> 3) * kTcM * 128 + r * 128 + (((c & 7) ^ (r & 7)) << 4)) =
-          val;
+          qv[u];
     }
     fence_proxy_async_smem();
     __syncwarp();
@@ -345,11 +369,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (lane == 0) mbar_arrive(&p_full[s]);
     }
 
-    float o[D / 8][4];
     if (p.cluster) {
-      // park this split's unnormalised O rows and (m, l) in the K/V ring
-      // (every TMA load and MMA of the CTA has completed once o_final fired)
-      const bool have = ok && n_tiles > 0 && mbar_wait(o_final, 0, p.err);
+      // keep this split's unnormalised O rows and (m, l) in registers for the
+      // push below (every TMA load and MMA of the CTA has completed once
+      // o_final fired)
+      have = ok && n_tiles > 0 && mbar_wait(o_final, 0, p.err);
 #pragma unroll
       for (int db = 0; db < D / 8; ++db)
 #pragma unroll
@@ -371,20 +395,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int hh = 0; hh < 2; ++hh) {
         l_run[hh] += __shfl_xor_sync(0xffffffffu, l_run[hh], 1);
         l_run[hh] += __shfl_xor_sync(0xffffffffu, l_run[hh], 2);
-      }
-      float* so = reinterpret_cast<float*>(smem);                  // [64][D + 8]
-      float2* sml = reinterpret_cast<float2*>(smem + C::kCombOffML); // [64]
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const int r = r0 + 8 * hh;
-#pragma unroll
-        for (int db = 0; db < D / 8; ++db) {
-          const int d = db * 8 + 2 * (lane & 3);
-          *reinterpret_cast<float2*>(so + r * (D + 8) + d) =
-              make_float2(o[db][2 * hh], o[db][2 * hh + 1]);
-        }
-        if ((lane & 3) == 0)
-          sml[r] = have ? make_float2(m_ref[hh], l_run[hh]) : make_float2(-INFINITY, 0.f);
+        m_fin[hh] = have ? m_ref[hh] : -INFINITY;
+        l_fin[hh] = have ? l_run[hh] : 0.f;
       }
     } else if (ok && mbar_wait(o_final, 0, p.err)) {
       tc_fence_after();
@@ -435,52 +447,57 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
 
   if (p.cluster) {
-    cluster_sync();
+    const int S = p.max_splits;
+    const int q = static_cast<int>(cluster_rank());
+    cluster_sync();  // every CTA of the cluster is done with its K/V ring
     if (warp >= 2) {
-      const int S = p.max_splits;
-      const int q = static_cast<int>(cluster_rank());
-      const int tid = threadIdx.x - 64;
-      const float* so = reinterpret_cast<const float*>(smem);
-      const float2* sml = reinterpret_cast<const float2*>(smem + C::kCombOffML);
-      float* wsc = reinterpret_cast<float*>(smem + C::kCombOffW);  // [64 / S rows][S]
-      const int my_rows = (p.R - q + S - 1) / S;                   // rows q, q + S, ...
-      // per-row weights 2^(m_p - M) / L of the S pieces
-      if (tid < my_rows) {
-        const int r = q + tid * S;
-        float mp[8], lp[8], M = -INFINITY;
-        for (int s = 0; s < S; ++s) {
-          const float4 t = ld_peer_f4(sml + (r & ~1), static_cast<uint32_t>(s));
-          mp[s] = (r & 1) ? t.z : t.x;
-          lp[s] = (r & 1) ? t.w : t.y;
-          M = fmaxf(M, mp[s]);
+      float* recv = reinterpret_cast<float*>(smem);                  // [slot][D + 8]
+      float2* recv_ml = reinterpret_cast<float2*>(smem + C::kCombOffML);
+      const int r0 = 16 * (warp & 3) + (lane >> 2);
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int r = r0 + 8 * hh;
+        if (r >= p.R) continue;
+        const uint32_t owner = static_cast<uint32_t>(r % S);
+        const int slot = (r / S) * S + q;
+#pragma unroll
+        for (int db = 0; db < D / 8; ++db) {
+          const int d = db * 8 + 2 * (lane & 3);
+          st_peer_f2(recv + slot * (D + 8) + d, owner, o[db][2 * hh], o[db][2 * hh + 1]);
         }
-        float L = 0.f;
-        for (int s = 0; s < S; ++s) {
-          mp[s] = mp[s] == -INFINITY ? 0.f : exp2f(mp[s] - M);
-          L += lp[s] * mp[s];
-        }
-        const float inv = 1.f / L;
-        for (int s = 0; s < S; ++s) wsc[tid * 8 + s] = mp[s] * inv;
+        if ((lane & 3) == 0) st_peer_f2(recv_ml + slot, owner, m_fin[hh], l_fin[hh]);
       }
-      named_bar_sync(2, 128);
+    }
+    cluster_sync();  // every push has landed
+    if (warp >= 2) {
+      const float* recv = reinterpret_cast<const float*>(smem);
+      const float2* recv_ml = reinterpret_cast<const float2*>(smem + C::kCombOffML);
+      const int tid = threadIdx.x - 64;
+      const int my_rows = (p.R - q + S - 1) / S;  // rows q, q + S, ...
       for (int item = tid; item < my_rows * (D / 4); item += 128) {
         const int lr = item / (D / 4), d = (item - lr * (D / 4)) * 4;
         const int r = q + lr * S;
+        float M = -INFINITY;
+        for (int src = 0; src < S; ++src) M = fmaxf(M, recv_ml[lr * S + src].x);
+        float L = 0.f;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int s = 0; s < S; ++s) {
-          const float w = wsc[lr * 8 + s];
-          const float4 t = ld_peer_f4(so + r * (D + 8) + d, static_cast<uint32_t>(s));
+        for (int src = 0; src < S; ++src) {
+          const float2 ml = recv_ml[lr * S + src];
+          const float w = ml.x == -INFINITY ? 0.f : exp2f(ml.x - M);
+          L += w * ml.y;
+          const float4 t = *reinterpret_cast<const float4*>(recv + (lr * S + src) * (D + 8) + d);
           acc.x += w * t.x;
           acc.y += w * t.y;
           acc.z += w * t.z;
           acc.w += w * t.w;
         }
+        const float inv = 1.f / L;
         const int i = r / p.G, g = r - (r / p.G) * p.G;
         f16* dst = p.o + (static_cast<size_t>(b * p.bs + i) * p.Hq + h * p.G + g) * D + d;
-        *reinterpret_cast<uint2*>(dst) = make_uint2(pack_f16x2(acc.x, acc.y), pack_f16x2(acc.z, acc.w));
+        *reinterpret_cast<uint2*>(dst) =
+            make_uint2(pack_f16x2(acc.x * inv, acc.y * inv), pack_f16x2(acc.z * inv, acc.w * inv));
       }
     }
-    cluster_sync();  // no CTA leaves while a peer may still read its shared memory
   }
 
   tc_fence_before();

@@ -86,8 +86,12 @@ struct GemmPlan {
 // rounded up to 16 (multiples of 8 rows keep every slot 1024-byte aligned).
 int gemm_a_rows(int M) { return M >= kGemmBM ? kGemmBM : std::max(16, (M + 15) / 16 * 16); }
 
+// Few-row (staged) GEMMs keep 4 stages in flight: measured on the Qwen3-8B
+// draft step, 4 stages stream the weights faster than 5 or 6 (and 2 or 3).
+constexpr int kGemmStagedStages = 4;
+
 int gemm_stages(int a_rows, int bn) {
-  int st = kGemmMaxStages;
+  int st = gemm_staged(a_rows) ? kGemmStagedStages : kGemmMaxStages;
   while (st > 2 && gemm_smem_bytes(a_rows, bn, st) > kGemmSmemLimit) --st;
   return st;
 }
@@ -114,11 +118,14 @@ GemmPlan plan_gemm(int M, int N, int K, int group, int num_sms, int force_bn = 0
   pl.BN = force_bn ? force_bn : 256;
   if (pl.BN < group || pl.BN % group) pl.BN = 256;
   const bool one_m_tile = pl.m_tiles == 1;
-  if (one_m_tile) {
-    // the staged epilogue (M <= 32) frees the accumulator as soon as it is
-    // copied out, so one buffer suffices there
+  if (M <= kGemmStagedRows) {
+    // staged epilogue: the accumulator is copied out at once (one buffer); the
+    // weight stream, not the MMA chain, paces these tiles (one chain)
+    pl.nacc = 1;
+    pl.nbuf = 1;
+  } else if (one_m_tile) {
     pl.nacc = pl.BN >= 256 ? 2 : 4;
-    pl.nbuf = (M > kGemmStagedRows && 2 * pl.nacc * pl.BN <= 512) ? 2 : 1;
+    pl.nbuf = (2 * pl.nacc * pl.BN <= 512) ? 2 : 1;
   } else {
     pl.nacc = pl.BN >= 256 ? 1 : pl.BN >= 128 ? 2 : 4;
     pl.nbuf = 2;

@@ -164,6 +164,12 @@ __device__ __forceinline__ float4 ld_peer_f4(const void* p, uint32_t rank) {
   return v;
 }
 
+__device__ __forceinline__ void st_peer_f2(void* p, uint32_t rank, float x, float y) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(p)), "r"(rank));
+  asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(remote), "f"(x), "f"(y) : "memory");
+}
+
 __device__ __forceinline__ void cta_sync() {
   __syncwarp();
   __syncthreads();

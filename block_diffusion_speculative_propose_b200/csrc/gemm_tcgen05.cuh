@@ -219,6 +219,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int lane = threadIdx.x & 31;
   pdl_trigger();
 
+  // The weights are never written by an earlier kernel: thread 0 (the TMA
+  // producer) requests the W tiles of the first `stages` k-blocks right after
+  // the barriers exist — before the tensor-memory allocation, which may wait
+  // for a co-resident CTA of the previous kernel to free its columns, and
+  // before waiting for the grid that produces A.  Fresh stages need no
+  // empty-slot wait.
+  int pre = 0;
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) {
       mbar_init(&full[s], 1);
@@ -231,6 +238,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     fence_barrier_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmW);
+    const uint64_t pol_w = policy_evict_first();
+    GemmSegIter it0(p);
+    GemmSeg s0;
+    while (pre < stages && it0.next(p, s0)) {
+      for (int kb = s0.kb0; kb < s0.kb1 && pre < stages; ++kb, ++pre) {
+        mbar_arrive_expect_tx(&full[pre], stage_tx);
+        tma_load_2d_hint(sB + pre * C::kBBytes, &tmW, &full[pre], w_x(p, kb),
+                         w_y<BN>(p, s0.n_tile, kb), pol_w);
+      }
+    }
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, static_cast<uint32_t>(p.tmem_cols));
@@ -247,21 +264,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (lane == 0) {
       const uint64_t pol_w = policy_evict_first();
       const uint64_t pol_a = policy_evict_last();
-      // The weights are never written by an earlier kernel: the W tiles of the
-      // first `stages` k-blocks are requested before waiting for the grid that
-      // produces A (the fresh stages need no empty-slot wait).
-      int pre = 0;
-      {
-        GemmSegIter it0(p);
-        GemmSeg s0;
-        while (pre < stages && it0.next(p, s0)) {
-          for (int kb = s0.kb0; kb < s0.kb1 && pre < stages; ++kb, ++pre) {
-            mbar_arrive_expect_tx(&full[pre], stage_tx);
-            tma_load_2d_hint(sB + pre * C::kBBytes, &tmW, &full[pre], w_x(p, kb),
-                             w_y<BN>(p, s0.n_tile, kb), pol_w);
-          }
-        }
-      }
       pdl_wait();
       uint32_t stage = 0, phase = 0;
       int idx = 0;
@@ -557,12 +559,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (p.cluster_s > 1) {
     // Every thread of every CTA of the cluster reaches both barriers exactly
     // once (no early exits above, all waits bounded).  Between them, CTA rank q
-    // reduces the column groups g = q, q + S, ... of the tile over the S
-    // staging tiles in rank order (deterministic) and runs the epilogue.
+    // owns the column groups g = q, q + S, ... of the tile: first all 128
+    // epilogue threads sum, per float4 of those groups, the S staging tiles in
+    // rank order (deterministic; S independent peer loads in flight per
+    // thread) into this CTA's own staging tile — peers only read the groups
+    // they own, never these — then each (row, group) item runs the epilogue.
     cluster_sync();
     if (warp >= 2) {
       constexpr int LD = BN + 4;
       constexpr int NG = BN / G;
+      constexpr int GF4 = G / 4;
       const int S = p.cluster_s;
       const int rank = static_cast<int>(cluster_rank());
       const int tile = blockIdx.x / S;
@@ -570,25 +576,41 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int rows = p.M;
       const int my_groups = (NG - rank + S - 1) / S;
       const int tid = threadIdx.x - 64;
+      for (int it = tid; it < my_groups * rows * GF4; it += 128) {
+        const int c4 = it % GF4, rest = it / GF4;
+        const int r = rest % rows, lg = rest / rows;
+        float* src = staging + r * LD + (rank + lg * S) * G + c4 * 4;
+        float4 t[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          if (q < S) t[q] = ld_peer_f4(src, static_cast<uint32_t>(q));
+        float4 acc = t[0];
+#pragma unroll
+        for (int q = 1; q < 8; ++q) {
+          if (q < S) {
+            acc.x += t[q].x;
+            acc.y += t[q].y;
+            acc.z += t[q].z;
+            acc.w += t[q].w;
+          }
+        }
+        *reinterpret_cast<float4*>(src) = acc;
+      }
+      named_bar_sync(1, 128);
       for (int item = tid; item < my_groups * rows; item += 128) {
         const int lg = item / rows, r = item - lg * rows;
         const int g = rank + lg * S;
         const int n0 = n_tile * BN + g * G;
         if (n0 >= p.N) continue;
         float v[G];
-#pragma unroll
-        for (int j = 0; j < G; ++j) v[j] = 0.f;
         const float* src = staging + r * LD + g * G;
-#pragma unroll 1
-        for (int q = 0; q < S; ++q) {
 #pragma unroll
-          for (int j = 0; j < G; j += 4) {
-            const float4 t = ld_peer_f4(src + j, static_cast<uint32_t>(q));
-            v[j] += t.x;
-            v[j + 1] += t.y;
-            v[j + 2] += t.z;
-            v[j + 3] += t.w;
-          }
+        for (int j = 0; j < G; j += 4) {
+          const float4 q4 = *reinterpret_cast<const float4*>(src + j);
+          v[j] = q4.x;
+          v[j + 1] = q4.y;
+          v[j + 2] = q4.z;
+          v[j + 3] = q4.w;
         }
         typename Epi::State st;
         epi.begin(st);
