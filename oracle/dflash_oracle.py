@@ -248,6 +248,73 @@ def paged_slots(positions, req_ids, block_table, page_size: int) -> np.ndarray:
 
 
 @dataclass
+class ProposalInputs:
+    positions: np.ndarray      # [n] corrected context positions (int64)
+    slot_mapping: np.ndarray   # [n] context slots, -1 for trailing padding rows (int64)
+    req_ids: np.ndarray        # [n] request of each row, -1 for padding (int64)
+    seq_lens: np.ndarray       # [B] post-verify sequence lengths (int64)
+    bonus: np.ndarray          # [B] bonus tokens (int64)
+
+
+def _valid_count(sampled, vocab: int) -> np.ndarray:
+    """Per request, the sampler outputs that are real tokens: != -1 and
+    < vocab ([NEURON] "Async Rejection and Position Correction")."""
+    s = np.asarray(sampled, dtype=np.int64)
+    return np.sum((s != -1) & (s < vocab), axis=1)
+
+
+def prepare_proposal_inputs(target_positions, last_token_indices, cur_sampled, cur_num_draft,
+                            block_table, page_size: int, vocab: int, prev_sampled=None,
+                            prev_num_draft=None) -> ProposalInputs:
+    """Device-side proposal-input preparation with the async correction,
+    [NEURON] "Async Rejection and Position Correction", "Paged KV
+    Integration" and "Draft Block Construction", in the pages' order:
+
+    1. the request of each target row follows from last_token_indices (rows
+       of request b end at last_token_indices[b]; rows past the last
+       request's end are trailing padding);
+    2. _correct_target_positions_for_async: prev_num_rejected =
+       (1 + prev_num_draft_tokens) - prev_valid_count, subtracted from each
+       row's optimistic position (no previous step: no correction);
+    3. _current_seq_lens: the post-verify length removes this step's
+       rejected positions from the optimistic length (the request's last
+       corrected position + 1), using cur_num_draft_tokens;
+    4. the bonus token is the last valid rejection-sampler output;
+    5. context slots from the paged-slot formula, -1 for padding rows."""
+    pos_in = np.asarray(target_positions, dtype=np.int64)
+    last = np.asarray(last_token_indices, dtype=np.int64)
+    n, B = pos_in.shape[0], last.shape[0]
+    req = np.full(n, -1, dtype=np.int64)
+    start = 0
+    for b in range(B):
+        for r in range(start, last[b] + 1):
+            req[r] = b
+        start = last[b] + 1
+    if prev_sampled is None:
+        prev_rej = np.zeros(B, dtype=np.int64)
+    else:
+        prev_rej = (1 + np.asarray(prev_num_draft, dtype=np.int64)) - _valid_count(prev_sampled,
+                                                                                    vocab)
+    pos = pos_in.copy()
+    for r in range(n):
+        if req[r] >= 0:
+            pos[r] = pos_in[r] - prev_rej[req[r]]
+    cur = np.asarray(cur_sampled, dtype=np.int64)
+    cur_rej = (1 + np.asarray(cur_num_draft, dtype=np.int64)) - _valid_count(cur, vocab)
+    seq_lens = np.array([pos[last[b]] + 1 - cur_rej[b] for b in range(B)], dtype=np.int64)
+    bonus = np.full(B, -1, dtype=np.int64)
+    for b in range(B):
+        for j in range(cur.shape[1]):
+            if cur[b, j] != -1 and cur[b, j] < vocab:
+                bonus[b] = cur[b, j]
+    slots = np.full(n, -1, dtype=np.int64)
+    live = req >= 0
+    if live.any():
+        slots[live] = paged_slots(pos[live], req[live], block_table, page_size)
+    return ProposalInputs(pos, slots, req, seq_lens, bonus)
+
+
+@dataclass
 class QueryBlock:
     input_ids: np.ndarray         # [B * bs]
     positions: np.ndarray         # [B * bs]
