@@ -48,7 +48,7 @@ TRAFFIC = {
     # gate/up GEMM of the batch-1 Qwen3-8B-shaped step: 201.55 MB read + 3.55 MB written
     # (ncu --set full, profiles/gemm_gate_up_qwen3_b1_ctx2048.md)
     ("qwen3_b1_ctx2048", "gemm_gate_up"): {"bytes_per_launch": 205106688,
-                                           "digest": "b23c2b028c04627c"},
+                                           "digest": "04b44d4801a112eb"},
 }
 
 
@@ -69,11 +69,17 @@ def parse_args():
     return a
 
 
-def source_digest() -> str:
+# Sources a kernel family is compiled from (its traffic figure is void once
+# any of them changes).
+FAMILY_SOURCES = {"gemm": ("gemm_tcgen05.cuh", "dflash_device.cuh"),
+                  "attention": ("attention_tc.cuh", "attention.cuh", "dflash_device.cuh")}
+
+
+def source_digest(family: str = "gemm") -> str:
     h = hashlib.sha256()
-    for p in sorted(glob.glob(os.path.join(ROOT, "block_diffusion_speculative_propose_b200",
-                                           "csrc", "*"))):
-        h.update(open(p, "rb").read())
+    for name in FAMILY_SOURCES["attention" if family == "attention" else "gemm"]:
+        h.update(open(os.path.join(ROOT, "block_diffusion_speculative_propose_b200", "csrc",
+                                   name), "rb").read())
     return h.hexdigest()[:16]
 
 
@@ -323,6 +329,80 @@ class GpuStep:
         return None
 
 
+def graph_seconds(fn, dev, reps: int = 10, iters: int = 5) -> float:
+    """Device seconds per call of `fn`, replayed from a CUDA graph of `reps`
+    calls (so host launch cost is excluded), median-free mean over `iters`."""
+    fn()
+    torch.cuda.synchronize(dev)
+    s = torch.cuda.Stream(device=dev)
+    s.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(s):
+        fn()
+    torch.cuda.synchronize(dev)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(reps):
+            fn()
+    g.replay()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(iters):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize(dev)
+    del g
+    return e0.elapsed_time(e1) / 1e3 / (iters * reps)
+
+
+def roof_of(byts: float, flops: float, seconds: float, peaks: dict) -> dict:
+    """Roofline fraction of work (bytes, flops) done in `seconds`: against the
+    slower of the HBM time and the tensor time (measured peaks)."""
+    t_hbm = byts / (peaks["hbm_gbs"] * 1e9)
+    tc = peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"]
+    t_tc = flops / (tc * 1e12)
+    bound = "tensor" if t_tc > t_hbm else "hbm"
+    return {"bound": bound, "roofline_us": max(t_hbm, t_tc) * 1e6, "us": seconds * 1e6,
+            "frac": max(t_hbm, t_tc) / seconds if seconds > 0 else None,
+            "algorithmic_bytes": byts, "algorithmic_flops": flops}
+
+
+def extra_measurements(st, peaks) -> dict:
+    """Sub-measurements of the same workload: the prefill injection of the
+    first request's whole context (batch-1 workloads) and the device-side
+    proposal-input preparation at the workload's batch."""
+    from block_diffusion_speculative_propose_b200 import paged_slots, prepare_proposal_inputs
+    c, dev, out = st.cfg, st.dev, {}
+    H, L, Hkv, d, T = (c["hidden"], c["n_layers"], c["n_kv_heads"], c["head_dim"],
+                       c["n_target_layers"])
+    if st.B == 1:
+        n = int(st.sb.ctx_lens[0])
+        g = torch.Generator(device=dev)
+        g.manual_seed(11)
+        aux = torch.randn(n, T * H, generator=g, device=dev).to(torch.bfloat16)
+        pos = torch.arange(n, dtype=torch.int64, device=dev)
+        req = torch.zeros(n, dtype=torch.int64, device=dev)
+        slots = paged_slots(pos, req, st.inp["block_table"], c["page_size"])
+        ws = torch.empty(st.h.inject_workspace_bytes(n), dtype=torch.uint8, device=dev)
+        t = graph_seconds(lambda: st.h.inject_context(aux, pos, slots, st.kc, st.vc,
+                                                       workspace=ws), dev, reps=4)
+        byts = 2.0 * (H * T * H + L * 2 * Hkv * d * H) + n * (T * H * 2 + L * 2 * Hkv * d * 2)
+        flops = 2.0 * n * (T * H * H + H * L * 2 * Hkv * d)
+        out["prefill_inject"] = dict(rows=n, **roof_of(byts, flops, t, peaks))
+        del aux, ws
+    K, B = st.K, st.B
+    starts = st.sb.seq_lens.to(torch.int64).to(dev)
+    tp = (starts[:, None] + torch.arange(K + 1, device=dev)[None, :]).reshape(-1)
+    last = ((torch.arange(B, device=dev) + 1) * (K + 1) - 1).to(torch.int32)
+    nd = torch.full((B,), K, dtype=torch.int32, device=dev)
+    ver = st.out["ver_tokens"]
+    t = graph_seconds(lambda: prepare_proposal_inputs(tp, last, ver, nd, st.inp["block_table"],
+                                                      c["page_size"], c["vocab"], ver, nd),
+                      dev, reps=20)
+    out["prepare_proposal_inputs"] = {"rows": int(tp.numel()), "us": t * 1e6}
+    return out
+
+
 def run_ours(a, rank, world, local):
     peaks, peaks_src = load_peaks()
     st = GpuStep(a.workload, local, shard_seed(a.seed, rank))
@@ -420,10 +500,25 @@ def run_ours(a, rank, world, local):
         roof = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s",
                 "frac": ach / peak}
     tr = TRAFFIC.get((a.workload, dom))
-    roof.update({"traffic": tr["bytes_per_launch"] if tr and tr["digest"] == source_digest()
+    roof.update({"traffic": tr["bytes_per_launch"] if tr and tr["digest"] == source_digest(dom)
                  else None, "kernel": dom, "algorithmic_bytes_per_launch": byts,
                  "algorithmic_flops_per_launch": flops, "launch_ms": per_launch_s * 1e3,
                  "peak_source": f"{peaks_src} ({'sustained bf16' if roof['bound'] == 'tensor' else 'HBM copy'})"})
+
+    # per-kernel and whole-step rooflines (event-bracketed launch times)
+    step_b, step_f = 0.0, 0.0
+    for k, v in shares.items():
+        alg_k = st.algorithmic(k)
+        if alg_k is None or v["launches_per_step"] <= 0:
+            continue
+        per = v["ms_per_step"] / 1e3 / v["launches_per_step"]
+        r = roof_of(alg_k[0], alg_k[1], per, peaks)
+        v.update({"bound": r["bound"], "frac": r["frac"],
+                  "algorithmic_bytes_per_launch": alg_k[0]})
+        step_b += alg_k[0] * v["launches_per_step"]
+        step_f += alg_k[1] * v["launches_per_step"]
+    step_roof = roof_of(step_b, step_f, t_step, peaks)
+    extras = extra_measurements(st, peaks) if rank == 0 else {}
 
     assert st.h.check_device_errors() == 0, "device error flags raised"
 
@@ -440,7 +535,9 @@ def run_ours(a, rank, world, local):
                    "l2": "inputs larger than L2: every step streams the draft weights "
                          f"({weight_bytes(st.cfg) / 1e9:.2f} GB) and the KV context"},
         "roofline": roof,
+        "step_roofline": step_roof,
         "kernels": shares,
+        "extras": extras,
         "gpu_launches": launches * a.steps,
         "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
         "clock_samples": clocks["samples"],

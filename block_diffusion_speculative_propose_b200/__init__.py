@@ -6,4 +6,5 @@ synthetic-input generator used by the tests and the benchmark.
 """
 
 from .dflash import (DFlash, DFlashError, Workspace, lib, paged_slots,  # noqa: F401
-                     status_string, verify_greedy, verify_workspace_bytes, version)
+                     prepare_proposal_inputs, status_string, verify_greedy,
+                     verify_workspace_bytes, version)

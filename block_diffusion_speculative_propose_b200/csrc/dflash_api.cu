@@ -1114,6 +1114,34 @@ dflash_status dflash_paged_slots(const int64_t* positions, const int64_t* req_id
   return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ERR_CUDA;
 }
 
+dflash_status dflash_prepare_proposal_inputs(
+    const int64_t* target_positions, int n, const int32_t* last_token_indices, int B,
+    const int32_t* cur_sampled, int cur_width, const int32_t* cur_num_draft,
+    const int32_t* prev_sampled, int prev_width, const int32_t* prev_num_draft,
+    const int32_t* block_table, int max_pages_per_seq, int page_size, int vocab,
+    int64_t* positions_out, int64_t* slot_mapping_out, int32_t* seq_lens_out,
+    int32_t* bonus_out, unsigned* device_error, void* stream) {
+  if (n < 0 || B < 0 || cur_width < 1 || max_pages_per_seq < 1 || page_size < 1 || vocab < 1)
+    return DFLASH_ERR_INVALID_ARG;
+  if ((prev_sampled == nullptr) != (prev_num_draft == nullptr)) return DFLASH_ERR_INVALID_ARG;
+  if (prev_sampled && prev_width < 1) return DFLASH_ERR_INVALID_ARG;
+  if (n == 0 && B == 0) return DFLASH_OK;
+  if ((n > 0 && (!target_positions || !positions_out || !slot_mapping_out)) ||
+      (B > 0 && (!cur_sampled || !cur_num_draft || !seq_lens_out || !bonus_out ||
+                 !last_token_indices || !block_table)))
+    return DFLASH_ERR_INVALID_ARG;
+  dflash_status s = set_device_for(static_cast<cudaStream_t>(stream),
+                                   n > 0 ? static_cast<const void*>(positions_out)
+                                         : static_cast<const void*>(seq_lens_out));
+  if (s != DFLASH_OK) return s;
+  launch_k(pdl_default(), prepare_proposal_kernel, dim3(cdiv(std::max(n, B), 256)), dim3(256), 0,
+           static_cast<cudaStream_t>(stream), target_positions, n, last_token_indices, B,
+           cur_sampled, cur_width, cur_num_draft, prev_sampled, prev_sampled ? prev_width : 1,
+           prev_num_draft, block_table, max_pages_per_seq, page_size, vocab, positions_out,
+           slot_mapping_out, seq_lens_out, bonus_out, device_error);
+  return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ERR_CUDA;
+}
+
 dflash_status dflash_inject_context(dflash_handle* h, const void* aux, const int64_t* positions,
                                     const int64_t* slot_mapping, int n, void* const* k_cache,
                                     void* const* v_cache, int num_pages, void* workspace,

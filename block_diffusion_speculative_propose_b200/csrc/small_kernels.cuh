@@ -246,6 +246,75 @@ __global__ void paged_slots_kernel(const int64_t* __restrict__ pos,
 }
 
 // In-place bf16 -> fp16 conversion of weights (exact in fp16's normal range).
+// Proposal-input preparation with the async rejection correction: threads
+// r < n handle target rows, threads b < B handle requests; nothing is shared
+// between threads (each recomputes the few per-request counts it needs).
+__device__ __forceinline__ int count_valid(const int32_t* s, int width, int vocab) {
+  int c = 0;
+  for (int j = 0; j < width; ++j) c += (s[j] != -1 && s[j] < vocab) ? 1 : 0;
+  return c;
+}
+
+__global__ void prepare_proposal_kernel(
+    const int64_t* __restrict__ target_positions, int n, const int32_t* __restrict__ last, int B,
+    const int32_t* __restrict__ cur_sampled, int cur_width, const int32_t* __restrict__ cur_num_draft,
+    const int32_t* __restrict__ prev_sampled, int prev_width,
+    const int32_t* __restrict__ prev_num_draft, const int32_t* __restrict__ table, int W, int P,
+    int vocab, int64_t* __restrict__ pos_out, int64_t* __restrict__ slot_out,
+    int32_t* __restrict__ seq_out, int32_t* __restrict__ bonus_out, unsigned* err) {
+  pdl_trigger();
+  pdl_wait();
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  auto prev_rejected = [&](int b) -> int {
+    if (!prev_sampled) return 0;
+    return 1 + prev_num_draft[b] -
+           count_valid(prev_sampled + static_cast<size_t>(b) * prev_width, prev_width, vocab);
+  };
+  if (t < n) {
+    // request of row t: first b with last[b] >= t (binary search)
+    int lo = 0, hi = B;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (last[mid] >= t) hi = mid;
+      else lo = mid + 1;
+    }
+    const int64_t p_in = target_positions[t];
+    if (lo >= B) {
+      pos_out[t] = p_in;      // trailing padding row
+      slot_out[t] = -1;
+    } else {
+      const int64_t p = p_in - prev_rejected(lo);
+      pos_out[t] = p;
+      if (p < 0) {
+        raise_error(err, DFLASH_DEVERR_INPUT);
+        slot_out[t] = -1;
+      } else {
+        const int64_t page_no = min(p / P, static_cast<int64_t>(W - 1));
+        const int64_t block = table[static_cast<int64_t>(lo) * W + page_no];
+        slot_out[t] = block * P + p % P;
+      }
+    }
+  }
+  if (t < B) {
+    const int lt = last[t];
+    if (lt >= n || lt < 0 || (t > 0 && last[t - 1] >= lt)) {
+      raise_error(err, DFLASH_DEVERR_INPUT);
+      seq_out[t] = 0;
+      bonus_out[t] = -1;
+      return;
+    }
+    const int32_t* cs = cur_sampled + static_cast<size_t>(t) * cur_width;
+    const int cur_rej = 1 + cur_num_draft[t] - count_valid(cs, cur_width, vocab);
+    const int64_t last_pos = target_positions[lt] - prev_rejected(t);
+    seq_out[t] = static_cast<int32_t>(last_pos + 1 - cur_rej);
+    int bonus = -1;
+    for (int j = 0; j < cur_width; ++j)
+      if (cs[j] != -1 && cs[j] < vocab) bonus = cs[j];
+    if (bonus == -1) raise_error(err, DFLASH_DEVERR_INPUT);
+    bonus_out[t] = bonus;
+  }
+}
+
 __global__ void bf16_to_f16_kernel(uint16_t* __restrict__ data, size_t n) {
   for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
        i += static_cast<size_t>(gridDim.x) * blockDim.x) {

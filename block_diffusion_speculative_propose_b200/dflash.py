@@ -82,6 +82,8 @@ def lib() -> ctypes.CDLL:
         "dflash_linear_workspace_bytes": ([vp, i32, i32, i32], sz),
         "dflash_attention_workspace_bytes": ([vp, i32, i32], sz),
         "dflash_paged_slots": ([vp, vp, i32, vp, i32, i32, vp, vp], i32),
+        "dflash_prepare_proposal_inputs": ([vp, i32, vp, i32, vp, i32, vp, vp, i32, vp, vp,
+                                            i32, i32, i32, vp, vp, vp, vp, vp, vp], i32),
         "dflash_inject_context": ([vp, vp, vp, vp, i32, _PP, _PP, i32, vp, sz, vp], i32),
         "dflash_propose": ([vp, vp, vp, vp, i32, i32, _PP, _PP, i32, vp, vp, vp, vp, sz, vp],
                            i32),
@@ -386,6 +388,36 @@ def paged_slots(positions, req_ids, block_table, page_size: int = 16, slots=None
                                     int(block_table.shape[1]), page_size, _ptr(slots),
                                     _stream(stream)), "dflash_paged_slots")
     return slots
+
+
+def prepare_proposal_inputs(target_positions, last_token_indices, cur_sampled, cur_num_draft,
+                            block_table, page_size: int, vocab: int, prev_sampled=None,
+                            prev_num_draft=None, device_error=None, stream=None):
+    """Proposal inputs with the async rejection correction on the device
+    (dflash_prepare_proposal_inputs).  Returns (positions, slot_mapping,
+    seq_lens, bonus) ready for DFlash.inject_context / DFlash.propose."""
+    n, B = int(target_positions.shape[0]), int(last_token_indices.shape[0])
+    _want(target_positions, torch.int64, "target_positions")
+    _want(last_token_indices, torch.int32, "last_token_indices")
+    _want(cur_sampled, torch.int32, "cur_sampled")
+    _want(cur_num_draft, torch.int32, "cur_num_draft")
+    _want(block_table, torch.int32, "block_table")
+    if prev_sampled is not None:
+        _want(prev_sampled, torch.int32, "prev_sampled")
+        _want(prev_num_draft, torch.int32, "prev_num_draft")
+    dev = target_positions.device
+    positions = torch.empty(n, dtype=torch.int64, device=dev)
+    slots = torch.empty(n, dtype=torch.int64, device=dev)
+    seq_lens = torch.empty(B, dtype=torch.int32, device=dev)
+    bonus = torch.empty(B, dtype=torch.int32, device=dev)
+    pw = int(prev_sampled.shape[1]) if prev_sampled is not None else 0
+    _check(lib().dflash_prepare_proposal_inputs(
+        _ptr(target_positions), n, _ptr(last_token_indices), B, _ptr(cur_sampled),
+        int(cur_sampled.shape[1]), _ptr(cur_num_draft), _ptr(prev_sampled), pw,
+        _ptr(prev_num_draft), _ptr(block_table), int(block_table.shape[1]), page_size, vocab,
+        _ptr(positions), _ptr(slots), _ptr(seq_lens), _ptr(bonus), _ptr(device_error),
+        _stream(stream)), "dflash_prepare_proposal_inputs")
+    return positions, slots, seq_lens, bonus
 
 
 def status_string(s: int) -> str:

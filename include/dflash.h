@@ -19,6 +19,9 @@
  *                            plus one bonus token; rejected slots are -1
  *                            (§"Async Rejection and Position Correction").
  *   dflash_paged_slots     — §"Paged KV Integration" (_paged_slots helper).
+ *   dflash_prepare_proposal_inputs — §"Async Rejection and Position Correction"
+ *                            (_correct_target_positions_for_async, _current_seq_lens),
+ *                            §"Paged KV Integration", §"Draft Block Construction".
  *
  * Conventions for every call
  *   - All tensor arguments are DEVICE pointers unless stated otherwise; bf16 means
@@ -65,6 +68,7 @@ typedef enum {
 #define DFLASH_DEVERR_TABLE     0x4u  /* position // page_size past the block-table row width   */
 #define DFLASH_DEVERR_TOKEN     0x8u  /* bonus token id outside [0, vocab)                      */
 #define DFLASH_DEVERR_POSITION  0x10u /* position outside [0, max_position) of the RoPE table   */
+#define DFLASH_DEVERR_INPUT     0x20u /* malformed proposal-preparation input (see below)       */
 
 /* Draft-model geometry.  block_size / mask_token_id / target_layer_ids are the
  * fields of the pages' DFlashConfig; the rest is the Qwen3 layer shape.
@@ -192,6 +196,49 @@ dflash_status dflash_paged_slots(const int64_t* positions, const int64_t* req_id
                                  int n, const int32_t* block_table,
                                  int max_pages_per_seq, int page_size,
                                  int64_t* slots, void* stream);
+
+/* Proposal-input preparation on the device, with the async rejection
+ * correction (§"Async Rejection and Position Correction", §"Paged KV
+ * Integration", §"Draft Block Construction"), so that a whole speculative step
+ * (verify -> prepare -> inject -> propose) runs on one stream with no host
+ * round trip.  In the pages' order:
+ *   1. request of target row r: the b with last_token_indices[b-1] < r <=
+ *      last_token_indices[b]; rows past last_token_indices[B-1] are trailing
+ *      padding;
+ *   2. prev_rejected[b] = (1 + prev_num_draft[b]) - #{j : prev_sampled[b][j] != -1
+ *      and prev_sampled[b][j] < vocab}; positions_out[r] = target_positions[r]
+ *      - prev_rejected[req(r)] (prev_sampled == NULL: no previous step, no
+ *      correction);
+ *   3. seq_lens_out[b] = positions_out[last_token_indices[b]] + 1 - cur_rejected[b],
+ *      cur_rejected[b] = (1 + cur_num_draft[b]) - #valid(cur_sampled[b]);
+ *   4. bonus_out[b] = the last valid entry of cur_sampled[b];
+ *   5. slot_mapping_out[r] = the _paged_slots formula at (positions_out[r],
+ *      req(r)) (with the page's clamp); -1 for padding rows (their position is
+ *      copied unchanged).
+ * Inputs (device): target_positions [n] int64; last_token_indices [B] int32,
+ * strictly increasing, < n; cur_sampled [B, cur_width] int32 (the rejection
+ * sampler's output of this step, -1 padded, e.g. out_tokens of
+ * dflash_verify_greedy); cur_num_draft [B] int32; prev_sampled
+ * [B, prev_width] int32 and prev_num_draft [B] int32, both NULL or both set;
+ * block_table [B, max_pages_per_seq] int32.  Outputs (device, caller-owned):
+ * positions_out, slot_mapping_out [n] int64; seq_lens_out, bonus_out [B]
+ * int32 — ready for dflash_inject_context (positions, slots) and
+ * dflash_propose (bonus_tokens, seq_lens).
+ * Host errors (DFLASH_ERR_INVALID_ARG) before any launch: n < 0, B < 0,
+ * widths < 1, page_size < 1, vocab < 1, a missing pointer (the per-request
+ * ones and the block table may be NULL only when B == 0: every row is then
+ * padding), prev_sampled / prev_num_draft given alone.  Device errors set DFLASH_DEVERR_INPUT in
+ * *device_error (a device word, nullable) and skip the value: indices not
+ * strictly increasing or past n, a request with no valid sampler output
+ * (bonus_out = -1), a corrected position < 0 (slot -1).  One launch; B == 0
+ * and n == 0 are no-ops. */
+dflash_status dflash_prepare_proposal_inputs(
+    const int64_t* target_positions, int n, const int32_t* last_token_indices, int B,
+    const int32_t* cur_sampled, int cur_width, const int32_t* cur_num_draft,
+    const int32_t* prev_sampled, int prev_width, const int32_t* prev_num_draft,
+    const int32_t* block_table, int max_pages_per_seq, int page_size, int vocab,
+    int64_t* positions_out, int64_t* slot_mapping_out, int32_t* seq_lens_out,
+    int32_t* bonus_out, unsigned* device_error, void* stream);
 
 /* precompute_and_store_context_kv (§"Context KV Injection (Precompute)"):
  *   ctx = hidden_norm(fc(aux))                       [n, H]

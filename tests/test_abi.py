@@ -65,6 +65,28 @@ def test_host_validation_without_gpu(L):
     assert L.dflash_verify_workspace_bytes(0, 15, 151936) == 0
     assert L.dflash_inject_workspace_bytes(None, 16) == 0
     assert L.dflash_propose_workspace_bytes(None, 1, 10) == 0
+    # proposal preparation: (n, B) = (0, 0) is a no-op; bad sizes / pointer
+    # combinations are rejected before any launch
+    prep = L.dflash_prepare_proposal_inputs
+    args = dict(tp=None, n=0, last=None, B=0, cur=None, cw=4, cnd=None, prev=None, pw=0,
+                pnd=None, bt=None, W=4, P=16, V=10, po=None, so=None, sl=None, bo=None,
+                err=None, st=None)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return prep(a["tp"], a["n"], a["last"], a["B"], a["cur"], a["cw"], a["cnd"], a["prev"],
+                    a["pw"], a["pnd"], a["bt"], a["W"], a["P"], a["V"], a["po"], a["so"],
+                    a["sl"], a["bo"], a["err"], a["st"])
+    assert call() == 0
+    assert call(n=-1) == -1
+    assert call(B=-1) == -1
+    assert call(cw=0) == -1
+    assert call(P=0) == -1
+    assert call(V=0) == -1
+    assert call(prev=16) == -1          # prev_sampled without prev_num_draft
+    assert call(pnd=16) == -1
+    assert call(n=4) == -1              # rows without their pointers
+    assert call(B=2) == -1
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
