@@ -500,7 +500,7 @@ dflash_status run_gemm(dflash_handle* h, int kind, bool f16, bool w_packed, cons
   } else if (!h->tmap(&tw, Wt, N, K, pl.BN, f16)) {
     return DFLASH_ERR_CUDA;
   }
-  GemmParams gp;
+  GemmParams gp{};
   gp.M = M;
   gp.N = N;
   gp.K = K;
