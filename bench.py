@@ -316,6 +316,10 @@ class GpuStep:
             return gemm(M, 2 * I, H, M * I * 2)
         if family == "gemm_down":
             return gemm(M, H, I, M * H * 8)
+        if family == "gemm_mlp":     # gate/up + down in one launch (few rows)
+            b1, f1 = gemm(M, 2 * I, H, M * I * 2)
+            b2, f2 = gemm(M, H, I, M * H * 8)
+            return b1 + b2, f1 + f2
         if family == "gemm_lm_head":
             return gemm(MK, V, H, MK * 8)
         if family == "gemm_fc":

@@ -139,7 +139,7 @@ GemmPlan plan_gemm(int M, int N, int K, int group, int num_sms, int force_bn = 0
   bool sk = one_m_tile ? fill < 0.9 : 2 * pl.tiles < num_sms;
   if (force_splits == 1) sk = false;
   if (force_splits >= 2) sk = true;
-  if (sk && pl.tiles > kCounterSlots) sk = false;
+  if (sk && pl.tiles > kCounterSlots - 2) sk = false;   // the last 2 slots: chain arrivals
   pl.total_iters = pl.tiles * pl.k_blocks;
   pl.a_rows = gemm_a_rows(M);
   if (!force_splits && cluster_cap && gemm_staged(pl.a_rows) && pl.tiles <= num_sms) {
@@ -292,6 +292,14 @@ struct dflash_handle {
   // hot-path kernels are launched with programmatic dependent launch (the
   // environment variable DFLASH_PDL=0 turns it off)
   bool pdl = pdl_default();
+  // few-row gate/up + down as one chain launch: opt-in (DFLASH_CHAIN=1 when the
+  // handle is created).  Measured on the batch-1 Qwen3-8B-shaped step it is
+  // 1-2% slower than two launches, whose down GEMM already prefetches on the
+  // SMs gate/up leaves free and reduces through clusters.
+  bool chain = [] {
+    const char* e = std::getenv("DFLASH_CHAIN");
+    return e && e[0] == '1';
+  }();
   std::vector<cudaEvent_t> prof_events;
   size_t prof_next = 0;
   std::vector<int> prof_kind;
@@ -489,7 +497,7 @@ dflash_status run_gemm(dflash_handle* h, int kind, bool f16, bool w_packed, cons
     const int* cap = gemm_cluster_caps<Epi>(h, pl.BN, pl.smem);
     if (cap) pl = plan_gemm(M, N, K, Epi::kGroup, h->num_sms, force_bn, force_splits, cap);
   }
-  if (pl.stream_k && pl.tiles > kCounterSlots) return DFLASH_ERR_UNSUPPORTED_SHAPE;
+  if (pl.stream_k && pl.tiles > kCounterSlots - 2) return DFLASH_ERR_UNSUPPORTED_SHAPE;
   if (pl.partial_bytes > partial_cap) return DFLASH_ERR_WORKSPACE;
   CUtensorMap ta, tw;
   if (!h->tmap(&ta, A, M, K, pl.a_rows, f16)) return DFLASH_ERR_CUDA;
@@ -540,6 +548,83 @@ dflash_status run_gemm(dflash_handle* h, int kind, bool f16, bool w_packed, cons
     default:
       return DFLASH_ERR_UNSUPPORTED_SHAPE;
   }
+  return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ERR_CUDA;
+}
+
+// Phase parameters of one GEMM of a chain launch (packed weights).
+template <class Epi>
+bool chain_phase(dflash_handle* h, const GemmPlan& pl, bool f16, const void* A, int M, int K,
+                 const void* Wt, int N, float* partials, unsigned* counters, CUtensorMap* ta,
+                 CUtensorMap* tw, GemmParams* gp) {
+  if (!h->tmap(ta, A, M, K, pl.a_rows, f16)) return false;
+  if (!h->tmap(tw, Wt, static_cast<uint64_t>(pl.n_tiles) * pl.k_blocks * kPackRows, kGemmBK,
+               kPackRows, f16))
+    return false;
+  *gp = GemmParams{};
+  gp->M = M;
+  gp->N = N;
+  gp->K = K;
+  gp->m_tiles = pl.m_tiles;
+  gp->n_tiles = pl.n_tiles;
+  gp->k_blocks = pl.k_blocks;
+  gp->tiles = pl.tiles;
+  gp->stream_k = pl.stream_k;
+  gp->cluster_s = 1;
+  gp->ipc = pl.ipc;
+  gp->total_iters = pl.total_iters;
+  gp->nacc = pl.nacc;
+  gp->nbuf = pl.nbuf;
+  gp->tmem_cols = pl.tmem_cols;
+  gp->a_rows = pl.a_rows;
+  gp->stages = pl.stages;
+  gp->f16 = f16 ? 1 : 0;
+  gp->w_packed = 1;
+  gp->slot_rows = pl.slot_rows;
+  gp->partials = partials;
+  gp->counters = counters;
+  gp->err = h->dev_err;
+  return true;
+}
+
+// True when two few-row GEMMs (packed weights) can run as one chain launch:
+// the staged epilogue on both sides with the same tile shape and ring.
+bool chain_ok(int M, int num_sms) {
+  return gemm_staged(gemm_a_rows(M)) && M > 0 && num_sms > 0;
+}
+
+// Phase 1: D1 = A1 W1^T with epilogue e1 (whole tiles, one per CTA, when they
+// occupy at least half of the SMs; else stream-K); phase 2: D2 = A2 W2^T with
+// e2 (stream-K), A2 written by phase 1.  One launch of one CTA per SM.
+template <class Epi1, class Epi2>
+dflash_status run_gemm_chain(dflash_handle* h, int kind, bool f16_1, const void* A1, int M,
+                             int K1, const void* W1, int N1, const Epi1& e1, bool f16_2,
+                             const void* A2, int K2, const void* W2, int N2, const Epi2& e2,
+                             float* partials, size_t partial_cap, cudaStream_t st) {
+  if (!chain_ok(M, h->num_sms)) return DFLASH_ERR_UNSUPPORTED_SHAPE;
+  const int t1 = cdiv(N1, kPackRows);
+  GemmPlan pl1 = plan_gemm(M, N1, K1, Epi1::kGroup, h->num_sms, kPackRows,
+                           2 * t1 >= h->num_sms && t1 <= h->num_sms ? 1 : 0);
+  GemmPlan pl2 = plan_gemm(M, N2, K2, Epi2::kGroup, h->num_sms, kPackRows, 0);
+  if (pl1.a_rows != pl2.a_rows || pl1.stages != pl2.stages || pl1.tmem_cols != pl2.tmem_cols ||
+      pl1.BN != 256 || pl2.BN != 256 || pl1.nbuf != 1 || pl2.nbuf != 1)
+    return DFLASH_ERR_UNSUPPORTED_SHAPE;
+  if (pl1.stream_k && pl2.stream_k &&
+      static_cast<size_t>(pl1.tiles) + pl2.tiles > static_cast<size_t>(kCounterSlots - 2))
+    return DFLASH_ERR_UNSUPPORTED_SHAPE;
+  const int grid = h->num_sms;
+  const size_t part = static_cast<size_t>(grid) * 2 * std::min(M, kGemmBM) * 256 * 4;
+  if ((pl1.stream_k || pl2.stream_k) && part > partial_cap) return DFLASH_ERR_WORKSPACE;
+  CUtensorMap ta1, tw1, ta2, tw2;
+  GemmParams g1, g2;
+  if (!chain_phase<Epi1>(h, pl1, f16_1, A1, M, K1, W1, N1, partials, h->counters, &ta1, &tw1,
+                         &g1) ||
+      !chain_phase<Epi2>(h, pl2, f16_2, A2, M, K2, W2, N2, partials,
+                         h->counters + (pl1.stream_k ? pl1.tiles : 0), &ta2, &tw2, &g2))
+    return DFLASH_ERR_CUDA;
+  unsigned* dep = h->counters + kCounterSlots - 2;
+  LaunchScope scope(h, kind, st);
+  launch_k(h->pdl, gemm_chain_kernel<256, Epi1, Epi2>, dim3(grid), dim3(kGemmThreads), pl1.smem,
+           st, ta1, tw1, g1, e1, ta2, tw2, g2, e2, dep);
   return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ERR_CUDA;
 }
 
@@ -803,15 +888,20 @@ dflash_status propose_layers(dflash_handle* h, const ProposeWs& lw, void* ws,
                c.rms_eps, 0, bs);
     }
     if (cudaGetLastError() != cudaSuccess) return DFLASH_ERR_CUDA;
-    // h = silu(gate) * up
+    // h = silu(gate) * up; x += Wd h — one launch for few rows
     EpiSwiGLU eg{hm, I};
-    s = run_gemm(h, DFLASH_KERNEL_GEMM_GATE_UP, true, true, nrm, M, H, h->wgu[l], 2 * I, eg, partial,
-                 lw.partial_cap, st);
-    if (s != DFLASH_OK) return s;
-    // x += Wd h
-    s = run_gemm(h, DFLASH_KERNEL_GEMM_DOWN, false, true, hm, M, I, h->wdown[l], H, er, partial,
-                 lw.partial_cap, st);
-    if (s != DFLASH_OK) return s;
+    if (h->chain && chain_ok(M, h->num_sms)) {
+      s = run_gemm_chain(h, DFLASH_KERNEL_GEMM_MLP, true, nrm, M, H, h->wgu[l], 2 * I, eg, false,
+                         hm, I, h->wdown[l], H, er, partial, lw.partial_cap, st);
+      if (s != DFLASH_OK) return s;
+    } else {
+      s = run_gemm(h, DFLASH_KERNEL_GEMM_GATE_UP, true, true, nrm, M, H, h->wgu[l], 2 * I, eg,
+                   partial, lw.partial_cap, st);
+      if (s != DFLASH_OK) return s;
+      s = run_gemm(h, DFLASH_KERNEL_GEMM_DOWN, false, true, hm, M, I, h->wdown[l], H, er, partial,
+                   lw.partial_cap, st);
+      if (s != DFLASH_OK) return s;
+    }
     LaunchScope scope(h, DFLASH_KERNEL_RMSNORM, st);
     if (l + 1 < c.n_layers) {
       launch_k(h->pdl, rmsnorm_rows_kernel, dim3(M), dim3(256), 0, st, x, h->in_norm_w[l + 1], nrm,
@@ -1061,7 +1151,10 @@ dflash_status dflash_create(const dflash_config* cfg, const dflash_weights* w, i
     return fail_st(DFLASH_ERR_CUDA);
 
   // kernel attributes (set once, outside any stream capture)
-  if (set_gemm_attrs_all<EpiStoreF32>() != cudaSuccess ||
+  if (cudaFuncSetAttribute(gemm_chain_kernel<256, EpiSwiGLU, EpiResidAdd>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           kGemmSmemLimit) != cudaSuccess ||
+      set_gemm_attrs_all<EpiStoreF32>() != cudaSuccess ||
       set_gemm_attrs_all<EpiResidAdd>() != cudaSuccess ||
       set_gemm_attrs_all<EpiSwiGLU>() != cudaSuccess ||
       set_gemm_attrs_all<EpiArgmax>() != cudaSuccess ||
@@ -1405,6 +1498,7 @@ const char* dflash_kernel_name(int kind) {
     case DFLASH_KERNEL_GEMM_FC: return "gemm_fc";
     case DFLASH_KERNEL_GEMM_KV_INJECT: return "gemm_kv_inject";
     case DFLASH_KERNEL_LINEAR: return "linear";
+    case DFLASH_KERNEL_GEMM_MLP: return "gemm_mlp";
   }
   return nullptr;
 }

@@ -187,168 +187,264 @@ __device__ __forceinline__ int w_y(const GemmParams& p, int n_tile, int kb) {
   return p.w_packed ? (n_tile * p.k_blocks + kb) * 256 : n_tile * BN;
 }
 
-template <int BN, class Epi>
-__global__ void __launch_bounds__(kGemmThreads, 1)
-    gemm_tcgen05_kernel(const __grid_constant__ CUtensorMap tmA,
-                        const __grid_constant__ CUtensorMap tmW, const GemmParams p,
-                        const Epi epi) {
-  using C = GemmCfg<BN>;
-  constexpr int G = Epi::kGroup;
-  static_assert(BN % G == 0, "epilogue group must divide the tile width");
+// Shared-memory carve-up, barriers and tensor-memory base of one CTA, common
+// to every phase of a launch.
+template <int BN>
+struct GemmCta {
+  uint8_t* sA;
+  uint8_t* sB;
+  uint64_t* full;
+  uint64_t* empty;
+  uint64_t* tfull;
+  uint64_t* tempty;
+  uint32_t* tmem_slot;
+  volatile int* last_flag;
+  // [2]: verdict of the elected epilogue wait, alternating by segment (a
+  // thread can be at most one segment ahead of the slowest reader)
+  volatile int* wait_flag;
+  float* staging;
+  int stages;
+  int a_bytes;
+  uint32_t stage_tx;
+  uint32_t tmem_base;
+  int acc_cols;   // TMEM columns of one accumulator buffer
+};
 
+// Ring positions of the producer / MMA thread and of the epilogue, carried
+// from one phase of a launch to the next.
+struct GemmRing {
+  uint32_t stage = 0, phase = 0;
+  bool ok = true;
+};
+struct GemmAccRing {
+  uint32_t acc = 0, acc_phase = 0, nseen = 0;
+  bool ok = true;
+};
+
+// Bounded wait until *ctr >= target (acquire): the arrival count of the CTAs
+// of this launch that finished an earlier phase.  Gives up like mbar_wait.
+__device__ __forceinline__ bool wait_count(const unsigned* ctr, unsigned target, unsigned* err) {
+  const long long t0 = clock64();
+  for (unsigned spin = 0;; ++spin) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+    if (v >= target) return true;
+    if ((spin & 63u) == 63u) {
+      if (clock64() - t0 > kWaitLimitCycles) {
+        raise_error(err, DFLASH_DEVERR_TIMEOUT);
+        return false;
+      }
+      if (err && (*reinterpret_cast<volatile unsigned*>(err) & DFLASH_DEVERR_TIMEOUT)) return false;
+    }
+    __nanosleep(64);
+  }
+}
+
+// Barrier init, the first weight stages of phase `p0` (thread 0), tensor-memory
+// allocation (warp 1) and the CTA barrier.  Returns the carve-up; `pre` = the
+// k-blocks of p0 whose W tile thread 0 has requested.
+template <int BN>
+__device__ __forceinline__ GemmCta<BN> gemm_setup(const GemmParams& p0, const CUtensorMap* tA,
+                                                  const CUtensorMap* tW, int& pre) {
+  using C = GemmCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  const int stages = p.stages;
-  const int a_bytes = p.a_rows * 128;
-  const uint32_t stage_tx = static_cast<uint32_t>(a_bytes + C::kBBytes);
-  uint8_t* sA = smem;
-  uint8_t* sB = smem + stages * a_bytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + stages * C::kBBytes);
-  uint64_t* empty = full + kGemmMaxStages;
-  uint64_t* tfull = empty + kGemmMaxStages;
-  uint64_t* tempty = tfull + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
-  volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  // [2]: verdict of the elected epilogue wait, alternating by segment (a
-  // thread can be at most one segment ahead of the slowest reader)
-  volatile int* wait_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
-  float* staging = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(full) + kGemmBarrierBytes);
-
+  GemmCta<BN> S;
+  S.stages = p0.stages;
+  S.a_bytes = p0.a_rows * 128;
+  S.stage_tx = static_cast<uint32_t>(S.a_bytes + C::kBBytes);
+  S.sA = smem;
+  S.sB = smem + S.stages * S.a_bytes;
+  S.full = reinterpret_cast<uint64_t*>(S.sB + S.stages * C::kBBytes);
+  S.empty = S.full + kGemmMaxStages;
+  S.tfull = S.empty + kGemmMaxStages;
+  S.tempty = S.tfull + 2;
+  S.tmem_slot = reinterpret_cast<uint32_t*>(S.tempty + 2);
+  S.last_flag = reinterpret_cast<volatile int*>(S.tmem_slot + 1);
+  S.wait_flag = reinterpret_cast<volatile int*>(S.tmem_slot + 2);
+  S.staging = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(S.full) + kGemmBarrierBytes);
+  S.acc_cols = p0.nacc * BN;
   const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  pdl_trigger();
-
   // The weights are never written by an earlier kernel: thread 0 (the TMA
   // producer) requests the W tiles of the first `stages` k-blocks right after
   // the barriers exist — before the tensor-memory allocation, which may wait
   // for a co-resident CTA of the previous kernel to free its columns, and
   // before waiting for the grid that produces A.  Fresh stages need no
   // empty-slot wait.
-  int pre = 0;
+  pre = 0;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < stages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+    for (int s = 0; s < S.stages; ++s) {
+      mbar_init(&S.full[s], 1);
+      mbar_init(&S.empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
-      mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 4);
+      mbar_init(&S.tfull[a], 1);
+      mbar_init(&S.tempty[a], 4);
     }
     fence_barrier_init();
-    tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmW);
+    tma_prefetch_desc(tA);
+    tma_prefetch_desc(tW);
     const uint64_t pol_w = policy_evict_first();
-    GemmSegIter it0(p);
+    GemmSegIter it0(p0);
     GemmSeg s0;
-    while (pre < stages && it0.next(p, s0)) {
-      for (int kb = s0.kb0; kb < s0.kb1 && pre < stages; ++kb, ++pre) {
-        mbar_arrive_expect_tx(&full[pre], stage_tx);
-        tma_load_2d_hint(sB + pre * C::kBBytes, &tmW, &full[pre], w_x(p, kb),
-                         w_y<BN>(p, s0.n_tile, kb), pol_w);
+    while (pre < S.stages && it0.next(p0, s0)) {
+      for (int kb = s0.kb0; kb < s0.kb1 && pre < S.stages; ++kb, ++pre) {
+        mbar_arrive_expect_tx(&S.full[pre], S.stage_tx);
+        tma_load_2d_hint(S.sB + pre * C::kBBytes, tW, &S.full[pre], w_x(p0, kb),
+                         w_y<BN>(p0, s0.n_tile, kb), pol_w);
       }
     }
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, static_cast<uint32_t>(p.tmem_cols));
+    tmem_alloc(S.tmem_slot, static_cast<uint32_t>(p0.tmem_cols));
     tmem_relinquish();
   }
   tc_fence_before();
   cta_sync();
   tc_fence_after();
-  const uint32_t tmem_base = *tmem_slot;
-  const int acc_cols = p.nacc * BN;   // TMEM columns of one accumulator buffer
+  S.tmem_base = *S.tmem_slot;
+  return S;
+}
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      const uint64_t pol_w = policy_evict_first();
-      const uint64_t pol_a = policy_evict_last();
-      pdl_wait();
-      uint32_t stage = 0, phase = 0;
-      int idx = 0;
-      bool ok = true;
-      GemmSegIter it(p);
-      GemmSeg sg;
-      while (ok && it.next(p, sg)) {
-        for (int kb = sg.kb0; kb < sg.kb1; ++kb, ++idx) {
-          if (idx >= pre) {
-            if (!mbar_wait(&empty[stage], phase ^ 1u, p.err)) {
-              ok = false;
-              break;
-            }
-            mbar_arrive_expect_tx(&full[stage], stage_tx);
-            tma_load_2d_hint(sB + stage * C::kBBytes, &tmW, &full[stage], w_x(p, kb),
-                             w_y<BN>(p, sg.n_tile, kb), pol_w);
-          }
-          tma_load_2d_hint(sA + stage * a_bytes, &tmA, &full[stage], kb * kGemmBK,
-                           sg.m_tile * kGemmBM, pol_a);
-          if (++stage == static_cast<uint32_t>(stages)) {
-            stage = 0;
-            phase ^= 1u;
-          }
+// TMA producer (one thread), one phase.  The W tiles of the first `pre`
+// k-blocks were already requested (with the whole stage's byte count).  With
+// `dep`, the phase's A operand is written by an earlier phase of the same
+// launch: the producer first requests the W tiles of as many k-blocks as there
+// are free stages, then waits (bounded) until `dep_target` CTAs have arrived
+// on *dep, then loads A (after a proxy fence, since A was written by other
+// CTAs through the generic proxy and is read here by TMA).
+template <int BN>
+__device__ void gemm_produce(const GemmParams& q, const CUtensorMap* tA, const CUtensorMap* tW,
+                             const GemmCta<BN>& S, GemmRing& R, int pre, const unsigned* dep,
+                             unsigned dep_target) {
+  using C = GemmCfg<BN>;
+  const uint64_t pol_w = policy_evict_first();
+  const uint64_t pol_a = policy_evict_last();
+  if (dep) {
+    GemmSegIter it0(q);
+    GemmSeg s0;
+    uint32_t stage = R.stage, phase = R.phase;
+    pre = 0;
+    while (R.ok && pre < S.stages && it0.next(q, s0)) {
+      for (int kb = s0.kb0; kb < s0.kb1 && pre < S.stages; ++kb, ++pre) {
+        if (!mbar_wait(&S.empty[stage], phase ^ 1u, q.err)) {
+          R.ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&S.full[stage], S.stage_tx);
+        tma_load_2d_hint(S.sB + stage * C::kBBytes, tW, &S.full[stage], w_x(q, kb),
+                         w_y<BN>(q, s0.n_tile, kb), pol_w);
+        if (++stage == static_cast<uint32_t>(S.stages)) {
+          stage = 0;
+          phase ^= 1u;
         }
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc = umma_idesc_f32acc(kGemmBM, BN, p.f16 != 0);
-      uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
-      bool ok = true;
-      GemmSegIter it(p);
-      GemmSeg sg;
-      while (ok && it.next(p, sg)) {
-        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, p.err)) break;
-        tc_fence_after();
-        const uint32_t d_base = tmem_base + acc * acc_cols;
-        int t = 0;   // K=16 step index within the segment; chain = t % nacc
-        for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
-          if (!mbar_wait(&full[stage], phase, p.err)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint64_t adesc = umma_desc_sw128(smem_u32(sA + stage * a_bytes));
-          const uint64_t bdesc = umma_desc_sw128(smem_u32(sB + stage * C::kBBytes));
+    if (R.ok && !wait_count(dep, dep_target, q.err)) R.ok = false;
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+  }
+  int idx = 0;
+  GemmSegIter it(q);
+  GemmSeg sg;
+  while (R.ok && it.next(q, sg)) {
+    for (int kb = sg.kb0; kb < sg.kb1; ++kb, ++idx) {
+      if (idx >= pre) {
+        if (!mbar_wait(&S.empty[R.stage], R.phase ^ 1u, q.err)) {
+          R.ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&S.full[R.stage], S.stage_tx);
+        tma_load_2d_hint(S.sB + R.stage * C::kBBytes, tW, &S.full[R.stage], w_x(q, kb),
+                         w_y<BN>(q, sg.n_tile, kb), pol_w);
+      }
+      tma_load_2d_hint(S.sA + R.stage * S.a_bytes, tA, &S.full[R.stage], kb * kGemmBK,
+                       sg.m_tile * kGemmBM, pol_a);
+      if (++R.stage == static_cast<uint32_t>(S.stages)) {
+        R.stage = 0;
+        R.phase ^= 1u;
+      }
+    }
+  }
+}
+
+// MMA issuer (one thread), one phase.
+template <int BN>
+__device__ void gemm_mma(const GemmParams& q, const GemmCta<BN>& S, GemmRing& R,
+                         GemmAccRing& A) {
+  using C = GemmCfg<BN>;
+  const uint32_t idesc = umma_idesc_f32acc(kGemmBM, BN, q.f16 != 0);
+  GemmSegIter it(q);
+  GemmSeg sg;
+  while (R.ok && it.next(q, sg)) {
+    if (!mbar_wait(&S.tempty[A.acc], A.acc_phase ^ 1u, q.err)) {
+      R.ok = false;
+      break;
+    }
+    tc_fence_after();
+    const uint32_t d_base = S.tmem_base + A.acc * S.acc_cols;
+    int t = 0;   // K=16 step index within the segment; chain = t % nacc
+    for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
+      if (!mbar_wait(&S.full[R.stage], R.phase, q.err)) {
+        R.ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint64_t adesc = umma_desc_sw128(smem_u32(S.sA + R.stage * S.a_bytes));
+      const uint64_t bdesc = umma_desc_sw128(smem_u32(S.sB + R.stage * C::kBBytes));
 #pragma unroll
-          for (int k = 0; k < kGemmBK / 16; ++k, ++t) {
-            // +32 bytes along K inside the 128-byte swizzle atom = +2 in the
-            // descriptor's (address >> 4) field
-            const int chain = t % p.nacc;
-            umma_f16kind(d_base + chain * BN, adesc + 2 * k, bdesc + 2 * k, idesc,
-                         t >= p.nacc ? 1u : 0u);
-          }
-          umma_commit(&empty[stage]);
-          if (++stage == static_cast<uint32_t>(stages)) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
-        if (!ok) break;
-        umma_commit(&tfull[acc]);
-        if (++acc == static_cast<uint32_t>(p.nbuf)) {
-          acc = 0;
-          acc_phase ^= 1u;
-        }
+      for (int k = 0; k < kGemmBK / 16; ++k, ++t) {
+        // +32 bytes along K inside the 128-byte swizzle atom = +2 in the
+        // descriptor's (address >> 4) field
+        const int chain = t % q.nacc;
+        umma_f16kind(d_base + chain * BN, adesc + 2 * k, bdesc + 2 * k, idesc,
+                     t >= q.nacc ? 1u : 0u);
+      }
+      umma_commit(&S.empty[R.stage]);
+      if (++R.stage == static_cast<uint32_t>(S.stages)) {
+        R.stage = 0;
+        R.phase ^= 1u;
       }
     }
-  } else if (gemm_staged(p.a_rows)) {
-    // ------------------------------------------------------------ staged epilogue
-    pdl_wait();
-    constexpr int LD = BN + 4;
-    constexpr int F4 = BN / 4;             // float4 per row
-    const int tid = threadIdx.x - 64;      // 0..127
-    const int sp = warp & 3;
-    uint32_t acc = 0, acc_phase = 0, nseen = 0;
-    GemmSegIter it(p);
-    GemmSeg sg;
-    while (it.next(p, sg)) {
+    if (!R.ok) break;
+    umma_commit(&S.tfull[A.acc]);
+    if (++A.acc == static_cast<uint32_t>(q.nbuf)) {
+      A.acc = 0;
+      A.acc_phase ^= 1u;
+    }
+  }
+}
+
+template <int BN, class Epi>
+__device__ void gemm_staged_epilogue(const GemmParams& p, const Epi& epi, const GemmCta<BN>& S,
+                                     GemmAccRing& A) {
+  constexpr int G = Epi::kGroup;
+  constexpr int LD = BN + 4;
+  constexpr int F4 = BN / 4;             // float4 per row
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tid = threadIdx.x - 64;      // 0..127
+  const int sp = warp & 3;
+  float* staging = S.staging;
+  volatile int* wait_flag = S.wait_flag;
+  volatile int* last_flag = S.last_flag;
+  uint64_t* tfull = S.tfull;
+  uint64_t* tempty = S.tempty;
+  const uint32_t tmem_base = S.tmem_base;
+  const int acc_cols = S.acc_cols;
+  uint32_t& acc = A.acc;
+  uint32_t& acc_phase = A.acc_phase;
+  uint32_t& nseen = A.nseen;
+  GemmSegIter it(p);
+  GemmSeg sg;
+  while (A.ok && it.next(p, sg)) {
       // one thread waits (bounded) and the verdict is shared, so that the
       // named barriers below are always reached by all 128 threads or none
       if (tid == 0) wait_flag[nseen & 1] = mbar_wait(&tfull[acc], acc_phase, p.err) ? 1 : 0;
       named_bar_sync(1, 128);
-      if (!wait_flag[nseen++ & 1]) break;
+      if (!wait_flag[nseen++ & 1]) {
+        A.ok = false;
+        break;
+      }
       tc_fence_after();
       if (sp == 0) {
         // rows 0..31 live in TMEM lanes 0..31: the sub-partition-0 warp reads
@@ -458,6 +554,47 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       named_bar_sync(1, 128);  // staging and last_flag are rewritten by the next segment
     }
+}
+
+template <int BN, class Epi>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_tcgen05_kernel(const __grid_constant__ CUtensorMap tmA,
+                        const __grid_constant__ CUtensorMap tmW, const GemmParams p,
+                        const Epi epi) {
+  constexpr int G = Epi::kGroup;
+  static_assert(BN % G == 0, "epilogue group must divide the tile width");
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  pdl_trigger();
+  int pre = 0;
+  const GemmCta<BN> S = gemm_setup<BN>(p, &tmA, &tmW, pre);
+  float* staging = S.staging;
+  volatile int* wait_flag = S.wait_flag;
+  volatile int* last_flag = S.last_flag;
+  uint64_t* tfull = S.tfull;
+  uint64_t* tempty = S.tempty;
+  const uint32_t tmem_base = S.tmem_base;
+  const int acc_cols = S.acc_cols;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      pdl_wait();
+      GemmRing R;
+      gemm_produce<BN>(p, &tmA, &tmW, S, R, pre, nullptr, 0);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      GemmRing R;
+      GemmAccRing A;
+      gemm_mma<BN>(p, S, R, A);
+    }
+  } else if (gemm_staged(p.a_rows)) {
+    // ------------------------------------------------------------ staged epilogue
+    pdl_wait();
+    GemmAccRing A;
+    gemm_staged_epilogue<BN, Epi>(p, epi, S, A);
   } else {
     // ------------------------------------------------------------ epilogue
     pdl_wait();
@@ -556,6 +693,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   }
 
+
   if (p.cluster_s > 1) {
     // Every thread of every CTA of the cluster reaches both barriers exactly
     // once (no early exits above, all waits bounded).  Between them, CTA rank q
@@ -626,6 +764,78 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, static_cast<uint32_t>(p.tmem_cols));
+  }
+}
+
+// Two GEMMs in one launch (few rows, staged epilogue, no clusters): phase 1
+// (A1 x W1^T, epilogue e1) then phase 2 (A2 x W2^T, e2) on the same CTAs, the
+// same pipeline ring and the same accumulator, where A2 is written by phase 1.
+// Every CTA's epilogue arrives on dep[0] once its phase-1 stores are out; a
+// producer loads A2 only after all gridDim.x CTAs have arrived, and meanwhile
+// streams phase 2's first weight stages — so the second weight stream starts
+// while the first one drains, without a kernel boundary.  The last CTA to
+// finish resets dep[0] and dep[1] to zero for the next launch.  Every CTA of
+// the grid must be able to become resident (the grid is at most one CTA per
+// SM, and nothing the CTAs wait on depends on them), so the wait ends.
+template <int BN, class Epi1, class Epi2>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_chain_kernel(const __grid_constant__ CUtensorMap tmA1,
+                      const __grid_constant__ CUtensorMap tmW1, const GemmParams p1,
+                      const Epi1 e1, const __grid_constant__ CUtensorMap tmA2,
+                      const __grid_constant__ CUtensorMap tmW2, const GemmParams p2,
+                      const Epi2 e2, unsigned* dep) {
+  static_assert(BN % Epi1::kGroup == 0 && BN % Epi2::kGroup == 0, "epilogue groups");
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  pdl_trigger();
+  int pre = 0;
+  const GemmCta<BN> S = gemm_setup<BN>(p1, &tmA1, &tmW1, pre);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      pdl_wait();
+      GemmRing R;
+      gemm_produce<BN>(p1, &tmA1, &tmW1, S, R, pre, nullptr, 0);
+      if (R.ok) {
+        tma_prefetch_desc(&tmA2);
+        tma_prefetch_desc(&tmW2);
+      }
+      gemm_produce<BN>(p2, &tmA2, &tmW2, S, R, 0, dep, gridDim.x);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      GemmRing R;
+      GemmAccRing A;
+      gemm_mma<BN>(p1, S, R, A);
+      gemm_mma<BN>(p2, S, R, A);
+    }
+  } else {
+    pdl_wait();
+    GemmAccRing A;
+    gemm_staged_epilogue<BN, Epi1>(p1, e1, S, A);
+    // phase-1 stores of this CTA are out: arrive
+    named_bar_sync(1, 128);
+    if (threadIdx.x == 64) {
+      __threadfence();
+      atomicAdd(&dep[0], 1u);
+    }
+    gemm_staged_epilogue<BN, Epi2>(p2, e2, S, A);
+  }
+
+  tc_fence_before();
+  cta_sync();
+  if (threadIdx.x == 0) {
+    // the last CTA out resets the arrival counters for the next launch
+    const unsigned prev = atomicAdd(&dep[1], 1u);
+    if (prev == gridDim.x - 1) {
+      dep[0] = 0u;
+      dep[1] = 0u;
+      __threadfence();
+    }
+  }
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(S.tmem_base, static_cast<uint32_t>(p1.tmem_cols));
   }
 }
 

@@ -28,7 +28,7 @@ STATUS = {
     -7: "DFLASH_ERR_DEVICE_TIMEOUT",
 }
 DEVERR_TIMEOUT, DEVERR_SLOT, DEVERR_TABLE, DEVERR_TOKEN, DEVERR_POSITION = 1, 2, 4, 8, 16
-KERNEL_KINDS = 13
+KERNEL_KINDS = 14
 
 
 class DFlashError(RuntimeError):

@@ -348,7 +348,8 @@ enum {
   DFLASH_KERNEL_GEMM_FC = 10,        /* fc over the tapped states                    */
   DFLASH_KERNEL_GEMM_KV_INJECT = 11, /* all layers' K/V + k_norm + RoPE + scatter    */
   DFLASH_KERNEL_LINEAR = 12,         /* dflash_linear / dflash_linear_ex             */
-  DFLASH_KERNEL_KINDS = 13
+  DFLASH_KERNEL_GEMM_MLP = 13,       /* few rows: gate/up + SwiGLU + down + residual, one launch */
+  DFLASH_KERNEL_KINDS = 14
 };
 
 /* Number of kernel launches the handle's calls have issued so far (launches

@@ -267,3 +267,26 @@ def test_qwen3_b1_step():
         assert excluded <= max_excluded(K)
     finally:
         h.close()
+
+
+def test_chain_launch_matches_oracle(monkeypatch):
+    """The opt-in one-launch gate/up + down schedule (few rows) gives the same
+    drafts as the oracle outside near-ties, like the default schedule."""
+    monkeypatch.setenv("DFLASH_CHAIN", "1")
+    cfg = dict(synth.model_config("qwen3_8b"), n_layers=1, vocab=8192, mask_token_id=8191)
+    Wt = synth.make_weights(cfg, seed=0)
+    h = DFlash(cfg, weights_to(Wt, DEV), max_position=4096)
+    try:
+        for ctx in ([700], [300, 1300]):
+            ch = Chain(cfg, Wt, h, ctx, seed=11 + len(ctx))
+            h.profile_enable(1024)
+            d, lo, blk = ch.gpu()
+            prof = h.profile_read()
+            h.profile_disable()
+            assert prof.get("gemm_mlp", (0, 0.0))[0] == cfg["n_layers"]   # the chain ran
+            assert prof.get("gemm_gate_up", (0, 0.0))[0] == 0
+            K = cfg["block_size"] - 1
+            excluded = compare_drafts(d, lo, ch.oracle("device"), ch.oracle("exact"), K)
+            assert excluded <= max_excluded(len(ctx) * K)
+    finally:
+        h.close()
