@@ -38,37 +38,46 @@
 
 namespace dflash {
 
-constexpr int kTcKeys = 128;        // keys per tile (8 pages)
+constexpr int kTcKeys = 128;        // keys per tile of the few-request (cluster) variant
+constexpr int kTcKeysSmall = 64;    // keys per tile of the many-request variant (2 CTAs per SM)
 constexpr int kTcStages = 2;        // K/V ring depth
 constexpr int kTcM = 64;            // MMA M: query rows of a kv group, zero-padded
 constexpr int kTcThreads = 192;     // warp 0 TMA, warp 1 MMA, warps 2..5 softmax
 constexpr float kTcLazyRescale = 8.f;  // log2 of the growth that forces an O rescale
 
-template <int D>
+// Per tile width KT (keys): 128-key tiles keep more keys in flight per CTA (few
+// requests, latency); 64-key tiles with one P buffer fit two CTAs per SM
+// (shared memory 100 KB, 256 TMEM columns) so that their pipelines hide each
+// other's latency (many requests, throughput).
+template <int D, int KT>
 struct TcAttnCfg {
   static constexpr int kHalves = D / 64;                      // 64-element halves of a row
-  static constexpr int kKVBytes = kHalves * kTcKeys * 128;    // one K (or V) tile
+  static constexpr int kKVBytes = kHalves * KT * 128;         // one K (or V) tile
   static constexpr int kQBytes = kHalves * kTcM * 128;
-  static constexpr int kPBytes = (kTcKeys / 64) * kTcM * 128; // P hi (or lo) of one tile
+  static constexpr int kPBytes = (KT / 64) * kTcM * 128;      // P hi (or lo) of one tile
+  static constexpr int kPBufs = KT == 64 ? 1 : 2;             // P buffers (ring of tiles)
   static constexpr int kOffV = kTcStages * kKVBytes;
   static constexpr int kOffQ = 2 * kTcStages * kKVBytes;
   static constexpr int kOffP = kOffQ + kQBytes;
-  static constexpr int kOffBar = kOffP + 4 * kPBytes;
+  static constexpr int kOffBar = kOffP + 2 * kPBufs * kPBytes;
   static constexpr int kSmem = 1024 + kOffBar + 256;
-  static constexpr int kOCol = 2 * kTcKeys;                   // TMEM column of O
+  static constexpr int kOCol = 2 * KT;                        // TMEM column of O
+  static constexpr int kTmemCols = kOCol + D <= 256 ? 256 : 512;
+  static constexpr int kMinBlocks = KT == 64 ? 2 : 1;
   // cluster combine, inside the (then idle) K/V ring: received O rows
   // [lr * S + src][D + 8] and (m, l) [lr * S + src] (S * ceil(64 / S) <= 71 slots)
   static constexpr int kCombSlots = kTcM + 7;
   static constexpr int kCombOffML = kCombSlots * (D + 8) * 4;
+  static_assert(KT == 64 || KT == 128, "tile width");
   static_assert(kCombOffML + kCombSlots * 8 <= 2 * kTcStages * kKVBytes, "combine buffers");
   static_assert(kOCol + D <= 512, "TMEM budget");
 };
 
-template <int D>
-__global__ void __launch_bounds__(kTcThreads, 1)
+template <int D, int KT>
+__global__ void __launch_bounds__(kTcThreads, TcAttnCfg<D, KT>::kMinBlocks)
     attn_block_tc_kernel(const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
-  using C = TcAttnCfg<D>;
+  using C = TcAttnCfg<D, KT>;
   pdl_trigger();
   pdl_wait();
   const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -78,7 +87,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (k0 >= n_keys && !p.cluster) return;
   const int k1 = min(n_keys, k0 + p.chunk_keys);
   const int n_splits_b = (n_keys + p.chunk_keys - 1) / p.chunk_keys;
-  const int n_tiles = k0 < n_keys ? (k1 - k0 + kTcKeys - 1) / kTcKeys : 0;
+  const int n_tiles = k0 < n_keys ? (k1 - k0 + KT - 1) / KT : 0;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   extern __shared__ uint8_t smem_raw[];
@@ -98,7 +107,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
   auto sK = [&](int s) { return smem + s * C::kKVBytes; };
   auto sV = [&](int s) { return smem + C::kOffV + s * C::kKVBytes; };
-  auto sP = [&](int lohi, int buf) { return smem + C::kOffP + (buf * 2 + lohi) * C::kPBytes; };
+  auto sP = [&](int lohi, int buf) {
+    return smem + C::kOffP + ((C::kPBufs == 1 ? 0 : buf) * 2 + lohi) * C::kPBytes;
+  };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
@@ -115,7 +126,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 512);
+    tmem_alloc(tmem_slot, C::kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -136,12 +147,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int t = 0; t < n_tiles; ++t) {
         const int s = t & 1, u = t >> 1;
         if (!mbar_wait(&kv_empty[s], (u & 1) ^ 1u, p.err)) break;
-        const int t0 = k0 + t * kTcKeys;
-        const int nvalid = min(kTcKeys, k1 - t0);
+        const int t0 = k0 + t * KT;
+        const int nvalid = min(KT, k1 - t0);
         const int npages = (nvalid + 15) >> 4;
         mbar_arrive_expect_tx(&kv_full[s],
-                              static_cast<uint32_t>(8 * C::kHalves * 2048 * 2));
-        for (int j = 0; j < 8; ++j) {
+                              static_cast<uint32_t>((KT / 16) * C::kHalves * 2048 * 2));
+        for (int j = 0; j < KT / 16; ++j) {
           int y = -16;  // pages past the range: fully out of bounds, TMA fills zeros
           if (j < npages) {
             const int pg = (t0 >> 4) + j;
@@ -155,7 +166,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
 #pragma unroll
           for (int hf = 0; hf < C::kHalves; ++hf) {
-            const int off = hf * kTcKeys * 128 + j * 2048;
+            const int off = hf * KT * 128 + j * 2048;
             tma_load_2d(sK(s) + off, &tmK, &kv_full[s], hf * 64, y);
             tma_load_2d(sV(s) + off, &tmV, &kv_full[s], hf * 64, y);
           }
@@ -165,7 +176,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc_qk = umma_idesc_bf16(kTcM, kTcKeys, false);
+      const uint32_t idesc_qk = umma_idesc_bf16(kTcM, KT, false);
       const uint32_t idesc_pv = umma_idesc_bf16(kTcM, D, true);
       bool ok = n_tiles > 0 && mbar_wait(q_full, 0, p.err);
       tc_fence_after();
@@ -178,8 +189,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int kk = 0; kk < D / 16; ++kk) {
           const int half = kk >> 2, w = kk & 3;
           const uint64_t ad = umma_desc_sw128(smem_u32(sQ + half * kTcM * 128 + w * 32));
-          const uint64_t bd = umma_desc_sw128(smem_u32(sK(s) + half * kTcKeys * 128 + w * 32));
-          umma_f16kind(tmem_base + s * kTcKeys, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+          const uint64_t bd = umma_desc_sw128(smem_u32(sK(s) + half * KT * 128 + w * 32));
+          umma_f16kind(tmem_base + s * KT, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
         }
         umma_commit(&s_full[s]);
         return true;
@@ -199,11 +210,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
         for (int lohi = 0; lohi < 2; ++lohi) {
 #pragma unroll
-          for (int kk = 0; kk < kTcKeys / 16; ++kk) {
+          for (int kk = 0; kk < KT / 16; ++kk) {
             const int kh = kk >> 2, w = kk & 3;
             const uint64_t ad = umma_desc_sw128(smem_u32(sP(lohi, s) + kh * kTcM * 128 + w * 32));
             const uint64_t bd = umma_desc_sw128_mn(smem_u32(sV(s) + kk * 16 * 128),
-                                                   kTcKeys * 128, 1024);
+                                                   KT * 128, 1024);
             umma_f16kind(tmem_base + C::kOCol, ad, bd, idesc_pv,
                          (t > 0 || lohi > 0 || kk > 0) ? 1u : 0u);
           }
@@ -257,19 +268,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         break;
       }
       tc_fence_after();
-      float sv[4 * (kTcKeys / 8)];
-      tmem_ld_16x256b_x8(tmem_base + lane_base + s * kTcKeys, sv);
-      tmem_ld_16x256b_x8(tmem_base + lane_base + s * kTcKeys + 64, sv + 32);
+      float sv[4 * (KT / 8)];
+#pragma unroll
+      for (int c = 0; c < KT / 64; ++c)
+        tmem_ld_16x256b_x8(tmem_base + lane_base + s * KT + c * 64, sv + 32 * c);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_empty[s]);
 
-      const int t0 = k0 + t * kTcKeys;
-      const int nvalid = min(kTcKeys, k1 - t0);
+      const int t0 = k0 + t * KT;
+      const int nvalid = min(KT, k1 - t0);
       float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
-      for (int j = 0; j < kTcKeys / 8; ++j) {
+      for (int j = 0; j < KT / 8; ++j) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int kt = j * 8 + 2 * (lane & 3) + (e & 1);
@@ -326,19 +338,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) ref[hh] = (m_ref[hh] == -INFINITY) ? 0.f : m_ref[hh];
 #pragma unroll
-      for (int q = 0; q < 4 * (kTcKeys / 8); ++q) {
+      for (int q = 0; q < 4 * (KT / 8); ++q) {
         const float pv = exp2f(sv[q] - ref[(q >> 1) & 1]);
         sv[q] = pv;
         l_run[(q >> 1) & 1] += pv;
       }
-      if (!mbar_wait(&p_empty[s], (u & 1) ^ 1u, p.err)) {
+      // the P buffer must be free: P V of the tile that used it has landed
+      // (two buffers: tile t-2, via p_empty; one buffer: tile t-1, via o_ready,
+      // which is at most one phase behind here)
+      const bool p_free = C::kPBufs == 2 ? mbar_wait(&p_empty[s], (u & 1) ^ 1u, p.err)
+                          : (t == 0 || mbar_wait(o_ready, (t - 1) & 1, p.err));
+      if (!p_free) {
         ok = false;
         break;
       }
       uint8_t* ph = sP(0, s);
       uint8_t* pl = sP(1, s);
 #pragma unroll
-      for (int j = 0; j < kTcKeys / 8; ++j) {
+      for (int j = 0; j < KT / 8; ++j) {
         const int kh = j >> 3, ch = j & 7;
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
@@ -359,7 +376,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const int hf = e / ((16 - rr0) * 8);
           const int rem = e - hf * (16 - rr0) * 8;
           const int rr = rr0 + rem / 8, cc = rem & 7;
-          *reinterpret_cast<uint4*>(sV(s) + hf * kTcKeys * 128 + jp * 2048 + rr * 128 + cc * 16) =
+          *reinterpret_cast<uint4*>(sV(s) + hf * KT * 128 + jp * 2048 + rr * 128 + cc * 16) =
               make_uint4(0, 0, 0, 0);
         }
       }
@@ -504,7 +521,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   cta_sync();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, 512);
+    tmem_dealloc(tmem_base, C::kTmemCols);
   }
 }
 

@@ -195,6 +195,7 @@ size_t gemm_partial_bound(int M, int num_sms) {
 struct AttnPlan {
   int chunk_keys = 0, max_splits = 0, R = 0, row_groups = 0, key_parts = 0, nwc = 0;
   bool tc = false;   // tcgen05 kernel (kv groups of up to 64 query rows)
+  int kt = 128;      // tcgen05 kernel: keys per tile
   bool cluster = false;  // tcgen05 kernel, splits of a (request, kv head) combined in a cluster
   size_t part_o_bytes = 0, part_ml_bytes = 0;
 };
@@ -205,7 +206,8 @@ AttnPlan plan_attention(int B, int Hkv, int W, int P, int bs, int G, int D, int 
   const double est = static_cast<double>(B) * Hkv * keys_max;
   a.R = bs * G;
   a.tc = a.R <= kTcM;
-  const int tile = a.tc ? kTcKeys : kAttnTileKeys;
+  a.kt = kTcKeysSmall;   // many requests: 64-key tiles, two CTAs per SM
+  const int tile = a.tc ? a.kt : kAttnTileKeys;
   int chunk = static_cast<int>(std::ceil(est / (4.0 * num_sms)));
   chunk = (chunk + tile - 1) / tile * tile;
   chunk = std::max(128, std::min(8192, chunk));
@@ -230,6 +232,7 @@ AttnPlan plan_attention(int B, int Hkv, int W, int P, int bs, int G, int D, int 
       const int splits = cdiv(keys_max, chunk);
       if (splits >= 2) {
         a.cluster = true;
+        a.kt = kTcKeys;      // few requests: 128-key tiles, more keys in flight per CTA
         a.chunk_keys = chunk;
         a.max_splits = splits;
         a.part_o_bytes = 0;
@@ -644,8 +647,13 @@ cudaError_t set_attn_attrs() {
   if ((e = cudaFuncSetAttribute(attn_block_kernel<D, 16>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, bytes)) != cudaSuccess)
     return e;
-  return cudaFuncSetAttribute(attn_block_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              TcAttnCfg<D>::kSmem);
+  if ((e = cudaFuncSetAttribute(attn_block_tc_kernel<D, kTcKeysSmall>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                TcAttnCfg<D, kTcKeysSmall>::kSmem)) != cudaSuccess)
+    return e;
+  return cudaFuncSetAttribute(attn_block_tc_kernel<D, kTcKeys>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              TcAttnCfg<D, kTcKeys>::kSmem);
 }
 
 template <int D>
@@ -665,8 +673,12 @@ dflash_status run_attention(dflash_handle* h, const AttnPlan& ap, AttnParams prm
   prm.cluster = ap.cluster ? 1 : 0;
   if (ap.tc) {
     LaunchScope scope(h, DFLASH_KERNEL_ATTENTION, st);
-    launch_kc(h->pdl, ap.cluster ? ap.max_splits : 1, attn_block_tc_kernel<D>, grid,
-              dim3(kTcThreads), TcAttnCfg<D>::kSmem, st, tk, tv, prm);
+    if (ap.kt == kTcKeysSmall)
+      launch_kc(h->pdl, ap.cluster ? ap.max_splits : 1, attn_block_tc_kernel<D, kTcKeysSmall>,
+                grid, dim3(kTcThreads), TcAttnCfg<D, kTcKeysSmall>::kSmem, st, tk, tv, prm);
+    else
+      launch_kc(h->pdl, ap.cluster ? ap.max_splits : 1, attn_block_tc_kernel<D, kTcKeys>, grid,
+                dim3(kTcThreads), TcAttnCfg<D, kTcKeys>::kSmem, st, tk, tv, prm);
   } else {
     LaunchScope scope(h, DFLASH_KERNEL_ATTENTION, st);
     if (ap.key_parts == 1)
