@@ -45,10 +45,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # dram__bytes_write.sum) for the kernel family that dominates a workload,
 # keyed by the digest of the kernel sources it was measured on.
 TRAFFIC = {
-    # gate/up GEMM of the batch-1 Qwen3-8B-shaped step: 201.55 MB read + 3.55 MB written
+    # gate/up GEMM of the batch-1 Qwen3-8B-shaped step: 201.54 MB read + 3.79 MB written
     # (ncu --set full, profiles/gemm_gate_up_qwen3_b1_ctx2048.md)
-    ("qwen3_b1_ctx2048", "gemm_gate_up"): {"bytes_per_launch": 205106688,
-                                           "digest": "04b44d4801a112eb"},
+    ("qwen3_b1_ctx2048", "gemm_gate_up"): {"bytes_per_launch": 205339392,
+                                           "digest": "3f8ab3c2e1ea80ae"},
 }
 
 
