@@ -100,8 +100,9 @@ int gemm_stages(int a_rows, int bn) {
 // weight-streaming regime, M <= 128): two accumulator chains in a single TMEM
 // buffer, and stream-K (the (tile, k-block) iterations split evenly over the
 // SMs) unless whole tiles already fill >= 90% of the last round.  Several M
-// tiles (tensor-bound): one chain, double-buffered, whole tiles round-robin;
-// stream-K only when the tiles cannot occupy half of the SMs.  force_bn /
+// tiles (tensor-bound): 256-wide tiles, or 128-wide ones when only those fill
+// >= 75% of the last round; double-buffered accumulator, whole tiles
+// round-robin; stream-K only when the tiles cannot occupy half of the SMs.  force_bn /
 // force_splits (0 = automatic) pin the tile width and the schedule: 1 = whole
 // tiles, n >= 2 = stream-K with ceil(k_blocks / n) iterations per CTA.
 //
@@ -116,6 +117,15 @@ GemmPlan plan_gemm(int M, int N, int K, int group, int num_sms, int force_bn = 0
   pl.k_blocks = K / kGemmBK;
   pl.m_tiles = cdiv(M, kGemmBM);
   pl.BN = force_bn ? force_bn : 256;
+  if (!force_bn && pl.m_tiles > 1 && group <= 128) {
+    // several M tiles (tensor-bound): 128-wide tiles when only they fill the
+    // SMs (e.g. 4 x 32 tiles of a 4096-wide output at 512 rows)
+    auto util = [&](int bn) {
+      const int t = pl.m_tiles * cdiv(N, bn);
+      return static_cast<double>(t) / (static_cast<double>(cdiv(t, num_sms)) * num_sms);
+    };
+    if (util(256) < 0.75 && util(128) >= 0.75) pl.BN = 128;
+  }
   if (pl.BN < group || pl.BN % group) pl.BN = 256;
   const bool one_m_tile = pl.m_tiles == 1;
   if (M <= kGemmStagedRows) {
@@ -494,7 +504,6 @@ dflash_status run_gemm(dflash_handle* h, int kind, bool f16, bool w_packed, cons
                    force_bn % Epi::kGroup))
     return DFLASH_ERR_INVALID_ARG;
   if (force_splits < 0 || force_splits > K / kGemmBK) return DFLASH_ERR_INVALID_ARG;
-  if (w_packed) force_bn = kPackRows;  // the packed layout fixes the tile width
   GemmPlan pl = plan_gemm(M, N, K, Epi::kGroup, h->num_sms, force_bn, force_splits);
   if (gemm_staged(pl.a_rows) && pl.tiles <= h->num_sms && !force_splits) {
     const int* cap = gemm_cluster_caps<Epi>(h, pl.BN, pl.smem);
@@ -505,8 +514,8 @@ dflash_status run_gemm(dflash_handle* h, int kind, bool f16, bool w_packed, cons
   CUtensorMap ta, tw;
   if (!h->tmap(&ta, A, M, K, pl.a_rows, f16)) return DFLASH_ERR_CUDA;
   if (w_packed) {
-    if (!h->tmap(&tw, Wt, static_cast<uint64_t>(pl.n_tiles) * pl.k_blocks * kPackRows, kGemmBK,
-                 kPackRows, f16))
+    if (!h->tmap(&tw, Wt, static_cast<uint64_t>(cdiv(N, kPackRows)) * pl.k_blocks * kPackRows,
+                 kGemmBK, pl.BN, f16))
       return DFLASH_ERR_CUDA;
   } else if (!h->tmap(&tw, Wt, N, K, pl.BN, f16)) {
     return DFLASH_ERR_CUDA;
@@ -560,8 +569,8 @@ bool chain_phase(dflash_handle* h, const GemmPlan& pl, bool f16, const void* A, 
                  const void* Wt, int N, float* partials, unsigned* counters, CUtensorMap* ta,
                  CUtensorMap* tw, GemmParams* gp) {
   if (!h->tmap(ta, A, M, K, pl.a_rows, f16)) return false;
-  if (!h->tmap(tw, Wt, static_cast<uint64_t>(pl.n_tiles) * pl.k_blocks * kPackRows, kGemmBK,
-               kPackRows, f16))
+  if (!h->tmap(tw, Wt, static_cast<uint64_t>(cdiv(N, kPackRows)) * pl.k_blocks * kPackRows,
+               kGemmBK, pl.BN, f16))
     return false;
   *gp = GemmParams{};
   gp->M = M;

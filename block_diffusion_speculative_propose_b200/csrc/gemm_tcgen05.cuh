@@ -178,13 +178,17 @@ __device__ __forceinline__ void tmem_load_sum32(uint32_t taddr, int nacc, float*
 }
 
 // Coordinates of the W box of (n_tile, k-block kb): row-major W is addressed by
-// (k, row); the tile-contiguous layout stores each 256 x 64 tile as one chunk.
+// (k, row); the tile-contiguous layout stores each 256 x 64 tile as one chunk
+// of 256 consecutive 128-byte rows, so a BN-row tile (BN dividing 256) is a
+// contiguous part of one chunk.
 __device__ __forceinline__ int w_x(const GemmParams& p, int kb) {
   return p.w_packed ? 0 : kb * kGemmBK;
 }
 template <int BN>
 __device__ __forceinline__ int w_y(const GemmParams& p, int n_tile, int kb) {
-  return p.w_packed ? (n_tile * p.k_blocks + kb) * 256 : n_tile * BN;
+  static_assert(256 % BN == 0, "tile width divides the packed chunk");
+  const int row0 = n_tile * BN;
+  return p.w_packed ? ((row0 >> 8) * p.k_blocks + kb) * 256 + (row0 & 255) : row0;
 }
 
 // Shared-memory carve-up, barriers and tensor-memory base of one CTA, common
