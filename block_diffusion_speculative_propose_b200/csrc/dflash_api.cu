@@ -210,7 +210,8 @@ struct AttnPlan {
   size_t part_o_bytes = 0, part_ml_bytes = 0;
 };
 
-AttnPlan plan_attention(int B, int Hkv, int W, int P, int bs, int G, int D, int num_sms) {
+AttnPlan plan_attention(int B, int Hkv, int W, int P, int bs, int G, int D, int num_sms,
+                        bool allow_cluster) {
   AttnPlan a;
   const int keys_max = W * P;
   const double est = static_cast<double>(B) * Hkv * keys_max;
@@ -232,10 +233,12 @@ AttnPlan plan_attention(int B, int Hkv, int W, int P, int bs, int G, int D, int 
       a.max_splits > 1 ? static_cast<size_t>(a.max_splits) * B * Hkv * a.R * D * 4 : 0;
   a.part_ml_bytes =
       a.max_splits > 1 ? static_cast<size_t>(a.max_splits) * B * Hkv * a.R * 2 * 4 : 0;
-  // Few (request, kv head) pairs: the key splits are what fills the GPU, and
-  // they are combined inside a cluster of up to 8 CTAs instead of through
-  // global partials and a second kernel.
-  if (a.tc && 2 * B * Hkv <= num_sms) {
+  // Opt-in: with few (request, kv head) pairs, combine the key splits inside a
+  // cluster of up to 8 CTAs (128-key tiles) instead of through global partials
+  // and a second kernel.  Measured slower than the default (64-key tiles, two
+  // CTAs per SM, combine kernel) at batch 1-4 of the Qwen3-8B shape
+  // (batch 1, context 2048: 18.2 vs 14.6 us per layer).
+  if (allow_cluster && a.tc && 2 * B * Hkv <= num_sms) {
     const int S = std::min(8, num_sms / (B * Hkv));
     if (S >= 2) {
       const int chunk = cdiv(cdiv(keys_max, S), kTcKeys) * kTcKeys;
@@ -311,6 +314,12 @@ struct dflash_handle {
   // SMs gate/up leaves free and reduces through clusters.
   bool chain = [] {
     const char* e = std::getenv("DFLASH_CHAIN");
+    return e && e[0] == '1';
+  }();
+  // cluster-combined attention splits for few requests: opt-in
+  // (DFLASH_ATTN_CLUSTER=1 when the handle is created)
+  bool attn_cluster = [] {
+    const char* e = std::getenv("DFLASH_ATTN_CLUSTER");
     return e && e[0] == '1';
   }();
   std::vector<cudaEvent_t> prof_events;
@@ -755,7 +764,8 @@ ProposeWs propose_layout(const dflash_handle* h, int B, int W) {
   size_t po = 0, pm = 0, pc = 0;
   // the attention split plan is not monotonic in the batch: cover every size
   for (int bb = 1; bb <= B; ++bb) {
-    const AttnPlan ap = plan_attention(bb, Hkv, W, c.page_size, bs, Hq / Hkv, D, h->num_sms);
+    const AttnPlan ap = plan_attention(bb, Hkv, W, c.page_size, bs, Hq / Hkv, D, h->num_sms,
+                                       h->attn_cluster);
     po = std::max(po, ap.part_o_bytes);
     pm = std::max(pm, ap.part_ml_bytes);
   }
@@ -849,7 +859,8 @@ dflash_status propose_layers(dflash_handle* h, const ProposeWs& lw, void* ws,
   bf16* hm = at<bf16>(ws, lw.hm);
   f16* frows = at<f16>(ws, lw.frows);
   float* partial = at<float>(ws, lw.partial);
-  const AttnPlan ap = plan_attention(B, Hkv, W, c.page_size, bs, Hq / Hkv, D, h->num_sms);
+  const AttnPlan ap = plan_attention(B, Hkv, W, c.page_size, bs, Hq / Hkv, D, h->num_sms,
+                                     h->attn_cluster);
   if (ap.part_o_bytes > lw.part_o_cap || ap.part_ml_bytes > lw.part_ml_cap)
     return DFLASH_ERR_WORKSPACE;
   AttnParams prm;
@@ -1456,7 +1467,7 @@ size_t dflash_attention_workspace_bytes(const dflash_handle* h, int B, int max_p
   const dflash_config& c = h->cfg;
   const AttnPlan ap = plan_attention(B, c.n_kv_heads, max_pages_per_seq, c.page_size,
                                      c.block_size, c.n_q_heads / c.n_kv_heads, c.head_dim,
-                                     h->num_sms);
+                                     h->num_sms, h->attn_cluster);
   return align_up(ap.part_o_bytes) + align_up(ap.part_ml_bytes) + kAlign;
 }
 
@@ -1476,7 +1487,7 @@ dflash_status dflash_block_attention(dflash_handle* h, const void* q, const int3
   DF_CUDA(use_device(h->device));
   const AttnPlan ap = plan_attention(B, c.n_kv_heads, max_pages_per_seq, c.page_size,
                                      c.block_size, c.n_q_heads / c.n_kv_heads, c.head_dim,
-                                     h->num_sms);
+                                     h->num_sms, h->attn_cluster);
   AttnParams prm;
   prm.q = static_cast<const bf16*>(q);
   prm.o = static_cast<f16*>(o);

@@ -175,6 +175,38 @@ def test_block_attention_matches_oracle(model, seq_lens):
         h.close()
 
 
+@pytest.mark.parametrize("model,seq_lens", [
+    ("qwen3_8b", [2048]),
+    ("qwen3_8b", [0, 7, 100, 1000, 5000]),
+    ("llama31_8b", [3, 333, 4097]),
+])
+def test_block_attention_cluster_combine(monkeypatch, model, seq_lens):
+    """The opt-in plan that combines a request's key splits inside a thread-
+    block cluster (distributed shared memory) instead of a second kernel."""
+    monkeypatch.setenv("DFLASH_ATTN_CLUSTER", "1")
+    cfg = synth.model_config(model)
+    small = dict(cfg, intermediate=256, vocab=1024, n_layers=1, mask_token_id=1023,
+                 n_target_layers=1)
+    h = DFlash(small, weights_to(synth.make_weights(small, seed=1), DEV), max_position=4096)
+    try:
+        q, kc, vc, table, ref = _attention_case(cfg, seq_lens, seed=len(seq_lens) + 7)
+        h.profile_enable(64)
+        o = h.block_attention(q.to(DEV), torch.tensor(seq_lens, dtype=torch.int32, device=DEV),
+                              torch.tensor(table, device=DEV), kc.to(DEV), vc.to(DEV))
+        torch.cuda.synchronize()
+        prof = h.profile_read()
+        h.profile_disable()
+        assert prof["attention"][0] == 1 and "attn_combine" not in prof   # combined in-cluster
+        got = to_np(o).astype(np.float64).reshape(ref.shape)
+        errs = [rel_l2(got[b * cfg["block_size"]:(b + 1) * cfg["block_size"]],
+                       ref[b * cfg["block_size"]:(b + 1) * cfg["block_size"]])
+                for b in range(len(seq_lens))]
+        assert max(errs) < 1e-3, errs
+        assert h.check_device_errors() == 0
+    finally:
+        h.close()
+
+
 # ----------------------------------------------------------------------------
 # verify / paged slots
 # ----------------------------------------------------------------------------

@@ -270,9 +270,11 @@ def test_qwen3_b1_step():
 
 
 def test_chain_launch_matches_oracle(monkeypatch):
-    """The opt-in one-launch gate/up + down schedule (few rows) gives the same
-    drafts as the oracle outside near-ties, like the default schedule."""
+    """The opt-in schedules — one-launch gate/up + down (few rows) and
+    cluster-combined attention splits — give the same drafts as the oracle
+    outside near-ties, like the default schedule."""
     monkeypatch.setenv("DFLASH_CHAIN", "1")
+    monkeypatch.setenv("DFLASH_ATTN_CLUSTER", "1")
     cfg = dict(synth.model_config("qwen3_8b"), n_layers=1, vocab=8192, mask_token_id=8191)
     Wt = synth.make_weights(cfg, seed=0)
     h = DFlash(cfg, weights_to(Wt, DEV), max_position=4096)
