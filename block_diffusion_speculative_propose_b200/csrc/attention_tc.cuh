@@ -41,6 +41,7 @@ namespace dflash {
 constexpr int kTcKeys = 128;        // keys per tile of the few-request (cluster) variant
 constexpr int kTcKeysSmall = 64;    // keys per tile of the many-request variant (2 CTAs per SM)
 constexpr int kTcStages = 2;        // K/V ring depth
+constexpr int kTcDeepStages = 6;    // K/V ring depth of the one-CTA-per-SM 64-key variant
 constexpr int kTcM = 64;            // MMA M: query rows of a kv group, zero-padded
 constexpr int kTcThreads = 192;     // warp 0 TMA, warp 1 MMA, warps 2..5 softmax
 constexpr float kTcLazyRescale = 8.f;  // log2 of the growth that forces an O rescale
@@ -49,35 +50,38 @@ constexpr float kTcLazyRescale = 8.f;  // log2 of the growth that forces an O re
 // requests, latency); 64-key tiles with one P buffer fit two CTAs per SM
 // (shared memory 100 KB, 256 TMEM columns) so that their pipelines hide each
 // other's latency (many requests, throughput).
-template <int D, int KT>
+template <int D, int KT, int ST = kTcStages>
 struct TcAttnCfg {
   static constexpr int kHalves = D / 64;                      // 64-element halves of a row
   static constexpr int kKVBytes = kHalves * KT * 128;         // one K (or V) tile
   static constexpr int kQBytes = kHalves * kTcM * 128;
   static constexpr int kPBytes = (KT / 64) * kTcM * 128;      // P hi (or lo) of one tile
   static constexpr int kPBufs = KT == 64 ? 1 : 2;             // P buffers (ring of tiles)
-  static constexpr int kOffV = kTcStages * kKVBytes;
-  static constexpr int kOffQ = 2 * kTcStages * kKVBytes;
+  static constexpr int kStages = ST;                          // K/V ring depth
+  static constexpr int kOffV = ST * kKVBytes;
+  static constexpr int kOffQ = 2 * ST * kKVBytes;
   static constexpr int kOffP = kOffQ + kQBytes;
   static constexpr int kOffBar = kOffP + 2 * kPBufs * kPBytes;
   static constexpr int kSmem = 1024 + kOffBar + 256;
   static constexpr int kOCol = 2 * KT;                        // TMEM column of O
   static constexpr int kTmemCols = kOCol + D <= 256 ? 256 : 512;
-  static constexpr int kMinBlocks = KT == 64 ? 2 : 1;
+  static constexpr int kMinBlocks = (KT == 64 && ST == 2) ? 2 : 1;
   // cluster combine, inside the (then idle) K/V ring: received O rows
   // [lr * S + src][D + 8] and (m, l) [lr * S + src] (S * ceil(64 / S) <= 71 slots)
   static constexpr int kCombSlots = kTcM + 7;
   static constexpr int kCombOffML = kCombSlots * (D + 8) * 4;
   static_assert(KT == 64 || KT == 128, "tile width");
-  static_assert(kCombOffML + kCombSlots * 8 <= 2 * kTcStages * kKVBytes, "combine buffers");
+  static_assert(kCombOffML + kCombSlots * 8 <= 2 * ST * kKVBytes, "combine buffers");
+  static_assert(ST >= 2 && ST <= 8, "ring depth");
+  static_assert(kSmem <= 232448, "shared memory");
   static_assert(kOCol + D <= 512, "TMEM budget");
 };
 
-template <int D, int KT>
-__global__ void __launch_bounds__(kTcThreads, TcAttnCfg<D, KT>::kMinBlocks)
+template <int D, int KT, int ST = kTcStages>
+__global__ void __launch_bounds__(kTcThreads, TcAttnCfg<D, KT, ST>::kMinBlocks)
     attn_block_tc_kernel(const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
-  using C = TcAttnCfg<D, KT>;
+  using C = TcAttnCfg<D, KT, ST>;
   pdl_trigger();
   pdl_wait();
   const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -95,16 +99,16 @@ __global__ void __launch_bounds__(kTcThreads, TcAttnCfg<D, KT>::kMinBlocks)
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sQ = smem + C::kOffQ;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
-  uint64_t* kv_full = bars;        // [2]
-  uint64_t* kv_empty = bars + 2;   // [2]
-  uint64_t* s_full = bars + 4;     // [2]
-  uint64_t* s_empty = bars + 6;    // [2]
-  uint64_t* p_full = bars + 8;     // [2]
-  uint64_t* p_empty = bars + 10;   // [2]
-  uint64_t* o_ready = bars + 12;   // one phase per tile: P V of that tile landed
-  uint64_t* q_full = bars + 13;
-  uint64_t* o_final = bars + 14;   // the last tile's P V landed
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
+  uint64_t* kv_full = bars;        // [ST] K/V ring (tile t -> stage t % ST)
+  uint64_t* kv_empty = bars + 8;   // [ST]
+  uint64_t* s_full = bars + 16;    // [2] S buffers (tile t -> t % 2)
+  uint64_t* s_empty = bars + 18;   // [2]
+  uint64_t* p_full = bars + 20;    // [2] P buffers
+  uint64_t* p_empty = bars + 22;   // [2]
+  uint64_t* o_ready = bars + 24;   // one phase per tile: P V of that tile landed
+  uint64_t* q_full = bars + 25;
+  uint64_t* o_final = bars + 26;   // the last tile's P V landed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 27);
   auto sK = [&](int s) { return smem + s * C::kKVBytes; };
   auto sV = [&](int s) { return smem + C::kOffV + s * C::kKVBytes; };
   auto sP = [&](int lohi, int buf) {
@@ -112,9 +116,11 @@ __global__ void __launch_bounds__(kTcThreads, TcAttnCfg<D, KT>::kMinBlocks)
   };
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < ST; ++i) {
       mbar_init(&kv_full[i], 1);
       mbar_init(&kv_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&s_empty[i], 4);
       mbar_init(&p_full[i], 4);
@@ -145,7 +151,7 @@ __global__ void __launch_bounds__(kTcThreads, TcAttnCfg<D, KT>::kMinBlocks)
       tma_prefetch_desc(&tmV);
       const int* bt = p.block_table + static_cast<size_t>(b) * p.W;
       for (int t = 0; t < n_tiles; ++t) {
-        const int s = t & 1, u = t >> 1;
+        const int s = t % ST, u = t / ST;
         if (!mbar_wait(&kv_empty[s], (u & 1) ^ 1u, p.err)) break;
         const int t0 = k0 + t * KT;
         const int nvalid = min(KT, k1 - t0);
@@ -181,15 +187,16 @@ __global__ void __launch_bounds__(kTcThreads, TcAttnCfg<D, KT>::kMinBlocks)
       bool ok = n_tiles > 0 && mbar_wait(q_full, 0, p.err);
       tc_fence_after();
       auto issue_qk = [&](int t) -> bool {
-        const int s = t & 1, u = t >> 1;
-        if (!mbar_wait(&kv_full[s], u & 1, p.err)) return false;
+        const int kv = t % ST, kvu = t / ST;      // K/V ring stage
+        const int s = t & 1, u = t >> 1;          // S buffer
+        if (!mbar_wait(&kv_full[kv], kvu & 1, p.err)) return false;
         if (!mbar_wait(&s_empty[s], (u & 1) ^ 1u, p.err)) return false;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int half = kk >> 2, w = kk & 3;
           const uint64_t ad = umma_desc_sw128(smem_u32(sQ + half * kTcM * 128 + w * 32));
-          const uint64_t bd = umma_desc_sw128(smem_u32(sK(s) + half * KT * 128 + w * 32));
+          const uint64_t bd = umma_desc_sw128(smem_u32(sK(kv) + half * KT * 128 + w * 32));
           umma_f16kind(tmem_base + s * KT, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
         }
         umma_commit(&s_full[s]);
@@ -201,7 +208,8 @@ __global__ void __launch_bounds__(kTcThreads, TcAttnCfg<D, KT>::kMinBlocks)
         // (its softmax then overlaps P V); otherwise P V(t) is issued first
         // instead of waiting on the load
         const int s1 = (t + 1) & 1, u1 = (t + 1) >> 1;
-        const bool qk_first = t + 1 < n_tiles && mbar_try_wait(&kv_full[s1], u1 & 1) &&
+        const int kv1 = (t + 1) % ST, kvu1 = (t + 1) / ST;
+        const bool qk_first = t + 1 < n_tiles && mbar_try_wait(&kv_full[kv1], kvu1 & 1) &&
                               mbar_try_wait(&s_empty[s1], (u1 & 1) ^ 1u);
         if (qk_first && !issue_qk(t + 1)) break;
         const int s = t & 1, u = t >> 1;
@@ -213,13 +221,13 @@ __global__ void __launch_bounds__(kTcThreads, TcAttnCfg<D, KT>::kMinBlocks)
           for (int kk = 0; kk < KT / 16; ++kk) {
             const int kh = kk >> 2, w = kk & 3;
             const uint64_t ad = umma_desc_sw128(smem_u32(sP(lohi, s) + kh * kTcM * 128 + w * 32));
-            const uint64_t bd = umma_desc_sw128_mn(smem_u32(sV(s) + kk * 16 * 128),
+            const uint64_t bd = umma_desc_sw128_mn(smem_u32(sV(t % ST) + kk * 16 * 128),
                                                    KT * 128, 1024);
             umma_f16kind(tmem_base + C::kOCol, ad, bd, idesc_pv,
                          (t > 0 || lohi > 0 || kk > 0) ? 1u : 0u);
           }
         }
-        umma_commit(&kv_empty[s]);
+        umma_commit(&kv_empty[t % ST]);
         umma_commit(&p_empty[s]);
         umma_commit(o_ready);
         if (t + 1 == n_tiles) umma_commit(o_final);
@@ -376,8 +384,8 @@ __global__ void __launch_bounds__(kTcThreads, TcAttnCfg<D, KT>::kMinBlocks)
           const int hf = e / ((16 - rr0) * 8);
           const int rem = e - hf * (16 - rr0) * 8;
           const int rr = rr0 + rem / 8, cc = rem & 7;
-          *reinterpret_cast<uint4*>(sV(s) + hf * KT * 128 + jp * 2048 + rr * 128 + cc * 16) =
-              make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4*>(sV(t % ST) + hf * KT * 128 + jp * 2048 + rr * 128 +
+                                    cc * 16) = make_uint4(0, 0, 0, 0);
         }
       }
       fence_proxy_async_smem();

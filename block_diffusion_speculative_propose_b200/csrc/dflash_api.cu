@@ -206,12 +206,15 @@ struct AttnPlan {
   int chunk_keys = 0, max_splits = 0, R = 0, row_groups = 0, key_parts = 0, nwc = 0;
   bool tc = false;   // tcgen05 kernel (kv groups of up to 64 query rows)
   int kt = 128;      // tcgen05 kernel: keys per tile
+  int st = 2;        // tcgen05 kernel: K/V ring depth (64-key tiles: 2 -> two CTAs per SM)
   bool cluster = false;  // tcgen05 kernel, splits of a (request, kv head) combined in a cluster
   size_t part_o_bytes = 0, part_ml_bytes = 0;
 };
 
+// forced_ring: K/V ring depth of the 64-key tcgen05 kernel (2 or 6), or 0 to
+// let the planner decide.
 AttnPlan plan_attention(int B, int Hkv, int W, int P, int bs, int G, int D, int num_sms,
-                        bool allow_cluster) {
+                        bool allow_cluster, int forced_ring) {
   AttnPlan a;
   const int keys_max = W * P;
   const double est = static_cast<double>(B) * Hkv * keys_max;
@@ -224,6 +227,14 @@ AttnPlan plan_attention(int B, int Hkv, int W, int P, int bs, int G, int D, int 
   chunk = std::max(128, std::min(8192, chunk));
   a.chunk_keys = chunk;
   a.max_splits = cdiv(keys_max, chunk);
+  // Ring depth: a split of at least 2 x 6 tiles keeps a six-deep ring busy, and
+  // one CTA per SM with six 64-key tiles in flight then beats two CTAs with two
+  // each.  Measured on the Qwen3-8B shape: batch 32, contexts U[512, 8192]
+  // (56-tile splits): 234 -> 191 us per layer; batch 32 x 8192: 366 -> 358 us;
+  // batch 128 x 4096: 586 -> 604 us; short splits (batch 2-4, 2-4 tiles) lose
+  // 25-30%, so they keep the two-CTA ring.
+  a.st = (chunk / kTcKeysSmall >= 2 * kTcDeepStages) ? kTcDeepStages : kTcStages;
+  if (forced_ring == kTcStages || forced_ring == kTcDeepStages) a.st = forced_ring;
   a.row_groups = cdiv(a.R, 16);
   a.key_parts = 1;
   while (a.key_parts < 4 && a.row_groups * a.key_parts * 2 <= kAttnMaxComputeWarps)
@@ -321,6 +332,12 @@ struct dflash_handle {
   bool attn_cluster = [] {
     const char* e = std::getenv("DFLASH_ATTN_CLUSTER");
     return e && e[0] == '1';
+  }();
+  // K/V ring depth of the 64-key attention kernel forced by DFLASH_ATTN_STAGES
+  // (2 or 6) when the handle is created; 0 lets the planner decide
+  int attn_ring = [] {
+    const char* e = std::getenv("DFLASH_ATTN_STAGES");
+    return e ? std::atoi(e) : 0;
   }();
   std::vector<cudaEvent_t> prof_events;
   size_t prof_next = 0;
@@ -669,6 +686,10 @@ cudaError_t set_attn_attrs() {
                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 TcAttnCfg<D, kTcKeysSmall>::kSmem)) != cudaSuccess)
     return e;
+  if ((e = cudaFuncSetAttribute(attn_block_tc_kernel<D, kTcKeysSmall, kTcDeepStages>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                TcAttnCfg<D, kTcKeysSmall, kTcDeepStages>::kSmem)) != cudaSuccess)
+    return e;
   return cudaFuncSetAttribute(attn_block_tc_kernel<D, kTcKeys>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize,
                               TcAttnCfg<D, kTcKeys>::kSmem);
@@ -691,7 +712,11 @@ dflash_status run_attention(dflash_handle* h, const AttnPlan& ap, AttnParams prm
   prm.cluster = ap.cluster ? 1 : 0;
   if (ap.tc) {
     LaunchScope scope(h, DFLASH_KERNEL_ATTENTION, st);
-    if (ap.kt == kTcKeysSmall)
+    if (ap.kt == kTcKeysSmall && ap.st == kTcDeepStages)
+      launch_kc(h->pdl, ap.cluster ? ap.max_splits : 1,
+                attn_block_tc_kernel<D, kTcKeysSmall, kTcDeepStages>, grid, dim3(kTcThreads),
+                TcAttnCfg<D, kTcKeysSmall, kTcDeepStages>::kSmem, st, tk, tv, prm);
+    else if (ap.kt == kTcKeysSmall)
       launch_kc(h->pdl, ap.cluster ? ap.max_splits : 1, attn_block_tc_kernel<D, kTcKeysSmall>,
                 grid, dim3(kTcThreads), TcAttnCfg<D, kTcKeysSmall>::kSmem, st, tk, tv, prm);
     else
@@ -765,7 +790,7 @@ ProposeWs propose_layout(const dflash_handle* h, int B, int W) {
   // the attention split plan is not monotonic in the batch: cover every size
   for (int bb = 1; bb <= B; ++bb) {
     const AttnPlan ap = plan_attention(bb, Hkv, W, c.page_size, bs, Hq / Hkv, D, h->num_sms,
-                                       h->attn_cluster);
+                                       h->attn_cluster, h->attn_ring);
     po = std::max(po, ap.part_o_bytes);
     pm = std::max(pm, ap.part_ml_bytes);
   }
@@ -860,7 +885,7 @@ dflash_status propose_layers(dflash_handle* h, const ProposeWs& lw, void* ws,
   f16* frows = at<f16>(ws, lw.frows);
   float* partial = at<float>(ws, lw.partial);
   const AttnPlan ap = plan_attention(B, Hkv, W, c.page_size, bs, Hq / Hkv, D, h->num_sms,
-                                     h->attn_cluster);
+                                     h->attn_cluster, h->attn_ring);
   if (ap.part_o_bytes > lw.part_o_cap || ap.part_ml_bytes > lw.part_ml_cap)
     return DFLASH_ERR_WORKSPACE;
   AttnParams prm;
@@ -1467,7 +1492,7 @@ size_t dflash_attention_workspace_bytes(const dflash_handle* h, int B, int max_p
   const dflash_config& c = h->cfg;
   const AttnPlan ap = plan_attention(B, c.n_kv_heads, max_pages_per_seq, c.page_size,
                                      c.block_size, c.n_q_heads / c.n_kv_heads, c.head_dim,
-                                     h->num_sms, h->attn_cluster);
+                                     h->num_sms, h->attn_cluster, h->attn_ring);
   return align_up(ap.part_o_bytes) + align_up(ap.part_ml_bytes) + kAlign;
 }
 
@@ -1487,7 +1512,7 @@ dflash_status dflash_block_attention(dflash_handle* h, const void* q, const int3
   DF_CUDA(use_device(h->device));
   const AttnPlan ap = plan_attention(B, c.n_kv_heads, max_pages_per_seq, c.page_size,
                                      c.block_size, c.n_q_heads / c.n_kv_heads, c.head_dim,
-                                     h->num_sms, h->attn_cluster);
+                                     h->num_sms, h->attn_cluster, h->attn_ring);
   AttnParams prm;
   prm.q = static_cast<const bf16*>(q);
   prm.o = static_cast<f16*>(o);

@@ -207,6 +207,36 @@ def test_block_attention_cluster_combine(monkeypatch, model, seq_lens):
         h.close()
 
 
+@pytest.mark.parametrize("ring", [2, 6])
+@pytest.mark.parametrize("model,seq_lens", [
+    ("tiny", [0, 1, 15, 16, 17, 63, 64, 65, 200]),
+    ("qwen3_8b", [0, 7, 100, 1000, 5000]),
+    ("llama31_8b", [3, 333, 4097]),
+])
+def test_block_attention_ring_depth(monkeypatch, ring, model, seq_lens):
+    """Both K/V ring depths of the 64-key kernel (two stages at two CTAs per
+    SM, six stages at one), forced regardless of what the planner picks."""
+    monkeypatch.setenv("DFLASH_ATTN_STAGES", str(ring))
+    cfg = synth.model_config(model)
+    small = dict(cfg, intermediate=256, vocab=1024, n_layers=1, mask_token_id=1023,
+                 n_target_layers=1)
+    h = DFlash(small, weights_to(synth.make_weights(small, seed=1), DEV), max_position=4096)
+    try:
+        q, kc, vc, table, ref = _attention_case(cfg, seq_lens, seed=len(seq_lens) + 11)
+        o = h.block_attention(q.to(DEV), torch.tensor(seq_lens, dtype=torch.int32, device=DEV),
+                              torch.tensor(table, device=DEV), kc.to(DEV), vc.to(DEV))
+        torch.cuda.synchronize()
+        got = to_np(o).astype(np.float64).reshape(ref.shape)
+        assert np.isfinite(got).all()
+        errs = [rel_l2(got[b * cfg["block_size"]:(b + 1) * cfg["block_size"]],
+                       ref[b * cfg["block_size"]:(b + 1) * cfg["block_size"]])
+                for b in range(len(seq_lens))]
+        assert max(errs) < 1e-3, errs
+        assert h.check_device_errors() == 0
+    finally:
+        h.close()
+
+
 # ----------------------------------------------------------------------------
 # verify / paged slots
 # ----------------------------------------------------------------------------
