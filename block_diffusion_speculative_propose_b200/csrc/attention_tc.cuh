@@ -6,11 +6,13 @@
 // heads, zero-padded to 64 rows) attends to the request's keys
 // [split * chunk, ...) of [0, seq_len + bs) with no mask inside the range.
 //
-//   warp 0      TMA producer: walks the block table, stages 128-key tiles of
-//               K and V (eight 16-key pages, 128-byte swizzle) in a 2-deep ring
+//   warp 0      TMA producer: walks the block table, stages KT-key tiles of K
+//               and V (KT / 16 pages of 16 keys, 128-byte swizzle) in a ring of
+//               ST tiles
 //   warp 1      MMA issuer (one thread): S = Q K^T into a double-buffered TMEM
-//               S (M=64 rows x 128 keys), then O += P_hi V + P_lo V into TMEM
-//               O (64 x d); S of tile t+1 is issued before P V of tile t
+//               S (M=64 rows x KT keys), then O += P_hi V + P_lo V into TMEM O
+//               (64 x d); S of tile t+1 is issued before P V of tile t when its
+//               K/V have landed
 //   warps 2..5  softmax: each reads its 16 rows of S with tcgen05.ld.16x256b
 //               (the mma.sync accumulator-fragment layout), applies the online
 //               softmax (row statistics by quad shuffles), writes P split into
@@ -19,11 +21,17 @@
 //               2^8 since the last rescale (the reference maximum is shared by P,
 //               the row sum and O, so the result is exact either way).
 //
-// Shared memory: K/V ring 2 x (K + V) tiles, Q (64 x d), P hi/lo x 2 buffers.
-// TMEM: S buffers at columns [0, 256), O at [256, 256 + d).  Every wait is
-// bounded; a wait that runs out sets the timeout bit and the CTA winds down.
+// Variants <D, KT, ST>: 128-key tiles with a 2-deep ring and two P buffers
+// (the opt-in cluster mode below); 64-key tiles with one P buffer and a 2-deep
+// ring (100 KB of shared memory: two CTAs per SM) or a 6-deep ring (231 KB:
+// one CTA per SM, six tiles in flight, for long key splits).
 //
-// Cluster mode (few requests: splitting the keys is what fills the GPU): the
+// Shared memory: K/V ring ST x (K + V) tiles, Q (64 x d), P hi/lo x 1 or 2
+// buffers, barriers.  TMEM: S buffers at columns [0, 2 KT), O at
+// [2 KT, 2 KT + d).  Every wait is bounded; a wait that runs out sets the
+// timeout bit and the CTA winds down.
+//
+// Cluster mode (opt-in; few requests: splitting the keys is what fills the GPU): the
 // splits of one (request, kv head) are the CTAs of one cluster; CTA rank q
 // owns rows q, q + S, ...  Once every CTA of the cluster is past its key loop
 // (first cluster barrier), each pushes its unnormalised O rows and (m, l)
@@ -46,10 +54,11 @@ constexpr int kTcM = 64;            // MMA M: query rows of a kv group, zero-pad
 constexpr int kTcThreads = 192;     // warp 0 TMA, warp 1 MMA, warps 2..5 softmax
 constexpr float kTcLazyRescale = 8.f;  // log2 of the growth that forces an O rescale
 
-// Per tile width KT (keys): 128-key tiles keep more keys in flight per CTA (few
-// requests, latency); 64-key tiles with one P buffer fit two CTAs per SM
-// (shared memory 100 KB, 256 TMEM columns) so that their pipelines hide each
-// other's latency (many requests, throughput).
+// Per tile width KT (keys) and ring depth ST: 128-key tiles keep more keys in
+// flight per CTA (the cluster mode); 64-key tiles with one P buffer and a
+// 2-deep ring fit two CTAs per SM (shared memory 100 KB, 256 TMEM columns) so
+// that their pipelines hide each other's latency; with a 6-deep ring one CTA
+// per SM keeps six tiles in flight.
 template <int D, int KT, int ST = kTcStages>
 struct TcAttnCfg {
   static constexpr int kHalves = D / 64;                      // 64-element halves of a row
