@@ -471,7 +471,46 @@ def extra_measurements(st, peaks) -> dict:
                                                       c["page_size"], c["vocab"], ver, nd),
                       dev, reps=20)
     out["prepare_proposal_inputs"] = {"rows": int(tp.numel()), "us": t * 1e6}
+    out["spec_step_graph"] = spec_step_graph(st)
     return out
+
+
+def spec_step_graph(st, reps: int = 20) -> dict:
+    """The closed-loop speculative step through the library's own CUDA graph
+    (dflash_step_graph_create / _launch): verify the workload's drafts against
+    its target logits, prepare the proposal inputs on the device, inject all
+    K+1 verified rows of every request and propose the next block — nothing
+    from the host between the stages.  The verified rows end where the
+    workload's context ends, so every block lies inside the block table."""
+    c, dev, K, B = st.cfg, st.dev, st.K, st.B
+    T, H = c["n_target_layers"], c["hidden"]
+    starts = (st.sb.seq_lens.to(torch.int64) - (K + 1)).clamp(min=0).to(dev)
+    tp = (starts[:, None] + torch.arange(K + 1, device=dev)[None, :]).reshape(-1)
+    last = ((torch.arange(B, device=dev) + 1) * (K + 1) - 1).to(torch.int32)
+    nd = torch.full((B,), K, dtype=torch.int32, device=dev)
+    g0 = torch.Generator(device=dev)
+    g0.manual_seed(13)
+    aux = torch.randn(B * (K + 1), T * H, generator=g0, device=dev).to(torch.bfloat16)
+    g = st.h.step_graph(st.inp["prev_drafts"], st.inp["target_logits"], tp, last, nd, aux,
+                        st.inp["block_table"], st.kc, st.vc)
+    try:
+        for _ in range(3):
+            g.launch()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            g.launch()
+        e1.record()
+        torch.cuda.synchronize(dev)
+        t = e0.elapsed_time(e1) / 1e3 / reps
+        if st.h.check_device_errors():
+            raise RuntimeError("device error in the closed-loop step")
+        acc = float(g.out["num_accepted"].float().mean())
+    finally:
+        g.close()
+    return {"rows": int(tp.numel()), "us": t * 1e6, "blocks_per_s": B / t,
+            "mean_accepted": acc, "launches": reps}
 
 
 def run_ours(a, rank, world, local):

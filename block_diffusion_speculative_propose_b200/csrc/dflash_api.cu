@@ -1446,6 +1446,163 @@ dflash_status dflash_verify_greedy(const int32_t* drafts, const float* target_lo
   return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ERR_CUDA;
 }
 
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// the whole speculative step
+// ---------------------------------------------------------------------------
+namespace {
+struct StepWs {
+  size_t ver = 0, inj = 0, prop = 0, total = 0;
+};
+StepWs step_layout(const dflash_handle* h, int B, int n, int W) {
+  StepWs w;
+  const int K = h->cfg.block_size - 1;
+  size_t off = 0;
+  w.ver = off;
+  off += align_up(std::max<size_t>(plan_verify(B, K, h->cfg.vocab).bytes, kAlign));
+  w.inj = off;
+  off += align_up(std::max<size_t>(inject_layout(h, n).total, kAlign));
+  w.prop = off;
+  off += align_up(propose_layout(h, B, W).total);
+  w.total = off;
+  return w;
+}
+
+// Every host check of the four calls of the step, before any launch.
+dflash_status check_step(const dflash_handle* h, const dflash_step_io* io, const void* ws,
+                         size_t bytes) {
+  if (!h || !io || io->B < 0 || io->n < 0) return DFLASH_ERR_INVALID_ARG;
+  if (io->B == 0) return DFLASH_OK;
+  const dflash_config& c = h->cfg;
+  const int K = c.block_size - 1;
+  if (io->n < io->B || K > 128 || io->max_pages_per_seq < 1 || io->num_pages < 1)
+    return DFLASH_ERR_INVALID_ARG;
+  if ((K > 0 && !io->prev_drafts) || !io->target_logits || !io->target_positions ||
+      !io->last_token_indices || !io->num_draft || !io->aux || !io->block_table ||
+      !io->k_cache || !io->v_cache || !io->out_tokens || !io->num_accepted || !io->positions ||
+      !io->slot_mapping || !io->seq_lens || !io->bonus || !io->draft_tokens || !ws)
+    return DFLASH_ERR_INVALID_ARG;
+  if ((io->prev_sampled == nullptr) != (io->prev_num_draft == nullptr))
+    return DFLASH_ERR_INVALID_ARG;
+  if (io->prev_sampled && io->prev_width < 1) return DFLASH_ERR_INVALID_ARG;
+  for (int l = 0; l < c.n_layers; ++l)
+    if (!io->k_cache[l] || !io->v_cache[l]) return DFLASH_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(ws) % kAlign) return DFLASH_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(io->target_logits) % 16 && c.vocab % 4 == 0)
+    return DFLASH_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(io->B) * c.block_size > (1 << 24))
+    return DFLASH_ERR_UNSUPPORTED_SHAPE;
+  if (bytes < step_layout(h, io->B, io->n, io->max_pages_per_seq).total)
+    return DFLASH_ERR_WORKSPACE;
+  return DFLASH_OK;
+}
+}  // namespace
+
+struct dflash_step_graph {
+  int device = 0;
+  cudaGraph_t graph = nullptr;
+  cudaGraphExec_t exec = nullptr;
+};
+
+extern "C" {
+
+size_t dflash_spec_step_workspace_bytes(const dflash_handle* h, int B, int n,
+                                        int max_pages_per_seq) {
+  if (!h || B <= 0 || n < B || max_pages_per_seq <= 0) return 0;
+  return step_layout(h, B, n, max_pages_per_seq).total;
+}
+
+dflash_status dflash_spec_step(dflash_handle* h, const dflash_step_io* io, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+  dflash_status s = check_step(h, io, workspace, workspace_bytes);
+  if (s != DFLASH_OK || io->B == 0) return s;
+  DF_CUDA(use_device(h->device));
+  const dflash_config& c = h->cfg;
+  const int B = io->B, n = io->n, K = c.block_size - 1, W = io->max_pages_per_seq;
+  const StepWs w = step_layout(h, B, n, W);
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  // 1. greedy verification of the previous drafts
+  s = dflash_verify_greedy(io->prev_drafts, io->target_logits, B, K, c.vocab, io->out_tokens,
+                           io->num_accepted, io->bonus, base + w.ver, w.inj - w.ver, stream);
+  if (s != DFLASH_OK) return s;
+  // 2. corrected positions, context slots, post-verify lengths, bonus tokens
+  s = dflash_prepare_proposal_inputs(
+      io->target_positions, n, io->last_token_indices, B, io->out_tokens, K + 1, io->num_draft,
+      io->prev_sampled, io->prev_width, io->prev_num_draft, io->block_table, W, c.page_size,
+      c.vocab, io->positions, io->slot_mapping, io->seq_lens, io->bonus,
+      io->device_error ? io->device_error : h->dev_err, stream);
+  if (s != DFLASH_OK) return s;
+  // 3. context fusion and K/V injection of the target rows
+  s = dflash_inject_context(h, io->aux, io->positions, io->slot_mapping, n, io->k_cache,
+                            io->v_cache, io->num_pages, base + w.inj, w.prop - w.inj, stream);
+  if (s != DFLASH_OK) return s;
+  // 4. the next block's drafts
+  return dflash_propose(h, io->bonus, io->seq_lens, io->block_table, B, W, io->k_cache,
+                        io->v_cache, io->num_pages, io->draft_tokens, io->block_tokens, nullptr,
+                        base + w.prop, w.total - w.prop, stream);
+}
+
+dflash_status dflash_step_graph_create(dflash_handle* h, const dflash_step_io* io,
+                                       void* workspace, size_t workspace_bytes,
+                                       dflash_step_graph** out) {
+  if (!out) return DFLASH_ERR_INVALID_ARG;
+  *out = nullptr;
+  dflash_status s = check_step(h, io, workspace, workspace_bytes);
+  if (s != DFLASH_OK) return s;
+  // per-launch profiling events would be baked into the graph
+  if (h->prof_on) return DFLASH_ERR_INVALID_ARG;
+  auto* g = new (std::nothrow) dflash_step_graph;
+  if (!g) return DFLASH_ERR_CUDA;
+  g->device = h->device;
+  if (io->B == 0) {  // nothing to run: launches are no-ops
+    *out = g;
+    return DFLASH_OK;
+  }
+  if (use_device(h->device) != cudaSuccess) {
+    delete g;
+    return DFLASH_ERR_CUDA;
+  }
+  cudaStream_t cs = nullptr;
+  if (cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking) != cudaSuccess) {
+    cudaGetLastError();
+    delete g;
+    return DFLASH_ERR_CUDA;
+  }
+  cudaError_t e = cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal);
+  if (e == cudaSuccess) {
+    s = dflash_spec_step(h, io, workspace, workspace_bytes, cs);
+    e = cudaStreamEndCapture(cs, &g->graph);
+  }
+  cudaStreamDestroy(cs);
+  if (s == DFLASH_OK && e == cudaSuccess && g->graph)
+    e = cudaGraphInstantiate(&g->exec, g->graph, 0);
+  if (s != DFLASH_OK || e != cudaSuccess || !g->exec) {
+    cudaGetLastError();
+    if (g->graph) cudaGraphDestroy(g->graph);
+    delete g;
+    return s != DFLASH_OK ? s : DFLASH_ERR_CUDA;
+  }
+  *out = g;
+  return DFLASH_OK;
+}
+
+dflash_status dflash_step_graph_launch(dflash_step_graph* g, void* stream) {
+  if (!g) return DFLASH_ERR_INVALID_ARG;
+  if (!g->exec) return DFLASH_OK;
+  DF_CUDA(use_device(g->device));
+  DF_CUDA(cudaGraphLaunch(g->exec, static_cast<cudaStream_t>(stream)));
+  return DFLASH_OK;
+}
+
+void dflash_step_graph_destroy(dflash_step_graph* g) {
+  if (!g) return;
+  use_device(g->device);
+  if (g->exec) cudaGraphExecDestroy(g->exec);
+  if (g->graph) cudaGraphDestroy(g->graph);
+  delete g;
+}
+
 size_t dflash_linear_workspace_bytes(const dflash_handle* h, int M, int N, int K) {
   if (!h || M <= 0 || N <= 0 || K <= 0) return 0;
   return align_up(std::max<size_t>(plan_gemm(M, N, K, 32, h->num_sms).partial_bytes, kAlign));

@@ -59,6 +59,21 @@ class _Weights(ctypes.Structure):
                            "k_norm_w", "w_gate", "w_up", "w_down")]
 
 
+class _StepIO(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("n", ctypes.c_int),
+                ("prev_drafts", ctypes.c_void_p), ("target_logits", ctypes.c_void_p),
+                ("target_positions", ctypes.c_void_p), ("last_token_indices", ctypes.c_void_p),
+                ("num_draft", ctypes.c_void_p), ("prev_sampled", ctypes.c_void_p),
+                ("prev_width", ctypes.c_int), ("prev_num_draft", ctypes.c_void_p),
+                ("aux", ctypes.c_void_p), ("block_table", ctypes.c_void_p),
+                ("max_pages_per_seq", ctypes.c_int), ("k_cache", _PP), ("v_cache", _PP),
+                ("num_pages", ctypes.c_int), ("out_tokens", ctypes.c_void_p),
+                ("num_accepted", ctypes.c_void_p), ("positions", ctypes.c_void_p),
+                ("slot_mapping", ctypes.c_void_p), ("seq_lens", ctypes.c_void_p),
+                ("bonus", ctypes.c_void_p), ("draft_tokens", ctypes.c_void_p),
+                ("block_tokens", ctypes.c_void_p), ("device_error", ctypes.c_void_p)]
+
+
 _lib = None
 
 
@@ -89,6 +104,12 @@ def lib() -> ctypes.CDLL:
                            i32),
         "dflash_verify_greedy": ([vp, vp, i32, i32, i32, vp, vp, vp, vp, sz, vp], i32),
         "dflash_verify_greedy_noalloc": ([vp, vp, i32, i32, i32, vp, vp, vp, vp], i32),
+        "dflash_spec_step_workspace_bytes": ([vp, i32, i32, i32], sz),
+        "dflash_spec_step": ([vp, ctypes.POINTER(_StepIO), vp, sz, vp], i32),
+        "dflash_step_graph_create": ([vp, ctypes.POINTER(_StepIO), vp, sz, ctypes.POINTER(vp)],
+                                     i32),
+        "dflash_step_graph_launch": ([vp, vp], i32),
+        "dflash_step_graph_destroy": ([vp], None),
         "dflash_linear": ([vp, vp, vp, i32, i32, i32, vp, vp, sz, vp], i32),
         "dflash_linear_ex": ([vp, vp, vp, i32, i32, i32, vp, i32, i32, vp, sz, vp], i32),
         "dflash_block_attention": ([vp, vp, vp, vp, i32, i32, vp, vp, i32, vp, vp, sz, vp],
@@ -264,6 +285,87 @@ class DFlash:
                "dflash_propose")
         return draft_tokens
 
+    def spec_step_workspace_bytes(self, B: int, n: int, max_pages_per_seq: int) -> int:
+        return lib().dflash_spec_step_workspace_bytes(self.h, B, n, max_pages_per_seq)
+
+    def _step_io(self, prev_drafts, target_logits, target_positions, last_token_indices,
+                 num_draft, aux, block_table, k_cache, v_cache, prev_sampled, prev_num_draft,
+                 out, device_error):
+        """Marshal the buffers of one speculative step into dflash_step_io;
+        returns (io, outputs, objects to keep alive)."""
+        B, n = int(last_token_indices.shape[0]), int(target_positions.shape[0])
+        bs = self.cfg["block_size"]
+        _want(prev_drafts, torch.int32, "prev_drafts")
+        _want(target_logits, torch.float32, "target_logits")
+        _want(target_positions, torch.int64, "target_positions")
+        _want(last_token_indices, torch.int32, "last_token_indices")
+        _want(num_draft, torch.int32, "num_draft")
+        _want(aux, torch.bfloat16, "aux")
+        _want(block_table, torch.int32, "block_table")
+        if prev_sampled is not None:
+            _want(prev_sampled, torch.int32, "prev_sampled")
+        if prev_num_draft is not None:
+            _want(prev_num_draft, torch.int32, "prev_num_draft")
+        dev = self.device
+        o = dict(out or {})
+        shapes = {"out_tokens": ((B, bs), torch.int32), "num_accepted": ((B,), torch.int32),
+                  "positions": ((n,), torch.int64), "slot_mapping": ((n,), torch.int64),
+                  "seq_lens": ((B,), torch.int32), "bonus": ((B,), torch.int32),
+                  "draft_tokens": ((B, bs - 1), torch.int32),
+                  "block_tokens": ((B, bs), torch.int32)}
+        for k, (shape, dt) in shapes.items():
+            if k not in o:
+                o[k] = torch.empty(shape, dtype=dt, device=dev)
+            _want(o[k], dt, k)
+        kp, ka = _ptr_array(k_cache)
+        vp, va = _ptr_array(v_cache)
+        io = _StepIO(B, n, _ptr(prev_drafts), _ptr(target_logits), _ptr(target_positions),
+                     _ptr(last_token_indices), _ptr(num_draft), _ptr(prev_sampled),
+                     int(prev_sampled.shape[1]) if prev_sampled is not None else 0,
+                     _ptr(prev_num_draft), _ptr(aux), _ptr(block_table),
+                     int(block_table.shape[1]), kp, vp, int(k_cache[0].shape[0]),
+                     _ptr(o["out_tokens"]), _ptr(o["num_accepted"]), _ptr(o["positions"]),
+                     _ptr(o["slot_mapping"]), _ptr(o["seq_lens"]), _ptr(o["bonus"]),
+                     _ptr(o["draft_tokens"]), _ptr(o["block_tokens"]), _ptr(device_error))
+        keep = [prev_drafts, target_logits, target_positions, last_token_indices, num_draft,
+                aux, block_table, list(k_cache), list(v_cache), prev_sampled, prev_num_draft,
+                device_error, ka, va]
+        return io, o, keep
+
+    def spec_step(self, prev_drafts, target_logits, target_positions, last_token_indices,
+                  num_draft, aux, block_table, k_cache, v_cache, prev_sampled=None,
+                  prev_num_draft=None, out=None, device_error=None, workspace=None,
+                  stream=None) -> Dict[str, torch.Tensor]:
+        """One whole speculative step (dflash_spec_step): verify -> prepare ->
+        inject -> propose on the device.  Returns the outputs by name
+        (out_tokens, num_accepted, positions, slot_mapping, seq_lens, bonus,
+        draft_tokens, block_tokens); tensors given in ``out`` are written in place."""
+        io, o, keep = self._step_io(prev_drafts, target_logits, target_positions,
+                                    last_token_indices, num_draft, aux, block_table, k_cache,
+                                    v_cache, prev_sampled, prev_num_draft, out, device_error)
+        need = self.spec_step_workspace_bytes(io.B, io.n, io.max_pages_per_seq) if io.B else 0
+        ws = workspace if workspace is not None else self.ws.get(need)
+        _check(lib().dflash_spec_step(self.h, ctypes.byref(io), _ptr(ws), ws.numel(),
+                                      _stream(stream)), "dflash_spec_step")
+        return o
+
+    def step_graph(self, prev_drafts, target_logits, target_positions, last_token_indices,
+                   num_draft, aux, block_table, k_cache, v_cache, prev_sampled=None,
+                   prev_num_draft=None, out=None, device_error=None,
+                   workspace=None) -> "StepGraph":
+        """The same step captured once into a library-owned CUDA graph
+        (dflash_step_graph_create) over these buffers; see StepGraph."""
+        io, o, keep = self._step_io(prev_drafts, target_logits, target_positions,
+                                    last_token_indices, num_draft, aux, block_table, k_cache,
+                                    v_cache, prev_sampled, prev_num_draft, out, device_error)
+        need = self.spec_step_workspace_bytes(io.B, io.n, io.max_pages_per_seq) if io.B else 0
+        ws = workspace if workspace is not None else torch.empty(
+            max(need, 256), dtype=torch.uint8, device=self.device)
+        g = ctypes.c_void_p()
+        _check(lib().dflash_step_graph_create(self.h, ctypes.byref(io), _ptr(ws), ws.numel(),
+                                              ctypes.byref(g)), "dflash_step_graph_create")
+        return StepGraph(self, g, o, keep + [ws, io])
+
     def linear(self, A, W, out=None, block_n: int = 0, splits: int = 0, workspace=None,
                stream=None):
         M, K = A.shape
@@ -322,6 +424,35 @@ class DFlash:
         bits = ctypes.c_uint(0)
         lib().dflash_check_device_errors(self.h, ctypes.byref(bits))
         return int(bits.value)
+
+
+class StepGraph:
+    """A speculative step captured into a CUDA graph owned by the library.
+    ``launch()`` replays it on a stream; ``out`` holds its output tensors.  The
+    graph keeps the pointers of the buffers it was built on (held here): write
+    new inputs into those tensors between launches."""
+
+    def __init__(self, owner: DFlash, g, out: Dict[str, torch.Tensor], keep: List):
+        self._owner = owner     # the handle must outlive the graph
+        self.g = g
+        self.out = out
+        self._keep = keep
+
+    def launch(self, stream=None) -> None:
+        _check(lib().dflash_step_graph_launch(self.g, _stream(stream)),
+               "dflash_step_graph_launch")
+
+    def close(self) -> None:
+        if getattr(self, "g", None):
+            torch.cuda.synchronize(self._owner.device)
+            lib().dflash_step_graph_destroy(self.g)
+            self.g = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 def verify_workspace_bytes(B: int, K: int, V: int) -> int:

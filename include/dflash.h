@@ -296,6 +296,109 @@ dflash_status dflash_verify_greedy(const int32_t* drafts, const float* target_lo
                                    void* workspace, size_t workspace_bytes,
                                    void* stream);
 
+/* ---- the whole speculative step ------------------------------------------ */
+
+/* Buffers of one speculative-decoding step (dflash_spec_step).  Device
+ * pointers, caller-owned; K = block_size - 1, V = vocab, n target rows.
+ * Inputs:
+ *   prev_drafts        [B, K] int32   the drafts the target has just scored
+ *   target_logits      [B, K+1, V] fp32  the target's predictions after each
+ *                      verified slot (as for dflash_verify_greedy)
+ *   target_positions   [n] int64      optimistic positions of the target rows
+ *   last_token_indices [B] int32      last target row of each request
+ *   num_draft          [B] int32      drafts verified this step per request
+ *                      (cur_num_draft of dflash_prepare_proposal_inputs)
+ *   prev_sampled       [B, prev_width] int32 and prev_num_draft [B] int32: the
+ *                      previous step's sampler output, both NULL on a first step
+ *   aux                [n, T*H] bf16  the target's tapped states of the rows
+ *   block_table        [B, max_pages_per_seq] int32
+ *   k_cache, v_cache   HOST arrays of n_layers device pointers (paged pools of
+ *                      num_pages pages, as for dflash_inject_context)
+ * Outputs:
+ *   out_tokens [B, K+1], num_accepted [B]     verification (the accepted
+ *                                             tokens of this step)
+ *   positions, slot_mapping [n] int64         corrected rows of the injection
+ *   seq_lens, bonus [B] int32                 the new block's start and first token
+ *   draft_tokens [B, K], block_tokens [B, bs] (nullable) the next proposal
+ *   device_error (device word)                input errors seen by the
+ *                                             preparation (DFLASH_DEVERR_INPUT);
+ *                                             NULL: the handle's error word
+ *                                             (dflash_check_device_errors) */
+typedef struct dflash_step_io {
+  int B;
+  int n;
+  const int32_t* prev_drafts;
+  const float* target_logits;
+  const int64_t* target_positions;
+  const int32_t* last_token_indices;
+  const int32_t* num_draft;
+  const int32_t* prev_sampled;
+  int prev_width;
+  const int32_t* prev_num_draft;
+  const void* aux;
+  const int32_t* block_table;
+  int max_pages_per_seq;
+  void* const* k_cache;
+  void* const* v_cache;
+  int num_pages;
+  int32_t* out_tokens;
+  int32_t* num_accepted;
+  int64_t* positions;
+  int64_t* slot_mapping;
+  int32_t* seq_lens;
+  int32_t* bonus;
+  int32_t* draft_tokens;
+  int32_t* block_tokens;
+  unsigned* device_error;
+} dflash_step_io;
+
+/* Workspace needed by dflash_spec_step (and dflash_step_graph_create) for B
+ * requests, n target rows and block tables max_pages_per_seq wide: the
+ * verification's, the injection's and the proposal's workspaces side by side
+ * (256-byte aligned pieces).  0 for invalid sizes. */
+size_t dflash_spec_step_workspace_bytes(const dflash_handle* h, int B, int n,
+                                        int max_pages_per_seq);
+
+/* One whole speculative step with no host round trip (§"Async Rejection and
+ * Position Correction": with the proposal inputs prepared on the device the
+ * step needs nothing from the host between its stages):
+ *   1. dflash_verify_greedy(prev_drafts, target_logits) -> out_tokens,
+ *      num_accepted (its bonus is written to `bonus`, then rewritten by 2.
+ *      with the same value: the last valid entry of out_tokens);
+ *   2. dflash_prepare_proposal_inputs(target_positions, last_token_indices,
+ *      cur_sampled = out_tokens (width K+1), num_draft, prev_sampled,
+ *      prev_num_draft) -> positions, slot_mapping, seq_lens, bonus;
+ *   3. dflash_inject_context over the n target rows (padding rows, slot -1,
+ *      are skipped);
+ *   4. dflash_propose(bonus, seq_lens) -> draft_tokens, block_tokens.
+ * Every argument is checked on the host before the first launch (the checks
+ * of the four calls, plus n >= B when B > 0); B == 0 is a no-op.  The calls
+ * only enqueue work on `stream`, so the step may be captured into a CUDA graph
+ * (dflash_step_graph_create does that). */
+dflash_status dflash_spec_step(dflash_handle* h, const dflash_step_io* io, void* workspace,
+                               size_t workspace_bytes, void* stream);
+
+/* A speculative step captured once into a CUDA graph owned by the library
+ * (every launch of dflash_spec_step with PDL edges kept), replayed by
+ * dflash_step_graph_launch on any stream of the handle's device.  The graph
+ * holds the pointers of `io` and `workspace` (and the handle's weights): the
+ * caller rewrites the inputs in place between launches and keeps every buffer
+ * alive until dflash_step_graph_destroy.  Feeding a step's drafts to the next
+ * step as prev_drafts means two graphs over two buffer sets, or a copy.
+ * create: the same host checks as dflash_spec_step (DFLASH_ERR_INVALID_ARG as
+ * well while launch profiling is enabled on the handle), captured on a stream
+ * of the handle's device; nothing runs until the first launch.  Errors:
+ * DFLASH_ERR_CUDA if capture or instantiation fails (e.g. a capture already
+ * open on the calling thread).  B == 0 gives a graph whose launches do
+ * nothing. */
+typedef struct dflash_step_graph dflash_step_graph;
+dflash_status dflash_step_graph_create(dflash_handle* h, const dflash_step_io* io,
+                                       void* workspace, size_t workspace_bytes,
+                                       dflash_step_graph** out);
+dflash_status dflash_step_graph_launch(dflash_step_graph* g, void* stream);
+/* NULL is a no-op; the caller makes sure no launch of the graph is pending. */
+void dflash_step_graph_destroy(dflash_step_graph* g);
+
 /* ---- component entry points (each runs one kernel family of the path) ---- */
 
 /* out[m, n] = sum_k A[m, k] * W[n, k] in fp32 — the tcgen05 GEMM that every

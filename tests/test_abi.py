@@ -89,6 +89,22 @@ def test_host_validation_without_gpu(L):
     assert call(B=2) == -1
 
 
+def test_spec_step_host_validation_without_gpu(L):
+    """The whole-step entry points reject a missing handle or buffers before
+    anything reaches the device, and the graph calls accept NULL as documented."""
+    io = D._StepIO()
+    io.B, io.n = 1, 16
+    assert L.dflash_spec_step(None, ctypes.byref(io), None, 0, None) == -1
+    assert L.dflash_spec_step(None, None, None, 0, None) == -1
+    out = ctypes.c_void_p(1)
+    assert L.dflash_step_graph_create(None, ctypes.byref(io), None, 0, ctypes.byref(out)) == -1
+    assert out.value is None                          # *out cleared on failure
+    assert L.dflash_step_graph_create(None, ctypes.byref(io), None, 0, None) == -1
+    assert L.dflash_step_graph_launch(None, None) == -1
+    L.dflash_step_graph_destroy(None)                 # no-op
+    assert L.dflash_spec_step_workspace_bytes(None, 1, 16, 8) == 0
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
 def test_create_without_device_fails_cleanly(L):
     from block_diffusion_speculative_propose_b200 import synth
