@@ -472,6 +472,36 @@ def extra_measurements(st, peaks) -> dict:
                       dev, reps=20)
     out["prepare_proposal_inputs"] = {"rows": int(tp.numel()), "us": t * 1e6}
     out["spec_step_graph"] = spec_step_graph(st)
+    out["vocab_parallel_propose"] = vocab_parallel_propose(st)
+    return out
+
+
+def vocab_parallel_propose(st, parts_list=(1, 2, 4, 8)) -> dict:
+    """One rank's share of a vocabulary-parallel proposal: the proposal with a
+    1/parts shard of the LM head (dflash_propose_keys on a shard handle), as
+    each rank of a parts-GPU group would run it before the all-reduce of its
+    8-byte keys per draft row.  The exchange itself is not timed (one GPU)."""
+    from block_diffusion_speculative_propose_b200 import DFlash
+    from block_diffusion_speculative_propose_b200.tensor_parallel import vocab_shards
+    c, dev, B, K = st.cfg, st.dev, st.B, st.K
+    keys = torch.empty(B, K, dtype=torch.int64, device=dev)
+    args = (st.inp["bonus"], st.inp["seq_lens"], st.inp["block_table"], st.kc, st.vc)
+    out = {}
+    for parts in parts_list:
+        start, count = vocab_shards(c["vocab"], parts)[0]
+        if parts == 1:
+            hs = st.h
+        else:
+            hs = DFlash(c, dict(st.W, lm_head=st.W["lm_head"][start:start + count]),
+                        device=dev.index, max_position=st.h.max_position,
+                        vocab_shard=(start, count))
+        try:
+            t = graph_seconds(lambda: hs.propose_keys(*args, draft_keys=keys,
+                                                      workspace=st.ws_prop), dev, reps=4)
+        finally:
+            if hs is not st.h:
+                hs.close()
+        out[str(parts)] = {"vocab_rows": count, "us": t * 1e6}
     return out
 
 

@@ -5,6 +5,6 @@ CUDA); ``dflash`` is its thin Python binding and ``synth`` the seeded
 synthetic-input generator used by the tests and the benchmark.
 """
 
-from .dflash import (DFlash, DFlashError, StepGraph, Workspace, lib,  # noqa: F401
-                     paged_slots, prepare_proposal_inputs, status_string, verify_greedy,
+from .dflash import (DFlash, DFlashError, StepGraph, Workspace, finalize_draft_keys,  # noqa: F401
+                     lib, paged_slots, prepare_proposal_inputs, status_string, verify_greedy,
                      verify_workspace_bytes, version)

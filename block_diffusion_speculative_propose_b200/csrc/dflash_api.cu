@@ -305,7 +305,10 @@ struct dflash_handle {
   std::vector<bf16*> wdown;         // W_down (bf16: multiplied against the bf16 MLP hidden)
   bf16* fcw = nullptr;              // fc (bf16: multiplied against the bf16 target states)
   f16* wkv = nullptr;               // all layers' [Wk; Wv], [L * 2 * Hkv * D, H]
-  f16* lm_head16 = nullptr;         // [V, H]
+  f16* lm_head16 = nullptr;         // [vocab_count, H]: rows [vocab_start, +vocab_count)
+  // vocabulary shard of the LM head (tensor-parallel proposal); the whole
+  // vocabulary unless created by dflash_create_vocab_shard
+  int vocab_start = 0, vocab_count = 0;
   bf16* knorm_all = nullptr;  // [L, D]
   float2* rope = nullptr;   // [max_position, D/2]
   unsigned* dev_err = nullptr;
@@ -997,10 +1000,19 @@ const char* dflash_version(void) { return "dflash-b200 0.1 (sm_100a)"; }
 
 dflash_status dflash_create(const dflash_config* cfg, const dflash_weights* w, int device,
                             dflash_handle** out) {
+  return dflash_create_vocab_shard(cfg, w, device, 0, cfg ? cfg->vocab : 0, out);
+}
+
+dflash_status dflash_create_vocab_shard(const dflash_config* cfg, const dflash_weights* w,
+                                        int device, int vocab_start, int vocab_count,
+                                        dflash_handle** out) {
   if (!out) return DFLASH_ERR_INVALID_ARG;
   *out = nullptr;
   if (!cfg || !w) return DFLASH_ERR_INVALID_ARG;
   const dflash_config& c = *cfg;
+  if (vocab_start < 0 || vocab_count <= 0 || vocab_count > c.vocab - vocab_start)
+    return DFLASH_ERR_INVALID_ARG;
+  if (vocab_start % 32 || vocab_count % 32) return DFLASH_ERR_UNSUPPORTED_SHAPE;
   if (c.hidden <= 0 || c.n_layers <= 0 || c.n_q_heads <= 0 || c.n_kv_heads <= 0 ||
       c.head_dim <= 0 || c.intermediate <= 0 || c.vocab <= 0 || c.n_target_layers <= 0 ||
       c.block_size <= 0 || c.page_size <= 0 || c.max_position <= 0 || !(c.rms_eps >= 0.f) ||
@@ -1041,6 +1053,8 @@ dflash_status dflash_create(const dflash_config* cfg, const dflash_weights* w, i
   dflash_handle* h = new (std::nothrow) dflash_handle();
   if (!h) return DFLASH_ERR_CUDA;
   h->cfg = c;
+  h->vocab_start = vocab_start;
+  h->vocab_count = vocab_count;
   if (c.target_layer_ids) h->target_layer_ids.assign(c.target_layer_ids, c.target_layer_ids + c.n_target_layers);
   h->cfg.target_layer_ids = h->target_layer_ids.empty() ? nullptr : h->target_layer_ids.data();
   h->device = device;
@@ -1131,8 +1145,8 @@ dflash_status dflash_create(const dflash_config* cfg, const dflash_weights* w, i
                         cudaMemcpyDeviceToDevice, st) != cudaSuccess)
       return fail_st(DFLASH_ERR_CUDA);
   }
-  if (cudaMalloc(&h->lm_head16, static_cast<size_t>(c.vocab) * rowb) != cudaSuccess ||
-      cudaMemcpyAsync(h->lm_head16, w->lm_head, static_cast<size_t>(c.vocab) * rowb,
+  if (cudaMalloc(&h->lm_head16, static_cast<size_t>(vocab_count) * rowb) != cudaSuccess ||
+      cudaMemcpyAsync(h->lm_head16, w->lm_head, static_cast<size_t>(vocab_count) * rowb,
                       cudaMemcpyDeviceToDevice, st) != cudaSuccess)
     return fail_st(DFLASH_ERR_CUDA);
   {
@@ -1147,7 +1161,7 @@ dflash_status dflash_create(const dflash_config* cfg, const dflash_weights* w, i
       ok = ok && to_f16(h->wo[l], static_cast<size_t>(H) * Hq * D);
     }
     ok = ok && to_f16(h->wkv, static_cast<size_t>(L) * 2 * kvrows * H);
-    ok = ok && to_f16(h->lm_head16, static_cast<size_t>(c.vocab) * H);
+    ok = ok && to_f16(h->lm_head16, static_cast<size_t>(vocab_count) * H);
     if (!ok) return fail_st(DFLASH_ERR_CUDA);
   }
   // every GEMM weight into the tile-contiguous layout
@@ -1181,7 +1195,7 @@ dflash_status dflash_create(const dflash_config* cfg, const dflash_weights* w, i
       ok = ok && repack(h->wo[l], H, Hq * D);
     }
     ok = ok && repack(h->wkv, L * 2 * Hkv * D, H);
-    ok = ok && repack(h->lm_head16, c.vocab, H);
+    ok = ok && repack(h->lm_head16, vocab_count, H);
     for (int l = 0; ok && l < L; ++l) {
       void* p = nullptr;
       ok = pack(w->w_down[l], H, I, &p);
@@ -1369,17 +1383,22 @@ dflash_status dflash_inject_context(dflash_handle* h, const void* aux, const int
 }
 
 
-dflash_status dflash_propose(dflash_handle* h, const int32_t* bonus_tokens,
-                             const int32_t* seq_lens, const int32_t* block_table, int B,
-                             int max_pages_per_seq, void* const* k_cache, void* const* v_cache,
-                             int num_pages, int32_t* draft_tokens, int32_t* block_tokens,
-                             float* logits_out, void* workspace, size_t workspace_bytes,
-                             void* stream) {
+}  // extern "C"
+
+namespace {
+// The proposal up to the LM head's greedy pick; then either the drafts
+// (draft_keys == nullptr) or this handle's vocabulary shard's ordered keys.
+dflash_status propose_impl(dflash_handle* h, const int32_t* bonus_tokens,
+                           const int32_t* seq_lens, const int32_t* block_table, int B,
+                           int max_pages_per_seq, void* const* k_cache, void* const* v_cache,
+                           int num_pages, int32_t* draft_tokens, int32_t* block_tokens,
+                           int64_t* draft_keys, float* logits_out, void* workspace,
+                           size_t workspace_bytes, void* stream) {
   if (!h || B < 0) return DFLASH_ERR_INVALID_ARG;
   if (B == 0) return DFLASH_OK;
   const dflash_config& c = h->cfg;
   if (!bonus_tokens || !seq_lens || !block_table || max_pages_per_seq <= 0 || !k_cache ||
-      !v_cache || num_pages <= 0 || !draft_tokens || !workspace)
+      !v_cache || num_pages <= 0 || !(draft_tokens || draft_keys) || !workspace)
     return DFLASH_ERR_INVALID_ARG;
   for (int l = 0; l < c.n_layers; ++l)
     if (!k_cache[l] || !v_cache[l]) return DFLASH_ERR_INVALID_ARG;
@@ -1409,16 +1428,65 @@ dflash_status dflash_propose(dflash_handle* h, const int32_t* bonus_tokens,
                         : propose_layers<64>(h, lw, workspace, seq_lens, block_table, B,
                                              max_pages_per_seq, k_cache, v_cache, num_pages, st);
   if (s != DFLASH_OK) return s;
-  // aliased target LM head with the greedy pick fused into its epilogue
-  EpiArgmax ea{keys, logits_out, c.vocab};
-  s = run_gemm(h, DFLASH_KERNEL_GEMM_LM_HEAD, true, true, frows, B * K, H, h->lm_head16, c.vocab, ea,
-               partial, lw.partial_cap, st);
+  // aliased target LM head (this handle's vocabulary rows) with the greedy
+  // pick fused into its epilogue
+  EpiArgmax ea{keys, logits_out, h->vocab_count, static_cast<uint32_t>(h->vocab_start)};
+  s = run_gemm(h, DFLASH_KERNEL_GEMM_LM_HEAD, true, true, frows, B * K, H, h->lm_head16,
+               h->vocab_count, ea, partial, lw.partial_cap, st);
   if (s != DFLASH_OK) return s;
   {
     LaunchScope scope(h, DFLASH_KERNEL_ARGMAX_FINALIZE, st);
-    launch_k(h->pdl, argmax_finalize_kernel, dim3(cdiv(M, 256)), dim3(256), 0, st, keys,
-             bonus_tokens, draft_tokens, block_tokens, B, bs);
+    if (draft_keys)
+      launch_k(h->pdl, keys_export_kernel, dim3(cdiv(B * K, 256)), dim3(256), 0, st, keys,
+               B * K, draft_keys);
+    else
+      launch_k(h->pdl, argmax_finalize_kernel, dim3(cdiv(M, 256)), dim3(256), 0, st, keys,
+               bonus_tokens, draft_tokens, block_tokens, B, bs);
   }
+  return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ERR_CUDA;
+}
+}  // namespace
+
+extern "C" {
+
+dflash_status dflash_propose(dflash_handle* h, const int32_t* bonus_tokens,
+                             const int32_t* seq_lens, const int32_t* block_table, int B,
+                             int max_pages_per_seq, void* const* k_cache, void* const* v_cache,
+                             int num_pages, int32_t* draft_tokens, int32_t* block_tokens,
+                             float* logits_out, void* workspace, size_t workspace_bytes,
+                             void* stream) {
+  // a vocabulary shard's own argmax is not a draft: dflash_propose_keys
+  if (h && h->vocab_count != h->cfg.vocab) return DFLASH_ERR_INVALID_ARG;
+  if (!draft_tokens && B > 0) return DFLASH_ERR_INVALID_ARG;
+  return propose_impl(h, bonus_tokens, seq_lens, block_table, B, max_pages_per_seq, k_cache,
+                      v_cache, num_pages, draft_tokens, block_tokens, nullptr, logits_out,
+                      workspace, workspace_bytes, stream);
+}
+
+dflash_status dflash_propose_keys(dflash_handle* h, const int32_t* bonus_tokens,
+                                  const int32_t* seq_lens, const int32_t* block_table, int B,
+                                  int max_pages_per_seq, void* const* k_cache,
+                                  void* const* v_cache, int num_pages, int64_t* draft_keys,
+                                  float* logits_out, void* workspace, size_t workspace_bytes,
+                                  void* stream) {
+  if (!draft_keys && B > 0) return DFLASH_ERR_INVALID_ARG;
+  return propose_impl(h, bonus_tokens, seq_lens, block_table, B, max_pages_per_seq, k_cache,
+                      v_cache, num_pages, nullptr, nullptr, draft_keys, logits_out, workspace,
+                      workspace_bytes, stream);
+}
+
+dflash_status dflash_finalize_draft_keys(const int64_t* draft_keys, const int32_t* bonus_tokens,
+                                         int B, int block_size, int vocab,
+                                         int32_t* draft_tokens, int32_t* block_tokens,
+                                         unsigned* device_error, void* stream) {
+  if (B < 0 || block_size < 2 || vocab < 1) return DFLASH_ERR_INVALID_ARG;
+  if (B == 0) return DFLASH_OK;
+  if (!draft_keys || !bonus_tokens || !draft_tokens) return DFLASH_ERR_INVALID_ARG;
+  dflash_status s = set_device_for(static_cast<cudaStream_t>(stream), draft_tokens);
+  if (s != DFLASH_OK) return s;
+  launch_k(pdl_default(), draft_keys_finalize_kernel, dim3(cdiv(B * block_size, 256)), dim3(256),
+           0, static_cast<cudaStream_t>(stream), draft_keys, bonus_tokens, B, block_size, vocab,
+           draft_tokens, block_tokens, device_error);
   return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ERR_CUDA;
 }
 
@@ -1473,6 +1541,7 @@ StepWs step_layout(const dflash_handle* h, int B, int n, int W) {
 dflash_status check_step(const dflash_handle* h, const dflash_step_io* io, const void* ws,
                          size_t bytes) {
   if (!h || !io || io->B < 0 || io->n < 0) return DFLASH_ERR_INVALID_ARG;
+  if (h->vocab_count != h->cfg.vocab) return DFLASH_ERR_INVALID_ARG;   // a vocabulary shard
   if (io->B == 0) return DFLASH_OK;
   const dflash_config& c = h->cfg;
   const int K = c.block_size - 1;

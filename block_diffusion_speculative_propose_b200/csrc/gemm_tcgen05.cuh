@@ -1072,12 +1072,14 @@ struct EpiArgmax {
   unsigned long long* keys;
   float* logits;
   int ldl;
+  uint32_t idx_base;   // vocabulary id of column 0 (a shard's first row)
   __device__ void begin(State& s) const { s.best = 0ull; }
   __device__ void apply(State& s, int m, int n0, int nv, const float* v) const {
 #pragma unroll
     for (int j = 0; j < kGroup; ++j) {
       if (j < nv) {
-        const unsigned long long k = argmax_key(v[j], static_cast<uint32_t>(n0 + j));
+        const unsigned long long k =
+            argmax_key(v[j], idx_base + static_cast<uint32_t>(n0 + j));
         s.best = k > s.best ? k : s.best;
       }
     }

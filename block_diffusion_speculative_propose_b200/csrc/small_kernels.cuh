@@ -143,6 +143,49 @@ __global__ void argmax_finalize_kernel(const unsigned long long* __restrict__ ke
   if (block) block[idx] = tok;
 }
 
+// A vocabulary shard's ordered argmax keys as signed 64-bit integers: each key
+// with its top bit flipped, so that the signed maximum over shards (an
+// all-reduce MAX over int64) is the unsigned maximum — the largest logit, and
+// among equal logits the lowest vocabulary id.
+__global__ void keys_export_kernel(const unsigned long long* __restrict__ keys, int n,
+                                   int64_t* __restrict__ out) {
+  pdl_trigger();
+  pdl_wait();
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) out[i] = static_cast<int64_t>(keys[i] ^ 0x8000000000000000ull);
+}
+
+// Drafts from exported keys (their maximum over the shards); block[b] =
+// [bonus_b, drafts[b]].  A key naming no vocabulary entry (no shard wrote the
+// row, or an id >= vocab) gives -1 and sets DFLASH_DEVERR_INPUT.
+__global__ void draft_keys_finalize_kernel(const int64_t* __restrict__ keys,
+                                           const int32_t* __restrict__ bonus, int B, int bs,
+                                           int vocab, int32_t* __restrict__ drafts,
+                                           int32_t* __restrict__ block, unsigned* err) {
+  pdl_trigger();
+  pdl_wait();
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= B * bs) return;
+  const int K = bs - 1;
+  const int b = idx / bs, i = idx - (idx / bs) * bs;
+  int32_t tok;
+  if (i == 0) {
+    tok = bonus[b];
+  } else {
+    const unsigned long long u =
+        static_cast<unsigned long long>(keys[b * K + i - 1]) ^ 0x8000000000000000ull;
+    const uint32_t id = argmax_key_index(u);
+    if (u == 0ull || id >= static_cast<uint32_t>(vocab)) {
+      raise_error(err, DFLASH_DEVERR_INPUT);
+      tok = -1;
+    } else {
+      tok = static_cast<int32_t>(id);
+    }
+    drafts[b * K + i - 1] = tok;
+  }
+  if (block) block[idx] = tok;
+}
+
 // Greedy verification, pass 1: per (row, chunk) ordered argmax key of the fp32
 // target logits.  Rows are [B * (K+1)], each V long.
 __global__ void __launch_bounds__(256) verify_partial_kernel(

@@ -90,6 +90,8 @@ def lib() -> ctypes.CDLL:
     sig = {
         "dflash_create": ([ctypes.POINTER(_Config), ctypes.POINTER(_Weights), i32,
                            ctypes.POINTER(vp)], i32),
+        "dflash_create_vocab_shard": ([ctypes.POINTER(_Config), ctypes.POINTER(_Weights), i32,
+                                       i32, i32, ctypes.POINTER(vp)], i32),
         "dflash_destroy": ([vp], None),
         "dflash_inject_workspace_bytes": ([vp, i32], sz),
         "dflash_propose_workspace_bytes": ([vp, i32, i32], sz),
@@ -102,6 +104,9 @@ def lib() -> ctypes.CDLL:
         "dflash_inject_context": ([vp, vp, vp, vp, i32, _PP, _PP, i32, vp, sz, vp], i32),
         "dflash_propose": ([vp, vp, vp, vp, i32, i32, _PP, _PP, i32, vp, vp, vp, vp, sz, vp],
                            i32),
+        "dflash_propose_keys": ([vp, vp, vp, vp, i32, i32, _PP, _PP, i32, vp, vp, vp, sz, vp],
+                                i32),
+        "dflash_finalize_draft_keys": ([vp, vp, i32, i32, i32, vp, vp, vp, vp], i32),
         "dflash_verify_greedy": ([vp, vp, i32, i32, i32, vp, vp, vp, vp, sz, vp], i32),
         "dflash_verify_greedy_noalloc": ([vp, vp, i32, i32, i32, vp, vp, vp, vp], i32),
         "dflash_spec_step_workspace_bytes": ([vp, i32, i32, i32], sz),
@@ -183,9 +188,13 @@ class DFlash:
 
     ``cfg`` uses the field names of ``dflash_config``; ``weights`` the names of
     ``dflash_weights`` (bf16 CUDA tensors; per-layer entries are lists).  The
-    handle keeps references to every tensor whose pointer the library keeps."""
+    handle keeps references to every tensor whose pointer the library keeps.
+    ``vocab_shard=(start, count)`` builds one rank's shard of the tensor-parallel
+    LM head (dflash_create_vocab_shard): ``weights["lm_head"]`` is then that
+    shard's [count, H] rows, and the handle proposes through propose_keys."""
 
-    def __init__(self, cfg: Dict, weights: Dict, device: int = 0, max_position: int = 0):
+    def __init__(self, cfg: Dict, weights: Dict, device: int = 0, max_position: int = 0,
+                 vocab_shard: Optional[Sequence[int]] = None):
         L = lib()
         self.cfg = dict(cfg)
         self.device = torch.device("cuda", device)
@@ -222,8 +231,15 @@ class DFlash:
             self._keep.append(arr)
             setattr(w, k, pp)
         h = ctypes.c_void_p()
-        _check(L.dflash_create(ctypes.byref(c), ctypes.byref(w), device, ctypes.byref(h)),
-               "dflash_create")
+        if vocab_shard is None:
+            self.vocab_shard = (0, cfg["vocab"])
+            _check(L.dflash_create(ctypes.byref(c), ctypes.byref(w), device, ctypes.byref(h)),
+                   "dflash_create")
+        else:
+            self.vocab_shard = (int(vocab_shard[0]), int(vocab_shard[1]))
+            _check(L.dflash_create_vocab_shard(ctypes.byref(c), ctypes.byref(w), device,
+                                               self.vocab_shard[0], self.vocab_shard[1],
+                                               ctypes.byref(h)), "dflash_create_vocab_shard")
         self.h = h
         self.ws = Workspace(self.device)
 
@@ -366,6 +382,31 @@ class DFlash:
                                               ctypes.byref(g)), "dflash_step_graph_create")
         return StepGraph(self, g, o, keep + [ws, io])
 
+    def propose_keys(self, bonus_tokens, seq_lens, block_table, k_cache, v_cache,
+                     draft_keys=None, logits_out=None, workspace: Optional[torch.Tensor] = None,
+                     stream=None):
+        """dflash_propose_keys: this handle's vocabulary shard's greedy-pick keys,
+        [B, K] int64, ready for an all-reduce MAX across the shards."""
+        B = int(bonus_tokens.shape[0])
+        bs = self.cfg["block_size"]
+        _want(bonus_tokens, torch.int32, "bonus_tokens")
+        _want(seq_lens, torch.int32, "seq_lens")
+        _want(block_table, torch.int32, "block_table")
+        W = int(block_table.shape[1])
+        if draft_keys is None:
+            draft_keys = torch.empty(B, bs - 1, dtype=torch.int64, device=self.device)
+        _want(draft_keys, torch.int64, "draft_keys")
+        need = self.propose_workspace_bytes(B, W) if B else 0
+        ws = workspace if workspace is not None else self.ws.get(need)
+        kp, ka = _ptr_array(k_cache)
+        vp, va = _ptr_array(v_cache)
+        _check(lib().dflash_propose_keys(self.h, _ptr(bonus_tokens), _ptr(seq_lens),
+                                         _ptr(block_table), B, W, kp, vp,
+                                         int(k_cache[0].shape[0]), _ptr(draft_keys),
+                                         _ptr(logits_out), _ptr(ws), ws.numel(),
+                                         _stream(stream)), "dflash_propose_keys")
+        return draft_keys
+
     def linear(self, A, W, out=None, block_n: int = 0, splits: int = 0, workspace=None,
                stream=None):
         M, K = A.shape
@@ -453,6 +494,25 @@ class StepGraph:
             self.close()
         except Exception:
             pass
+
+
+def finalize_draft_keys(draft_keys, bonus_tokens, block_size: int, vocab: int,
+                        draft_tokens=None, block_tokens=None, device_error=None, stream=None):
+    """dflash_finalize_draft_keys: drafts [B, K] (and block tokens [B, bs])
+    from the keys exchanged across vocabulary shards."""
+    B = int(bonus_tokens.shape[0])
+    _want(draft_keys, torch.int64, "draft_keys")
+    _want(bonus_tokens, torch.int32, "bonus_tokens")
+    dev = draft_keys.device
+    if draft_tokens is None:
+        draft_tokens = torch.empty(B, block_size - 1, dtype=torch.int32, device=dev)
+    if block_tokens is None:
+        block_tokens = torch.empty(B, block_size, dtype=torch.int32, device=dev)
+    _check(lib().dflash_finalize_draft_keys(_ptr(draft_keys), _ptr(bonus_tokens), B, block_size,
+                                            vocab, _ptr(draft_tokens), _ptr(block_tokens),
+                                            _ptr(device_error), _stream(stream)),
+           "dflash_finalize_draft_keys")
+    return draft_tokens, block_tokens
 
 
 def verify_workspace_bytes(B: int, K: int, V: int) -> int:

@@ -140,6 +140,21 @@ typedef struct dflash_handle dflash_handle;
 dflash_status dflash_create(const dflash_config* cfg, const dflash_weights* w,
                             int device, dflash_handle** out);
 
+/* A handle whose LM head holds only the vocabulary rows [vocab_start,
+ * vocab_start + vocab_count): one rank's shard of the tensor-parallel LM head
+ * (§"DFlashQwen3ForCausalLM": the aliased head is a column-parallel linear
+ * over the vocabulary; every rank runs the rest of the draft in full).
+ * w->lm_head points at that shard, [vocab_count, H] bf16; w->embed stays the
+ * whole [vocab, H] table; cfg->vocab is the whole vocabulary.  vocab_start and
+ * vocab_count must be multiples of 32 (DFLASH_ERR_UNSUPPORTED_SHAPE), with
+ * vocab_count >= 1 and vocab_start + vocab_count <= vocab (DFLASH_ERR_INVALID_ARG).
+ * A shard handle proposes through dflash_propose_keys (dflash_propose and
+ * dflash_spec_step reject it: a shard's own argmax is not a draft); the
+ * whole-vocabulary shard (0, vocab) is what dflash_create builds. */
+dflash_status dflash_create_vocab_shard(const dflash_config* cfg, const dflash_weights* w,
+                                        int device, int vocab_start, int vocab_count,
+                                        dflash_handle** out);
+
 /* Frees everything the handle owns.  The caller must make sure no work that
  * uses the handle is still pending.  NULL is a no-op. */
 void dflash_destroy(dflash_handle* h);
@@ -280,6 +295,37 @@ dflash_status dflash_propose(dflash_handle* h, const int32_t* bonus_tokens,
                              int32_t* draft_tokens, int32_t* block_tokens,
                              float* logits_out, void* workspace,
                              size_t workspace_bytes, void* stream);
+
+/* The proposal of dflash_propose up to the LM head's greedy pick, over this
+ * handle's vocabulary rows, exported for a cross-rank exchange instead of
+ * turned into drafts:
+ *   draft_keys [B, K] int64 out: for draft row (b, i) the key
+ *     ((ordered bits of the row's largest logit) << 32 | (2^32 - 1 - its
+ *     vocabulary id)) with bit 63 flipped, where the ordered bits of a float
+ *     sort like the float (-0 as +0, NaN as -inf).  The signed int64 maximum of
+ *     the keys of all shards (an all-reduce MAX, 8 bytes per row) is the key
+ *     of the whole vocabulary's greedy pick, ties -> lowest id.
+ *   logits_out [B*K, vocab_count] fp32 out (debug; this shard's columns);
+ *     may be NULL.
+ * Everything else (arguments, workspace, errors) as dflash_propose; a
+ * whole-vocabulary handle works too.  Then dflash_finalize_draft_keys. */
+dflash_status dflash_propose_keys(dflash_handle* h, const int32_t* bonus_tokens,
+                                  const int32_t* seq_lens, const int32_t* block_table, int B,
+                                  int max_pages_per_seq, void* const* k_cache,
+                                  void* const* v_cache, int num_pages, int64_t* draft_keys,
+                                  float* logits_out, void* workspace, size_t workspace_bytes,
+                                  void* stream);
+
+/* Drafts from the exchanged keys of dflash_propose_keys: draft_tokens [B, K]
+ * int32 = the vocabulary id in each key; block_tokens [B, block_size] int32
+ * (nullable) = cat(bonus_tokens[b], drafts[b]).  A key that names no id below
+ * `vocab` (no shard wrote the row) gives -1 and sets DFLASH_DEVERR_INPUT in
+ * *device_error (nullable).  Host errors: B < 0, block_size < 2, vocab < 1, a
+ * missing pointer.  One launch on the device of `stream`; B == 0 is a no-op. */
+dflash_status dflash_finalize_draft_keys(const int64_t* draft_keys, const int32_t* bonus_tokens,
+                                         int B, int block_size, int vocab,
+                                         int32_t* draft_tokens, int32_t* block_tokens,
+                                         unsigned* device_error, void* stream);
 
 /* Greedy verification.  target_logits row j (j = 0..K) of request b is the
  * target's prediction after block slot j (slot 0 = previous bonus token,
