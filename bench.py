@@ -45,10 +45,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # dram__bytes_write.sum) for the kernel family that dominates a workload,
 # keyed by the digest of the kernel sources it was measured on.
 TRAFFIC = {
-    # gate/up GEMM of the batch-1 Qwen3-8B-shaped step: 201.54 MB read + 3.99 MB written
+    # gate/up GEMM of the batch-1 Qwen3-8B-shaped step: 201.57 MB read + 3.55 MB written
     # (ncu --set full, profiles/gemm_gate_up_qwen3_b1_ctx2048.md)
-    ("qwen3_b1_ctx2048", "gemm_gate_up"): {"bytes_per_launch": 205528832,
-                                           "digest": "b870578c09aea03c"},
+    ("qwen3_b1_ctx2048", "gemm_gate_up"): {"bytes_per_launch": 205118208,
+                                           "digest": "59a7f03b8506a4c8"},
 }
 
 
