@@ -29,6 +29,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -552,8 +553,11 @@ def run_ours(a, rank, world, local):
         st.capture()
 
     # ---------------------------------------------------------- timed value loop
-    os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
-    sampler = ClockSampler(local, os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv"))
+    # the raw nvidia-smi samples go to BENCH_CLOCKS_DIR (default: the system
+    # temporary directory); their summary is in the JSON line
+    clocks_dir = os.environ.get("BENCH_CLOCKS_DIR") or tempfile.gettempdir()
+    os.makedirs(clocks_dir, exist_ok=True)
+    sampler = ClockSampler(local, os.path.join(clocks_dir, f"clocks_rank{rank}.csv"))
     for _ in range(a.warmup):
         st.step()
     torch.cuda.synchronize(dev)
