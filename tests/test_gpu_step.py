@@ -195,6 +195,34 @@ def test_qwen3_heads_spec_step():
         h.close()
 
 
+def test_spec_step_empty_batch_is_a_noop(tiny):
+    """B == 0: nothing runs, eager or as a graph (whose launches do nothing)."""
+    cfg, Wt, h = tiny
+    z32 = torch.zeros(0, dtype=torch.int32, device=DEV)
+    inp = dict(prev_drafts=torch.zeros(0, cfg["block_size"] - 1, dtype=torch.int32, device=DEV),
+               target_logits=torch.zeros(0, cfg["block_size"], cfg["vocab"], device=DEV),
+               target_positions=torch.zeros(0, dtype=torch.int64, device=DEV),
+               last_token_indices=z32, num_draft=z32,
+               aux=torch.zeros(0, cfg["n_target_layers"] * cfg["hidden"], dtype=torch.bfloat16,
+                               device=DEV),
+               block_table=torch.zeros(0, 4, dtype=torch.int32, device=DEV))
+    shape = (4, cfg["n_kv_heads"], cfg["page_size"], cfg["head_dim"])
+    kc = [torch.zeros(shape, dtype=torch.bfloat16, device=DEV) for _ in range(cfg["n_layers"])]
+    vc = [torch.zeros(shape, dtype=torch.bfloat16, device=DEV) for _ in range(cfg["n_layers"])]
+    before = h.launch_count()
+    out = h.spec_step(k_cache=kc, v_cache=vc, workspace=torch.empty(256, dtype=torch.uint8,
+                                                                     device=DEV), **inp)
+    g = h.step_graph(k_cache=kc, v_cache=vc, **inp)
+    try:
+        g.launch()
+        torch.cuda.synchronize()
+    finally:
+        g.close()
+    assert h.launch_count() == before
+    assert all(t.numel() == 0 for t in out.values())
+    assert h.check_device_errors() == 0
+
+
 def test_spec_step_host_errors(tiny):
     cfg, Wt, h = tiny
     case = StepCase(cfg, Wt, [20, 30], [1, 2], seed=3)
