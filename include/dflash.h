@@ -22,13 +22,21 @@
  *   dflash_prepare_proposal_inputs — §"Async Rejection and Position Correction"
  *                            (_correct_target_positions_for_async, _current_seq_lens),
  *                            §"Paged KV Integration", §"Draft Block Construction".
+ *   dflash_spec_step, dflash_step_graph_* — the four calls above as one step with
+ *                            nothing from the host between them, eager or as one
+ *                            CUDA graph owned by the library.
+ *   dflash_create_vocab_shard, dflash_propose_keys, dflash_finalize_draft_keys —
+ *                            §"DFlashQwen3ForCausalLM": the aliased LM head split over
+ *                            the vocabulary across tensor-parallel ranks, combined
+ *                            by one all-reduce MAX of 8 bytes per draft row.
  *
  * Conventions for every call
  *   - All tensor arguments are DEVICE pointers unless stated otherwise; bf16 means
  *     IEEE bfloat16 stored as uint16.  Row-major, densely packed.
  *   - `stream` is a cudaStream_t passed as void*.  Calls only enqueue work on it:
- *     no call synchronizes the stream, and no call other than dflash_create
- *     allocates memory.  Work may be captured into a CUDA graph.
+ *     no call synchronizes the stream, and no call other than dflash_create* and
+ *     dflash_step_graph_create (the graph and its capture stream) allocates
+ *     memory.  Work may be captured into a CUDA graph.
  *   - The caller owns every buffer it passes; the handle owns only the packed
  *     weight copies and small tables it builds in dflash_create.
  *   - Shape and argument errors are detected on the host before any launch and
