@@ -542,4 +542,449 @@ __global__ void __launch_bounds__(kTcThreads, TcAttnCfg<D, KT, ST>::kMinBlocks)
   }
 }
 
+
+// ---------------------------------------------------------------------------
+// Persistent variant of the 64-key, six-deep-ring kernel: gridDim.x CTAs (one
+// per SM) walk the (key split, kv head, request) items in the order of the
+// non-persistent grid (split fastest), CTA c taking items c, c + gridDim.x, ...
+// Every ring, S/P buffer and O barrier runs on a tile counter that continues
+// across items, so the producer streams the next item's K/V while the softmax
+// warps finish the previous item: the softmax warps load the next item's Q as
+// soon as the MMA warp has issued the current item's last S (q_empty), then
+// write the current item's output, then start the next item's tiles.  The
+// barrier / TMEM set-up is paid once per CTA instead of once per item.  No
+// cluster mode.  Same results as attn_block_tc_kernel<D, 64, ST> item by item.
+// ---------------------------------------------------------------------------
+template <int D, int ST>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    attn_block_tc_persistent_kernel(const __grid_constant__ CUtensorMap tmK,
+                                    const __grid_constant__ CUtensorMap tmV,
+                                    const AttnParams p) {
+  constexpr int KT = kTcKeysSmall;
+  using C = TcAttnCfg<D, KT, ST>;
+  static_assert(C::kPBufs == 1, "one P buffer");
+  pdl_trigger();
+  pdl_wait();
+  const int n_items = p.max_splits * p.Hkv * p.B;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // item -> (split, head, request, key range); false when it has no keys
+  auto item_at = [&](int it, int& split, int& h, int& b, int& k0, int& k1, int& n_tiles) {
+    split = it % p.max_splits;
+    const int r = it / p.max_splits;
+    h = r % p.Hkv;
+    b = r / p.Hkv;
+    const int n_keys = p.seq_lens[b] + p.bs;
+    k0 = split * p.chunk_keys;
+    k1 = min(n_keys, k0 + p.chunk_keys);
+    n_tiles = k0 < n_keys ? (k1 - k0 + KT - 1) / KT : 0;
+    return n_tiles > 0;
+  };
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sQ = smem + C::kOffQ;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint64_t* kv_full = bars;        // [ST] K/V ring (tile g -> stage g % ST)
+  uint64_t* kv_empty = bars + 8;   // [ST]
+  uint64_t* s_full = bars + 16;    // [2] S buffers (tile g -> g % 2)
+  uint64_t* s_empty = bars + 18;   // [2]
+  uint64_t* p_full = bars + 20;    // [2] (one P buffer: barrier g % 2 of it)
+  uint64_t* o_ready = bars + 24;   // one phase per tile: P V of that tile landed
+  uint64_t* q_full = bars + 25;    // one phase per item: its Q is in shared memory
+  uint64_t* o_final = bars + 26;   // one phase per item: its last P V landed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 27);
+  uint64_t* q_empty = bars + 28;   // one phase per item: its last S was issued and ran
+  auto sK = [&](int s) { return smem + s * C::kKVBytes; };
+  auto sV = [&](int s) { return smem + C::kOffV + s * C::kKVBytes; };
+  uint8_t* sPh = smem + C::kOffP;
+  uint8_t* sPl = smem + C::kOffP + C::kPBytes;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < ST; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_empty[i], 4);
+      mbar_init(&p_full[i], 4);
+    }
+    mbar_init(o_ready, 1);
+    mbar_init(q_full, 4);
+    mbar_init(o_final, 1);
+    mbar_init(q_empty, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  cta_sync();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      uint32_t g = 0;
+      bool ok = true;
+      for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
+        int split, h, b, k0, k1, n_tiles;
+        if (!item_at(it, split, h, b, k0, k1, n_tiles)) continue;
+        const int* bt = p.block_table + static_cast<size_t>(b) * p.W;
+        for (int t = 0; t < n_tiles; ++t, ++g) {
+          const int s = static_cast<int>(g % ST);
+          const uint32_t u = g / ST;
+          if (!mbar_wait(&kv_empty[s], (u & 1) ^ 1u, p.err)) {
+            ok = false;
+            break;
+          }
+          const int t0 = k0 + t * KT;
+          const int nvalid = min(KT, k1 - t0);
+          const int npages = (nvalid + 15) >> 4;
+          mbar_arrive_expect_tx(&kv_full[s],
+                                static_cast<uint32_t>((KT / 16) * C::kHalves * 2048 * 2));
+          for (int j = 0; j < KT / 16; ++j) {
+            int y = -16;  // pages past the range: fully out of bounds, TMA fills zeros
+            if (j < npages) {
+              const int pg = (t0 >> 4) + j;
+              if (pg >= p.W) {
+                raise_error(p.err, DFLASH_DEVERR_TABLE);
+              } else {
+                const int page = bt[pg];
+                if (page < 0 || page >= p.num_pages) raise_error(p.err, DFLASH_DEVERR_SLOT);
+                else y = (page * p.Hkv + h) * 16;
+              }
+            }
+#pragma unroll
+            for (int hf = 0; hf < C::kHalves; ++hf) {
+              const int off = hf * KT * 128 + j * 2048;
+              tma_load_2d(sK(s) + off, &tmK, &kv_full[s], hf * 64, y);
+              tma_load_2d(sV(s) + off, &tmV, &kv_full[s], hf * 64, y);
+            }
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_qk = umma_idesc_bf16(kTcM, KT, false);
+      const uint32_t idesc_pv = umma_idesc_bf16(kTcM, D, true);
+      uint32_t g = 0, q_phase = 0;
+      bool ok = true;
+      for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
+        int split, h, b, k0, k1, n_tiles;
+        if (!item_at(it, split, h, b, k0, k1, n_tiles)) continue;
+        if (!mbar_wait(q_full, q_phase & 1, p.err)) break;
+        ++q_phase;
+        tc_fence_after();
+        const uint32_t g0 = g;
+        // S of the item's tile t; the item's last S also releases its Q
+        auto issue_qk = [&](int t) -> bool {
+          const uint32_t gt = g0 + t;
+          const int kv = static_cast<int>(gt % ST);
+          const uint32_t kvu = gt / ST;
+          const int s = static_cast<int>(gt & 1);
+          const uint32_t u = gt >> 1;
+          if (!mbar_wait(&kv_full[kv], kvu & 1, p.err)) return false;
+          if (!mbar_wait(&s_empty[s], (u & 1) ^ 1u, p.err)) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const int half = kk >> 2, w = kk & 3;
+            const uint64_t ad = umma_desc_sw128(smem_u32(sQ + half * kTcM * 128 + w * 32));
+            const uint64_t bd = umma_desc_sw128(smem_u32(sK(kv) + half * KT * 128 + w * 32));
+            umma_f16kind(tmem_base + s * KT, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&s_full[s]);
+          if (t == n_tiles - 1) umma_commit(q_empty);
+          return true;
+        };
+        ok = issue_qk(0);
+        for (int t = 0; ok && t < n_tiles; ++t) {
+          const uint32_t gt = g0 + t, g1 = gt + 1;
+          const bool qk_first = t + 1 < n_tiles &&
+                                mbar_try_wait(&kv_full[g1 % ST], (g1 / ST) & 1) &&
+                                mbar_try_wait(&s_empty[g1 & 1], ((g1 >> 1) & 1) ^ 1u);
+          if (qk_first && !issue_qk(t + 1)) {
+            ok = false;
+            break;
+          }
+          const int s = static_cast<int>(gt & 1);
+          if (!mbar_wait(&p_full[s], (gt >> 1) & 1, p.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int kv = static_cast<int>(gt % ST);
+#pragma unroll
+          for (int lohi = 0; lohi < 2; ++lohi) {
+#pragma unroll
+            for (int kk = 0; kk < KT / 16; ++kk) {
+              const int kh = kk >> 2, w = kk & 3;
+              const uint64_t ad =
+                  umma_desc_sw128(smem_u32((lohi ? sPl : sPh) + kh * kTcM * 128 + w * 32));
+              const uint64_t bd = umma_desc_sw128_mn(smem_u32(sV(kv) + kk * 16 * 128),
+                                                     KT * 128, 1024);
+              umma_f16kind(tmem_base + C::kOCol, ad, bd, idesc_pv,
+                           (t > 0 || lohi > 0 || kk > 0) ? 1u : 0u);
+            }
+          }
+          umma_commit(&kv_empty[kv]);
+          umma_commit(o_ready);
+          if (t + 1 == n_tiles) umma_commit(o_final);
+          if (!qk_first && t + 1 < n_tiles && !issue_qk(t + 1)) {
+            ok = false;
+            break;
+          }
+        }
+        g += n_tiles;
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ softmax warps
+    const int sp = warp & 3;                    // TMEM sub-partition = 16-row group
+    const int tid = threadIdx.x - 64;           // 0..127
+    const uint32_t lane_base = static_cast<uint32_t>(32 * sp) << 16;
+    const int r0 = 16 * sp + (lane >> 2);       // this thread's rows r0 and r0 + 8
+    // Q rows r = i * G + g of item (h, b) -> K-major, 128B-swizzled operand
+    auto load_q = [&](int h, int b) {
+      constexpr int kQPer = kTcM * (D / 8) / 128;
+      uint4 qv[kQPer];
+#pragma unroll
+      for (int u = 0; u < kQPer; ++u) {
+        const int e = tid + u * 128;
+        const int r = e / (D / 8), c = e - r * (D / 8);
+        qv[u] = make_uint4(0, 0, 0, 0);
+        if (r < p.R) {
+          const int i = r / p.G, gq = r - (r / p.G) * p.G;
+          const bf16* src = p.q + (static_cast<size_t>(b * p.bs + i) * p.Hq + h * p.G + gq) * D;
+          qv[u] = *reinterpret_cast<const uint4*>(src + c * 8);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kQPer; ++u) {
+        const int e = tid + u * 128;
+        const int r = e / (D / 8), c = e - r * (D / 8);
+        *reinterpret_cast<uint4*>(sQ + (c >> 3) * kTcM * 128 + r * 128 +
+                                  (((c & 7) ^ (r & 7)) << 4)) = qv[u];
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(q_full);
+    };
+    // the next item with keys at or after `it` (n_items if none)
+    auto next_item = [&](int it) {
+      int split, h, b, k0, k1, n_tiles;
+      while (it < n_items && !item_at(it, split, h, b, k0, k1, n_tiles)) it += gridDim.x;
+      return it;
+    };
+
+    uint32_t g = 0, item_phase = 0;
+    bool ok = true;
+    int it = next_item(blockIdx.x);
+    if (it < n_items) {
+      int split, h, b, k0, k1, n_tiles;
+      item_at(it, split, h, b, k0, k1, n_tiles);
+      load_q(h, b);
+    }
+    while (ok && it < n_items) {
+      int split, h, b, k0, k1, n_tiles;
+      item_at(it, split, h, b, k0, k1, n_tiles);
+      const int n_keys = p.seq_lens[b] + p.bs;
+      const int n_splits_b = (n_keys + p.chunk_keys - 1) / p.chunk_keys;
+      float m_ref[2] = {-INFINITY, -INFINITY};
+      float l_run[2] = {0.f, 0.f};
+      for (int t = 0; t < n_tiles; ++t) {
+        const uint32_t gt = g + t;
+        const int s = static_cast<int>(gt & 1);
+        if (!mbar_wait(&s_full[s], (gt >> 1) & 1, p.err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        float sv[4 * (KT / 8)];
+        tmem_ld_16x256b_x8(tmem_base + lane_base + s * KT, sv);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_empty[s]);
+
+        const int t0 = k0 + t * KT;
+        const int nvalid = min(KT, k1 - t0);
+        float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+        for (int j = 0; j < KT / 8; ++j) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int kt = j * 8 + 2 * (lane & 3) + (e & 1);
+            const float v = sv[4 * j + e] * p.scale_log2;
+            sv[4 * j + e] = (kt < nvalid) ? v : -INFINITY;
+            mx[e >> 1] = fmaxf(mx[e >> 1], sv[4 * j + e]);
+          }
+        }
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          mx[hh] = fmaxf(mx[hh], __shfl_xor_sync(0xffffffffu, mx[hh], 1));
+          mx[hh] = fmaxf(mx[hh], __shfl_xor_sync(0xffffffffu, mx[hh], 2));
+        }
+        bool need[2];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh)
+          need[hh] = mx[hh] != -INFINITY &&
+                     (m_ref[hh] == -INFINITY || mx[hh] > m_ref[hh] + kTcLazyRescale);
+        if (__any_sync(0xffffffffu, need[0] || need[1])) {
+          float nref[2], alpha[2];
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            nref[hh] = need[hh] ? mx[hh] : m_ref[hh];
+            alpha[hh] = (m_ref[hh] == -INFINITY) ? 0.f : exp2f(m_ref[hh] - nref[hh]);
+          }
+          if (t > 0) {
+            // O holds this item's P V of tiles < t: rescale it once the
+            // previous tile's P V has landed (o_ready is at most one phase
+            // behind, so its parity names tile gt - 1)
+            if (!mbar_wait(o_ready, (gt - 1) & 1, p.err)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int c = 0; c < D / 64; ++c) {
+              float ov[32];
+              tmem_ld_16x256b_x8(tmem_base + lane_base + C::kOCol + c * 64, ov);
+              tmem_ld_wait();
+#pragma unroll
+              for (int q = 0; q < 32; ++q) ov[q] *= alpha[(q >> 1) & 1];
+              tmem_st_16x256b_x8(tmem_base + lane_base + C::kOCol + c * 64, ov);
+            }
+            tmem_st_wait();
+          }
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            l_run[hh] *= alpha[hh];
+            m_ref[hh] = nref[hh];
+          }
+        }
+        float ref[2];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) ref[hh] = (m_ref[hh] == -INFINITY) ? 0.f : m_ref[hh];
+#pragma unroll
+        for (int q = 0; q < 4 * (KT / 8); ++q) {
+          const float pv = exp2f(sv[q] - ref[(q >> 1) & 1]);
+          sv[q] = pv;
+          l_run[(q >> 1) & 1] += pv;
+        }
+        // the P buffer is free once P V of the previous tile (any item) landed
+        if (gt > 0 && !mbar_wait(o_ready, (gt - 1) & 1, p.err)) {
+          ok = false;
+          break;
+        }
+#pragma unroll
+        for (int j = 0; j < KT / 8; ++j) {
+          const int kh = j >> 3, ch = j & 7;
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const int r = r0 + 8 * hh;
+            uint32_t hi, lo;
+            split_bf16x2(sv[4 * j + 2 * hh], sv[4 * j + 2 * hh + 1], hi, lo);
+            const int off = kh * kTcM * 128 + r * 128 + ((ch ^ (r & 7)) << 4) + (lane & 3) * 4;
+            *reinterpret_cast<uint32_t*>(sPh + off) = hi;
+            *reinterpret_cast<uint32_t*>(sPl + off) = lo;
+          }
+        }
+        if (sp == 0 && (nvalid & 15)) {
+          // rows past the last key of a partly used page may hold anything
+          // (NaN patterns included): zero them so that P = 0 rows add 0
+          const int jp = nvalid >> 4, rr0 = nvalid & 15;
+          const int n16 = (16 - rr0) * C::kHalves * 8;
+          for (int e = lane; e < n16; e += 32) {
+            const int hf = e / ((16 - rr0) * 8);
+            const int rem = e - hf * (16 - rr0) * 8;
+            const int rr = rr0 + rem / 8, cc = rem & 7;
+            *reinterpret_cast<uint4*>(sV(static_cast<int>(gt % ST)) + hf * KT * 128 + jp * 2048 +
+                                      rr * 128 + cc * 16) = make_uint4(0, 0, 0, 0);
+          }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[s]);
+      }
+      if (!ok) break;
+      g += n_tiles;
+      // the next item's Q, as soon as this item's last S has run
+      const int nxt = next_item(it + gridDim.x);
+      if (nxt < n_items) {
+        if (!mbar_wait(q_empty, item_phase & 1, p.err)) break;
+        int s2, h2, b2, a0, a1, nt2;
+        item_at(nxt, s2, h2, b2, a0, a1, nt2);
+        load_q(h2, b2);
+      }
+      // this item's output
+      if (!mbar_wait(o_final, item_phase & 1, p.err)) break;
+      ++item_phase;
+      tc_fence_after();
+      float o[D / 8][4];
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) {
+        float ov[32];
+        tmem_ld_16x256b_x8(tmem_base + lane_base + C::kOCol + c * 64, ov);
+        tmem_ld_wait();
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) o[c * 8 + jj][e] = ov[4 * jj + e];
+      }
+      tc_fence_before();
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        l_run[hh] += __shfl_xor_sync(0xffffffffu, l_run[hh], 1);
+        l_run[hh] += __shfl_xor_sync(0xffffffffu, l_run[hh], 2);
+      }
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int r = r0 + hh * 8;
+        if (r >= p.R) continue;
+        if (n_splits_b == 1) {
+          const int i = r / p.G, gq = r - (r / p.G) * p.G;
+          f16* dst = p.o + (static_cast<size_t>(b * p.bs + i) * p.Hq + h * p.G + gq) * D;
+          const float inv = 1.f / l_run[hh];
+#pragma unroll
+          for (int db = 0; db < D / 8; ++db) {
+            const int d = db * 8 + 2 * (lane & 3);
+            *reinterpret_cast<uint32_t*>(dst + d) =
+                pack_f16x2(o[db][2 * hh] * inv, o[db][2 * hh + 1] * inv);
+          }
+        } else {
+          const size_t prow = (static_cast<size_t>(split) * p.B + b) * p.Hkv + h;
+          float* dst = p.part_o + (prow * p.R + r) * D;
+#pragma unroll
+          for (int db = 0; db < D / 8; ++db) {
+            const int d = db * 8 + 2 * (lane & 3);
+            *reinterpret_cast<float2*>(dst + d) = make_float2(o[db][2 * hh], o[db][2 * hh + 1]);
+          }
+          if ((lane & 3) == 0) {
+            *reinterpret_cast<float2*>(p.part_ml + (prow * p.R + r) * 2) =
+                make_float2(m_ref[hh], l_run[hh]);
+          }
+        }
+      }
+      it = nxt;
+    }
+  }
+
+  tc_fence_before();
+  cta_sync();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
 }  // namespace dflash

@@ -207,14 +207,15 @@ struct AttnPlan {
   bool tc = false;   // tcgen05 kernel (kv groups of up to 64 query rows)
   int kt = 128;      // tcgen05 kernel: keys per tile
   int st = 2;        // tcgen05 kernel: K/V ring depth (64-key tiles: 2 -> two CTAs per SM)
+  bool persist = false;  // six-deep ring: persistent CTAs (one per SM) walk the items
   bool cluster = false;  // tcgen05 kernel, splits of a (request, kv head) combined in a cluster
   size_t part_o_bytes = 0, part_ml_bytes = 0;
 };
 
 // forced_ring: K/V ring depth of the 64-key tcgen05 kernel (2 or 6), or 0 to
-// let the planner decide.
+// let the planner decide; persist: the six-deep ring as persistent CTAs.
 AttnPlan plan_attention(int B, int Hkv, int W, int P, int bs, int G, int D, int num_sms,
-                        bool allow_cluster, int forced_ring) {
+                        bool allow_cluster, int forced_ring, bool persist = false) {
   AttnPlan a;
   const int keys_max = W * P;
   const double est = static_cast<double>(B) * Hkv * keys_max;
@@ -235,6 +236,7 @@ AttnPlan plan_attention(int B, int Hkv, int W, int P, int bs, int G, int D, int 
   // 25-30%, so they keep the two-CTA ring.
   a.st = (chunk / kTcKeysSmall >= 2 * kTcDeepStages) ? kTcDeepStages : kTcStages;
   if (forced_ring == kTcStages || forced_ring == kTcDeepStages) a.st = forced_ring;
+  a.persist = persist && a.tc && a.st == kTcDeepStages;
   a.row_groups = cdiv(a.R, 16);
   a.key_parts = 1;
   while (a.key_parts < 4 && a.row_groups * a.key_parts * 2 <= kAttnMaxComputeWarps)
@@ -341,6 +343,12 @@ struct dflash_handle {
   int attn_ring = [] {
     const char* e = std::getenv("DFLASH_ATTN_STAGES");
     return e ? std::atoi(e) : 0;
+  }();
+  // six-deep-ring attention as persistent CTAs: opt-in (DFLASH_ATTN_PERSIST=1
+  // when the handle is created)
+  bool attn_persist = [] {
+    const char* e = std::getenv("DFLASH_ATTN_PERSIST");
+    return e && e[0] == '1';
   }();
   std::vector<cudaEvent_t> prof_events;
   size_t prof_next = 0;
@@ -693,6 +701,10 @@ cudaError_t set_attn_attrs() {
                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 TcAttnCfg<D, kTcKeysSmall, kTcDeepStages>::kSmem)) != cudaSuccess)
     return e;
+  if ((e = cudaFuncSetAttribute(attn_block_tc_persistent_kernel<D, kTcDeepStages>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                TcAttnCfg<D, kTcKeysSmall, kTcDeepStages>::kSmem)) != cudaSuccess)
+    return e;
   return cudaFuncSetAttribute(attn_block_tc_kernel<D, kTcKeys>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize,
                               TcAttnCfg<D, kTcKeys>::kSmem);
@@ -715,7 +727,12 @@ dflash_status run_attention(dflash_handle* h, const AttnPlan& ap, AttnParams prm
   prm.cluster = ap.cluster ? 1 : 0;
   if (ap.tc) {
     LaunchScope scope(h, DFLASH_KERNEL_ATTENTION, st);
-    if (ap.kt == kTcKeysSmall && ap.st == kTcDeepStages)
+    if (ap.kt == kTcKeysSmall && ap.persist) {
+      const int items = ap.max_splits * c.n_kv_heads * prm.B;
+      launch_k(h->pdl, attn_block_tc_persistent_kernel<D, kTcDeepStages>,
+               dim3(std::min(items, h->num_sms)), dim3(kTcThreads),
+               TcAttnCfg<D, kTcKeysSmall, kTcDeepStages>::kSmem, st, tk, tv, prm);
+    } else if (ap.kt == kTcKeysSmall && ap.st == kTcDeepStages)
       launch_kc(h->pdl, ap.cluster ? ap.max_splits : 1,
                 attn_block_tc_kernel<D, kTcKeysSmall, kTcDeepStages>, grid, dim3(kTcThreads),
                 TcAttnCfg<D, kTcKeysSmall, kTcDeepStages>::kSmem, st, tk, tv, prm);
@@ -793,7 +810,8 @@ ProposeWs propose_layout(const dflash_handle* h, int B, int W) {
   // the attention split plan is not monotonic in the batch: cover every size
   for (int bb = 1; bb <= B; ++bb) {
     const AttnPlan ap = plan_attention(bb, Hkv, W, c.page_size, bs, Hq / Hkv, D, h->num_sms,
-                                       h->attn_cluster, h->attn_ring);
+                                       h->attn_cluster, h->attn_ring,
+                                     h->attn_persist);
     po = std::max(po, ap.part_o_bytes);
     pm = std::max(pm, ap.part_ml_bytes);
   }
@@ -888,7 +906,8 @@ dflash_status propose_layers(dflash_handle* h, const ProposeWs& lw, void* ws,
   f16* frows = at<f16>(ws, lw.frows);
   float* partial = at<float>(ws, lw.partial);
   const AttnPlan ap = plan_attention(B, Hkv, W, c.page_size, bs, Hq / Hkv, D, h->num_sms,
-                                     h->attn_cluster, h->attn_ring);
+                                     h->attn_cluster, h->attn_ring,
+                                     h->attn_persist);
   if (ap.part_o_bytes > lw.part_o_cap || ap.part_ml_bytes > lw.part_ml_cap)
     return DFLASH_ERR_WORKSPACE;
   AttnParams prm;
@@ -1718,7 +1737,8 @@ size_t dflash_attention_workspace_bytes(const dflash_handle* h, int B, int max_p
   const dflash_config& c = h->cfg;
   const AttnPlan ap = plan_attention(B, c.n_kv_heads, max_pages_per_seq, c.page_size,
                                      c.block_size, c.n_q_heads / c.n_kv_heads, c.head_dim,
-                                     h->num_sms, h->attn_cluster, h->attn_ring);
+                                     h->num_sms, h->attn_cluster, h->attn_ring,
+                                     h->attn_persist);
   return align_up(ap.part_o_bytes) + align_up(ap.part_ml_bytes) + kAlign;
 }
 
@@ -1738,7 +1758,8 @@ dflash_status dflash_block_attention(dflash_handle* h, const void* q, const int3
   DF_CUDA(use_device(h->device));
   const AttnPlan ap = plan_attention(B, c.n_kv_heads, max_pages_per_seq, c.page_size,
                                      c.block_size, c.n_q_heads / c.n_kv_heads, c.head_dim,
-                                     h->num_sms, h->attn_cluster, h->attn_ring);
+                                     h->num_sms, h->attn_cluster, h->attn_ring,
+                                     h->attn_persist);
   AttnParams prm;
   prm.q = static_cast<const bf16*>(q);
   prm.o = static_cast<f16*>(o);

@@ -237,6 +237,45 @@ def test_block_attention_ring_depth(monkeypatch, ring, model, seq_lens):
         h.close()
 
 
+@pytest.mark.parametrize("model,seq_lens", [
+    ("tiny", [0, 1, 15, 16, 17, 63, 64, 65, 200]),
+    ("qwen3_8b", [0, 7, 100, 1000, 5000]),
+    ("qwen3_8b", [3000] * 40 + [0, 64, 17]),
+    ("llama31_8b", [3, 333, 4097]),
+])
+def test_block_attention_persistent(monkeypatch, model, seq_lens):
+    """The persistent six-deep-ring kernel (CTAs walking the (split, head,
+    request) items, counters carried across items) gives the same bits as the
+    one-item-per-CTA six-deep-ring kernel, and the oracle's values."""
+    cfg = synth.model_config(model)
+    small = dict(cfg, intermediate=256, vocab=1024, n_layers=1, mask_token_id=1023,
+                 n_target_layers=1)
+    W = weights_to(synth.make_weights(small, seed=1), DEV)
+    q, kc, vc, table, ref = _attention_case(cfg, seq_lens, seed=len(seq_lens) + 5)
+    args = (q.to(DEV), torch.tensor(seq_lens, dtype=torch.int32, device=DEV),
+            torch.tensor(table, device=DEV), kc.to(DEV), vc.to(DEV))
+    outs = []
+    for persist in ("0", "1"):
+        monkeypatch.setenv("DFLASH_ATTN_STAGES", "6")
+        monkeypatch.setenv("DFLASH_ATTN_PERSIST", persist)
+        h = DFlash(small, W, max_position=8192)
+        try:
+            h.profile_enable(16)
+            outs.append(h.block_attention(*args))
+            torch.cuda.synchronize()
+            assert h.profile_read()["attention"][0] == 1
+            h.profile_disable()
+            assert h.check_device_errors() == 0
+        finally:
+            h.close()
+    assert torch.equal(outs[0], outs[1])
+    got = to_np(outs[1]).astype(np.float64).reshape(ref.shape)
+    errs = [rel_l2(got[b * cfg["block_size"]:(b + 1) * cfg["block_size"]],
+                   ref[b * cfg["block_size"]:(b + 1) * cfg["block_size"]])
+            for b in range(len(seq_lens))]
+    assert max(errs) < 1e-3, errs
+
+
 # ----------------------------------------------------------------------------
 # verify / paged slots
 # ----------------------------------------------------------------------------
