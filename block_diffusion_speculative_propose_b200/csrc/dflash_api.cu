@@ -221,7 +221,7 @@ AttnPlan plan_attention(int B, int Hkv, int W, int P, int bs, int G, int D, int 
   const double est = static_cast<double>(B) * Hkv * keys_max;
   a.R = bs * G;
   a.tc = a.R <= kTcM;
-  a.kt = kTcKeysSmall;   // many requests: 64-key tiles, two CTAs per SM
+  a.kt = kTcKeysSmall;   // 64-key tiles (the ring depth is chosen below)
   const int tile = a.tc ? a.kt : kAttnTileKeys;
   int chunk = static_cast<int>(std::ceil(est / (4.0 * num_sms)));
   chunk = (chunk + tile - 1) / tile * tile;
