@@ -116,3 +116,61 @@ def test_composes_with_greedy_verification():
     got = O.prepare_proposal_inputs(pos, last, ver.out_tokens, np.full(B, K), table, 16, V)
     np.testing.assert_array_equal(got.seq_lens, starts + ver.num_accepted + 1)
     np.testing.assert_array_equal(got.bonus, ver.bonus)
+
+
+def test_injecting_rejected_rows_changes_no_proposal():
+    """The whole step injects all K+1 verified rows of a request, the rejected
+    ones included; they sit at positions >= the post-verify length, which the
+    next block covers, so the proposal equals the one made after injecting
+    the accepted rows only (the plain reading: n + 1 rows at [seq_len,
+    seq_len + n + 1))."""
+    from block_diffusion_speculative_propose_b200 import synth
+    cfg = synth.model_config("tiny")
+    oc = O.OracleConfig.from_mapping(cfg)
+    W = {k: ([x.float().numpy() for x in v] if isinstance(v, list) else v.float().numpy())
+         for k, v in synth.make_weights(cfg, seed=4).items()}
+    rng = np.random.default_rng(8)
+    K, bs, P, V = cfg["block_size"] - 1, cfg["block_size"], cfg["page_size"], cfg["vocab"]
+    ctx = [21, 50, 3]
+    B = len(ctx)
+    need = [-(-(c + 2 * bs + 1) // P) for c in ctx]
+    table = np.zeros((B, max(need)), dtype=np.int64)
+    perm = rng.permutation(sum(need))
+    cur = 0
+    for b, n in enumerate(need):
+        table[b, :n] = perm[cur:cur + n]
+        cur += n
+    pre_pos = np.concatenate([np.arange(c) for c in ctx]).astype(np.int64)
+    pre_req = np.concatenate([np.full(c, b) for b, c in enumerate(ctx)]).astype(np.int64)
+    pre_aux = rng.standard_normal((len(pre_pos), cfg["n_target_layers"] * cfg["hidden"]))
+    drafts = rng.integers(0, V, size=(B, K))
+    logits = rng.standard_normal((B, K + 1, V)).astype(np.float32)
+    accept = [0, 2, K]
+    for b in range(B):
+        for j in range(K):
+            if j < accept[b]:
+                logits[b, j, drafts[b, j]] = logits[b, j].max() + 1
+            else:
+                logits[b, j, drafts[b, j]] = logits[b, j].min() - 1
+    ver = O.verify_greedy(drafts, logits)
+    aux = rng.standard_normal((B * (K + 1), cfg["n_target_layers"] * cfg["hidden"]))
+    tpos = np.concatenate([c + np.arange(K + 1) for c in ctx]).astype(np.int64)
+    last = (np.arange(1, B + 1) * (K + 1) - 1)
+    nd = np.full(B, K)
+    pi = O.prepare_proposal_inputs(tpos, last, ver.out_tokens, nd, table, P, V)
+
+    def proposal(rows):
+        kc, vc = O.empty_caches(oc, sum(need))
+        O.inject_context(oc, W, pre_aux, pre_pos, O.paged_slots(pre_pos, pre_req, table, P),
+                         kc, vc, "exact")
+        O.inject_context(oc, W, aux[rows], pi.positions[rows], pi.slot_mapping[rows], kc, vc,
+                         "exact")
+        return O.propose(oc, W, pi.bonus, pi.seq_lens, table, kc, vc, "exact")
+
+    every = proposal(np.arange(B * (K + 1)))
+    kept = np.concatenate([b * (K + 1) + np.arange(int(ver.num_accepted[b]) + 1)
+                           for b in range(B)])
+    accepted_only = proposal(kept)
+    np.testing.assert_array_equal(pi.seq_lens, np.asarray(ctx) + ver.num_accepted + 1)
+    np.testing.assert_array_equal(every.draft_tokens, accepted_only.draft_tokens)
+    np.testing.assert_array_equal(every.logits, accepted_only.logits)
