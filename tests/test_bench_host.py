@@ -61,3 +61,39 @@ def test_reference_arm_prints_one_json_line():
     assert d["impl"] == "reference" and d["value"] > 0 and d["unit"] == "blocks/s"
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["steps"] == 2 and d["warmup"] == 3
+
+
+def test_reference_arm_bounds_its_run(monkeypatch, capsys):
+    """With many timed steps, the reference arm runs only as many whole oracle
+    steps as fit its wall-clock bound, spread over the K steps, and says so."""
+    sys.path.insert(0, ROOT)
+    import time
+    import types
+
+    import bench
+
+    class FakeOracle:
+        calls = 0
+
+        def __init__(self, wl_name, seed):
+            self.n, self.B, self.cfg = 1, 1, {"block_size": 4}
+
+        def step(self):
+            FakeOracle.calls += 1
+            time.sleep(0.02)
+
+    monkeypatch.setattr(bench, "OracleStep", FakeOracle)
+    monkeypatch.setattr(bench, "REF_BUDGET_S", 0.1)
+    a = types.SimpleNamespace(workload="tiny_b1_ctx64", seed=1, steps=200, warmup=3)
+    bench.run_reference(a, 0, 1)
+    d = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    timed = d["oracle_steps_timed"]
+    assert 1 <= timed <= 6 and FakeOracle.calls == timed + 1     # + the calibration step
+    assert d["steps"] == 200 and d["value"] > 0
+    assert f"{timed} whole oracle step" in d["cpu_baseline"]["sample"]
+    # few steps: all of them run
+    FakeOracle.calls = 0
+    a.steps = 2
+    bench.run_reference(a, 0, 1)
+    d = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert d["oracle_steps_timed"] == 2 and FakeOracle.calls == 3
