@@ -1691,6 +1691,28 @@ void dflash_step_graph_destroy(dflash_step_graph* g) {
   delete g;
 }
 
+dflash_status dflash_plan_attention_info(int B, int n_kv_heads, int max_pages_per_seq,
+                                         int page_size, int block_size, int q_per_kv,
+                                         int head_dim, int num_sms, int forced_ring, int flags,
+                                         dflash_attention_plan* out) {
+  if (!out || B <= 0 || n_kv_heads <= 0 || max_pages_per_seq <= 0 || page_size <= 0 ||
+      block_size <= 0 || q_per_kv <= 0 || head_dim <= 0 || num_sms <= 0)
+    return DFLASH_ERR_INVALID_ARG;
+  const AttnPlan ap = plan_attention(B, n_kv_heads, max_pages_per_seq, page_size, block_size,
+                                     q_per_kv, head_dim, num_sms, (flags & 1) != 0, forced_ring,
+                                     (flags & 2) != 0);
+  out->tcgen05 = ap.tc ? 1 : 0;
+  out->keys_per_tile = ap.tc ? ap.kt : kAttnTileKeys;
+  out->ring_depth = ap.tc ? (ap.kt == kTcKeysSmall ? ap.st : kTcStages) : 0;
+  out->ctas_per_sm =
+      ap.tc && ap.kt == kTcKeysSmall && ap.st == kTcStages && !ap.cluster ? 2 : 1;
+  out->chunk_keys = ap.chunk_keys;
+  out->max_splits = ap.max_splits;
+  out->cluster = ap.cluster ? 1 : 0;
+  out->persistent = ap.persist && !ap.cluster && ap.kt == kTcKeysSmall ? 1 : 0;
+  return DFLASH_OK;
+}
+
 size_t dflash_linear_workspace_bytes(const dflash_handle* h, int M, int N, int K) {
   if (!h || M <= 0 || N <= 0 || K <= 0) return 0;
   return align_up(std::max<size_t>(plan_gemm(M, N, K, 32, h->num_sms).partial_bytes, kAlign));

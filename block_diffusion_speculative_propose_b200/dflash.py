@@ -74,6 +74,12 @@ class _StepIO(ctypes.Structure):
                 ("block_tokens", ctypes.c_void_p), ("device_error", ctypes.c_void_p)]
 
 
+class _AttnPlan(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in ("tcgen05", "keys_per_tile", "ring_depth",
+                                            "ctas_per_sm", "chunk_keys", "max_splits",
+                                            "cluster", "persistent")]
+
+
 _lib = None
 
 
@@ -119,6 +125,7 @@ def lib() -> ctypes.CDLL:
         "dflash_linear_ex": ([vp, vp, vp, i32, i32, i32, vp, i32, i32, vp, sz, vp], i32),
         "dflash_block_attention": ([vp, vp, vp, vp, i32, i32, vp, vp, i32, vp, vp, sz, vp],
                                    i32),
+        "dflash_plan_attention_info": ([i32] * 10 + [ctypes.POINTER(_AttnPlan)], i32),
         "dflash_check_device_errors": ([vp, ctypes.POINTER(ctypes.c_uint)], i32),
         "dflash_launch_count": ([vp], ctypes.c_ulonglong),
         "dflash_kernel_name": ([i32], ctypes.c_char_p),
@@ -513,6 +520,21 @@ def finalize_draft_keys(draft_keys, bonus_tokens, block_size: int, vocab: int,
                                             _ptr(device_error), _stream(stream)),
            "dflash_finalize_draft_keys")
     return draft_tokens, block_tokens
+
+
+def attention_plan(B: int, n_kv_heads: int, max_pages_per_seq: int, block_size: int,
+                   q_per_kv: int, head_dim: int = 128, page_size: int = 16, num_sms: int = 148,
+                   forced_ring: int = 0, cluster: bool = False,
+                   persistent: bool = False) -> Dict[str, int]:
+    """dflash_plan_attention_info: the attention launch plan for this geometry
+    (host only)."""
+    out = _AttnPlan()
+    flags = (1 if cluster else 0) | (2 if persistent else 0)
+    _check(lib().dflash_plan_attention_info(B, n_kv_heads, max_pages_per_seq, page_size,
+                                            block_size, q_per_kv, head_dim, num_sms,
+                                            forced_ring, flags, ctypes.byref(out)),
+           "dflash_plan_attention_info")
+    return {n: getattr(out, n) for n, _ in _AttnPlan._fields_}
 
 
 def verify_workspace_bytes(B: int, K: int, V: int) -> int:

@@ -488,6 +488,28 @@ dflash_status dflash_block_attention(dflash_handle* h, const void* q, const int3
                                      void* o, void* workspace, size_t workspace_bytes,
                                      void* stream);
 
+/* The attention launch plan that a proposal with this geometry uses
+ * (diagnostics; host only, no device needed): kv groups of bs * G query rows
+ * (G = query heads per kv head), block tables of W pages of P keys, on
+ * `num_sms` SMs.  forced_ring: 0 (the planner's choice), 2 or 6 as
+ * DFLASH_ATTN_STAGES forces it; flags: bit 0 the opt-in cluster combine,
+ * bit 1 the opt-in persistent kernel.  Written to *out; DFLASH_ERR_INVALID_ARG
+ * for a non-positive size or a NULL out. */
+typedef struct dflash_attention_plan {
+  int tcgen05;        /* 1: the tcgen05 kernel (bs * G <= 64), 0: the mma.sync kernel */
+  int keys_per_tile;  /* tcgen05 kernel: 64 or 128 */
+  int ring_depth;     /* tcgen05 kernel: K/V tiles in flight per CTA (2 or 6) */
+  int ctas_per_sm;    /* tcgen05 kernel: 2 for the two-deep 64-key ring, else 1 */
+  int chunk_keys;     /* keys per split */
+  int max_splits;     /* splits of the longest request */
+  int cluster;        /* splits combined inside a thread-block cluster */
+  int persistent;     /* persistent CTAs walking the items */
+} dflash_attention_plan;
+dflash_status dflash_plan_attention_info(int B, int n_kv_heads, int max_pages_per_seq,
+                                         int page_size, int block_size, int q_per_kv,
+                                         int head_dim, int num_sms, int forced_ring, int flags,
+                                         dflash_attention_plan* out);
+
 /* ---- launch accounting and per-launch timing (diagnostics) ---- */
 
 /* Kernel families launched by the calls above (ids for dflash_profile_read). */
