@@ -5,5 +5,5 @@ and the CPU-baseline leg of ``bench.py``; never by the library package.
 """
 from .dflash_oracle import *  # noqa: F401,F403
 from .dflash_oracle import (OracleConfig, Proposal, ProposalInputs, QueryBlock,  # noqa: F401
-                            Verification,
+                            TPSlices, Verification,
                             STORAGE_POINTS, FP16_WEIGHTS)

@@ -612,3 +612,134 @@ def top2_gap_f32(logits: np.ndarray) -> np.ndarray:
     f = np.asarray(logits).astype(np.float32).astype(np.float64)
     part = np.partition(f, -2, axis=-1)
     return part[..., -1] - part[..., -2]
+
+
+# ----------------------------------------------------------------------------
+# tensor parallelism across ranks (the next step of the path; exact mode only)
+#
+# [NEURON] "Context KV Injection": each rank projects and stores "this rank's
+# KV heads only"; [NEURON] "DFlashQwen3ForCausalLM": the aliased LM head is a
+# column-parallel linear over the vocabulary.  Reading of what the pages leave
+# open (the usual column-/row-parallel split of a decoder layer): rank r of S
+# holds the contiguous kv heads [r Hkv/S, (r+1) Hkv/S) with their query heads
+# (each kv head keeps its own query group) and the MLP features
+# [r I/S, (r+1) I/S); the O and down projections are row-parallel, so each
+# rank forms a partial sum of the layer's output and the partials are added
+# across ranks (an all-reduce) before the residual add.  Every norm, the
+# embedding, fc + hidden_norm and the residual stream are replicated.
+# ----------------------------------------------------------------------------
+@dataclass
+class TPSlices:
+    q_heads: slice      # query heads of this rank
+    kv_heads: slice     # kv heads of this rank
+    features: slice     # MLP features of this rank
+
+
+def tp_slices(cfg: OracleConfig, rank: int, size: int) -> TPSlices:
+    """Rank `rank` of `size`: its kv heads, their query heads, its MLP
+    features (contiguous blocks); `size` must divide n_kv_heads and intermediate."""
+    Hq, Hkv, I = cfg.n_q_heads, cfg.n_kv_heads, cfg.intermediate
+    if size < 1 or Hkv % size or I % size or not 0 <= rank < size:
+        raise ValueError(f"cannot split {Hkv} kv heads / {I} features over {size} ranks")
+    hk, hq, fi = Hkv // size, Hq // size, I // size
+    return TPSlices(slice(rank * hq, (rank + 1) * hq), slice(rank * hk, (rank + 1) * hk),
+                    slice(rank * fi, (rank + 1) * fi))
+
+
+def _rows(w: np.ndarray, heads: slice, d: int) -> np.ndarray:
+    """The output rows of a [heads * d, in] projection that belong to `heads`."""
+    return np.asarray(w)[heads.start * d:heads.stop * d]
+
+
+def empty_caches_tp(cfg: OracleConfig, num_pages: int, size: int):
+    """Per rank, per layer zeroed K and V pools of the rank's kv heads,
+    [num_pages, Hkv / size, page, d]."""
+    shape = (num_pages, cfg.n_kv_heads // size, cfg.page_size, cfg.head_dim)
+    return ([[np.zeros(shape) for _ in range(cfg.n_layers)] for _ in range(size)],
+            [[np.zeros(shape) for _ in range(cfg.n_layers)] for _ in range(size)])
+
+
+def inject_context_tp(cfg: OracleConfig, W: Mapping, aux, positions, slot_mapping,
+                      k_caches, v_caches, size: int) -> None:
+    """inject_context with each rank projecting and storing its kv heads only
+    ([NEURON] "Context KV Injection"); k_caches[r][l] is rank r's layer-l pool."""
+    aux = np.asarray(aux, dtype=np.float64)
+    if aux.shape[0] == 0:
+        return
+    d = cfg.head_dim
+    ctx = context_fusion(cfg, W, aux, "exact")             # replicated on every rank
+    for r in range(size):
+        sl = tp_slices(cfg, r, size)
+        for l in range(cfg.n_layers):
+            k = linear(ctx, _rows(W["wk"][l], sl.kv_heads, d)).reshape(ctx.shape[0], -1, d)
+            v = linear(ctx, _rows(W["wv"][l], sl.kv_heads, d)).reshape(ctx.shape[0], -1, d)
+            k = apply_rope(rms_norm(k, W["k_norm_w"][l], cfg.rms_eps), positions,
+                           cfg.rope_theta)
+            write_slots(k_caches[r][l], slot_mapping, k, cfg.page_size)
+            write_slots(v_caches[r][l], slot_mapping, v, cfg.page_size)
+
+
+def draft_layer_tp(cfg: OracleConfig, W: Mapping, l: int, x: np.ndarray, qb: QueryBlock,
+                   block_table, seq_lens, k_caches, v_caches, size: int) -> np.ndarray:
+    """draft_layer split over `size` ranks: each rank's heads attend over its
+    own cache shard, its O and down projections give partial sums, and the
+    partials are added across ranks (in rank order) before each residual add."""
+    eps, d, M = cfg.rms_eps, cfg.head_dim, x.shape[0]
+    n = rms_norm(x, W["in_norm_w"][l], eps)
+    attn_parts = []
+    for r in range(size):
+        sl = tp_slices(cfg, r, size)
+        hq, hk = sl.q_heads.stop - sl.q_heads.start, sl.kv_heads.stop - sl.kv_heads.start
+        q = linear(n, _rows(W["wq"][l], sl.q_heads, d)).reshape(M, hq, d)
+        k = linear(n, _rows(W["wk"][l], sl.kv_heads, d)).reshape(M, hk, d)
+        v = linear(n, _rows(W["wv"][l], sl.kv_heads, d)).reshape(M, hk, d)
+        q = apply_rope(rms_norm(q, W["q_norm_w"][l], eps), qb.positions, cfg.rope_theta)
+        k = apply_rope(rms_norm(k, W["k_norm_w"][l], eps), qb.positions, cfg.rope_theta)
+        slots = paged_slots(qb.positions, qb.req_ids, block_table, cfg.page_size)
+        write_slots(k_caches[r][l], slots, k, cfg.page_size)
+        write_slots(v_caches[r][l], slots, v, cfg.page_size)
+        rank_cfg = OracleConfig(**{**cfg.__dict__, "n_q_heads": hq, "n_kv_heads": hk})
+        o = block_attention(rank_cfg, q, k_caches[r][l], v_caches[r][l], block_table, seq_lens)
+        wo_cols = np.asarray(W["wo"][l])[:, sl.q_heads.start * d:sl.q_heads.stop * d]
+        attn_parts.append(linear(o.reshape(M, hq * d), wo_cols))
+    x = x + sum(attn_parts)                                  # all-reduce of the O partials
+    n2 = rms_norm(x, W["post_norm_w"][l], eps)
+    mlp_parts = []
+    for r in range(size):
+        f = tp_slices(cfg, r, size).features
+        h = silu(linear(n2, np.asarray(W["w_gate"][l])[f])) * linear(n2, np.asarray(W["w_up"][l])[f])
+        mlp_parts.append(linear(h, np.asarray(W["w_down"][l])[:, f]))
+    return x + sum(mlp_parts)                                # all-reduce of the down partials
+
+
+def propose_tp(cfg: OracleConfig, W: Mapping, bonus_tokens, seq_lens, block_table,
+               k_caches, v_caches, size: int, vocab_shards) -> Proposal:
+    """propose over `size` ranks: draft_layer_tp for the stack, then the LM
+    head over the vocabulary shards [(start, count), ...] (a column-parallel
+    linear, [NEURON] "DFlashQwen3ForCausalLM"): each shard's greedy pick (its
+    largest float32 logit, lowest id on ties) and the best of those across
+    shards (largest value, lowest id on ties)."""
+    bonus = np.asarray(bonus_tokens, dtype=np.int64)
+    B, bs, K = bonus.shape[0], cfg.block_size, cfg.num_drafts
+    qb = build_query_block(bonus, seq_lens, bs, cfg.mask_token_id)
+    x = np.asarray(W["embed"])[qb.input_ids].astype(np.float64)
+    for l in range(cfg.n_layers):
+        x = draft_layer_tp(cfg, W, l, x, qb, block_table, seq_lens, k_caches, v_caches, size)
+    f = rms_norm(x[qb.keep_idx], W["final_norm_w"], cfg.rms_eps)
+    lm = np.asarray(W["lm_head"])
+    parts, picks = [], []
+    for start, count in vocab_shards:
+        lg = linear(f, lm[start:start + count])
+        parts.append(lg)
+        loc = argmax_f32(lg)
+        picks.append((lg.astype(np.float32)[np.arange(lg.shape[0]), loc], loc + start))
+    vals = np.stack([p[0] for p in picks])                   # [shards, rows] float32
+    ids = np.stack([p[1] for p in picks])
+    vals = np.where(np.isnan(vals), -np.inf, vals)
+    best = np.empty(f.shape[0], dtype=np.int64)
+    for row in range(f.shape[0]):
+        top = vals[:, row].max()
+        best[row] = ids[vals[:, row] == top, row].min()
+    drafts = best.reshape(B, K)
+    block = np.concatenate([bonus[:, None], drafts], axis=1)
+    return Proposal(drafts, block, np.concatenate(parts, axis=1), x)
