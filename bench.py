@@ -39,7 +39,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "draft blocks/sec and draft tokens/sec at batch B; % HBM / tensor-core roofline"
-DEFAULT_WORKLOAD = "qwen3_b1_ctx2048"
+DEFAULT_WORKLOAD = "qwen3_b128_ctx8192_32768"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM traffic per launch measured with ncu (dram__bytes_read.sum +
@@ -47,7 +47,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # keyed by the digest of the kernel sources it was measured on.
 TRAFFIC = {
     # gate/up GEMM of the batch-1 Qwen3-8B-shaped step: 201.57 MB read + 3.55 MB written
-    # (ncu --set full, profiles/gemm_gate_up_qwen3_b1_ctx2048.md)
+    # (ncu --set full on one launch)
     ("qwen3_b1_ctx2048", "gemm_gate_up"): {"bytes_per_launch": 205118208,
                                            "digest": "59a7f03b8506a4c8"},
 }
@@ -56,7 +56,7 @@ TRAFFIC = {
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
@@ -770,6 +770,13 @@ class OracleStep:
         O.propose(self.oc, self.W, self.bonus, self.seq, self.table, self.kc, self.vc, "device")
 
 
+def one_thread():
+    """The oracle runs single-threaded: numpy's BLAS pool limited to one thread
+    for the duration of the CPU legs."""
+    from threadpoolctl import threadpool_limits
+    return threadpool_limits(limits=1, user_api="blas")
+
+
 def blas_threads() -> int:
     try:
         from threadpoolctl import threadpool_info
@@ -779,21 +786,36 @@ def blas_threads() -> int:
         return os.cpu_count() or 1
 
 
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except Exception:
+        pass
+    return "unknown"
+
+
 def cpu_baseline(wl_name: str, seed: int, target_s: float = 10.0) -> dict:
     os_ = OracleStep(wl_name, seed)
-    t0 = time.perf_counter()
-    n = 0
-    while True:
-        os_.step()
-        n += 1
-        if time.perf_counter() - t0 >= target_s:
-            break
-    dt = (time.perf_counter() - t0) / n
-    return {"value": os_.n / dt, "unit": "blocks/s", "cores": blas_threads(), "kind": "oracle",
+    with one_thread():
+        threads = blas_threads()
+        t0 = time.perf_counter()
+        n = 0
+        while True:
+            os_.step()
+            n += 1
+            if time.perf_counter() - t0 >= target_s:
+                break
+        dt = (time.perf_counter() - t0) / n
+    extrap = os_.n < os_.B
+    return {"value": os_.n / dt, "unit": "blocks/s", "cores": threads, "kind": "oracle",
             "sample": f"{n} oracle step(s) of {os_.n} of {os_.B} request(s) (verify + inject + "
-                      f"propose, device storage precision), {dt:.2f} s per step; numpy float64, "
-                      f"BLAS threads = cores",
-            "host_cores": os.cpu_count()}
+                      f"propose, device storage precision, whole contexts), {dt:.2f} s per step; "
+                      f"numpy float64 on one thread"
+                      + (f"; requests are independent, so the per-request rate of the sample "
+                         f"stands for the batch of {os_.B} (extrapolated)" if extrap else ""),
+            "extrapolated": extrap, "host_cores": os.cpu_count(), "cpu_model": cpu_model()}
 
 
 # Wall-clock bound of the reference arm's timed steps: one oracle step of a
@@ -807,6 +829,8 @@ def run_reference(a, rank, world):
     if rank != 0:
         return
     os_ = OracleStep(a.workload, a.seed)
+    lim = one_thread()
+    threads = blas_threads()
     # warm-up: one whole oracle step, which also times it (taken even when W = 0)
     t0 = time.perf_counter()
     os_.step()
@@ -819,6 +843,7 @@ def run_reference(a, rank, world):
             os_.step()
             done += 1
     elapsed = time.perf_counter() - t0
+    lim.restore_original_limits()
     dt = elapsed / a.steps
     value = done * os_.n / elapsed
     line = {
@@ -829,14 +854,17 @@ def run_reference(a, rank, world):
         "data": "synthetic",
         "config": {"workload": a.workload, "batch_per_gpu": os_.B,
                    "block_size": os_.cfg["block_size"]},
-        "cpu_baseline": {"value": value, "unit": "blocks/s", "cores": blas_threads(),
+        "cpu_baseline": {"value": value, "unit": "blocks/s", "cores": threads,
                          "kind": "oracle",
                          "sample": f"{done} whole oracle step(s) of {os_.n} of {os_.B} "
                                    f"request(s) (verify + inject + propose at the device "
-                                   f"storage precision, {t_one:.1f} s each) spread evenly over "
-                                   f"the {a.steps} timed steps to bound the run at "
-                                   f"{REF_BUDGET_S:.0f} s; value = requests processed / "
-                                   f"elapsed time"},
+                                   f"storage precision, whole contexts, {t_one:.1f} s each, one "
+                                   f"thread) spread evenly over the {a.steps} timed steps to "
+                                   f"bound the run at {REF_BUDGET_S:.0f} s; value = requests "
+                                   f"processed / elapsed time"
+                                   + ("; the per-request rate of the sample stands for the "
+                                      "whole batch (extrapolated)" if os_.n < os_.B else ""),
+                         "extrapolated": os_.n < os_.B, "cpu_model": cpu_model()},
         "oracle_steps_timed": done,
         "e2e": {"value": value, "unit": "blocks/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},

@@ -5,6 +5,7 @@ CUDA); ``dflash`` is its thin Python binding and ``synth`` the seeded
 synthetic-input generator used by the tests and the benchmark.
 """
 
-from .dflash import (DFlash, DFlashError, StepGraph, Workspace, finalize_draft_keys,  # noqa: F401
-                     lib, paged_slots, prepare_proposal_inputs, status_string, verify_greedy,
+from .dflash import (DFlash, DFlashError, StepGraph, TargetModel, Workspace,  # noqa: F401
+                     aux_capture_layers, finalize_draft_keys, lib, paged_slots,
+                     prepare_proposal_inputs, set_wait_limit, status_string, verify_greedy,
                      verify_workspace_bytes, version)

@@ -21,12 +21,15 @@
 #include "dflash.h"
 #include "gemm_tcgen05.cuh"
 #include "small_kernels.cuh"
+#include "target_model.cuh"
 
 using namespace dflash;
 
 namespace {
 
 constexpr int kCounterSlots = 1 << 16;
+constexpr float kFp16Max = 65504.f;            // largest finite fp16
+constexpr double kFp16SubnormalLimit = 0.01;   // fraction of fp16-subnormal weights refused
 constexpr size_t kAlign = 256;
 
 size_t align_up(size_t v, size_t a = kAlign) { return (v + a - 1) / a * a; }
@@ -315,6 +318,11 @@ struct dflash_handle {
   float2* rope = nullptr;   // [max_position, D/2]
   unsigned* dev_err = nullptr;
   unsigned* counters = nullptr;
+  // fp16 range of the weights stored in fp16 (checked by dflash_create)
+  unsigned* range_stats = nullptr;
+  float fp16_weight_absmax = 0.f;
+  double fp16_subnormal_fraction = 0.0;
+  double norm_output_bound = 0.0;
   std::mutex mu;
   std::map<std::tuple<const void*, uint64_t, uint64_t, uint32_t, bool>, CUtensorMap> tmaps;
   std::map<std::pair<const void*, int>, std::array<int, 9>> cluster_caps;
@@ -386,6 +394,7 @@ void free_handle(dflash_handle* h) {
   cudaFree(h->rope);
   cudaFree(h->dev_err);
   cudaFree(h->counters);
+  cudaFree(h->range_stats);
   delete h;
 }
 
@@ -671,9 +680,26 @@ dflash_status run_gemm_chain(dflash_handle* h, int kind, bool f16_1, const void*
                          h->counters + (pl1.stream_k ? pl1.tiles : 0), &ta2, &tw2, &g2))
     return DFLASH_ERR_CUDA;
   unsigned* dep = h->counters + kCounterSlots - 2;
+  // every CTA waits for all the others' phase-1 stores: the grid must be
+  // co-resident, which a cooperative launch guarantees (or refuses)
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gemm_chain_kernel<256, Epi1, Epi2>,
+                                                    kGemmThreads, pl1.smem) != cudaSuccess ||
+      per_sm < 1)
+    return DFLASH_ERR_UNSUPPORTED_SHAPE;
   LaunchScope scope(h, kind, st);
-  launch_k(h->pdl, gemm_chain_kernel<256, Epi1, Epi2>, dim3(grid), dim3(kGemmThreads), pl1.smem,
-           st, ta1, tw1, g1, e1, ta2, tw2, g2, e2, dep);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = pl1.smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, gemm_chain_kernel<256, Epi1, Epi2>, ta1, tw1, g1, e1, ta2, tw2, g2, e2,
+                     dep);
   return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ERR_CUDA;
 }
 
@@ -1011,11 +1037,26 @@ const char* dflash_status_string(dflash_status s) {
     case DFLASH_ERR_DEVICE_BOUNDS: return "DFLASH_ERR_DEVICE_BOUNDS";
     case DFLASH_ERR_UNIMPLEMENTED: return "DFLASH_ERR_UNIMPLEMENTED";
     case DFLASH_ERR_DEVICE_TIMEOUT: return "DFLASH_ERR_DEVICE_TIMEOUT";
+    case DFLASH_ERR_RANGE: return "DFLASH_ERR_RANGE";
   }
   return "DFLASH_ERR_UNKNOWN";
 }
 
 const char* dflash_version(void) { return "dflash-b200 0.1 (sm_100a)"; }
+
+dflash_status dflash_set_wait_limit(int device, long long cycles) {
+  if (cycles <= 0) return DFLASH_ERR_INVALID_ARG;
+  DF_CUDA(use_device(device));
+  DF_CUDA(cudaMemcpyToSymbol(g_wait_limit_cycles, &cycles, sizeof(cycles)));
+  return DFLASH_OK;
+}
+
+dflash_status dflash_selftest_wait_timeout(dflash_handle* h, void* stream) {
+  if (!h) return DFLASH_ERR_INVALID_ARG;
+  DF_CUDA(use_device(h->device));
+  wait_timeout_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(h->dev_err);
+  return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ERR_CUDA;
+}
 
 dflash_status dflash_create(const dflash_config* cfg, const dflash_weights* w, int device,
                             dflash_handle** out) {
@@ -1168,12 +1209,27 @@ dflash_status dflash_create_vocab_shard(const dflash_config* cfg, const dflash_w
       cudaMemcpyAsync(h->lm_head16, w->lm_head, static_cast<size_t>(vocab_count) * rowb,
                       cudaMemcpyDeviceToDevice, st) != cudaSuccess)
     return fail_st(DFLASH_ERR_CUDA);
+  // fp16 range statistics of the converted weights and of the norm weights
+  // whose RMSNorm outputs are stored in fp16 (device words, read back below)
+  unsigned* stats = nullptr;
+  if (cudaMalloc(&stats, 4 * sizeof(unsigned)) != cudaSuccess) return fail_st(DFLASH_ERR_CUDA);
+  h->range_stats = stats;
+  if (cudaMemsetAsync(stats, 0, 4 * sizeof(unsigned), st) != cudaSuccess)
+    return fail_st(DFLASH_ERR_CUDA);
+  size_t f16_values = 0;
   {
     auto to_f16 = [&](void* ptr, size_t n) {
-      bf16_to_f16_kernel<<<1184, 256, 0, st>>>(static_cast<uint16_t*>(ptr), n);
+      bf16_to_f16_kernel<<<1184, 256, 0, st>>>(static_cast<uint16_t*>(ptr), n, stats);
+      f16_values += n;
       return cudaGetLastError() == cudaSuccess;
     };
-    bool ok = true;
+    auto norm_max = [&](const bf16* w, int n) {
+      absmax_bf16_kernel<<<1, 256, 0, st>>>(w, n, stats);
+      return cudaGetLastError() == cudaSuccess;
+    };
+    bool ok = norm_max(h->hidden_norm_w, H) && norm_max(h->final_norm_w, H);
+    for (int l = 0; l < L; ++l)
+      ok = ok && norm_max(h->in_norm_w[l], H) && norm_max(h->post_norm_w[l], H);
     for (int l = 0; l < L; ++l) {
       ok = ok && to_f16(h->wqkv[l], static_cast<size_t>(Hq + 2 * Hkv) * D * H);
       ok = ok && to_f16(h->wgu[l], static_cast<size_t>(2 * I) * H);
@@ -1255,6 +1311,22 @@ dflash_status dflash_create_vocab_shard(const dflash_config* cfg, const dflash_w
       set_attn_attrs<64>() != cudaSuccess || set_attn_attrs<128>() != cudaSuccess)
     return fail_st(DFLASH_ERR_CUDA);
   if (cudaStreamSynchronize(st) != cudaSuccess) return fail_st(DFLASH_ERR_CUDA);
+  // the fp16 storage of the path holds these weights and norm outputs only in
+  // fp16's range: refuse weights beyond it, weights so small that more than 1%
+  // of them would be fp16 subnormals, and norm weights whose RMSNorm outputs
+  // (|y_i| <= sqrt(hidden) * max|w|) could overflow fp16
+  unsigned hs[4] = {0, 0, 0, 0};
+  if (cudaMemcpy(hs, stats, sizeof(hs), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return fail_st(DFLASH_ERR_CUDA);
+  float wmax, nmax;
+  std::memcpy(&wmax, &hs[0], 4);
+  std::memcpy(&nmax, &hs[2], 4);
+  h->fp16_weight_absmax = wmax;
+  h->fp16_subnormal_fraction = f16_values ? static_cast<double>(hs[1]) / f16_values : 0.0;
+  h->norm_output_bound = std::sqrt(static_cast<double>(H)) * nmax;
+  if (!(wmax <= kFp16Max) || h->fp16_subnormal_fraction > kFp16SubnormalLimit ||
+      !(h->norm_output_bound <= kFp16Max))
+    return fail_st(DFLASH_ERR_RANGE);
   cudaStreamDestroy(st);
   *out = h;
   return DFLASH_OK;
@@ -1275,6 +1347,11 @@ size_t dflash_propose_workspace_bytes(const dflash_handle* h, int max_batch,
                                       int max_pages_per_seq) {
   if (!h || max_batch <= 0 || max_pages_per_seq <= 0) return 0;
   return propose_layout(h, max_batch, max_pages_per_seq).total;
+}
+
+size_t dflash_propose_final_rows_offset(const dflash_handle* h, int B, int max_pages_per_seq) {
+  if (!h || B <= 0 || max_pages_per_seq <= 0) return static_cast<size_t>(-1);
+  return propose_layout(h, B, max_pages_per_seq).frows;
 }
 
 
@@ -1515,6 +1592,7 @@ dflash_status dflash_verify_greedy(const int32_t* drafts, const float* target_lo
                                    void* stream) {
   if (B < 0 || K < 0 || V <= 0 || K > 128) return DFLASH_ERR_INVALID_ARG;
   if (B == 0) return DFLASH_OK;
+  if (static_cast<int64_t>(B) * (K + 1) > (1 << 30)) return DFLASH_ERR_UNSUPPORTED_SHAPE;
   if ((K > 0 && !drafts) || !target_logits || !out_tokens || !num_accepted || !bonus ||
       !workspace)
     return DFLASH_ERR_INVALID_ARG;
@@ -1526,8 +1604,8 @@ dflash_status dflash_verify_greedy(const int32_t* drafts, const float* target_lo
   dflash_status s = set_device_for(st, out_tokens);
   if (s != DFLASH_OK) return s;
   unsigned long long* part = static_cast<unsigned long long*>(workspace);
-  launch_k(pdl_default(), verify_partial_kernel, dim3(vp.chunks, B * (K + 1)), dim3(256), 0, st,
-           target_logits, V, vp.chunk_len, vp.chunks, part);
+  launch_k(pdl_default(), verify_partial_kernel, dim3(vp.chunks, std::min(B * (K + 1), 65535)),
+           dim3(256), 0, st, target_logits, V, vp.chunk_len, vp.chunks, B * (K + 1), part);
   launch_k(pdl_default(), verify_final_kernel, dim3(B), dim3(256), 0, st, part, vp.chunks, drafts,
            K, out_tokens, num_accepted, bonus);
   return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ERR_CUDA;
@@ -1915,25 +1993,60 @@ static __device__ __align__(256) unsigned long long g_verify_scratch[kNoAllocVer
 
 constexpr int kNoAllocMaxDevices = 64;
 std::mutex g_verify_scratch_mu;
-unsigned long long* g_verify_scratch_dev[kNoAllocMaxDevices] = {};
+struct ScratchAddr {
+  unsigned long long ctx_id = 0;       // context the address belongs to (0: none yet)
+  unsigned long long* ptr = nullptr;
+};
+ScratchAddr g_verify_scratch_dev[kNoAllocMaxDevices];
+
+// Unique id of the calling thread's current CUDA context (driver entry points
+// looked up once; no link-time libcuda dependency).  0 if unavailable.
+unsigned long long current_context_id() {
+  typedef CUresult (*GetCurrentFn)(CUcontext*);
+  typedef CUresult (*GetIdFn)(CUcontext, unsigned long long*);
+  static GetCurrentFn get_current = nullptr;
+  static GetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<GetCurrentFn>(p);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<GetIdFn>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx ||
+      get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
 
 // On the host, g_verify_scratch only names the symbol; a kernel given that
 // name would read the wrong memory.  The array's device address is looked up
-// once per device (with that device current) and cached.
+// per device (with that device current) and cached together with the id of
+// the context it belongs to: after a device reset the runtime builds a new
+// context, the id changes, and the address is looked up again.
 dflash_status verify_scratch_on_current_device(unsigned long long** out) {
   int dev = -1;
   DF_CUDA(cudaGetDevice(&dev));
   if (dev < 0 || dev >= kNoAllocMaxDevices) return DFLASH_ERR_UNSUPPORTED_SHAPE;
+  const unsigned long long ctx = current_context_id();   // 0 before the context exists
   std::lock_guard<std::mutex> lk(g_verify_scratch_mu);
-  if (!g_verify_scratch_dev[dev]) {
+  ScratchAddr& a = g_verify_scratch_dev[dev];
+  if (!a.ptr || ctx == 0 || a.ctx_id != ctx) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_verify_scratch) != cudaSuccess || p == nullptr) {
       cudaGetLastError();
       return DFLASH_ERR_CUDA;
     }
-    g_verify_scratch_dev[dev] = static_cast<unsigned long long*>(p);
+    a.ptr = static_cast<unsigned long long*>(p);
+    a.ctx_id = current_context_id();
   }
-  *out = g_verify_scratch_dev[dev];
+  *out = a.ptr;
   return DFLASH_OK;
 }
 
@@ -1946,6 +2059,7 @@ extern "C" dflash_status dflash_verify_greedy_noalloc(const int32_t* drafts,
                                                       void* stream) {
   if (B < 0 || K < 0 || V <= 0 || K > 128) return DFLASH_ERR_INVALID_ARG;
   if (B == 0) return DFLASH_OK;
+  if (static_cast<int64_t>(B) * (K + 1) > (1 << 30)) return DFLASH_ERR_UNSUPPORTED_SHAPE;
   if ((K > 0 && !drafts) || !target_logits || !out_tokens || !num_accepted || !bonus)
     return DFLASH_ERR_INVALID_ARG;
   const VerifyPlan vp = plan_verify(B, K, V);
@@ -1961,9 +2075,231 @@ extern "C" dflash_status dflash_verify_greedy_noalloc(const int32_t* drafts,
   if (s != DFLASH_OK) return s;
   // Nothing in the scratch has to start at zero: the second kernel reads only
   // the keys the first one writes in this same call.
-  launch_k(pdl_default(), verify_partial_kernel, dim3(vp.chunks, B * (K + 1)), dim3(256), 0, st,
-           target_logits, V, vp.chunk_len, vp.chunks, part);
+  launch_k(pdl_default(), verify_partial_kernel, dim3(vp.chunks, std::min(B * (K + 1), 65535)),
+           dim3(256), 0, st, target_logits, V, vp.chunk_len, vp.chunks, B * (K + 1), part);
   launch_k(pdl_default(), verify_final_kernel, dim3(B), dim3(256), 0, st, part, vp.chunks, drafts,
            K, out_tokens, num_accepted, bonus);
   return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ERR_CUDA;
 }
+
+// ===========================================================================
+// A small causal target model on the device (the on-device lossless loop)
+// ===========================================================================
+struct dflash_target {
+  dflash_target_config cfg{};
+  std::vector<int> capture;          // pre-layer capture indices, request order
+  int device = 0;
+  const float *embed = nullptr, *final_norm_w = nullptr, *lm_head = nullptr;
+  std::vector<const float*> in_norm_w, post_norm_w, q_norm_w, k_norm_w, wo, wdown;
+  std::vector<float*> wqkv, wgu;     // owned: [Wq; Wk; Wv] and [Wgate; Wup] per layer
+  float *kcache = nullptr, *vcache = nullptr;   // owned: [L][max_len][Hkv][D] each
+  unsigned* dev_err = nullptr;
+};
+
+namespace {
+struct TargetWs {
+  size_t x, y, qkv, q, o, gu, hm, total;
+};
+TargetWs target_layout(const dflash_target_config& c, int n) {
+  TargetWs w{};
+  size_t off = 0;
+  auto take = [&off](size_t floats) {
+    const size_t at = off;
+    off += align_up(floats * 4);
+    return at;
+  };
+  const size_t rows = static_cast<size_t>(n);
+  w.x = take(rows * c.hidden);
+  w.y = take(rows * c.hidden);
+  w.qkv = take(rows * (c.n_q_heads + 2 * c.n_kv_heads) * c.head_dim);
+  w.q = take(rows * c.n_q_heads * c.head_dim);
+  w.o = take(rows * c.n_q_heads * c.head_dim);
+  w.gu = take(rows * 2 * c.intermediate);
+  w.hm = take(rows * c.intermediate);
+  w.total = off;
+  return w;
+}
+void free_target(dflash_target* t) {
+  if (!t) return;
+  for (auto p : t->wqkv) cudaFree(p);
+  for (auto p : t->wgu) cudaFree(p);
+  cudaFree(t->kcache);
+  cudaFree(t->vcache);
+  cudaFree(t->dev_err);
+  delete t;
+}
+}  // namespace
+
+extern "C" {
+
+dflash_status dflash_aux_capture_layers(const int* target_layer_ids, int n, int target_n_layers,
+                                        int* capture_layers) {
+  if (n < 0 || target_n_layers <= 0 || (n > 0 && (!target_layer_ids || !capture_layers)))
+    return DFLASH_ERR_INVALID_ARG;
+  for (int i = 0; i < n; ++i) {
+    // the state after layer i is the state before layer i + 1
+    const int j = target_layer_ids[i] + 1;
+    if (target_layer_ids[i] < 0 || j > target_n_layers) return DFLASH_ERR_INVALID_ARG;
+    capture_layers[i] = j;
+  }
+  return DFLASH_OK;
+}
+
+dflash_status dflash_target_create(const dflash_target_config* cfg, const dflash_target_weights* w,
+                                   int device, dflash_target** out) {
+  if (!out) return DFLASH_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!cfg || !w) return DFLASH_ERR_INVALID_ARG;
+  const dflash_target_config& c = *cfg;
+  if (c.hidden <= 0 || c.n_layers <= 0 || c.n_q_heads <= 0 || c.n_kv_heads <= 0 ||
+      c.head_dim <= 0 || c.intermediate <= 0 || c.vocab <= 0 || c.max_len <= 0 ||
+      c.n_capture < 0 || (c.n_capture > 0 && !c.capture_layers) || !(c.rms_eps >= 0.f) ||
+      !(c.rope_theta > 0.f))
+    return DFLASH_ERR_INVALID_ARG;
+  if (c.head_dim % 32 || c.head_dim > 128 || c.n_q_heads % c.n_kv_heads || c.head_dim % 2)
+    return DFLASH_ERR_UNSUPPORTED_SHAPE;
+  for (int i = 0; i < c.n_capture; ++i)
+    if (c.capture_layers[i] < 0 || c.capture_layers[i] > c.n_layers) return DFLASH_ERR_INVALID_ARG;
+  const int L = c.n_layers;
+  if (!w->embed || !w->final_norm_w || !w->lm_head || !w->in_norm_w || !w->post_norm_w ||
+      !w->wq || !w->wk || !w->wv || !w->wo || !w->q_norm_w || !w->k_norm_w || !w->w_gate ||
+      !w->w_up || !w->w_down)
+    return DFLASH_ERR_INVALID_ARG;
+  for (int l = 0; l < L; ++l)
+    if (!w->in_norm_w[l] || !w->post_norm_w[l] || !w->wq[l] || !w->wk[l] || !w->wv[l] ||
+        !w->wo[l] || !w->q_norm_w[l] || !w->k_norm_w[l] || !w->w_gate[l] || !w->w_up[l] ||
+        !w->w_down[l])
+      return DFLASH_ERR_INVALID_ARG;
+  dflash_target* t = new (std::nothrow) dflash_target();
+  if (!t) return DFLASH_ERR_CUDA;
+  t->cfg = c;
+  t->capture.assign(c.capture_layers, c.capture_layers + c.n_capture);
+  t->cfg.capture_layers = t->capture.empty() ? nullptr : t->capture.data();
+  t->device = device;
+  auto fail = [t](dflash_status s) {
+    free_target(t);
+    return s;
+  };
+  if (cudaSetDevice(device) != cudaSuccess) return fail(DFLASH_ERR_CUDA);
+  const int H = c.hidden, D = c.head_dim, Hq = c.n_q_heads, Hkv = c.n_kv_heads, I = c.intermediate;
+  t->embed = w->embed;
+  t->final_norm_w = w->final_norm_w;
+  t->lm_head = w->lm_head;
+  const size_t row = static_cast<size_t>(H) * 4;
+  for (int l = 0; l < L; ++l) {
+    t->in_norm_w.push_back(w->in_norm_w[l]);
+    t->post_norm_w.push_back(w->post_norm_w[l]);
+    t->q_norm_w.push_back(w->q_norm_w[l]);
+    t->k_norm_w.push_back(w->k_norm_w[l]);
+    t->wo.push_back(w->wo[l]);
+    t->wdown.push_back(w->w_down[l]);
+    float* p = nullptr;
+    if (cudaMalloc(&p, static_cast<size_t>(Hq + 2 * Hkv) * D * row) != cudaSuccess)
+      return fail(DFLASH_ERR_CUDA);
+    t->wqkv.push_back(p);
+    if (cudaMemcpy(p, w->wq[l], static_cast<size_t>(Hq) * D * row, cudaMemcpyDeviceToDevice) !=
+            cudaSuccess ||
+        cudaMemcpy(p + static_cast<size_t>(Hq) * D * H, w->wk[l], static_cast<size_t>(Hkv) * D * row,
+                   cudaMemcpyDeviceToDevice) != cudaSuccess ||
+        cudaMemcpy(p + static_cast<size_t>(Hq + Hkv) * D * H, w->wv[l],
+                   static_cast<size_t>(Hkv) * D * row, cudaMemcpyDeviceToDevice) != cudaSuccess)
+      return fail(DFLASH_ERR_CUDA);
+    if (cudaMalloc(&p, static_cast<size_t>(2 * I) * row) != cudaSuccess) return fail(DFLASH_ERR_CUDA);
+    t->wgu.push_back(p);
+    if (cudaMemcpy(p, w->w_gate[l], static_cast<size_t>(I) * row, cudaMemcpyDeviceToDevice) !=
+            cudaSuccess ||
+        cudaMemcpy(p + static_cast<size_t>(I) * H, w->w_up[l], static_cast<size_t>(I) * row,
+                   cudaMemcpyDeviceToDevice) != cudaSuccess)
+      return fail(DFLASH_ERR_CUDA);
+  }
+  const size_t cache = static_cast<size_t>(L) * c.max_len * Hkv * D * 4;
+  if (cudaMalloc(&t->kcache, cache) != cudaSuccess || cudaMalloc(&t->vcache, cache) != cudaSuccess ||
+      cudaMemset(t->kcache, 0, cache) != cudaSuccess || cudaMemset(t->vcache, 0, cache) != cudaSuccess ||
+      cudaMalloc(&t->dev_err, sizeof(unsigned)) != cudaSuccess ||
+      cudaMemset(t->dev_err, 0, sizeof(unsigned)) != cudaSuccess ||
+      cudaDeviceSynchronize() != cudaSuccess)
+    return fail(DFLASH_ERR_CUDA);
+  *out = t;
+  return DFLASH_OK;
+}
+
+void dflash_target_destroy(dflash_target* t) {
+  if (!t) return;
+  cudaSetDevice(t->device);
+  free_target(t);
+}
+
+size_t dflash_target_workspace_bytes(const dflash_target* t, int n) {
+  if (!t || n <= 0) return 0;
+  return target_layout(t->cfg, n).total;
+}
+
+dflash_status dflash_target_forward(dflash_target* t, const int32_t* tokens, int n, int start_pos,
+                                    float* logits, void* aux, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
+  if (!t || n < 0) return DFLASH_ERR_INVALID_ARG;
+  if (n == 0) return DFLASH_OK;
+  const dflash_target_config& c = t->cfg;
+  if (!tokens || !logits || !workspace || (c.n_capture > 0 && !aux)) return DFLASH_ERR_INVALID_ARG;
+  if (start_pos < 0 || static_cast<int64_t>(start_pos) + n > c.max_len)
+    return DFLASH_ERR_INVALID_ARG;
+  const TargetWs ws = target_layout(c, n);
+  if (workspace_bytes < ws.total) return DFLASH_ERR_WORKSPACE;
+  DF_CUDA(use_device(t->device));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int H = c.hidden, D = c.head_dim, Hq = c.n_q_heads, Hkv = c.n_kv_heads,
+            I = c.intermediate, V = c.vocab, L = c.n_layers;
+  float* x = at<float>(workspace, ws.x);
+  float* y = at<float>(workspace, ws.y);
+  float* qkv = at<float>(workspace, ws.qkv);
+  float* q = at<float>(workspace, ws.q);
+  float* o = at<float>(workspace, ws.o);
+  float* gu = at<float>(workspace, ws.gu);
+  float* hm = at<float>(workspace, ws.hm);
+  bf16* ax = static_cast<bf16*>(aux);
+  TargetDims d{H, Hq, Hkv, D, I, V, c.max_len, c.rms_eps, c.rope_theta};
+  auto linear = [&](const float* a, const float* W, int N, int K, float* dst, int acc) {
+    target_linear_kernel<<<dim3(cdiv(N, 8), n), 256, 0, st>>>(a, W, N, K, dst, acc);
+  };
+  auto capture = [&](int layer) {
+    for (int k = 0; k < c.n_capture; ++k)
+      if (t->capture[k] == layer)
+        target_capture_kernel<<<cdiv(n * H, 256), 256, 0, st>>>(x, n, H, c.n_capture, k, ax);
+  };
+  target_embed_kernel<<<n, 256, 0, st>>>(tokens, t->embed, H, V, x, t->dev_err);
+  const size_t layer_cache = static_cast<size_t>(c.max_len) * Hkv * D;
+  for (int l = 0; l < L; ++l) {
+    capture(l);
+    target_rmsnorm_kernel<<<n, 256, 0, st>>>(x, t->in_norm_w[l], H, c.rms_eps, y);
+    linear(y, t->wqkv[l], (Hq + 2 * Hkv) * D, H, qkv, 0);
+    target_qkv_kernel<<<cdiv(n * (Hq + Hkv), 8), 256, 0, st>>>(
+        qkv, n, start_pos, d, t->q_norm_w[l], t->k_norm_w[l], q, t->kcache + l * layer_cache,
+        t->vcache + l * layer_cache, t->dev_err);
+    target_attention_kernel<<<cdiv(n * Hq, 8), 256, 0, st>>>(
+        q, n, start_pos, d, t->kcache + l * layer_cache, t->vcache + l * layer_cache, o);
+    linear(o, t->wo[l], H, Hq * D, x, 1);
+    target_rmsnorm_kernel<<<n, 256, 0, st>>>(x, t->post_norm_w[l], H, c.rms_eps, y);
+    linear(y, t->wgu[l], 2 * I, H, gu, 0);
+    target_swiglu_kernel<<<cdiv(n * I, 256), 256, 0, st>>>(gu, I, n, hm);
+    linear(hm, t->wdown[l], H, I, x, 1);
+  }
+  capture(L);
+  target_rmsnorm_kernel<<<n, 256, 0, st>>>(x, t->final_norm_w, H, c.rms_eps, y);
+  linear(y, t->lm_head, V, H, logits, 0);
+  return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ERR_CUDA;
+}
+
+dflash_status dflash_target_check_device_errors(dflash_target* t, unsigned* bits) {
+  if (bits) *bits = 0;
+  if (!t) return DFLASH_ERR_INVALID_ARG;
+  DF_CUDA(use_device(t->device));
+  DF_CUDA(cudaDeviceSynchronize());
+  unsigned v = 0;
+  DF_CUDA(cudaMemcpy(&v, t->dev_err, sizeof(unsigned), cudaMemcpyDeviceToHost));
+  DF_CUDA(cudaMemset(t->dev_err, 0, sizeof(unsigned)));
+  if (bits) *bits = v;
+  return v ? DFLASH_ERR_DEVICE_BOUNDS : DFLASH_OK;
+}
+
+}  // extern "C"
+

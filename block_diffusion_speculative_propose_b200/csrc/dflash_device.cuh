@@ -24,9 +24,11 @@ __device__ __forceinline__ void raise_error(unsigned* err, unsigned bit) {
   if (err) atomicOr(err, bit);
 }
 
-// Pipeline waits give up after this many SM cycles (about 2 s at 1.9 GHz):
-// a wait that long means the pipeline is broken, never that it is busy.
+// Pipeline waits give up after this many SM cycles (default about 2 s at
+// 1.9 GHz): a wait that long means the pipeline is broken, never that it is
+// busy.  One value per device, set by dflash_set_wait_limit (diagnostics).
 constexpr long long kWaitLimitCycles = 4000000000LL;
+__device__ long long g_wait_limit_cycles = kWaitLimitCycles;
 
 // ---------------------------------------------------------------------------
 // small conversions
@@ -109,7 +111,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsign
   const long long t0 = clock64();
   for (unsigned spin = 1; !mbar_try_wait(bar, parity); ++spin) {
     if ((spin & 1023u) == 0) {
-      if (clock64() - t0 > kWaitLimitCycles) {
+      if (clock64() - t0 > *reinterpret_cast<volatile long long*>(&g_wait_limit_cycles)) {
         raise_error(err, DFLASH_DEVERR_TIMEOUT);
         return false;
       }

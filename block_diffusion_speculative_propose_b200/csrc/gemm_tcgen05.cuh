@@ -234,7 +234,7 @@ __device__ __forceinline__ bool wait_count(const unsigned* ctr, unsigned target,
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
     if (v >= target) return true;
     if ((spin & 63u) == 63u) {
-      if (clock64() - t0 > kWaitLimitCycles) {
+      if (clock64() - t0 > *reinterpret_cast<volatile long long*>(&g_wait_limit_cycles)) {
         raise_error(err, DFLASH_DEVERR_TIMEOUT);
         return false;
       }

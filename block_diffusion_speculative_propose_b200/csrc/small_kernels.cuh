@@ -189,12 +189,13 @@ __global__ void draft_keys_finalize_kernel(const int64_t* __restrict__ keys,
 // Greedy verification, pass 1: per (row, chunk) ordered argmax key of the fp32
 // target logits.  Rows are [B * (K+1)], each V long.
 __global__ void __launch_bounds__(256) verify_partial_kernel(
-    const float* __restrict__ logits, int V, int chunk_len, int chunks,
+    const float* __restrict__ logits, int V, int chunk_len, int chunks, int rows,
     unsigned long long* __restrict__ part) {
   pdl_trigger();
   pdl_wait();
   __shared__ unsigned long long red[32];
-  const size_t row = blockIdx.y;
+  // grid.y is capped at 65535: CTAs step over the rows
+  for (size_t row = blockIdx.y; row < static_cast<size_t>(rows); row += gridDim.y) {
   const int beg = blockIdx.x * chunk_len;
   const int end = min(V, beg + chunk_len);
   const float* src = logits + row * static_cast<size_t>(V);
@@ -226,6 +227,8 @@ __global__ void __launch_bounds__(256) verify_partial_kernel(
     unsigned long long t = lane < (blockDim.x >> 5) ? red[lane] : 0ull;
     t = warp_max_u64(t);
     if (lane == 0) part[row * chunks + blockIdx.x] = t;
+  }
+  __syncthreads();   // red[] is reused by the next row
   }
 }
 
@@ -358,13 +361,55 @@ __global__ void prepare_proposal_kernel(
   }
 }
 
-__global__ void bf16_to_f16_kernel(uint16_t* __restrict__ data, size_t n) {
+// fp16 range statistics of converted weights: stats[0] = the largest |x| seen
+// (float bits, which order like the values for x >= 0; NaN sorts above
+// infinity), stats[1] = the number of nonzero values below fp16's smallest
+// normal number (2^-14), which fp16 holds only as subnormals.
+__device__ __forceinline__ void range_stats_add(unsigned* stats, unsigned amax_bits,
+                                                unsigned small) {
+  __shared__ unsigned s_max, s_small;
+  if (threadIdx.x == 0) {
+    s_max = 0u;
+    s_small = 0u;
+  }
+  __syncthreads();
+  for (int o = 16; o > 0; o >>= 1) {
+    amax_bits = max(amax_bits, __shfl_xor_sync(0xffffffffu, amax_bits, o));
+    small += __shfl_xor_sync(0xffffffffu, small, o);
+  }
+  if ((threadIdx.x & 31) == 0) {
+    atomicMax(&s_max, amax_bits);
+    atomicAdd(&s_small, small);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    atomicMax(&stats[0], s_max);
+    atomicAdd(&stats[1], s_small);
+  }
+}
+
+__global__ void bf16_to_f16_kernel(uint16_t* __restrict__ data, size_t n, unsigned* stats) {
+  unsigned amax = 0u, small = 0u;
   for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
        i += static_cast<size_t>(gridDim.x) * blockDim.x) {
     const bf16 v = *reinterpret_cast<const bf16*>(data + i);
-    const f16 o = __float2half_rn(__bfloat162float(v));
+    const float f = __bfloat162float(v);
+    const unsigned a = __float_as_uint(f) & 0x7fffffffu;
+    amax = max(amax, a);
+    small += (a != 0u && a < 0x38800000u) ? 1u : 0u;   // 0 < |f| < 2^-14
+    const f16 o = __float2half_rn(f);
     data[i] = *reinterpret_cast<const uint16_t*>(&o);
   }
+  range_stats_add(stats, amax, small);
+}
+
+// Largest |x| of a bf16 vector into stats[2] (float bits, as above).
+__global__ void absmax_bf16_kernel(const bf16* __restrict__ x, int n, unsigned* stats) {
+  unsigned amax = 0u;
+  for (int i = threadIdx.x; i < n; i += blockDim.x)
+    amax = max(amax, __float_as_uint(__bfloat162float(x[i])) & 0x7fffffffu);
+  for (int o = 16; o > 0; o >>= 1) amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if ((threadIdx.x & 31) == 0) atomicMax(&stats[2], amax);
 }
 
 // Tile-contiguous GEMM weight layout: the kPackRows x 64 tile (n_tile, k_block)
@@ -412,6 +457,20 @@ __global__ void rope_table_kernel(float2* __restrict__ table, int max_pos, int h
     const double a = static_cast<double>(pos) * inv;
     table[static_cast<size_t>(pos) * half + j] =
         make_float2(static_cast<float>(cos(a)), static_cast<float>(sin(a)));
+  }
+}
+
+// Diagnostics: one bounded wait that runs out.  Thread 0 initialises an
+// mbarrier that expects one arrival and waits for its first phase with the
+// pipelines' own bounded wait; nothing ever arrives, so the wait gives up after
+// the device's wait limit and sets DFLASH_DEVERR_TIMEOUT in *err.  No fault, no
+// trap: the kernel then returns normally.
+__global__ void wait_timeout_selftest_kernel(unsigned* err) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+    mbar_wait(&bar, 0, err);
   }
 }
 

@@ -26,6 +26,7 @@ STATUS = {
     -5: "DFLASH_ERR_DEVICE_BOUNDS",
     -6: "DFLASH_ERR_UNIMPLEMENTED",
     -7: "DFLASH_ERR_DEVICE_TIMEOUT",
+    -8: "DFLASH_ERR_RANGE",
 }
 DEVERR_TIMEOUT, DEVERR_SLOT, DEVERR_TABLE, DEVERR_TOKEN, DEVERR_POSITION = 1, 2, 4, 8, 16
 KERNEL_KINDS = 14
@@ -74,6 +75,24 @@ class _StepIO(ctypes.Structure):
                 ("block_tokens", ctypes.c_void_p), ("device_error", ctypes.c_void_p)]
 
 
+class _TargetConfig(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in ("hidden", "n_layers", "n_q_heads", "n_kv_heads",
+                                            "head_dim", "intermediate", "vocab")] + \
+               [("rms_eps", ctypes.c_float), ("rope_theta", ctypes.c_float),
+                ("max_len", ctypes.c_int), ("n_capture", ctypes.c_int),
+                ("capture_layers", ctypes.POINTER(ctypes.c_int))]
+
+
+_TARGET_SINGLE = ("embed", "final_norm_w", "lm_head")
+_TARGET_LAYER = ("in_norm_w", "post_norm_w", "wq", "wk", "wv", "wo", "q_norm_w", "k_norm_w",
+                 "w_gate", "w_up", "w_down")
+
+
+class _TargetWeights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in _TARGET_SINGLE] + \
+               [(n, _PP) for n in _TARGET_LAYER]
+
+
 class _AttnPlan(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in ("tcgen05", "keys_per_tile", "ring_depth",
                                             "ctas_per_sm", "chunk_keys", "max_splits",
@@ -101,6 +120,17 @@ def lib() -> ctypes.CDLL:
         "dflash_destroy": ([vp], None),
         "dflash_inject_workspace_bytes": ([vp, i32], sz),
         "dflash_propose_workspace_bytes": ([vp, i32, i32], sz),
+        "dflash_propose_final_rows_offset": ([vp, i32, i32], sz),
+        "dflash_set_wait_limit": ([i32, ctypes.c_longlong], i32),
+        "dflash_aux_capture_layers": ([ctypes.POINTER(ctypes.c_int), i32, i32,
+                                       ctypes.POINTER(ctypes.c_int)], i32),
+        "dflash_target_create": ([ctypes.POINTER(_TargetConfig), ctypes.POINTER(_TargetWeights),
+                                  i32, ctypes.POINTER(vp)], i32),
+        "dflash_target_destroy": ([vp], None),
+        "dflash_target_workspace_bytes": ([vp, i32], sz),
+        "dflash_target_forward": ([vp, vp, i32, i32, vp, vp, vp, sz, vp], i32),
+        "dflash_target_check_device_errors": ([vp, ctypes.POINTER(ctypes.c_uint)], i32),
+        "dflash_selftest_wait_timeout": ([vp, vp], i32),
         "dflash_verify_workspace_bytes": ([i32, i32, i32], sz),
         "dflash_linear_workspace_bytes": ([vp, i32, i32, i32], sz),
         "dflash_attention_workspace_bytes": ([vp, i32, i32], sz),
@@ -268,6 +298,17 @@ class DFlash:
 
     def propose_workspace_bytes(self, B: int, max_pages_per_seq: int) -> int:
         return lib().dflash_propose_workspace_bytes(self.h, B, max_pages_per_seq)
+
+    def propose_final_rows(self, workspace: torch.Tensor, B: int,
+                           max_pages_per_seq: int) -> torch.Tensor:
+        """View of the [B*K, hidden] fp16 rows that the last proposal with this
+        workspace handed to the LM head (diagnostics)."""
+        off = int(lib().dflash_propose_final_rows_offset(self.h, B, max_pages_per_seq))
+        K, H = self.cfg["block_size"] - 1, self.cfg["hidden"]
+        n = B * K * H * 2
+        if off < 0 or off + n > workspace.numel():
+            raise DFlashError(-1, "dflash_propose_final_rows_offset")
+        return workspace[off:off + n].view(torch.float16).view(B * K, H)
 
     # ---------------------------------------------------------------- calls
     def inject_context(self, aux, positions, slot_mapping, k_cache, v_cache,
@@ -472,6 +513,107 @@ class DFlash:
         bits = ctypes.c_uint(0)
         lib().dflash_check_device_errors(self.h, ctypes.byref(bits))
         return int(bits.value)
+
+    def check_device_status(self):
+        """(status, bits) of dflash_check_device_errors."""
+        bits = ctypes.c_uint(0)
+        s = int(lib().dflash_check_device_errors(self.h, ctypes.byref(bits)))
+        return s, int(bits.value)
+
+    def selftest_wait_timeout(self, stream=None) -> None:
+        """Enqueue a kernel whose one bounded wait runs out (diagnostics)."""
+        _check(lib().dflash_selftest_wait_timeout(self.h, _stream(stream)),
+               "dflash_selftest_wait_timeout")
+
+
+def aux_capture_layers(target_layer_ids: Sequence[int], target_n_layers: int) -> List[int]:
+    """Capture layers (pre-layer states) for a draft checkpoint's
+    target_layer_ids (states after layer i): each id plus one."""
+    n = len(target_layer_ids)
+    ids = (ctypes.c_int * max(n, 1))(*target_layer_ids)
+    out = (ctypes.c_int * max(n, 1))()
+    _check(lib().dflash_aux_capture_layers(ids, n, int(target_n_layers), out),
+           "dflash_aux_capture_layers")
+    return [int(out[i]) for i in range(n)]
+
+
+class TargetModel:
+    """The library's small causal target model (dflash_target_*): fp32
+    weights (CUDA tensors, names of ``dflash_target_weights``), one sequence.
+    ``forward(tokens, start_pos)`` returns (logits [n, V] fp32, aux
+    [n, n_capture * H] bf16)."""
+
+    def __init__(self, cfg: Dict, weights: Dict, capture_layers: Sequence[int],
+                 max_len: int, device: int = 0):
+        L = lib()
+        self.cfg = dict(cfg)
+        self.device = torch.device("cuda", device)
+        self.n_capture = len(capture_layers)
+        self._keep: List = []
+        cap = (ctypes.c_int * max(self.n_capture, 1))(*capture_layers)
+        self._keep.append(cap)
+        c = _TargetConfig(cfg["hidden"], cfg["n_layers"], cfg["n_q_heads"], cfg["n_kv_heads"],
+                          cfg["head_dim"], cfg["intermediate"], cfg["vocab"],
+                          cfg.get("rms_eps", 1e-6), cfg.get("rope_theta", 1e6), int(max_len),
+                          self.n_capture, ctypes.cast(cap, ctypes.POINTER(ctypes.c_int)))
+        w = _TargetWeights()
+        for k in _TARGET_SINGLE:
+            t = weights[k]
+            _want(t, torch.float32, k)
+            self._keep.append(t)
+            setattr(w, k, _ptr(t))
+        for k in _TARGET_LAYER:
+            ts = list(weights[k])
+            if len(ts) != cfg["n_layers"]:
+                raise ValueError(f"{k}: expected {cfg['n_layers']} layers")
+            for t in ts:
+                _want(t, torch.float32, k)
+            self._keep.extend(ts)
+            pp, arr = _ptr_array(ts)
+            self._keep.append(arr)
+            setattr(w, k, pp)
+        h = ctypes.c_void_p()
+        _check(L.dflash_target_create(ctypes.byref(c), ctypes.byref(w), device, ctypes.byref(h)),
+               "dflash_target_create")
+        self.h = h
+        self.ws = Workspace(self.device)
+
+    def close(self) -> None:
+        if getattr(self, "h", None):
+            torch.cuda.synchronize(self.device)
+            lib().dflash_target_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def forward(self, tokens: torch.Tensor, start_pos: int, logits=None, aux=None, stream=None):
+        _want(tokens, torch.int32, "tokens")
+        n = int(tokens.numel())
+        H, V = self.cfg["hidden"], self.cfg["vocab"]
+        if logits is None:
+            logits = torch.empty(n, V, dtype=torch.float32, device=self.device)
+        if aux is None and self.n_capture:
+            aux = torch.empty(n, self.n_capture * H, dtype=torch.bfloat16, device=self.device)
+        ws = self.ws.get(lib().dflash_target_workspace_bytes(self.h, max(n, 1)))
+        _check(lib().dflash_target_forward(self.h, _ptr(tokens), n, int(start_pos), _ptr(logits),
+                                           _ptr(aux), _ptr(ws), ws.numel(), _stream(stream)),
+               "dflash_target_forward")
+        return logits, aux
+
+    def check_device_errors(self) -> int:
+        bits = ctypes.c_uint(0)
+        lib().dflash_target_check_device_errors(self.h, ctypes.byref(bits))
+        return int(bits.value)
+
+
+def set_wait_limit(device: int, cycles: int) -> None:
+    """Cycles after which every bounded wait of the library's kernels on
+    `device` gives up (diagnostics; default 4e9)."""
+    _check(lib().dflash_set_wait_limit(int(device), int(cycles)), "dflash_set_wait_limit")
 
 
 class StepGraph:

@@ -118,6 +118,26 @@ def make_weights(cfg: dict, seed: int = 0, device="cpu",
     return W
 
 
+def target_config(draft_cfg: dict, n_layers: int) -> dict:
+    """A small causal target for a draft: the draft's layer shape and
+    vocabulary with its own depth."""
+    keys = ("hidden", "n_q_heads", "n_kv_heads", "head_dim", "intermediate", "vocab",
+            "rms_eps", "rope_theta")
+    return dict({k: draft_cfg[k] for k in keys}, n_layers=n_layers)
+
+
+def make_target_weights(tcfg: dict, seed: int = 0, device="cpu",
+                        std: float = 0.05) -> Dict[str, object]:
+    """Random-init target weights as float32 tensors holding bf16 values (so
+    that a draft's bf16 aliases of the embedding and LM head carry the same
+    numbers).  Same names and layouts as make_weights, without fc / hidden_norm."""
+    W = make_weights(dict(tcfg, n_target_layers=1, block_size=2, mask_token_id=0), seed,
+                     device, std)
+    del W["fc_w"], W["hidden_norm_w"]
+    return {k: ([x.float() for x in v] if isinstance(v, list) else v.float())
+            for k, v in W.items()}
+
+
 # ----------------------------------------------------------------------------
 # one step's batch
 # ----------------------------------------------------------------------------

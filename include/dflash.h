@@ -67,7 +67,8 @@ typedef enum {
   DFLASH_ERR_UNSUPPORTED_SHAPE = -4, /* geometry outside what the kernels are built for       */
   DFLASH_ERR_DEVICE_BOUNDS = -5,     /* returned by dflash_check_device_errors (see above)    */
   DFLASH_ERR_UNIMPLEMENTED = -6,
-  DFLASH_ERR_DEVICE_TIMEOUT = -7     /* returned by dflash_check_device_errors                */
+  DFLASH_ERR_DEVICE_TIMEOUT = -7,    /* returned by dflash_check_device_errors                */
+  DFLASH_ERR_RANGE = -8              /* weights outside the fp16 range the path stores them in */
 } dflash_status;
 
 /* Device error bits reported by dflash_check_device_errors(). */
@@ -144,7 +145,13 @@ typedef struct dflash_handle dflash_handle;
 /* Validates the geometry, makes `device` current, packs the weights and builds
  * the RoPE table (cos/sin of pos * theta^(-2i/d), evaluated in double precision
  * on the device).  Synchronizes the device once at the end.  On success *out
- * receives the handle; on failure *out is NULL and nothing is leaked. */
+ * receives the handle; on failure *out is NULL and nothing is leaked.
+ * Range of the fp16 storage (DFLASH_ERR_RANGE otherwise): every weight copied
+ * to fp16 (wq, wk, wv, wo, w_gate, w_up, lm_head) has |w| <= 65504 and at most
+ * 1% of the nonzero ones lie below 2^-14 (where fp16 keeps them only as
+ * subnormals); the norm weights whose RMSNorm outputs are stored in fp16
+ * (hidden_norm_w, in_norm_w, post_norm_w, final_norm_w) have
+ * sqrt(hidden) * max|w| <= 65504, the bound of those outputs. */
 dflash_status dflash_create(const dflash_config* cfg, const dflash_weights* w,
                             int device, dflash_handle** out);
 
@@ -176,6 +183,16 @@ size_t dflash_inject_workspace_bytes(const dflash_handle* h, int max_rows);
 size_t dflash_propose_workspace_bytes(const dflash_handle* h, int max_batch,
                                       int max_pages_per_seq);
 
+/* Diagnostics: byte offset, inside the workspace of a dflash_propose /
+ * dflash_propose_keys call with this B and max_pages_per_seq, of the rows that
+ * call hands to the LM head: [B * K, hidden] fp16, row b * K + i the
+ * final-RMSNormed hidden state of block slot 1 + i of request b
+ * (§"DFlashQwen3ForCausalLM": the kept rows of compute_draft_tokens).  Valid
+ * after the call until the workspace is reused, so that the LM head's greedy
+ * pick can be checked on exactly the rows it saw.  (size_t)-1 for a NULL
+ * handle or non-positive sizes. */
+size_t dflash_propose_final_rows_offset(const dflash_handle* h, int B, int max_pages_per_seq);
+
 /* Workspace needed by dflash_verify_greedy for [B, K+1, V] target logits. */
 size_t dflash_verify_workspace_bytes(int B, int K, int V);
 
@@ -194,8 +211,9 @@ size_t dflash_verify_workspace_bytes(int B, int K, int V);
  * library's device memory, present on every device that loads the library
  * until the process exits; the call allocates nothing.
  *   - The first call on a device looks up that array's device address (with
- *     the device current) and caches it; make that first call before any
- *     stream capture.
+ *     the device current) and caches it with the id of the device's current
+ *     context; make that first call before any stream capture.  After a device
+ *     reset (a new context) the next call looks the address up again.
  *   - Every call shares the one array and leaves its last contents behind.
  *     Calls that overlap on the GPU (e.g. on two streams at once) race on it
  *     and give wrong results; order them on one stream.
@@ -343,7 +361,8 @@ dflash_status dflash_finalize_draft_keys(const int64_t* draft_keys, const int32_
  *   out_tokens[b] = [drafts[b][0..n-1], t_n, -1, ..., -1]   ([B, K+1] int32)
  *   num_accepted[b] = n, bonus[b] = t_n                      ([B] int32 each)
  * drafts [B, K] int32; target_logits [B, K+1, V] fp32.  Bit-exact by construction.
- * B == 0 is a no-op.  Needs dflash_verify_workspace_bytes(B, K, V). */
+ * B == 0 is a no-op; B * (K + 1) > 2^30 rows is DFLASH_ERR_UNSUPPORTED_SHAPE.
+ * Needs dflash_verify_workspace_bytes(B, K, V). */
 dflash_status dflash_verify_greedy(const int32_t* drafts, const float* target_logits,
                                    int B, int K, int V, int32_t* out_tokens,
                                    int32_t* num_accepted, int32_t* bonus,
@@ -510,6 +529,107 @@ dflash_status dflash_plan_attention_info(int B, int n_kv_heads, int max_pages_pe
                                          int head_dim, int num_sms, int forced_ring, int flags,
                                          dflash_attention_plan* out);
 
+/* ---- a small causal target model on the device ---------------------------
+ *
+ * DFlash reads the target model's auxiliary hidden states (§"Target Auxiliary
+ * Hidden State Extraction"): the target captures the residual stream BEFORE
+ * the requested layers and returns the captured states concatenated, one
+ * [n, n_capture * hidden] tensor per forward, the input of
+ * dflash_inject_context.  The draft checkpoint's target_layer_ids name the
+ * state AFTER layer i (HuggingFace output hidden-state ids), so the runner
+ * asks the target for layer i + 1 (the page's "crucial off-by-one").
+ *
+ * dflash_target_* is a small Qwen3-style causal LM with that capture
+ * interface (the same layer as the draft's, with causal attention and an
+ * un-aliased final norm + LM head), so that the whole speculative loop —
+ * target forward, greedy verification, injection, proposal — runs on the
+ * device and can be checked against plain greedy decoding of the same target.
+ * It is built for exact reproducibility, not speed: fp32 weights and
+ * activations, and every output element reduced in one fixed order that does
+ * not depend on how many rows a call processes, so a token at a position gets
+ * bit-identical logits whether decoded alone or inside a block.  One sequence
+ * per instance; its K/V cache ([n_layers][max_len][n_kv_heads][head_dim] fp32)
+ * is owned by the instance. */
+
+/* capture_layers[i] = target_layer_ids[i] + 1 (host arrays of n entries); each
+ * id must lie in [0, target_n_layers - 1] (DFLASH_ERR_INVALID_ARG otherwise):
+ * capture layer target_n_layers is the last layer's output, before the final
+ * norm. */
+dflash_status dflash_aux_capture_layers(const int* target_layer_ids, int n, int target_n_layers,
+                                        int* capture_layers);
+
+typedef struct dflash_target_config {
+  int hidden;
+  int n_layers;
+  int n_q_heads;
+  int n_kv_heads;
+  int head_dim;                /* a multiple of 32, <= 128 */
+  int intermediate;
+  int vocab;
+  float rms_eps;
+  float rope_theta;
+  int max_len;                 /* the sequence's positions [0, max_len) */
+  int n_capture;               /* captured states per row (may be 0) */
+  const int* capture_layers;   /* HOST [n_capture]: pre-layer index in [0, n_layers] */
+} dflash_target_config;
+
+/* DEVICE pointers, fp32, row-major [out, in]; per-layer entries are HOST arrays
+ * of n_layers device pointers; all used in place except wq|wk|wv and
+ * w_gate|w_up, which the instance stacks into copies of its own.
+ *   embed, lm_head [vocab, hidden]; final_norm_w, in_norm_w, post_norm_w [hidden];
+ *   wq [Hq*d, hidden]; wk, wv [Hkv*d, hidden]; wo [hidden, Hq*d];
+ *   q_norm_w, k_norm_w [d]; w_gate, w_up [I, hidden]; w_down [hidden, I] */
+typedef struct dflash_target_weights {
+  const float* embed;
+  const float* final_norm_w;
+  const float* lm_head;
+  const float* const* in_norm_w;
+  const float* const* post_norm_w;
+  const float* const* wq;
+  const float* const* wk;
+  const float* const* wv;
+  const float* const* wo;
+  const float* const* q_norm_w;
+  const float* const* k_norm_w;
+  const float* const* w_gate;
+  const float* const* w_up;
+  const float* const* w_down;
+} dflash_target_weights;
+
+typedef struct dflash_target dflash_target;
+
+/* Allocates the instance (weight copies, K/V cache, error word) on `device`
+ * and synchronizes it.  DFLASH_ERR_INVALID_ARG for missing pointers or sizes,
+ * a capture layer outside [0, n_layers]; DFLASH_ERR_UNSUPPORTED_SHAPE for a
+ * head_dim that is not a multiple of 32 up to 128, or n_q_heads not a multiple
+ * of n_kv_heads. */
+dflash_status dflash_target_create(const dflash_target_config* cfg,
+                                   const dflash_target_weights* w, int device,
+                                   dflash_target** out);
+void dflash_target_destroy(dflash_target* t);
+size_t dflash_target_workspace_bytes(const dflash_target* t, int n);
+
+/* Forward of tokens[0..n) (DEVICE int32) at positions [start_pos, start_pos + n)
+ * of the instance's sequence: writes their K/V into the cache, attends
+ * causally over [0, position], and writes
+ *   logits [n, vocab] fp32 (DEVICE): the prediction after each token;
+ *   aux [n, n_capture * hidden] bf16 (DEVICE; may be NULL when n_capture == 0):
+ *     row r, slot k = the residual state of token r before layer
+ *     capture_layers[k] (the embedding for 0, the last layer's output for
+ *     n_layers).
+ * Positions at or past start_pos + n of the cache are untouched (stale rows of
+ * rejected tokens are overwritten by the next forward that covers them).
+ * Host errors: start_pos < 0 or start_pos + n > max_len, missing pointers
+ * (DFLASH_ERR_INVALID_ARG), a workspace below dflash_target_workspace_bytes
+ * (DFLASH_ERR_WORKSPACE).  A token outside [0, vocab) embeds as zeros and sets
+ * DFLASH_DEVERR_TOKEN (dflash_target_check_device_errors). */
+dflash_status dflash_target_forward(dflash_target* t, const int32_t* tokens, int n, int start_pos,
+                                    float* logits, void* aux, void* workspace,
+                                    size_t workspace_bytes, void* stream);
+
+/* Synchronizes the device, reads and clears the instance's device error word. */
+dflash_status dflash_target_check_device_errors(dflash_target* t, unsigned* bits);
+
 /* ---- launch accounting and per-launch timing (diagnostics) ---- */
 
 /* Kernel families launched by the calls above (ids for dflash_profile_read). */
@@ -555,6 +675,23 @@ dflash_status dflash_profile_disable(dflash_handle* h);
  * raw DFLASH_DEVERR_* mask.  (verify and paged_slots take no handle and have
  * no device-detected error conditions.) */
 dflash_status dflash_check_device_errors(dflash_handle* h, unsigned* bits);
+
+/* Diagnostics.  Every bounded wait of the library's kernels (pipeline
+ * barriers, cross-CTA arrival counters) gives up after `cycles` SM clock
+ * cycles on `device`, sets DFLASH_DEVERR_TIMEOUT and lets its kernel wind down
+ * (default 4e9 cycles, about 2 s).  One value per device for the whole
+ * process; set it only while no kernel of the library runs on the device
+ * (the call synchronizes with the device).  DFLASH_ERR_INVALID_ARG for
+ * cycles <= 0. */
+dflash_status dflash_set_wait_limit(int device, long long cycles);
+
+/* Diagnostics: enqueues one kernel on `stream` whose single bounded wait can
+ * never complete (an mbarrier that nothing arrives on), so that it runs out
+ * after the device's wait limit and sets DFLASH_DEVERR_TIMEOUT in the handle's
+ * error word; dflash_check_device_errors then returns
+ * DFLASH_ERR_DEVICE_TIMEOUT.  Nothing faults or traps and the context stays
+ * usable; the handle's next calls run normally once the bit is read. */
+dflash_status dflash_selftest_wait_timeout(dflash_handle* h, void* stream);
 
 /* Static, human-readable name of a status code. */
 const char* dflash_status_string(dflash_status s);

@@ -35,3 +35,23 @@ def rel_l2(a, b) -> float:
     a = np.asarray(a, dtype=np.float64)
     b = np.asarray(b, dtype=np.float64)
     return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
+
+
+# ----------------------------------------------------------------------------
+# parity bookkeeping: rows whose greedy pick is a near-tie are excluded from the
+# bit-exact comparison; every exclusion is recorded and summarised at the end
+# of the pytest run (tests/conftest.py), and written as JSON lines to the file
+# named by DFLASH_PARITY_RECORD when that variable is set.
+# ----------------------------------------------------------------------------
+PARITY_LOG: list = []
+
+
+def record_parity(name: str, **fields) -> None:
+    import json
+    import os
+    entry = dict(name=name, **fields)
+    PARITY_LOG.append(entry)
+    path = os.environ.get("DFLASH_PARITY_RECORD")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps(entry) + "\n")

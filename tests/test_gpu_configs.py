@@ -18,7 +18,7 @@ import oracle as O
 from block_diffusion_speculative_propose_b200 import (DFlash, paged_slots, synth,
                                                       verify_greedy)
 from tests._util import rel_l2, to_np, weights_np, weights_to
-from tests.test_gpu_propose import compare_drafts, max_excluded
+from tests.test_gpu_propose import check_lm_head_stage, compare_drafts, max_excluded
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
@@ -71,13 +71,23 @@ def test_full_step_at_bench_size(workload, samples):
         out_tok, n_acc, new_bonus = verify_greedy(dv["prev_drafts"], dv["target_logits"])
         slots = paged_slots(dv["inject_positions"], dv["inject_req_ids"], dv["block_table"], P)
         h.inject_context(dv["aux"], dv["inject_positions"], slots, kc, vc)
-        logits = torch.empty(B * K, V, dtype=torch.float32, device=DEV)
+        Wpages = int(sb.block_table.shape[1])
+        ws = torch.empty(h.propose_workspace_bytes(B, Wpages), dtype=torch.uint8, device=DEV)
         drafts = h.propose(dv["bonus"], dv["seq_lens"], dv["block_table"], kc, vc,
-                           logits_out=logits)
+                           workspace=ws)
         torch.cuda.synchronize()
         assert h.check_device_errors() == 0
-        # same step without the debug logits gives the same drafts
-        drafts2 = h.propose(dv["bonus"], dv["seq_lens"], dv["block_table"], kc, vc)
+        # the LM head's greedy pick on the rows it saw, stage-isolated: every
+        # sampled request's rows plus random rows of the whole batch
+        Wn = weights_np(Wt)
+        lm_rows = sorted({*np.concatenate([np.arange(b * K, (b + 1) * K) for b in pick]).tolist(),
+                          *rng.choice(B * K, min(B * K, 64), replace=False).tolist()})
+        check_lm_head_stage(h, ws, B, Wpages, to_np(drafts), Wn, lm_rows,
+                            f"{workload} lm-head")
+        # the same step with the debug logits gives the same drafts
+        logits = torch.empty(B * K, V, dtype=torch.float32, device=DEV)
+        drafts2 = h.propose(dv["bonus"], dv["seq_lens"], dv["block_table"], kc, vc,
+                            logits_out=logits)
         torch.cuda.synchronize()
         assert torch.equal(drafts, drafts2)
 
@@ -110,7 +120,6 @@ def test_full_step_at_bench_size(workload, samples):
         local_req = np.searchsorted(np.array(pick), req[sel])
         local_slots = O.paged_slots(pos, local_req, table, P)
         aux = to_np(sb.aux)[sel].astype(np.float64)
-        Wn = weights_np(Wt)
         del Wt
         res = {}
         for mode in ("device", "exact"):
@@ -118,7 +127,8 @@ def test_full_step_at_bench_size(workload, samples):
             vo = [v.astype(np.float64) for v in v_pre]
             O.inject_context(oc, Wn, aux, pos, local_slots, ko, vo, mode)
             res[mode] = O.propose(oc, Wn, to_np(sb.bonus)[pick], seq[pick], table, ko, vo, mode)
-        excluded = compare_drafts(gpu_drafts, gpu_logits, res["device"], res["exact"], K)
+        excluded = compare_drafts(gpu_drafts, gpu_logits, res["device"], res["exact"], K,
+                                  name=f"{workload} chain")
         assert excluded <= max_excluded(len(pick) * K)
     finally:
         h.close()

@@ -122,7 +122,8 @@ def check_step(case, out, ver, pi, prop):
     np.testing.assert_array_equal(to_np(out["slot_mapping"]), pi.slot_mapping)
     np.testing.assert_array_equal(to_np(out["seq_lens"]), pi.seq_lens)
     np.testing.assert_array_equal(to_np(out["bonus"]), pi.bonus)
-    excluded = compare_drafts(to_np(out["draft_tokens"]), None, prop, None, case.K)
+    excluded = compare_drafts(to_np(out["draft_tokens"]), None, prop, None, case.K,
+                              name=f"spec step chain B={case.B}")
     assert excluded <= max_excluded(case.B * case.K)
     blk = to_np(out["block_tokens"])
     np.testing.assert_array_equal(blk[:, 0], pi.bonus)

@@ -63,7 +63,7 @@ def run_shards(cfg, Wt, ctx_lens, parts_list, seed):
             gd, fd = to_np(d).reshape(-1), d_full.reshape(-1)
             assert np.array_equal(gd[same], fd[same])
             excluded = compare_drafts(to_np(d), to_np(torch.cat(logits, dim=1)), prop_io,
-                                      ch.oracle("exact"), K)
+                                      ch.oracle("exact"), K, name=f"vocab-parallel chain x{parts}")
             assert excluded <= max_excluded(ch.B * K)
             assert np.array_equal(to_np(blk)[:, 0], to_np(ch.bonus))
             assert np.array_equal(to_np(blk)[:, 1:], to_np(d))
