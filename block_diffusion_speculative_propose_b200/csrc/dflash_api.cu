@@ -18,6 +18,7 @@
 
 #include "attention.cuh"
 #include "attention_tc.cuh"
+#include "attention_tc2.cuh"
 #include "dflash.h"
 #include "gemm_tcgen05.cuh"
 #include "small_kernels.cuh"
@@ -212,13 +213,15 @@ struct AttnPlan {
   int st = 2;        // tcgen05 kernel: K/V ring depth (64-key tiles: 2 -> two CTAs per SM)
   bool persist = false;  // six-deep ring: persistent CTAs (one per SM) walk the items
   bool cluster = false;  // tcgen05 kernel, splits of a (request, kv head) combined in a cluster
+  bool tc2 = false;      // head_dim 128: two CTAs per SM, P V transposed (attention_tc2.cuh)
   size_t part_o_bytes = 0, part_ml_bytes = 0;
 };
 
 // forced_ring: K/V ring depth of the 64-key tcgen05 kernel (2 or 6), or 0 to
 // let the planner decide; persist: the six-deep ring as persistent CTAs.
 AttnPlan plan_attention(int B, int Hkv, int W, int P, int bs, int G, int D, int num_sms,
-                        bool allow_cluster, int forced_ring, bool persist = false) {
+                        bool allow_cluster, int forced_ring, bool persist = false,
+                        int tc2_keys = 64) {
   AttnPlan a;
   const int keys_max = W * P;
   const double est = static_cast<double>(B) * Hkv * keys_max;
@@ -240,6 +243,21 @@ AttnPlan plan_attention(int B, int Hkv, int W, int P, int bs, int G, int D, int 
   a.st = (chunk / kTcKeysSmall >= 2 * kTcDeepStages) ? kTcDeepStages : kTcStages;
   if (forced_ring == kTcStages || forced_ring == kTcDeepStages) a.st = forced_ring;
   a.persist = persist && a.tc && a.st == kTcDeepStages;
+  // head_dim 128 (every configuration of the pages' models): unless a ring
+  // depth, the persistent or the cluster variant is asked for, the kernel
+  // with two CTAs per SM and P V transposed; its splits are sized for 8
+  // CTAs per SM (two resident at a time) so that mixed context lengths
+  // balance over several waves
+  if (a.tc && D == 128 && forced_ring == 0 && !persist && !allow_cluster) {
+    a.tc2 = true;
+    a.kt = tc2_keys;
+    a.st = tc2_keys == 64 ? Tc2Cfg<64>::ST : Tc2Cfg<32>::ST;
+    chunk = static_cast<int>(std::ceil(est / (8.0 * num_sms)));
+    chunk = (chunk + tile - 1) / tile * tile;
+    chunk = std::max(128, std::min(8192, chunk));
+    a.chunk_keys = chunk;
+    a.max_splits = cdiv(keys_max, chunk);
+  }
   a.row_groups = cdiv(a.R, 16);
   a.key_parts = 1;
   while (a.key_parts < 4 && a.row_groups * a.key_parts * 2 <= kAttnMaxComputeWarps)
@@ -314,6 +332,9 @@ struct dflash_handle {
   // vocabulary shard of the LM head (tensor-parallel proposal); the whole
   // vocabulary unless created by dflash_create_vocab_shard
   int vocab_start = 0, vocab_count = 0;
+  // tensor-parallel shard (dflash_create_tp_shard): rank and group size; the
+  // cfg above then holds this shard's head and MLP-feature counts
+  int tp_rank = 0, tp_size = 1;
   bf16* knorm_all = nullptr;  // [L, D]
   float2* rope = nullptr;   // [max_position, D/2]
   unsigned* dev_err = nullptr;
@@ -357,6 +378,13 @@ struct dflash_handle {
   bool attn_persist = [] {
     const char* e = std::getenv("DFLASH_ATTN_PERSIST");
     return e && e[0] == '1';
+  }();
+  // keys per tile of the two-CTA-per-SM head_dim-128 kernel (DFLASH_ATTN_TILE
+  // = 32 or 64 when the handle is created; 64 otherwise: measured at 128
+  // requests x 8k-32k keys, 64-key tiles stream 4.2 TB/s, 32-key ones 3.7)
+  int attn_tile = [] {
+    const char* e = std::getenv("DFLASH_ATTN_TILE");
+    return (e && std::atoi(e) == 32) ? 32 : 64;
   }();
   std::vector<cudaEvent_t> prof_events;
   size_t prof_next = 0;
@@ -727,6 +755,16 @@ cudaError_t set_attn_attrs() {
                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 TcAttnCfg<D, kTcKeysSmall, kTcDeepStages>::kSmem)) != cudaSuccess)
     return e;
+  if constexpr (D == 128) {
+    if ((e = cudaFuncSetAttribute(attn_block_tc2_kernel<64>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  Tc2Cfg<64>::kSmem)) != cudaSuccess)
+      return e;
+    if ((e = cudaFuncSetAttribute(attn_block_tc2_kernel<32>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  Tc2Cfg<32>::kSmem)) != cudaSuccess)
+      return e;
+  }
   if ((e = cudaFuncSetAttribute(attn_block_tc_persistent_kernel<D, kTcDeepStages>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 TcAttnCfg<D, kTcKeysSmall, kTcDeepStages>::kSmem)) != cudaSuccess)
@@ -751,7 +789,17 @@ dflash_status run_attention(dflash_handle* h, const AttnPlan& ap, AttnParams prm
   prm.row_groups = ap.row_groups;
   prm.key_parts = ap.key_parts;
   prm.cluster = ap.cluster ? 1 : 0;
-  if (ap.tc) {
+  if (ap.tc2) {
+    LaunchScope scope(h, DFLASH_KERNEL_ATTENTION, st);
+    if constexpr (D == 128) {
+      if (ap.kt == 64)
+        launch_k(h->pdl, attn_block_tc2_kernel<64>, grid, dim3(kTcThreads), Tc2Cfg<64>::kSmem,
+                 st, tk, tv, prm);
+      else
+        launch_k(h->pdl, attn_block_tc2_kernel<32>, grid, dim3(kTcThreads), Tc2Cfg<32>::kSmem,
+                 st, tk, tv, prm);
+    }
+  } else if (ap.tc) {
     LaunchScope scope(h, DFLASH_KERNEL_ATTENTION, st);
     if (ap.kt == kTcKeysSmall && ap.persist) {
       const int items = ap.max_splits * c.n_kv_heads * prm.B;
@@ -809,7 +857,7 @@ InjectWs inject_layout(const dflash_handle* h, int n) {
 
 struct ProposeWs {
   size_t x = 0, nrm = 0, q = 0, o = 0, hm = 0, frows = 0, keys = 0, part_o = 0, part_ml = 0,
-         partial = 0, total = 0, partial_cap = 0, part_o_cap = 0, part_ml_cap = 0;
+         partial = 0, total = 0, partial_cap = 0, part_o_cap = 0, part_ml_cap = 0, xpart = 0;
 };
 size_t propose_partial_need(const dflash_handle* h, int B) {
   return gemm_partial_bound(B * h->cfg.block_size, h->num_sms);
@@ -837,7 +885,7 @@ ProposeWs propose_layout(const dflash_handle* h, int B, int W) {
   for (int bb = 1; bb <= B; ++bb) {
     const AttnPlan ap = plan_attention(bb, Hkv, W, c.page_size, bs, Hq / Hkv, D, h->num_sms,
                                        h->attn_cluster, h->attn_ring,
-                                     h->attn_persist);
+                                     h->attn_persist, h->attn_tile);
     po = std::max(po, ap.part_o_bytes);
     pm = std::max(pm, ap.part_ml_bytes);
   }
@@ -848,6 +896,9 @@ ProposeWs propose_layout(const dflash_handle* h, int B, int W) {
   w.part_ml_cap = pm;
   w.partial = take(pc);
   w.partial_cap = pc;
+  // tensor-parallel shard: this rank's partial sums of the O / down
+  // projections, all-reduced in place by the caller's exchange hook
+  if (h->tp_size > 1) w.xpart = take(static_cast<size_t>(M) * H * 4);
   w.total = off;
   return w;
 }
@@ -920,7 +971,7 @@ template <int D>
 dflash_status propose_layers(dflash_handle* h, const ProposeWs& lw, void* ws,
                              const int32_t* seq_lens, const int32_t* block_table, int B, int W,
                              void* const* k_cache, void* const* v_cache, int num_pages,
-                             cudaStream_t st) {
+                             cudaStream_t st, dflash_allreduce_fn exchange, void* user) {
   const dflash_config& c = h->cfg;
   const int bs = c.block_size, M = B * bs, H = c.hidden, Hq = c.n_q_heads, Hkv = c.n_kv_heads,
             I = c.intermediate, K = bs - 1;
@@ -933,7 +984,7 @@ dflash_status propose_layers(dflash_handle* h, const ProposeWs& lw, void* ws,
   float* partial = at<float>(ws, lw.partial);
   const AttnPlan ap = plan_attention(B, Hkv, W, c.page_size, bs, Hq / Hkv, D, h->num_sms,
                                      h->attn_cluster, h->attn_ring,
-                                     h->attn_persist);
+                                     h->attn_persist, h->attn_tile);
   if (ap.part_o_bytes > lw.part_o_cap || ap.part_ml_bytes > lw.part_ml_cap)
     return DFLASH_ERR_WORKSPACE;
   AttnParams prm;
@@ -982,6 +1033,41 @@ dflash_status propose_layers(dflash_handle* h, const ProposeWs& lw, void* ws,
     // non-causal block attention over context + block
     s = run_attention<D>(h, ap, prm, k_cache[l], v_cache[l], num_pages, st);
     if (s != DFLASH_OK) return s;
+    if (h->tp_size > 1) {
+      // tensor-parallel shard: Wo and W_down are row-parallel, so this rank
+      // forms partial sums of both projections over its heads / features;
+      // the caller's hook sums them over the ranks (an all-reduce) before
+      // each residual add
+      float* xpart = at<float>(ws, lw.xpart);
+      EpiStoreF32 es{xpart, H};
+      s = run_gemm(h, DFLASH_KERNEL_GEMM_O, true, true, o, M, Hq * D, h->wo[l], H, es, partial,
+                   lw.partial_cap, st);
+      if (s != DFLASH_OK) return s;
+      if (exchange(xpart, static_cast<size_t>(M) * H, st, user) != 0) return DFLASH_ERR_EXCHANGE;
+      {
+        LaunchScope scope(h, DFLASH_KERNEL_RMSNORM, st);
+        launch_k(h->pdl, add_rmsnorm_rows_kernel, dim3(M), dim3(256), 0, st, x,
+                 static_cast<const float*>(xpart), h->post_norm_w[l], nrm, H, c.rms_eps, 0, bs);
+      }
+      if (cudaGetLastError() != cudaSuccess) return DFLASH_ERR_CUDA;
+      EpiSwiGLU eg{hm, I};
+      s = run_gemm(h, DFLASH_KERNEL_GEMM_GATE_UP, true, true, nrm, M, H, h->wgu[l], 2 * I, eg,
+                   partial, lw.partial_cap, st);
+      if (s != DFLASH_OK) return s;
+      s = run_gemm(h, DFLASH_KERNEL_GEMM_DOWN, false, true, hm, M, I, h->wdown[l], H, es,
+                   partial, lw.partial_cap, st);
+      if (s != DFLASH_OK) return s;
+      if (exchange(xpart, static_cast<size_t>(M) * H, st, user) != 0) return DFLASH_ERR_EXCHANGE;
+      LaunchScope scope(h, DFLASH_KERNEL_RMSNORM, st);
+      if (l + 1 < c.n_layers)
+        launch_k(h->pdl, add_rmsnorm_rows_kernel, dim3(M), dim3(256), 0, st, x,
+                 static_cast<const float*>(xpart), h->in_norm_w[l + 1], nrm, H, c.rms_eps, 0, bs);
+      else
+        launch_k(h->pdl, add_rmsnorm_rows_kernel, dim3(B * K), dim3(256), 0, st, x,
+                 static_cast<const float*>(xpart), h->final_norm_w, frows, H, c.rms_eps, K, bs);
+      if (cudaGetLastError() != cudaSuccess) return DFLASH_ERR_CUDA;
+      continue;
+    }
     // x += Wo o
     EpiResidAdd er{x, H};
     s = run_gemm(h, DFLASH_KERNEL_GEMM_O, true, true, o, M, Hq * D, h->wo[l], H, er, partial,
@@ -1025,6 +1111,12 @@ dflash_status propose_layers(dflash_handle* h, const ProposeWs& lw, void* ws,
 // ===========================================================================
 // C ABI
 // ===========================================================================
+namespace {
+dflash_status create_handle(const dflash_config* cfg, const dflash_weights* w, int device,
+                            int vocab_start, int vocab_count, int tp_rank, int tp_size,
+                            dflash_handle** out);
+}  // namespace
+
 extern "C" {
 
 const char* dflash_status_string(dflash_status s) {
@@ -1038,6 +1130,7 @@ const char* dflash_status_string(dflash_status s) {
     case DFLASH_ERR_UNIMPLEMENTED: return "DFLASH_ERR_UNIMPLEMENTED";
     case DFLASH_ERR_DEVICE_TIMEOUT: return "DFLASH_ERR_DEVICE_TIMEOUT";
     case DFLASH_ERR_RANGE: return "DFLASH_ERR_RANGE";
+    case DFLASH_ERR_EXCHANGE: return "DFLASH_ERR_EXCHANGE";
   }
   return "DFLASH_ERR_UNKNOWN";
 }
@@ -1066,6 +1159,29 @@ dflash_status dflash_create(const dflash_config* cfg, const dflash_weights* w, i
 dflash_status dflash_create_vocab_shard(const dflash_config* cfg, const dflash_weights* w,
                                         int device, int vocab_start, int vocab_count,
                                         dflash_handle** out) {
+  return create_handle(cfg, w, device, vocab_start, vocab_count, 0, 1, out);
+}
+
+dflash_status dflash_create_tp_shard(const dflash_config* cfg, const dflash_weights* w,
+                                     int device, int tp_rank, int tp_size, int vocab_start,
+                                     int vocab_count, dflash_handle** out) {
+  if (tp_size < 1 || tp_rank < 0 || tp_rank >= tp_size) {
+    if (out) *out = nullptr;
+    return DFLASH_ERR_INVALID_ARG;
+  }
+  return create_handle(cfg, w, device, vocab_start, vocab_count, tp_rank, tp_size, out);
+}
+
+}  // extern "C"
+
+namespace {
+// A handle over the whole model (tp_size 1) or over tensor-parallel rank
+// tp_rank's slice of it: kv heads [r Hkv/S, (r+1) Hkv/S) with their query
+// heads, MLP features [r I/S, (r+1) I/S), the matching columns of Wo and
+// W_down, and the LM-head vocabulary rows [vocab_start, + vocab_count).
+dflash_status create_handle(const dflash_config* cfg, const dflash_weights* w, int device,
+                            int vocab_start, int vocab_count, int tp_rank, int tp_size,
+                            dflash_handle** out) {
   if (!out) return DFLASH_ERR_INVALID_ARG;
   *out = nullptr;
   if (!cfg || !w) return DFLASH_ERR_INVALID_ARG;
@@ -1085,6 +1201,9 @@ dflash_status dflash_create_vocab_shard(const dflash_config* cfg, const dflash_w
       c.block_size > 64 || c.n_layers > kMaxLayers)
     return DFLASH_ERR_UNSUPPORTED_SHAPE;
   if (c.block_size * (c.n_q_heads / c.n_kv_heads) > 16 * kAttnMaxComputeWarps)
+    return DFLASH_ERR_UNSUPPORTED_SHAPE;
+  // tensor-parallel slices: whole kv groups per rank, MLP features in 64s
+  if (c.n_kv_heads % tp_size || c.intermediate % (64 * tp_size))
     return DFLASH_ERR_UNSUPPORTED_SHAPE;
   const int L = c.n_layers;
   if (!w->fc_w || !w->hidden_norm_w || !w->embed || !w->lm_head || !w->final_norm_w ||
@@ -1113,6 +1232,12 @@ dflash_status dflash_create_vocab_shard(const dflash_config* cfg, const dflash_w
   dflash_handle* h = new (std::nothrow) dflash_handle();
   if (!h) return DFLASH_ERR_CUDA;
   h->cfg = c;
+  // a shard's geometry is its slice of the heads and MLP features
+  h->cfg.n_q_heads = c.n_q_heads / tp_size;
+  h->cfg.n_kv_heads = c.n_kv_heads / tp_size;
+  h->cfg.intermediate = c.intermediate / tp_size;
+  h->tp_rank = tp_rank;
+  h->tp_size = tp_size;
   h->vocab_start = vocab_start;
   h->vocab_count = vocab_count;
   if (c.target_layer_ids) h->target_layer_ids.assign(c.target_layer_ids, c.target_layer_ids + c.n_target_layers);
@@ -1129,8 +1254,16 @@ dflash_status dflash_create_vocab_shard(const dflash_config* cfg, const dflash_w
   cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, device);
   if (major != 10) return fail(DFLASH_ERR_UNSUPPORTED_SHAPE);
 
-  const int H = c.hidden, D = c.head_dim, Hq = c.n_q_heads, Hkv = c.n_kv_heads,
-            I = c.intermediate;
+  // local (this shard's) sizes, and where its slices start in the whole weights
+  const int H = c.hidden, D = c.head_dim, Hq = h->cfg.n_q_heads, Hkv = h->cfg.n_kv_heads,
+            I = h->cfg.intermediate;
+  const int Hq_all = c.n_q_heads, I_all = c.intermediate;
+  auto rows_at = [](const void* base, size_t row, size_t row_len) {
+    return static_cast<const void*>(static_cast<const uint16_t*>(base) + row * row_len);
+  };
+  const size_t q_row0 = static_cast<size_t>(tp_rank) * Hq * D;     // wq rows, wo columns
+  const size_t kv_row0 = static_cast<size_t>(tp_rank) * Hkv * D;   // wk / wv rows
+  const size_t f_row0 = static_cast<size_t>(tp_rank) * I;          // gate/up rows, down columns
   h->hidden_norm_w = static_cast<const bf16*>(w->hidden_norm_w);
   h->embed = static_cast<const bf16*>(w->embed);
   h->final_norm_w = static_cast<const bf16*>(w->final_norm_w);
@@ -1156,12 +1289,12 @@ dflash_status dflash_create_vocab_shard(const dflash_config* cfg, const dflash_w
     if (cudaMalloc(&p, static_cast<size_t>(Hq + 2 * Hkv) * D * rowb) != cudaSuccess)
       return fail_st(DFLASH_ERR_CUDA);
     h->wqkv.push_back(p);
-    if (cudaMemcpyAsync(p, w->wq[l], static_cast<size_t>(Hq) * D * rowb,
+    if (cudaMemcpyAsync(p, rows_at(w->wq[l], q_row0, H), static_cast<size_t>(Hq) * D * rowb,
                         cudaMemcpyDeviceToDevice, st) != cudaSuccess ||
-        cudaMemcpyAsync(p + static_cast<size_t>(Hq) * D * H, w->wk[l],
+        cudaMemcpyAsync(p + static_cast<size_t>(Hq) * D * H, rows_at(w->wk[l], kv_row0, H),
                         static_cast<size_t>(Hkv) * D * rowb, cudaMemcpyDeviceToDevice,
                         st) != cudaSuccess ||
-        cudaMemcpyAsync(p + static_cast<size_t>(Hq + Hkv) * D * H, w->wv[l],
+        cudaMemcpyAsync(p + static_cast<size_t>(Hq + Hkv) * D * H, rows_at(w->wv[l], kv_row0, H),
                         static_cast<size_t>(Hkv) * D * rowb, cudaMemcpyDeviceToDevice,
                         st) != cudaSuccess)
       return fail_st(DFLASH_ERR_CUDA);
@@ -1172,10 +1305,11 @@ dflash_status dflash_create_vocab_shard(const dflash_config* cfg, const dflash_w
     if (cudaMalloc(&p, static_cast<size_t>(2 * I) * rowb) != cudaSuccess)
       return fail_st(DFLASH_ERR_CUDA);
     h->wgu.push_back(p);
-    if (cudaMemcpy2DAsync(p, 32 * rowb, w->w_gate[l], 16 * rowb, 16 * rowb, I / 16,
-                          cudaMemcpyDeviceToDevice, st) != cudaSuccess ||
-        cudaMemcpy2DAsync(p + 16 * static_cast<size_t>(H), 32 * rowb, w->w_up[l], 16 * rowb,
-                          16 * rowb, I / 16, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    if (cudaMemcpy2DAsync(p, 32 * rowb, rows_at(w->w_gate[l], f_row0, H), 16 * rowb, 16 * rowb,
+                          I / 16, cudaMemcpyDeviceToDevice, st) != cudaSuccess ||
+        cudaMemcpy2DAsync(p + 16 * static_cast<size_t>(H), 32 * rowb,
+                          rows_at(w->w_up[l], f_row0, H), 16 * rowb, 16 * rowb, I / 16,
+                          cudaMemcpyDeviceToDevice, st) != cudaSuccess)
       return fail_st(DFLASH_ERR_CUDA);
   }
   // all layers' K/V projections stacked: per layer [wk; wv]
@@ -1183,10 +1317,10 @@ dflash_status dflash_create_vocab_shard(const dflash_config* cfg, const dflash_w
   if (cudaMalloc(&h->wkv, static_cast<size_t>(L) * 2 * kvrows * rowb) != cudaSuccess)
     return fail_st(DFLASH_ERR_CUDA);
   for (int l = 0; l < L; ++l) {
-    if (cudaMemcpyAsync(h->wkv + (2 * l) * kvrows * H, w->wk[l], kvrows * rowb,
-                        cudaMemcpyDeviceToDevice, st) != cudaSuccess ||
-        cudaMemcpyAsync(h->wkv + (2 * l + 1) * kvrows * H, w->wv[l], kvrows * rowb,
-                        cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    if (cudaMemcpyAsync(h->wkv + (2 * l) * kvrows * H, rows_at(w->wk[l], kv_row0, H),
+                        kvrows * rowb, cudaMemcpyDeviceToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(h->wkv + (2 * l + 1) * kvrows * H, rows_at(w->wv[l], kv_row0, H),
+                        kvrows * rowb, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
       return fail_st(DFLASH_ERR_CUDA);
   }
   if (cudaMalloc(&h->knorm_all, static_cast<size_t>(L) * D * 2) != cudaSuccess)
@@ -1201,8 +1335,10 @@ dflash_status dflash_create_vocab_shard(const dflash_config* cfg, const dflash_w
     if (cudaMalloc(&p, static_cast<size_t>(H) * Hq * D * 2) != cudaSuccess)
       return fail_st(DFLASH_ERR_CUDA);
     h->wo.push_back(p);
-    if (cudaMemcpyAsync(p, w->wo[l], static_cast<size_t>(H) * Hq * D * 2,
-                        cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    // this shard's columns of Wo [H, Hq_all * D] (all of them for one shard)
+    if (cudaMemcpy2DAsync(p, static_cast<size_t>(Hq) * D * 2, rows_at(w->wo[l], q_row0, 1),
+                          static_cast<size_t>(Hq_all) * D * 2, static_cast<size_t>(Hq) * D * 2, H,
+                          cudaMemcpyDeviceToDevice, st) != cudaSuccess)
       return fail_st(DFLASH_ERR_CUDA);
   }
   if (cudaMalloc(&h->lm_head16, static_cast<size_t>(vocab_count) * rowb) != cudaSuccess ||
@@ -1242,14 +1378,15 @@ dflash_status dflash_create_vocab_shard(const dflash_config* cfg, const dflash_w
   // every GEMM weight into the tile-contiguous layout
   {
     // packs row-major [N, K] `src` into a new buffer stored at *out
-    auto pack = [&](const void* src, int N, int K, void** out) {
+    auto pack = [&](const void* src, int N, int K, void** out, int ld = 0) {
       const size_t bytes = static_cast<size_t>(cdiv(N, kPackRows)) * kPackRows * K * 2;
       if (cudaMalloc(out, bytes) != cudaSuccess) {
         *out = nullptr;
         return false;
       }
       pack_tiles_kernel<<<1184, 256, 0, st>>>(static_cast<const uint16_t*>(src),
-                                              static_cast<uint16_t*>(*out), N, K, bytes / 16, 0);
+                                              static_cast<uint16_t*>(*out), N, K, ld ? ld : K,
+                                              bytes / 16, 0);
       return cudaGetLastError() == cudaSuccess;
     };
     // replaces a row-major copy owned by the handle with its packed form
@@ -1273,7 +1410,7 @@ dflash_status dflash_create_vocab_shard(const dflash_config* cfg, const dflash_w
     ok = ok && repack(h->lm_head16, vocab_count, H);
     for (int l = 0; ok && l < L; ++l) {
       void* p = nullptr;
-      ok = pack(w->w_down[l], H, I, &p);
+      ok = pack(rows_at(w->w_down[l], f_row0, 1), H, I, &p, I_all);
       if (p) h->wdown.push_back(static_cast<bf16*>(p));
     }
     if (ok) {
@@ -1331,6 +1468,9 @@ dflash_status dflash_create_vocab_shard(const dflash_config* cfg, const dflash_w
   *out = h;
   return DFLASH_OK;
 }
+}  // namespace
+
+extern "C" {
 
 void dflash_destroy(dflash_handle* h) {
   if (!h) return;
@@ -1489,8 +1629,12 @@ dflash_status propose_impl(dflash_handle* h, const int32_t* bonus_tokens,
                            int max_pages_per_seq, void* const* k_cache, void* const* v_cache,
                            int num_pages, int32_t* draft_tokens, int32_t* block_tokens,
                            int64_t* draft_keys, float* logits_out, void* workspace,
-                           size_t workspace_bytes, void* stream) {
+                           size_t workspace_bytes, void* stream,
+                           dflash_allreduce_fn exchange = nullptr, void* user = nullptr) {
   if (!h || B < 0) return DFLASH_ERR_INVALID_ARG;
+  // a tensor-parallel shard proposes only through dflash_propose_tp (with an
+  // exchange hook), and only a shard takes one
+  if ((h->tp_size > 1) != (exchange != nullptr)) return DFLASH_ERR_INVALID_ARG;
   if (B == 0) return DFLASH_OK;
   const dflash_config& c = h->cfg;
   if (!bonus_tokens || !seq_lens || !block_table || max_pages_per_seq <= 0 || !k_cache ||
@@ -1520,9 +1664,11 @@ dflash_status propose_impl(dflash_handle* h, const int32_t* bonus_tokens,
   if (cudaGetLastError() != cudaSuccess) return DFLASH_ERR_CUDA;
   dflash_status s = (c.head_dim == 128)
                         ? propose_layers<128>(h, lw, workspace, seq_lens, block_table, B,
-                                              max_pages_per_seq, k_cache, v_cache, num_pages, st)
+                                              max_pages_per_seq, k_cache, v_cache, num_pages, st,
+                                              exchange, user)
                         : propose_layers<64>(h, lw, workspace, seq_lens, block_table, B,
-                                             max_pages_per_seq, k_cache, v_cache, num_pages, st);
+                                             max_pages_per_seq, k_cache, v_cache, num_pages, st,
+                                             exchange, user);
   if (s != DFLASH_OK) return s;
   // aliased target LM head (this handle's vocabulary rows) with the greedy
   // pick fused into its epilogue
@@ -1569,6 +1715,19 @@ dflash_status dflash_propose_keys(dflash_handle* h, const int32_t* bonus_tokens,
   return propose_impl(h, bonus_tokens, seq_lens, block_table, B, max_pages_per_seq, k_cache,
                       v_cache, num_pages, nullptr, nullptr, draft_keys, logits_out, workspace,
                       workspace_bytes, stream);
+}
+
+dflash_status dflash_propose_tp(dflash_handle* h, const int32_t* bonus_tokens,
+                                const int32_t* seq_lens, const int32_t* block_table, int B,
+                                int max_pages_per_seq, void* const* k_cache,
+                                void* const* v_cache, int num_pages, int64_t* draft_keys,
+                                float* logits_out, void* workspace, size_t workspace_bytes,
+                                void* stream, dflash_allreduce_fn exchange, void* user) {
+  if (!h || h->tp_size < 2 || !exchange) return DFLASH_ERR_INVALID_ARG;
+  if (!draft_keys && B > 0) return DFLASH_ERR_INVALID_ARG;
+  return propose_impl(h, bonus_tokens, seq_lens, block_table, B, max_pages_per_seq, k_cache,
+                      v_cache, num_pages, nullptr, nullptr, draft_keys, logits_out, workspace,
+                      workspace_bytes, stream, exchange, user);
 }
 
 dflash_status dflash_finalize_draft_keys(const int64_t* draft_keys, const int32_t* bonus_tokens,
@@ -1639,6 +1798,7 @@ dflash_status check_step(const dflash_handle* h, const dflash_step_io* io, const
                          size_t bytes) {
   if (!h || !io || io->B < 0 || io->n < 0) return DFLASH_ERR_INVALID_ARG;
   if (h->vocab_count != h->cfg.vocab) return DFLASH_ERR_INVALID_ARG;   // a vocabulary shard
+  if (h->tp_size > 1) return DFLASH_ERR_INVALID_ARG;                   // a head-parallel shard
   if (io->B == 0) return DFLASH_OK;
   const dflash_config& c = h->cfg;
   const int K = c.block_size - 1;
@@ -1778,12 +1938,13 @@ dflash_status dflash_plan_attention_info(int B, int n_kv_heads, int max_pages_pe
     return DFLASH_ERR_INVALID_ARG;
   const AttnPlan ap = plan_attention(B, n_kv_heads, max_pages_per_seq, page_size, block_size,
                                      q_per_kv, head_dim, num_sms, (flags & 1) != 0, forced_ring,
-                                     (flags & 2) != 0);
+                                     (flags & 2) != 0, (flags & 4) ? 32 : 64);
   out->tcgen05 = ap.tc ? 1 : 0;
   out->keys_per_tile = ap.tc ? ap.kt : kAttnTileKeys;
-  out->ring_depth = ap.tc ? (ap.kt == kTcKeysSmall ? ap.st : kTcStages) : 0;
+  out->ring_depth = ap.tc ? (ap.tc2 || ap.kt == kTcKeysSmall ? ap.st : kTcStages) : 0;
   out->ctas_per_sm =
-      ap.tc && ap.kt == kTcKeysSmall && ap.st == kTcStages && !ap.cluster ? 2 : 1;
+      ap.tc2 || (ap.tc && ap.kt == kTcKeysSmall && ap.st == kTcStages && !ap.cluster) ? 2 : 1;
+  out->transposed_pv = ap.tc2 ? 1 : 0;
   out->chunk_keys = ap.chunk_keys;
   out->max_splits = ap.max_splits;
   out->cluster = ap.cluster ? 1 : 0;
@@ -1838,7 +1999,7 @@ size_t dflash_attention_workspace_bytes(const dflash_handle* h, int B, int max_p
   const AttnPlan ap = plan_attention(B, c.n_kv_heads, max_pages_per_seq, c.page_size,
                                      c.block_size, c.n_q_heads / c.n_kv_heads, c.head_dim,
                                      h->num_sms, h->attn_cluster, h->attn_ring,
-                                     h->attn_persist);
+                                     h->attn_persist, h->attn_tile);
   return align_up(ap.part_o_bytes) + align_up(ap.part_ml_bytes) + kAlign;
 }
 
@@ -1859,7 +2020,7 @@ dflash_status dflash_block_attention(dflash_handle* h, const void* q, const int3
   const AttnPlan ap = plan_attention(B, c.n_kv_heads, max_pages_per_seq, c.page_size,
                                      c.block_size, c.n_q_heads / c.n_kv_heads, c.head_dim,
                                      h->num_sms, h->attn_cluster, h->attn_ring,
-                                     h->attn_persist);
+                                     h->attn_persist, h->attn_tile);
   AttnParams prm;
   prm.q = static_cast<const bf16*>(q);
   prm.o = static_cast<f16*>(o);

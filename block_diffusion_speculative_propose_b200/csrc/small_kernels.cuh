@@ -122,6 +122,44 @@ __global__ void __launch_bounds__(256) rmsnorm_rows_kernel(
   }
 }
 
+// Tensor-parallel residual add: x[src(r)] += part[src(r)] (the all-reduced sum
+// of every rank's row-parallel O or down projection), then out[r] = fp16 of
+// RMSNorm(x[src(r)]) * w exactly as rmsnorm_rows_kernel (same src(r) rule).
+__global__ void __launch_bounds__(256) add_rmsnorm_rows_kernel(
+    float* __restrict__ x, const float* __restrict__ part, const bf16* __restrict__ w,
+    f16* __restrict__ out, int H, float eps, int gather_k, int bs) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ float red[32];
+  const int r = blockIdx.x;
+  const int src = gather_k > 0 ? (r / gather_k) * bs + 1 + (r - (r / gather_k) * gather_k) : r;
+  float* xr = x + static_cast<size_t>(src) * H;
+  const float* pr = part + static_cast<size_t>(src) * H;
+  float ss = 0.f;
+  for (int j = threadIdx.x * 4; j < H; j += blockDim.x * 4) {
+    float4 a = *reinterpret_cast<const float4*>(xr + j);
+    const float4 c = *reinterpret_cast<const float4*>(pr + j);
+    a.x += c.x;
+    a.y += c.y;
+    a.z += c.z;
+    a.w += c.w;
+    *reinterpret_cast<float4*>(xr + j) = a;
+    ss += a.x * a.x + a.y * a.y + a.z * a.z + a.w * a.w;
+  }
+  ss = block_sum(ss, red);
+  const float rinv = rsqrtf(ss / H + eps);
+  f16* orow = out + static_cast<size_t>(r) * H;
+  for (int j = threadIdx.x * 4; j < H; j += blockDim.x * 4) {
+    const float4 a = *reinterpret_cast<const float4*>(xr + j);
+    const uint2 wq = *reinterpret_cast<const uint2*>(w + j);
+    const bf16* wb = reinterpret_cast<const bf16*>(&wq);
+    uint2 o;
+    o.x = pack_f16x2(a.x * rinv * bf2f(wb[0]), a.y * rinv * bf2f(wb[1]));
+    o.y = pack_f16x2(a.z * rinv * bf2f(wb[2]), a.w * rinv * bf2f(wb[3]));
+    *reinterpret_cast<uint2*>(orow + j) = o;
+  }
+}
+
 // drafts[b, i] = argmax of LM-head row (b, i); block[b] = [bonus_b, drafts[b]].
 __global__ void argmax_finalize_kernel(const unsigned long long* __restrict__ keys,
                                        const int32_t* __restrict__ bonus,
@@ -416,11 +454,13 @@ __global__ void absmax_bf16_kernel(const bf16* __restrict__ x, int n, unsigned* 
 // of a row-major W [N, K] becomes one contiguous chunk (kPackRows rows of 128
 // bytes, in order) at chunk index n_tile * (K / 64) + k_block; rows past N are
 // zero.  Every TMA box of the weight stream is then a single contiguous read.
+// The source rows are `ld` elements apart (a column slice of a wider matrix
+// when ld > K; 16-byte aligned starts).
 // With to_f16 the bf16 values are converted to fp16 on the way.
 constexpr int kPackRows = 256;
 
 __global__ void pack_tiles_kernel(const uint16_t* __restrict__ src, uint16_t* __restrict__ dst,
-                                  int N, int K, size_t units, int to_f16) {
+                                  int N, int K, int ld, size_t units, int to_f16) {
   const int kb_count = K / 64;
   for (size_t u = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; u < units;
        u += static_cast<size_t>(gridDim.x) * blockDim.x) {
@@ -432,7 +472,7 @@ __global__ void pack_tiles_kernel(const uint16_t* __restrict__ src, uint16_t* __
     const int row = nt * kPackRows + r;
     uint4 v = make_uint4(0, 0, 0, 0);
     if (row < N)
-      v = *reinterpret_cast<const uint4*>(src + static_cast<size_t>(row) * K + kb * 64 + j8 * 8);
+      v = *reinterpret_cast<const uint4*>(src + static_cast<size_t>(row) * ld + kb * 64 + j8 * 8);
     if (to_f16) {
       uint32_t* w = reinterpret_cast<uint32_t*>(&v);
 #pragma unroll

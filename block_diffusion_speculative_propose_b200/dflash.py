@@ -96,7 +96,7 @@ class _TargetWeights(ctypes.Structure):
 class _AttnPlan(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in ("tcgen05", "keys_per_tile", "ring_depth",
                                             "ctas_per_sm", "chunk_keys", "max_splits",
-                                            "cluster", "persistent")]
+                                            "cluster", "persistent", "transposed_pv")]
 
 
 _lib = None
@@ -667,11 +667,11 @@ def finalize_draft_keys(draft_keys, bonus_tokens, block_size: int, vocab: int,
 def attention_plan(B: int, n_kv_heads: int, max_pages_per_seq: int, block_size: int,
                    q_per_kv: int, head_dim: int = 128, page_size: int = 16, num_sms: int = 148,
                    forced_ring: int = 0, cluster: bool = False,
-                   persistent: bool = False) -> Dict[str, int]:
+                   persistent: bool = False, tile32: bool = False) -> Dict[str, int]:
     """dflash_plan_attention_info: the attention launch plan for this geometry
     (host only)."""
     out = _AttnPlan()
-    flags = (1 if cluster else 0) | (2 if persistent else 0)
+    flags = (1 if cluster else 0) | (2 if persistent else 0) | (4 if tile32 else 0)
     _check(lib().dflash_plan_attention_info(B, n_kv_heads, max_pages_per_seq, page_size,
                                             block_size, q_per_kv, head_dim, num_sms,
                                             forced_ring, flags, ctypes.byref(out)),

@@ -68,7 +68,8 @@ typedef enum {
   DFLASH_ERR_DEVICE_BOUNDS = -5,     /* returned by dflash_check_device_errors (see above)    */
   DFLASH_ERR_UNIMPLEMENTED = -6,
   DFLASH_ERR_DEVICE_TIMEOUT = -7,    /* returned by dflash_check_device_errors                */
-  DFLASH_ERR_RANGE = -8              /* weights outside the fp16 range the path stores them in */
+  DFLASH_ERR_RANGE = -8,             /* weights outside the fp16 range the path stores them in */
+  DFLASH_ERR_EXCHANGE = -9           /* the caller's all-reduce hook reported a failure        */
 } dflash_status;
 
 /* Device error bits reported by dflash_check_device_errors(). */
@@ -169,6 +170,26 @@ dflash_status dflash_create(const dflash_config* cfg, const dflash_weights* w,
 dflash_status dflash_create_vocab_shard(const dflash_config* cfg, const dflash_weights* w,
                                         int device, int vocab_start, int vocab_count,
                                         dflash_handle** out);
+
+/* Tensor-parallel rank tp_rank of tp_size (§"Context KV Injection": each rank
+ * projects and stores "this rank's KV heads only"; §"DFlashQwen3ForCausalLM":
+ * the aliased LM head is a column-parallel linear over the vocabulary).  The
+ * handle holds rank r's slice of the draft: kv heads [r Hkv/S, (r+1) Hkv/S)
+ * with their query heads (each kv head keeps its query group), MLP features
+ * [r I/S, (r+1) I/S), the matching columns of Wo and W_down (row-parallel:
+ * each rank forms a partial sum of the layer's O and down outputs), and the
+ * LM-head vocabulary rows [vocab_start, vocab_start + vocab_count).  fc,
+ * hidden_norm, the norms and the embedding are replicated.  cfg and w describe
+ * the WHOLE model (every rank passes the same); the slices are copied out of
+ * w.  Requires n_kv_heads % tp_size == 0 and intermediate % (64 tp_size) == 0
+ * (DFLASH_ERR_UNSUPPORTED_SHAPE), 0 <= tp_rank < tp_size and the vocabulary
+ * rules of dflash_create_vocab_shard.  The handle's KV pools hold its own kv
+ * heads only ([num_pages, n_kv_heads / tp_size, page_size, head_dim]):
+ * dflash_inject_context on it projects and writes those heads; it proposes
+ * through dflash_propose_tp.  tp_size 1 gives a whole-model handle. */
+dflash_status dflash_create_tp_shard(const dflash_config* cfg, const dflash_weights* w,
+                                     int device, int tp_rank, int tp_size, int vocab_start,
+                                     int vocab_count, dflash_handle** out);
 
 /* Frees everything the handle owns.  The caller must make sure no work that
  * uses the handle is still pending.  NULL is a no-op. */
@@ -342,6 +363,33 @@ dflash_status dflash_propose_keys(dflash_handle* h, const int32_t* bonus_tokens,
                                   float* logits_out, void* workspace, size_t workspace_bytes,
                                   void* stream);
 
+/* The exchange of a tensor-parallel proposal: sum `count` fp32 values at the
+ * DEVICE pointer `data` element-wise over every rank of the group, in place
+ * (an all-reduce SUM, e.g. ncclAllReduce with ncclSum), ordered after the work
+ * already enqueued on `stream` and before the work enqueued after the call
+ * returns (the library enqueues its next kernels on `stream` right after).
+ * `user` is passed through.  Return 0 on success. */
+typedef int (*dflash_allreduce_fn)(float* data, size_t count, void* stream, void* user);
+
+/* dflash_propose_keys on a tensor-parallel shard (dflash_create_tp_shard):
+ * every layer runs on this rank's heads and MLP features; after the O
+ * projection and after the down projection the rank's partial sums (the
+ * [B * block_size, hidden] fp32 rows, in the workspace) go through
+ * `exchange`, and the summed rows are added to the replicated residual
+ * stream.  Every rank of the group must make the same call (same B, block
+ * tables, bonus tokens and sequence lengths; each with its own KV pools of its
+ * kv heads).  Output: this rank's vocabulary shard's greedy-pick keys, as
+ * dflash_propose_keys; an all-reduce MAX of them over the ranks, then
+ * dflash_finalize_draft_keys, gives the drafts.  DFLASH_ERR_INVALID_ARG for a
+ * whole-model handle or a NULL exchange; DFLASH_ERR_EXCHANGE if the hook
+ * returns non-zero (the kernels enqueued before it stay enqueued). */
+dflash_status dflash_propose_tp(dflash_handle* h, const int32_t* bonus_tokens,
+                                const int32_t* seq_lens, const int32_t* block_table, int B,
+                                int max_pages_per_seq, void* const* k_cache,
+                                void* const* v_cache, int num_pages, int64_t* draft_keys,
+                                float* logits_out, void* workspace, size_t workspace_bytes,
+                                void* stream, dflash_allreduce_fn exchange, void* user);
+
 /* Drafts from the exchanged keys of dflash_propose_keys: draft_tokens [B, K]
  * int32 = the vocabulary id in each key; block_tokens [B, block_size] int32
  * (nullable) = cat(bonus_tokens[b], drafts[b]).  A key that names no id below
@@ -511,18 +559,24 @@ dflash_status dflash_block_attention(dflash_handle* h, const void* q, const int3
  * (diagnostics; host only, no device needed): kv groups of bs * G query rows
  * (G = query heads per kv head), block tables of W pages of P keys, on
  * `num_sms` SMs.  forced_ring: 0 (the planner's choice), 2 or 6 as
- * DFLASH_ATTN_STAGES forces it; flags: bit 0 the opt-in cluster combine,
- * bit 1 the opt-in persistent kernel.  Written to *out; DFLASH_ERR_INVALID_ARG
- * for a non-positive size or a NULL out. */
+ * DFLASH_ATTN_STAGES forces it (the one-CTA-per-tile kernel with that ring);
+ * flags: bit 0 the opt-in cluster combine, bit 1 the opt-in persistent
+ * kernel, bit 2 32-key tiles for the two-CTA kernel (DFLASH_ATTN_TILE=32).
+ * Without bits 0-1 or a forced ring, head_dim 128 takes the two-CTA-per-SM
+ * kernel with P V transposed (64-key tiles in a two-deep ring; with bit 2,
+ * 32-key tiles in a four-deep ring),
+ * its splits sized for 8 CTAs per SM.  Written to *out;
+ * DFLASH_ERR_INVALID_ARG for a non-positive size or a NULL out. */
 typedef struct dflash_attention_plan {
   int tcgen05;        /* 1: the tcgen05 kernel (bs * G <= 64), 0: the mma.sync kernel */
-  int keys_per_tile;  /* tcgen05 kernel: 64 or 128 */
-  int ring_depth;     /* tcgen05 kernel: K/V tiles in flight per CTA (2 or 6) */
-  int ctas_per_sm;    /* tcgen05 kernel: 2 for the two-deep 64-key ring, else 1 */
+  int keys_per_tile;  /* tcgen05 kernels: 32, 64 or 128 */
+  int ring_depth;     /* tcgen05 kernels: K/V tiles in flight per CTA (2, 4 or 6) */
+  int ctas_per_sm;    /* tcgen05 kernels: 2 for the two-CTA kernels, else 1 */
   int chunk_keys;     /* keys per split */
   int max_splits;     /* splits of the longest request */
   int cluster;        /* splits combined inside a thread-block cluster */
   int persistent;     /* persistent CTAs walking the items */
+  int transposed_pv;  /* head_dim 128 default: two CTAs per SM, O^T = V^T P^T (M = 128) */
 } dflash_attention_plan;
 dflash_status dflash_plan_attention_info(int B, int n_kv_heads, int max_pages_per_seq,
                                          int page_size, int block_size, int q_per_kv,

