@@ -1341,8 +1341,12 @@ dflash_status create_handle(const dflash_config* cfg, const dflash_weights* w, i
                           cudaMemcpyDeviceToDevice, st) != cudaSuccess)
       return fail_st(DFLASH_ERR_CUDA);
   }
+  // the LM head rows of this handle: a vocabulary shard (dflash_create_vocab_shard)
+  // is given its rows; a tensor-parallel shard takes them out of the whole head
+  const void* lm_src = tp_size > 1 ? rows_at(w->lm_head, static_cast<size_t>(vocab_start), H)
+                                   : w->lm_head;
   if (cudaMalloc(&h->lm_head16, static_cast<size_t>(vocab_count) * rowb) != cudaSuccess ||
-      cudaMemcpyAsync(h->lm_head16, w->lm_head, static_cast<size_t>(vocab_count) * rowb,
+      cudaMemcpyAsync(h->lm_head16, lm_src, static_cast<size_t>(vocab_count) * rowb,
                       cudaMemcpyDeviceToDevice, st) != cudaSuccess)
     return fail_st(DFLASH_ERR_CUDA);
   // fp16 range statistics of the converted weights and of the norm weights

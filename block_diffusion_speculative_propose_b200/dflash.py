@@ -27,6 +27,7 @@ STATUS = {
     -6: "DFLASH_ERR_UNIMPLEMENTED",
     -7: "DFLASH_ERR_DEVICE_TIMEOUT",
     -8: "DFLASH_ERR_RANGE",
+    -9: "DFLASH_ERR_EXCHANGE",
 }
 DEVERR_TIMEOUT, DEVERR_SLOT, DEVERR_TABLE, DEVERR_TOKEN, DEVERR_POSITION = 1, 2, 4, 8, 16
 KERNEL_KINDS = 14
@@ -50,6 +51,9 @@ class _Config(ctypes.Structure):
 
 
 _PP = ctypes.POINTER(ctypes.c_void_p)
+# dflash_allreduce_fn: int (*)(float* data, size_t count, void* stream, void* user)
+ALLREDUCE_FN = ctypes.CFUNCTYPE(ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p,
+                                ctypes.c_void_p)
 
 
 class _Weights(ctypes.Structure):
@@ -122,6 +126,10 @@ def lib() -> ctypes.CDLL:
         "dflash_propose_workspace_bytes": ([vp, i32, i32], sz),
         "dflash_propose_final_rows_offset": ([vp, i32, i32], sz),
         "dflash_set_wait_limit": ([i32, ctypes.c_longlong], i32),
+        "dflash_create_tp_shard": ([ctypes.POINTER(_Config), ctypes.POINTER(_Weights), i32, i32,
+                                    i32, i32, i32, ctypes.POINTER(vp)], i32),
+        "dflash_propose_tp": ([vp, vp, vp, vp, i32, i32, _PP, _PP, i32, vp, vp, vp, sz, vp,
+                               ALLREDUCE_FN, vp], i32),
         "dflash_aux_capture_layers": ([ctypes.POINTER(ctypes.c_int), i32, i32,
                                        ctypes.POINTER(ctypes.c_int)], i32),
         "dflash_target_create": ([ctypes.POINTER(_TargetConfig), ctypes.POINTER(_TargetWeights),
@@ -231,7 +239,7 @@ class DFlash:
     shard's [count, H] rows, and the handle proposes through propose_keys."""
 
     def __init__(self, cfg: Dict, weights: Dict, device: int = 0, max_position: int = 0,
-                 vocab_shard: Optional[Sequence[int]] = None):
+                 vocab_shard: Optional[Sequence[int]] = None, tp: Optional[Sequence[int]] = None):
         L = lib()
         self.cfg = dict(cfg)
         self.device = torch.device("cuda", device)
@@ -268,7 +276,17 @@ class DFlash:
             self._keep.append(arr)
             setattr(w, k, pp)
         h = ctypes.c_void_p()
-        if vocab_shard is None:
+        self.tp = (0, 1) if tp is None else (int(tp[0]), int(tp[1]))
+        if tp is not None:
+            # one tensor-parallel rank: `weights` is the whole model (every rank
+            # passes the same); the library copies out this rank's slices
+            self.vocab_shard = ((0, cfg["vocab"]) if vocab_shard is None else
+                                (int(vocab_shard[0]), int(vocab_shard[1])))
+            _check(L.dflash_create_tp_shard(ctypes.byref(c), ctypes.byref(w), device,
+                                            self.tp[0], self.tp[1], self.vocab_shard[0],
+                                            self.vocab_shard[1], ctypes.byref(h)),
+                   "dflash_create_tp_shard")
+        elif vocab_shard is None:
             self.vocab_shard = (0, cfg["vocab"])
             _check(L.dflash_create(ctypes.byref(c), ctypes.byref(w), device, ctypes.byref(h)),
                    "dflash_create")
@@ -453,6 +471,39 @@ class DFlash:
                                          int(k_cache[0].shape[0]), _ptr(draft_keys),
                                          _ptr(logits_out), _ptr(ws), ws.numel(),
                                          _stream(stream)), "dflash_propose_keys")
+        return draft_keys
+
+    def propose_tp(self, bonus_tokens, seq_lens, block_table, k_cache, v_cache, exchange,
+                   draft_keys=None, logits_out=None, workspace: Optional[torch.Tensor] = None,
+                   stream=None):
+        """dflash_propose_tp on a tensor-parallel shard: `exchange(data_ptr,
+        count, stream_ptr) -> int` must sum the `count` fp32 values at the
+        device pointer over every rank, in place, ordered on that stream (0 on
+        success).  Returns this rank's vocabulary shard's keys [B, K] int64."""
+        B = int(bonus_tokens.shape[0])
+        bs = self.cfg["block_size"]
+        _want(bonus_tokens, torch.int32, "bonus_tokens")
+        _want(seq_lens, torch.int32, "seq_lens")
+        _want(block_table, torch.int32, "block_table")
+        W = int(block_table.shape[1])
+        if draft_keys is None:
+            draft_keys = torch.empty(B, bs - 1, dtype=torch.int64, device=self.device)
+        need = self.propose_workspace_bytes(B, W) if B else 0
+        ws = workspace if workspace is not None else self.ws.get(need)
+        kp, ka = _ptr_array(k_cache)
+        vp, va = _ptr_array(v_cache)
+
+        def hook(data, count, st, user):
+            try:
+                return int(exchange(int(data), int(count), st))
+            except Exception:
+                return 1
+        cb = ALLREDUCE_FN(hook)
+        _check(lib().dflash_propose_tp(self.h, _ptr(bonus_tokens), _ptr(seq_lens),
+                                       _ptr(block_table), B, W, kp, vp,
+                                       int(k_cache[0].shape[0]), _ptr(draft_keys),
+                                       _ptr(logits_out), _ptr(ws), ws.numel(), _stream(stream),
+                                       cb, None), "dflash_propose_tp")
         return draft_keys
 
     def linear(self, A, W, out=None, block_n: int = 0, splits: int = 0, workspace=None,

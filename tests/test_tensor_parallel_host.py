@@ -130,3 +130,55 @@ def test_gloo_ranks_exchange_keys(world):
     want = [reference_pick(lg[r]) for r in range(lg.shape[0])]
     for r in range(world):
         assert res[r] == want
+
+
+# ----------------------------------------------------------------------------
+# head-parallel layers: the exchange hook of dflash_propose_tp between gloo ranks
+# ----------------------------------------------------------------------------
+def _hook_rank_main(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world))
+    sys.path.insert(0, ROOT)
+    import torch
+    import torch.distributed as dist
+    from block_diffusion_speculative_propose_b200.tensor_parallel import allreduce_hook
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        # a host "workspace" whose middle holds this rank's partial sums; the
+        # hook receives only the pointer and the count, as from the library
+        ws = torch.zeros(4096, dtype=torch.uint8)
+        off, count = 1024, 100
+        part = ws[off:off + 4 * count].view(torch.float32)
+        g = torch.Generator().manual_seed(rank)
+        part.copy_(torch.randn(count, generator=g))
+        hook = allreduce_hook(ws)
+        rc = hook(ws.data_ptr() + off, count)
+        bad = hook(ws.data_ptr() + 4000, 100)    # past the workspace: refused, nothing sent
+        q.put((rank, rc, bad, part.tolist(), ws[:off].abs().sum().item(),
+               ws[off + 4 * count:].abs().sum().item()))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_gloo_ranks_sum_partials_in_place(world):
+    """The hook sums every rank's row-parallel partials in place, touching
+    nothing else of the workspace, and refuses a range outside it."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = 29560 + world
+    procs = [ctx.Process(target=_hook_rank_main, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = {}
+    for _ in range(world):
+        rank, rc, bad, vals, before, after = q.get(timeout=120)
+        res[rank] = vals
+        assert rc == 0 and bad == 1 and before == 0 and after == 0
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    import torch
+    want = sum(torch.randn(100, generator=torch.Generator().manual_seed(r)) for r in range(world))
+    for r in range(world):
+        np.testing.assert_allclose(res[r], want.numpy(), rtol=1e-6, atol=1e-6)
