@@ -73,7 +73,9 @@ struct Tc2Cfg {
   static constexpr int kOffL = kOffAlpha + 2 * kTcM * 4;       // [64] fp32 row sums
   static constexpr int kOffM = kOffL + kTcM * 4;               // [64] fp32 row references
   static constexpr int kOffBar = kOffM + kTcM * 4;
-  static constexpr int kSmem = 1024 + kOffBar + 256;
+  static constexpr int kOffPages = kOffBar + 256;              // the split's page rows
+  static constexpr int kMaxPages = 8192 / 16 + 1;              // pages of the longest split
+  static constexpr int kSmem = 1024 + kOffPages + kMaxPages * 4;
   static constexpr int kOCol = 2 * KT;                         // TMEM column of O^T
   static constexpr int kTmemCols = KT == 64 ? 256 : 128;
   static_assert(KT == 64 || KT == 32, "tile width");
@@ -166,6 +168,9 @@ __global__ void __launch_bounds__(kTcThreads, 2)
   uint64_t* q_full = bars + 25;
   uint64_t* o_final = bars + 26;   // the last tile's P V landed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 27);
+  // rows of this split's pages in the [pages * Hkv * 16, D] views of the pools,
+  // (-16: a page past the table or the pool; the loads then fill zeros)
+  int* s_rows = reinterpret_cast<int*>(smem + C::kOffPages);
   auto sK = [&](int s) { return smem + s * C::kKVBytes; };
   auto sV = [&](int s) { return smem + C::kOffV + s * C::kKVBytes; };
 
@@ -202,29 +207,31 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     // as S of tile tk - ST has run, V of tile tv (never ahead of K) as soon as
     // P V of tile tv - ST has.  (One thread, so that the two rings never wait
     // on each other through a divergent warp.)
+    // the split's page rows, read from the block table once (all 32 lanes),
+    // checked against the table width and the pool
+    const int pg0 = k0 >> 4, npg = min(C::kMaxPages, ((k1 - 1) >> 4) - pg0 + 1);
+    const int* bt = p.block_table + static_cast<size_t>(b) * p.W;
+    for (int j = lane; j < npg; j += 32) {
+      const int pg = pg0 + j;
+      int y = -16;
+      if (pg >= p.W) {
+        raise_error(p.err, DFLASH_DEVERR_TABLE);
+      } else {
+        const int page = bt[pg];
+        if (page < 0 || page >= p.num_pages) raise_error(p.err, DFLASH_DEVERR_SLOT);
+        else y = (page * p.Hkv + h) * 16;
+      }
+      s_rows[j] = y;
+    }
+    __syncwarp();
     if (lane == 0) {
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      const int* bt = p.block_table + static_cast<size_t>(b) * p.W;
-      // the rows of this tile's pages in the [pages * Hkv * 16, D] views
-      // (-16: a page past the range, fully out of bounds, which TMA fills with zeros)
+      // the rows of tile t's pages (-16 past the split: TMA fills zeros)
       auto page_rows = [&](int t, int* y) {
-        const int t0 = k0 + t * KT;
-        const int npages = (min(KT, k1 - t0) + 15) >> 4;
+        const int npages = (min(KT, k1 - (k0 + t * KT)) + 15) >> 4;
 #pragma unroll
-        for (int j = 0; j < KT / 16; ++j) {
-          y[j] = -16;
-          if (j < npages) {
-            const int pg = (t0 >> 4) + j;
-            if (pg >= p.W) {
-              raise_error(p.err, DFLASH_DEVERR_TABLE);
-            } else {
-              const int page = bt[pg];
-              if (page < 0 || page >= p.num_pages) raise_error(p.err, DFLASH_DEVERR_SLOT);
-              else y[j] = (page * p.Hkv + h) * 16;
-            }
-          }
-        }
+        for (int j = 0; j < KT / 16; ++j) y[j] = j < npages ? s_rows[t * (KT / 16) + j] : -16;
       };
       auto issue = [&](int t, bool is_v) {
         const int s = t % ST;
@@ -244,12 +251,14 @@ __global__ void __launch_bounds__(kTcThreads, 2)
       long long idle_since = clock64();
       while (tv < n_tiles) {
         bool progress = false;
-        if (tk < n_tiles && mbar_test_wait(&k_empty[tk % ST], ((tk / ST) & 1) ^ 1u)) {
-          issue(tk++, false);
-          progress = true;
-        }
+        // V first: P V of tile tv waits on it, while K of tile tk (released
+        // right after S) still has the softmax and P V of a tile as slack
         if (tv < tk && mbar_test_wait(&v_empty[tv % ST], ((tv / ST) & 1) ^ 1u)) {
           issue(tv++, true);
+          progress = true;
+        }
+        if (tk < n_tiles && mbar_test_wait(&k_empty[tk % ST], ((tk / ST) & 1) ^ 1u)) {
+          issue(tk++, false);
           progress = true;
         }
         if (progress) {
