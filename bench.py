@@ -50,6 +50,12 @@ TRAFFIC = {
     # (ncu --set full on one launch)
     ("qwen3_b1_ctx2048", "gemm_gate_up"): {"bytes_per_launch": 205118208,
                                            "digest": "59a7f03b8506a4c8"},
+    # attention of the batch-128, 8k-32k-context step, scaled from one launch on a
+    # 16-request case of the same context distribution (1.2523 GB read + 24.4 MB
+    # written for 1.2525 GB of algorithmic bytes: ratio 1.0193) to the launch's
+    # algorithmic bytes
+    ("qwen3_b128_ctx8192_32768", "attention"): {"ratio_to_algorithmic": 1.0193,
+                                                "digest": "fec19f3b5522f0a2"},
 }
 
 
@@ -63,6 +69,10 @@ def parse_args():
     ap.add_argument("--no-graph", action="store_true", help="eager launches for the value loop")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-extras", action="store_true", help="skip the sub-measurements")
+    ap.add_argument("--ncu-case", choices=["attention", "gemms", "verify"], default=None,
+                    help="run one kernel family twice on a reduced case of the workload "
+                         "(for a profiler capture of the second run) and exit")
     ap.add_argument("--seed", type=int, default=1)
     a = ap.parse_args()
     a.warmup = max(a.warmup, 3)
@@ -73,7 +83,8 @@ def parse_args():
 # Sources a kernel family is compiled from (its traffic figure is void once
 # any of them changes).
 FAMILY_SOURCES = {"gemm": ("gemm_tcgen05.cuh", "dflash_device.cuh"),
-                  "attention": ("attention_tc.cuh", "attention.cuh", "dflash_device.cuh")}
+                  "attention": ("attention_tc2.cuh", "attention_tc.cuh", "attention.cuh",
+                                "dflash_device.cuh")}
 
 
 def source_digest(family: str = "gemm") -> str:
@@ -649,8 +660,11 @@ def run_ours(a, rank, world, local):
         roof = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s",
                 "frac": ach / peak}
     tr = TRAFFIC.get((a.workload, dom))
-    roof.update({"traffic": tr["bytes_per_launch"] if tr and tr["digest"] == source_digest(dom)
-                 else None, "kernel": dom, "algorithmic_bytes_per_launch": byts,
+    traffic = None
+    if tr and tr["digest"] == source_digest(dom):
+        traffic = (tr["bytes_per_launch"] if "bytes_per_launch" in tr
+                   else tr["ratio_to_algorithmic"] * byts)
+    roof.update({"traffic": traffic, "kernel": dom, "algorithmic_bytes_per_launch": byts,
                  "algorithmic_flops_per_launch": flops, "launch_ms": per_launch_s * 1e3,
                  "peak_source": f"{peaks_src} ({'sustained bf16' if roof['bound'] == 'tensor' else 'HBM copy'})"})
 
@@ -667,7 +681,7 @@ def run_ours(a, rank, world, local):
         step_b += alg_k[0] * v["launches_per_step"]
         step_f += alg_k[1] * v["launches_per_step"]
     step_roof = roof_of(step_b, step_f, t_step, peaks)
-    extras = extra_measurements(st, peaks) if rank == 0 else {}
+    extras = extra_measurements(st, peaks) if rank == 0 and not a.no_extras else {}
 
     assert st.h.check_device_errors() == 0, "device error flags raised"
 
@@ -872,8 +886,93 @@ def run_reference(a, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def ncu_case(a):
+    """Reduced cases of the workload's hot kernel families, each run twice, so
+    that a profiler can capture the second launch on a few GB of device memory:
+      attention  one layer of block attention for 16 requests drawn from the
+                 workload's context-length distribution (paged, shuffled pages)
+      gemms      injection + proposal at the workload's batch with 64-token
+                 contexts: the GEMM shapes of the full step (block rows, LM-head
+                 rows, injected rows) with a small KV pool
+      verify     greedy verification of the workload's [B, K+1, V] fp32 logits"""
+    from block_diffusion_speculative_propose_b200 import DFlash, paged_slots, synth, verify_greedy
+    wl = synth.WORKLOADS[a.workload]
+    cfg = synth.model_config(wl["model"])
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev)
+    g.manual_seed(a.seed)
+    B, bs, P = wl["batch"], cfg["block_size"], cfg["page_size"]
+    Hkv, d = cfg["n_kv_heads"], cfg["head_dim"]
+    if a.ncu_case == "verify":
+        V, K = cfg["vocab"], bs - 1
+        lo = torch.randn(B, K + 1, V, generator=g, device=dev)
+        dr = torch.randint(0, V, (B, K), generator=g, device=dev).to(torch.int32)
+        for _ in range(2):
+            verify_greedy(dr, lo)
+        torch.cuda.synchronize()
+        print(json.dumps({"ncu_case": "verify", "algorithmic_bytes": lo.numel() * 4.0}))
+        return
+    if a.ncu_case == "attention":
+        c1 = dict(cfg, n_layers=1, vocab=2048, mask_token_id=2047)
+        h = DFlash(c1, synth.make_weights(c1, seed=0, device=dev),
+                   max_position=wl["ctx_hi"] + 2 * bs)
+        rng = np.random.default_rng(a.seed)
+        n = 16
+        seq = rng.integers(wl["ctx_lo"], wl["ctx_hi"] + 1, size=n).astype(np.int32)
+        need = [-(-(int(s) + bs) // P) for s in seq]
+        perm = rng.permutation(sum(need))
+        table = np.zeros((n, max(need)), dtype=np.int32)
+        cur = 0
+        for b, m in enumerate(need):
+            table[b, :m] = perm[cur:cur + m]
+            cur += m
+        shape = (sum(need), Hkv, P, d)
+        kc = torch.randn(shape, generator=g, device=dev).to(torch.bfloat16)
+        vc = torch.randn(shape, generator=g, device=dev).to(torch.bfloat16)
+        q = torch.randn(n * bs, cfg["n_q_heads"], d, generator=g, device=dev).to(torch.bfloat16)
+        seq_t, table_t = torch.tensor(seq, device=dev), torch.tensor(table, device=dev)
+        for _ in range(2):
+            h.block_attention(q, seq_t, table_t, kc, vc)
+        torch.cuda.synchronize()
+        keys = float((seq.astype(np.float64) + bs).sum())
+        byts = keys * Hkv * d * 2 * 2 + 2 * n * bs * cfg["n_q_heads"] * d * 2
+        print(json.dumps({"ncu_case": "attention", "requests": n, "algorithmic_bytes": byts,
+                          "device_errors": h.check_device_errors()}))
+        h.close()
+        return
+    # gemms
+    h = DFlash(cfg, synth.make_weights(cfg, seed=0, device=dev), max_position=4096)
+    ctx = 64
+    per = -(-(ctx + 2 * bs) // P)
+    table = torch.arange(B * per, dtype=torch.int32, device=dev).view(B, per)
+    shape = (B * per, Hkv, P, d)
+    kc = [torch.randn(shape, generator=g, device=dev).to(torch.bfloat16)
+          for _ in range(cfg["n_layers"])]
+    vc = [torch.randn(shape, generator=g, device=dev).to(torch.bfloat16)
+          for _ in range(cfg["n_layers"])]
+    rows_per = 6 if wl["accept"] == "geometric" else (bs + 1) // 2
+    rows = B * rows_per
+    req = (torch.arange(rows, device=dev) % B).to(torch.int64)
+    pos = (ctx - rows_per + torch.arange(rows, device=dev) // B).to(torch.int64)
+    slots = paged_slots(pos, req, table, P)
+    aux = torch.randn(rows, cfg["n_target_layers"] * cfg["hidden"], generator=g,
+                      device=dev).to(torch.bfloat16)
+    bonus = torch.randint(0, cfg["vocab"] - 1, (B,), generator=g, device=dev).to(torch.int32)
+    seq = torch.full((B,), ctx, dtype=torch.int32, device=dev)
+    for _ in range(2):
+        h.inject_context(aux, pos, slots, kc, vc)
+        h.propose(bonus, seq, table, kc, vc)
+    torch.cuda.synchronize()
+    print(json.dumps({"ncu_case": "gemms", "block_rows": B * bs, "injected_rows": rows,
+                      "device_errors": h.check_device_errors()}))
+    h.close()
+
+
 def main():
     a = parse_args()
+    if a.ncu_case:
+        ncu_case(a)
+        return
     rank, world, local = dist_init(a.gpus)
     try:
         if a.impl == "reference":

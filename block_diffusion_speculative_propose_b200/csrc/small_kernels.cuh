@@ -239,7 +239,30 @@ __global__ void __launch_bounds__(256) verify_partial_kernel(
   const float* src = logits + row * static_cast<size_t>(V);
   unsigned long long best = 0ull;
   if ((V & 3) == 0) {
-    for (int j = beg + threadIdx.x * 4; j < end; j += blockDim.x * 4) {
+    // four 16-byte loads in flight per thread (a row is streamed once, so the
+    // loads, not the compares, set the pace)
+    constexpr int U = 4;
+    const int step = blockDim.x * 4;
+    int j = beg + threadIdx.x * 4;
+    for (; j + (U - 1) * step < end; j += U * step) {
+      float4 v[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) v[u] = __ldcs(reinterpret_cast<const float4*>(src + j + u * step));
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int jj = j + u * step;
+        unsigned long long k;
+        k = argmax_key(v[u].x, jj);
+        best = k > best ? k : best;
+        k = argmax_key(v[u].y, jj + 1);
+        best = k > best ? k : best;
+        k = argmax_key(v[u].z, jj + 2);
+        best = k > best ? k : best;
+        k = argmax_key(v[u].w, jj + 3);
+        best = k > best ? k : best;
+      }
+    }
+    for (; j < end; j += step) {
       const float4 v = __ldcs(reinterpret_cast<const float4*>(src + j));
       unsigned long long k;
       k = argmax_key(v.x, j);
