@@ -46,10 +46,6 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # dram__bytes_write.sum) for the kernel family that dominates a workload,
 # keyed by the digest of the kernel sources it was measured on.
 TRAFFIC = {
-    # gate/up GEMM of the batch-1 Qwen3-8B-shaped step: 201.57 MB read + 3.55 MB written
-    # (ncu --set full on one launch)
-    ("qwen3_b1_ctx2048", "gemm_gate_up"): {"bytes_per_launch": 205118208,
-                                           "digest": "59a7f03b8506a4c8"},
     # attention of the batch-128, 8k-32k-context step, scaled from one launch on a
     # 16-request case of the same context distribution (1.2523 GB read + 24.4 MB
     # written for 1.2525 GB of algorithmic bytes: ratio 1.0193) to the launch's
@@ -82,7 +78,7 @@ def parse_args():
 
 # Sources a kernel family is compiled from (its traffic figure is void once
 # any of them changes).
-FAMILY_SOURCES = {"gemm": ("gemm_tcgen05.cuh", "dflash_device.cuh"),
+FAMILY_SOURCES = {"gemm": ("gemm_tcgen05.cuh", "gemm_pair.cuh", "dflash_device.cuh"),
                   "attention": ("attention_tc2.cuh", "attention_tc.cuh", "attention.cuh",
                                 "dflash_device.cuh")}
 

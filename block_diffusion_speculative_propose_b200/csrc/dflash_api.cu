@@ -21,6 +21,7 @@
 #include "attention_tc2.cuh"
 #include "dflash.h"
 #include "gemm_tcgen05.cuh"
+#include "gemm_pair.cuh"
 #include "small_kernels.cuh"
 #include "target_model.cuh"
 
@@ -386,6 +387,16 @@ struct dflash_handle {
     const char* e = std::getenv("DFLASH_ATTN_TILE");
     return (e && std::atoi(e) == 32) ? 32 : 64;
   }();
+  // whole-tile GEMMs over several 128-row M tiles run on CTA pairs (one MMA of
+  // 256 x 256 over two SMs, gemm_pair.cuh) unless DFLASH_GEMM_PAIR=0 when the
+  // handle is created
+  bool gemm_pair = [] {
+    const char* e = std::getenv("DFLASH_GEMM_PAIR");
+    return !(e && e[0] == '0');
+  }();
+  // two-CTA clusters of each pair-GEMM instantiation that can be resident at
+  // once (occupancy query, per kernel)
+  std::map<const void*, int> pair_clusters;
   std::vector<cudaEvent_t> prof_events;
   size_t prof_next = 0;
   std::vector<int> prof_kind;
@@ -495,7 +506,10 @@ cudaError_t set_gemm_attr() {
 
 template <class Epi>
 cudaError_t set_gemm_attrs_all() {
-  cudaError_t e = cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(gemm_pair_kernel<Epi>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       kGemmSmemLimit);
+  if (e != cudaSuccess) return e;
   if constexpr (256 % Epi::kGroup == 0)
     if ((e = set_gemm_attr<256, Epi>()) != cudaSuccess) return e;
   if constexpr (128 % Epi::kGroup == 0)
@@ -565,6 +579,92 @@ const int* gemm_cluster_caps(dflash_handle* h, int bn, int smem) {
   return nullptr;
 }
 
+// True when a plan of whole 256-wide tiles over several 128-row M tiles (no
+// stream-K, no cluster split-K, not the staged few-row epilogue) can run on
+// CTA pairs instead.
+bool gemm_pair_plan(const GemmPlan& pl) {
+  return !pl.stream_k && pl.cluster_s == 1 && !gemm_staged(pl.a_rows) && pl.BN == kPairBN &&
+         pl.m_tiles >= 2 && pl.nacc == 1;
+}
+
+// Two-CTA clusters of gemm_pair_kernel<Epi> with `smem` bytes each that fit
+// on the GPU at once (cached per handle); 0 if the query fails.
+template <class Epi>
+int gemm_pair_capacity(dflash_handle* h, int smem) {
+  const void* key = reinterpret_cast<const void*>(gemm_pair_kernel<Epi>);
+  std::lock_guard<std::mutex> lk(h->mu);
+  auto it = h->pair_clusters.find(key);
+  if (it != h->pair_clusters.end()) return it->second;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2);
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, gemm_pair_kernel<Epi>, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    n = 0;
+  }
+  h->pair_clusters.emplace(key, n);
+  return n;
+}
+
+// The whole-tile plan `pl` on CTA pairs: 256 x 256 tiles, one cluster of two
+// CTAs per pair of SMs walking them; W boxes of 128 rows (each CTA loads its
+// half of a tile's W rows).
+template <class Epi>
+dflash_status run_gemm_pair(dflash_handle* h, int kind, bool f16, bool w_packed, const void* A,
+                            int M, int K, const void* Wt, int N, const Epi& epi,
+                            const GemmPlan& pl, cudaStream_t st) {
+  const int stages = gemm_pair_max_stages();
+  const int smem = gemm_pair_smem_bytes(stages);
+  CUtensorMap ta, tw;
+  if (!h->tmap(&ta, A, M, K, kPairRows, f16)) return DFLASH_ERR_CUDA;
+  if (w_packed) {
+    if (!h->tmap(&tw, Wt, static_cast<uint64_t>(cdiv(N, kPackRows)) * pl.k_blocks * kPackRows,
+                 kGemmBK, kPairRows, f16))
+      return DFLASH_ERR_CUDA;
+  } else if (!h->tmap(&tw, Wt, N, K, kPairRows, f16)) {
+    return DFLASH_ERR_CUDA;
+  }
+  GemmParams gp{};
+  gp.M = M;
+  gp.N = N;
+  gp.K = K;
+  gp.m_tiles = cdiv(M, 2 * kPairRows);
+  gp.n_tiles = cdiv(N, kPairBN);
+  gp.k_blocks = pl.k_blocks;
+  gp.tiles = gp.m_tiles * gp.n_tiles;
+  gp.stream_k = 0;
+  gp.cluster_s = 2;
+  gp.ipc = pl.k_blocks;
+  gp.total_iters = gp.tiles * pl.k_blocks;
+  gp.nacc = 1;
+  gp.nbuf = 2;
+  gp.tmem_cols = kPairTmemCols;
+  gp.a_rows = kPairRows;
+  gp.stages = stages;
+  gp.f16 = f16 ? 1 : 0;
+  gp.w_packed = w_packed ? 1 : 0;
+  gp.slot_rows = 0;
+  gp.partials = nullptr;
+  gp.counters = h->counters;
+  gp.err = h->dev_err;
+  int clusters = gemm_pair_capacity<Epi>(h, smem);
+  if (clusters <= 0) clusters = h->num_sms / 2;
+  clusters = std::max(1, std::min(clusters, gp.tiles));
+  LaunchScope scope(h, kind, st);
+  launch_kc(h->pdl, 2, gemm_pair_kernel<Epi>, dim3(2 * clusters), dim3(kGemmThreads), smem, st,
+            ta, tw, gp, epi);
+  return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ERR_CUDA;
+}
+
 // D = A[M, K] * W[N, K]^T with epilogue `epi`.  `partials` must hold
 // plan.partial_bytes.
 template <class Epi>
@@ -585,6 +685,8 @@ dflash_status run_gemm(dflash_handle* h, int kind, bool f16, bool w_packed, cons
   }
   if (pl.stream_k && pl.tiles > kCounterSlots - 2) return DFLASH_ERR_UNSUPPORTED_SHAPE;
   if (pl.partial_bytes > partial_cap) return DFLASH_ERR_WORKSPACE;
+  if (h->gemm_pair && !force_bn && !force_splits && gemm_pair_plan(pl))
+    return run_gemm_pair(h, kind, f16, w_packed, A, M, K, Wt, N, epi, pl, st);
   CUtensorMap ta, tw;
   if (!h->tmap(&ta, A, M, K, pl.a_rows, f16)) return DFLASH_ERR_CUDA;
   if (w_packed) {

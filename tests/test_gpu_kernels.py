@@ -56,6 +56,13 @@ GEMM_CASES = [
     (512, 4096, 4096, 256, 1),
     (1000, 2080, 640, 0, 0),
     (2048, 1024, 1024, 256, 1),
+    # whole 256-wide tiles over several M tiles: CTA pairs (256 x 256 tiles),
+    # each cluster walking several tiles; ragged M and N; a pair whose second
+    # half lies wholly past M (300 rows)
+    (1024, 4096, 4096, 0, 0),
+    (2048, 6144, 1024, 0, 0),
+    (1000, 8224, 704, 0, 0),
+    (300, 6400, 256, 0, 0),
 ]
 
 
@@ -73,6 +80,29 @@ def test_linear_matches_float64_matmul(tiny, M, N, K, bn, splits):
     scale = ref.abs().max().item()
     assert err <= 2e-5 * scale + 1e-6, (err, scale)
     assert h.check_device_errors() == 0
+
+
+def test_linear_pair_and_single_sm_agree(monkeypatch, tiny):
+    """The same many-row product through CTA pairs (default) and through the
+    one-SM kernel (DFLASH_GEMM_PAIR=0 when the handle is created): both within
+    the float64 bound, and within a few fp32 ulps of each other."""
+    monkeypatch.setenv("DFLASH_GEMM_PAIR", "0")
+    cfg = tiny[0]
+    single = DFlash(cfg, weights_to(tiny[1], DEV), max_position=256)
+    try:
+        g = torch.Generator().manual_seed(11)
+        A = torch.randn(700, 1024, generator=g).to(torch.bfloat16)
+        W = (0.05 * torch.randn(5024, 1024, generator=g)).to(torch.bfloat16)
+        ref = A.double() @ W.double().T
+        a = tiny[2].linear(A.to(DEV), W.to(DEV)).cpu().double()
+        b = single.linear(A.to(DEV), W.to(DEV)).cpu().double()
+        scale = ref.abs().max().item()
+        for got in (a, b):
+            assert (got - ref).abs().max().item() <= 2e-5 * scale + 1e-6
+        assert (a - b).abs().max().item() <= 1e-6 * scale
+        assert tiny[2].check_device_errors() == 0 and single.check_device_errors() == 0
+    finally:
+        single.close()
 
 
 def test_linear_split_k_is_deterministic(tiny):
