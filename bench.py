@@ -46,11 +46,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # dram__bytes_write.sum) for the kernel family that dominates a workload,
 # keyed by the digest of the kernel sources it was measured on.
 TRAFFIC = {
-    # attention of the batch-128, 8k-32k-context step, scaled from one launch on a
-    # 16-request case of the same context distribution (1.2523 GB read + 24.4 MB
-    # written for 1.2525 GB of algorithmic bytes: ratio 1.0193) to the launch's
-    # algorithmic bytes
-    ("qwen3_b128_ctx8192_32768", "attention"): {"ratio_to_algorithmic": 1.0193,
+    # attention of the batch-128, 8k-32k-context step, scaled from one launch of
+    # `bench.py --ncu-case attention` (16 requests of the same context
+    # distribution: 1.3737 GB read + 29.4 MB written for 1.3738 GB of
+    # algorithmic bytes, ratio 1.0214) to the launch's algorithmic bytes
+    ("qwen3_b128_ctx8192_32768", "attention"): {"ratio_to_algorithmic": 1.0214,
                                                 "digest": "fec19f3b5522f0a2"},
 }
 
@@ -481,6 +481,7 @@ def extra_measurements(st, peaks) -> dict:
     out["prepare_proposal_inputs"] = {"rows": int(tp.numel()), "us": t * 1e6}
     out["spec_step_graph"] = spec_step_graph(st)
     out["vocab_parallel_propose"] = vocab_parallel_propose(st)
+    out["head_parallel_propose"] = head_parallel_propose(st)
     return out
 
 
@@ -510,6 +511,41 @@ def vocab_parallel_propose(st, parts_list=(1, 2, 4, 8)) -> dict:
             if hs is not st.h:
                 hs.close()
         out[str(parts)] = {"vocab_rows": count, "us": t * 1e6}
+    return out
+
+
+def head_parallel_propose(st, sizes=(2, 4, 8)) -> dict:
+    """One rank's share of a head-parallel proposal (dflash_propose_tp on the
+    rank-0 shard of `size`: its kv heads with their query groups, its MLP
+    features and its vocabulary shard), on that rank's own K/V pool of the same
+    pages.  The exchange hook is a no-op here (one GPU: the two all-reduces per
+    layer are not timed), so the figure is the rank's compute alone."""
+    from block_diffusion_speculative_propose_b200 import DFlash
+    from block_diffusion_speculative_propose_b200.tensor_parallel import vocab_shards
+    c, dev, B, K = st.cfg, st.dev, st.B, st.K
+    out = {}
+    args = (st.inp["bonus"], st.inp["seq_lens"], st.inp["block_table"])
+    for size in sizes:
+        if c["n_kv_heads"] % size:
+            continue
+        shard = DFlash(c, st.W, device=dev.index, max_position=st.h.max_position,
+                       tp=(0, size), vocab_shard=vocab_shards(c["vocab"], size)[0])
+        kc = vc = None
+        try:
+            shape = (st.kc[0].shape[0], c["n_kv_heads"] // size) + tuple(st.kc[0].shape[2:])
+            kc = [torch.empty(shape, dtype=torch.bfloat16, device=dev) for _ in st.kc]
+            vc = [torch.empty(shape, dtype=torch.bfloat16, device=dev) for _ in st.vc]
+            for x in kc + vc:
+                x.normal_()
+            keys = torch.empty(B, K, dtype=torch.int64, device=dev)
+            t = graph_seconds(lambda: shard.propose_tp(*args, kc, vc, lambda d, n, s: 0,
+                                                       draft_keys=keys), dev, reps=4)
+            out[str(size)] = {"kv_heads": c["n_kv_heads"] // size,
+                              "intermediate": c["intermediate"] // size, "us": t * 1e6}
+        finally:
+            shard.close()
+            del kc, vc
+            torch.cuda.empty_cache()
     return out
 
 
