@@ -63,6 +63,10 @@ GEMM_CASES = [
     (2048, 6144, 1024, 0, 0),
     (1000, 8224, 704, 0, 0),
     (300, 6400, 256, 0, 0),
+    # 256 x 128 pair tiles (too few 256-wide ones to fill the SMs): 512 rows
+    # against a 4096-wide output, and ragged M and N in place of a stream-K plan
+    (512, 4096, 1024, 0, 0),
+    (500, 4128, 704, 0, 0),
 ]
 
 
