@@ -506,10 +506,15 @@ cudaError_t set_gemm_attr() {
 
 template <class Epi>
 cudaError_t set_gemm_attrs_all() {
-  cudaError_t e = cudaFuncSetAttribute(gemm_pair_kernel<Epi>,
+  cudaError_t e = cudaFuncSetAttribute(gemm_pair_kernel<256, Epi>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        kGemmSmemLimit);
   if (e != cudaSuccess) return e;
+  if constexpr (128 % Epi::kGroup == 0)
+    if ((e = cudaFuncSetAttribute(gemm_pair_kernel<128, Epi>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  kGemmSmemLimit)) != cudaSuccess)
+      return e;
   if constexpr (256 % Epi::kGroup == 0)
     if ((e = set_gemm_attr<256, Epi>()) != cudaSuccess) return e;
   if constexpr (128 % Epi::kGroup == 0)
@@ -579,19 +584,34 @@ const int* gemm_cluster_caps(dflash_handle* h, int bn, int smem) {
   return nullptr;
 }
 
-// True when a plan of whole 256-wide tiles over several 128-row M tiles (no
-// stream-K, no cluster split-K, not the staged few-row epilogue) can run on
-// CTA pairs instead.
-bool gemm_pair_plan(const GemmPlan& pl) {
-  return !pl.stream_k && pl.cluster_s == 1 && !gemm_staged(pl.a_rows) && pl.BN == kPairBN &&
-         pl.m_tiles >= 2 && pl.nacc == 1;
+// Tile width of the CTA-pair kernel for a plan over several 128-row M tiles
+// (not the staged few-row epilogue, no cluster split-K), or 0 to keep the
+// one-SM plan.  256-wide pair tiles read half the operand bytes per MMA cycle
+// that a one-SM 128 x 256 tile does; 256 x 128 pair tiles read as many as the
+// one-SM tile (about 3/4 of the wide pair's rate, as measured on the draft
+// GEMMs) but are twice as many, so they are taken only when that fills the
+// SMs enough better (e.g. the O and down projections of 512 rows: 32 wide
+// pair tiles for 74 pairs of SMs, or 64 narrow ones).  A one-SM stream-K
+// plan (too few whole tiles) is replaced only when the pair tiles fill at
+// least half of the SMs.
+int gemm_pair_width(const GemmPlan& pl, int M, int N, int group, int num_sms) {
+  if (pl.cluster_s != 1 || gemm_staged(pl.a_rows) || pl.m_tiles < 2) return 0;
+  const int ncl = std::max(1, num_sms / 2);
+  auto fill = [&](int bn) {
+    const int tiles = cdiv(M, 2 * kPairRows) * cdiv(N, bn);
+    return static_cast<double>(tiles) / (static_cast<double>(cdiv(tiles, ncl)) * ncl);
+  };
+  const double wide = fill(256), narrow = 0.75 * fill(128);
+  const int bn = (group <= 128 && narrow > wide + 0.05) ? 128 : 256;
+  if (pl.stream_k && std::max(wide, narrow) < 0.5) return 0;
+  return bn;
 }
 
-// Two-CTA clusters of gemm_pair_kernel<Epi> with `smem` bytes each that fit
-// on the GPU at once (cached per handle); 0 if the query fails.
-template <class Epi>
+// Two-CTA clusters of gemm_pair_kernel<BN, Epi> with `smem` bytes each that
+// fit on the GPU at once (cached per handle); 0 if the query fails.
+template <int BN, class Epi>
 int gemm_pair_capacity(dflash_handle* h, int smem) {
-  const void* key = reinterpret_cast<const void*>(gemm_pair_kernel<Epi>);
+  const void* key = reinterpret_cast<const void*>(gemm_pair_kernel<BN, Epi>);
   std::lock_guard<std::mutex> lk(h->mu);
   auto it = h->pair_clusters.find(key);
   if (it != h->pair_clusters.end()) return it->second;
@@ -607,7 +627,7 @@ int gemm_pair_capacity(dflash_handle* h, int smem) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, gemm_pair_kernel<Epi>, &cfg) != cudaSuccess) {
+  if (cudaOccupancyMaxActiveClusters(&n, gemm_pair_kernel<BN, Epi>, &cfg) != cudaSuccess) {
     cudaGetLastError();
     n = 0;
   }
@@ -615,22 +635,23 @@ int gemm_pair_capacity(dflash_handle* h, int smem) {
   return n;
 }
 
-// The whole-tile plan `pl` on CTA pairs: 256 x 256 tiles, one cluster of two
-// CTAs per pair of SMs walking them; W boxes of 128 rows (each CTA loads its
-// half of a tile's W rows).
-template <class Epi>
+// The plan `pl` on CTA pairs: 256 x BN tiles, one cluster of two CTAs per
+// pair of SMs walking them; W boxes of BN / 2 rows (each CTA loads its half of
+// a tile's W rows).
+template <int BN, class Epi>
 dflash_status run_gemm_pair(dflash_handle* h, int kind, bool f16, bool w_packed, const void* A,
                             int M, int K, const void* Wt, int N, const Epi& epi,
                             const GemmPlan& pl, cudaStream_t st) {
-  const int stages = gemm_pair_max_stages();
-  const int smem = gemm_pair_smem_bytes(stages);
+  using PC = PairCfg<BN>;
+  const int stages = PC::kStages;
+  const int smem = PC::kSmem;
   CUtensorMap ta, tw;
   if (!h->tmap(&ta, A, M, K, kPairRows, f16)) return DFLASH_ERR_CUDA;
   if (w_packed) {
     if (!h->tmap(&tw, Wt, static_cast<uint64_t>(cdiv(N, kPackRows)) * pl.k_blocks * kPackRows,
-                 kGemmBK, kPairRows, f16))
+                 kGemmBK, PC::kWRows, f16))
       return DFLASH_ERR_CUDA;
-  } else if (!h->tmap(&tw, Wt, N, K, kPairRows, f16)) {
+  } else if (!h->tmap(&tw, Wt, N, K, PC::kWRows, f16)) {
     return DFLASH_ERR_CUDA;
   }
   GemmParams gp{};
@@ -638,7 +659,7 @@ dflash_status run_gemm_pair(dflash_handle* h, int kind, bool f16, bool w_packed,
   gp.N = N;
   gp.K = K;
   gp.m_tiles = cdiv(M, 2 * kPairRows);
-  gp.n_tiles = cdiv(N, kPairBN);
+  gp.n_tiles = cdiv(N, BN);
   gp.k_blocks = pl.k_blocks;
   gp.tiles = gp.m_tiles * gp.n_tiles;
   gp.stream_k = 0;
@@ -647,7 +668,7 @@ dflash_status run_gemm_pair(dflash_handle* h, int kind, bool f16, bool w_packed,
   gp.total_iters = gp.tiles * pl.k_blocks;
   gp.nacc = 1;
   gp.nbuf = 2;
-  gp.tmem_cols = kPairTmemCols;
+  gp.tmem_cols = PC::kTmemCols;
   gp.a_rows = kPairRows;
   gp.stages = stages;
   gp.f16 = f16 ? 1 : 0;
@@ -656,11 +677,11 @@ dflash_status run_gemm_pair(dflash_handle* h, int kind, bool f16, bool w_packed,
   gp.partials = nullptr;
   gp.counters = h->counters;
   gp.err = h->dev_err;
-  int clusters = gemm_pair_capacity<Epi>(h, smem);
+  int clusters = gemm_pair_capacity<BN, Epi>(h, smem);
   if (clusters <= 0) clusters = h->num_sms / 2;
   clusters = std::max(1, std::min(clusters, gp.tiles));
   LaunchScope scope(h, kind, st);
-  launch_kc(h->pdl, 2, gemm_pair_kernel<Epi>, dim3(2 * clusters), dim3(kGemmThreads), smem, st,
+  launch_kc(h->pdl, 2, gemm_pair_kernel<BN, Epi>, dim3(2 * clusters), dim3(kGemmThreads), smem, st,
             ta, tw, gp, epi);
   return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ERR_CUDA;
 }
@@ -685,8 +706,13 @@ dflash_status run_gemm(dflash_handle* h, int kind, bool f16, bool w_packed, cons
   }
   if (pl.stream_k && pl.tiles > kCounterSlots - 2) return DFLASH_ERR_UNSUPPORTED_SHAPE;
   if (pl.partial_bytes > partial_cap) return DFLASH_ERR_WORKSPACE;
-  if (h->gemm_pair && !force_bn && !force_splits && gemm_pair_plan(pl))
-    return run_gemm_pair(h, kind, f16, w_packed, A, M, K, Wt, N, epi, pl, st);
+  if (h->gemm_pair && !force_bn && !force_splits) {
+    const int pbn = gemm_pair_width(pl, M, N, Epi::kGroup, h->num_sms);
+    if (pbn == 256) return run_gemm_pair<256>(h, kind, f16, w_packed, A, M, K, Wt, N, epi, pl, st);
+    if constexpr (128 % Epi::kGroup == 0)
+      if (pbn == 128)
+        return run_gemm_pair<128>(h, kind, f16, w_packed, A, M, K, Wt, N, epi, pl, st);
+  }
   CUtensorMap ta, tw;
   if (!h->tmap(&ta, A, M, K, pl.a_rows, f16)) return DFLASH_ERR_CUDA;
   if (w_packed) {

@@ -1,11 +1,12 @@
 // gemm_pair.cuh — the many-row GEMM on CTA pairs: one tcgen05.mma with
-// cta_group::2 computes a 256 x 256 x 16 block over two SMs.
+// cta_group::2 computes a 256 x 256 x 16 (or 256 x 128 x 16) block over two SMs.
 //
 // Same product and epilogue functors as gemm_tcgen05_kernel
 // (D[m, n] = sum_k A[m, k] W[n, k], fp32 accumulation, the epilogue applied per
-// output row and column group), for plans of whole 256-wide tiles over several
-// 128-row M tiles (the proposal's GEMMs at batch >= 16, the LM head at batch
-// >= 9, the injection of >= 129 rows).
+// output row and column group), for plans of whole tiles over several 128-row
+// M tiles (the proposal's GEMMs at batch >= 16, the LM head at batch >= 9, the
+// injection of >= 129 rows).  Tiles are 256 x 256, or 256 x 128 where only the
+// narrower tiles keep the SMs busy (few rows against a narrow output).
 //
 // Why: on one SM a 128 x 256 x 16 MMA takes ~128 cycles and reads 12 KB of
 // operands from shared memory, while TMA writes the next 12 KB of the ring: about
@@ -17,11 +18,11 @@
 // 8 KB.
 //
 // A cluster of two CTAs; rank 0 leads.  In each CTA warp 0 is the TMA producer
-// for its own rows (A rows [m0 + 128 rank, +128) and W rows [n0 + 128 rank,
-// +128) of every k-block, into its own ring) and counts the bytes on the
-// leader's full barrier; warp 1 of the leader issues the MMAs and commits to
-// both CTAs' barriers at once; warps 2..5 of each CTA drain its 128
-// accumulator rows (TMEM lanes) x 256 columns and release the buffer on the
+// for its own rows (A rows [m0 + 128 rank, +128) and W rows
+// [n0 + rank BN / 2, +BN / 2) of every k-block, into its own ring) and counts
+// the bytes on the leader's full barrier; warp 1 of the leader issues the MMAs
+// and commits to both CTAs' barriers at once; warps 2..5 of each CTA drain its
+// 128 accumulator rows (TMEM lanes) x BN columns and release the buffer on the
 // leader's barrier.  Both CTAs allocate the same TMEM columns.  No TMA load
 // here multicasts: each CTA loads only the rows it holds.
 //
@@ -33,18 +34,22 @@
 
 namespace dflash {
 
-constexpr int kPairRows = 128;                           // A rows and W rows per CTA
-constexpr int kPairBN = 256;                             // output columns of a pair tile
-constexpr int kPairHalfBytes = kPairRows * kGemmBK * 2;  // one 128 x 64 operand box
-constexpr int kPairStageBytes = 2 * kPairHalfBytes;      // A and W half of one k-block
-constexpr int kPairTmemCols = 512;                       // two 256-column accumulators
+constexpr int kPairRows = 128;                           // A rows per CTA
+constexpr int kPairHalfBytes = kPairRows * kGemmBK * 2;  // one 128 x 64 A box
 
-__host__ __device__ inline int gemm_pair_smem_bytes(int stages) {
-  return 1024 + stages * kPairStageBytes + kGemmBarrierBytes;
-}
-__host__ __device__ inline int gemm_pair_max_stages() {
-  return (kGemmSmemLimit - 1024 - kGemmBarrierBytes) / kPairStageBytes;
-}
+// A pair tile is 256 rows x BN columns (BN = 256, or 128 when only the
+// narrower tiles fill the SMs); each CTA holds BN / 2 of its W rows.
+template <int BN>
+struct PairCfg {
+  static_assert(BN == 256 || BN == 128, "pair tile width");
+  static constexpr int kWRows = BN / 2;                       // W rows per CTA
+  static constexpr int kWBytes = kWRows * kGemmBK * 2;        // its W box
+  static constexpr int kStageBytes = kPairHalfBytes + kWBytes;
+  static constexpr int kTmemCols = 2 * BN;                    // two accumulators
+  static constexpr int kMaxStages = (kGemmSmemLimit - 1024 - kGemmBarrierBytes) / kStageBytes;
+  static constexpr int kStages = kMaxStages < kGemmMaxStages ? kMaxStages : kGemmMaxStages;
+  static constexpr int kSmem = 1024 + kStages * kStageBytes + kGemmBarrierBytes;
+};
 
 // Address of this CTA's shared variable at `saddr` in the CTA of cluster rank
 // `rank` (shared::cluster window).
@@ -107,15 +112,16 @@ __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m
       : "memory");
 }
 
-// p.m_tiles = 256-row pair tiles, p.n_tiles = 256-column tiles, p.tiles their
-// product (m fastest); p.stages ring depth; W boxes are 128 rows.
-template <class Epi>
+// p.m_tiles = 256-row pair tiles, p.n_tiles = BN-column tiles, p.tiles their
+// product (m fastest); p.stages ring depth; W boxes are BN / 2 rows.
+template <int BN, class Epi>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                      const __grid_constant__ CUtensorMap tmW, const GemmParams p,
                      const Epi epi) {
+  using PC = PairCfg<BN>;
   constexpr int G = Epi::kGroup;
-  static_assert(kPairBN % G == 0, "epilogue group must divide the tile width");
+  static_assert(BN % G == 0, "epilogue group must divide the tile width");
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();
@@ -126,8 +132,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                              ~static_cast<uintptr_t>(1023));
   const int stages = p.stages;
   uint8_t* sA = smem;                                   // [stages][128 x 128 B]
-  uint8_t* sW = smem + stages * kPairHalfBytes;         // [stages][128 x 128 B]
-  uint64_t* full = reinterpret_cast<uint64_t*>(sW + stages * kPairHalfBytes);
+  uint8_t* sW = smem + stages * kPairHalfBytes;         // [stages][BN / 2 x 128 B]
+  uint64_t* full = reinterpret_cast<uint64_t*>(sW + stages * PC::kWBytes);
   uint64_t* empty = full + kGemmMaxStages;
   uint64_t* tfull = empty + kGemmMaxStages;
   uint64_t* tempty = tfull + 2;
@@ -148,7 +154,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tma_prefetch_desc(&tmW);
   }
   if (warp == 1) {
-    tmem_alloc_pair(tmem_slot, kPairTmemCols);
+    tmem_alloc_pair(tmem_slot, PC::kTmemCols);
     tmem_relinquish_pair();
   }
   tc_fence_before();
@@ -170,16 +176,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int t = cl; ok && t < p.tiles; t += n_cl) {
         const int mp = t % p.m_tiles, nt = t / p.m_tiles;
         const int a_row = mp * 2 * kPairRows + static_cast<int>(rank) * kPairRows;
-        const int w_tile = nt * 2 + static_cast<int>(rank);   // 128-row W tile index
+        const int w_tile = nt * 2 + static_cast<int>(rank);   // BN / 2-row W tile index
         for (int kb = 0; kb < p.k_blocks; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, p.err)) {
             ok = false;
             break;
           }
-          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2u * kPairStageBytes);
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2u * PC::kStageBytes);
           const uint32_t fb = full_lead + stage * 8u;
-          tma_load_2d_pair(sW + stage * kPairHalfBytes, &tmW, fb, w_x(p, kb),
-                           w_y<kPairRows>(p, w_tile, kb), pol_w);
+          tma_load_2d_pair(sW + stage * PC::kWBytes, &tmW, fb, w_x(p, kb),
+                           w_y<PC::kWRows>(p, w_tile, kb), pol_w);
           tma_load_2d_pair(sA + stage * kPairHalfBytes, &tmA, fb, kb * kGemmBK, a_row, pol_a);
           if (++stage == static_cast<uint32_t>(stages)) {
             stage = 0;
@@ -200,13 +206,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (leader)
     if (rank == 0 && lane == 0) {
-      const uint32_t idesc = umma_idesc_f32acc(2 * kPairRows, kPairBN, p.f16 != 0);
+      const uint32_t idesc = umma_idesc_f32acc(2 * kPairRows, BN, p.f16 != 0);
       uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
       bool ok = true;
       for (int t = cl; ok && t < p.tiles; t += n_cl) {
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, p.err)) break;
         tc_fence_after();
-        const uint32_t d = tmem_base + acc * kPairBN;
+        const uint32_t d = tmem_base + acc * BN;
         for (int kb = 0; kb < p.k_blocks; ++kb) {
           if (!mbar_wait(&full[stage], phase, p.err)) {
             ok = false;
@@ -214,7 +220,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           tc_fence_after();
           const uint64_t ad = umma_desc_sw128(smem_u32(sA + stage * kPairHalfBytes));
-          const uint64_t bd = umma_desc_sw128(smem_u32(sW + stage * kPairHalfBytes));
+          const uint64_t bd = umma_desc_sw128(smem_u32(sW + stage * PC::kWBytes));
 #pragma unroll
           for (int k = 0; k < kGemmBK / 16; ++k)
             umma_pair_f16kind(d, ad + 2 * k, bd + 2 * k, idesc, (kb > 0 || k > 0) ? 1u : 0u);
@@ -249,16 +255,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int mp = t % p.m_tiles, nt = t / p.m_tiles;
       const int m = mp * 2 * kPairRows + static_cast<int>(rank) * kPairRows + row;
       const bool row_ok = m < p.M;
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(sp * 32) << 16) + acc * kPairBN;
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(sp * 32) << 16) + acc * BN;
       typename Epi::State st;
       epi.begin(st);
 #pragma unroll 1
-      for (int g = 0; g < kPairBN / G; ++g) {
+      for (int g = 0; g < BN / G; ++g) {
         float v[G];
 #pragma unroll
         for (int c = 0; c < G / 32; ++c) tmem_ld_32x32b_x32(taddr + g * G + c * 32, v + c * 32);
         tmem_ld_wait();
-        const int n0 = nt * kPairBN + g * G;
+        const int n0 = nt * BN + g * G;
         if (row_ok && n0 < p.N) epi.apply(st, m, n0, min(G, p.N - n0), v);
       }
       epi.end(st, m, row_ok);
@@ -276,7 +282,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   cluster_sync();   // the pair's MMAs, TMEM reads and remote arrivals are over
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc_pair(tmem_base, kPairTmemCols);
+    tmem_dealloc_pair(tmem_base, PC::kTmemCols);
   }
 }
 
