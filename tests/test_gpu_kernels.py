@@ -400,6 +400,14 @@ def test_verify_bit_exact(B, K, V):
         T[0, 1, :] = 0.5                        # all-equal row -> index 0
         T[1, 0, 7] = float("nan")
         T[2, 1, :] = float("-inf")
+        T[0, 2, :] = float("nan")               # all NaN: counts as -inf -> index 0
+        T[1, 1, :] = -1.0                       # -0 ties +0 as the maximum -> lower index
+        T[1, 1, 5] = -0.0
+        T[1, 1, V - 7] = 0.0
+        T[2, 0, :] = 0.0                        # ties inside one thread's elements
+        T[2, 0, 1027 % V] = 100.0               # (indices 3 and 1027) and across chunks
+        T[2, 0, 3] = 100.0
+        T[2, 0, V - 1] = 100.0
     ref = O.verify_greedy(to_np(drafts), to_np(T))
     out, n, bonus = verify_greedy(drafts.to(DEV), T.to(DEV))
     torch.cuda.synchronize()
