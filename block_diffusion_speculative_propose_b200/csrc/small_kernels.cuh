@@ -237,13 +237,24 @@ __global__ void __launch_bounds__(256) verify_partial_kernel(
   const int beg = blockIdx.x * chunk_len;
   const int end = min(V, beg + chunk_len);
   const float* src = logits + row * static_cast<size_t>(V);
-  unsigned long long best = 0ull;
+  // Each thread visits its elements in increasing index order and keeps the
+  // first largest (strict compare: NaN never wins, so it counts as -inf; -0
+  // ties +0; ties keep the lower index); its result enters the ordered 64-bit
+  // key once.  A thread that sees only -inf / NaN reports -inf at its first
+  // index, which is what the key order picks among them.
+  float bv = -INFINITY;
+  int bi = -1;
+  auto take = [&](float v, int j) {
+    const bool gt = v > bv;
+    bv = gt ? v : bv;
+    bi = gt ? j : bi;
+  };
   if ((V & 3) == 0) {
-    // four 16-byte loads in flight per thread (a row is streamed once, so the
-    // loads, not the compares, set the pace)
+    // four 16-byte loads in flight per thread (a row is streamed once)
     constexpr int U = 4;
     const int step = blockDim.x * 4;
     int j = beg + threadIdx.x * 4;
+    if (j < end) bi = j;
     for (; j + (U - 1) * step < end; j += U * step) {
       float4 v[U];
 #pragma unroll
@@ -251,35 +262,25 @@ __global__ void __launch_bounds__(256) verify_partial_kernel(
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int jj = j + u * step;
-        unsigned long long k;
-        k = argmax_key(v[u].x, jj);
-        best = k > best ? k : best;
-        k = argmax_key(v[u].y, jj + 1);
-        best = k > best ? k : best;
-        k = argmax_key(v[u].z, jj + 2);
-        best = k > best ? k : best;
-        k = argmax_key(v[u].w, jj + 3);
-        best = k > best ? k : best;
+        take(v[u].x, jj);
+        take(v[u].y, jj + 1);
+        take(v[u].z, jj + 2);
+        take(v[u].w, jj + 3);
       }
     }
     for (; j < end; j += step) {
       const float4 v = __ldcs(reinterpret_cast<const float4*>(src + j));
-      unsigned long long k;
-      k = argmax_key(v.x, j);
-      best = k > best ? k : best;
-      k = argmax_key(v.y, j + 1);
-      best = k > best ? k : best;
-      k = argmax_key(v.z, j + 2);
-      best = k > best ? k : best;
-      k = argmax_key(v.w, j + 3);
-      best = k > best ? k : best;
+      take(v.x, j);
+      take(v.y, j + 1);
+      take(v.z, j + 2);
+      take(v.w, j + 3);
     }
   } else {
-    for (int j = beg + threadIdx.x; j < end; j += blockDim.x) {
-      const unsigned long long k = argmax_key(__ldcs(src + j), j);
-      best = k > best ? k : best;
-    }
+    int j = beg + threadIdx.x;
+    if (j < end) bi = j;
+    for (; j < end; j += blockDim.x) take(__ldcs(src + j), j);
   }
+  unsigned long long best = bi >= 0 ? argmax_key(bv, static_cast<uint32_t>(bi)) : 0ull;
   best = warp_max_u64(best);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (lane == 0) red[warp] = best;
