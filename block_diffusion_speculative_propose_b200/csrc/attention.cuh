@@ -417,50 +417,69 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const AttnParams p) {
   auto row_of = [&](int s) {
     return ((static_cast<size_t>(s) * p.B + b) * p.Hkv + h) * p.R + r;
   };
-  float mmax = -INFINITY;
-  for (int s = lane; s < ns; s += 32) mmax = fmaxf(mmax, p.part_ml[row_of(s) * 2]);
+  // The (m, l) pairs of the first 32 splits are read lane-parallel and the
+  // first kGroup splits' rows are requested at the same time, before the
+  // maximum is known, so that a row with up to kGroup splits costs one round
+  // trip to memory; more splits follow in groups of kGroup, in index order.
+  constexpr int kGroup = 8;
+  auto load_row = [&](int s, float* v) {
+    const float* src = p.part_o + row_of(s) * D + lane * PER;
+    if constexpr (PER == 4) {
+      const float4 q = *reinterpret_cast<const float4*>(src);
+      v[0] = q.x;
+      v[1] = q.y;
+      v[2] = q.z;
+      v[3] = q.w;
+    } else {
+      const float2 q = *reinterpret_cast<const float2*>(src);
+      v[0] = q.x;
+      v[1] = q.y;
+    }
+  };
+  float2 ml0 = make_float2(-INFINITY, 0.f);
+  if (lane < ns) ml0 = *reinterpret_cast<const float2*>(p.part_ml + row_of(lane) * 2);
+  float v[kGroup][PER];
+#pragma unroll
+  for (int u = 0; u < kGroup; ++u) {
+    if (u < ns) {
+      load_row(u, v[u]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < PER; ++e) v[u][e] = 0.f;
+    }
+  }
+  float mmax = ml0.x;
+  for (int s = lane + 32; s < ns; s += 32) mmax = fmaxf(mmax, p.part_ml[row_of(s) * 2]);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) mmax = fmaxf(mmax, __shfl_xor_sync(0xffffffffu, mmax, off));
   float acc[PER];
 #pragma unroll
-  for (int j = 0; j < PER; ++j) acc[j] = 0.f;
+  for (int e = 0; e < PER; ++e) acc[e] = 0.f;
   float l = 0.f;
   for (int s0 = 0; s0 < ns; s0 += 32) {
     float w = 0.f, wl = 0.f;
     if (s0 + lane < ns) {
-      const float2 ml = *reinterpret_cast<const float2*>(p.part_ml + row_of(s0 + lane) * 2);
+      const float2 ml = s0 == 0 ? ml0
+                                : *reinterpret_cast<const float2*>(p.part_ml + row_of(s0 + lane) * 2);
       w = exp2f(ml.x - mmax);
       wl = w * ml.y;
     }
     l += wl;
     const int cnt = min(32, ns - s0);
-    // four splits' loads in flight at a time; past-the-end slots reread the
-    // last split with weight 0
-    for (int j = 0; j < cnt; j += 4) {
-      float ws[4];
-      float v[4][PER];
+    for (int j = 0; j < cnt; j += kGroup) {
+      if (s0 > 0 || j > 0) {
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int jj = min(j + u, cnt - 1);
-        const float wsu = __shfl_sync(0xffffffffu, w, jj);
-        ws[u] = (j + u < cnt) ? wsu : 0.f;
-        const float* src = p.part_o + row_of(s0 + jj) * D + lane * PER;
-        if constexpr (PER == 4) {
-          const float4 q = *reinterpret_cast<const float4*>(src);
-          v[u][0] = q.x;
-          v[u][1] = q.y;
-          v[u][2] = q.z;
-          v[u][3] = q.w;
-        } else {
-          const float2 q = *reinterpret_cast<const float2*>(src);
-          v[u][0] = q.x;
-          v[u][1] = q.y;
-        }
+        for (int u = 0; u < kGroup; ++u)
+          if (j + u < cnt) load_row(s0 + j + u, v[u]);
       }
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
+      for (int u = 0; u < kGroup; ++u) {
+        const float wsu = __shfl_sync(0xffffffffu, w, (j + u) & 31);
+        if (j + u < cnt) {
 #pragma unroll
-        for (int e = 0; e < PER; ++e) acc[e] += ws[u] * v[u][e];
+          for (int e = 0; e < PER; ++e) acc[e] += wsu * v[u][e];
+        }
+      }
     }
   }
 #pragma unroll
