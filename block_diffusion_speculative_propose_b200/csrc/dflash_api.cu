@@ -394,6 +394,12 @@ struct dflash_handle {
     const char* e = std::getenv("DFLASH_GEMM_PAIR");
     return !(e && e[0] == '0');
   }();
+  // few wide pair tiles with a long K split over two pairs (a cluster of four)
+  // unless DFLASH_GEMM_SPLIT=0 when the handle is created
+  bool gemm_split = [] {
+    const char* e = std::getenv("DFLASH_GEMM_SPLIT");
+    return !(e && e[0] == '0');
+  }();
   // two-CTA clusters of each pair-GEMM instantiation that can be resident at
   // once (occupancy query, per kernel)
   std::map<const void*, int> pair_clusters;
@@ -506,12 +512,16 @@ cudaError_t set_gemm_attr() {
 
 template <class Epi>
 cudaError_t set_gemm_attrs_all() {
-  cudaError_t e = cudaFuncSetAttribute(gemm_pair_kernel<256, Epi>,
+  cudaError_t e = cudaFuncSetAttribute(gemm_pair_kernel<256, 1, Epi>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        kGemmSmemLimit);
   if (e != cudaSuccess) return e;
+  if ((e = cudaFuncSetAttribute(gemm_pair_kernel<256, 2, Epi>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemLimit)) !=
+      cudaSuccess)
+    return e;
   if constexpr (128 % Epi::kGroup == 0)
-    if ((e = cudaFuncSetAttribute(gemm_pair_kernel<128, Epi>,
+    if ((e = cudaFuncSetAttribute(gemm_pair_kernel<128, 1, Epi>,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   kGemmSmemLimit)) != cudaSuccess)
       return e;
@@ -594,40 +604,62 @@ const int* gemm_cluster_caps(dflash_handle* h, int bn, int smem) {
 // pair tiles for 74 pairs of SMs, or 64 narrow ones).  A one-SM stream-K
 // plan (too few whole tiles) is replaced only when the pair tiles fill at
 // least half of the SMs.
-int gemm_pair_width(const GemmPlan& pl, int M, int N, int group, int num_sms) {
-  if (pl.cluster_s != 1 || gemm_staged(pl.a_rows) || pl.m_tiles < 2) return 0;
+// A third option for few wide tiles with a long K (>= 96 k-blocks, so that
+// each half still amortises the reduction): split K over two pairs (a cluster
+// of four, one tile per cluster; the second pair's partial reduced through
+// distributed shared memory), taken when the tiles fit one round as split
+// units and that fills the SMs enough better (0.85 of the wide rate for the
+// reduction).  Measured at 512 rows: down (K = 12288, 32 wide tiles -> 64
+// pairs) 0.48 -> 0.61 of the sustained bf16 figure, fc 0.29 -> 0.44; O
+// (K = 4096) lost 0.33 -> 0.31, hence the K floor.
+struct PairChoice {
+  int bn = 0, ks = 1;   // bn = 0: keep the one-SM plan
+};
+PairChoice gemm_pair_choice(const GemmPlan& pl, int M, int N, int group, int num_sms,
+                            int split_cap) {
+  PairChoice c;
+  if (pl.cluster_s != 1 || gemm_staged(pl.a_rows) || pl.m_tiles < 2) return c;
   const int ncl = std::max(1, num_sms / 2);
   auto fill = [&](int bn) {
     const int tiles = cdiv(M, 2 * kPairRows) * cdiv(N, bn);
     return static_cast<double>(tiles) / (static_cast<double>(cdiv(tiles, ncl)) * ncl);
   };
+  const int wide_tiles = cdiv(M, 2 * kPairRows) * cdiv(N, 256);
   const double wide = fill(256), narrow = 0.75 * fill(128);
-  const int bn = (group <= 128 && narrow > wide + 0.05) ? 128 : 256;
-  if (pl.stream_k && std::max(wide, narrow) < 0.5) return 0;
-  return bn;
+  const double split = (pl.k_blocks >= 96 && wide_tiles <= split_cap)
+                           ? 0.85 * static_cast<double>(2 * wide_tiles) / ncl : 0.0;
+  const double best = std::max(wide, std::max(narrow, split));
+  if (pl.stream_k && best < 0.5) return c;
+  if (split > wide + 0.05 && split >= narrow) {
+    c.bn = 256;
+    c.ks = 2;
+  } else {
+    c.bn = (group <= 128 && narrow > wide + 0.05) ? 128 : 256;
+  }
+  return c;
 }
 
-// Two-CTA clusters of gemm_pair_kernel<BN, Epi> with `smem` bytes each that
-// fit on the GPU at once (cached per handle); 0 if the query fails.
-template <int BN, class Epi>
+// Clusters of 2 KS CTAs of gemm_pair_kernel<BN, KS, Epi> with `smem` bytes each
+// that fit on the GPU at once (cached per handle); 0 if the query fails.
+template <int BN, int KS, class Epi>
 int gemm_pair_capacity(dflash_handle* h, int smem) {
-  const void* key = reinterpret_cast<const void*>(gemm_pair_kernel<BN, Epi>);
+  const void* key = reinterpret_cast<const void*>(gemm_pair_kernel<BN, KS, Epi>);
   std::lock_guard<std::mutex> lk(h->mu);
   auto it = h->pair_clusters.find(key);
   if (it != h->pair_clusters.end()) return it->second;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2);
   cfg.blockDim = dim3(kGemmThreads);
   cfg.dynamicSmemBytes = smem;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.x = 2 * KS;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  cfg.gridDim = dim3(2 * KS);
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, gemm_pair_kernel<BN, Epi>, &cfg) != cudaSuccess) {
+  if (cudaOccupancyMaxActiveClusters(&n, gemm_pair_kernel<BN, KS, Epi>, &cfg) != cudaSuccess) {
     cudaGetLastError();
     n = 0;
   }
@@ -638,7 +670,7 @@ int gemm_pair_capacity(dflash_handle* h, int smem) {
 // The plan `pl` on CTA pairs: 256 x BN tiles, one cluster of two CTAs per
 // pair of SMs walking them; W boxes of BN / 2 rows (each CTA loads its half of
 // a tile's W rows).
-template <int BN, class Epi>
+template <int BN, int KS, class Epi>
 dflash_status run_gemm_pair(dflash_handle* h, int kind, bool f16, bool w_packed, const void* A,
                             int M, int K, const void* Wt, int N, const Epi& epi,
                             const GemmPlan& pl, cudaStream_t st) {
@@ -663,7 +695,7 @@ dflash_status run_gemm_pair(dflash_handle* h, int kind, bool f16, bool w_packed,
   gp.k_blocks = pl.k_blocks;
   gp.tiles = gp.m_tiles * gp.n_tiles;
   gp.stream_k = 0;
-  gp.cluster_s = 2;
+  gp.cluster_s = 2 * KS;
   gp.ipc = pl.k_blocks;
   gp.total_iters = gp.tiles * pl.k_blocks;
   gp.nacc = 1;
@@ -677,11 +709,13 @@ dflash_status run_gemm_pair(dflash_handle* h, int kind, bool f16, bool w_packed,
   gp.partials = nullptr;
   gp.counters = h->counters;
   gp.err = h->dev_err;
-  int clusters = gemm_pair_capacity<BN, Epi>(h, smem);
-  if (clusters <= 0) clusters = h->num_sms / 2;
+  int clusters = gemm_pair_capacity<BN, KS, Epi>(h, smem);
+  if (clusters <= 0) clusters = h->num_sms / (2 * KS);
   clusters = std::max(1, std::min(clusters, gp.tiles));
+  if (KS == 2) clusters = gp.tiles;   // one tile per cluster (the planner keeps it to one round)
   LaunchScope scope(h, kind, st);
-  launch_kc(h->pdl, 2, gemm_pair_kernel<BN, Epi>, dim3(2 * clusters), dim3(kGemmThreads), smem, st,
+  launch_kc(h->pdl, 2 * KS, gemm_pair_kernel<BN, KS, Epi>, dim3(2 * KS * clusters),
+            dim3(kGemmThreads), smem, st,
             ta, tw, gp, epi);
   return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ERR_CUDA;
 }
@@ -707,11 +741,15 @@ dflash_status run_gemm(dflash_handle* h, int kind, bool f16, bool w_packed, cons
   if (pl.stream_k && pl.tiles > kCounterSlots - 2) return DFLASH_ERR_UNSUPPORTED_SHAPE;
   if (pl.partial_bytes > partial_cap) return DFLASH_ERR_WORKSPACE;
   if (h->gemm_pair && !force_bn && !force_splits) {
-    const int pbn = gemm_pair_width(pl, M, N, Epi::kGroup, h->num_sms);
-    if (pbn == 256) return run_gemm_pair<256>(h, kind, f16, w_packed, A, M, K, Wt, N, epi, pl, st);
+    const int cap = h->gemm_split ? gemm_pair_capacity<256, 2, Epi>(h, PairCfg<256>::kSmem) : 0;
+    const PairChoice pc = gemm_pair_choice(pl, M, N, Epi::kGroup, h->num_sms, cap);
+    if (pc.bn == 256 && pc.ks == 2)
+      return run_gemm_pair<256, 2>(h, kind, f16, w_packed, A, M, K, Wt, N, epi, pl, st);
+    if (pc.bn == 256)
+      return run_gemm_pair<256, 1>(h, kind, f16, w_packed, A, M, K, Wt, N, epi, pl, st);
     if constexpr (128 % Epi::kGroup == 0)
-      if (pbn == 128)
-        return run_gemm_pair<128>(h, kind, f16, w_packed, A, M, K, Wt, N, epi, pl, st);
+      if (pc.bn == 128)
+        return run_gemm_pair<128, 1>(h, kind, f16, w_packed, A, M, K, Wt, N, epi, pl, st);
   }
   CUtensorMap ta, tw;
   if (!h->tmap(&ta, A, M, K, pl.a_rows, f16)) return DFLASH_ERR_CUDA;

@@ -91,9 +91,8 @@ __device__ __forceinline__ void umma_pair_f16kind(uint32_t d_tmem, uint64_t a_de
       : "memory");
 }
 // Once the pair's earlier MMAs retired: arrive on the barrier at `bar`'s
-// offset in both CTAs of the pair.
-__device__ __forceinline__ void umma_pair_commit_both(uint64_t* bar) {
-  const uint16_t mask = 3;
+// offset in both CTAs of the pair (cluster ranks given by `mask`).
+__device__ __forceinline__ void umma_pair_commit_both(uint64_t* bar, uint16_t mask) {
   asm volatile(
       "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
       " [%0], %1;" ::"r"(smem_u32(bar)),
@@ -114,7 +113,14 @@ __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m
 
 // p.m_tiles = 256-row pair tiles, p.n_tiles = BN-column tiles, p.tiles their
 // product (m fastest); p.stages ring depth; W boxes are BN / 2 rows.
-template <int BN, class Epi>
+//
+// KS = 2 (split K over two pairs, a cluster of four, one tile per cluster):
+// pair q (cluster ranks 2q, 2q + 1) accumulates k-blocks [q * kh, (q+1) * kh);
+// once every MMA of the cluster has retired, each CTA of pair 1 writes its
+// fp32 accumulator rows into the idle stage ring of the CTA of pair 0 that
+// holds the same rows (distributed shared memory), and pair 0 adds them to its
+// own, in that fixed order, and runs the epilogue.
+template <int BN, int KS, class Epi>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                      const __grid_constant__ CUtensorMap tmW, const GemmParams p,
@@ -122,9 +128,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   using PC = PairCfg<BN>;
   constexpr int G = Epi::kGroup;
   static_assert(BN % G == 0, "epilogue group must divide the tile width");
+  static_assert(KS == 1 || KS == 2, "K splits");
+  constexpr int LD = BN + 4;   // padded row of the split-K partial (fp32)
+  static_assert(KS == 1 || kPairRows * LD * 4 <= 7 * PC::kStageBytes, "partial fits the ring");
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();
+  const uint32_t pr = rank & 1u;          // CTA of the pair: rows [128 pr, +128) of a tile
+  const uint32_t q = rank >> 1;           // K part (0 when KS == 1)
+  const uint32_t lead = rank & ~1u;       // the pair's leader
+  const uint16_t pair_mask = static_cast<uint16_t>(3u << lead);
+  const int kh = (p.k_blocks + KS - 1) / KS;
+  const int kb0 = static_cast<int>(q) * kh, kb1 = min(p.k_blocks, kb0 + kh);
   pdl_trigger();
 
   extern __shared__ uint8_t smem_raw[];
@@ -161,8 +176,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   cluster_sync();   // both CTAs' barriers exist before any remote arrival or byte count
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int n_cl = static_cast<int>(gridDim.x >> 1);
-  const int cl = static_cast<int>(blockIdx.x >> 1);
+  const int n_cl = static_cast<int>(gridDim.x) / (2 * KS);
+  const int cl = static_cast<int>(blockIdx.x) / (2 * KS);
+  bool epi_ok = false;   // split K: this CTA's accumulator is complete
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -170,19 +186,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       pdl_wait();
       const uint64_t pol_w = policy_evict_first();
       const uint64_t pol_a = policy_evict_last();
-      const uint32_t full_lead = cluster_addr(smem_u32(full), 0);
+      const uint32_t full_lead = cluster_addr(smem_u32(full), lead);
       uint32_t stage = 0, phase = 0;
       bool ok = true;
       for (int t = cl; ok && t < p.tiles; t += n_cl) {
         const int mp = t % p.m_tiles, nt = t / p.m_tiles;
-        const int a_row = mp * 2 * kPairRows + static_cast<int>(rank) * kPairRows;
-        const int w_tile = nt * 2 + static_cast<int>(rank);   // BN / 2-row W tile index
-        for (int kb = 0; kb < p.k_blocks; ++kb) {
+        const int a_row = mp * 2 * kPairRows + static_cast<int>(pr) * kPairRows;
+        const int w_tile = nt * 2 + static_cast<int>(pr);   // BN / 2-row W tile index
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, p.err)) {
             ok = false;
             break;
           }
-          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2u * PC::kStageBytes);
+          if (pr == 0) mbar_arrive_expect_tx(&full[stage], 2u * PC::kStageBytes);
           const uint32_t fb = full_lead + stage * 8u;
           tma_load_2d_pair(sW + stage * PC::kWBytes, &tmW, fb, w_x(p, kb),
                            w_y<PC::kWRows>(p, w_tile, kb), pol_w);
@@ -205,7 +221,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (leader)
-    if (rank == 0 && lane == 0) {
+    if (pr == 0 && lane == 0) {
       const uint32_t idesc = umma_idesc_f32acc(2 * kPairRows, BN, p.f16 != 0);
       uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
       bool ok = true;
@@ -213,7 +229,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, p.err)) break;
         tc_fence_after();
         const uint32_t d = tmem_base + acc * BN;
-        for (int kb = 0; kb < p.k_blocks; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&full[stage], phase, p.err)) {
             ok = false;
             break;
@@ -223,15 +239,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const uint64_t bd = umma_desc_sw128(smem_u32(sW + stage * PC::kWBytes));
 #pragma unroll
           for (int k = 0; k < kGemmBK / 16; ++k)
-            umma_pair_f16kind(d, ad + 2 * k, bd + 2 * k, idesc, (kb > 0 || k > 0) ? 1u : 0u);
-          umma_pair_commit_both(&empty[stage]);
+            umma_pair_f16kind(d, ad + 2 * k, bd + 2 * k, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+          umma_pair_commit_both(&empty[stage], pair_mask);
           if (++stage == static_cast<uint32_t>(stages)) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        umma_pair_commit_both(&tfull[acc]);
+        umma_pair_commit_both(&tfull[acc], pair_mask);
         if (++acc == 2u) {
           acc = 0;
           acc_phase ^= 1u;
@@ -244,7 +260,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int ew = warp - 2;
     const int sp = warp & 3;            // TMEM sub-partition this warp may read
     const int row = sp * 32 + lane;
-    const uint32_t tempty_lead = cluster_addr(smem_u32(tempty), 0);
+    const uint32_t tempty_lead = cluster_addr(smem_u32(tempty), lead);
     uint32_t acc = 0, acc_phase = 0, nseen = 0;
     for (int t = cl; t < p.tiles; t += n_cl) {
       if (ew == 0 && lane == 0)
@@ -252,8 +268,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       named_bar_sync(1, 128);
       if (!wait_flag[nseen++ & 1]) break;
       tc_fence_after();
+      if constexpr (KS == 2) {
+        epi_ok = true;   // one tile per cluster: reduced and stored below
+        break;
+      }
       const int mp = t % p.m_tiles, nt = t / p.m_tiles;
-      const int m = mp * 2 * kPairRows + static_cast<int>(rank) * kPairRows + row;
+      const int m = mp * 2 * kPairRows + static_cast<int>(pr) * kPairRows + row;
       const bool row_ok = m < p.M;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(sp * 32) << 16) + acc * BN;
       typename Epi::State st;
@@ -275,6 +295,62 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         acc = 0;
         acc_phase ^= 1u;
       }
+    }
+  }
+
+  if constexpr (KS == 2) {
+    // every MMA of the cluster has retired (each epilogue saw its tfull): the
+    // stage rings are idle and pair 1 can write its partial into pair 0's
+    float* stg = reinterpret_cast<float*>(smem);   // [128][LD] fp32, over the ring
+    const int sp = warp & 3, row = sp * 32 + lane;
+    const uint32_t taddr = tmem_base + (static_cast<uint32_t>(sp * 32) << 16);
+    tc_fence_before();
+    cluster_sync();
+    tc_fence_after();
+    if (warp >= 2 && q == 1 && epi_ok) {
+      const uint32_t dst = cluster_addr(smem_u32(stg + row * LD), rank - 2u);
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        float v[32];
+        tmem_ld_32x32b_x32(taddr + c * 32, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(
+                           dst + static_cast<uint32_t>((c * 32 + 4 * j) * 4)),
+                       "f"(v[4 * j]), "f"(v[4 * j + 1]), "f"(v[4 * j + 2]), "f"(v[4 * j + 3])
+                       : "memory");
+      }
+    }
+    tc_fence_before();
+    cluster_sync();   // pair 1's partials are in pair 0's shared memory
+    tc_fence_after();
+    if (warp >= 2 && q == 0 && epi_ok) {
+      const int t = cl;
+      const int mp = t % p.m_tiles, nt = t / p.m_tiles;
+      const int m = mp * 2 * kPairRows + static_cast<int>(pr) * kPairRows + row;
+      const bool row_ok = m < p.M;
+      const float* own = stg + row * LD;
+      typename Epi::State st;
+      epi.begin(st);
+#pragma unroll 1
+      for (int g = 0; g < BN / G; ++g) {
+        float v[G];
+#pragma unroll
+        for (int c = 0; c < G / 32; ++c) tmem_ld_32x32b_x32(taddr + g * G + c * 32, v + c * 32);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < G; j += 4) {
+          const float4 r4 = *reinterpret_cast<const float4*>(own + g * G + j);
+          v[j] += r4.x;
+          v[j + 1] += r4.y;
+          v[j + 2] += r4.z;
+          v[j + 3] += r4.w;
+        }
+        const int n0 = nt * BN + g * G;
+        if (row_ok && n0 < p.N) epi.apply(st, m, n0, min(G, p.N - n0), v);
+      }
+      epi.end(st, m, row_ok);
     }
   }
 

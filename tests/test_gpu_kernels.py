@@ -67,6 +67,10 @@ GEMM_CASES = [
     # against a 4096-wide output, and ragged M and N in place of a stream-K plan
     (512, 4096, 1024, 0, 0),
     (500, 4128, 704, 0, 0),
+    # few wide pair tiles with a long K: K split over two pairs (clusters of
+    # four, the second pair's partial reduced through distributed shared memory)
+    (512, 4096, 6144, 0, 0),
+    (500, 4128, 6144, 0, 0),
 ]
 
 
@@ -107,6 +111,32 @@ def test_linear_pair_and_single_sm_agree(monkeypatch, tiny):
         assert tiny[2].check_device_errors() == 0 and single.check_device_errors() == 0
     finally:
         single.close()
+
+
+def test_linear_pair_split_k_matches_unsplit(monkeypatch, tiny):
+    """512 rows against a 4096-wide output with K = 6144: the split-K pair plan
+    (default) and the narrow pair tiles (DFLASH_GEMM_SPLIT=0) both within the
+    float64 bound, and the split plan deterministic.  (The two accumulate the
+    6144 products in different orders and MMA shapes; the tensor cores' fp32
+    accumulation is not exactly rounded, so they are compared with float64,
+    not with each other.)"""
+    monkeypatch.setenv("DFLASH_GEMM_SPLIT", "0")
+    unsplit = DFlash(tiny[0], weights_to(tiny[1], DEV), max_position=256)
+    try:
+        g = torch.Generator().manual_seed(12)
+        A = torch.randn(512, 6144, generator=g).to(torch.bfloat16)
+        W = (0.05 * torch.randn(4096, 6144, generator=g)).to(torch.bfloat16)
+        ref = A.double() @ W.double().T
+        a = tiny[2].linear(A.to(DEV), W.to(DEV)).cpu().double()
+        a2 = tiny[2].linear(A.to(DEV), W.to(DEV)).cpu().double()
+        b = unsplit.linear(A.to(DEV), W.to(DEV)).cpu().double()
+        scale = ref.abs().max().item()
+        for got in (a, b):
+            assert (got - ref).abs().max().item() <= 2e-5 * scale + 1e-6
+        assert torch.equal(a, a2)
+        assert tiny[2].check_device_errors() == 0 and unsplit.check_device_errors() == 0
+    finally:
+        unsplit.close()
 
 
 def test_linear_split_k_is_deterministic(tiny):
