@@ -2122,6 +2122,37 @@ dflash_status dflash_plan_attention_info(int B, int n_kv_heads, int max_pages_pe
   return DFLASH_OK;
 }
 
+dflash_status dflash_plan_gemm_info(int M, int N, int K, int group, int num_sms,
+                                    int pair_split_cap, dflash_gemm_plan* out) {
+  if (!out || M <= 0 || N <= 0 || K <= 0 || K % kGemmBK || num_sms < 2 || pair_split_cap < 0 ||
+      (group != 32 && group != 64 && group != 128))
+    return DFLASH_ERR_INVALID_ARG;
+  std::array<int, 9> cap{};
+  for (int S = 2; S <= 8; ++S) cap[S] = num_sms / S;
+  GemmPlan pl = plan_gemm(M, N, K, group, num_sms);
+  if (gemm_staged(pl.a_rows) && pl.tiles <= num_sms)
+    pl = plan_gemm(M, N, K, group, num_sms, 0, 0, cap.data());
+  const PairChoice pc = gemm_pair_choice(pl, M, N, group, num_sms, pair_split_cap);
+  *out = dflash_gemm_plan{};
+  if (pc.bn) {
+    out->pair = 1;
+    out->tile_m = 2 * kPairRows;
+    out->tile_n = pc.bn;
+    out->k_splits = pc.ks;
+    out->tiles = cdiv(M, 2 * kPairRows) * cdiv(N, pc.bn);
+    out->grid = pc.ks == 2 ? 4 * out->tiles : 2 * std::min(out->tiles, num_sms / 2);
+  } else {
+    out->tile_m = kGemmBM;
+    out->tile_n = pl.BN;
+    out->k_splits = pl.cluster_s;
+    out->stream_k = pl.stream_k;
+    out->staged = gemm_staged(pl.a_rows) ? 1 : 0;
+    out->tiles = pl.tiles;
+    out->grid = pl.grid;
+  }
+  return DFLASH_OK;
+}
+
 size_t dflash_linear_workspace_bytes(const dflash_handle* h, int M, int N, int K) {
   if (!h || M <= 0 || N <= 0 || K <= 0) return 0;
   return align_up(std::max<size_t>(plan_gemm(M, N, K, 32, h->num_sms).partial_bytes, kAlign));

@@ -126,6 +126,7 @@ def lib() -> ctypes.CDLL:
         "dflash_propose_workspace_bytes": ([vp, i32, i32], sz),
         "dflash_propose_final_rows_offset": ([vp, i32, i32], sz),
         "dflash_set_wait_limit": ([i32, ctypes.c_longlong], i32),
+        "dflash_plan_gemm_info": ([i32] * 6 + [ctypes.POINTER(_GemmPlan)], i32),
         "dflash_create_tp_shard": ([ctypes.POINTER(_Config), ctypes.POINTER(_Weights), i32, i32,
                                     i32, i32, i32, ctypes.POINTER(vp)], i32),
         "dflash_propose_tp": ([vp, vp, vp, vp, i32, i32, _PP, _PP, i32, vp, vp, vp, sz, vp,
@@ -728,6 +729,20 @@ def attention_plan(B: int, n_kv_heads: int, max_pages_per_seq: int, block_size: 
                                             forced_ring, flags, ctypes.byref(out)),
            "dflash_plan_attention_info")
     return {n: getattr(out, n) for n, _ in _AttnPlan._fields_}
+
+
+class _GemmPlan(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in ("pair", "tile_m", "tile_n", "k_splits", "stream_k",
+                                            "staged", "tiles", "grid")]
+
+
+def gemm_plan(M: int, N: int, K: int, group: int = 32, num_sms: int = 148,
+              pair_split_cap: int = 37) -> Dict[str, int]:
+    """dflash_plan_gemm_info: the GEMM launch plan for this shape (host only)."""
+    out = _GemmPlan()
+    _check(lib().dflash_plan_gemm_info(M, N, K, group, num_sms, pair_split_cap,
+                                       ctypes.byref(out)), "dflash_plan_gemm_info")
+    return {n: getattr(out, n) for n, _ in _GemmPlan._fields_}
 
 
 def verify_workspace_bytes(B: int, K: int, V: int) -> int:

@@ -583,6 +583,27 @@ dflash_status dflash_plan_attention_info(int B, int n_kv_heads, int max_pages_pe
                                          int head_dim, int num_sms, int forced_ring, int flags,
                                          dflash_attention_plan* out);
 
+/* The GEMM launch plan the library takes for D[M, N] = A[M, K] W[N, K]^T
+ * with an epilogue that groups `group` output columns (32, 64 or 128), host
+ * only (no device, no allocation).  On a device the library queries how many
+ * thread-block clusters fit at once; here those capacities are parameters:
+ * clusters of S CTAs for the few-row cluster split-K are taken as
+ * num_sms / S, and pair_split_cap is the number of four-CTA clusters of the
+ * split-K pair kernel that fit (0: never split).  K must be a multiple of 64.
+ * DFLASH_ERR_INVALID_ARG for sizes out of range. */
+typedef struct dflash_gemm_plan {
+  int pair;           /* 1: CTA pairs (tcgen05.mma.cta_group::2), 0: one SM per tile */
+  int tile_m;         /* rows of a tile (256 for pairs, 128 otherwise) */
+  int tile_n;         /* columns of a tile */
+  int k_splits;       /* pairs: K split over this many pairs; one SM: cluster split-K size */
+  int stream_k;       /* one SM: (tile, k-block) iterations dealt in equal ranges */
+  int staged;         /* one SM: the few-row staged epilogue (M <= 32) */
+  int tiles;          /* output tiles */
+  int grid;           /* CTAs launched (pairs: an upper bound before the occupancy query) */
+} dflash_gemm_plan;
+dflash_status dflash_plan_gemm_info(int M, int N, int K, int group, int num_sms,
+                                    int pair_split_cap, dflash_gemm_plan* out);
+
 /* ---- a small causal target model on the device ---------------------------
  *
  * DFlash reads the target model's auxiliary hidden states (§"Target Auxiliary

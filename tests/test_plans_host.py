@@ -7,7 +7,7 @@ import itertools
 
 import pytest
 
-from block_diffusion_speculative_propose_b200.dflash import DFlashError, attention_plan
+from block_diffusion_speculative_propose_b200.dflash import DFlashError, attention_plan, gemm_plan
 
 
 def test_benchmark_workloads_plans():
@@ -71,3 +71,58 @@ def test_attention_plan_rejects_bad_sizes():
         attention_plan(0, 8, 130, 16, 4)
     with pytest.raises(DFlashError):
         attention_plan(1, 8, 0, 16, 4)
+
+
+# ----------------------------------------------------------------------------
+# GEMM plans (dflash_plan_gemm_info)
+# ----------------------------------------------------------------------------
+def test_gemm_plans_of_the_draft_step():
+    # batch 128 (2048 block rows, 1920 LM-head rows): 256 x 256 CTA-pair tiles
+    for M, N, K, g in ((2048, 6144, 4096, 128), (2048, 4096, 4096, 32), (2048, 24576, 4096, 32),
+                       (2048, 4096, 12288, 32), (1920, 151936, 4096, 32)):
+        p = gemm_plan(M, N, K, g)
+        assert (p["pair"], p["tile_m"], p["tile_n"], p["k_splits"]) == (1, 256, 256, 1), (M, N, K)
+    # batch 32 (512 rows): QKV wide pairs (48 tiles), O narrow pairs (64 tiles
+    # of 256 x 128), down and fc with K split over two pairs (32 tiles -> 64 pairs)
+    assert gemm_plan(512, 6144, 4096, 128)["tile_n"] == 256
+    p = gemm_plan(512, 4096, 4096)
+    assert (p["pair"], p["tile_n"], p["k_splits"], p["tiles"]) == (1, 128, 1, 64)
+    for M, K in ((512, 12288), (282, 20480)):
+        p = gemm_plan(M, 4096, K)
+        assert (p["pair"], p["tile_n"], p["k_splits"], p["tiles"], p["grid"]) == (1, 256, 2, 32, 128)
+    # no split when the split clusters cannot all run at once, or K is short
+    assert gemm_plan(512, 4096, 12288, pair_split_cap=20)["k_splits"] == 1
+    assert gemm_plan(512, 4096, 4096, pair_split_cap=37)["k_splits"] == 1
+    # batch 1 (16 rows): the staged one-SM kernel; few tiles -> cluster split-K,
+    # the LM head's 594 tiles -> stream-K
+    p = gemm_plan(16, 4096, 12288)
+    assert (p["pair"], p["staged"], p["k_splits"], p["grid"]) == (0, 1, 8, 128)
+    p = gemm_plan(15, 151936, 4096)
+    assert (p["pair"], p["staged"], p["stream_k"], p["grid"]) == (0, 1, 1, 148)
+
+
+@pytest.mark.parametrize("M", [1, 16, 32, 33, 128, 129, 256, 300, 512, 768, 2048])
+@pytest.mark.parametrize("N,K", [(1024, 1024), (4096, 4096), (6144, 4096), (4096, 12288),
+                                 (24576, 4096), (151936, 4096)])
+def test_gemm_plan_rules(M, N, K):
+    for g in (32, 128):
+        p = gemm_plan(M, N, K, g)
+        assert p["tiles"] == -(-M // p["tile_m"]) * -(-N // p["tile_n"])
+        if p["pair"]:
+            # pairs only for several 128-row M tiles, never the staged epilogue
+            assert M > 128 and not p["staged"] and not p["stream_k"]
+            assert p["tile_m"] == 256 and p["tile_n"] in (128, 256) and p["tile_n"] % g == 0
+            if p["k_splits"] == 2:
+                assert p["tile_n"] == 256 and K // 64 >= 96 and p["tiles"] <= 37
+                assert p["grid"] == 4 * p["tiles"]
+            else:
+                assert p["k_splits"] == 1 and p["grid"] <= 148 and p["grid"] % 2 == 0
+        else:
+            assert p["tile_m"] == 128 and p["grid"] <= 148
+            assert p["staged"] == (1 if M <= 32 else 0)
+
+
+def test_gemm_plan_rejects_bad_sizes():
+    for args in ((0, 1024, 1024), (16, 0, 1024), (16, 1024, 100), (16, 1024, 1024, 48)):
+        with pytest.raises(DFlashError):
+            gemm_plan(*args)
