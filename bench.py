@@ -52,6 +52,18 @@ TRAFFIC = {
     # algorithmic bytes, ratio 1.0216) to the launch's algorithmic bytes
     ("qwen3_b128_ctx8192_32768", "attention"): {"ratio_to_algorithmic": 1.0216,
                                                 "digest": "a57e69be73424de9"},
+    # the same for the batch-32, 512-8192-context workload (16 requests: 298.2 MB
+    # read + 18.7 MB written for 298.7 MB) and the Llama-paired batch-128 one
+    # (590.3 MB + 16.5 MB for 590.2 MB)
+    ("qwen3_b32_ctx512_8192", "attention"): {"ratio_to_algorithmic": 1.0612,
+                                             "digest": "a57e69be73424de9"},
+    ("llama_b128_ctx1024_16384", "attention"): {"ratio_to_algorithmic": 1.0282,
+                                                "digest": "a57e69be73424de9"},
+    # gate/up GEMM of the batch-1 step, one launch of `bench.py --workload
+    # qwen3_b1_ctx2048 --ncu-case gemms` (the step's shapes): 201.5 MB read +
+    # 3.5 MB written
+    ("qwen3_b1_ctx2048", "gemm_gate_up"): {"bytes_per_launch": 205062144,
+                                           "digest": "6384f9db5e3108f3"},
 }
 
 
