@@ -48,17 +48,17 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 TRAFFIC = {
     # attention of the batch-128, 8k-32k-context step, scaled from one launch of
     # `bench.py --ncu-case attention` (16 requests of the same context
-    # distribution: 1.3738 GB read + 29.7 MB written for 1.3738 GB of
-    # algorithmic bytes, ratio 1.0216) to the launch's algorithmic bytes
-    ("qwen3_b128_ctx8192_32768", "attention"): {"ratio_to_algorithmic": 1.0216,
-                                                "digest": "a57e69be73424de9"},
-    # the same for the batch-32, 512-8192-context workload (16 requests: 298.2 MB
-    # read + 18.7 MB written for 298.7 MB) and the Llama-paired batch-128 one
-    # (590.3 MB + 16.5 MB for 590.2 MB)
-    ("qwen3_b32_ctx512_8192", "attention"): {"ratio_to_algorithmic": 1.0612,
-                                             "digest": "a57e69be73424de9"},
-    ("llama_b128_ctx1024_16384", "attention"): {"ratio_to_algorithmic": 1.0282,
-                                                "digest": "a57e69be73424de9"},
+    # distribution: 1.3782 GB read + 27.4 MB written for 1.3738 GB of
+    # algorithmic bytes, ratio 1.0232) to the launch's algorithmic bytes
+    ("qwen3_b128_ctx8192_32768", "attention"): {"ratio_to_algorithmic": 1.0232,
+                                                "digest": "2f2ef01b70758d65"},
+    # the same for the batch-32, 512-8192-context workload (16 requests: 300.6 MB
+    # read + 16.4 MB written for 298.7 MB) and the Llama-paired batch-128 one
+    # (592.1 MB + 16.7 MB for 590.2 MB)
+    ("qwen3_b32_ctx512_8192", "attention"): {"ratio_to_algorithmic": 1.0614,
+                                             "digest": "2f2ef01b70758d65"},
+    ("llama_b128_ctx1024_16384", "attention"): {"ratio_to_algorithmic": 1.0316,
+                                                "digest": "2f2ef01b70758d65"},
     # gate/up GEMM of the batch-1 step, one launch of `bench.py --workload
     # qwen3_b1_ctx2048 --ncu-case gemms` (the step's shapes): 201.5 MB read +
     # 3.5 MB written

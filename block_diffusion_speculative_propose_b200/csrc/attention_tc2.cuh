@@ -20,6 +20,13 @@
 //     with M = head_dim = 128 (the full-rate shape) instead of M = 64 rows;
 //     V (MN-major) and P (K-major) keep their shared-memory layouts, only the
 //     roles swap.  O^T lives in TMEM as 128 lanes (d) x 64 columns (rows).
+//   - The grid is split-major (x = kv head, y = request, z = split): the CTAs
+//     are dispatched roughly in linear block order, so every request's full
+//     first splits go out before the later ones, and the last wave is made of
+//     the partial last splits (shorter by half on average) instead of full
+//     8192-key splits of the last requests.  Outputs are unchanged (each CTA
+//     writes its own partial); 128 requests x 8k-32k keys: 5.46 -> 5.60 TB/s
+//     alone, 0.64 -> 0.70 of the copy figure inside the whole step.
 //   - The softmax keeps one reference m_r per row, fixed at the first tile's
 //     row maximum.  Later tiles compute p = 2^(s * scale - m_r) directly, with
 //     no per-tile maximum: exp2 of anything up to 2^kTc2Headroom stays well
@@ -137,7 +144,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
   constexpr int D = C::D, ST = C::ST, NB = C::kPBufs;
   pdl_trigger();
   pdl_wait();
-  const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int h = blockIdx.x, b = blockIdx.y, split = blockIdx.z;   // split-major grid
   const int n_keys = p.seq_lens[b] + p.bs;
   const int k0 = split * p.chunk_keys;
   if (k0 >= n_keys) return;

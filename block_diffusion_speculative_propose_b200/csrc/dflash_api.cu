@@ -958,11 +958,14 @@ dflash_status run_attention(dflash_handle* h, const AttnPlan& ap, AttnParams prm
   if (ap.tc2) {
     LaunchScope scope(h, DFLASH_KERNEL_ATTENTION, st);
     if constexpr (D == 128) {
+      // split-major: every request's first splits are dispatched first and the
+      // partial last splits fill the tail
+      const dim3 grid2(c.n_kv_heads, prm.B, ap.max_splits);
       if (ap.kt == 64)
-        launch_k(h->pdl, attn_block_tc2_kernel<64>, grid, dim3(kTcThreads), Tc2Cfg<64>::kSmem,
+        launch_k(h->pdl, attn_block_tc2_kernel<64>, grid2, dim3(kTcThreads), Tc2Cfg<64>::kSmem,
                  st, tk, tv, prm);
       else
-        launch_k(h->pdl, attn_block_tc2_kernel<32>, grid, dim3(kTcThreads), Tc2Cfg<32>::kSmem,
+        launch_k(h->pdl, attn_block_tc2_kernel<32>, grid2, dim3(kTcThreads), Tc2Cfg<32>::kSmem,
                  st, tk, tv, prm);
     }
   } else if (ap.tc) {
