@@ -97,3 +97,18 @@ def test_reference_arm_bounds_its_run(monkeypatch, capsys):
     bench.run_reference(a, 0, 1)
     d = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
     assert d["oracle_steps_timed"] == 2 and FakeOracle.calls == 3
+
+
+def test_traffic_records_match_the_kernel_sources():
+    """Every ncu traffic record in bench.py was taken on the kernel sources as
+    they stand: a kernel change without a new capture would make the bench
+    line's roofline.traffic read null."""
+    import bench
+    for (workload, family), rec in bench.TRAFFIC.items():
+        fam = "attention" if family == "attention" else "gemm"
+        assert rec["digest"] == bench.source_digest(fam), (workload, family)
+        assert ("ratio_to_algorithmic" in rec) != ("bytes_per_launch" in rec)
+        if "ratio_to_algorithmic" in rec:
+            assert 1.0 <= rec["ratio_to_algorithmic"] < 1.2
+    # the default workload's dominant kernel has a record
+    assert (bench.DEFAULT_WORKLOAD, "attention") in bench.TRAFFIC
