@@ -207,6 +207,10 @@ size_t gemm_partial_bound(int M, int num_sms) {
 // ---------------------------------------------------------------------------
 // attention planning
 // ---------------------------------------------------------------------------
+// Requests per attention launch: the request index is a grid dimension (y for
+// the two-CTA kernel, z for the others), at most 65535.
+constexpr int kMaxAttnRequests = 65535;
+
 struct AttnPlan {
   int chunk_keys = 0, max_splits = 0, R = 0, row_groups = 0, key_parts = 0, nwc = 0;
   bool tc = false;   // tcgen05 kernel (kv groups of up to 64 query rows)
@@ -1816,7 +1820,9 @@ dflash_status propose_impl(dflash_handle* h, const int32_t* bonus_tokens,
   for (int l = 0; l < c.n_layers; ++l)
     if (!k_cache[l] || !v_cache[l]) return DFLASH_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return DFLASH_ERR_INVALID_ARG;
-  if (static_cast<int64_t>(B) * c.block_size > (1 << 24)) return DFLASH_ERR_UNSUPPORTED_SHAPE;
+  // (the attention grid carries the request index in its y dimension)
+  if (static_cast<int64_t>(B) * c.block_size > (1 << 24) || B > kMaxAttnRequests)
+    return DFLASH_ERR_UNSUPPORTED_SHAPE;
   const ProposeWs lw = propose_layout(h, B, max_pages_per_seq);
   if (workspace_bytes < lw.total) return DFLASH_ERR_WORKSPACE;
   DF_CUDA(use_device(h->device));
@@ -1990,7 +1996,7 @@ dflash_status check_step(const dflash_handle* h, const dflash_step_io* io, const
   if (reinterpret_cast<uintptr_t>(ws) % kAlign) return DFLASH_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(io->target_logits) % 16 && c.vocab % 4 == 0)
     return DFLASH_ERR_INVALID_ARG;
-  if (static_cast<int64_t>(io->B) * c.block_size > (1 << 24))
+  if (static_cast<int64_t>(io->B) * c.block_size > (1 << 24) || io->B > kMaxAttnRequests)
     return DFLASH_ERR_UNSUPPORTED_SHAPE;
   if (bytes < step_layout(h, io->B, io->n, io->max_pages_per_seq).total)
     return DFLASH_ERR_WORKSPACE;
@@ -2218,6 +2224,7 @@ dflash_status dflash_block_attention(dflash_handle* h, const void* q, const int3
       num_pages <= 0 || !o || !workspace)
     return DFLASH_ERR_INVALID_ARG;
   const dflash_config& c = h->cfg;
+  if (B > kMaxAttnRequests) return DFLASH_ERR_UNSUPPORTED_SHAPE;
   if (workspace_bytes < dflash_attention_workspace_bytes(h, B, max_pages_per_seq))
     return DFLASH_ERR_WORKSPACE;
   DF_CUDA(use_device(h->device));

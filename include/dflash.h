@@ -334,7 +334,8 @@ dflash_status dflash_inject_context(dflash_handle* h, const void* aux,
  *                 block slots 1..bs-1 (ties -> lowest id; NaN counts as -inf)
  *   block_tokens  [B, bs] int32 out, cat(bonus, drafts); may be NULL
  *   logits_out    [B*K, V] fp32 out (debug); may be NULL
- * B == 0 is a no-op.  Needs dflash_propose_workspace_bytes(h, B, max_pages_per_seq). */
+ * B == 0 is a no-op; B > 65535 (requests per attention launch) or B * bs > 2^24 is
+ * DFLASH_ERR_UNSUPPORTED_SHAPE.  Needs dflash_propose_workspace_bytes(h, B, max_pages_per_seq). */
 dflash_status dflash_propose(dflash_handle* h, const int32_t* bonus_tokens,
                              const int32_t* seq_lens, const int32_t* block_table,
                              int B, int max_pages_per_seq, void* const* k_cache,
@@ -547,6 +548,7 @@ dflash_status dflash_linear_ex(dflash_handle* h, const void* A, const void* W, i
  *   o [B*bs, n_q_heads*head_dim] fp16 out (as the proposal path stores it)
  * Request b attends to its logical keys [0, seq_lens[b] + bs), located through
  * block_table exactly as in dflash_propose; scale 1/sqrt(head_dim).
+ * B > 65535 is DFLASH_ERR_UNSUPPORTED_SHAPE.
  * Needs dflash_attention_workspace_bytes(h, B, max_pages_per_seq). */
 size_t dflash_attention_workspace_bytes(const dflash_handle* h, int B, int max_pages_per_seq);
 dflash_status dflash_block_attention(dflash_handle* h, const void* q, const int32_t* seq_lens,

@@ -8,6 +8,8 @@
   nothing arrives on) gives up after the device's wait limit, the handle
   reports DFLASH_ERR_DEVICE_TIMEOUT, and the context stays usable: the next
   proposal is clean and identical to one taken before.
+- Request count: more requests than an attention launch can index are refused
+  on the host before any launch.
 """
 
 from __future__ import annotations
@@ -24,6 +26,7 @@ DEV = "cuda:0"
 DEVERR_TIMEOUT = 1
 ERR_RANGE = -8
 ERR_DEVICE_TIMEOUT = -7
+ERR_UNSUPPORTED_SHAPE = -4
 
 
 def _tiny():
@@ -93,5 +96,38 @@ def test_bounded_wait_runs_out_and_context_survives():
         after = _propose(h, cfg)
         assert h.check_device_errors() == 0
         np.testing.assert_array_equal(before, after)
+    finally:
+        h.close()
+
+
+def test_request_count_limit_refused_before_any_launch():
+    """The attention grid carries the request index in one of its dimensions
+    (at most 65535): a proposal or an attention call for 65536 requests is
+    DFLASH_ERR_UNSUPPORTED_SHAPE on the host, before any launch or buffer
+    access (the buffers passed here are deliberately too small to be read)."""
+    cfg, W = _tiny()
+    h = DFlash(cfg, W, max_position=1024)
+    try:
+        B = 65536
+        bonus = torch.zeros(B, dtype=torch.int32, device=DEV)
+        seq = torch.zeros(B, dtype=torch.int32, device=DEV)
+        table = torch.zeros(B, 1, dtype=torch.int32, device=DEV)
+        shape = (1, cfg["n_kv_heads"], cfg["page_size"], cfg["head_dim"])
+        kc = [torch.zeros(shape, dtype=torch.bfloat16, device=DEV) for _ in range(cfg["n_layers"])]
+        vc = [torch.zeros(shape, dtype=torch.bfloat16, device=DEV) for _ in range(cfg["n_layers"])]
+        ws = torch.zeros(1024, dtype=torch.uint8, device=DEV)
+        with pytest.raises(DFlashError) as e:
+            h.propose(bonus, seq, table, kc, vc, workspace=ws)
+        assert e.value.status == ERR_UNSUPPORTED_SHAPE
+        q = torch.zeros(cfg["block_size"], cfg["n_q_heads"], cfg["head_dim"], dtype=torch.bfloat16,
+                        device=DEV)
+        with pytest.raises(DFlashError) as e:
+            h.block_attention(q, seq, table, kc[0], vc[0], workspace=ws)
+        assert e.value.status == ERR_UNSUPPORTED_SHAPE
+        torch.cuda.synchronize()
+        assert h.check_device_errors() == 0
+        # the handle still proposes
+        _propose(h, cfg)
+        assert h.check_device_errors() == 0
     finally:
         h.close()
